@@ -1,0 +1,431 @@
+"""Benchmark of the DSA decode step (lightning indexer + top-k + sparse latent
+attention) on B200, one process per GPU.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload 4] [--no-cpu-baseline]
+
+A step is one decode step of the whole batch (B sequences) of the chosen
+workload (default: B = 8 sequences at 131072 tokens, the 128K-context case):
+rotate/quantise the new queries and key, append the key, score every cached
+key, select the top 2048, run the sparse latent attention.  Under torchrun each
+rank runs its own batch (independent sequences, no collective on the data
+path: weak scaling); the timed region is bracketed by a barrier and a device
+synchronise, and the slowest rank's time counts.
+
+Rank 0 prints ONE JSON line.  `--impl reference` times the CPU oracle instead
+(the only reference implementation there is), on a bounded sample of the same
+workload, on rank 0 only.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+import torch
+
+import workloads
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+N_COPIES = 3            # rotating device copies of the decode state (each > L2)
+
+
+def _peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            p = json.load(f)
+        return float(p["hbm_gbs"]), "measured"
+    return 6650.0, "fallback"
+
+
+# --------------------------------------------------------------------------- #
+# distributed plumbing
+# --------------------------------------------------------------------------- #
+def _dist_init():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        backend = "nccl" if torch.cuda.is_available() else "gloo"
+        if torch.cuda.is_available():
+            torch.cuda.set_device(local)
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(local)
+    return world, rank, local
+
+
+def _barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def _max_over_ranks(world, value: float) -> float:
+    if world == 1:
+        return value
+    import torch.distributed as dist
+    t = torch.tensor([value], dtype=torch.float64,
+                     device="cuda" if torch.cuda.is_available() else "cpu")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# --------------------------------------------------------------------------- #
+# clocks sampled during the timed region
+# --------------------------------------------------------------------------- #
+class ClockSampler:
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.dev = device_index
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.dev), f"--query-gpu={self.QUERY}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        self.lines = []
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                out, _ = self.proc.communicate(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+                out, _ = self.proc.communicate()
+            self.lines = [l for l in out.splitlines() if l.strip()]
+
+    def summary(self):
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in getattr(self, "lines", []):
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx.append(float(f[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx),
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# --------------------------------------------------------------------------- #
+# device state of the decode step
+# --------------------------------------------------------------------------- #
+def build_state(dsa, wl, rank_seed_offset=0):
+    """Device state for one decode step of wl (B sequences), N_COPIES rotating copies."""
+    dev = "cuda"
+    B, T = wl.B, wl.T
+    dt = torch.bfloat16 if wl.attn_dtype == "bf16" else torch.float32
+    k_cache = torch.empty(B, T, wl.D, dtype=torch.uint8, device=dev)
+    k_scale = torch.empty(B, T, dtype=torch.float32, device=dev)
+    kv = torch.empty(B, T, wl.dqk, dtype=dt, device=dev)
+    q_idx = torch.empty(B, wl.H, wl.D, device=dev)
+    w = torch.empty(B, wl.H, device=dev)
+    k_new = torch.empty(B, wl.D, device=dev)
+    q_mla = torch.empty(B, wl.Hq, wl.dqk, dtype=dt, device=dev)
+    for b in range(B):
+        s = workloads.decode_sequence(wl, b + rank_seed_offset)
+        dsa.dsa_indexer_quant(s["keys"][:T - 1].to(dev), k_cache[b], k_scale[b])
+        kv[b] = s["kv"].to(dev)
+        q_idx[b] = s["q_idx"].to(dev)
+        w[b] = s["w"].to(dev)
+        k_new[b] = s["keys"][T - 1].to(dev)
+        q_mla[b] = s["q_mla"].to(dev)
+        del s
+    K = wl.K
+    dtc = dsa.DSA_BF16 if dt == torch.bfloat16 else dsa.DSA_F32
+    need = dsa.dsa_decode_step_workspace_size(B, wl.H, wl.D, T, wl.topk, wl.Hq, wl.dc, wl.dr, dtc)
+    copies = []
+    for c in range(N_COPIES):
+        copies.append(dict(
+            k_cache=k_cache if c == 0 else k_cache.clone(),
+            k_scale=k_scale if c == 0 else k_scale.clone(),
+            kv=kv if c == 0 else kv.clone(),
+            q_idx=q_idx.clone(), w=w.clone(), k_new=k_new.clone(), q_mla=q_mla.clone(),
+            idx=torch.empty(B, K, dtype=torch.int32, device=dev),
+            out=torch.empty(B, wl.Hq, wl.dc, dtype=dt, device=dev),
+            lse=torch.empty(B, wl.Hq, dtype=torch.float32, device=dev),
+            ws=torch.empty(need, dtype=torch.uint8, device=dev), T=T))
+    return copies
+
+
+def decode_step(dsa, wl, st, stream=None):
+    dsa.dsa_decode_step(st["q_idx"], st["w"], st["k_new"], st["k_cache"], st["k_scale"],
+                        st["kv"], st["q_mla"], st["T"], wl.topk, wl.softmax_scale_idx,
+                        wl.sm_scale, st["idx"], st["out"], st["lse"], st["ws"], stream=stream)
+
+
+def count_launches_per_step(wl, dsa, st) -> tuple[int, list[str]]:
+    """Kernels one decode step launches, counted by the profiler on an untimed step."""
+    from torch.profiler import ProfilerActivity, profile
+    torch.cuda.synchronize()
+    with profile(activities=[ProfilerActivity.CUDA]) as prof:
+        decode_step(dsa, wl, st)
+        torch.cuda.synchronize()
+    names = [e.name for e in prof.events() if e.device_type.name == "CUDA"
+             and "memcpy" not in e.name.lower() and "memset" not in e.name.lower()]
+    return len(names), sorted(set(names))
+
+
+# --------------------------------------------------------------------------- #
+# dominant kernel: the indexer scorer, timed alone on the same inputs
+# --------------------------------------------------------------------------- #
+def time_scorer(dsa, wl, copies, iters):
+    """Average duration of the index-scoring launch over the full cache, with
+    CUDA events on the launching stream, rotating the state copies."""
+    dev = "cuda"
+    B, T = wl.B, wl.T
+    q_fp8 = torch.empty(B, 1, wl.H, wl.D, dtype=torch.uint8, device=dev)
+    q_scale = torch.empty(B, 1, wl.H, dtype=torch.float32, device=dev)
+    dsa.dsa_indexer_quant(copies[0]["q_idx"], q_fp8, q_scale)
+    w = copies[0]["w"].reshape(B, 1, wl.H).contiguous()
+    scores = torch.empty(B, 1, T, dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream()
+    for i in range(3):
+        st = copies[i % len(copies)]
+        dsa.dsa_index_scores(q_fp8, q_scale, w, st["k_cache"], st["k_scale"], T - 1, T,
+                             wl.softmax_scale_idx, scores)
+    torch.cuda.synchronize()
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for i in range(iters):
+        st = copies[i % len(copies)]
+        dsa.dsa_index_scores(q_fp8, q_scale, w, st["k_cache"], st["k_scale"], T - 1, T,
+                             wl.softmax_scale_idx, scores)
+    t1.record(stream)
+    t1.synchronize()
+    return t0.elapsed_time(t1) / iters * 1e-3      # seconds per launch
+
+
+# --------------------------------------------------------------------------- #
+# the CPU oracle as a baseline (bounded sample)
+# --------------------------------------------------------------------------- #
+def oracle_decode_sample(wl, n_seq: int, repeats: int = 1):
+    """Time the oracle's per-step work (quantise q and the new key, score the
+    T cached keys, select, attend) on n_seq sequences; the cache itself is
+    quantised once, untimed, as a decode cache would already hold it."""
+    import oracle
+    per_seq = []
+    for b in range(n_seq):
+        s = workloads.decode_sequence(wl, b)
+        keys = s["keys"].numpy()
+        T = keys.shape[0]
+        k_fp8, k_sc = oracle.indexer_quant(keys[:T - 1])
+        k_fp8 = np.concatenate([k_fp8, np.zeros((1, wl.D), np.uint8)])[None]
+        k_sc = np.concatenate([k_sc, np.zeros(1, np.float32)])[None]
+        q_mla = s["q_mla"].float().numpy()[None, None]
+        kv = s["kv"].float().numpy()[None]
+        for _ in range(repeats):
+            t0 = time.perf_counter()
+            nk, ns = oracle.indexer_quant(keys[T - 1:T])
+            k_fp8[0, T - 1], k_sc[0, T - 1] = nk[0], ns[0]
+            qf, qs = oracle.indexer_quant(s["q_idx"].numpy())
+            sc = oracle.index_scores(qf[None, None], qs[None, None], s["w"].numpy()[None, None],
+                                     k_fp8, k_sc, T - 1, T, wl.softmax_scale_idx)
+            idx = oracle.topk_select(sc, T - 1, wl.topk)
+            oracle.sparse_mla(q_mla, kv, idx, T - 1, wl.sm_scale, wl.dc)
+            per_seq.append(time.perf_counter() - t0)
+    return per_seq
+
+
+def run_reference(args, wl, world, rank):
+    if rank != 0:
+        return
+    # one "step" of the reference arm = the oracle's decode pass for ONE
+    # sequence of the batch; steps/s of the whole batch = 1 / (B * t_seq)
+    warm = oracle_decode_sample(wl, 1, repeats=max(args.warmup, 0)) if args.warmup else []
+    times = []
+    for k in range(args.steps):
+        times += oracle_decode_sample(wl, 1, repeats=1)
+    t_seq = sum(times) / len(times)
+    value = 1.0 / (wl.B * t_seq)
+    line = {
+        "metric": "dsa_decode_steps_per_s", "value": value, "unit": "steps/s", "n_gpus": 1,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": wl.B * t_seq * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "impl": "reference",
+        "config": {"workload": wl.name, "B": wl.B, "T": wl.T, "H": wl.H, "D": wl.D,
+                   "topk": wl.topk, "Hq": wl.Hq, "dc": wl.dc, "dr": wl.dr},
+        "cpu_baseline": {"value": value, "unit": "steps/s", "cores": 1, "kind": "oracle",
+                         "sample": f"sequence 0 of {wl.B}, one decode step per timed step "
+                                   f"(T={wl.T}), extrapolated x{wl.B}; cache prebuilt"},
+        "e2e": {"value": value, "unit": "steps/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+        "indexer_gscores_per_s": wl.T / t_seq / 1e9,
+    }
+    print(json.dumps(line), flush=True)
+
+
+# --------------------------------------------------------------------------- #
+# our arm
+# --------------------------------------------------------------------------- #
+def run_ours(args, wl, world, rank, local):
+    from top_kv_selection_b200 import build as _build
+    _build.build()
+    import top_kv_selection_b200 as dsa
+
+    copies = build_state(dsa, wl, rank_seed_offset=0)
+    torch.cuda.synchronize()
+    per_step_launches, kernel_names = count_launches_per_step(wl, dsa, copies[0])
+
+    stream = torch.cuda.current_stream()
+    for i in range(args.warmup):
+        decode_step(dsa, wl, copies[i % N_COPIES])
+    torch.cuda.synchronize()
+    if dsa.dsa_get_device_error() != 0:
+        raise RuntimeError("device error word set during warm-up")
+
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    _barrier(world)
+    torch.cuda.synchronize()
+    with ClockSampler(torch.cuda.current_device()) as clk:
+        start.record(stream)
+        for i in range(args.steps):
+            decode_step(dsa, wl, copies[i % N_COPIES])
+        end.record(stream)
+        end.synchronize()
+    torch.cuda.synchronize()
+    _barrier(world)
+    elapsed = start.elapsed_time(end) * 1e-3
+    elapsed = _max_over_ranks(world, elapsed)
+    ms_per_step = elapsed / args.steps * 1e3
+    value = world * args.steps / elapsed
+    gscores = world * args.steps * wl.B * wl.T / elapsed / 1e9
+
+    # e2e: per-step inputs from pinned host memory, result back to the host
+    e2e = run_e2e(dsa, wl, copies, args, world)
+
+    # dominant kernel roofline (indexer scorer over the full cache)
+    peak, peak_kind = _peaks()
+    t_score = time_scorer(dsa, wl, copies, iters=max(10, args.steps))
+    score_bytes = wl.B * wl.T * (wl.D + 4) + wl.B * wl.H * (wl.D + 4 + 4)
+    achieved = score_bytes / t_score / 1e9
+    step_bytes = wl.B * (wl.T * (wl.D + 4) + wl.K * wl.dqk * 2 + wl.H * wl.D * 4
+                         + wl.Hq * wl.dqk * 2 + wl.Hq * wl.dc * 2)
+
+    line = {
+        "metric": "dsa_decode_steps_per_s", "value": value, "unit": "steps/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "fp8_e4m3+bf16", "data": "synthetic",
+        "config": {"workload": wl.name, "B": wl.B, "T": wl.T, "H": wl.H, "D": wl.D,
+                   "topk": wl.topk, "Hq": wl.Hq, "dc": wl.dc, "dr": wl.dr,
+                   "l2": f"{N_COPIES} rotating state copies, each larger than L2",
+                   "parallelism": f"dp{world} (independent batches per rank)"},
+        "indexer_gscores_per_s": gscores,
+        "step_roofline": {"bytes": step_bytes, "achieved_gbs": step_bytes / (ms_per_step * 1e-3)
+                          / 1e9, "frac": step_bytes / (ms_per_step * 1e-3) / 1e9 / peak},
+        "roofline": {"kernel": "index_scores", "bound": "hbm", "achieved": achieved,
+                     "peak": peak, "peak_kind": f"{peak_kind} hbm_gbs", "unit": "GB/s",
+                     "frac": achieved / peak, "traffic": None,
+                     "avg_launch_us": t_score * 1e6},
+        "e2e": e2e,
+        "gpu_launches": per_step_launches * args.steps,
+        "kernels_per_step": per_step_launches, "kernels": kernel_names,
+        "clocks": clk.summary(),
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        times = oracle_decode_sample(wl, 2)
+        t_seq = sum(times) / len(times)
+        line["cpu_baseline"] = {
+            "value": 1.0 / (wl.B * t_seq), "unit": "steps/s", "cores": 1, "kind": "oracle",
+            "sample": f"sequences 0-1 of {wl.B}, one decode step each at T={wl.T} "
+                      f"({sum(times):.1f} s), extrapolated x{wl.B}; cache prebuilt"}
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
+def run_e2e(dsa, wl, copies, args, world):
+    """Same step through the public API with host buffers: the step's inputs are
+    copied from pinned host memory and the result read back, inside the timed region."""
+    B = wl.B
+    st = copies[0]
+    host_in = {k: st[k].cpu().pin_memory() for k in ("q_idx", "w", "k_new", "q_mla")}
+    new_row = st["kv"][:, wl.T - 1].cpu().pin_memory()
+    host_idx = torch.empty(st["idx"].shape, dtype=torch.int32).pin_memory()
+    host_out = torch.empty(st["out"].shape, dtype=st["out"].dtype).pin_memory()
+    h2d = sum(t.numel() * t.element_size() for t in host_in.values()) + \
+        new_row.numel() * new_row.element_size()
+    d2h = host_idx.numel() * 4 + host_out.numel() * host_out.element_size()
+    stream = torch.cuda.current_stream()
+
+    def one(i):
+        s = copies[i % N_COPIES]
+        for k, t in host_in.items():
+            s[k].copy_(t, non_blocking=True)
+        s["kv"][:, wl.T - 1].copy_(new_row, non_blocking=True)
+        decode_step(dsa, wl, s)
+        host_idx.copy_(s["idx"], non_blocking=True)
+        host_out.copy_(s["out"], non_blocking=True)
+
+    for i in range(max(args.warmup, 1)):
+        one(i)
+    torch.cuda.synchronize()
+    _barrier(world)
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for i in range(args.steps):
+        one(i)
+    t1.record(stream)
+    t1.synchronize()
+    el = _max_over_ranks(world, t0.elapsed_time(t1) * 1e-3)
+    return {"value": world * args.steps / el, "unit": "steps/s", "h2d_bytes_per_step": h2d,
+            "d2h_bytes_per_step": d2h}
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", type=int, default=4)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args(argv)
+    wl = workloads.WORKLOADS[args.workload]
+    if wl.mode != "decode":
+        raise SystemExit("bench.py times decode workloads (1, 2 or 4)")
+    world, rank, local = _dist_init()
+    try:
+        if args.impl == "reference":
+            run_reference(args, wl, world, rank)
+        else:
+            if not torch.cuda.is_available():
+                raise SystemExit("no CUDA device: the product path has no CPU fallback")
+            run_ours(args, wl, world, rank, local)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

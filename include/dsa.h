@@ -1,0 +1,188 @@
+/*
+ * dsa.h -- C ABI of libdsa: the data-parallel hot path of DeepSeek Sparse
+ * Attention on NVIDIA B200 (sm_100a).
+ *
+ * The path (lightning indexer, top-k token selection, sparse latent attention)
+ * follows these pages:
+ *   "DeepSeek-V3.2-Exp - Split indexer heads": the Indexer.forward excerpt
+ *       (inference/model.py, lines 457-487): rotate_activation, act_quant,
+ *       the key-cache write, the weight fold, fp8_index, the additive mask and
+ *       topk(min(index_topk, end_pos)).
+ *   "DeepSeek-V3.2-Exp - Causal mask": Transformer.forward (mask =
+ *       full(-inf).triu_(1) when seqlen > 1) and the MLA prefill excerpt
+ *       (model.py 574-589: index_mask = full(-inf).scatter_(topk, 0) + mask).
+ *   "DeepSeek Sparse Attention, one decode step in one layer (V3.2 sizes)"
+ *       diagram: I(t,s) = sum_j w_j ReLU(q_j . k_s), k = 2048, core attention
+ *       in MQA mode over the gathered latents, each latent row key and value.
+ *
+ * Conventions for every entry point:
+ *   - Memory: every tensor argument is a caller-owned DEVICE pointer, row-major
+ *     and contiguous with the layout stated below, 16-byte aligned.  The
+ *     library allocates nothing.  Scratch memory is passed in as `workspace`
+ *     (size from the matching *_workspace_size call); it need not be zeroed.
+ *   - Execution: every call only enqueues kernels on `stream` and returns; it
+ *     never synchronises.  Calls on one stream run in order.  Two calls that
+ *     share a workspace must not run concurrently.
+ *   - Errors: argument checks run on the host before anything is launched and
+ *     return DSA_ERR_INVALID_ARG / DSA_ERR_UNSUPPORTED / DSA_ERR_WORKSPACE with
+ *     nothing enqueued.  A failed launch returns DSA_ERR_CUDA.  Problems found
+ *     on the device (an index out of range) never trap: the kernel skips the
+ *     access and records a code in a sticky device word that
+ *     dsa_get_device_error() reads.
+ *   - Empty problems (a zero batch or zero vectors) return DSA_OK without a
+ *     launch.
+ *   - Indices are int32; -1 marks an empty selection slot.
+ */
+#ifndef DSA_H
+#define DSA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same type as cudaStream_t; NULL is the legacy default stream. */
+typedef struct CUstream_st *dsa_stream_t;
+
+typedef enum dsa_status {
+    DSA_OK = 0,
+    DSA_ERR_INVALID_ARG = 1,   /* null pointer, bad size, misaligned pointer  */
+    DSA_ERR_UNSUPPORTED = 2,   /* valid but not built (e.g. D not 64 or 128)  */
+    DSA_ERR_CUDA = 3,          /* a CUDA runtime call or launch failed        */
+    DSA_ERR_TIMEOUT = 4,       /* a bounded device-side wait expired          */
+    DSA_ERR_DEVICE = 5,        /* device-side check failed (see device word)  */
+    DSA_ERR_WORKSPACE = 6      /* workspace missing or smaller than required  */
+} dsa_status;
+
+typedef enum dsa_dtype {
+    DSA_F32 = 0,               /* IEEE binary32 */
+    DSA_BF16 = 1               /* bfloat16      */
+} dsa_dtype;
+
+/* Text for a status code (static storage, never NULL). */
+const char *dsa_status_string(dsa_status status);
+
+/* Library version: major * 10000 + minor * 100 + patch. */
+int dsa_version(void);
+
+/*
+ * Waits for `stream`, then returns in *device_status the first code a kernel
+ * of this library recorded on the current device since the last call (DSA_OK
+ * if none) and clears it.  Returns DSA_ERR_INVALID_ARG if device_status is
+ * NULL, DSA_ERR_CUDA if the wait or the read fails.
+ */
+dsa_status dsa_get_device_error(dsa_stream_t stream, int32_t *device_status);
+
+/*
+ * rotate_activation + act_quant (Indexer.forward, "Split indexer heads"):
+ * each d-vector is rotated by the orthonormal Walsh-Hadamard transform
+ * (butterflies in fp32 with strides 1, 2, ..., d/2, then one multiply by
+ * fp32(d^-1/2)) and quantised to FP8 e4m3 with one scale per vector:
+ * scale = max(amax, 1e-4) / 448, code = e4m3_rn_satfinite(x / scale), both
+ * divisions correctly rounded.
+ *
+ *   x          [n_rows, n_vec, d]  F32 or BF16 (x_dtype), contiguous
+ *   out_fp8    vector (r, v) -> out_fp8 + r * out_row_stride + v * d  (bytes)
+ *   out_scale  vector (r, v) -> out_scale + r * scale_row_stride + v  (floats)
+ *
+ * Queries: n_rows = 1, n_vec = B*S*H, strides unused (pass 0).
+ * Keys appended to a cache k_cache[B, t_max, d] / k_scale[B, t_max] at
+ * start_pos: x = keys[B, S, d], n_rows = B, n_vec = S, out_fp8 = k_cache +
+ * start_pos * d, out_row_stride = t_max * d, out_scale = k_scale + start_pos,
+ * scale_row_stride = t_max.
+ * d must be 64 or 128 (else DSA_ERR_UNSUPPORTED).  out_row_stride must be a
+ * multiple of 16 when n_rows > 1.
+ */
+dsa_status dsa_indexer_quant(const void *x, dsa_dtype x_dtype, int64_t n_rows, int64_t n_vec,
+                             int d, uint8_t *out_fp8, int64_t out_row_stride, float *out_scale,
+                             int64_t scale_row_stride, dsa_stream_t stream);
+
+/*
+ * fp8_index with the weight fold and the additive causal mask
+ * (Indexer.forward; mask from Transformer.forward; formula from the diagram):
+ *   w'[b,s,h]  = fp32(fp32(fp32(w * fp32(H^-1/2)) * q_scale) * softmax_scale)
+ *   I[b,s,t]   = k_scale[b,t] * sum_h w'[b,s,h] * ReLU(q_fp8[b,s,h,:] . k_cache[b,t,:])
+ *   I[b,s,t]   = -inf for t > start_pos + s
+ * Dot products of the decoded FP8 values accumulate in fp32.
+ *
+ *   q_fp8   [B,S,H,D] e4m3 codes     q_scale [B,S,H] fp32     w [B,S,H] fp32
+ *   k_cache [B,t_max,D] e4m3 codes   k_scale [B,t_max] fp32
+ *   scores  [B,S,T] fp32 (T = end_pos <= t_max; start_pos + S <= T)
+ * D must be 64 or 128; 1 <= H <= 256.
+ */
+dsa_status dsa_index_scores(const uint8_t *q_fp8, const float *q_scale, const float *w,
+                            const uint8_t *k_cache, const float *k_scale, int64_t t_max, int B,
+                            int S, int H, int D, int64_t start_pos, int64_t T,
+                            float softmax_scale, float *scores, dsa_stream_t stream);
+
+/*
+ * topk(min(index_topk, end_pos)) (Indexer.forward), restricted to the causal
+ * positions t <= start_pos + s of each row:
+ *   idx[b,s,:] holds the m = min(K, start_pos+s+1, T) positions with the
+ *   largest scores, K = min(k, T), ties broken towards the lower position,
+ *   written in ascending position order; slots m..K-1 hold -1.
+ * Scores are compared as fp32 values (-0 equals +0; NaN ranks below -inf).
+ *
+ *   scores [B,S,T] fp32     idx [B,S,K] int32
+ */
+size_t dsa_topk_select_workspace_size(int B, int S, int64_t T, int k);
+dsa_status dsa_topk_select(const float *scores, int B, int S, int64_t T, int64_t start_pos,
+                           int k, int32_t *idx, void *workspace, size_t workspace_bytes,
+                           dsa_stream_t stream);
+
+/*
+ * Sparse latent attention, MQA mode (diagram "core attention"; semantics of
+ * the MLA prefill excerpt with the index mask and the causal mask):
+ *   for each (b, s, head) over the selected rows c_j = kv_cache[b, idx_j, :]:
+ *   z_j = sm_scale * (q[:dc] . c_j[:dc] + q[dc:] . c_j[dc:])
+ *   out = sum_j softmax(z)_j * c_j[:dc],   lse = log sum_j exp(z_j)
+ * Slots with idx < 0 or idx > start_pos + s are skipped (the -1 sentinel and
+ * the causal mask).  A row with no valid slot gives out = 0, lse = -inf.
+ * Indices must be distinct within a row and below t_max; an index >= t_max
+ * is skipped and recorded as DSA_ERR_DEVICE in the device word.
+ *
+ *   q        [B,S,Hq,dc+dr]   kv_cache [B,t_max,dc+dr]   (dtype dt)
+ *   idx      [B,S,k] int32
+ *   out      [B,S,Hq,dc] (dtype dt)     lse [B,S,Hq] fp32 or NULL
+ * dt = DSA_BF16 (tensor-core path, fp32 softmax and accumulation) or DSA_F32
+ * (test mode: fp32 FMA throughout).
+ */
+size_t dsa_sparse_mla_attn_workspace_size(int B, int S, int Hq, int dc, int dr, int k,
+                                          dsa_dtype dt);
+dsa_status dsa_sparse_mla_attn(const void *q, const void *kv_cache, int64_t t_max,
+                               const int32_t *idx, int B, int S, int Hq, int dc, int dr, int k,
+                               int64_t start_pos, float sm_scale, dsa_dtype dt, void *out,
+                               float *lse, void *workspace, size_t workspace_bytes,
+                               dsa_stream_t stream);
+
+/*
+ * One DSA decode step for B sequences that each see T tokens (end_pos = T,
+ * the new token at position T-1; no mask, as seqlen == 1):
+ *   1. rotate + quantise the new token's indexer queries and key; append the
+ *      key to k_cache / k_scale at position T-1 (Indexer.forward cache write);
+ *   2. score all T cached keys (fp8_index with the weight fold);
+ *   3. select the top K = min(index_topk, T) positions into idx;
+ *   4. sparse latent attention of q_mla over the selected latent rows.
+ *
+ *   q_idx [B,H,D] fp32   w [B,H] fp32   k_new [B,D] fp32
+ *   k_cache [B,t_max,D] e4m3 (written at T-1)   k_scale [B,t_max] fp32
+ *   kv_cache [B,t_max,dc+dr] (dt): row T-1 must already hold the new latent
+ *   q_mla [B,Hq,dc+dr] (dt)   idx [B,K] int32   out [B,Hq,dc] (dt)
+ *   lse [B,Hq] fp32 or NULL
+ */
+size_t dsa_decode_step_workspace_size(int B, int H, int D, int64_t T, int index_topk, int Hq,
+                                      int dc, int dr, dsa_dtype dt);
+dsa_status dsa_decode_step(const float *q_idx, const float *w, const float *k_new,
+                           uint8_t *k_cache, float *k_scale, int64_t t_max,
+                           const void *kv_cache, const void *q_mla, int B, int H, int D, int Hq,
+                           int dc, int dr, int64_t T, int index_topk, float softmax_scale,
+                           float sm_scale, dsa_dtype dt, int32_t *idx, void *out, float *lse,
+                           void *workspace, size_t workspace_bytes, dsa_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* DSA_H */

@@ -1,0 +1,69 @@
+"""Comparison rules shared by the GPU parity tests.
+
+Tolerances:
+  * FP8 codes and scales: bit-identical.
+  * scores: |gpu - ref| <= 1e-3 * max(|ref|, rms(ref row)) on finite entries; the
+    masked (-inf) pattern must match exactly.
+  * selections from identical fp32 scores: identical (same tie rule).
+  * selections from each side's own scores: every position in one set and not
+    the other must have an oracle score within the score tolerance of the
+    oracle's k-th score (a boundary tie); the -1 padding must match exactly.
+  * attention: 2e-2 absolute in bf16, 1e-4 absolute in fp32 test mode; lse 1e-3
+    absolute (bf16 inputs) / 1e-5 (fp32).
+"""
+import numpy as np
+
+SCORE_RTOL = 1e-3
+ATTN_ATOL = {"bf16": 2e-2, "f32": 1e-4}
+LSE_ATOL = {"bf16": 1e-3, "f32": 1e-5}
+
+
+def assert_scores_close(gpu, ref):
+    gpu = np.asarray(gpu, dtype=np.float32)
+    ref = np.asarray(ref, dtype=np.float32)
+    assert gpu.shape == ref.shape
+    fin = np.isfinite(ref)
+    assert np.array_equal(np.isfinite(gpu), fin), "mask pattern differs"
+    assert np.all(gpu[~fin] == ref[~fin])
+    r = np.where(fin, ref, 0.0).astype(np.float64)
+    g = np.where(fin, gpu, 0.0).astype(np.float64)
+    rms = np.sqrt((r ** 2).sum(-1, keepdims=True) / np.maximum(fin.sum(-1, keepdims=True), 1))
+    tol = SCORE_RTOL * np.maximum(np.abs(r), rms)
+    bad = np.abs(g - r) > tol
+    assert not bad.any(), (f"{bad.sum()} scores out of tolerance; worst "
+                           f"{np.max(np.abs(g - r) / np.maximum(tol, 1e-30)):.3g}x tol")
+
+
+def assert_selection_matches(gpu_idx, ref_idx, ref_scores_row):
+    """One row: gpu_idx, ref_idx [K]; ref_scores_row [T] = the oracle's scores."""
+    gpu_idx = np.asarray(gpu_idx)
+    ref_idx = np.asarray(ref_idx)
+    assert np.array_equal(gpu_idx < 0, ref_idx < 0), "padding differs"
+    g = set(gpu_idx[gpu_idx >= 0].tolist())
+    r = set(ref_idx[ref_idx >= 0].tolist())
+    assert len(g) == int((gpu_idx >= 0).sum()), "duplicate indices"
+    if g == r:
+        return 0
+    sc = np.asarray(ref_scores_row, dtype=np.float64)
+    kth = min(sc[list(r)])
+    fin = np.isfinite(sc)
+    rms = np.sqrt((sc[fin] ** 2).mean())
+    tol = SCORE_RTOL * max(abs(kth), rms)
+    for t in g ^ r:
+        assert abs(sc[t] - kth) <= tol, f"position {t} score {sc[t]} vs k-th {kth} (tol {tol})"
+    return len(g ^ r) // 2
+
+
+def assert_attention_close(gpu_out, ref_out, dtype, gpu_lse=None, ref_lse=None):
+    gpu_out = np.asarray(gpu_out, dtype=np.float64)
+    ref_out = np.asarray(ref_out, dtype=np.float64)
+    err = np.abs(gpu_out - ref_out).max() if gpu_out.size else 0.0
+    assert err <= ATTN_ATOL[dtype], f"attention max abs err {err}"
+    if gpu_lse is not None:
+        gl = np.asarray(gpu_lse, dtype=np.float64)
+        rl = np.asarray(ref_lse, dtype=np.float64)
+        inf = ~np.isfinite(rl)
+        assert np.array_equal(~np.isfinite(gl), inf)
+        if (~inf).any():
+            e = np.abs(gl[~inf] - rl[~inf]).max()
+            assert e <= LSE_ATOL[dtype], f"lse max abs err {e}"

@@ -1,0 +1,120 @@
+"""The C ABI loads and exports what include/dsa.h declares; host-side argument
+checks reject bad calls before anything is launched (no GPU needed)."""
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "dsa.h")
+
+
+@pytest.fixture(scope="module")
+def dsa():
+    from top_kv_selection_b200 import build
+    build.build()
+    import top_kv_selection_b200 as m
+    return m
+
+
+def header_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(dsa_[a-z0-9_]+)\s*\(", text)))
+
+
+def test_header_declares_the_hot_path_entry_points():
+    names = header_functions()
+    for n in ("dsa_indexer_quant", "dsa_index_scores", "dsa_topk_select",
+              "dsa_sparse_mla_attn", "dsa_decode_step"):
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol(dsa):
+    out = subprocess.run(["nm", "-D", "--defined-only", dsa.LIB_PATH], capture_output=True,
+                         text=True, check=True).stdout
+    exported = set(re.findall(r"\sT\s(dsa_\w+)", out))
+    missing = [n for n in header_functions() if n not in exported]
+    assert not missing, missing
+    assert set(header_functions()) == set(dsa.EXPORTED)
+
+
+def test_status_strings_and_version(dsa):
+    assert dsa.version() >= 100
+    for code in range(7):
+        assert dsa.status_string(code) and dsa.status_string(code) != "unknown status"
+    assert dsa.status_string(99) == "unknown status"
+
+
+NULL = None
+FAKE = ctypes.c_void_p(1 << 20)        # aligned, never dereferenced: checks fail first
+ODD = ctypes.c_void_p((1 << 20) + 4)   # misaligned
+
+
+def test_indexer_quant_argument_checks(dsa):
+    L = dsa._lib
+    assert L.dsa_indexer_quant(FAKE, 0, 1, 8, 96, FAKE, 0, FAKE, 0, NULL) == dsa.DSA_ERR_UNSUPPORTED
+    assert L.dsa_indexer_quant(FAKE, 7, 1, 8, 128, FAKE, 0, FAKE, 0, NULL) == dsa.DSA_ERR_INVALID_ARG
+    assert L.dsa_indexer_quant(NULL, 0, 1, 8, 128, FAKE, 0, FAKE, 0, NULL) == dsa.DSA_ERR_INVALID_ARG
+    assert L.dsa_indexer_quant(ODD, 0, 1, 8, 128, FAKE, 0, FAKE, 0, NULL) == dsa.DSA_ERR_INVALID_ARG
+    assert L.dsa_indexer_quant(FAKE, 0, -1, 8, 128, FAKE, 0, FAKE, 0, NULL) == dsa.DSA_ERR_INVALID_ARG
+    # cache append with a row stride shorter than a row
+    assert L.dsa_indexer_quant(FAKE, 0, 2, 8, 128, FAKE, 512, FAKE, 8, NULL) == dsa.DSA_ERR_INVALID_ARG
+    # empty problems succeed without a launch (no GPU here)
+    assert L.dsa_indexer_quant(NULL, 0, 1, 0, 128, NULL, 0, NULL, 0, NULL) == dsa.DSA_OK
+
+
+def test_index_scores_argument_checks(dsa):
+    L = dsa._lib
+    args = lambda **kw: [kw.get("q", FAKE), FAKE, FAKE, kw.get("k", FAKE), FAKE,
+                         kw.get("t_max", 64), kw.get("B", 1), kw.get("S", 1), kw.get("H", 64),
+                         kw.get("D", 128), kw.get("sp", 63), kw.get("T", 64), 0.1, FAKE, NULL]
+    assert L.dsa_index_scores(*args(D=32)) == dsa.DSA_ERR_UNSUPPORTED
+    assert L.dsa_index_scores(*args(H=300)) == dsa.DSA_ERR_UNSUPPORTED
+    assert L.dsa_index_scores(*args(T=65)) == dsa.DSA_ERR_INVALID_ARG       # T > t_max
+    assert L.dsa_index_scores(*args(sp=64)) == dsa.DSA_ERR_INVALID_ARG      # start_pos + S > T
+    assert L.dsa_index_scores(*args(q=NULL)) == dsa.DSA_ERR_INVALID_ARG
+    assert L.dsa_index_scores(*args(k=ODD)) == dsa.DSA_ERR_INVALID_ARG
+    assert L.dsa_index_scores(*args(B=0)) == dsa.DSA_OK
+
+
+def test_topk_argument_checks(dsa):
+    L = dsa._lib
+    assert L.dsa_topk_select(FAKE, 1, 1, 100, 99, 0, FAKE, NULL, 0, NULL) == dsa.DSA_ERR_INVALID_ARG
+    assert L.dsa_topk_select(FAKE, 1, 2, 100, 99, 8, FAKE, NULL, 0, NULL) == dsa.DSA_ERR_INVALID_ARG
+    assert L.dsa_topk_select(NULL, 1, 1, 100, 99, 8, FAKE, NULL, 0, NULL) == dsa.DSA_ERR_INVALID_ARG
+    assert L.dsa_topk_select(NULL, 0, 1, 100, 99, 8, NULL, NULL, 0, NULL) == dsa.DSA_OK
+    need = L.dsa_topk_select_workspace_size(8, 1, 131072, 2048)
+    if need:
+        assert L.dsa_topk_select(FAKE, 8, 1, 131072, 131071, 2048, FAKE, FAKE, need - 1,
+                                 NULL) == dsa.DSA_ERR_WORKSPACE
+
+
+def test_sparse_mla_argument_checks(dsa):
+    L = dsa._lib
+    base = lambda **kw: [FAKE, FAKE, kw.get("t_max", 4096), FAKE, 1, 1, 128, kw.get("dc", 512),
+                         kw.get("dr", 64), 2048, kw.get("sp", 4095), 0.04, kw.get("dt", 1),
+                         kw.get("out", FAKE), NULL, FAKE, 1 << 30, NULL]
+    assert L.dsa_sparse_mla_attn(*base(dc=500)) == dsa.DSA_ERR_UNSUPPORTED
+    assert L.dsa_sparse_mla_attn(*base(dc=512, dr=128)) == dsa.DSA_ERR_UNSUPPORTED
+    assert L.dsa_sparse_mla_attn(*base(dt=5)) == dsa.DSA_ERR_INVALID_ARG
+    assert L.dsa_sparse_mla_attn(*base(sp=4096)) == dsa.DSA_ERR_INVALID_ARG
+    assert L.dsa_sparse_mla_attn(*base(out=ODD)) == dsa.DSA_ERR_INVALID_ARG
+
+
+def test_decode_step_argument_checks(dsa):
+    L = dsa._lib
+    need = L.dsa_decode_step_workspace_size(8, 64, 128, 131072, 2048, 128, 512, 64, 1)
+    assert need >= 8 * 64 * 128 + 8 * 64 * 4
+    def call(**kw):
+        return L.dsa_decode_step(FAKE, FAKE, FAKE, FAKE, FAKE, kw.get("t_max", 131072), FAKE,
+                                 FAKE, 8, 64, kw.get("D", 128), 128, 512, 64, kw.get("T", 131072),
+                                 2048, 0.088, 0.041, 1, FAKE, FAKE, NULL, kw.get("ws", FAKE),
+                                 kw.get("ws_bytes", need), NULL)
+    assert call(D=96) == dsa.DSA_ERR_UNSUPPORTED
+    assert call(T=131073) == dsa.DSA_ERR_INVALID_ARG
+    assert call(T=0) == dsa.DSA_ERR_INVALID_ARG
+    assert call(ws_bytes=need - 1) == dsa.DSA_ERR_WORKSPACE
+    assert call(ws=NULL) == dsa.DSA_ERR_WORKSPACE

@@ -1,0 +1,91 @@
+"""The fused decode step on the GPU vs the oracle's decode pass, sequence by sequence."""
+import dataclasses
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import workloads
+from gpu_pipelines import decode_batch, run_decode
+from parity import assert_attention_close, assert_selection_matches
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def dsa():
+    import top_kv_selection_b200 as m
+    return m
+
+
+def _check_sequence(wl, seq, state, b, T):
+    r = oracle.decode_step(seq["q_idx"].numpy(), seq["w"].numpy(), seq["keys"].numpy(),
+                           seq["q_mla"].float().numpy(), seq["kv"].float().numpy(), topk=wl.topk,
+                           softmax_scale_idx=wl.softmax_scale_idx, sm_scale=wl.sm_scale, dc=wl.dc)
+    # the appended key
+    assert np.array_equal(state["k_cache"][b, T - 1].cpu().numpy(), r["k_fp8"][T - 1])
+    assert state["k_scale"][b, T - 1].item() == r["k_scale"][T - 1]
+    assert_selection_matches(state["idx"][b].cpu().numpy(), r["idx"], r["scores"])
+    assert_attention_close(state["out"][b].float().cpu().numpy(), r["out"], wl.attn_dtype,
+                           state["lse"][b].cpu().numpy(), r["lse"])
+    return r
+
+
+@pytest.mark.parametrize("cfg,T,B", [
+    (1, 5000, 2),      # V3.2 shapes, ragged context
+    (1, 1, 1),         # a single token: K = 1
+    (1, 2048, 2),      # T == k: every position
+    (1, 700, 1),       # T < k: padded with -1? no: K = min(k, T) = T slots, all filled
+    (0, 300, 2),       # tiny heads, fp32 test mode
+])
+def test_decode_step_small(dsa, cfg, T, B):
+    wl = workloads.WORKLOADS[cfg]
+    if cfg == 0:
+        wl = dataclasses.replace(wl, mode="decode")
+    seqs, st = decode_batch(dsa, wl, T=T, B=B)
+    for b in range(B):
+        _check_sequence(wl, seqs[b], st, b, T)
+    assert dsa.dsa_get_device_error() == 0
+
+
+def test_decode_step_cache_capacity_larger_than_context(dsa):
+    wl = workloads.WORKLOADS[1]
+    seqs, st = decode_batch(dsa, wl, T=3000, B=2, t_max=4096)
+    for b in range(2):
+        _check_sequence(wl, seqs[b], st, b, 3000)
+
+
+def test_decode_step_v32_4k_full(dsa):
+    wl = workloads.WORKLOADS[1]
+    seqs, st = decode_batch(dsa, wl)
+    _check_sequence(wl, seqs[0], st, 0, wl.T)
+
+
+def test_decode_step_batched_32k_sampled(dsa):
+    wl = workloads.WORKLOADS[2]
+    seqs, st = decode_batch(dsa, wl)
+    for b in (0, 17, 31):
+        _check_sequence(wl, seqs[b], st, b, wl.T)
+
+
+def test_decode_step_long_context_128k(dsa):
+    """B = 8 at 131072 tokens with 1% planted keys: every planted position is
+    selected in every sequence; two sequences compared in full with the oracle."""
+    wl = workloads.WORKLOADS[4]
+    seqs, st = decode_batch(dsa, wl)
+    idx = st["idx"].cpu().numpy()
+    for b in range(wl.B):
+        assert np.isin(seqs[b]["planted"].numpy(), idx[b]).all()
+        assert len(np.unique(idx[b])) == wl.topk and (idx[b] >= 0).all()
+    for b in (0, 7):
+        _check_sequence(wl, seqs[b], st, b, wl.T)
+
+
+def test_decode_step_deterministic(dsa):
+    wl = workloads.WORKLOADS[1]
+    seqs, st = decode_batch(dsa, wl, T=6000, B=2)
+    idx1, out1 = st["idx"].clone(), st["out"].clone()
+    run_decode(dsa, wl, st)
+    torch.cuda.synchronize()
+    assert torch.equal(idx1, st["idx"]) and torch.equal(out1, st["out"])

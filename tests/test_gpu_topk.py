@@ -1,0 +1,83 @@
+"""Top-k selection on the GPU: identical to the oracle when both see the same fp32 scores."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import workloads
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def dsa():
+    import top_kv_selection_b200 as m
+    return m
+
+
+def _gpu_topk(dsa, scores, start_pos, k):
+    B, S, T = scores.shape
+    K = min(k, T)
+    sc = torch.from_numpy(np.ascontiguousarray(scores)).cuda()
+    idx = torch.empty(B, S, K, dtype=torch.int32, device="cuda")
+    need = dsa.dsa_topk_select_workspace_size(B, S, T, k)
+    ws = torch.empty(max(need, 1), dtype=torch.uint8, device="cuda")
+    dsa.dsa_topk_select(sc, start_pos, k, idx, ws)
+    return idx.cpu().numpy()
+
+
+@pytest.mark.parametrize("B,S,T,sp,k,ties", [
+    (1, 1, 4096, 4095, 2048, 0.0),       # V3.2 decode, 4K context
+    (4, 1, 5003, 5002, 2048, 0.0),       # ragged
+    (2, 1, 1500, 1499, 2048, 0.0),       # T < k: everything selected
+    (2, 1, 2048, 2047, 2048, 0.0),       # T == k
+    (3, 1, 9000, 8999, 2048, 0.3),       # many exact ties, also at the boundary
+    (1, 1, 3000, 2999, 1, 0.0),          # k = 1
+    (1, 64, 64, 0, 16, 0.0),             # prefill causal rows, short rows padded with -1
+    (1, 40, 600, 560, 100, 0.1),         # query chunk with start_pos > 0
+])
+def test_topk_identical_to_oracle(dsa, B, S, T, sp, k, ties):
+    sc = workloads.score_rows(B * S, T, seed=T + k, tie_frac=ties).numpy().reshape(B, S, T)
+    got = _gpu_topk(dsa, sc, sp, k)
+    ref = oracle.topk_select(sc, sp, k)
+    assert np.array_equal(got, ref)
+
+
+def test_topk_special_values(dsa):
+    T = 3000
+    sc = workloads.score_rows(4, T, seed=9).numpy()
+    sc[0, ::3] = -np.inf                 # masked-looking entries inside the causal range
+    sc[1, :] = 0.0
+    sc[1, ::2] = -0.0                    # signed zeros tie
+    sc[2, :2500] = -np.inf               # fewer finite scores than k
+    sc[3] = np.abs(sc[3])                # all positive
+    sc = sc.reshape(4, 1, T)
+    got = _gpu_topk(dsa, sc, T - 1, 2048)
+    ref = oracle.topk_select(sc, T - 1, 2048)
+    assert np.array_equal(got, ref)
+
+
+def test_topk_long_context_rows(dsa):
+    """Rows of 131072 scores (the 128K decode) with k = 2048."""
+    T = 131072
+    sc = workloads.score_rows(8, T, seed=4).numpy().reshape(8, 1, T)
+    got = _gpu_topk(dsa, sc, T - 1, 2048)
+    ref = oracle.topk_select(sc, T - 1, 2048)
+    assert np.array_equal(got, ref)
+
+
+def test_topk_prefill_full_size_sampled_rows(dsa):
+    """8192 causal rows of 8192 scores, top-2048 each; rows compared one by one."""
+    T = 8192
+    sc = workloads.score_rows(T, T, seed=8).numpy().reshape(1, T, T)
+    got = _gpu_topk(dsa, sc, 0, 2048)
+    for s in (0, 1, 2046, 2047, 2048, 4000, 8191):
+        ref = oracle.topk_select(sc[:, s:s + 1], s, 2048)
+        assert np.array_equal(got[:, s:s + 1], ref)
+
+
+def test_topk_deterministic(dsa):
+    sc = workloads.score_rows(4, 20000, seed=11, tie_frac=0.2).numpy().reshape(4, 1, 20000)
+    a = _gpu_topk(dsa, sc, 19999, 2048)
+    b = _gpu_topk(dsa, sc, 19999, 2048)
+    assert np.array_equal(a, b)

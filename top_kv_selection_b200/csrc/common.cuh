@@ -1,0 +1,108 @@
+// common.cuh -- internal helpers shared by the libdsa CUDA sources.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+#include <cuda_fp8.h>
+#include <stdint.h>
+
+#include "dsa.h"
+
+namespace dsa {
+
+// ---------------------------------------------------------------- host side
+// Device pointer of the sticky error word of the current device (the word
+// lives in api.cu).  Returns nullptr if the runtime cannot resolve it.
+int *device_error_word();
+
+inline bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+inline dsa_status launch_status() {
+    return cudaGetLastError() == cudaSuccess ? DSA_OK : DSA_ERR_CUDA;
+}
+
+inline int num_sms() {
+    int dev = 0, n = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 148;
+    return n;
+}
+
+inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+// -------------------------------------------------------------- device side
+__device__ __forceinline__ void record_error(int *word, int code) {
+    if (word) atomicCAS(word, 0, code);
+}
+
+// Order-preserving map from an fp32 score to an unsigned key: a > b as floats
+// <=> key(a) > key(b).  -0 maps to the key of +0; NaN maps to 0, below -inf.
+__device__ __forceinline__ uint32_t score_key(float f) {
+    uint32_t u = __float_as_uint(f);
+    if ((u & 0x7fffffffu) > 0x7f800000u) return 0u;   // NaN
+    if ((u & 0x7fffffffu) == 0u) u = 0u;              // -0 -> +0
+    return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    return v;
+}
+
+__device__ __forceinline__ float warp_max(float v) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+    return v;
+}
+
+// e4m3 code -> fp32 (exact).
+__device__ __forceinline__ float e4m3_to_f32(uint8_t c) {
+    __nv_fp8_e4m3 v;
+    v.__x = c;
+    return static_cast<float>(v);
+}
+
+// Four packed e4m3 codes (little-endian in a 32-bit word) -> fp32.
+__device__ __forceinline__ void e4m3x4_to_f32(uint32_t w, float &a, float &b, float &c, float &d) {
+    __nv_fp8x2_e4m3 lo, hi;
+    lo.__x = static_cast<__nv_fp8x2_storage_t>(w & 0xffffu);
+    hi.__x = static_cast<__nv_fp8x2_storage_t>(w >> 16);
+    float2 l = static_cast<float2>(lo);
+    float2 h = static_cast<float2>(hi);
+    a = l.x; b = l.y; c = h.x; d = h.y;
+}
+
+template <typename T> __device__ __forceinline__ float to_f32(T v);
+template <> __device__ __forceinline__ float to_f32<float>(float v) { return v; }
+template <> __device__ __forceinline__ float to_f32<__nv_bfloat16>(__nv_bfloat16 v) {
+    return __bfloat162float(v);
+}
+
+template <typename T> __device__ __forceinline__ T from_f32(float v);
+template <> __device__ __forceinline__ float from_f32<float>(float v) { return v; }
+template <> __device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(float v) {
+    return __float2bfloat16_rn(v);
+}
+
+// ------------------------------------------------ internal launchers (no checks)
+dsa_status launch_indexer_quant(const void *x, dsa_dtype x_dtype, int64_t n_rows, int64_t n_vec,
+                                int d, uint8_t *out_fp8, int64_t out_row_stride, float *out_scale,
+                                int64_t scale_row_stride, cudaStream_t stream);
+
+dsa_status launch_index_scores(const uint8_t *q_fp8, const float *q_scale, const float *w,
+                               const uint8_t *k_cache, const float *k_scale, int64_t t_max, int B,
+                               int S, int H, int D, int64_t start_pos, int64_t T,
+                               float softmax_scale, float *scores, cudaStream_t stream);
+
+size_t topk_workspace_bytes(int B, int S, int64_t T, int k);
+dsa_status launch_topk_select(const float *scores, int B, int S, int64_t T, int64_t start_pos,
+                              int k, int32_t *idx, void *ws, cudaStream_t stream);
+
+size_t sparse_mla_workspace_bytes(int B, int S, int Hq, int dc, int dr, int k, dsa_dtype dt);
+dsa_status launch_sparse_mla(const void *q, const void *kv, int64_t t_max, const int32_t *idx,
+                             int B, int S, int Hq, int dc, int dr, int k, int64_t start_pos,
+                             float sm_scale, dsa_dtype dt, void *out, float *lse, void *ws,
+                             cudaStream_t stream);
+
+}  // namespace dsa

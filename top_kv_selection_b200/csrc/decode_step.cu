@@ -1,0 +1,93 @@
+// decode_step.cu -- one DSA decode step for a batch of sequences.
+//
+// Order of Indexer.forward ("DeepSeek-V3.2-Exp - Split indexer heads") with
+// seqlen == 1 (no mask, "DeepSeek-V3.2-Exp - Causal mask"), followed by the
+// diagram's sparse core attention in MQA mode:
+//   rotate+quantise q and k_new, append k_new at T-1, fp8_index over the T
+//   cached keys, top-min(index_topk, T), sparse latent attention.
+// Everything is enqueued on one stream; nothing synchronises with the host.
+#include "common.cuh"
+
+namespace dsa {
+namespace {
+
+struct DecodeWs {
+    uint8_t *q_fp8;    // [B,H,D]
+    float *q_scale;    // [B,H]
+    float *scores;     // [B,T]
+    void *topk_ws;
+    void *attn_ws;
+    size_t total;
+};
+
+DecodeWs carve(void *base, int B, int H, int D, int64_t T, int index_topk, int Hq, int dc, int dr,
+               dsa_dtype dt) {
+    DecodeWs w{};
+    size_t off = 0;
+    char *p = static_cast<char *>(base);
+    auto take = [&](size_t bytes) {
+        char *r = p ? p + off : nullptr;
+        off = align_up(off + bytes, 256);
+        return r;
+    };
+    w.q_fp8 = reinterpret_cast<uint8_t *>(take((size_t)B * H * D));
+    w.q_scale = reinterpret_cast<float *>(take((size_t)B * H * sizeof(float)));
+    w.scores = reinterpret_cast<float *>(take((size_t)B * T * sizeof(float)));
+    w.topk_ws = take(topk_workspace_bytes(B, 1, T, index_topk));
+    const int K = (int64_t)index_topk < T ? index_topk : (int)T;
+    w.attn_ws = take(sparse_mla_workspace_bytes(B, 1, Hq, dc, dr, K, dt));
+    w.total = off;
+    return w;
+}
+
+}  // namespace
+}  // namespace dsa
+
+extern "C" size_t dsa_decode_step_workspace_size(int B, int H, int D, int64_t T, int index_topk,
+                                                 int Hq, int dc, int dr, dsa_dtype dt) {
+    if (B <= 0 || H <= 0 || T <= 0 || index_topk <= 0) return 0;
+    return dsa::carve(nullptr, B, H, D, T, index_topk, Hq, dc, dr, dt).total;
+}
+
+extern "C" dsa_status dsa_decode_step(const float *q_idx, const float *w, const float *k_new,
+                                      uint8_t *k_cache, float *k_scale, int64_t t_max,
+                                      const void *kv_cache, const void *q_mla, int B, int H,
+                                      int D, int Hq, int dc, int dr, int64_t T, int index_topk,
+                                      float softmax_scale, float sm_scale, dsa_dtype dt,
+                                      int32_t *idx, void *out, float *lse, void *workspace,
+                                      size_t workspace_bytes, dsa_stream_t stream) {
+    if (B < 0 || H < 1 || Hq < 1 || index_topk < 1 || T < 1 || T > t_max || T > INT32_MAX)
+        return DSA_ERR_INVALID_ARG;
+    if (dt != DSA_F32 && dt != DSA_BF16) return DSA_ERR_INVALID_ARG;
+    if (D != 64 && D != 128) return DSA_ERR_UNSUPPORTED;
+    if (H > 256) return DSA_ERR_UNSUPPORTED;
+    if (dc == 0 || dc % 32 != 0 || dc > 512 || dr < 0 || dr % 8 != 0 || dc + dr > 576)
+        return DSA_ERR_UNSUPPORTED;
+    if (B == 0) return DSA_OK;
+    if (!q_idx || !w || !k_new || !k_cache || !k_scale || !kv_cache || !q_mla || !idx || !out)
+        return DSA_ERR_INVALID_ARG;
+    if (!dsa::aligned16(q_idx) || !dsa::aligned16(k_new) || !dsa::aligned16(k_cache) ||
+        !dsa::aligned16(kv_cache) || !dsa::aligned16(q_mla) || !dsa::aligned16(out) ||
+        ((t_max * D) & 15))
+        return DSA_ERR_INVALID_ARG;
+    const dsa::DecodeWs ws = dsa::carve(workspace, B, H, D, T, index_topk, Hq, dc, dr, dt);
+    if (!workspace || workspace_bytes < ws.total || !dsa::aligned16(workspace))
+        return DSA_ERR_WORKSPACE;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    dsa_status st;
+    if ((st = dsa::launch_indexer_quant(q_idx, DSA_F32, 1, (int64_t)B * H, D, ws.q_fp8, 0,
+                                        ws.q_scale, 0, s)) != DSA_OK)
+        return st;
+    if ((st = dsa::launch_indexer_quant(k_new, DSA_F32, B, 1, D, k_cache + (T - 1) * D,
+                                        t_max * D, k_scale + (T - 1), t_max, s)) != DSA_OK)
+        return st;
+    if ((st = dsa::launch_index_scores(ws.q_fp8, ws.q_scale, w, k_cache, k_scale, t_max, B, 1, H,
+                                       D, T - 1, T, softmax_scale, ws.scores, s)) != DSA_OK)
+        return st;
+    if ((st = dsa::launch_topk_select(ws.scores, B, 1, T, T - 1, index_topk, idx, ws.topk_ws,
+                                      s)) != DSA_OK)
+        return st;
+    const int K = (int64_t)index_topk < T ? index_topk : (int)T;
+    return dsa::launch_sparse_mla(q_mla, kv_cache, t_max, idx, B, 1, Hq, dc, dr, K, T - 1,
+                                  sm_scale, dt, out, lse, ws.attn_ws, s);
+}
