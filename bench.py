@@ -22,7 +22,6 @@ import argparse
 import json
 import os
 import statistics
-import subprocess
 import sys
 import time
 
@@ -83,54 +82,67 @@ def _max_over_ranks(world, value: float) -> float:
 # clocks sampled during the timed region
 # --------------------------------------------------------------------------- #
 class ClockSampler:
-    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
-             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    """Polls NVML (SM clock, max SM clock, clock-event reasons) in a background
+    thread for as long as the context is open; open it around the timed region."""
+    REASONS = {0x4: "sw_power_cap", 0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown",
+               0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown"}
 
     def __init__(self, device_index: int):
         self.dev = device_index
-        self.proc = None
+        self.samples = []
+        self.max_mhz = None
+        self._stop = False
+        self._thread = None
+
+    def _handle(self):
+        import pynvml
+        pynvml.nvmlInit()
+        p = torch.cuda.get_device_properties(self.dev)
+        try:
+            bus = f"{p.pci_domain_id:08X}:{p.pci_bus_id:02X}:{p.pci_device_id:02X}.0"
+            return pynvml.nvmlDeviceGetHandleByPciBusId(bus)
+        except Exception:
+            return pynvml.nvmlDeviceGetHandleByIndex(self.dev)
+
+    def _run(self, h):
+        import pynvml
+        while not self._stop:
+            try:
+                clk = pynvml.nvmlDeviceGetClockInfo(h, pynvml.NVML_CLOCK_SM)
+                rs = pynvml.nvmlDeviceGetCurrentClocksEventReasons(h)
+                self.samples.append((clk, rs))
+            except Exception:
+                break
+            time.sleep(0.001)
 
     def __enter__(self):
+        import threading
         try:
-            self.proc = subprocess.Popen(
-                ["nvidia-smi", "-i", str(self.dev), f"--query-gpu={self.QUERY}",
-                 "--format=csv,noheader,nounits", "-lms", "100"],
-                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
-        except OSError:
-            self.proc = None
+            import pynvml
+            h = self._handle()
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(h, pynvml.NVML_CLOCK_SM)
+            self._thread = threading.Thread(target=self._run, args=(h,), daemon=True)
+            self._thread.start()
+        except Exception:
+            self._thread = None
         return self
 
     def __exit__(self, *exc):
-        self.lines = []
-        if self.proc is not None:
-            self.proc.terminate()
-            try:
-                out, _ = self.proc.communicate(timeout=5)
-            except subprocess.TimeoutExpired:
-                self.proc.kill()
-                out, _ = self.proc.communicate()
-            self.lines = [l for l in out.splitlines() if l.strip()]
+        self._stop = True
+        if self._thread is not None:
+            self._thread.join(timeout=5)
 
     def summary(self):
-        sm, mx, reasons = [], [], set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for line in getattr(self, "lines", []):
-            f = [x.strip() for x in line.split(",")]
-            if len(f) < 9:
-                continue
-            try:
-                sm.append(float(f[1]))
-                mx.append(float(f[2]))
-            except ValueError:
-                continue
-            for n, v in zip(names, f[5:9]):
-                if v.lower().startswith("active"):
-                    reasons.add(n)
-        if not sm:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
-        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx),
-                "reasons": sorted(reasons), "samples": len(sm)}
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": [], "samples": 0}
+        reasons = set()
+        for _, rs in self.samples:
+            for bit, name in self.REASONS.items():
+                if rs & bit:
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(c for c, _ in self.samples),
+                "sm_max_mhz": self.max_mhz, "reasons": sorted(reasons),
+                "samples": len(self.samples), "source": "nvml"}
 
 
 # --------------------------------------------------------------------------- #
@@ -285,8 +297,8 @@ def run_reference(args, wl, world, rank):
 # our arm
 # --------------------------------------------------------------------------- #
 def run_ours(args, wl, world, rank, local):
-    from top_kv_selection_b200 import build as _build
-    _build.build()
+    import __graft_entry__
+    __graft_entry__._builder().build()
     import top_kv_selection_b200 as dsa
 
     copies = build_state(dsa, wl, rank_seed_offset=0)
@@ -350,12 +362,12 @@ def run_ours(args, wl, world, rank, local):
         "clocks": clk.summary(),
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        times = oracle_decode_sample(wl, 2)
-        t_seq = sum(times) / len(times)
+        times = oracle_decode_sample(wl, wl.B)
+        t_step = sum(times)
         line["cpu_baseline"] = {
-            "value": 1.0 / (wl.B * t_seq), "unit": "steps/s", "cores": 1, "kind": "oracle",
-            "sample": f"sequences 0-1 of {wl.B}, one decode step each at T={wl.T} "
-                      f"({sum(times):.1f} s), extrapolated x{wl.B}; cache prebuilt"}
+            "value": 1.0 / t_step, "unit": "steps/s", "cores": 1, "kind": "oracle",
+            "sample": f"all {wl.B} sequences of one decode step at T={wl.T} "
+                      f"({t_step:.1f} s, single thread); caches prebuilt, untimed"}
     if world > 1:
         import torch.distributed as dist
         dist.barrier()
@@ -404,7 +416,7 @@ def run_e2e(dsa, wl, copies, args, world):
 def main(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--steps", type=int, default=2000)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", type=int, default=4)

@@ -13,8 +13,8 @@ HEADER = os.path.join(ROOT, "include", "dsa.h")
 
 @pytest.fixture(scope="module")
 def dsa():
-    from top_kv_selection_b200 import build
-    build.build()
+    import __graft_entry__
+    __graft_entry__._builder().build()
     import top_kv_selection_b200 as m
     return m
 

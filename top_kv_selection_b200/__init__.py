@@ -5,7 +5,7 @@ and only marshals arguments: torch tensors become device pointers, shapes
 become the integer arguments, the current torch stream becomes the stream
 argument.  Every computation runs in libdsa's CUDA kernels; there is no CPU or
 PyTorch fallback.  Importing the package fails if libdsa.so has not been built
-(``python -m top_kv_selection_b200.build``).
+(``python top_kv_selection_b200/build.py``).
 """
 from __future__ import annotations
 
@@ -19,7 +19,7 @@ LIB_PATH = os.path.join(_PKG, "libdsa.so")
 
 if not os.path.exists(LIB_PATH):
     raise ImportError(f"libdsa.so is not built at {LIB_PATH}; run "
-                      "`python -m top_kv_selection_b200.build`")
+                      "`python top_kv_selection_b200/build.py`")
 
 _lib = ctypes.CDLL(LIB_PATH)
 
@@ -189,3 +189,4 @@ def dsa_decode_step(q_idx: torch.Tensor, w: torch.Tensor, k_new: torch.Tensor,
         _ptr(q_mla), B, H, D, Hq, dc, dqk - dc, T, index_topk, softmax_scale, sm_scale,
         _dtype(q_mla), _ptr(idx), _ptr(out), _ptr(lse), _ptr(workspace),
         workspace.numel() * workspace.element_size(), _stream(stream)))
+

@@ -1,6 +1,8 @@
 """Build libdsa.so in-tree with nvcc for sm_100a.
 
-    python -m top_kv_selection_b200.build [--force] [--verbose]
+    python top_kv_selection_b200/build.py [--force] [--verbose]
+
+(run it by path: importing the package loads the library being rebuilt)
 
 Every ``csrc/*.cu`` is compiled separately (in parallel) and linked into
 ``top_kv_selection_b200/libdsa.so`` with the CUDA runtime linked statically, so
