@@ -181,6 +181,34 @@ dsa_status dsa_decode_step(const float *q_idx, const float *w, const float *k_ne
                            float sm_scale, dsa_dtype dt, int32_t *idx, void *out, float *lse,
                            void *workspace, size_t workspace_bytes, dsa_stream_t stream);
 
+/*
+ * The decode step without a workspace, for callers that cannot allocate device
+ * memory (a plugin living in another engine's memory pool, code launched while
+ * a CUDA graph owned by someone else is being captured, a host that links only
+ * this library).  The pages have no counterpart: this is a packaging variant
+ * of dsa_decode_step, with the same arguments minus the workspace and the same
+ * results.
+ *
+ * Scratch comes from a fixed device array of DSA_NOALLOC_SCRATCH_BYTES inside
+ * the library; every GPU that loads the library holds it until the process
+ * exits.  No call allocates or frees memory.  A problem whose
+ * dsa_decode_step_workspace_size() exceeds DSA_NOALLOC_SCRATCH_BYTES is
+ * rejected with DSA_ERR_WORKSPACE before anything is launched.
+ *   - The first call on a device resolves the array's device address (with
+ *     that device current); make that first call before any stream capture.
+ *   - All calls on a device share the one array and it keeps the previous
+ *     call's contents (nothing in it needs to start at zero).  Calls that
+ *     overlap on the GPU (other streams, other threads) race on it: serialise
+ *     them, e.g. by issuing them on one stream.
+ */
+#define DSA_NOALLOC_SCRATCH_BYTES (32u << 20)
+dsa_status dsa_decode_step_noalloc(const float *q_idx, const float *w, const float *k_new,
+                                   uint8_t *k_cache, float *k_scale, int64_t t_max,
+                                   const void *kv_cache, const void *q_mla, int B, int H, int D,
+                                   int Hq, int dc, int dr, int64_t T, int index_topk,
+                                   float softmax_scale, float sm_scale, dsa_dtype dt,
+                                   int32_t *idx, void *out, float *lse, dsa_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

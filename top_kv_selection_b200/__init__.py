@@ -26,6 +26,7 @@ _lib = ctypes.CDLL(LIB_PATH)
 DSA_OK, DSA_ERR_INVALID_ARG, DSA_ERR_UNSUPPORTED, DSA_ERR_CUDA = 0, 1, 2, 3
 DSA_ERR_TIMEOUT, DSA_ERR_DEVICE, DSA_ERR_WORKSPACE = 4, 5, 6
 DSA_F32, DSA_BF16 = 0, 1
+DSA_NOALLOC_SCRATCH_BYTES = 32 << 20
 
 _P, _i32, _i64, _f32, _sz = (ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_float,
                              ctypes.c_size_t)
@@ -46,6 +47,8 @@ _SIGNATURES = {
                                        _sz),
     "dsa_decode_step": ([_P, _P, _P, _P, _P, _i64, _P, _P, _i32, _i32, _i32, _i32, _i32, _i32,
                          _i64, _i32, _f32, _f32, _i32, _P, _P, _P, _P, _sz, _P], _i32),
+    "dsa_decode_step_noalloc": ([_P, _P, _P, _P, _P, _i64, _P, _P, _i32, _i32, _i32, _i32, _i32,
+                                 _i32, _i64, _i32, _f32, _f32, _i32, _P, _P, _P, _P], _i32),
 }
 
 for _name, (_args, _res) in _SIGNATURES.items():
@@ -190,3 +193,20 @@ def dsa_decode_step(q_idx: torch.Tensor, w: torch.Tensor, k_new: torch.Tensor,
         _dtype(q_mla), _ptr(idx), _ptr(out), _ptr(lse), _ptr(workspace),
         workspace.numel() * workspace.element_size(), _stream(stream)))
 
+
+def dsa_decode_step_noalloc(q_idx: torch.Tensor, w: torch.Tensor, k_new: torch.Tensor,
+                            k_cache: torch.Tensor, k_scale: torch.Tensor, kv_cache: torch.Tensor,
+                            q_mla: torch.Tensor, T: int, index_topk: int, softmax_scale: float,
+                            sm_scale: float, idx: torch.Tensor, out: torch.Tensor,
+                            lse: torch.Tensor | None, stream=None) -> None:
+    """dsa_decode_step without a workspace: for callers that cannot allocate device
+    memory, scratch comes from a fixed DSA_NOALLOC_SCRATCH_BYTES array inside libdsa
+    (shared by all calls on a device; calls overlapping on the GPU race)."""
+    B, H, D = q_idx.shape
+    Hq, dqk = q_mla.shape[1], q_mla.shape[2]
+    dc = out.shape[-1]
+    t_max = k_cache.shape[1]
+    _check("dsa_decode_step_noalloc", _lib.dsa_decode_step_noalloc(
+        _ptr(q_idx), _ptr(w), _ptr(k_new), _ptr(k_cache), _ptr(k_scale), t_max, _ptr(kv_cache),
+        _ptr(q_mla), B, H, D, Hq, dc, dqk - dc, T, index_topk, softmax_scale, sm_scale,
+        _dtype(q_mla), _ptr(idx), _ptr(out), _ptr(lse), _stream(stream)))
