@@ -81,3 +81,38 @@ def test_topk_deterministic(dsa):
     a = _gpu_topk(dsa, sc, 19999, 2048)
     b = _gpu_topk(dsa, sc, 19999, 2048)
     assert np.array_equal(a, b)
+
+
+@pytest.mark.parametrize("T", [20000, 40000, 70000, 300000, 700000])
+def test_topk_every_cluster_size_and_fallback(dsa, T):
+    """Row lengths that take 2, 4, 8 and 16 CTAs per row, and the one-CTA
+    global-memory kernel beyond that."""
+    sc = workloads.score_rows(2, T, seed=T % 997, tie_frac=0.05).numpy().reshape(2, 1, T)
+    got = _gpu_topk(dsa, sc, T - 1, 2048)
+    ref = oracle.topk_select(sc, T - 1, 2048)
+    assert np.array_equal(got, ref)
+
+
+def test_topk_outlier_and_flat_rows(dsa):
+    """A huge outlier squeezes every other score into one linear bin; a flat
+    row has no spread at all; both must still select exactly."""
+    T = 50000
+    sc = workloads.score_rows(3, T, seed=12).numpy()
+    sc[0, 777] = 3.0e38
+    sc[1, :] = 0.25
+    sc[2, 5] = -3.0e38
+    sc[2, 9] = np.inf
+    sc = sc.reshape(3, 1, T)
+    got = _gpu_topk(dsa, sc, T - 1, 2048)
+    ref = oracle.topk_select(sc, T - 1, 2048)
+    assert np.array_equal(got, ref)
+
+
+def test_topk_query_chunk_rows_of_different_lengths(dsa):
+    """S rows of a chunk share a cluster size but see different causal prefixes."""
+    B, S, T = 2, 6, 40000
+    sp = T - S
+    sc = workloads.score_rows(B * S, T, seed=13, tie_frac=0.02).numpy().reshape(B, S, T)
+    got = _gpu_topk(dsa, sc, sp, 2048)
+    ref = oracle.topk_select(sc, sp, 2048)
+    assert np.array_equal(got, ref)

@@ -5,70 +5,272 @@
 //   index_score = fp8_index(q_fp8, weights, k_cache, k_scale); index_score += mask
 // and the diagram's I(t,s) = sum_j w_j ReLU(q_j . k_s).
 //
-// General kernel: one CTA scores 128 consecutive tokens of one query row
-// (b, s); each thread owns one token, decodes its FP8 key into registers and
-// runs the per-head dot products against the query tile held in shared
-// memory (fp32, read as broadcasts).  The weight fold is computed once per CTA.
+// Tensor-core scorer (sm_100a).  One CTA owns a contiguous range of 128-token
+// tiles of one query row (b, s) and streams them once from HBM:
+//   warp 0      TMA producer: 128 x D FP8 key tiles (swizzled) into a ring of
+//               shared-memory stages, L2 evict-first;
+//   warp 1      allocates TMEM and issues tcgen05.mma kind::f8f6f4 with
+//               M = 128 tokens, N = heads (padded to 16), K = D in steps of 32,
+//               accumulating fp32 in a double-buffered TMEM tile;
+//   warps 2..5  epilogue: each thread owns one token (one TMEM lane), reads its
+//               N head dot products, and computes
+//               k_scale[t] * sum_h w'_h * max(dot_h, 0)  (ReLU, weighted head
+//               sum, key scale), storing one fp32 score per token.
+// The key cache is the only large operand: 132 bytes per token (D + 4).
 #include "common.cuh"
+#include "tc_ptx.cuh"
+#include "tmap.cuh"
 
 namespace dsa {
 namespace {
 
-constexpr int kTokPerCta = 128;
+constexpr int kTile = 128;       // tokens per tile = MMA M
+constexpr int kStages = 6;       // key-tile ring depth
+constexpr int kAcc = 2;          // TMEM accumulator buffers
+constexpr int kThreads = 192;    // warp 0 TMA, warp 1 MMA, warps 2..5 epilogue
+constexpr int kMaxHeads = 256;
+
+struct ScoreArgs {
+    const uint8_t *q_fp8;
+    const float *q_scale;
+    const float *w;
+    const float *k_scale;
+    float *scores;
+    int64_t t_max;
+    int64_t start_pos;
+    int64_t T;
+    int S, H, NH, chunks;
+    uint32_t tmem_cols;
+    float head_scale, softmax_scale;
+    int *err;
+};
+
+template <int D> struct KSwizzle;
+template <> struct KSwizzle<128> {
+    static constexpr tc::Swizzle kind = tc::kSwizzle128B;
+    static constexpr uint32_t sbo = 1024;    // 8 rows x 128 B
+    __device__ static int chunk(int row, int c) { return c ^ (row & 7); }
+};
+template <> struct KSwizzle<64> {
+    static constexpr tc::Swizzle kind = tc::kSwizzle64B;
+    static constexpr uint32_t sbo = 512;     // 8 rows x 64 B
+    __device__ static int chunk(int row, int c) { return c ^ ((row >> 1) & 3); }
+};
 
 template <int D>
-__global__ void __launch_bounds__(kTokPerCta)
-index_scores_simt_kernel(const uint8_t *__restrict__ q_fp8, const float *__restrict__ q_scale,
-                         const float *__restrict__ w, const uint8_t *__restrict__ k_cache,
-                         const float *__restrict__ k_scale, int64_t t_max, int S, int H,
-                         int64_t start_pos, int64_t T, float head_scale, float softmax_scale,
-                         float *__restrict__ scores) {
-    extern __shared__ float smem[];
-    float *qs = smem;                 // [H][D] decoded query codes
-    float *wf = smem + H * D;         // [H] folded weights
-    const int64_t row = blockIdx.x;   // b * S + s
-    const int64_t b = row / S, s = row - b * S;
-    const uint8_t *qrow = q_fp8 + row * H * D;
-    for (int i = threadIdx.x; i < H * D; i += blockDim.x) qs[i] = e4m3_to_f32(qrow[i]);
-    for (int h = threadIdx.x; h < H; h += blockDim.x) {
-        float t = __fmul_rn(w[row * H + h], head_scale);
-        t = __fmul_rn(t, q_scale[row * H + h]);
-        wf[h] = __fmul_rn(t, softmax_scale);
-    }
-    __syncthreads();
+__host__ __device__ constexpr size_t score_smem_bytes(int NH) {
+    return 1024 + (size_t)kStages * kTile * D + (size_t)NH * D + kMaxHeads * sizeof(float) +
+           (2 * kStages + 2 * kAcc) * sizeof(uint64_t) + 16;
+}
 
-    const int64_t t = (int64_t)blockIdx.y * kTokPerCta + threadIdx.x;
-    if (t >= T) return;
-    float *dst = scores + row * T + t;
-    if (t > start_pos + s) {
-        *dst = -INFINITY;
-        return;
-    }
-    float kf[D];
-    const uint4 *krow = reinterpret_cast<const uint4 *>(k_cache + (b * t_max + t) * D);
-#pragma unroll
-    for (int c = 0; c < D / 16; c++) {
-        uint4 v = __ldg(krow + c);
-        e4m3x4_to_f32(v.x, kf[16 * c + 0], kf[16 * c + 1], kf[16 * c + 2], kf[16 * c + 3]);
-        e4m3x4_to_f32(v.y, kf[16 * c + 4], kf[16 * c + 5], kf[16 * c + 6], kf[16 * c + 7]);
-        e4m3x4_to_f32(v.z, kf[16 * c + 8], kf[16 * c + 9], kf[16 * c + 10], kf[16 * c + 11]);
-        e4m3x4_to_f32(v.w, kf[16 * c + 12], kf[16 * c + 13], kf[16 * c + 14], kf[16 * c + 15]);
-    }
-    float acc = 0.f;
-    for (int h = 0; h < H; h++) {
-        const float4 *qh = reinterpret_cast<const float4 *>(qs + h * D);
-        float dot = 0.f;
-#pragma unroll
-        for (int d4 = 0; d4 < D / 4; d4++) {
-            float4 q4 = qh[d4];
-            dot = fmaf(q4.x, kf[4 * d4 + 0], dot);
-            dot = fmaf(q4.y, kf[4 * d4 + 1], dot);
-            dot = fmaf(q4.z, kf[4 * d4 + 2], dot);
-            dot = fmaf(q4.w, kf[4 * d4 + 3], dot);
+template <int D>
+__global__ void __launch_bounds__(kThreads)
+score_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const ScoreArgs a) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t *sk = smem;
+    uint8_t *sq = sk + kStages * kTile * D;
+    float *wf = reinterpret_cast<float *>(sq + a.NH * D);
+    uint64_t *full = reinterpret_cast<uint64_t *>(wf + kMaxHeads);
+    uint64_t *empty = full + kStages;
+    uint64_t *accf = empty + kStages;
+    uint64_t *acce = accf + kAcc;
+    uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(acce + kAcc);
+    volatile int *abort = reinterpret_cast<volatile int *>(tmem_holder + 1);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int64_t row = blockIdx.x / a.chunks;
+    const int chunk = blockIdx.x - (int)(row * a.chunks);
+    const int64_t b = row / a.S, s = row - b * a.S;
+    const int64_t limit = a.start_pos + s;
+    const int64_t n_vis = a.T < limit + 1 ? a.T : limit + 1;
+    const int64_t n_tiles = (n_vis + kTile - 1) / kTile;
+    const int64_t tile_lo = chunk * n_tiles / a.chunks;
+    const int64_t tile_hi = (chunk + 1) * n_tiles / a.chunks;
+    const int n_my = (int)(tile_hi - tile_lo);
+
+    // causally masked positions of this row (prefill only), shared by the chunks
+    for (int64_t t = n_vis + (int64_t)chunk * kThreads + threadIdx.x; t < a.T;
+         t += (int64_t)a.chunks * kThreads)
+        a.scores[row * a.T + t] = -INFINITY;
+    if (n_my <= 0) return;
+
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < kStages; i++) {
+            tc::mbar_init(&full[i], 1);
+            tc::mbar_init(&empty[i], 1);
         }
-        acc = fmaf(wf[h], fmaxf(dot, 0.f), acc);
+        for (int i = 0; i < kAcc; i++) {
+            tc::mbar_init(&accf[i], 1);
+            tc::mbar_init(&acce[i], 4 * 32);
+        }
+        *abort = 0;
+        tc::fence_mbar_init();
+        tc::tma_prefetch_desc(&tmap_k);
     }
-    *dst = k_scale[b * t_max + t] * acc;
+    if (warp == 1) {
+        tc::tmem_alloc(tmem_holder, a.tmem_cols);
+        tc::tmem_relinquish();
+    }
+    // query codes of this row -> K-major swizzled tile (padded heads are zero)
+    constexpr int kChunks = D / 16;
+    const uint8_t *qrow = a.q_fp8 + row * a.H * D;
+    for (int i = threadIdx.x; i < a.NH * kChunks; i += kThreads) {
+        const int h = i / kChunks, c = i - h * kChunks;
+        uint4 v = make_uint4(0, 0, 0, 0);
+        if (h < a.H) v = *reinterpret_cast<const uint4 *>(qrow + h * D + c * 16);
+        *reinterpret_cast<uint4 *>(sq + h * D + KSwizzle<D>::chunk(h, c) * 16) = v;
+    }
+    // weight fold: w' = ((w * H^-1/2) * q_scale) * softmax_scale, fp32, in that order
+    for (int h = threadIdx.x; h < kMaxHeads; h += kThreads) {
+        float t = 0.f;
+        if (h < a.H) {
+            t = __fmul_rn(a.w[row * a.H + h], a.head_scale);
+            t = __fmul_rn(t, a.q_scale[row * a.H + h]);
+            t = __fmul_rn(t, a.softmax_scale);
+        }
+        wf[h] = t;
+    }
+    tc::fence_proxy_async_smem();
+    tc::tc_fence_before();
+    __syncthreads();
+    tc::tc_fence_after();
+    const uint32_t tmem_base = *tmem_holder;
+
+    if (warp == 0) {
+        if (lane == 0) {
+            const uint64_t pol = tc::l2_evict_first_policy();
+            int issued = 0;
+            for (int i = 0; i < n_my; i++) {
+                const int st = i % kStages;
+                const uint32_t ph = (uint32_t)(i / kStages) & 1u;
+                if (!tc::mbar_wait(&empty[st], ph ^ 1u, a.err, abort)) break;
+                tc::mbar_arrive_expect_tx(&full[st], kTile * D);
+                tc::tma_load_3d(sk + st * kTile * D, &tmap_k, 0, (int)((tile_lo + i) * kTile),
+                                (int)b, &full[st], pol);
+                issued = i + 1;
+            }
+            // wait (bounded) for the last loads still landing in shared memory
+            for (int j = issued > kStages ? issued - kStages : 0; j < issued; j++)
+                tc::mbar_wait(&full[j % kStages], (uint32_t)(j / kStages) & 1u, a.err, abort);
+        }
+    } else if (warp == 1) {
+        if (lane == 0) {
+            const uint32_t idesc = tc::instr_desc(tc::kFmtE4M3, tc::kFmtE4M3, kTile, a.NH);
+            const uint32_t sk_addr = tc::smem_u32(sk), sq_addr = tc::smem_u32(sq);
+            for (int i = 0; i < n_my; i++) {
+                const int st = i % kStages, ac = i % kAcc;
+                if (!tc::mbar_wait(&full[st], (uint32_t)(i / kStages) & 1u, a.err, abort)) break;
+                if (!tc::mbar_wait(&acce[ac], ((uint32_t)(i / kAcc) & 1u) ^ 1u, a.err, abort))
+                    break;
+                tc::tc_fence_after();
+                const uint32_t d_tmem = tmem_base + (uint32_t)(ac * a.NH);
+#pragma unroll
+                for (int k = 0; k < D / 32; k++) {
+                    const uint64_t ad = tc::smem_desc(sk_addr + st * kTile * D + k * 32,
+                                                      KSwizzle<D>::sbo, KSwizzle<D>::kind);
+                    const uint64_t bd =
+                        tc::smem_desc(sq_addr + k * 32, KSwizzle<D>::sbo, KSwizzle<D>::kind);
+                    tc::mma_f8f6f4(d_tmem, ad, bd, idesc, k > 0);
+                }
+                tc::tc_commit(&empty[st]);
+                tc::tc_commit(&accf[ac]);
+            }
+        }
+    } else {
+        const int quarter = warp & 3;                 // TMEM lanes this warp may read
+        const int tok = quarter * 32 + lane;          // token within the tile
+        const uint32_t lane_addr = (uint32_t)(quarter * 32) << 16;
+        const float *ks_row = a.k_scale + b * a.t_max;
+        float *out = a.scores + row * a.T;
+        for (int i = 0; i < n_my; i++) {
+            const int ac = i % kAcc;
+            const int64_t t = (tile_lo + i) * kTile + tok;
+            const float ks = t < n_vis ? __ldg(ks_row + t) : 0.f;
+            if (!tc::mbar_wait(&accf[ac], (uint32_t)(i / kAcc) & 1u, a.err, abort)) break;
+            tc::tc_fence_after();
+            const uint32_t taddr = tmem_base + lane_addr + (uint32_t)(ac * a.NH);
+            float acc = 0.f;
+            for (int c0 = 0; c0 < a.NH; c0 += 64) {
+                uint32_t r[4][16];
+#pragma unroll
+                for (int j = 0; j < 4; j++)
+                    if (c0 + 16 * j < a.NH) tc::tmem_ld16(taddr + c0 + 16 * j, r[j]);
+                tc::tmem_wait_ld();
+#pragma unroll
+                for (int j = 0; j < 4; j++) {
+                    if (c0 + 16 * j >= a.NH) break;
+#pragma unroll
+                    for (int e = 0; e < 16; e++)
+                        acc = fmaf(wf[c0 + 16 * j + e], fmaxf(__uint_as_float(r[j][e]), 0.f), acc);
+                }
+            }
+            tc::tc_fence_before();
+            tc::mbar_arrive(&acce[ac]);
+            if (t < n_vis) out[t] = ks * acc;
+        }
+    }
+
+    tc::tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc::tc_fence_after();
+        tc::tmem_dealloc(tmem_base, a.tmem_cols);
+    }
+}
+
+uint32_t pow2_cols(int n) {
+    uint32_t c = 32;
+    while (c < (uint32_t)n) c <<= 1;
+    return c;
+}
+
+template <int D>
+dsa_status launch_tc(const uint8_t *q_fp8, const float *q_scale, const float *w,
+                     const uint8_t *k_cache, const float *k_scale, int64_t t_max, int B, int S,
+                     int H, int64_t start_pos, int64_t T, float softmax_scale, float *scores,
+                     cudaStream_t stream) {
+    CUtensorMap tmap;
+    const uint64_t dims[3] = {(uint64_t)D, (uint64_t)t_max, (uint64_t)B};
+    const uint64_t strides[2] = {(uint64_t)D, (uint64_t)t_max * D};
+    const uint32_t box[3] = {(uint32_t)D, (uint32_t)kTile, 1};
+    const CUtensorMapSwizzle swz =
+        D == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
+    if (!encode_tmap(&tmap, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, k_cache, dims, strides, box, swz))
+        return DSA_ERR_CUDA;
+
+    ScoreArgs a;
+    a.q_fp8 = q_fp8;
+    a.q_scale = q_scale;
+    a.w = w;
+    a.k_scale = k_scale;
+    a.scores = scores;
+    a.t_max = t_max;
+    a.start_pos = start_pos;
+    a.T = T;
+    a.S = S;
+    a.H = H;
+    a.NH = (H + 15) / 16 * 16;
+    a.tmem_cols = pow2_cols(kAcc * a.NH);
+    a.head_scale = (float)(1.0 / sqrt((double)H));
+    a.softmax_scale = softmax_scale;
+    a.err = device_error_word();
+
+    const size_t smem = score_smem_bytes<D>(a.NH);
+    const int per_sm = smem * 2 <= 227 * 1024 && a.tmem_cols <= 256 ? 2 : 1;
+    const int64_t rows = (int64_t)B * S;
+    const int64_t vis_max = T < start_pos + S ? T : start_pos + S;
+    const int64_t max_tiles = (vis_max + kTile - 1) / kTile;
+    int64_t chunks = (int64_t)num_sms() * per_sm / rows;
+    if (chunks > max_tiles) chunks = max_tiles;
+    if (chunks < 1) chunks = 1;
+    a.chunks = (int)chunks;
+    if (cudaFuncSetAttribute(score_tc_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)smem) != cudaSuccess)
+        return DSA_ERR_CUDA;
+    score_tc_kernel<D><<<(unsigned)(rows * chunks), kThreads, smem, stream>>>(tmap, a);
+    return launch_status();
 }
 
 }  // namespace
@@ -78,23 +280,11 @@ dsa_status launch_index_scores(const uint8_t *q_fp8, const float *q_scale, const
                                int S, int H, int D, int64_t start_pos, int64_t T,
                                float softmax_scale, float *scores, cudaStream_t stream) {
     if ((int64_t)B * S * T == 0) return DSA_OK;
-    const float head_scale = (float)(1.0 / sqrt((double)H));
-    const size_t smem = (size_t)H * D * sizeof(float) + (size_t)H * sizeof(float);
-    dim3 grid((unsigned)(B * S), (unsigned)((T + kTokPerCta - 1) / kTokPerCta));
-    if (D == 128) {
-        cudaFuncSetAttribute(index_scores_simt_kernel<128>,
-                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        index_scores_simt_kernel<128><<<grid, kTokPerCta, smem, stream>>>(
-            q_fp8, q_scale, w, k_cache, k_scale, t_max, S, H, start_pos, T, head_scale,
-            softmax_scale, scores);
-    } else {
-        cudaFuncSetAttribute(index_scores_simt_kernel<64>,
-                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        index_scores_simt_kernel<64><<<grid, kTokPerCta, smem, stream>>>(
-            q_fp8, q_scale, w, k_cache, k_scale, t_max, S, H, start_pos, T, head_scale,
-            softmax_scale, scores);
-    }
-    return launch_status();
+    if (D == 128)
+        return launch_tc<128>(q_fp8, q_scale, w, k_cache, k_scale, t_max, B, S, H, start_pos, T,
+                              softmax_scale, scores, stream);
+    return launch_tc<64>(q_fp8, q_scale, w, k_cache, k_scale, t_max, B, S, H, start_pos, T,
+                         softmax_scale, scores, stream);
 }
 
 }  // namespace dsa
@@ -109,7 +299,8 @@ extern "C" dsa_status dsa_index_scores(const uint8_t *q_fp8, const float *q_scal
     if (H > 256) return DSA_ERR_UNSUPPORTED;
     if ((int64_t)B * S * T == 0) return DSA_OK;
     if (T > t_max || start_pos + S > T) return DSA_ERR_INVALID_ARG;
-    if ((T + 127) / 128 > 65535) return DSA_ERR_UNSUPPORTED;
+    if (t_max > INT32_MAX || B > 65535 || (int64_t)B * S > INT32_MAX / 512)
+        return DSA_ERR_UNSUPPORTED;
     if (!q_fp8 || !q_scale || !w || !k_cache || !k_scale || !scores) return DSA_ERR_INVALID_ARG;
     if (!dsa::aligned16(q_fp8) || !dsa::aligned16(k_cache)) return DSA_ERR_INVALID_ARG;
     return dsa::launch_index_scores(q_fp8, q_scale, w, k_cache, k_scale, t_max, B, S, H, D,

@@ -6,24 +6,43 @@
 // Rows with fewer causal positions than K are padded with -1 (the warm-up
 // sentinel of the DeepSeek-V4 mask visualiser) instead of masked positions.
 //
-// Selection = exact radix select on order-preserving 32-bit keys:
-//   pass p (p = 0..3) histograms byte (3-p) of the keys that match the
-//   prefix chosen so far and keeps the bin holding the m-th largest key;
-//   after four passes the threshold key tau and the number of tau-equal keys
-//   still needed are known.  A final pass writes every position with
-//   key > tau plus the first `need` positions with key == tau, in ascending
-//   position order (block-wide ballot scans), so ties go to the lower
-//   position and the output is deterministic.
+// Contract: row (b, s) selects the m = min(K, n_valid) largest scores among
+// positions t < n_valid = min(T, start_pos + s + 1), ties going to the lower
+// position, and writes them in ascending position order.  This is the same as
+// finding tau = the m-th largest value and q = m - #(x > tau), then taking
+// every x > tau plus the first q positions with x == tau.
+//
+// Cluster kernel (rows up to ~300K positions): a thread-block cluster of CN
+// CTAs owns one row; CTA p keeps the scores of positions [p*L, (p+1)*L) in
+// shared memory.  tau is found in rounds whose histograms are merged through
+// distributed shared memory by CTA 0, which broadcasts the decision:
+//   round 0: 2048 bins linear in value between the row's finite min and max
+//            (well spread for smooth score distributions, so shared-memory
+//            atomics rarely collide and the threshold bin is small);
+//   rounds 1-3: exact radix select on the order-preserving 32-bit keys
+//            (11 + 11 + 10 bits), over the threshold-bin candidates only.
+// Then every CTA counts its x > tau and x == tau, the counts are exchanged,
+// and each CTA writes its selected positions at its offset in position order.
+// Cluster barriers are hardware barriers between co-scheduled CTAs.
+//
+// Fallback kernel (longer rows): one CTA per row, four 8-bit radix passes
+// over the row in global memory, then the same ordered compaction.
+#include <cooperative_groups.h>
+
 #include "common.cuh"
+
+namespace cg = cooperative_groups;
 
 namespace dsa {
 namespace {
 
 constexpr int kThreads = 1024;
 constexpr int kWarps = kThreads / 32;
+constexpr int kBins = 2048;
+constexpr int kMaxSlice = 36864;     // scores per CTA kept in shared memory
 
-// Block-wide exclusive scan of a 0/1 flag; returns the exclusive prefix and
-// writes the block total to *total.  All threads must call it.
+// Block-wide exclusive scan of a 0/1 flag; *total receives the block total.
+// All threads must call it.
 __device__ __forceinline__ int block_scan_flag(bool flag, int *warp_tot, int *total) {
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const unsigned ballot = __ballot_sync(0xffffffffu, flag);
@@ -38,7 +57,7 @@ __device__ __forceinline__ int block_scan_flag(bool flag, int *warp_tot, int *to
             int n = __shfl_up_sync(0xffffffffu, incl, o);
             if (lane >= o) incl += n;
         }
-        if (lane < kWarps) warp_tot[lane] = incl - v;   // exclusive
+        if (lane < kWarps) warp_tot[lane] = incl - v;
         if (lane == 31) warp_tot[32] = incl;
     }
     __syncthreads();
@@ -48,6 +67,264 @@ __device__ __forceinline__ int block_scan_flag(bool flag, int *warp_tot, int *to
     return r;
 }
 
+// Block-wide sum of an int (result in every thread).
+__device__ __forceinline__ int block_sum(int v, int *tmp) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    if ((threadIdx.x & 31) == 0) tmp[threadIdx.x >> 5] = v;
+    __syncthreads();
+    int r = 0;
+    for (int w = 0; w < kWarps; w++) r += tmp[w];
+    __syncthreads();
+    return r;
+}
+
+// Finds, in a histogram of `nb` bins counted from the top, the bin where the
+// running count reaches `rank` (1-based); returns the bin and the rank left
+// inside it.  Executed by the whole block; `hist` is in shared memory.
+__device__ __forceinline__ void find_rank_bin(const unsigned *hist, int nb, unsigned rank,
+                                              unsigned *out_bin, unsigned *out_rank,
+                                              unsigned *scan_tmp) {
+    // inclusive suffix sums over bins, in chunks of kThreads bins from the top
+    unsigned above = 0;
+    for (int base = nb - 1; base >= 0; base -= kThreads) {
+        const int bin = base - (int)threadIdx.x;
+        unsigned v = bin >= 0 ? hist[bin] : 0u;
+        // inclusive scan in thread order (= descending bins)
+        unsigned incl = v;
+        const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            unsigned n = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl += n;
+        }
+        if (lane == 31) scan_tmp[warp] = incl;
+        __syncthreads();
+        if (warp == 0) {
+            unsigned wv = scan_tmp[lane];
+            unsigned wi = wv;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                unsigned n = __shfl_up_sync(0xffffffffu, wi, o);
+                if (lane >= o) wi += n;
+            }
+            scan_tmp[lane] = wi - wv;       // exclusive prefix of warp totals
+            if (lane == 31) scan_tmp[32] = wi;
+        }
+        __syncthreads();
+        const unsigned before = above + scan_tmp[warp] + incl - v;   // count strictly above bin
+        if (bin >= 0 && before < rank && before + v >= rank) {
+            *out_bin = (unsigned)bin;
+            *out_rank = rank - before;
+        }
+        above += scan_tmp[32];
+        __syncthreads();
+        if (above >= rank) break;
+    }
+    __syncthreads();
+}
+
+__device__ __forceinline__ int linear_bin(float x, float lo, float scale) {
+    if (!(x >= lo)) return 0;                       // NaN, -inf
+    const float t = __fmul_rn(__fsub_rn(x, lo), scale);
+    return t >= (float)(kBins - 1) ? kBins - 1 : (int)t;
+}
+
+struct ClusterCtl {
+    float lo, hi;           // this CTA's finite min / max
+    unsigned bin, rank;     // broadcast by CTA 0
+    int n_gt, n_eq;         // this CTA's counts of x > tau, x == tau
+};
+
+__global__ void __launch_bounds__(kThreads, 1)
+topk_cluster_kernel(const float *__restrict__ scores, int S, int64_t T, int64_t start_pos, int K,
+                    int L, int32_t *__restrict__ idx) {
+    cg::cluster_group cl = cg::this_cluster();
+    const int CN = (int)cl.num_blocks();
+    const int p = (int)cl.block_rank();
+    const int64_t row = blockIdx.x / CN;
+    const int64_t s = row % S;
+    int64_t n_valid = start_pos + s + 1;
+    if (n_valid > T) n_valid = T;
+    const int m = (int64_t)K < n_valid ? K : (int)n_valid;
+    int32_t *dst = idx + row * K;
+
+    if (m == n_valid) {                   // every causal position is selected
+        for (int i = p * kThreads + threadIdx.x; i < K; i += CN * kThreads)
+            dst[i] = i < m ? i : -1;
+        return;                           // uniform across the cluster
+    }
+
+    extern __shared__ float sv[];                                   // [L] scores
+    uint16_t *cand = reinterpret_cast<uint16_t *>(sv + L);          // [L] candidate slots
+    __shared__ unsigned hist[kBins];
+    __shared__ unsigned scan_tmp[33];
+    __shared__ int itmp[33];
+    __shared__ ClusterCtl ctl;
+    __shared__ float s_lo, s_hi;
+    __shared__ unsigned s_bin, s_rank;
+
+    const int64_t t0 = (int64_t)p * L;
+    int64_t t1 = t0 + L;
+    if (t1 > n_valid) t1 = n_valid;
+    const int len = t1 > t0 ? (int)(t1 - t0) : 0;
+    const float *src = scores + row * T + t0;
+
+    // load the slice, finite min / max
+    float lo = INFINITY, hi = -INFINITY;
+    for (int i = threadIdx.x; i < len; i += kThreads) {
+        const float x = src[i];
+        sv[i] = x;
+        if (isfinite(x)) {
+            lo = fminf(lo, x);
+            hi = fmaxf(hi, x);
+        }
+    }
+    lo = -warp_max(-lo);
+    hi = warp_max(hi);
+    if ((threadIdx.x & 31) == 0) {
+        reinterpret_cast<float *>(itmp)[threadIdx.x >> 5] = lo;
+        scan_tmp[threadIdx.x >> 5] = __float_as_uint(hi);
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        float l = INFINITY, h = -INFINITY;
+        for (int w = 0; w < kWarps; w++) {
+            l = fminf(l, reinterpret_cast<float *>(itmp)[w]);
+            h = fmaxf(h, __uint_as_float(scan_tmp[w]));
+        }
+        ctl.lo = l;
+        ctl.hi = h;
+    }
+    for (int i = threadIdx.x; i < kBins; i += kThreads) hist[i] = 0;
+    cl.sync();
+    if (threadIdx.x == 0) {
+        float l = INFINITY, h = -INFINITY;
+        for (int r = 0; r < CN; r++) {
+            const ClusterCtl *rc = cl.map_shared_rank(&ctl, r);
+            l = fminf(l, rc->lo);
+            h = fmaxf(h, rc->hi);
+        }
+        s_lo = l;
+        s_hi = h;
+    }
+    __syncthreads();
+    const float g_lo = s_lo, g_hi = s_hi;
+    const float scale = (g_hi > g_lo && isfinite(g_hi - g_lo)) ? __fdiv_rn((float)kBins, g_hi - g_lo)
+                                                                  : 0.f;
+
+    // round 0: linear bins
+    for (int i = threadIdx.x; i < len; i += kThreads) atomicAdd(&hist[linear_bin(sv[i], g_lo, scale)], 1u);
+    cl.sync();
+    if (p == 0) {
+        for (int b = threadIdx.x; b < kBins; b += kThreads) {
+            unsigned v = hist[b];
+            for (int r = 1; r < CN; r++) v += cl.map_shared_rank(hist, r)[b];
+            hist[b] = v;    // own histogram is no longer needed by anyone else
+        }
+        __syncthreads();
+        find_rank_bin(hist, kBins, (unsigned)m, &s_bin, &s_rank, scan_tmp);
+        if (threadIdx.x < CN) {
+            ClusterCtl *rc = cl.map_shared_rank(&ctl, (int)threadIdx.x);
+            rc->bin = s_bin;
+            rc->rank = s_rank;
+        }
+    }
+    cl.sync();
+    const int tb = (int)ctl.bin;
+    unsigned rank = ctl.rank;
+
+    // candidates of the threshold bin, in position order
+    int n_cand = 0;
+    for (int base = 0; base < len; base += kThreads) {
+        const int i = base + threadIdx.x;
+        const bool f = i < len && linear_bin(sv[i], g_lo, scale) == tb;
+        int tot;
+        const int pos = block_scan_flag(f, itmp, &tot);
+        if (f) cand[n_cand + pos] = (uint16_t)i;
+        n_cand += tot;
+    }
+
+    // rounds 1-3: exact radix select among the candidates
+    uint32_t prefix = 0, mask = 0;
+    const int shifts[3] = {21, 10, 0};
+    const int widths[3] = {11, 11, 10};
+    for (int rd = 0; rd < 3; rd++) {
+        const int sh = shifts[rd];
+        const uint32_t dm = (1u << widths[rd]) - 1u;
+        for (int i = threadIdx.x; i < kBins; i += kThreads) hist[i] = 0;
+        __syncthreads();
+        for (int j = threadIdx.x; j < n_cand; j += kThreads) {
+            const uint32_t key = score_key(sv[cand[j]]);
+            if ((key & mask) == prefix) atomicAdd(&hist[(key >> sh) & dm], 1u);
+        }
+        cl.sync();
+        if (p == 0) {
+            for (int b = threadIdx.x; b <= (int)dm; b += kThreads) {
+                unsigned v = hist[b];
+                for (int r = 1; r < CN; r++) v += cl.map_shared_rank(hist, r)[b];
+                hist[b] = v;
+            }
+            __syncthreads();
+            find_rank_bin(hist, (int)dm + 1, rank, &s_bin, &s_rank, scan_tmp);
+            if (threadIdx.x < CN) {
+                ClusterCtl *rc = cl.map_shared_rank(&ctl, (int)threadIdx.x);
+                rc->bin = s_bin;
+                rc->rank = s_rank;
+            }
+        }
+        cl.sync();
+        prefix |= ctl.bin << sh;
+        mask |= dm << sh;
+        rank = ctl.rank;
+    }
+    const uint32_t tau = prefix;
+    const int q = (int)rank;            // tau-equal positions still to take
+
+    // counts, exchanged through the cluster, give each CTA its output offset
+    int gt = 0, eq = 0;
+    for (int i = threadIdx.x; i < len; i += kThreads) {
+        const uint32_t key = score_key(sv[i]);
+        gt += key > tau;
+        eq += key == tau;
+    }
+    gt = block_sum(gt, itmp);
+    eq = block_sum(eq, itmp);
+    if (threadIdx.x == 0) {
+        ctl.n_gt = gt;
+        ctl.n_eq = eq;
+    }
+    cl.sync();
+    int off = 0, eq_before = 0;
+    for (int r = 0; r < p; r++) {
+        const ClusterCtl *rc = cl.map_shared_rank(&ctl, r);
+        int quota = q - eq_before;
+        quota = quota < 0 ? 0 : (quota > rc->n_eq ? rc->n_eq : quota);
+        off += rc->n_gt + quota;
+        eq_before += rc->n_eq;
+    }
+    cl.sync();                            // no CTA leaves while others read its counts
+    const int my_quota = q - eq_before;   // may exceed eq or be negative: compared below
+
+    int eq_seen = 0, out = 0;
+    for (int base = 0; base < len; base += kThreads) {
+        const int i = base + threadIdx.x;
+        const uint32_t key = i < len ? score_key(sv[i]) : 0u;
+        const bool is_eq = i < len && key == tau;
+        int eq_tot;
+        const int eq_rank = block_scan_flag(is_eq, itmp, &eq_tot);
+        const bool sel = i < len && (key > tau || (is_eq && eq_seen + eq_rank < my_quota));
+        int sel_tot;
+        const int pos = block_scan_flag(sel, itmp, &sel_tot);
+        if (sel && off + out + pos < m) dst[off + out + pos] = (int32_t)(t0 + i);
+        out += sel_tot;
+        eq_seen += eq_tot;
+    }
+    for (int i = m + p * kThreads + threadIdx.x; i < K; i += CN * kThreads) dst[i] = -1;
+}
+
+// One CTA per row, the row read from global memory (rows too long for the
+// cluster kernel's shared memory).
 __global__ void __launch_bounds__(kThreads)
 topk_row_kernel(const float *__restrict__ scores, int S, int64_t T, int64_t start_pos, int K,
                 int32_t *__restrict__ idx) {
@@ -63,13 +340,12 @@ topk_row_kernel(const float *__restrict__ scores, int S, int64_t T, int64_t star
     const float *src = scores + row * T;
     int32_t *dst = idx + row * K;
 
-    if (m == n_valid) {                       // every causal position is selected
+    if (m == n_valid) {
         for (int i = threadIdx.x; i < K; i += kThreads) dst[i] = i < m ? i : -1;
         return;
     }
-
     uint32_t prefix = 0, mask = 0;
-    unsigned remaining = (unsigned)m;         // rank still to find among matching keys
+    unsigned remaining = (unsigned)m;
     for (int shift = 24; shift >= 0; shift -= 8) {
         for (int i = threadIdx.x; i < 256; i += kThreads) hist[i] = 0;
         __syncthreads();
@@ -96,7 +372,6 @@ topk_row_kernel(const float *__restrict__ scores, int S, int64_t T, int64_t star
     }
     const uint32_t tau = prefix;
     const int need_eq = (int)remaining;
-
     int out_base = 0, eq_seen = 0;
     for (int64_t start = 0; start < n_valid; start += kThreads) {
         const int64_t t = start + threadIdx.x;
@@ -116,6 +391,25 @@ topk_row_kernel(const float *__restrict__ scores, int S, int64_t T, int64_t star
     for (int i = m + threadIdx.x; i < K; i += kThreads) dst[i] = -1;
 }
 
+// Cluster size and slice length for rows of up to `n` positions; CN = 0 if
+// the cluster kernel cannot hold them.
+void cluster_plan(int64_t n, int *cn, int *slice) {
+    int c = 1;
+    while (c < 8 && (n + c - 1) / c > 16384) c *= 2;
+    int64_t l = (n + c - 1) / c;
+    if (l > kMaxSlice) {
+        c = 16;
+        l = (n + c - 1) / c;
+    }
+    if (l > kMaxSlice) {
+        *cn = 0;
+        *slice = 0;
+        return;
+    }
+    *cn = c;
+    *slice = (int)((l + 7) / 8 * 8);
+}
+
 }  // namespace
 
 size_t topk_workspace_bytes(int, int, int64_t, int) { return 0; }
@@ -124,7 +418,37 @@ dsa_status launch_topk_select(const float *scores, int B, int S, int64_t T, int6
                               int k, int32_t *idx, void *, cudaStream_t stream) {
     if ((int64_t)B * S * T == 0) return DSA_OK;
     const int K = (int64_t)k < T ? k : (int)T;
-    topk_row_kernel<<<(unsigned)(B * S), kThreads, 0, stream>>>(scores, S, T, start_pos, K, idx);
+    const int64_t rows = (int64_t)B * S;
+    const int64_t n_max = T < start_pos + S ? T : start_pos + S;
+    int cn, L;
+    cluster_plan(n_max, &cn, &L);
+    if (cn == 0) {
+        topk_row_kernel<<<(unsigned)rows, kThreads, 0, stream>>>(scores, S, T, start_pos, K, idx);
+        return launch_status();
+    }
+    const size_t smem = (size_t)L * (sizeof(float) + sizeof(uint16_t));
+    if (cudaFuncSetAttribute(topk_cluster_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)smem) != cudaSuccess)
+        return DSA_ERR_CUDA;
+    if (cn > 8 && cudaFuncSetAttribute(topk_cluster_kernel,
+                                       cudaFuncAttributeNonPortableClusterSizeAllowed,
+                                       1) != cudaSuccess)
+        return DSA_ERR_CUDA;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)(rows * cn));
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = (unsigned)cn;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (cudaLaunchKernelEx(&cfg, topk_cluster_kernel, scores, S, T, start_pos, K, L, idx) !=
+        cudaSuccess)
+        return DSA_ERR_CUDA;
     return launch_status();
 }
 
@@ -141,6 +465,7 @@ extern "C" dsa_status dsa_topk_select(const float *scores, int B, int S, int64_t
     if (B < 0 || S < 0 || T < 0 || start_pos < 0 || k < 1) return DSA_ERR_INVALID_ARG;
     if ((int64_t)B * S * T == 0) return DSA_OK;
     if (T > INT32_MAX || start_pos + S > T) return DSA_ERR_INVALID_ARG;
+    if ((int64_t)B * S * 16 > INT32_MAX) return DSA_ERR_UNSUPPORTED;
     if (!scores || !idx) return DSA_ERR_INVALID_ARG;
     const size_t need = dsa::topk_workspace_bytes(B, S, T, k);
     if (need > 0 && (!workspace || workspace_bytes < need)) return DSA_ERR_WORKSPACE;
