@@ -70,3 +70,52 @@ def test_sparse_mla_masks_future_and_sentinels(dsa):
     empty = torch.full((1, 1, 8), -1, dtype=torch.int32)
     out0, lse0 = _gpu(dsa, q[:, :1], kv, empty, 500, sm, dc)
     assert np.all(out0 == 0) and np.all(lse0 == -np.inf)
+
+
+def test_sparse_mla_single_split_many_rows(dsa):
+    """Enough rows that each (row, half) gets one CTA: output written directly."""
+    B, Hq, dc, dr, t_max, k = 80, 128, 512, 64, 700, 256
+    q, kv, idx = _case(B, 1, Hq, dc, dr, t_max, k, t_max - 1, torch.bfloat16, seed=21, fill=0.9)
+    sm = 576 ** -0.5
+    out, lse = _gpu(dsa, q, kv, idx, t_max - 1, sm, dc)
+    for b in (0, 41, 79):
+        ref, ref_lse = oracle.sparse_mla(q[b:b + 1].float().numpy(), kv[b:b + 1].float().numpy(),
+                                         idx[b:b + 1].numpy(), t_max - 1, sm, dc)
+        assert_attention_close(out[b:b + 1], ref, "bf16", lse[b:b + 1], ref_lse)
+
+
+def test_sparse_mla_growing_logits_force_rescale(dsa):
+    """Logits grow along the (ascending) selection, so the running max keeps
+    rising by more than the lazy-rescale threshold from tile to tile."""
+    B, Hq, dc, dr, t_max, k = 2, 128, 512, 64, 4096, 2048
+    g = torch.Generator().manual_seed(22)
+    q = torch.randn(B, 1, Hq, dc + dr, generator=g)
+    base = torch.randn(B, t_max, dc + dr, generator=g)
+    ramp = torch.linspace(0, 6, t_max).reshape(1, t_max, 1)
+    kv = base * 0.3 + ramp * q[:, 0, :1, :].sign()      # aligned with head 0's query signs
+    q, kv = q.to(torch.bfloat16), kv.to(torch.bfloat16)
+    idx = torch.sort(torch.randperm(t_max, generator=g)[:k].to(torch.int32)).values
+    idx = idx.reshape(1, 1, k).repeat(B, 1, 1)
+    sm = 576 ** -0.5
+    out, lse = _gpu(dsa, q, kv, idx, t_max - 1, sm, dc)
+    ref, ref_lse = oracle.sparse_mla(q.float().numpy(), kv.float().numpy(), idx.numpy(),
+                                     t_max - 1, sm, dc)
+    assert_attention_close(out, ref, "bf16", lse, ref_lse)
+
+
+def test_sparse_mla_all_slots_empty_bf16(dsa):
+    B, Hq, dc, dr, t_max = 3, 128, 512, 64, 300
+    q, kv, _ = _case(B, 1, Hq, dc, dr, t_max, 8, t_max - 1, torch.bfloat16, seed=23)
+    idx = torch.full((B, 1, 2048), -1, dtype=torch.int32)
+    out, lse = _gpu(dsa, q, kv, idx, t_max - 1, 0.04, dc)
+    assert np.all(out == 0) and np.all(lse == -np.inf)
+
+
+def test_sparse_mla_prefill_rows_bf16(dsa):
+    """S > 1 query rows with their own causal limits (start_pos + s)."""
+    B, S, Hq, dc, dr, t_max, k, sp = 1, 5, 128, 512, 64, 2000, 512, 1500
+    q, kv, idx = _case(B, S, Hq, dc, dr, t_max, k, sp, torch.bfloat16, seed=24)
+    sm = 576 ** -0.5
+    out, lse = _gpu(dsa, q, kv, idx, sp, sm, dc)
+    ref, ref_lse = oracle.sparse_mla(q.float().numpy(), kv.float().numpy(), idx.numpy(), sp, sm, dc)
+    assert_attention_close(out, ref, "bf16", lse, ref_lse)

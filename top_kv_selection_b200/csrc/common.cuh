@@ -100,6 +100,11 @@ dsa_status launch_topk_select(const float *scores, int B, int S, int64_t T, int6
                               int k, int32_t *idx, void *ws, cudaStream_t stream);
 
 size_t sparse_mla_workspace_bytes(int B, int S, int Hq, int dc, int dr, int k, dsa_dtype dt);
+bool sparse_mla_tc_supported(int Hq, int dc, int dr, int k, dsa_dtype dt);
+size_t sparse_mla_tc_workspace_bytes(int B, int S, int k);
+dsa_status launch_sparse_mla_tc(const void *q, const void *kv, int64_t t_max, const int32_t *idx,
+                                int B, int S, int k, int64_t start_pos, float sm_scale, void *out,
+                                float *lse, void *ws, cudaStream_t stream);
 dsa_status launch_sparse_mla(const void *q, const void *kv, int64_t t_max, const int32_t *idx,
                              int B, int S, int Hq, int dc, int dr, int k, int64_t start_pos,
                              float sm_scale, dsa_dtype dt, void *out, float *lse, void *ws,

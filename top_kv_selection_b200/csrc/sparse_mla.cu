@@ -7,7 +7,8 @@
 // plus the causal mask, softmax, value mix).  The latent row is [c | k_pe]
 // (wkv_a output order); the query is already in latent space.
 //
-// SIMT kernel (used for the fp32 test mode and as the general fallback shape):
+// bf16 at the V3.2 shapes (128 heads, 512 + 64) runs the tensor-core kernel of
+// sparse_mla_tc.cu.  SIMT kernel (the fp32 test mode and other shapes):
 // a warp owns one head of one query row and walks the selected rows with an
 // online softmax; lane l holds dims l, l+32, ... of the query and of the
 // output accumulator.
@@ -85,13 +86,19 @@ sparse_mla_simt_kernel(const T *__restrict__ q, const T *__restrict__ kv, int64_
 
 }  // namespace
 
-size_t sparse_mla_workspace_bytes(int, int, int, int, int, int, dsa_dtype) { return 0; }
+size_t sparse_mla_workspace_bytes(int B, int S, int Hq, int dc, int dr, int k, dsa_dtype dt) {
+    if (sparse_mla_tc_supported(Hq, dc, dr, k, dt)) return sparse_mla_tc_workspace_bytes(B, S, k);
+    return 0;
+}
 
 dsa_status launch_sparse_mla(const void *q, const void *kv, int64_t t_max, const int32_t *idx,
                              int B, int S, int Hq, int dc, int dr, int k, int64_t start_pos,
-                             float sm_scale, dsa_dtype dt, void *out, float *lse, void *,
+                             float sm_scale, dsa_dtype dt, void *out, float *lse, void *ws,
                              cudaStream_t stream) {
     if ((int64_t)B * S * Hq == 0) return DSA_OK;
+    if (sparse_mla_tc_supported(Hq, dc, dr, k, dt))
+        return launch_sparse_mla_tc(q, kv, t_max, idx, B, S, k, start_pos, sm_scale, out, lse, ws,
+                                    stream);
     dim3 grid((unsigned)(B * S), (unsigned)((Hq + kHeadsPerCta - 1) / kHeadsPerCta));
     int *err = device_error_word();
     if (dt == DSA_BF16)
@@ -126,6 +133,7 @@ extern "C" dsa_status dsa_sparse_mla_attn(const void *q, const void *kv_cache, i
         return DSA_ERR_UNSUPPORTED;
     if ((int64_t)B * S * Hq == 0) return DSA_OK;
     if (start_pos + S > t_max) return DSA_ERR_INVALID_ARG;
+    if ((int64_t)B * t_max > INT32_MAX || (int64_t)B * S * Hq > INT32_MAX) return DSA_ERR_UNSUPPORTED;
     if (!q || !kv_cache || !idx || !out) return DSA_ERR_INVALID_ARG;
     if (!dsa::aligned16(q) || !dsa::aligned16(kv_cache) || !dsa::aligned16(out))
         return DSA_ERR_INVALID_ARG;
