@@ -148,8 +148,8 @@ class ClockSampler:
 # --------------------------------------------------------------------------- #
 # device state of the decode step
 # --------------------------------------------------------------------------- #
-def build_state(dsa, wl, rank_seed_offset=0):
-    """Device state for one decode step of wl (B sequences), N_COPIES rotating copies."""
+def build_state(dsa, wl, rank_seed_offset=0, n_copies=N_COPIES):
+    """Device state for one decode step of wl (B sequences), n_copies rotating copies."""
     dev = "cuda"
     B, T = wl.B, wl.T
     dt = torch.bfloat16 if wl.attn_dtype == "bf16" else torch.float32
@@ -173,7 +173,7 @@ def build_state(dsa, wl, rank_seed_offset=0):
     dtc = dsa.DSA_BF16 if dt == torch.bfloat16 else dsa.DSA_F32
     need = dsa.dsa_decode_step_workspace_size(B, wl.H, wl.D, T, wl.topk, wl.Hq, wl.dc, wl.dr, dtc)
     copies = []
-    for c in range(N_COPIES):
+    for c in range(n_copies):
         copies.append(dict(
             k_cache=k_cache if c == 0 else k_cache.clone(),
             k_scale=k_scale if c == 0 else k_scale.clone(),
@@ -207,31 +207,57 @@ def count_launches_per_step(wl, dsa, st) -> tuple[int, list[str]]:
 # --------------------------------------------------------------------------- #
 # dominant kernel: the indexer scorer, timed alone on the same inputs
 # --------------------------------------------------------------------------- #
-def time_scorer(dsa, wl, copies, iters):
-    """Average duration of the index-scoring launch over the full cache, with
-    CUDA events on the launching stream, rotating the state copies."""
+def time_stages(dsa, wl, copies, iters):
+    """Average device time of each stage of the decode step, each launched
+    through its own entry point on the same inputs, with CUDA events on the
+    launching stream and the state copies rotating as in the timed steps.
+    Returns {stage: seconds per launch}; "index_scores" is the dominant kernel."""
     dev = "cuda"
     B, T = wl.B, wl.T
     q_fp8 = torch.empty(B, 1, wl.H, wl.D, dtype=torch.uint8, device=dev)
     q_scale = torch.empty(B, 1, wl.H, dtype=torch.float32, device=dev)
-    dsa.dsa_indexer_quant(copies[0]["q_idx"], q_fp8, q_scale)
     w = copies[0]["w"].reshape(B, 1, wl.H).contiguous()
     scores = torch.empty(B, 1, T, dtype=torch.float32, device=dev)
+    idx = torch.empty(B, 1, wl.K, dtype=torch.int32, device=dev)
+    dt = dsa.DSA_BF16 if wl.attn_dtype == "bf16" else dsa.DSA_F32
+    ws = torch.empty(max(1, dsa.dsa_sparse_mla_attn_workspace_size(B, 1, wl.Hq, wl.dc, wl.dr,
+                                                                    wl.K, dt)),
+                     dtype=torch.uint8, device=dev)
+    q_mla = copies[0]["q_mla"].reshape(B, 1, wl.Hq, wl.dqk).contiguous()
+    out = torch.empty(B, 1, wl.Hq, wl.dc, dtype=copies[0]["out"].dtype, device=dev)
+    lse = torch.empty(B, 1, wl.Hq, dtype=torch.float32, device=dev)
+
+    def quant(st):
+        dsa.dsa_indexer_quant(st["q_idx"], q_fp8, q_scale)
+        dsa.dsa_indexer_quant(st["k_new"], st["k_cache"][:, T - 1:], st["k_scale"][:, T - 1:],
+                              n_rows=B, out_row_stride=st["k_cache"].shape[1] * wl.D,
+                              scale_row_stride=st["k_cache"].shape[1])
+
+    def score(st):
+        dsa.dsa_index_scores(q_fp8, q_scale, w, st["k_cache"], st["k_scale"], T - 1, T,
+                             wl.softmax_scale_idx, scores)
+
+    def topk(st):
+        dsa.dsa_topk_select(scores, T - 1, wl.topk, idx)
+
+    def attn(st):
+        dsa.dsa_sparse_mla_attn(q_mla, st["kv"], idx, T - 1, wl.sm_scale, out, lse, ws)
+
     stream = torch.cuda.current_stream()
-    for i in range(3):
-        st = copies[i % len(copies)]
-        dsa.dsa_index_scores(q_fp8, q_scale, w, st["k_cache"], st["k_scale"], T - 1, T,
-                             wl.softmax_scale_idx, scores)
-    torch.cuda.synchronize()
-    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    t0.record(stream)
-    for i in range(iters):
-        st = copies[i % len(copies)]
-        dsa.dsa_index_scores(q_fp8, q_scale, w, st["k_cache"], st["k_scale"], T - 1, T,
-                             wl.softmax_scale_idx, scores)
-    t1.record(stream)
-    t1.synchronize()
-    return t0.elapsed_time(t1) / iters * 1e-3      # seconds per launch
+    result = {}
+    for name, fn in (("indexer_quant", quant), ("index_scores", score), ("topk_select", topk),
+                     ("sparse_mla_attn", attn)):
+        for i in range(3):
+            fn(copies[i % len(copies)])
+        torch.cuda.synchronize()
+        t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        t0.record(stream)
+        for i in range(iters):
+            fn(copies[i % len(copies)])
+        t1.record(stream)
+        t1.synchronize()
+        result[name] = t0.elapsed_time(t1) / iters * 1e-3
+    return result
 
 
 # --------------------------------------------------------------------------- #
@@ -301,13 +327,13 @@ def run_ours(args, wl, world, rank, local):
     __graft_entry__._builder().build()
     import top_kv_selection_b200 as dsa
 
-    copies = build_state(dsa, wl, rank_seed_offset=0)
+    copies = build_state(dsa, wl, rank_seed_offset=0, n_copies=args.copies)
     torch.cuda.synchronize()
     per_step_launches, kernel_names = count_launches_per_step(wl, dsa, copies[0])
 
     stream = torch.cuda.current_stream()
     for i in range(args.warmup):
-        decode_step(dsa, wl, copies[i % N_COPIES])
+        decode_step(dsa, wl, copies[i % len(copies)])
     torch.cuda.synchronize()
     if dsa.dsa_get_device_error() != 0:
         raise RuntimeError("device error word set during warm-up")
@@ -318,7 +344,7 @@ def run_ours(args, wl, world, rank, local):
     with ClockSampler(torch.cuda.current_device()) as clk:
         start.record(stream)
         for i in range(args.steps):
-            decode_step(dsa, wl, copies[i % N_COPIES])
+            decode_step(dsa, wl, copies[i % len(copies)])
         end.record(stream)
         end.synchronize()
     torch.cuda.synchronize()
@@ -334,7 +360,8 @@ def run_ours(args, wl, world, rank, local):
 
     # dominant kernel roofline (indexer scorer over the full cache)
     peak, peak_kind = _peaks()
-    t_score = time_scorer(dsa, wl, copies, iters=max(10, args.steps))
+    stages = time_stages(dsa, wl, copies, iters=max(10, min(args.steps, 500)))
+    t_score = stages["index_scores"]
     score_bytes = wl.B * wl.T * (wl.D + 4) + wl.B * wl.H * (wl.D + 4 + 4)
     achieved = score_bytes / t_score / 1e9
     step_bytes = wl.B * (wl.T * (wl.D + 4) + wl.K * wl.dqk * 2 + wl.H * wl.D * 4
@@ -347,7 +374,7 @@ def run_ours(args, wl, world, rank, local):
         "dtype": "fp8_e4m3+bf16", "data": "synthetic",
         "config": {"workload": wl.name, "B": wl.B, "T": wl.T, "H": wl.H, "D": wl.D,
                    "topk": wl.topk, "Hq": wl.Hq, "dc": wl.dc, "dr": wl.dr,
-                   "l2": f"{N_COPIES} rotating state copies, each larger than L2",
+                   "l2": f"{len(copies)} rotating state copies, each larger than L2",
                    "parallelism": f"dp{world} (independent batches per rank)"},
         "indexer_gscores_per_s": gscores,
         "step_roofline": {"bytes": step_bytes, "achieved_gbs": step_bytes / (ms_per_step * 1e-3)
@@ -359,6 +386,7 @@ def run_ours(args, wl, world, rank, local):
         "e2e": e2e,
         "gpu_launches": per_step_launches * args.steps,
         "kernels_per_step": per_step_launches, "kernels": kernel_names,
+        "stage_us": {k: round(v * 1e6, 2) for k, v in stages.items()},
         "clocks": clk.summary(),
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -390,7 +418,7 @@ def run_e2e(dsa, wl, copies, args, world):
     stream = torch.cuda.current_stream()
 
     def one(i):
-        s = copies[i % N_COPIES]
+        s = copies[i % len(copies)]
         for k, t in host_in.items():
             s[k].copy_(t, non_blocking=True)
         s["kv"][:, wl.T - 1].copy_(new_row, non_blocking=True)
@@ -413,6 +441,42 @@ def run_e2e(dsa, wl, copies, args, world):
             "d2h_bytes_per_step": d2h}
 
 
+def measure_fp8_peak(n=8192, iters=20):
+    """Dense e4m3 GEMM throughput (torch._scaled_mm, N^3, best of `iters`) -- the
+    FP8 tensor-core denominator for the prefill scorer's roofline."""
+    a = torch.randn(n, n, device="cuda").to(torch.float8_e4m3fn)
+    b = torch.randn(n, n, device="cuda").to(torch.float8_e4m3fn).t()
+    one = torch.ones((), device="cuda")
+    for _ in range(3):
+        torch._scaled_mm(a, b, scale_a=one, scale_b=one, out_dtype=torch.bfloat16)
+    torch.cuda.synchronize()
+    best = float("inf")
+    for _ in range(iters):
+        t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        t0.record()
+        torch._scaled_mm(a, b, scale_a=one, scale_b=one, out_dtype=torch.bfloat16)
+        t1.record()
+        t1.synchronize()
+        best = min(best, t0.elapsed_time(t1) * 1e-3)
+    with ClockSampler(torch.cuda.current_device()) as clk:
+        t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        t0.record()
+        k = 0
+        while True:
+            for _ in range(50):
+                torch._scaled_mm(a, b, scale_a=one, scale_b=one, out_dtype=torch.bfloat16)
+            k += 50
+            t1.record()
+            t1.synchronize()
+            if t0.elapsed_time(t1) > 4000:
+                break
+    sustained = 2 * n ** 3 * k / (t0.elapsed_time(t1) * 1e-3) / 1e12
+    return {"fp8_e4m3_tflops": 2 * n ** 3 / best / 1e12, "fp8_e4m3_tflops_sustained": sustained,
+            "n": n, "how": "torch._scaled_mm e4m3 x e4m3 -> bf16, N^3, best of "
+                           f"{iters} (burst) and back to back for 4 s (sustained)",
+            "clocks": clk.summary()}
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -421,7 +485,14 @@ def main(argv=None):
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", type=int, default=4)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--fp8-peak", action="store_true",
+                    help="measure the dense FP8 GEMM peak and exit")
+    ap.add_argument("--copies", type=int, default=N_COPIES,
+                    help="rotating device copies of the decode state (each larger than L2)")
     args = ap.parse_args(argv)
+    if args.fp8_peak:
+        print(json.dumps(measure_fp8_peak()), flush=True)
+        return
     wl = workloads.WORKLOADS[args.workload]
     if wl.mode != "decode":
         raise SystemExit("bench.py times decode workloads (1, 2 or 4)")

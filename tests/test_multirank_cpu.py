@@ -1,0 +1,61 @@
+"""The N > 1 path of bench.py on CPU: world_size-2 gloo ranks.
+
+The hot path partitions over independent sequences, so ranks share no data;
+the only cross-rank steps are the barrier around the timed region and the max
+over ranks of the elapsed time.  These run here with the gloo backend.
+"""
+import json
+import os
+import subprocess
+import sys
+
+import pytest
+import torch.multiprocessing as mp
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _max_worker(rank, world, port, out_q):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank),
+                      WORLD_SIZE=str(world), LOCAL_RANK=str(rank))
+    sys.path.insert(0, ROOT)
+    import bench
+    w, r, _ = bench._dist_init()
+    try:
+        bench._barrier(w)
+        # each rank reports a different elapsed time; all must agree on the max
+        out_q.put((r, bench._max_over_ranks(w, 1.0 + r * 0.5)))
+    finally:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+def test_max_over_ranks_gloo():
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = 29517
+    procs = [ctx.Process(target=_max_worker, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    for p in procs:
+        p.join(120)
+        assert p.exitcode == 0
+    got = dict(q.get(timeout=10) for _ in range(2))
+    assert got == {0: 1.5, 1: 1.5}
+
+
+@pytest.mark.slow
+def test_bench_reference_arm_under_torchrun_two_ranks():
+    """`bench.py --impl reference` launched like the driver's N=2 run: rank 0
+    prints one JSON line, rank 1 exits 0 without work."""
+    env = dict(os.environ, CUDA_VISIBLE_DEVICES="")
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", "--nproc-per-node=2",
+           "--master-addr", "127.0.0.1", "--master-port", "29533", "bench.py", "--impl",
+           "reference", "--workload", "1", "--steps", "1", "--warmup", "0"]
+    r = subprocess.run(cmd, cwd=ROOT, env=env, capture_output=True, text=True, timeout=600)
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = [l for l in r.stdout.splitlines() if l.startswith("{")]
+    assert len(lines) == 1
+    d = json.loads(lines[0])
+    assert d["impl"] == "reference" and d["value"] > 0 and d["cpu_baseline"]["kind"] == "oracle"
+    assert d["e2e"]["h2d_bytes_per_step"] == 0

@@ -95,6 +95,13 @@ dsa_status launch_index_scores(const uint8_t *q_fp8, const float *q_scale, const
                                int S, int H, int D, int64_t start_pos, int64_t T,
                                float softmax_scale, float *scores, cudaStream_t stream);
 
+// Decode step: rotate + quantise the new queries and key inside the scorer,
+// append the key at T-1, score positions 0..T-1 of each sequence.
+dsa_status launch_decode_scores(const float *q_raw, const float *w, const float *k_new,
+                                uint8_t *k_cache, float *k_scale, int64_t t_max, int B, int H,
+                                int D, int64_t T, float softmax_scale, float *scores,
+                                cudaStream_t stream);
+
 size_t topk_workspace_bytes(int B, int S, int64_t T, int k);
 dsa_status launch_topk_select(const float *scores, int B, int S, int64_t T, int64_t start_pos,
                               int k, int32_t *idx, void *ws, cudaStream_t stream);

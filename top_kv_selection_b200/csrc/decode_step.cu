@@ -4,7 +4,8 @@
 // seqlen == 1 (no mask, "DeepSeek-V3.2-Exp - Causal mask"), followed by the
 // diagram's sparse core attention in MQA mode:
 //   rotate+quantise q and k_new, append k_new at T-1, fp8_index over the T
-//   cached keys, top-min(index_topk, T), sparse latent attention.
+//   cached keys (one fused tensor-core kernel), top-min(index_topk, T), sparse
+//   latent attention.
 // Everything is enqueued on one stream; nothing synchronises with the host.
 #include "common.cuh"
 
@@ -12,15 +13,13 @@ namespace dsa {
 namespace {
 
 struct DecodeWs {
-    uint8_t *q_fp8;    // [B,H,D]
-    float *q_scale;    // [B,H]
     float *scores;     // [B,T]
     void *topk_ws;
     void *attn_ws;
     size_t total;
 };
 
-DecodeWs carve(void *base, int B, int H, int D, int64_t T, int index_topk, int Hq, int dc, int dr,
+DecodeWs carve(void *base, int B, int, int, int64_t T, int index_topk, int Hq, int dc, int dr,
                dsa_dtype dt) {
     DecodeWs w{};
     size_t off = 0;
@@ -30,8 +29,6 @@ DecodeWs carve(void *base, int B, int H, int D, int64_t T, int index_topk, int H
         off = align_up(off + bytes, 256);
         return r;
     };
-    w.q_fp8 = reinterpret_cast<uint8_t *>(take((size_t)B * H * D));
-    w.q_scale = reinterpret_cast<float *>(take((size_t)B * H * sizeof(float)));
     w.scores = reinterpret_cast<float *>(take((size_t)B * T * sizeof(float)));
     w.topk_ws = take(topk_workspace_bytes(B, 1, T, index_topk));
     const int K = (int64_t)index_topk < T ? index_topk : (int)T;
@@ -75,14 +72,8 @@ extern "C" dsa_status dsa_decode_step(const float *q_idx, const float *w, const 
         return DSA_ERR_WORKSPACE;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     dsa_status st;
-    if ((st = dsa::launch_indexer_quant(q_idx, DSA_F32, 1, (int64_t)B * H, D, ws.q_fp8, 0,
-                                        ws.q_scale, 0, s)) != DSA_OK)
-        return st;
-    if ((st = dsa::launch_indexer_quant(k_new, DSA_F32, B, 1, D, k_cache + (T - 1) * D,
-                                        t_max * D, k_scale + (T - 1), t_max, s)) != DSA_OK)
-        return st;
-    if ((st = dsa::launch_index_scores(ws.q_fp8, ws.q_scale, w, k_cache, k_scale, t_max, B, 1, H,
-                                       D, T - 1, T, softmax_scale, ws.scores, s)) != DSA_OK)
+    if ((st = dsa::launch_decode_scores(q_idx, w, k_new, k_cache, k_scale, t_max, B, H, D, T,
+                                        softmax_scale, ws.scores, s)) != DSA_OK)
         return st;
     if ((st = dsa::launch_topk_select(ws.scores, B, 1, T, T - 1, index_topk, idx, ws.topk_ws,
                                       s)) != DSA_OK)

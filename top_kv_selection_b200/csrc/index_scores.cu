@@ -17,7 +17,16 @@
 //               k_scale[t] * sum_h w'_h * max(dot_h, 0)  (ReLU, weighted head
 //               sum, key scale), storing one fp32 score per token.
 // The key cache is the only large operand: 132 bytes per token (D + 4).
+//
+// The producer starts streaming at once; the query operand is built in
+// parallel by the epilogue warps, either from given FP8 codes or -- in the
+// decode step -- by rotating and quantising the new token's fp32 queries
+// (rotate_activation + act_quant, bit-identical to dsa_indexer_quant).  In the
+// decode step the CTA holding position T-1 also quantises the new key and
+// appends it to the cache (the cache write of Indexer.forward) before its last
+// tile is fetched.
 #include "common.cuh"
+#include "quant.cuh"
 #include "tc_ptx.cuh"
 #include "tmap.cuh"
 
@@ -31,8 +40,12 @@ constexpr int kThreads = 192;    // warp 0 TMA, warp 1 MMA, warps 2..5 epilogue
 constexpr int kMaxHeads = 256;
 
 struct ScoreArgs {
-    const uint8_t *q_fp8;
+    const uint8_t *q_fp8;      // query codes [rows, H, D] and scales, or ...
     const float *q_scale;
+    const float *q_raw;        // ... the new token's fp32 queries [B, H, D] (decode)
+    const float *k_new;        // decode: new key [B, D], appended at position T-1
+    uint8_t *k_cache_w;
+    float *k_scale_w;
     const float *w;
     const float *k_scale;
     float *scores;
@@ -60,7 +73,70 @@ template <> struct KSwizzle<64> {
 template <int D>
 __host__ __device__ constexpr size_t score_smem_bytes(int NH) {
     return 1024 + (size_t)kStages * kTile * D + (size_t)NH * D + kMaxHeads * sizeof(float) +
-           (2 * kStages + 2 * kAcc) * sizeof(uint64_t) + 16;
+           (2 * kStages + 2 * kAcc + 2) * sizeof(uint64_t) + 16;
+}
+
+// Query operand (K-major, swizzled, padded heads zero) and folded weights
+// w' = ((w * H^-1/2) * q_scale) * softmax_scale; run by the four epilogue
+// warps.  In decode mode the first of them first appends the new key.
+template <int D>
+__device__ __forceinline__ void build_query(const ScoreArgs &a, int64_t row, int64_t b,
+                                            uint8_t *sq, float *wf, bool append,
+                                            float *knew_scale, uint64_t *k_ready) {
+    constexpr int E = D / 32;
+    constexpr int kChunks = D / 16;
+    const int t = threadIdx.x - 64;           // 0..127 over the epilogue warps
+    const int wi = t >> 5, lane = t & 31;
+    if (a.q_raw) {
+        if (append && wi == 0) {
+            float r[E];
+            load_lane_slice<D, float>(a.k_new + b * D, r);
+            float ks;
+            const uint32_t packed = rotate_quant_warp<D>(r, &ks);
+            uint8_t *dst = a.k_cache_w + (b * a.t_max + a.T - 1) * D + lane * E;
+            if constexpr (E == 4) *reinterpret_cast<uint32_t *>(dst) = packed;
+            else *reinterpret_cast<uint16_t *>(dst) = static_cast<uint16_t>(packed);
+            if (lane == 0) {
+                a.k_scale_w[b * a.t_max + a.T - 1] = ks;
+                *knew_scale = ks;
+            }
+            // the key row is read next by TMA (async proxy)
+            asm volatile("fence.proxy.async.global;" ::: "memory");
+            __syncwarp();
+            if (lane == 0) tc::mbar_arrive(k_ready);
+        }
+        for (int h = wi; h < a.H; h += 4) {
+            float r[E];
+            load_lane_slice<D, float>(a.q_raw + (row * a.H + h) * D, r);
+            float qs;
+            const uint32_t packed = rotate_quant_warp<D>(r, &qs);
+            const int byte = lane * E;
+            uint8_t *dst = sq + h * D + KSwizzle<D>::chunk(h, byte >> 4) * 16 + (byte & 15);
+            if constexpr (E == 4) *reinterpret_cast<uint32_t *>(dst) = packed;
+            else *reinterpret_cast<uint16_t *>(dst) = static_cast<uint16_t>(packed);
+            if (lane == 0) {
+                float x = __fmul_rn(a.w[row * a.H + h], a.head_scale);
+                x = __fmul_rn(x, qs);
+                wf[h] = __fmul_rn(x, a.softmax_scale);
+            }
+        }
+    } else {
+        const uint8_t *qrow = a.q_fp8 + row * a.H * D;
+        for (int i = t; i < a.H * kChunks; i += 128) {
+            const int h = i / kChunks, c = i - h * kChunks;
+            *reinterpret_cast<uint4 *>(sq + h * D + KSwizzle<D>::chunk(h, c) * 16) =
+                *reinterpret_cast<const uint4 *>(qrow + h * D + c * 16);
+        }
+        for (int h = t; h < a.H; h += 128) {
+            float x = __fmul_rn(a.w[row * a.H + h], a.head_scale);
+            x = __fmul_rn(x, a.q_scale[row * a.H + h]);
+            wf[h] = __fmul_rn(x, a.softmax_scale);
+        }
+    }
+    for (int i = t; i < (a.NH - a.H) * kChunks; i += 128)
+        *reinterpret_cast<uint4 *>(sq + (a.H + i / kChunks) * D + (i % kChunks) * 16) =
+            make_uint4(0, 0, 0, 0);
+    for (int h = a.H + t; h < kMaxHeads; h += 128) wf[h] = 0.f;
 }
 
 template <int D>
@@ -76,8 +152,10 @@ score_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const ScoreArgs a) {
     uint64_t *empty = full + kStages;
     uint64_t *accf = empty + kStages;
     uint64_t *acce = accf + kAcc;
-    uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(acce + kAcc);
+    uint64_t *q_ready = acce + kAcc, *k_ready = q_ready + 1;
+    uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(k_ready + 1);
     volatile int *abort = reinterpret_cast<volatile int *>(tmem_holder + 1);
+    float *knew_scale = reinterpret_cast<float *>(tmem_holder + 2);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int64_t row = blockIdx.x / a.chunks;
@@ -89,6 +167,8 @@ score_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const ScoreArgs a) {
     const int64_t tile_lo = chunk * n_tiles / a.chunks;
     const int64_t tile_hi = (chunk + 1) * n_tiles / a.chunks;
     const int n_my = (int)(tile_hi - tile_lo);
+    // decode: this CTA appends the new key if its last tile holds position T-1
+    const bool append = a.k_new != nullptr && n_my > 0 && tile_hi == n_tiles;
 
     // causally masked positions of this row (prefill only), shared by the chunks
     for (int64_t t = n_vis + (int64_t)chunk * kThreads + threadIdx.x; t < a.T;
@@ -105,6 +185,8 @@ score_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const ScoreArgs a) {
             tc::mbar_init(&accf[i], 1);
             tc::mbar_init(&acce[i], 4 * 32);
         }
+        tc::mbar_init(q_ready, 4 * 32);
+        tc::mbar_init(k_ready, 1);
         *abort = 0;
         tc::fence_mbar_init();
         tc::tma_prefetch_desc(&tmap_k);
@@ -113,26 +195,6 @@ score_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const ScoreArgs a) {
         tc::tmem_alloc(tmem_holder, a.tmem_cols);
         tc::tmem_relinquish();
     }
-    // query codes of this row -> K-major swizzled tile (padded heads are zero)
-    constexpr int kChunks = D / 16;
-    const uint8_t *qrow = a.q_fp8 + row * a.H * D;
-    for (int i = threadIdx.x; i < a.NH * kChunks; i += kThreads) {
-        const int h = i / kChunks, c = i - h * kChunks;
-        uint4 v = make_uint4(0, 0, 0, 0);
-        if (h < a.H) v = *reinterpret_cast<const uint4 *>(qrow + h * D + c * 16);
-        *reinterpret_cast<uint4 *>(sq + h * D + KSwizzle<D>::chunk(h, c) * 16) = v;
-    }
-    // weight fold: w' = ((w * H^-1/2) * q_scale) * softmax_scale, fp32, in that order
-    for (int h = threadIdx.x; h < kMaxHeads; h += kThreads) {
-        float t = 0.f;
-        if (h < a.H) {
-            t = __fmul_rn(a.w[row * a.H + h], a.head_scale);
-            t = __fmul_rn(t, a.q_scale[row * a.H + h]);
-            t = __fmul_rn(t, a.softmax_scale);
-        }
-        wf[h] = t;
-    }
-    tc::fence_proxy_async_smem();
     tc::tc_fence_before();
     __syncthreads();
     tc::tc_fence_after();
@@ -146,6 +208,7 @@ score_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const ScoreArgs a) {
                 const int st = i % kStages;
                 const uint32_t ph = (uint32_t)(i / kStages) & 1u;
                 if (!tc::mbar_wait(&empty[st], ph ^ 1u, a.err, abort)) break;
+                if (append && i == n_my - 1 && !tc::mbar_wait(k_ready, 0, a.err, abort)) break;
                 tc::mbar_arrive_expect_tx(&full[st], kTile * D);
                 tc::tma_load_3d(sk + st * kTile * D, &tmap_k, 0, (int)((tile_lo + i) * kTile),
                                 (int)b, &full[st], pol);
@@ -159,7 +222,8 @@ score_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const ScoreArgs a) {
         if (lane == 0) {
             const uint32_t idesc = tc::instr_desc(tc::kFmtE4M3, tc::kFmtE4M3, kTile, a.NH);
             const uint32_t sk_addr = tc::smem_u32(sk), sq_addr = tc::smem_u32(sq);
-            for (int i = 0; i < n_my; i++) {
+            const bool q_ok = tc::mbar_wait(q_ready, 0, a.err, abort);
+            for (int i = 0; q_ok && i < n_my; i++) {
                 const int st = i % kStages, ac = i % kAcc;
                 if (!tc::mbar_wait(&full[st], (uint32_t)(i / kStages) & 1u, a.err, abort)) break;
                 if (!tc::mbar_wait(&acce[ac], ((uint32_t)(i / kAcc) & 1u) ^ 1u, a.err, abort))
@@ -179,6 +243,10 @@ score_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const ScoreArgs a) {
             }
         }
     } else {
+        build_query<D>(a, row, b, sq, wf, append, knew_scale, k_ready);
+        tc::fence_proxy_async_smem();
+        asm volatile("bar.sync 1, 128;" ::: "memory");   // folded weights of all heads
+        tc::mbar_arrive(q_ready);
         const int quarter = warp & 3;                 // TMEM lanes this warp may read
         const int tok = quarter * 32 + lane;          // token within the tile
         const uint32_t lane_addr = (uint32_t)(quarter * 32) << 16;
@@ -187,11 +255,13 @@ score_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const ScoreArgs a) {
         for (int i = 0; i < n_my; i++) {
             const int ac = i % kAcc;
             const int64_t t = (tile_lo + i) * kTile + tok;
-            const float ks = t < n_vis ? __ldg(ks_row + t) : 0.f;
+            const float ks = t >= n_vis ? 0.f : (append && t == a.T - 1) ? *knew_scale
+                                                                          : __ldg(ks_row + t);
             if (!tc::mbar_wait(&accf[ac], (uint32_t)(i / kAcc) & 1u, a.err, abort)) break;
             tc::tc_fence_after();
             const uint32_t taddr = tmem_base + lane_addr + (uint32_t)(ac * a.NH);
-            float acc = 0.f;
+            // four independent partial sums keep the FMA chain short
+            float acc4[4] = {0.f, 0.f, 0.f, 0.f};
             for (int c0 = 0; c0 < a.NH; c0 += 64) {
                 uint32_t r[4][16];
 #pragma unroll
@@ -201,11 +271,18 @@ score_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const ScoreArgs a) {
 #pragma unroll
                 for (int j = 0; j < 4; j++) {
                     if (c0 + 16 * j >= a.NH) break;
+                    const float4 *w4 = reinterpret_cast<const float4 *>(wf + c0 + 16 * j);
 #pragma unroll
-                    for (int e = 0; e < 16; e++)
-                        acc = fmaf(wf[c0 + 16 * j + e], fmaxf(__uint_as_float(r[j][e]), 0.f), acc);
+                    for (int e = 0; e < 4; e++) {
+                        const float4 wv = w4[e];
+                        acc4[0] = fmaf(wv.x, fmaxf(__uint_as_float(r[j][4 * e + 0]), 0.f), acc4[0]);
+                        acc4[1] = fmaf(wv.y, fmaxf(__uint_as_float(r[j][4 * e + 1]), 0.f), acc4[1]);
+                        acc4[2] = fmaf(wv.z, fmaxf(__uint_as_float(r[j][4 * e + 2]), 0.f), acc4[2]);
+                        acc4[3] = fmaf(wv.w, fmaxf(__uint_as_float(r[j][4 * e + 3]), 0.f), acc4[3]);
+                    }
                 }
             }
+            const float acc = (acc4[0] + acc4[1]) + (acc4[2] + acc4[3]);
             tc::tc_fence_before();
             tc::mbar_arrive(&acce[ac]);
             if (t < n_vis) out[t] = ks * acc;
@@ -227,34 +304,22 @@ uint32_t pow2_cols(int n) {
 }
 
 template <int D>
-dsa_status launch_tc(const uint8_t *q_fp8, const float *q_scale, const float *w,
-                     const uint8_t *k_cache, const float *k_scale, int64_t t_max, int B, int S,
-                     int H, int64_t start_pos, int64_t T, float softmax_scale, float *scores,
-                     cudaStream_t stream) {
+dsa_status launch_tc(ScoreArgs a, const uint8_t *k_cache, int B, int S, int64_t start_pos,
+                     int64_t T, cudaStream_t stream) {
     CUtensorMap tmap;
-    const uint64_t dims[3] = {(uint64_t)D, (uint64_t)t_max, (uint64_t)B};
-    const uint64_t strides[2] = {(uint64_t)D, (uint64_t)t_max * D};
+    const uint64_t dims[3] = {(uint64_t)D, (uint64_t)a.t_max, (uint64_t)B};
+    const uint64_t strides[2] = {(uint64_t)D, (uint64_t)a.t_max * D};
     const uint32_t box[3] = {(uint32_t)D, (uint32_t)kTile, 1};
     const CUtensorMapSwizzle swz =
         D == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
     if (!encode_tmap(&tmap, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, k_cache, dims, strides, box, swz))
         return DSA_ERR_CUDA;
-
-    ScoreArgs a;
-    a.q_fp8 = q_fp8;
-    a.q_scale = q_scale;
-    a.w = w;
-    a.k_scale = k_scale;
-    a.scores = scores;
-    a.t_max = t_max;
     a.start_pos = start_pos;
     a.T = T;
     a.S = S;
-    a.H = H;
-    a.NH = (H + 15) / 16 * 16;
+    a.NH = (a.H + 15) / 16 * 16;
     a.tmem_cols = pow2_cols(kAcc * a.NH);
-    a.head_scale = (float)(1.0 / sqrt((double)H));
-    a.softmax_scale = softmax_scale;
+    a.head_scale = (float)(1.0 / sqrt((double)a.H));
     a.err = device_error_word();
 
     const size_t smem = score_smem_bytes<D>(a.NH);
@@ -280,11 +345,37 @@ dsa_status launch_index_scores(const uint8_t *q_fp8, const float *q_scale, const
                                int S, int H, int D, int64_t start_pos, int64_t T,
                                float softmax_scale, float *scores, cudaStream_t stream) {
     if ((int64_t)B * S * T == 0) return DSA_OK;
-    if (D == 128)
-        return launch_tc<128>(q_fp8, q_scale, w, k_cache, k_scale, t_max, B, S, H, start_pos, T,
-                              softmax_scale, scores, stream);
-    return launch_tc<64>(q_fp8, q_scale, w, k_cache, k_scale, t_max, B, S, H, start_pos, T,
-                         softmax_scale, scores, stream);
+    ScoreArgs a = {};
+    a.q_fp8 = q_fp8;
+    a.q_scale = q_scale;
+    a.w = w;
+    a.k_scale = k_scale;
+    a.scores = scores;
+    a.t_max = t_max;
+    a.H = H;
+    a.softmax_scale = softmax_scale;
+    return D == 128 ? launch_tc<128>(a, k_cache, B, S, start_pos, T, stream)
+                    : launch_tc<64>(a, k_cache, B, S, start_pos, T, stream);
+}
+
+dsa_status launch_decode_scores(const float *q_raw, const float *w, const float *k_new,
+                                uint8_t *k_cache, float *k_scale, int64_t t_max, int B, int H,
+                                int D, int64_t T, float softmax_scale, float *scores,
+                                cudaStream_t stream) {
+    if ((int64_t)B * T == 0) return DSA_OK;
+    ScoreArgs a = {};
+    a.q_raw = q_raw;
+    a.k_new = k_new;
+    a.k_cache_w = k_cache;
+    a.k_scale_w = k_scale;
+    a.w = w;
+    a.k_scale = k_scale;
+    a.scores = scores;
+    a.t_max = t_max;
+    a.H = H;
+    a.softmax_scale = softmax_scale;
+    return D == 128 ? launch_tc<128>(a, k_cache, B, 1, T - 1, T, stream)
+                    : launch_tc<64>(a, k_cache, B, 1, T - 1, T, stream);
 }
 
 }  // namespace dsa

@@ -1,0 +1,93 @@
+// quant.cuh -- rotate_activation + act_quant of one D-vector by one warp.
+//
+// Page: "DeepSeek-V3.2-Exp - Split indexer heads", Indexer.forward
+// (rotate_activation, then act_quant with one scale per vector).
+//
+// Lane L holds elements [E*L, E*L + E), E = D / 32.  Butterfly stage h pairs
+// element i with i ^ h: for h < E both live in the lane's registers,
+// otherwise in lane L ^ (h / E) at the same register slot.  The lower element
+// becomes a + b and the upper a - b, in fp32, stages in the order h = 1, 2, 4,
+// ..., D/2 -- the same dataflow as the plain in-place transform, so the result
+// is bit-identical to it.  Then one multiply by fp32(D^-1/2), a warp max of
+// |x|, scale = max(amax, 1e-4) / 448 and the e4m3 codes of x / scale (round to
+// nearest even, saturate to +-448), both divisions correctly rounded.
+#pragma once
+
+#include "common.cuh"
+
+namespace dsa {
+
+template <int D> struct HadamardScale;
+template <> struct HadamardScale<64> { static constexpr float value = 0.125f; };
+// nearest fp32 to 128^-1/2 = sqrt(2)/16: 0x3DB504F3
+template <> struct HadamardScale<128> { static constexpr float value = 0x1.6a09e6p-4f; };
+
+// Two fp32 -> two e4m3 codes packed as (lo | hi << 8); the first PTX source
+// operand fills the upper byte.
+__device__ __forceinline__ uint32_t e4m3x2_rn_sat(float lo, float hi) {
+    uint16_t r;
+    asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(hi), "f"(lo));
+    return r;
+}
+
+// Rotates and quantises the vector held in r (this lane's E elements).
+// Returns this lane's E codes packed little-endian; *scale gets the vector's
+// scale (same value in every lane).  All 32 lanes must call it.
+template <int D>
+__device__ __forceinline__ uint32_t rotate_quant_warp(float (&r)[D / 32], float *scale) {
+    constexpr int E = D / 32;
+    const int lane = threadIdx.x & 31;
+#pragma unroll
+    for (int h = 1; h < E; h <<= 1) {
+#pragma unroll
+        for (int e = 0; e < E; e++) {
+            if (e & h) continue;
+            const float a = r[e], b = r[e + h];
+            r[e] = a + b;
+            r[e + h] = a - b;
+        }
+    }
+#pragma unroll
+    for (int m = 1; m < 32; m <<= 1) {
+        const bool upper = (lane & m) != 0;
+#pragma unroll
+        for (int e = 0; e < E; e++) {
+            const float p = __shfl_xor_sync(0xffffffffu, r[e], m);
+            r[e] = upper ? __fsub_rn(p, r[e]) : __fadd_rn(r[e], p);
+        }
+    }
+    float amax = 0.f;
+#pragma unroll
+    for (int e = 0; e < E; e++) {
+        r[e] = __fmul_rn(r[e], HadamardScale<D>::value);
+        amax = fmaxf(amax, fabsf(r[e]));
+    }
+    amax = warp_max(amax);
+    const float s = __fdiv_rn(fmaxf(amax, 1e-4f), 448.0f);
+    uint32_t packed = 0;
+#pragma unroll
+    for (int e = 0; e < E; e += 2)
+        packed |= e4m3x2_rn_sat(__fdiv_rn(r[e], s), __fdiv_rn(r[e + 1], s)) << (8 * e);
+    *scale = s;
+    return packed;
+}
+
+// Loads this lane's E elements of a D-vector (fp32 or bf16).
+template <int D, typename T>
+__device__ __forceinline__ void load_lane_slice(const T *vec, float (&r)[D / 32]) {
+    constexpr int E = D / 32;
+    const int lane = threadIdx.x & 31;
+    const T *src = vec + lane * E;
+    if constexpr (E == 4 && sizeof(T) == 4) {
+        const float4 t = *reinterpret_cast<const float4 *>(src);
+        r[0] = t.x; r[1] = t.y; r[2] = t.z; r[3] = t.w;
+    } else if constexpr (E == 2 && sizeof(T) == 4) {
+        const float2 t = *reinterpret_cast<const float2 *>(src);
+        r[0] = t.x; r[1] = t.y;
+    } else {
+#pragma unroll
+        for (int e = 0; e < E; e++) r[e] = to_f32<T>(src[e]);
+    }
+}
+
+}  // namespace dsa

@@ -9,21 +9,27 @@
 // Shapes: Hq = 128 heads (the MMA M), rows [c (512) | k_pe (64)] bf16.
 // One CTA computes, for one query row, one 256-wide half of the output over
 // one share ("split") of the selected rows:
-//   warp 0      gathers 32 selected rows per tile with TMA tile::gather4 into
-//               a 4-stage ring; each tile is nine 64-column blocks of 32 rows
-//               x 128 B, 128B-swizzled (no multicast);
-//   warp 1      S = Q C^T: 36 tcgen05.mma kind::f16 (M=128, N=32, K=16), with
-//               Q columns 0..319 read from TMEM and 320..575 from shared
-//               memory; O += P C[:, half]: 2 MMAs (N=256, K=16) whose A = P
-//               comes from TMEM and whose B is the same shared tile read as an
-//               MN-major operand (no transpose copy);
-//   warps 2..5  one thread per head: online softmax in the exp2 domain with
+//   warps 5..8  gather 32 selected rows per tile into a 2-stage ring with
+//               16-byte cp.async, straight into the 128B-swizzled K-major
+//               layout (nine 64-column blocks of 32 rows x 128 B); each warp
+//               copies 8 rows, consecutive lanes consecutive 16-byte pieces;
+//               a tile is published (wait, proxy fence, arrive) two tiles
+//               later, or at once before the producer would block;
+//   warp 0      S = Q C^T: 36 tcgen05.mma kind::f16 (M=128, N=32, K=16) per
+//               tile with both operands in shared memory (the whole query,
+//               144 KB, is loaded once by TMA); O += P C[:, half]: 2 MMAs
+//               (N=256, K=16) with A = P from TMEM and B = the same shared
+//               tile read as an MN-major operand (no transpose copy).  The
+//               previous tile's PV is slotted between this tile's QK column
+//               blocks as soon as its P is ready, so its stage is freed early;
+//   warps 1..4  one thread per head: online softmax in the exp2 domain with
 //               lazy rescaling (the fp32 accumulator in TMEM is rescaled only
 //               when a head's running max grows by more than 8), P written to
 //               TMEM as bf16, then the epilogue.
-// TMEM (512 columns): O 256 | S 2 x 32 | P 2 x 16 | Q 160.  The logits are
-// computed by both halves of a row (the output accumulator alone fills TMEM),
-// so each gathered row is read twice from L2 but once from HBM.
+// TMEM: O 256 | S 2 x 32 | P 2 x 16 columns.  The logits are computed by both
+// halves of a row (the output accumulator alone fills half of TMEM and the
+// query fills most of shared memory), so each gathered row is read twice from
+// L2 but once from HBM.
 // With several splits per row, unnormalised partial outputs and (max, sum)
 // pairs go to the workspace and a combine kernel merges them.
 #include "common.cuh"
@@ -37,23 +43,23 @@ constexpr int kHq = 128, kDc = 512, kDr = 64, kDqk = kDc + kDr;
 constexpr int kNB = kDqk / 64;                  // 64-column blocks per row: 9
 constexpr int kDh = 256;                        // output columns per CTA
 constexpr int kRows = 32;                       // gathered rows per tile
-constexpr int kStages = 4;
-constexpr int kQT = 5;                          // Q blocks held in TMEM (dims 0..319)
-constexpr int kQS = kNB - kQT;                  // Q blocks in shared memory
-constexpr int kThreads = 192;
+constexpr int kStages = 2;
+constexpr int kThreads = 288;               // warp 0 MMA, 1..4 softmax, 5..8 gather
 constexpr int kMaxSel = 2048;                   // selection slots held in shared memory
-constexpr uint32_t kColO = 0, kColS = 256, kColP = 320, kColQ = 352, kTmemCols = 512;
+constexpr uint32_t kColO = 0, kColS = 256, kColP = 320, kTmemCols = 512;
 constexpr int kBlk = kRows * 128;               // bytes of one column block of a tile
 constexpr int kTileBytes = kNB * kBlk;          // 36864
 constexpr int kQBlk = kHq * 128;                // 16384
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
 
-constexpr size_t kSmemBytes = 1024 + (size_t)kStages * kTileBytes + (size_t)kQS * kQBlk +
+constexpr size_t kSmemBytes = 1024 + (size_t)kStages * kTileBytes + (size_t)kNB * kQBlk +
                               kMaxSel * sizeof(int32_t) + 32 * sizeof(uint64_t) + 64;
+constexpr int kLag = 2;                          // gather tiles in flight per thread beyond the one issued
 
 struct MlaArgs {
     const __nv_bfloat16 *q;
+    const __nv_bfloat16 *kv;
     const int32_t *idx;
     __nv_bfloat16 *out;
     float *lse;
@@ -66,7 +72,16 @@ struct MlaArgs {
     int *err;
 };
 
-__device__ __forceinline__ int block_scan_flag192(bool flag, int *warp_tot, int *total) {
+__device__ __forceinline__ void cp_async16(void *dst, const void *src) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(tc::smem_u32(dst)), "l"(src)
+                 : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N> __device__ __forceinline__ void cp_async_wait() {
+    asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+
+__device__ __forceinline__ int block_scan_flag_all(bool flag, int *warp_tot, int *total) {
     constexpr int kW = kThreads / 32;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const unsigned ballot = __ballot_sync(0xffffffffu, flag);
@@ -90,14 +105,13 @@ __device__ __forceinline__ int block_scan_flag192(bool flag, int *warp_tot, int 
 }
 
 __global__ void __launch_bounds__(kThreads, 1)
-sparse_mla_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
-                     const __grid_constant__ CUtensorMap tm_kv, const MlaArgs a) {
+sparse_mla_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const MlaArgs a) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t *sc = smem;                                      // C tiles
-    uint8_t *sq = sc + kStages * kTileBytes;                 // Q blocks kQT..kNB-1
-    int32_t *list = reinterpret_cast<int32_t *>(sq + kQS * kQBlk);
+    uint8_t *sq = sc + kStages * kTileBytes;                 // Q, nine 64-column blocks
+    int32_t *list = reinterpret_cast<int32_t *>(sq + kNB * kQBlk);
     uint64_t *bars = reinterpret_cast<uint64_t *>(list + kMaxSel);
     uint64_t *c_full = bars, *c_empty = bars + kStages;
     uint64_t *s_full = bars + 2 * kStages, *s_empty = s_full + 2;
@@ -105,7 +119,7 @@ sparse_mla_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
     uint64_t *q_full = pv_done + 2, *q_ready = q_full + 1;
     uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(q_ready + 1);
     volatile int *abort = reinterpret_cast<volatile int *>(tmem_holder + 1);
-    int *scan_tmp = const_cast<int *>(abort) + 1;            // 8 ints
+    int *scan_tmp = const_cast<int *>(abort) + 1;            // 10 ints
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int unit = blockIdx.x;                             // (row * 2 + half) * splits + sp
@@ -114,16 +128,60 @@ sparse_mla_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
     const int64_t row = unit / (a.splits * 2);
     const int64_t b = row / a.S, s = row - b * a.S;
     const int64_t limit = a.start_pos + s;
+    const bool is_softmax = warp >= 1 && warp <= 4;
+    const int quarter = warp & 3;                            // softmax warps: TMEM lane quarter
+    const int h = quarter * 32 + lane;                       // softmax warps: head
+    const uint32_t lane_addr = (uint32_t)(quarter * 32) << 16;
+
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < kStages; i++) {
+            tc::mbar_init(&c_full[i], 128);
+            tc::mbar_init(&c_empty[i], 1);
+        }
+        for (int i = 0; i < 2; i++) {
+            tc::mbar_init(&s_full[i], 1);
+            tc::mbar_init(&s_empty[i], 128);
+            tc::mbar_init(&p_full[i], 128);
+            tc::mbar_init(&pv_done[i], 1);
+        }
+        tc::mbar_init(q_full, 1);
+        *abort = 0;
+        tc::fence_mbar_init();
+        tc::tma_prefetch_desc(&tm_q);
+    }
+    if (warp == 0) {
+        tc::tmem_alloc(tmem_holder, kTmemCols);
+        tc::tmem_relinquish();
+    }
+    tc::tc_fence_before();
+    __syncthreads();
+    tc::tc_fence_after();
+    const uint32_t tmem = *tmem_holder;
+
+    // the query does not depend on the preceding kernel: load it first
+    if (threadIdx.x == 160) {
+        tc::mbar_arrive_expect_tx(q_full, kNB * kQBlk);
+        for (int j = 0; j < kNB; j++)
+            tc::tma_load_2d(sq + j * kQBlk, &tm_q, j * 64, (int)(row * kHq), q_full);
+    }
 
     // valid selections of this row, in slot order
+    constexpr int kPer = (kMaxSel + kThreads - 1) / kThreads;
+    int32_t slot[kPer];
+#pragma unroll
+    for (int r = 0; r < kPer; r++) {
+        const int j = r * kThreads + threadIdx.x;
+        slot[r] = j < a.k ? __ldg(a.idx + row * a.k + j) : -1;
+    }
     int n = 0;
-    for (int base = 0; base < a.k; base += kThreads) {
-        const int j = base + threadIdx.x;
-        const int32_t t = j < a.k ? a.idx[row * a.k + j] : -1;
+#pragma unroll
+    for (int r = 0; r < kPer; r++) {
+        if (r * kThreads >= a.k) break;
+        const int32_t t = slot[r];
         const bool v = t >= 0 && (int64_t)t <= limit && (int64_t)t < a.t_max;
         if (t >= 0 && (int64_t)t <= limit && (int64_t)t >= a.t_max) record_error(a.err, DSA_ERR_DEVICE);
         int tot;
-        const int pos = block_scan_flag192(v, scan_tmp, &tot);
+        const int pos = block_scan_flag_all(v, scan_tmp, &tot);
         if (v) list[n + pos] = t;
         n += tot;
     }
@@ -132,8 +190,8 @@ sparse_mla_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
     const int n_tiles = (n_my + kRows - 1) / kRows;
 
     if (n_tiles == 0) {                                      // nothing selected here
-        if (warp >= 2) {
-            const int h = (warp & 3) * 32 + lane;
+        if (threadIdx.x == 160) tc::mbar_wait(q_full, 0, a.err, abort);   // Q copy landed
+        if (is_softmax) {
             if (a.splits > 1) {
                 float4 *po = reinterpret_cast<float4 *>(a.part_o + ((int64_t)unit * kHq + h) * kDh);
                 for (int c = 0; c < kDh / 4; c++) po[c] = make_float4(0.f, 0.f, 0.f, 0.f);
@@ -144,101 +202,59 @@ sparse_mla_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
                 if (half == 0 && a.lse) a.lse[row * kHq + h] = -INFINITY;
             }
         }
-        return;
-    }
-
-    if (threadIdx.x == 0) {
-        for (int i = 0; i < kStages; i++) {
-            tc::mbar_init(&c_full[i], 1);
-            tc::mbar_init(&c_empty[i], 1);
-        }
-        for (int i = 0; i < 2; i++) {
-            tc::mbar_init(&s_full[i], 1);
-            tc::mbar_init(&s_empty[i], 128);
-            tc::mbar_init(&p_full[i], 128);
-            tc::mbar_init(&pv_done[i], 1);
-        }
-        tc::mbar_init(q_full, 1);
-        tc::mbar_init(q_ready, 128);
-        *abort = 0;
-        tc::fence_mbar_init();
-        tc::tma_prefetch_desc(&tm_q);
-        tc::tma_prefetch_desc(&tm_kv);
-    }
-    if (warp == 1) {
-        tc::tmem_alloc(tmem_holder, kTmemCols);
-        tc::tmem_relinquish();
-    }
-    tc::tc_fence_before();
-    __syncthreads();
-    tc::tc_fence_after();
-    const uint32_t tmem = *tmem_holder;
-
-    if (warp == 0) {
-        if (lane == 0) {
-            tc::mbar_arrive_expect_tx(q_full, kQS * kQBlk);
-            for (int j = 0; j < kQS; j++)
-                tc::tma_load_2d(sq + j * kQBlk, &tm_q, (kQT + j) * 64, (int)(row * kHq), q_full);
-            const int64_t rbase = b * a.t_max;
-            int issued = 0;
-            for (int i = 0; i < n_tiles; i++) {
-                const int st = i % kStages;
-                if (!tc::mbar_wait(&c_empty[st], ((uint32_t)(i / kStages) & 1u) ^ 1u, a.err, abort))
-                    break;
-                tc::mbar_arrive_expect_tx(&c_full[st], kTileBytes);
-                uint8_t *dst = sc + st * kTileBytes;
-                for (int g = 0; g < kRows / 4; g++) {
-                    int r[4];
-#pragma unroll
-                    for (int e = 0; e < 4; e++) {
-                        int j = i * kRows + g * 4 + e;
-                        if (j >= n_my) j = n_my - 1;                 // padding: a valid row
-                        r[e] = (int)(rbase + list[lo + j]);
-                    }
-#pragma unroll
-                    for (int cb = 0; cb < kNB; cb++)
-                        tc::tma_gather4(dst + cb * kBlk + g * 512, &tm_kv, cb * 64, r[0], r[1],
-                                        r[2], r[3], &c_full[st]);
-                }
-                issued = i + 1;
+    } else if (warp >= 5) {
+        // ---- gather: warp w copies rows 8w..8w+7 of each tile; lane l copies
+        // the 16-byte pieces l, l+32, l+64 (< 72) of each row
+        const int pw = warp - 5;
+        const int64_t rbase = b * a.t_max;
+        int issued = 0, signalled = 0;
+        for (int i = 0; i < n_tiles; i++) {
+            const int st = i % kStages;
+            const uint32_t ph = ((uint32_t)(i / kStages) & 1u) ^ 1u;
+            if (!tc::mbar_test_wait(&c_empty[st], ph)) {
+                // about to block: first publish every tile issued so far, since
+                // the stage we wait for is freed only after they are consumed
+                cp_async_wait<0>();
+                tc::fence_proxy_async_smem();
+                for (; signalled < issued; signalled++) tc::mbar_arrive(&c_full[signalled % kStages]);
+                if (!tc::mbar_wait(&c_empty[st], ph, a.err, abort)) break;
             }
-            for (int j = issued > kStages ? issued - kStages : 0; j < issued; j++)
-                tc::mbar_wait(&c_full[j % kStages], (uint32_t)(j / kStages) & 1u, a.err, abort);
+            uint8_t *tile = sc + st * kTileBytes;
+#pragma unroll 1
+            for (int jj = 0; jj < 8; jj++) {
+                const int j = pw * 8 + jj;
+                int r = i * kRows + j;
+                if (r >= n_my) r = n_my - 1;                 // padding: a valid row
+                const __nv_bfloat16 *src = a.kv + (rbase + list[lo + r]) * kDqk;
+#pragma unroll
+                for (int u = 0; u < 3; u++) {
+                    const int c = lane + 32 * u;
+                    if (c < 72)
+                        cp_async16(tile + (c >> 3) * kBlk + j * 128 + (((c & 7) ^ (j & 7)) << 4),
+                                   src + c * 8);
+                }
+            }
+            cp_async_commit();
+            issued = i + 1;
+            if (issued - signalled > kLag) {
+                cp_async_wait<kLag>();
+                tc::fence_proxy_async_smem();
+                tc::mbar_arrive(&c_full[signalled % kStages]);
+                signalled++;
+            }
         }
-    } else if (warp == 1) {
+        cp_async_wait<0>();
+        tc::fence_proxy_async_smem();
+        for (; signalled < issued; signalled++) tc::mbar_arrive(&c_full[signalled % kStages]);
+    } else if (warp == 0) {
         if (lane == 0) {
             const uint32_t id_qk = tc::instr_desc(tc::kFmtBF16, tc::kFmtBF16, 128, kRows);
             const uint32_t id_pv = tc::instr_desc(tc::kFmtBF16, tc::kFmtBF16, 128, kDh, true);
             const uint32_t sc_addr = tc::smem_u32(sc), sq_addr = tc::smem_u32(sq);
-            bool ok = tc::mbar_wait(q_full, 0, a.err, abort) && tc::mbar_wait(q_ready, 0, a.err, abort);
-            auto qk = [&](int i) -> bool {
-                const int st = i % kStages, sb = i & 1;
-                if (!tc::mbar_wait(&c_full[st], (uint32_t)(i / kStages) & 1u, a.err, abort)) return false;
-                if (!tc::mbar_wait(&s_empty[sb], ((uint32_t)(i >> 1) & 1u) ^ 1u, a.err, abort)) return false;
-                tc::tc_fence_after();
-                const uint32_t d = tmem + kColS + sb * kRows;
-#pragma unroll 1
-                for (int cb = 0; cb < kNB; cb++) {
-#pragma unroll
-                    for (int ks = 0; ks < 4; ks++) {
-                        const uint64_t bd = tc::smem_desc(sc_addr + st * kTileBytes + cb * kBlk + ks * 32,
-                                                          1024, tc::kSwizzle128B);
-                        const bool acc = (cb | ks) != 0;
-                        if (cb < kQT) {
-                            tc::mma_f16_ts(d, tmem + kColQ + cb * 32 + ks * 8, bd, id_qk, acc);
-                        } else {
-                            const uint64_t ad = tc::smem_desc(sq_addr + (cb - kQT) * kQBlk + ks * 32,
-                                                              1024, tc::kSwizzle128B);
-                            tc::mma_f16(d, ad, bd, id_qk, acc);
-                        }
-                    }
-                }
-                tc::tc_commit(&s_full[sb]);
-                return true;
-            };
-            auto pv = [&](int j) -> bool {
+            bool ok = tc::mbar_wait(q_full, 0, a.err, abort);
+            // O += P C[:, half] for tile j (P(j) must be published)
+            auto pv_issue = [&](int j) {
                 const int st = j % kStages, pb = j & 1;
-                if (!tc::mbar_wait(&p_full[pb], (uint32_t)(j >> 1) & 1u, a.err, abort)) return false;
                 tc::tc_fence_after();
 #pragma unroll
                 for (int ks = 0; ks < kRows / 16; ks++) {
@@ -250,33 +266,45 @@ sparse_mla_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
                 }
                 tc::tc_commit(&c_empty[st]);
                 tc::tc_commit(&pv_done[pb]);
+            };
+            // S = Q C^T for tile i, one 64-column block at a time; the PV of the
+            // previous tile (pend >= 0) is slotted in as soon as its P is
+            // published, so its stage is released without waiting for all of
+            // this tile's MMAs
+            auto qk = [&](int i, int pend) -> bool {
+                const int st = i % kStages, sb = i & 1;
+                if (!tc::mbar_wait(&c_full[st], (uint32_t)(i / kStages) & 1u, a.err, abort)) return false;
+                if (!tc::mbar_wait(&s_empty[sb], ((uint32_t)(i >> 1) & 1u) ^ 1u, a.err, abort)) return false;
+                tc::tc_fence_after();
+                const uint32_t d = tmem + kColS + sb * kRows;
+#pragma unroll 1
+                for (int cb = 0; cb < kNB; cb++) {
+                    if (pend >= 0 && tc::mbar_test_wait(&p_full[pend & 1], (uint32_t)(pend >> 1) & 1u)) {
+                        pv_issue(pend);
+                        pend = -1;
+                    }
+#pragma unroll
+                    for (int ks = 0; ks < 4; ks++) {
+                        const uint64_t ad = tc::smem_desc(sq_addr + cb * kQBlk + ks * 32, 1024, tc::kSwizzle128B);
+                        const uint64_t bd = tc::smem_desc(sc_addr + st * kTileBytes + cb * kBlk + ks * 32,
+                                                          1024, tc::kSwizzle128B);
+                        tc::mma_f16(d, ad, bd, id_qk, (cb | ks) != 0);
+                    }
+                }
+                tc::tc_commit(&s_full[sb]);
+                if (pend >= 0) {
+                    if (!tc::mbar_wait(&p_full[pend & 1], (uint32_t)(pend >> 1) & 1u, a.err, abort)) return false;
+                    pv_issue(pend);
+                }
                 return true;
             };
-            if (ok) ok = qk(0);
-            for (int i = 1; ok && i < n_tiles; i++) ok = qk(i) && pv(i - 1);
-            if (ok) pv(n_tiles - 1);
+            if (ok) ok = qk(0, -1);
+            for (int i = 1; ok && i < n_tiles; i++) ok = qk(i, i - 1);
+            if (ok && tc::mbar_wait(&p_full[(n_tiles - 1) & 1], (uint32_t)((n_tiles - 1) >> 1) & 1u, a.err, abort))
+                pv_issue(n_tiles - 1);
         }
     } else {
-        const int quarter = warp & 3;
-        const int h = quarter * 32 + lane;
-        const uint32_t lane_addr = (uint32_t)(quarter * 32) << 16;
-        // Q columns 0..319 -> TMEM (two bf16 per column)
-        {
-            const uint4 *qrow = reinterpret_cast<const uint4 *>(a.q + (row * kHq + h) * kDqk);
-#pragma unroll 1
-            for (int c0 = 0; c0 < kQT * 32; c0 += 16) {
-                uint32_t r[16];
-#pragma unroll
-                for (int v = 0; v < 4; v++) {
-                    const uint4 x = __ldg(qrow + c0 / 4 + v);
-                    r[4 * v] = x.x; r[4 * v + 1] = x.y; r[4 * v + 2] = x.z; r[4 * v + 3] = x.w;
-                }
-                tc::tmem_st16(tmem + lane_addr + kColQ + c0, r);
-            }
-            tc::tmem_wait_st();
-            tc::tc_fence_before();
-            tc::mbar_arrive(q_ready);
-        }
+        // ---- softmax warps
         float m_run = -INFINITY, l = 0.f;
         bool ok = true;
         for (int i = 0; i < n_tiles && ok; i++) {
@@ -378,48 +406,49 @@ sparse_mla_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
 
     tc::tc_fence_before();
     __syncthreads();
-    if (warp == 1) {
+    if (warp == 0) {
         tc::tc_fence_after();
         tc::tmem_dealloc(tmem, kTmemCols);
     }
 }
 
 // Merges the splits of each (row, half): out = sum_s 2^(m_s - m) O_s / sum_s 2^(m_s - m) l_s.
-__global__ void __launch_bounds__(128)
+// One warp per head; lane l covers output columns 8l..8l+7 (coalesced rows).
+constexpr int kCombineHeads = 8;
+__global__ void __launch_bounds__(32 * kCombineHeads)
 sparse_mla_combine_kernel(const float *__restrict__ part_o, const float2 *__restrict__ part_ml,
                           int splits, __nv_bfloat16 *__restrict__ out, float *__restrict__ lse) {
-    const int64_t row = blockIdx.x >> 1;
-    const int half = blockIdx.x & 1;
-    const int h = threadIdx.x;
-    const int64_t u0 = (row * 2 + half) * splits;
+    const int groups = kHq / kCombineHeads;
+    const int64_t rh = blockIdx.x / groups;                 // row * 2 + half
+    const int64_t row = rh >> 1;
+    const int half = (int)(rh & 1);
+    const int h = (int)(blockIdx.x % groups) * kCombineHeads + (threadIdx.x >> 5);
+    const int lane = threadIdx.x & 31;
+    const int64_t u0 = rh * splits;
     float m = -INFINITY;
     for (int sp = 0; sp < splits; sp++) m = fmaxf(m, part_ml[(u0 + sp) * kHq + h].x);
     float L = 0.f;
+    float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
     for (int sp = 0; sp < splits; sp++) {
         const float2 ml = part_ml[(u0 + sp) * kHq + h];
-        if (ml.x != -INFINITY) L += exp2f(ml.x - m) * ml.y;
+        if (ml.x == -INFINITY) continue;
+        const float w = exp2f(ml.x - m);
+        L += w * ml.y;
+        const float4 *po = reinterpret_cast<const float4 *>(part_o + ((u0 + sp) * kHq + h) * kDh) + 2 * lane;
+        const float4 x = po[0], y = po[1];
+        acc[0] += w * x.x; acc[1] += w * x.y; acc[2] += w * x.z; acc[3] += w * x.w;
+        acc[4] += w * y.x; acc[5] += w * y.y; acc[6] += w * y.z; acc[7] += w * y.w;
     }
     const float inv = L > 0.f ? 1.f / L : 0.f;
-    uint4 *o16 = reinterpret_cast<uint4 *>(out + (row * kHq + h) * kDc + half * kDh);
-    for (int c0 = 0; c0 < kDh; c0 += 8) {
-        float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-        for (int sp = 0; sp < splits; sp++) {
-            const float mx = part_ml[(u0 + sp) * kHq + h].x;
-            if (mx == -INFINITY) continue;
-            const float w = exp2f(mx - m);
-            const float4 *po = reinterpret_cast<const float4 *>(part_o + ((u0 + sp) * kHq + h) * kDh + c0);
-            const float4 x = po[0], y = po[1];
-            acc[0] += w * x.x; acc[1] += w * x.y; acc[2] += w * x.z; acc[3] += w * x.w;
-            acc[4] += w * y.x; acc[5] += w * y.y; acc[6] += w * y.z; acc[7] += w * y.w;
-        }
-        uint32_t wv[4];
-        for (int e = 0; e < 4; e++) {
-            const __nv_bfloat162 v = __floats2bfloat162_rn(acc[2 * e] * inv, acc[2 * e + 1] * inv);
-            wv[e] = *reinterpret_cast<const uint32_t *>(&v);
-        }
-        o16[c0 / 8] = make_uint4(wv[0], wv[1], wv[2], wv[3]);
+    uint32_t wv[4];
+#pragma unroll
+    for (int e = 0; e < 4; e++) {
+        const __nv_bfloat162 v = __floats2bfloat162_rn(acc[2 * e] * inv, acc[2 * e + 1] * inv);
+        wv[e] = *reinterpret_cast<const uint32_t *>(&v);
     }
-    if (half == 0 && lse) lse[row * kHq + h] = L > 0.f ? (m + log2f(L)) * kLn2 : -INFINITY;
+    reinterpret_cast<uint4 *>(out + (row * kHq + h) * kDc + half * kDh)[lane] =
+        make_uint4(wv[0], wv[1], wv[2], wv[3]);
+    if (half == 0 && lse && lane == 0) lse[row * kHq + h] = L > 0.f ? (m + log2f(L)) * kLn2 : -INFINITY;
 }
 
 int mla_splits(int64_t rows, int k) {
@@ -450,7 +479,7 @@ dsa_status launch_sparse_mla_tc(const void *q, const void *kv, int64_t t_max, co
                                 int B, int S, int k, int64_t start_pos, float sm_scale, void *out,
                                 float *lse, void *ws, cudaStream_t stream) {
     const int64_t rows = (int64_t)B * S;
-    CUtensorMap tm_q, tm_kv;
+    CUtensorMap tm_q;
     {
         const uint64_t dims[2] = {(uint64_t)kDqk, (uint64_t)(rows * kHq)};
         const uint64_t strides[1] = {(uint64_t)kDqk * 2};
@@ -459,16 +488,9 @@ dsa_status launch_sparse_mla_tc(const void *q, const void *kv, int64_t t_max, co
                          CU_TENSOR_MAP_SWIZZLE_128B))
             return DSA_ERR_CUDA;
     }
-    {
-        const uint64_t dims[2] = {(uint64_t)kDqk, (uint64_t)(B * t_max)};
-        const uint64_t strides[1] = {(uint64_t)kDqk * 2};
-        const uint32_t box[2] = {64, 1};
-        if (!encode_tmap(&tm_kv, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, kv, dims, strides, box,
-                         CU_TENSOR_MAP_SWIZZLE_128B))
-            return DSA_ERR_CUDA;
-    }
     MlaArgs a;
     a.q = static_cast<const __nv_bfloat16 *>(q);
+    a.kv = static_cast<const __nv_bfloat16 *>(kv);
     a.idx = idx;
     a.out = static_cast<__nv_bfloat16 *>(out);
     a.lse = lse;
@@ -490,12 +512,11 @@ dsa_status launch_sparse_mla_tc(const void *q, const void *kv, int64_t t_max, co
     if (cudaFuncSetAttribute(sparse_mla_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)kSmemBytes) != cudaSuccess)
         return DSA_ERR_CUDA;
-    sparse_mla_tc_kernel<<<(unsigned)(rows * 2 * a.splits), kThreads, kSmemBytes, stream>>>(
-        tm_q, tm_kv, a);
+    sparse_mla_tc_kernel<<<(unsigned)(rows * 2 * a.splits), kThreads, kSmemBytes, stream>>>(tm_q, a);
     dsa_status st = launch_status();
     if (st != DSA_OK || a.splits == 1) return st;
-    sparse_mla_combine_kernel<<<(unsigned)(rows * 2), kHq, 0, stream>>>(
-        a.part_o, a.part_ml, a.splits, a.out, lse);
+    sparse_mla_combine_kernel<<<(unsigned)(rows * 2 * (kHq / kCombineHeads)), 32 * kCombineHeads,
+                                0, stream>>>(a.part_o, a.part_ml, a.splits, a.out, lse);
     return launch_status();
 }
 

@@ -18,9 +18,11 @@
 // distributed shared memory by CTA 0, which broadcasts the decision:
 //   round 0: 2048 bins linear in value between the row's finite min and max
 //            (well spread for smooth score distributions, so shared-memory
-//            atomics rarely collide and the threshold bin is small);
-//   rounds 1-3: exact radix select on the order-preserving 32-bit keys
-//            (11 + 11 + 10 bits), over the threshold-bin candidates only.
+//            atomics rarely collide and the threshold bin is small), merged
+//            into CTA 0 with distributed shared-memory atomics;
+//   then the threshold-bin candidates' keys are gathered into CTA 0, which
+//   finds the exact k-th key alone (11 + 11 + 10-bit radix passes); if there
+//   are too many candidates, the radix passes run cluster-wide instead.
 // Then every CTA counts its x > tau and x == tau, the counts are exchanged,
 // and each CTA writes its selected positions at its offset in position order.
 // Cluster barriers are hardware barriers between co-scheduled CTAs.
@@ -39,7 +41,7 @@ namespace {
 constexpr int kThreads = 1024;
 constexpr int kWarps = kThreads / 32;
 constexpr int kBins = 2048;
-constexpr int kMaxSlice = 36864;     // scores per CTA kept in shared memory
+constexpr int kMaxSlice = 28672;     // scores per CTA kept in shared memory
 
 // Block-wide exclusive scan of a 0/1 flag; *total receives the block total.
 // All threads must call it.
@@ -63,6 +65,35 @@ __device__ __forceinline__ int block_scan_flag(bool flag, int *warp_tot, int *to
     __syncthreads();
     const int r = warp_tot[warp] + in_warp;
     *total = warp_tot[32];
+    __syncthreads();
+    return r;
+}
+
+// Block-wide exclusive scan of an int; *total receives the block total.
+__device__ __forceinline__ int block_scan_int(int v, int *tmp, int *total) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    int incl = v;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int n = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += n;
+    }
+    if (lane == 31) tmp[warp] = incl;
+    __syncthreads();
+    if (warp == 0) {
+        const int wv = lane < kWarps ? tmp[lane] : 0;
+        int wi = wv;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int n = __shfl_up_sync(0xffffffffu, wi, o);
+            if (lane >= o) wi += n;
+        }
+        if (lane < kWarps) tmp[lane] = wi - wv;
+        if (lane == 31) tmp[32] = wi;
+    }
+    __syncthreads();
+    const int r = tmp[warp] + incl - v;
+    *total = tmp[32];
     __syncthreads();
     return r;
 }
@@ -133,8 +164,43 @@ __device__ __forceinline__ int linear_bin(float x, float lo, float scale) {
 struct ClusterCtl {
     float lo, hi;           // this CTA's finite min / max
     unsigned bin, rank;     // broadcast by CTA 0
+    int n_cand;             // this CTA's threshold-bin candidates
     int n_gt, n_eq;         // this CTA's counts of x > tau, x == tau
 };
+
+// Slice element i lives at sv[pad(i)]: one spare word every 32 keeps the
+// per-thread contiguous segments (stride seg words) off a single bank.
+__device__ __forceinline__ int pad(int i) { return i + (i >> 5); }
+
+// Exact rank search among n keys held in shared memory by one CTA: the
+// rank-th largest key (11 + 11 + 10-bit radix passes) and the rank left
+// among the keys equal to it.
+__device__ void cta_select_keys(const uint32_t *keys, int n, unsigned rank, unsigned *hist,
+                                unsigned *scan_tmp, unsigned *s_bin, unsigned *s_rank,
+                                uint32_t *tau_out, unsigned *rank_out) {
+    uint32_t prefix = 0, mask = 0;
+    const int shifts[3] = {21, 10, 0};
+    const int widths[3] = {11, 11, 10};
+    for (int rd = 0; rd < 3; rd++) {
+        const uint32_t dm = (1u << widths[rd]) - 1u;
+        for (int i = threadIdx.x; i <= (int)dm; i += kThreads) hist[i] = 0;
+        __syncthreads();
+        for (int j = threadIdx.x; j < n; j += kThreads) {
+            const uint32_t key = keys[j];
+            if ((key & mask) == prefix) atomicAdd(&hist[(key >> shifts[rd]) & dm], 1u);
+        }
+        __syncthreads();
+        find_rank_bin(hist, (int)dm + 1, rank, s_bin, s_rank, scan_tmp);
+        prefix |= *s_bin << shifts[rd];
+        mask |= dm << shifts[rd];
+        rank = *s_rank;
+        __syncthreads();
+    }
+    *tau_out = prefix;
+    *rank_out = rank;
+}
+
+constexpr int kGather = 8192;      // candidates CTA 0 can select alone
 
 __global__ void __launch_bounds__(kThreads, 1)
 topk_cluster_kernel(const float *__restrict__ scores, int S, int64_t T, int64_t start_pos, int K,
@@ -155,14 +221,17 @@ topk_cluster_kernel(const float *__restrict__ scores, int S, int64_t T, int64_t 
         return;                           // uniform across the cluster
     }
 
-    extern __shared__ float sv[];                                   // [L] scores
-    uint16_t *cand = reinterpret_cast<uint16_t *>(sv + L);          // [L] candidate slots
-    __shared__ unsigned hist[kBins];
+    extern __shared__ float sv[];                                   // [pad(L)] scores
+    uint32_t *gath = reinterpret_cast<uint32_t *>(sv + pad(L) + 1);  // [kGather] keys (CTA 0)
+    uint16_t *cand = reinterpret_cast<uint16_t *>(gath + kGather);  // [L] candidate slots
+    __shared__ unsigned hist[kBins];          // local histogram
+    __shared__ unsigned hmerged[kBins];       // cluster histogram (CTA 0)
     __shared__ unsigned scan_tmp[33];
     __shared__ int itmp[33];
     __shared__ ClusterCtl ctl;
-    __shared__ float s_lo, s_hi;
     __shared__ unsigned s_bin, s_rank;
+    __shared__ uint32_t s_tau;
+    __shared__ float s_lo, s_hi;
 
     const int64_t t0 = (int64_t)p * L;
     int64_t t1 = t0 + L;
@@ -170,15 +239,19 @@ topk_cluster_kernel(const float *__restrict__ scores, int S, int64_t T, int64_t 
     const int len = t1 > t0 ? (int)(t1 - t0) : 0;
     const float *src = scores + row * T + t0;
 
-    // load the slice, finite min / max
+    // load the slice, finite min / max; clear the histograms
     float lo = INFINITY, hi = -INFINITY;
     for (int i = threadIdx.x; i < len; i += kThreads) {
         const float x = src[i];
-        sv[i] = x;
+        sv[pad(i)] = x;
         if (isfinite(x)) {
             lo = fminf(lo, x);
             hi = fmaxf(hi, x);
         }
+    }
+    for (int i = threadIdx.x; i < kBins; i += kThreads) {
+        hist[i] = 0;
+        hmerged[i] = 0;
     }
     lo = -warp_max(-lo);
     hi = warp_max(hi);
@@ -196,8 +269,7 @@ topk_cluster_kernel(const float *__restrict__ scores, int S, int64_t T, int64_t 
         ctl.lo = l;
         ctl.hi = h;
     }
-    for (int i = threadIdx.x; i < kBins; i += kThreads) hist[i] = 0;
-    cl.sync();
+    cl.sync();                                                            // (1)
     if (threadIdx.x == 0) {
         float l = INFINITY, h = -INFINITY;
         for (int r = 0; r < CN; r++) {
@@ -213,88 +285,126 @@ topk_cluster_kernel(const float *__restrict__ scores, int S, int64_t T, int64_t 
     const float scale = (g_hi > g_lo && isfinite(g_hi - g_lo)) ? __fdiv_rn((float)kBins, g_hi - g_lo)
                                                                   : 0.f;
 
-    // round 0: linear bins
-    for (int i = threadIdx.x; i < len; i += kThreads) atomicAdd(&hist[linear_bin(sv[i], g_lo, scale)], 1u);
-    cl.sync();
+    // round 0: linear bins, merged into CTA 0 with distributed shared-memory atomics
+    for (int i = threadIdx.x; i < len; i += kThreads)
+        atomicAdd(&hist[linear_bin(sv[pad(i)], g_lo, scale)], 1u);
+    __syncthreads();
+    {
+        unsigned *h0 = cl.map_shared_rank(hmerged, 0);
+        for (int b = threadIdx.x; b < kBins; b += kThreads)
+            if (hist[b]) atomicAdd(h0 + b, hist[b]);
+    }
+    cl.sync();                                                            // (2)
     if (p == 0) {
-        for (int b = threadIdx.x; b < kBins; b += kThreads) {
-            unsigned v = hist[b];
-            for (int r = 1; r < CN; r++) v += cl.map_shared_rank(hist, r)[b];
-            hist[b] = v;    // own histogram is no longer needed by anyone else
-        }
-        __syncthreads();
-        find_rank_bin(hist, kBins, (unsigned)m, &s_bin, &s_rank, scan_tmp);
+        find_rank_bin(hmerged, kBins, (unsigned)m, &s_bin, &s_rank, scan_tmp);
         if (threadIdx.x < CN) {
             ClusterCtl *rc = cl.map_shared_rank(&ctl, (int)threadIdx.x);
             rc->bin = s_bin;
             rc->rank = s_rank;
         }
     }
-    cl.sync();
+    cl.sync();                                                            // (3)
     const int tb = (int)ctl.bin;
     unsigned rank = ctl.rank;
 
-    // candidates of the threshold bin, in position order
-    int n_cand = 0;
-    for (int base = 0; base < len; base += kThreads) {
-        const int i = base + threadIdx.x;
-        const bool f = i < len && linear_bin(sv[i], g_lo, scale) == tb;
-        int tot;
-        const int pos = block_scan_flag(f, itmp, &tot);
-        if (f) cand[n_cand + pos] = (uint16_t)i;
-        n_cand += tot;
+    // threshold-bin candidates, in position order: thread i scans the
+    // contiguous segment [i*seg, (i+1)*seg) of the slice
+    const int seg = (len + kThreads - 1) / kThreads;
+    const int s0 = threadIdx.x * seg < len ? threadIdx.x * seg : len;
+    const int s1 = s0 + seg < len ? s0 + seg : len;
+    int n_cand;
+    {
+        int c = 0;
+        for (int i = s0; i < s1; i++) c += linear_bin(sv[pad(i)], g_lo, scale) == tb;
+        int pos = block_scan_int(c, itmp, &n_cand);
+        for (int i = s0; i < s1; i++)
+            if (linear_bin(sv[pad(i)], g_lo, scale) == tb) cand[pos++] = (uint16_t)i;
+    }
+    if (threadIdx.x == 0) ctl.n_cand = n_cand;
+    cl.sync();                                                            // (4)
+    int cand_off = 0, E = 0;
+    for (int r = 0; r < CN; r++) {
+        const int c = cl.map_shared_rank(&ctl, r)->n_cand;
+        if (r < p) cand_off += c;
+        E += c;
     }
 
-    // rounds 1-3: exact radix select among the candidates
-    uint32_t prefix = 0, mask = 0;
-    const int shifts[3] = {21, 10, 0};
-    const int widths[3] = {11, 11, 10};
-    for (int rd = 0; rd < 3; rd++) {
-        const int sh = shifts[rd];
-        const uint32_t dm = (1u << widths[rd]) - 1u;
-        for (int i = threadIdx.x; i < kBins; i += kThreads) hist[i] = 0;
-        __syncthreads();
-        for (int j = threadIdx.x; j < n_cand; j += kThreads) {
-            const uint32_t key = score_key(sv[cand[j]]);
-            if ((key & mask) == prefix) atomicAdd(&hist[(key >> sh) & dm], 1u);
-        }
-        cl.sync();
+    uint32_t tau;
+    int q;
+    if (E <= kGather) {
+        // few candidates: CTA 0 selects among all of them alone
+        uint32_t *g0 = cl.map_shared_rank(gath, 0);
+        for (int j = threadIdx.x; j < n_cand; j += kThreads) g0[cand_off + j] = score_key(sv[pad(cand[j])]);
+        cl.sync();                                                        // (5)
         if (p == 0) {
-            for (int b = threadIdx.x; b <= (int)dm; b += kThreads) {
-                unsigned v = hist[b];
-                for (int r = 1; r < CN; r++) v += cl.map_shared_rank(hist, r)[b];
-                hist[b] = v;
-            }
-            __syncthreads();
-            find_rank_bin(hist, (int)dm + 1, rank, &s_bin, &s_rank, scan_tmp);
+            unsigned rk;
+            cta_select_keys(gath, E, rank, hist, scan_tmp, &s_bin, &s_rank, &s_tau, &rk);
             if (threadIdx.x < CN) {
                 ClusterCtl *rc = cl.map_shared_rank(&ctl, (int)threadIdx.x);
-                rc->bin = s_bin;
-                rc->rank = s_rank;
+                rc->bin = s_tau;
+                rc->rank = rk;
             }
         }
-        cl.sync();
-        prefix |= ctl.bin << sh;
-        mask |= dm << sh;
-        rank = ctl.rank;
+        cl.sync();                                                        // (6)
+        tau = ctl.bin;
+        q = (int)ctl.rank;
+    } else {
+        // many candidates: radix rounds over each CTA's own candidates,
+        // histograms merged into CTA 0 with distributed atomics
+        uint32_t prefix = 0, mask = 0;
+        const int shifts[3] = {21, 10, 0};
+        const int widths[3] = {11, 11, 10};
+        for (int rd = 0; rd < 3; rd++) {
+            const int sh = shifts[rd];
+            const uint32_t dm = (1u << widths[rd]) - 1u;
+            for (int i = threadIdx.x; i < kBins; i += kThreads) {
+                hist[i] = 0;
+                hmerged[i] = 0;
+            }
+            cl.sync();
+            for (int j = threadIdx.x; j < n_cand; j += kThreads) {
+                const uint32_t key = score_key(sv[pad(cand[j])]);
+                if ((key & mask) == prefix) atomicAdd(&hist[(key >> sh) & dm], 1u);
+            }
+            __syncthreads();
+            {
+                unsigned *h0 = cl.map_shared_rank(hmerged, 0);
+                for (int b = threadIdx.x; b <= (int)dm; b += kThreads)
+                    if (hist[b]) atomicAdd(h0 + b, hist[b]);
+            }
+            cl.sync();
+            if (p == 0) {
+                find_rank_bin(hmerged, (int)dm + 1, rank, &s_bin, &s_rank, scan_tmp);
+                if (threadIdx.x < CN) {
+                    ClusterCtl *rc = cl.map_shared_rank(&ctl, (int)threadIdx.x);
+                    rc->bin = s_bin;
+                    rc->rank = s_rank;
+                }
+            }
+            cl.sync();
+            prefix |= ctl.bin << sh;
+            mask |= dm << sh;
+            rank = ctl.rank;
+        }
+        tau = prefix;
+        q = (int)rank;
     }
-    const uint32_t tau = prefix;
-    const int q = (int)rank;            // tau-equal positions still to take
 
     // counts, exchanged through the cluster, give each CTA its output offset
     int gt = 0, eq = 0;
-    for (int i = threadIdx.x; i < len; i += kThreads) {
-        const uint32_t key = score_key(sv[i]);
+    for (int i = s0; i < s1; i++) {
+        const uint32_t key = score_key(sv[pad(i)]);
         gt += key > tau;
         eq += key == tau;
     }
-    gt = block_sum(gt, itmp);
-    eq = block_sum(eq, itmp);
+    int cta_gt, cta_eq;
+    block_scan_int(gt, itmp, &cta_gt);
+    const int eq_before_me = block_scan_int(eq, itmp, &cta_eq);
     if (threadIdx.x == 0) {
-        ctl.n_gt = gt;
-        ctl.n_eq = eq;
+        ctl.n_gt = cta_gt;
+        ctl.n_eq = cta_eq;
     }
-    cl.sync();
+    cl.sync();                                                            // (7)
     int off = 0, eq_before = 0;
     for (int r = 0; r < p; r++) {
         const ClusterCtl *rc = cl.map_shared_rank(&ctl, r);
@@ -303,22 +413,20 @@ topk_cluster_kernel(const float *__restrict__ scores, int S, int64_t T, int64_t 
         off += rc->n_gt + quota;
         eq_before += rc->n_eq;
     }
-    cl.sync();                            // no CTA leaves while others read its counts
-    const int my_quota = q - eq_before;   // may exceed eq or be negative: compared below
-
-    int eq_seen = 0, out = 0;
-    for (int base = 0; base < len; base += kThreads) {
-        const int i = base + threadIdx.x;
-        const uint32_t key = i < len ? score_key(sv[i]) : 0u;
-        const bool is_eq = i < len && key == tau;
-        int eq_tot;
-        const int eq_rank = block_scan_flag(is_eq, itmp, &eq_tot);
-        const bool sel = i < len && (key > tau || (is_eq && eq_seen + eq_rank < my_quota));
-        int sel_tot;
-        const int pos = block_scan_flag(sel, itmp, &sel_tot);
-        if (sel && off + out + pos < m) dst[off + out + pos] = (int32_t)(t0 + i);
-        out += sel_tot;
-        eq_seen += eq_tot;
+    cl.sync();                            // (8) no CTA leaves while others read its counts
+    // tau-equal positions this thread takes: the first (q - earlier ones)
+    int my_q = q - eq_before - eq_before_me;
+    my_q = my_q < 0 ? 0 : (my_q > eq ? eq : my_q);
+    int tot;
+    int pos = off + block_scan_int(gt + my_q, itmp, &tot);
+    for (int i = s0; i < s1; i++) {
+        const uint32_t key = score_key(sv[pad(i)]);
+        bool take = key > tau;
+        if (key == tau && my_q > 0) {
+            take = true;
+            my_q--;
+        }
+        if (take && pos < m) dst[pos++] = (int32_t)(t0 + i);
     }
     for (int i = m + p * kThreads + threadIdx.x; i < K; i += CN * kThreads) dst[i] = -1;
 }
@@ -426,7 +534,8 @@ dsa_status launch_topk_select(const float *scores, int B, int S, int64_t T, int6
         topk_row_kernel<<<(unsigned)rows, kThreads, 0, stream>>>(scores, S, T, start_pos, K, idx);
         return launch_status();
     }
-    const size_t smem = (size_t)L * (sizeof(float) + sizeof(uint16_t));
+    const size_t smem = (size_t)(L + L / 32 + 1) * sizeof(float) + kGather * sizeof(uint32_t) +
+                        (size_t)L * sizeof(uint16_t);
     if (cudaFuncSetAttribute(topk_cluster_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)smem) != cudaSuccess)
         return DSA_ERR_CUDA;
