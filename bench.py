@@ -34,6 +34,42 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 N_COPIES = 3            # rotating device copies of the decode state (each > L2)
 
 
+# Source files of the dominant kernel (the indexer scorer); the committed ncu
+# summary records their hash, so its DRAM traffic is reported only while the
+# kernel is unchanged.
+SCORER_SOURCES = ("top_kv_selection_b200/csrc/index_scores.cu", "top_kv_selection_b200/csrc/quant.cuh",
+                  "top_kv_selection_b200/csrc/tc_ptx.cuh", "top_kv_selection_b200/csrc/common.cuh")
+SCORER_PROFILE = "profiles/index_scores_decode_B8_T131072.md"
+
+
+def scorer_source_hash() -> str:
+    import hashlib
+    h = hashlib.sha256()
+    for f in SCORER_SOURCES:
+        with open(os.path.join(ROOT, f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic():
+    """DRAM bytes per scorer launch from the committed ncu summary, or None if
+    the summary is missing or was taken on different kernel sources."""
+    path = os.path.join(ROOT, SCORER_PROFILE)
+    if not os.path.exists(path):
+        return None
+    fields = {}
+    for line in open(path):
+        if ":" in line and line.startswith("- "):
+            k, v = line[2:].split(":", 1)
+            fields[k.strip()] = v.strip().strip("`")
+    if fields.get("source_sha256") != scorer_source_hash():
+        return None
+    try:
+        return float(fields["dram_bytes_per_launch"])
+    except (KeyError, ValueError):
+        return None
+
+
 def _peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(path):
@@ -211,13 +247,11 @@ def time_stages(dsa, wl, copies, iters):
     """Average device time of each stage of the decode step, each launched
     through its own entry point on the same inputs, with CUDA events on the
     launching stream and the state copies rotating as in the timed steps.
-    Returns {stage: seconds per launch}; "index_scores" is the dominant kernel."""
+    Returns {stage: seconds per launch}; "decode_index_scores" is the dominant kernel."""
     dev = "cuda"
     B, T = wl.B, wl.T
-    q_fp8 = torch.empty(B, 1, wl.H, wl.D, dtype=torch.uint8, device=dev)
-    q_scale = torch.empty(B, 1, wl.H, dtype=torch.float32, device=dev)
-    w = copies[0]["w"].reshape(B, 1, wl.H).contiguous()
     scores = torch.empty(B, 1, T, dtype=torch.float32, device=dev)
+    scores2d = scores.view(B, T)
     idx = torch.empty(B, 1, wl.K, dtype=torch.int32, device=dev)
     dt = dsa.DSA_BF16 if wl.attn_dtype == "bf16" else dsa.DSA_F32
     ws = torch.empty(max(1, dsa.dsa_sparse_mla_attn_workspace_size(B, 1, wl.Hq, wl.dc, wl.dr,
@@ -227,15 +261,10 @@ def time_stages(dsa, wl, copies, iters):
     out = torch.empty(B, 1, wl.Hq, wl.dc, dtype=copies[0]["out"].dtype, device=dev)
     lse = torch.empty(B, 1, wl.Hq, dtype=torch.float32, device=dev)
 
-    def quant(st):
-        dsa.dsa_indexer_quant(st["q_idx"], q_fp8, q_scale)
-        dsa.dsa_indexer_quant(st["k_new"], st["k_cache"][:, T - 1:], st["k_scale"][:, T - 1:],
-                              n_rows=B, out_row_stride=st["k_cache"].shape[1] * wl.D,
-                              scale_row_stride=st["k_cache"].shape[1])
-
     def score(st):
-        dsa.dsa_index_scores(q_fp8, q_scale, w, st["k_cache"], st["k_scale"], T - 1, T,
-                             wl.softmax_scale_idx, scores)
+        # the indexer half of the step, the same kernel the decode step launches
+        dsa.dsa_decode_index_scores(st["q_idx"], st["w"], st["k_new"], st["k_cache"],
+                                    st["k_scale"], T, wl.softmax_scale_idx, scores2d)
 
     def topk(st):
         dsa.dsa_topk_select(scores, T - 1, wl.topk, idx)
@@ -245,7 +274,7 @@ def time_stages(dsa, wl, copies, iters):
 
     stream = torch.cuda.current_stream()
     result = {}
-    for name, fn in (("indexer_quant", quant), ("index_scores", score), ("topk_select", topk),
+    for name, fn in (("decode_index_scores", score), ("topk_select", topk),
                      ("sparse_mla_attn", attn)):
         for i in range(3):
             fn(copies[i % len(copies)])
@@ -361,8 +390,10 @@ def run_ours(args, wl, world, rank, local):
     # dominant kernel roofline (indexer scorer over the full cache)
     peak, peak_kind = _peaks()
     stages = time_stages(dsa, wl, copies, iters=max(10, min(args.steps, 500)))
-    t_score = stages["index_scores"]
-    score_bytes = wl.B * wl.T * (wl.D + 4) + wl.B * wl.H * (wl.D + 4 + 4)
+    t_score = stages["decode_index_scores"]
+    # keys + scales of every cached token, plus the new tokens' fp32 queries,
+    # weights and keys (the scores written are not algorithmic)
+    score_bytes = wl.B * wl.T * (wl.D + 4) + wl.B * (wl.H * wl.D * 4 + wl.H * 4 + wl.D * 4)
     achieved = score_bytes / t_score / 1e9
     step_bytes = wl.B * (wl.T * (wl.D + 4) + wl.K * wl.dqk * 2 + wl.H * wl.D * 4
                          + wl.Hq * wl.dqk * 2 + wl.Hq * wl.dc * 2)
@@ -379,9 +410,9 @@ def run_ours(args, wl, world, rank, local):
         "indexer_gscores_per_s": gscores,
         "step_roofline": {"bytes": step_bytes, "achieved_gbs": step_bytes / (ms_per_step * 1e-3)
                           / 1e9, "frac": step_bytes / (ms_per_step * 1e-3) / 1e9 / peak},
-        "roofline": {"kernel": "index_scores", "bound": "hbm", "achieved": achieved,
+        "roofline": {"kernel": "decode_index_scores", "bound": "hbm", "achieved": achieved,
                      "peak": peak, "peak_kind": f"{peak_kind} hbm_gbs", "unit": "GB/s",
-                     "frac": achieved / peak, "traffic": None,
+                     "frac": achieved / peak, "traffic": profiled_traffic(),
                      "avg_launch_us": t_score * 1e6},
         "e2e": e2e,
         "gpu_launches": per_step_launches * args.steps,

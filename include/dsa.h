@@ -118,6 +118,19 @@ dsa_status dsa_index_scores(const uint8_t *q_fp8, const float *q_scale, const fl
                             float softmax_scale, float *scores, dsa_stream_t stream);
 
 /*
+ * The indexer half of a decode step (Indexer.forward with seqlen == 1): rotate
+ * and quantise the new token's queries q_idx [B,H,D] fp32 and key k_new [B,D]
+ * fp32 exactly as dsa_indexer_quant does, append the key's codes and scale to
+ * k_cache / k_scale at position T-1, and write scores [B,T] fp32 for positions
+ * 0..T-1 as dsa_index_scores does (start_pos = T-1, no mask).  One kernel.
+ * Same constraints as dsa_index_scores; t_max * D must be a multiple of 16.
+ */
+dsa_status dsa_decode_index_scores(const float *q_idx, const float *w, const float *k_new,
+                                   uint8_t *k_cache, float *k_scale, int64_t t_max, int B, int H,
+                                   int D, int64_t T, float softmax_scale, float *scores,
+                                   dsa_stream_t stream);
+
+/*
  * topk(min(index_topk, end_pos)) (Indexer.forward), restricted to the causal
  * positions t <= start_pos + s of each row:
  *   idx[b,s,:] holds the m = min(K, start_pos+s+1, T) positions with the

@@ -64,3 +64,30 @@ def test_scores_prefill_full_size_sampled_rows(dsa):
         ref = oracle.index_scores(qf[:, s:s + 1], qs[:, s:s + 1], w[:, s:s + 1], kf, ks, s, T,
                                   wl.softmax_scale_idx)
         assert_scores_close(got[:, s:s + 1], ref)
+
+
+@pytest.mark.parametrize("cfg,B,T,t_max", [(1, 3, 5000, 5003), (1, 1, 1, 8), (0, 2, 300, 300)])
+def test_decode_index_scores_matches_oracle(dsa, cfg, B, T, t_max):
+    """The indexer half of a decode step: quantise the new queries and key, append
+    the key at T-1, score every cached position."""
+    wl = workloads.WORKLOADS[cfg]
+    D, H = wl.D, wl.H
+    seqs = [workloads.decode_sequence(wl, b, T=T) for b in range(B)]
+    k_cache = torch.zeros(B, t_max, D, dtype=torch.uint8, device="cuda")
+    k_scale = torch.zeros(B, t_max, dtype=torch.float32, device="cuda")
+    for b, s in enumerate(seqs):
+        if T > 1:
+            dsa.dsa_indexer_quant(s["keys"][:T - 1].cuda(), k_cache[b], k_scale[b])
+    q = torch.stack([s["q_idx"] for s in seqs]).cuda()
+    w = torch.stack([s["w"] for s in seqs]).cuda()
+    k_new = torch.stack([s["keys"][T - 1] for s in seqs]).cuda()
+    scores = torch.empty(B, T, dtype=torch.float32, device="cuda")
+    dsa.dsa_decode_index_scores(q, w, k_new, k_cache, k_scale, T, wl.softmax_scale_idx, scores)
+    for b, s in enumerate(seqs):
+        kf, ks = oracle.indexer_quant(s["keys"].numpy())
+        qf, qs = oracle.indexer_quant(s["q_idx"].numpy())
+        assert np.array_equal(k_cache[b, T - 1].cpu().numpy(), kf[T - 1])
+        assert k_scale[b, T - 1].item() == ks[T - 1]
+        ref = oracle.index_scores(qf[None, None], qs[None, None], s["w"].numpy()[None, None],
+                                  kf[None], ks[None], T - 1, T, wl.softmax_scale_idx)
+        assert_scores_close(scores[b:b + 1].cpu().numpy()[:, None], ref)

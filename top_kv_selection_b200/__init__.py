@@ -38,6 +38,8 @@ _SIGNATURES = {
     "dsa_indexer_quant": ([_P, _i32, _i64, _i64, _i32, _P, _i64, _P, _i64, _P], _i32),
     "dsa_index_scores": ([_P, _P, _P, _P, _P, _i64, _i32, _i32, _i32, _i32, _i64, _i64, _f32,
                           _P, _P], _i32),
+    "dsa_decode_index_scores": ([_P, _P, _P, _P, _P, _i64, _i32, _i32, _i32, _i64, _f32, _P, _P],
+                                _i32),
     "dsa_topk_select_workspace_size": ([_i32, _i32, _i64, _i32], _sz),
     "dsa_topk_select": ([_P, _i32, _i32, _i64, _i64, _i32, _P, _P, _sz, _P], _i32),
     "dsa_sparse_mla_attn_workspace_size": ([_i32, _i32, _i32, _i32, _i32, _i32, _i32], _sz),
@@ -134,6 +136,18 @@ def dsa_index_scores(q_fp8: torch.Tensor, q_scale: torch.Tensor, w: torch.Tensor
     _check("dsa_index_scores", _lib.dsa_index_scores(
         _ptr(q_fp8), _ptr(q_scale), _ptr(w), _ptr(k_cache), _ptr(k_scale), t_max, B, S, H, D,
         start_pos, T, softmax_scale, _ptr(scores), _stream(stream)))
+
+
+def dsa_decode_index_scores(q_idx: torch.Tensor, w: torch.Tensor, k_new: torch.Tensor,
+                            k_cache: torch.Tensor, k_scale: torch.Tensor, T: int,
+                            softmax_scale: float, scores: torch.Tensor, stream=None) -> None:
+    """Indexer half of a decode step: q_idx [B,H,D], w [B,H], k_new [B,D] fp32; appends the
+    key at T-1 of k_cache [B,t_max,D] / k_scale [B,t_max]; scores [B,T] fp32."""
+    B, H, D = q_idx.shape
+    t_max = k_cache.shape[1]
+    _check("dsa_decode_index_scores", _lib.dsa_decode_index_scores(
+        _ptr(q_idx), _ptr(w), _ptr(k_new), _ptr(k_cache), _ptr(k_scale), t_max, B, H, D, T,
+        softmax_scale, _ptr(scores), _stream(stream)))
 
 
 def dsa_topk_select_workspace_size(B: int, S: int, T: int, k: int) -> int:

@@ -252,11 +252,20 @@ score_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const ScoreArgs a) {
         const uint32_t lane_addr = (uint32_t)(quarter * 32) << 16;
         const float *ks_row = a.k_scale + b * a.t_max;
         float *out = a.scores + row * a.T;
+        // key scales are loaded three tiles ahead so their HBM latency is hidden
+        auto load_ks = [&](int ii) -> float {
+            const int64_t tt = (tile_lo + ii) * kTile + tok;
+            if (ii >= n_my || tt >= n_vis) return 0.f;
+            return (append && tt == a.T - 1) ? *knew_scale : __ldg(ks_row + tt);
+        };
+        float ks0 = load_ks(0), ks1 = load_ks(1), ks2 = load_ks(2);
         for (int i = 0; i < n_my; i++) {
             const int ac = i % kAcc;
             const int64_t t = (tile_lo + i) * kTile + tok;
-            const float ks = t >= n_vis ? 0.f : (append && t == a.T - 1) ? *knew_scale
-                                                                          : __ldg(ks_row + t);
+            const float ks = ks0;
+            ks0 = ks1;
+            ks1 = ks2;
+            ks2 = load_ks(i + 3);
             if (!tc::mbar_wait(&accf[ac], (uint32_t)(i / kAcc) & 1u, a.err, abort)) break;
             tc::tc_fence_after();
             const uint32_t taddr = tmem_base + lane_addr + (uint32_t)(ac * a.NH);
@@ -397,4 +406,21 @@ extern "C" dsa_status dsa_index_scores(const uint8_t *q_fp8, const float *q_scal
     return dsa::launch_index_scores(q_fp8, q_scale, w, k_cache, k_scale, t_max, B, S, H, D,
                                     start_pos, T, softmax_scale, scores,
                                     reinterpret_cast<cudaStream_t>(stream));
+}
+
+extern "C" dsa_status dsa_decode_index_scores(const float *q_idx, const float *w,
+                                              const float *k_new, uint8_t *k_cache,
+                                              float *k_scale, int64_t t_max, int B, int H, int D,
+                                              int64_t T, float softmax_scale, float *scores,
+                                              dsa_stream_t stream) {
+    if (B < 0 || T < 1 || H < 1 || T > t_max) return DSA_ERR_INVALID_ARG;
+    if (D != 64 && D != 128) return DSA_ERR_UNSUPPORTED;
+    if (H > 256 || t_max > INT32_MAX || B > 65535) return DSA_ERR_UNSUPPORTED;
+    if (B == 0) return DSA_OK;
+    if (!q_idx || !w || !k_new || !k_cache || !k_scale || !scores) return DSA_ERR_INVALID_ARG;
+    if (!dsa::aligned16(q_idx) || !dsa::aligned16(k_new) || !dsa::aligned16(k_cache) ||
+        ((t_max * D) & 15))
+        return DSA_ERR_INVALID_ARG;
+    return dsa::launch_decode_scores(q_idx, w, k_new, k_cache, k_scale, t_max, B, H, D, T,
+                                     softmax_scale, scores, reinterpret_cast<cudaStream_t>(stream));
 }

@@ -425,19 +425,34 @@ sparse_mla_combine_kernel(const float *__restrict__ part_o, const float2 *__rest
     const int h = (int)(blockIdx.x % groups) * kCombineHeads + (threadIdx.x >> 5);
     const int lane = threadIdx.x & 31;
     const int64_t u0 = rh * splits;
+    // all (max, sum) pairs first, then the partial rows four splits at a time,
+    // so that the loads of a batch are in flight together
     float m = -INFINITY;
     for (int sp = 0; sp < splits; sp++) m = fmaxf(m, part_ml[(u0 + sp) * kHq + h].x);
     float L = 0.f;
     float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-    for (int sp = 0; sp < splits; sp++) {
-        const float2 ml = part_ml[(u0 + sp) * kHq + h];
-        if (ml.x == -INFINITY) continue;
-        const float w = exp2f(ml.x - m);
-        L += w * ml.y;
-        const float4 *po = reinterpret_cast<const float4 *>(part_o + ((u0 + sp) * kHq + h) * kDh) + 2 * lane;
-        const float4 x = po[0], y = po[1];
-        acc[0] += w * x.x; acc[1] += w * x.y; acc[2] += w * x.z; acc[3] += w * x.w;
-        acc[4] += w * y.x; acc[5] += w * y.y; acc[6] += w * y.z; acc[7] += w * y.w;
+    for (int sp0 = 0; sp0 < splits; sp0 += 4) {
+        float2 ml[4];
+        float4 x[4], y[4];
+#pragma unroll
+        for (int u = 0; u < 4; u++) {
+            const int sp = sp0 + u;
+            ml[u] = sp < splits ? part_ml[(u0 + sp) * kHq + h] : make_float2(-INFINITY, 0.f);
+            if (sp < splits) {
+                const float4 *po =
+                    reinterpret_cast<const float4 *>(part_o + ((u0 + sp) * kHq + h) * kDh) + 2 * lane;
+                x[u] = po[0];
+                y[u] = po[1];
+            }
+        }
+#pragma unroll
+        for (int u = 0; u < 4; u++) {
+            if (ml[u].x == -INFINITY) continue;
+            const float w = exp2f(ml[u].x - m);
+            L += w * ml[u].y;
+            acc[0] += w * x[u].x; acc[1] += w * x[u].y; acc[2] += w * x[u].z; acc[3] += w * x[u].w;
+            acc[4] += w * y[u].x; acc[5] += w * y[u].y; acc[6] += w * y[u].z; acc[7] += w * y[u].w;
+        }
     }
     const float inv = L > 0.f ? 1.f / L : 0.f;
     uint32_t wv[4];

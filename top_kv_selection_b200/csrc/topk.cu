@@ -240,13 +240,51 @@ topk_cluster_kernel(const float *__restrict__ scores, int S, int64_t T, int64_t 
     const float *src = scores + row * T + t0;
 
     // load the slice, finite min / max; clear the histograms
+    // (loads are issued in batches of eight per thread so their latencies overlap)
     float lo = INFINITY, hi = -INFINITY;
-    for (int i = threadIdx.x; i < len; i += kThreads) {
-        const float x = src[i];
-        sv[pad(i)] = x;
-        if (isfinite(x)) {
-            lo = fminf(lo, x);
-            hi = fmaxf(hi, x);
+    const bool vec = ((reinterpret_cast<uintptr_t>(src) & 15) == 0);
+    if (vec) {
+        const int n4 = len >> 2;
+        for (int base = 0; base < n4; base += 8 * kThreads) {
+            float4 v[8];
+#pragma unroll
+            for (int u = 0; u < 8; u++) {
+                const int j = base + u * kThreads + threadIdx.x;
+                v[u] = j < n4 ? __ldg(reinterpret_cast<const float4 *>(src) + j)
+                              : make_float4(NAN, NAN, NAN, NAN);
+            }
+#pragma unroll
+            for (int u = 0; u < 8; u++) {
+                const int j = base + u * kThreads + threadIdx.x;
+                if (j >= n4) continue;
+                const float xs[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
+#pragma unroll
+                for (int e = 0; e < 4; e++) {
+                    sv[pad(4 * j + e)] = xs[e];
+                    if (isfinite(xs[e])) {
+                        lo = fminf(lo, xs[e]);
+                        hi = fmaxf(hi, xs[e]);
+                    }
+                }
+            }
+        }
+    }
+    for (int base = vec ? (len & ~3) : 0; base < len; base += 8 * kThreads) {
+        float v[8];
+#pragma unroll
+        for (int u = 0; u < 8; u++) {
+            const int i = base + u * kThreads + threadIdx.x;
+            v[u] = i < len ? __ldg(src + i) : NAN;
+        }
+#pragma unroll
+        for (int u = 0; u < 8; u++) {
+            const int i = base + u * kThreads + threadIdx.x;
+            if (i >= len) continue;
+            sv[pad(i)] = v[u];
+            if (isfinite(v[u])) {
+                lo = fminf(lo, v[u]);
+                hi = fmaxf(hi, v[u]);
+            }
         }
     }
     for (int i = threadIdx.x; i < kBins; i += kThreads) {
