@@ -1,4 +1,6 @@
 """fp8_index scoring on the GPU vs the oracle (1e-3 relative, exact mask)."""
+import dataclasses
+
 import numpy as np
 import pytest
 import torch
@@ -66,11 +68,20 @@ def test_scores_prefill_full_size_sampled_rows(dsa):
         assert_scores_close(got[:, s:s + 1], ref)
 
 
-@pytest.mark.parametrize("cfg,B,T,t_max", [(1, 3, 5000, 5003), (1, 1, 1, 8), (0, 2, 300, 300)])
-def test_decode_index_scores_matches_oracle(dsa, cfg, B, T, t_max):
+@pytest.mark.parametrize("cfg,B,T,t_max,H", [
+    (1, 3, 5000, 5003, None),
+    (1, 1, 1, 8, None),
+    (0, 2, 300, 300, None),        # D = 64, 4 heads: one lane per head, padded heads
+    (1, 2, 4193, 4200, 128),       # two passes over the heads; T-1 in the last quarter
+    (1, 1, 2081, 2081, 256),       # four passes; T-1 in the second quarter
+    (1, 2, 129, 129, 64),          # T-1 opens a tile of its own
+])
+def test_decode_index_scores_matches_oracle(dsa, cfg, B, T, t_max, H):
     """The indexer half of a decode step: quantise the new queries and key, append
     the key at T-1, score every cached position."""
     wl = workloads.WORKLOADS[cfg]
+    if H is not None:
+        wl = dataclasses.replace(wl, H=H)
     D, H = wl.D, wl.H
     seqs = [workloads.decode_sequence(wl, b, T=T) for b in range(B)]
     k_cache = torch.zeros(B, t_max, D, dtype=torch.uint8, device="cuda")

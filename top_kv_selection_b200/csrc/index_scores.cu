@@ -21,10 +21,12 @@
 // The producer starts streaming at once; the query operand is built in
 // parallel by the epilogue warps, either from given FP8 codes or -- in the
 // decode step -- by rotating and quantising the new token's fp32 queries
-// (rotate_activation + act_quant, bit-identical to dsa_indexer_quant).  In the
-// decode step the CTA holding position T-1 also quantises the new key and
-// appends it to the cache (the cache write of Indexer.forward) before its last
-// tile is fetched.
+// (rotate_activation + act_quant, bit-identical to dsa_indexer_quant).  Their
+// global loads are issued at kernel entry, before the key stream fills the
+// memory queues, and the rotation keeps 64 elements per lane so that it is
+// almost all register arithmetic.  In the decode step the CTA holding position
+// T-1 also quantises the new key and appends it to the cache (the cache write
+// of Indexer.forward) before its last tile is fetched.
 #include "common.cuh"
 #include "quant.cuh"
 #include "tc_ptx.cuh"
@@ -77,70 +79,94 @@ __host__ __device__ constexpr size_t score_smem_bytes(int NH) {
 }
 
 // Query operand (K-major, swizzled, padded heads zero) and folded weights
-// w' = ((w * H^-1/2) * q_scale) * softmax_scale; run by the four epilogue
-// warps.  In decode mode the first of them first appends the new key.
-template <int D>
-__device__ __forceinline__ void build_query(const ScoreArgs &a, int64_t row, int64_t b,
-                                            uint8_t *sq, float *wf, bool append,
-                                            float *knew_scale, uint64_t *k_ready) {
-    constexpr int E = D / 32;
-    constexpr int kChunks = D / 16;
-    const int t = threadIdx.x - 64;           // 0..127 over the epilogue warps
-    const int wi = t >> 5, lane = t & 31;
-    if (a.q_raw) {
-        if (append && wi == 0) {
-            float r[E];
-            load_lane_slice<D, float>(a.k_new + b * D, r);
-            float ks;
-            const uint32_t packed = rotate_quant_warp<D>(r, &ks);
-            uint8_t *dst = a.k_cache_w + (b * a.t_max + a.T - 1) * D + lane * E;
-            if constexpr (E == 4) *reinterpret_cast<uint32_t *>(dst) = packed;
-            else *reinterpret_cast<uint16_t *>(dst) = static_cast<uint16_t>(packed);
-            if (lane == 0) {
-                a.k_scale_w[b * a.t_max + a.T - 1] = ks;
-                *knew_scale = ks;
+// w' = ((w * H^-1/2) * q_scale) * softmax_scale, built by the four epilogue
+// warps.  G = D / 64 adjacent lanes own one head, 64 bytes of its row each, so
+// one pass over the warps covers 4 * 32 / G heads.  The first pass's global
+// loads are issued at kernel entry (QueryPrefetch), ahead of the key stream
+// that would otherwise queue in front of them.
+template <int D, bool kRaw> struct QueryPrefetch {
+    static constexpr int G = D / 64;            // lanes per head
+    static constexpr int kPass = 4 * 32 / G;    // heads per pass
+    float r[kRaw ? 64 : 1];                     // fp32 query slice (decode)
+    uint4 c[4];                                 // FP8 code slice (64 bytes)
+    float w, qs;
+
+    __device__ __forceinline__ static int head(int pass) {
+        const int t = threadIdx.x - 64;
+        return pass * kPass + (t >> 5) * (32 / G) + (t & 31) / G;
+    }
+    __device__ __forceinline__ void load(const ScoreArgs &a, int64_t row, int pass) {
+        const int h = head(pass), part = (threadIdx.x - 64) % G;
+        const bool ok = h < a.H;
+        w = ok && part == 0 ? a.w[row * a.H + h] : 0.f;
+        if constexpr (kRaw) {
+            qs = 0.f;
+            const float4 *src =
+                reinterpret_cast<const float4 *>(a.q_raw + (row * a.H + h) * D + part * 64);
+#pragma unroll
+            for (int j = 0; j < 16; j++) {
+                const float4 v = ok ? src[j] : make_float4(0.f, 0.f, 0.f, 0.f);
+                r[4 * j] = v.x; r[4 * j + 1] = v.y; r[4 * j + 2] = v.z; r[4 * j + 3] = v.w;
             }
-            // the key row is read next by TMA (async proxy)
-            asm volatile("fence.proxy.async.global;" ::: "memory");
-            __syncwarp();
-            if (lane == 0) tc::mbar_arrive(k_ready);
+        } else {
+            qs = ok && part == 0 ? a.q_scale[row * a.H + h] : 0.f;
+            const uint4 *src =
+                reinterpret_cast<const uint4 *>(a.q_fp8 + (row * a.H + h) * D + part * 64);
+#pragma unroll
+            for (int j = 0; j < 4; j++) c[j] = ok ? src[j] : make_uint4(0, 0, 0, 0);
         }
-        for (int h = wi; h < a.H; h += 4) {
-            float r[E];
-            load_lane_slice<D, float>(a.q_raw + (row * a.H + h) * D, r);
-            float qs;
-            const uint32_t packed = rotate_quant_warp<D>(r, &qs);
-            const int byte = lane * E;
-            uint8_t *dst = sq + h * D + KSwizzle<D>::chunk(h, byte >> 4) * 16 + (byte & 15);
-            if constexpr (E == 4) *reinterpret_cast<uint32_t *>(dst) = packed;
-            else *reinterpret_cast<uint16_t *>(dst) = static_cast<uint16_t>(packed);
-            if (lane == 0) {
-                float x = __fmul_rn(a.w[row * a.H + h], a.head_scale);
-                x = __fmul_rn(x, qs);
-                wf[h] = __fmul_rn(x, a.softmax_scale);
-            }
+    }
+    // Rotates / quantises (decode) or copies (codes) the loaded slice into the
+    // operand and writes the head's folded weight.
+    __device__ __forceinline__ void store(const ScoreArgs &a, int pass, uint8_t *sq, float *wf) {
+        const int h = head(pass), part = (threadIdx.x - 64) % G;
+        float scale = qs;
+        if constexpr (kRaw) {
+            uint32_t codes[16];
+            rotate_quant_lanes<D>(r, codes, &scale);
+#pragma unroll
+            for (int j = 0; j < 4; j++)
+                c[j] = make_uint4(codes[4 * j], codes[4 * j + 1], codes[4 * j + 2],
+                                  codes[4 * j + 3]);
         }
-    } else {
-        const uint8_t *qrow = a.q_fp8 + row * a.H * D;
-        for (int i = t; i < a.H * kChunks; i += 128) {
-            const int h = i / kChunks, c = i - h * kChunks;
-            *reinterpret_cast<uint4 *>(sq + h * D + KSwizzle<D>::chunk(h, c) * 16) =
-                *reinterpret_cast<const uint4 *>(qrow + h * D + c * 16);
+        if (h < a.NH) {
+#pragma unroll
+            for (int j = 0; j < 4; j++)
+                *reinterpret_cast<uint4 *>(sq + h * D + KSwizzle<D>::chunk(h, part * 4 + j) * 16) =
+                    c[j];
         }
-        for (int h = t; h < a.H; h += 128) {
-            float x = __fmul_rn(a.w[row * a.H + h], a.head_scale);
-            x = __fmul_rn(x, a.q_scale[row * a.H + h]);
+        if (h < a.H && part == 0) {
+            float x = __fmul_rn(w, a.head_scale);
+            x = __fmul_rn(x, scale);
             wf[h] = __fmul_rn(x, a.softmax_scale);
         }
     }
-    for (int i = t; i < (a.NH - a.H) * kChunks; i += 128)
-        *reinterpret_cast<uint4 *>(sq + (a.H + i / kChunks) * D + (i % kChunks) * 16) =
-            make_uint4(0, 0, 0, 0);
-    for (int h = a.H + t; h < kMaxHeads; h += 128) wf[h] = 0.f;
+};
+
+// Decode: quantise the new key and append it at position T-1 of the cache
+// (one warp, the lane layout of rotate_quant_warp); its TMA read follows.
+template <int D>
+__device__ __forceinline__ void append_key(const ScoreArgs &a, int64_t b, float (&kr)[D / 32],
+                                           float *knew_scale, uint64_t *k_ready) {
+    constexpr int E = D / 32;
+    const int lane = threadIdx.x & 31;
+    float ks;
+    const uint32_t packed = rotate_quant_warp<D>(kr, &ks);
+    uint8_t *dst = a.k_cache_w + (b * a.t_max + a.T - 1) * D + lane * E;
+    if constexpr (E == 4) *reinterpret_cast<uint32_t *>(dst) = packed;
+    else *reinterpret_cast<uint16_t *>(dst) = static_cast<uint16_t>(packed);
+    if (lane == 0) {
+        a.k_scale_w[b * a.t_max + a.T - 1] = ks;
+        *knew_scale = ks;
+    }
+    // the key row is read next by TMA (async proxy)
+    asm volatile("fence.proxy.async.global;" ::: "memory");
+    __syncwarp();
+    if (lane == 0) tc::mbar_arrive(k_ready);
 }
 
-template <int D>
-__global__ void __launch_bounds__(kThreads)
+template <int D, bool kRaw>
+__global__ void __launch_bounds__(kThreads, 2)
 score_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const ScoreArgs a) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>(
@@ -168,13 +194,38 @@ score_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const ScoreArgs a) {
     const int64_t tile_hi = (chunk + 1) * n_tiles / a.chunks;
     const int n_my = (int)(tile_hi - tile_lo);
     // decode: this CTA appends the new key if its last tile holds position T-1
-    const bool append = a.k_new != nullptr && n_my > 0 && tile_hi == n_tiles;
+    const bool append = kRaw && n_my > 0 && tile_hi == n_tiles;
 
     // causally masked positions of this row (prefill only), shared by the chunks
     for (int64_t t = n_vis + (int64_t)chunk * kThreads + threadIdx.x; t < a.T;
          t += (int64_t)a.chunks * kThreads)
         a.scores[row * a.T + t] = -INFINITY;
     if (n_my <= 0) return;
+
+    // epilogue warps: issue the query, weight, first key-scale and new-key
+    // loads before the key stream starts
+    using Prefetch = QueryPrefetch<D, kRaw>;
+    Prefetch pf;
+    float kr[D / 32];
+    const int tok = (warp & 3) * 32 + lane;       // token within a tile (epilogue)
+    const float *ks_row = a.k_scale + b * a.t_max;
+    // key scales are loaded three tiles ahead so their HBM latency is hidden
+    auto load_ks = [&](int ii) -> float {
+        const int64_t tt = (tile_lo + ii) * kTile + tok;
+        if (ii >= n_my || tt >= n_vis) return 0.f;
+        return (append && tt == a.T - 1) ? *knew_scale : __ldg(ks_row + tt);
+    };
+    // the epilogue warp whose tokens include position T-1 appends the new key,
+    // so the key's scale passes between lanes of one warp
+    const bool appender = append && warp >= 2 && (warp & 3) == (int)(((a.T - 1) % kTile) >> 5);
+    float ks0 = 0.f, ks1 = 0.f, ks2 = 0.f;
+    if (warp >= 2) {
+        pf.load(a, row, 0);
+        if (appender) load_lane_slice<D, float>(a.k_new + b * D, kr);
+        ks0 = load_ks(0);     // the new key's entry is reloaded once it is appended
+        ks1 = load_ks(1);
+        ks2 = load_ks(2);
+    }
 
     if (threadIdx.x == 0) {
         for (int i = 0; i < kStages; i++) {
@@ -243,22 +294,23 @@ score_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const ScoreArgs a) {
             }
         }
     } else {
-        build_query<D>(a, row, b, sq, wf, append, knew_scale, k_ready);
+        for (int pass = 0; pass * Prefetch::kPass < a.NH; pass++) {
+            if (pass > 0) pf.load(a, row, pass);
+            pf.store(a, pass, sq, wf);
+        }
+        for (int h = a.H + (threadIdx.x - 64); h < kMaxHeads; h += 128) wf[h] = 0.f;
         tc::fence_proxy_async_smem();
         asm volatile("bar.sync 1, 128;" ::: "memory");   // folded weights of all heads
         tc::mbar_arrive(q_ready);
-        const int quarter = warp & 3;                 // TMEM lanes this warp may read
-        const int tok = quarter * 32 + lane;          // token within the tile
-        const uint32_t lane_addr = (uint32_t)(quarter * 32) << 16;
-        const float *ks_row = a.k_scale + b * a.t_max;
+        if (appender) {
+            append_key<D>(a, b, kr, knew_scale, k_ready);
+            __syncwarp();
+            ks0 = load_ks(0);
+            ks1 = load_ks(1);
+            ks2 = load_ks(2);
+        }
+        const uint32_t lane_addr = (uint32_t)((warp & 3) * 32) << 16;
         float *out = a.scores + row * a.T;
-        // key scales are loaded three tiles ahead so their HBM latency is hidden
-        auto load_ks = [&](int ii) -> float {
-            const int64_t tt = (tile_lo + ii) * kTile + tok;
-            if (ii >= n_my || tt >= n_vis) return 0.f;
-            return (append && tt == a.T - 1) ? *knew_scale : __ldg(ks_row + tt);
-        };
-        float ks0 = load_ks(0), ks1 = load_ks(1), ks2 = load_ks(2);
         for (int i = 0; i < n_my; i++) {
             const int ac = i % kAcc;
             const int64_t t = (tile_lo + i) * kTile + tok;
@@ -312,7 +364,7 @@ uint32_t pow2_cols(int n) {
     return c;
 }
 
-template <int D>
+template <int D, bool kRaw>
 dsa_status launch_tc(ScoreArgs a, const uint8_t *k_cache, int B, int S, int64_t start_pos,
                      int64_t T, cudaStream_t stream) {
     CUtensorMap tmap;
@@ -340,10 +392,10 @@ dsa_status launch_tc(ScoreArgs a, const uint8_t *k_cache, int B, int S, int64_t 
     if (chunks > max_tiles) chunks = max_tiles;
     if (chunks < 1) chunks = 1;
     a.chunks = (int)chunks;
-    if (cudaFuncSetAttribute(score_tc_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)smem) != cudaSuccess)
+    if (cudaFuncSetAttribute(score_tc_kernel<D, kRaw>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
         return DSA_ERR_CUDA;
-    score_tc_kernel<D><<<(unsigned)(rows * chunks), kThreads, smem, stream>>>(tmap, a);
+    score_tc_kernel<D, kRaw><<<(unsigned)(rows * chunks), kThreads, smem, stream>>>(tmap, a);
     return launch_status();
 }
 
@@ -363,8 +415,8 @@ dsa_status launch_index_scores(const uint8_t *q_fp8, const float *q_scale, const
     a.t_max = t_max;
     a.H = H;
     a.softmax_scale = softmax_scale;
-    return D == 128 ? launch_tc<128>(a, k_cache, B, S, start_pos, T, stream)
-                    : launch_tc<64>(a, k_cache, B, S, start_pos, T, stream);
+    return D == 128 ? launch_tc<128, false>(a, k_cache, B, S, start_pos, T, stream)
+                    : launch_tc<64, false>(a, k_cache, B, S, start_pos, T, stream);
 }
 
 dsa_status launch_decode_scores(const float *q_raw, const float *w, const float *k_new,
@@ -383,8 +435,8 @@ dsa_status launch_decode_scores(const float *q_raw, const float *w, const float 
     a.t_max = t_max;
     a.H = H;
     a.softmax_scale = softmax_scale;
-    return D == 128 ? launch_tc<128>(a, k_cache, B, 1, T - 1, T, stream)
-                    : launch_tc<64>(a, k_cache, B, 1, T - 1, T, stream);
+    return D == 128 ? launch_tc<128, true>(a, k_cache, B, 1, T - 1, T, stream)
+                    : launch_tc<64, true>(a, k_cache, B, 1, T - 1, T, stream);
 }
 
 }  // namespace dsa

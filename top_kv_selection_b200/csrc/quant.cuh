@@ -1,4 +1,5 @@
-// quant.cuh -- rotate_activation + act_quant of one D-vector by one warp.
+// quant.cuh -- rotate_activation + act_quant of one D-vector by one warp
+// (rotate_quant_warp) or by D / 64 lanes (rotate_quant_lanes).
 //
 // Page: "DeepSeek-V3.2-Exp - Split indexer heads", Indexer.forward
 // (rotate_activation, then act_quant with one scale per vector).
@@ -70,6 +71,50 @@ __device__ __forceinline__ uint32_t rotate_quant_warp(float (&r)[D / 32], float 
         packed |= e4m3x2_rn_sat(__fdiv_rn(r[e], s), __fdiv_rn(r[e + 1], s)) << (8 * e);
     *scale = s;
     return packed;
+}
+
+// The same rotation and quantisation with the vector split over G = D / 64
+// adjacent lanes, 64 contiguous elements each (lane part p holds elements
+// [64p, 64p + 64)).  Stages h = 1 .. 32 stay in registers; for D = 128 the last
+// stage h = 64 pairs part 0 (lower: a + b) with part 1 (upper: a - b) of the
+// lane pair L, L ^ 1.  Every lane of the warp must call it (lanes of a vector
+// that does not exist pass zeros).  codes[j] holds the e4m3 codes of elements
+// 4j .. 4j + 3 of this lane's slice, little-endian.
+template <int D>
+__device__ __forceinline__ void rotate_quant_lanes(float (&r)[64], uint32_t (&codes)[16],
+                                                   float *scale) {
+    static_assert(D == 64 || D == 128, "one or two lanes per vector");
+#pragma unroll
+    for (int h = 1; h < 64; h <<= 1) {
+#pragma unroll
+        for (int e = 0; e < 64; e++) {
+            if (e & h) continue;
+            const float a = r[e], b = r[e + h];
+            r[e] = a + b;
+            r[e + h] = a - b;
+        }
+    }
+    if constexpr (D == 128) {
+        const bool upper = (threadIdx.x & 1) != 0;
+#pragma unroll
+        for (int e = 0; e < 64; e++) {
+            const float p = __shfl_xor_sync(0xffffffffu, r[e], 1);
+            r[e] = upper ? __fsub_rn(p, r[e]) : __fadd_rn(r[e], p);
+        }
+    }
+    float amax = 0.f;
+#pragma unroll
+    for (int e = 0; e < 64; e++) {
+        r[e] = __fmul_rn(r[e], HadamardScale<D>::value);
+        amax = fmaxf(amax, fabsf(r[e]));
+    }
+    if constexpr (D == 128) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
+    const float s = __fdiv_rn(fmaxf(amax, 1e-4f), 448.0f);
+#pragma unroll
+    for (int j = 0; j < 16; j++)
+        codes[j] = e4m3x2_rn_sat(__fdiv_rn(r[4 * j], s), __fdiv_rn(r[4 * j + 1], s)) |
+                   e4m3x2_rn_sat(__fdiv_rn(r[4 * j + 2], s), __fdiv_rn(r[4 * j + 3], s)) << 16;
+    *scale = s;
 }
 
 // Loads this lane's E elements of a D-vector (fp32 or bf16).
