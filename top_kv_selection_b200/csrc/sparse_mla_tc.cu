@@ -7,29 +7,35 @@
 // value mix).
 //
 // Shapes: Hq = 128 heads (the MMA M), rows [c (512) | k_pe (64)] bf16.
-// One CTA computes, for one query row, one 256-wide half of the output over
-// one share ("split") of the selected rows:
-//   warps 5..8  gather 32 selected rows per tile into a 2-stage ring with
-//               16-byte cp.async, straight into the 128B-swizzled K-major
-//               layout (nine 64-column blocks of 32 rows x 128 B); each warp
-//               copies 8 rows, consecutive lanes consecutive 16-byte pieces;
-//               a tile is published (wait, proxy fence, arrive) two tiles
-//               later, or at once before the producer would block;
-//   warp 0      S = Q C^T: 36 tcgen05.mma kind::f16 (M=128, N=32, K=16) per
-//               tile with both operands in shared memory (the whole query,
-//               144 KB, is loaded once by TMA); O += P C[:, half]: 2 MMAs
-//               (N=256, K=16) with A = P from TMEM and B = the same shared
-//               tile read as an MN-major operand (no transpose copy).  The
-//               previous tile's PV is slotted between this tile's QK column
-//               blocks as soon as its P is ready, so its stage is freed early;
-//   warps 1..4  one thread per head: online softmax in the exp2 domain with
-//               lazy rescaling (the fp32 accumulator in TMEM is rescaled only
-//               when a head's running max grows by more than 8), P written to
-//               TMEM as bf16, then the epilogue.
-// TMEM: O 256 | S 2 x 32 | P 2 x 16 columns.  The logits are computed by both
-// halves of a row (the output accumulator alone fills half of TMEM and the
-// query fills most of shared memory), so each gathered row is read twice from
-// L2 but once from HBM.
+// A cluster of two CTAs computes one query row over one share ("split") of
+// its selected rows.  CTA r of the pair owns
+//   - columns [256r, 256r + 320) of the query and of every gathered row
+//     (five 64-column blocks; block 4 of CTA 0 and block 0 of CTA 1 are the
+//     same columns 256..319),
+//   - the logit contraction over columns [288r, 288r + 288), i.e. half of
+//     q . [c | k_pe], and
+//   - output columns [256r, 256r + 256).
+// Per tile of 64 gathered rows:
+//   warps 5..8  gather the CTA's 640 bytes of each row with 16-byte cp.async
+//               straight into the 128B-swizzled K-major layout (a 2-stage
+//               ring; a tile is published two tiles later, or at once before
+//               the producer would block);
+//   warp 0      S_r = Q_r C_r^T: 18 tcgen05.mma kind::f16 (M=128, N=64, K=16)
+//               with both operands in shared memory; O += P C[:, own 256]:
+//               4 MMAs (N=256, K=16) with A = P from TMEM and B = the same
+//               shared tile read as an MN-major operand.  The previous tile's
+//               PV is slotted between this tile's QK blocks once its P is
+//               ready;
+//   warps 1..4  one thread per head: read the partial logits S_r from TMEM,
+//               send them to the partner CTA's shared memory (DSMEM), add
+//               the partner's (S_0 + S_1 in both CTAs: the same bits, since
+//               fp32 addition commutes), then the online softmax in the exp2
+//               domain with lazy rescaling (the TMEM accumulator is rescaled
+//               only when a head's running max grows by more than 8), P to
+//               TMEM as bf16, and the epilogue.
+// Both CTAs run the same softmax on the same logits, so their P, running max
+// and sum agree exactly; each accumulates its own half of the output.
+// TMEM: O 256 | S 2 x 64 | P 2 x 32 columns.
 // With several splits per row, unnormalised partial outputs and (max, sum)
 // pairs go to the workspace and a combine kernel merges them.
 #include "common.cuh"
@@ -40,22 +46,26 @@ namespace dsa {
 namespace {
 
 constexpr int kHq = 128, kDc = 512, kDr = 64, kDqk = kDc + kDr;
-constexpr int kNB = kDqk / 64;                  // 64-column blocks per row: 9
+constexpr int kLB = 5;                          // 64-column blocks held per CTA
 constexpr int kDh = 256;                        // output columns per CTA
-constexpr int kRows = 32;                       // gathered rows per tile
-constexpr int kStages = 2;
+constexpr int kRows = 64;                       // gathered rows per tile (QK N)
+constexpr int kStages = 4;
 constexpr int kThreads = 288;               // warp 0 MMA, 1..4 softmax, 5..8 gather
 constexpr int kMaxSel = 2048;                   // selection slots held in shared memory
-constexpr uint32_t kColO = 0, kColS = 256, kColP = 320, kTmemCols = 512;
+// TMEM columns: O (fp32) | S (fp32) | P (bf16 pairs) | Q (bf16 pairs, this CTA's 320)
+constexpr uint32_t kColO = 0, kColS = 256, kColP = 320, kColQ = 352, kTmemCols = 512;
+static_assert(kColQ + kLB * 64 / 2 == kTmemCols, "the query fills the last TMEM columns");
 constexpr int kBlk = kRows * 128;               // bytes of one column block of a tile
-constexpr int kTileBytes = kNB * kBlk;          // 36864
-constexpr int kQBlk = kHq * 128;                // 16384
+constexpr int kTileBytes = kLB * kBlk;          // 40960
+constexpr int kChunks = kLB * 8;                // 16-byte pieces of a row per CTA: 40
+constexpr int kRxBytes = kHq * kRows * 4;       // partner's partial logits
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
 
-constexpr size_t kSmemBytes = 1024 + (size_t)kStages * kTileBytes + (size_t)kNB * kQBlk +
+constexpr size_t kSmemBytes = 1024 + (size_t)kStages * kTileBytes + kRxBytes +
                               kMaxSel * sizeof(int32_t) + 32 * sizeof(uint64_t) + 64;
-constexpr int kLag = 2;                          // gather tiles in flight per thread beyond the one issued
+constexpr int kLag = 1;                          // gather tiles in flight per thread beyond the one issued
+constexpr int kQBlk = kHq * 128;                 // one 64-column block of the query (TMA box)
 
 struct MlaArgs {
     const __nv_bfloat16 *q;
@@ -63,7 +73,7 @@ struct MlaArgs {
     const int32_t *idx;
     __nv_bfloat16 *out;
     float *lse;
-    float *part_o;      // [units][128][256]  (splits > 1)
+    float *part_o;      // [units][128][256]  (splits > 1), unit = (row * splits + sp) * 2 + r
     float2 *part_ml;    // [units][128]
     int64_t t_max;
     int64_t start_pos;
@@ -81,51 +91,32 @@ template <int N> __device__ __forceinline__ void cp_async_wait() {
     asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
 }
 
-__device__ __forceinline__ int block_scan_flag_all(bool flag, int *warp_tot, int *total) {
-    constexpr int kW = kThreads / 32;
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    const unsigned ballot = __ballot_sync(0xffffffffu, flag);
-    const int in_warp = __popc(ballot & ((1u << lane) - 1u));
-    if (lane == 0) warp_tot[warp] = __popc(ballot);
-    __syncthreads();
-    if (threadIdx.x == 0) {
-        int acc = 0;
-        for (int w = 0; w < kW; w++) {
-            const int v = warp_tot[w];
-            warp_tot[w] = acc;
-            acc += v;
-        }
-        warp_tot[kW] = acc;
-    }
-    __syncthreads();
-    const int r = warp_tot[warp] + in_warp;
-    *total = warp_tot[kW];
-    __syncthreads();
-    return r;
-}
-
 __global__ void __launch_bounds__(kThreads, 1)
 sparse_mla_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const MlaArgs a) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t *sc = smem;                                      // C tiles
-    uint8_t *sq = sc + kStages * kTileBytes;                 // Q, nine 64-column blocks
-    int32_t *list = reinterpret_cast<int32_t *>(sq + kNB * kQBlk);
+    float4 *rx = reinterpret_cast<float4 *>(sc + kStages * kTileBytes);   // partner's logits [16][128]
+    int32_t *list = reinterpret_cast<int32_t *>(sc + kStages * kTileBytes + kRxBytes);
     uint64_t *bars = reinterpret_cast<uint64_t *>(list + kMaxSel);
     uint64_t *c_full = bars, *c_empty = bars + kStages;
-    uint64_t *s_full = bars + 2 * kStages, *s_empty = s_full + 2;
-    uint64_t *p_full = s_empty + 2, *pv_done = p_full + 2;
-    uint64_t *q_full = pv_done + 2, *q_ready = q_full + 1;
-    uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(q_ready + 1);
+    uint64_t *s_full = bars + 2 * kStages, *s_empty = s_full + 1;
+    uint64_t *p_full = s_empty + 1, *pv_done = p_full + 1;
+    uint64_t *q_ready = pv_done + 1;    // the query is in TMEM
+    uint64_t *q_full = q_ready + 1;     // the query's TMA copy (ring stages 2..3) landed
+    uint64_t *q_free = q_full + 1;      // ... and has been moved to TMEM
+    uint64_t *rx_full = q_free + 1;     // partner's logits of the current tile landed
+    uint64_t *tx_ok = rx_full + 1;      // partner has read what this CTA sent last
+    uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(tx_ok + 1);
     volatile int *abort = reinterpret_cast<volatile int *>(tmem_holder + 1);
     int *scan_tmp = const_cast<int *>(abort) + 1;            // 10 ints
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int unit = blockIdx.x;                             // (row * 2 + half) * splits + sp
-    const int sp = unit % a.splits;
-    const int half = (unit / a.splits) & 1;
-    const int64_t row = unit / (a.splits * 2);
+    const int unit = blockIdx.x;                             // (row * splits + sp) * 2 + r
+    const int cr = unit & 1;                                 // rank in the pair
+    const int sp = (unit >> 1) % a.splits;
+    const int64_t row = (unit >> 1) / a.splits;
     const int64_t b = row / a.S, s = row - b * a.S;
     const int64_t limit = a.start_pos + s;
     const bool is_softmax = warp >= 1 && warp <= 4;
@@ -138,13 +129,15 @@ sparse_mla_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const MlaArgs a) 
             tc::mbar_init(&c_full[i], 128);
             tc::mbar_init(&c_empty[i], 1);
         }
-        for (int i = 0; i < 2; i++) {
-            tc::mbar_init(&s_full[i], 1);
-            tc::mbar_init(&s_empty[i], 128);
-            tc::mbar_init(&p_full[i], 128);
-            tc::mbar_init(&pv_done[i], 1);
-        }
+        tc::mbar_init(s_full, 1);
+        tc::mbar_init(s_empty, 128);
+        tc::mbar_init(p_full, 128);
+        tc::mbar_init(pv_done, 1);
+        tc::mbar_init(q_ready, 128);
         tc::mbar_init(q_full, 1);
+        tc::mbar_init(q_free, 128);
+        tc::mbar_init(rx_full, 128);
+        tc::mbar_init(tx_ok, 128);
         *abort = 0;
         tc::fence_mbar_init();
         tc::tma_prefetch_desc(&tm_q);
@@ -154,59 +147,107 @@ sparse_mla_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const MlaArgs a) 
         tc::tmem_relinquish();
     }
     tc::tc_fence_before();
-    __syncthreads();
+    tc::cluster_sync_all();          // both CTAs' barriers exist before any remote arrive
     tc::tc_fence_after();
     const uint32_t tmem = *tmem_holder;
-
-    // the query does not depend on the preceding kernel: load it first
-    if (threadIdx.x == 160) {
-        tc::mbar_arrive_expect_tx(q_full, kNB * kQBlk);
-        for (int j = 0; j < kNB; j++)
-            tc::tma_load_2d(sq + j * kQBlk, &tm_q, j * 64, (int)(row * kHq), q_full);
+    if (threadIdx.x == 0) {
+        // this CTA's five 64-column blocks of the query, staged in ring
+        // stages 2..3 until the softmax warps have moved them to TMEM
+        tc::mbar_arrive_expect_tx(q_full, kLB * kQBlk);
+        for (int j = 0; j < kLB; j++)
+            tc::tma_load_2d(sc + 2 * kTileBytes + j * kQBlk, &tm_q, (cr * 4 + j) * 64,
+                            (int)(row * kHq), q_full);
     }
 
-    // valid selections of this row, in slot order
-    constexpr int kPer = (kMaxSel + kThreads - 1) / kThreads;
-    int32_t slot[kPer];
+    // valid selections of this row, in slot order (the same list in both CTAs):
+    // threads 0..255 take 8 consecutive slots each, one block-wide scan
+    constexpr int kPer = kMaxSel / 256;
+    int32_t v8[kPer];
+    int cnt = 0;
 #pragma unroll
-    for (int r = 0; r < kPer; r++) {
-        const int j = r * kThreads + threadIdx.x;
-        slot[r] = j < a.k ? __ldg(a.idx + row * a.k + j) : -1;
+    for (int e = 0; e < kPer; e++) {
+        const int j = threadIdx.x * kPer + e;
+        int32_t t = threadIdx.x < 256 && j < a.k ? __ldg(a.idx + row * a.k + j) : -1;
+        if (t >= 0 && (int64_t)t <= limit) {
+            if ((int64_t)t >= a.t_max) {
+                record_error(a.err, DSA_ERR_DEVICE);
+                t = -1;
+            }
+        } else {
+            t = -1;
+        }
+        v8[e] = t;
+        cnt += t >= 0 ? 1 : 0;
     }
-    int n = 0;
+    int incl = cnt;
 #pragma unroll
-    for (int r = 0; r < kPer; r++) {
-        if (r * kThreads >= a.k) break;
-        const int32_t t = slot[r];
-        const bool v = t >= 0 && (int64_t)t <= limit && (int64_t)t < a.t_max;
-        if (t >= 0 && (int64_t)t <= limit && (int64_t)t >= a.t_max) record_error(a.err, DSA_ERR_DEVICE);
-        int tot;
-        const int pos = block_scan_flag_all(v, scan_tmp, &tot);
-        if (v) list[n + pos] = t;
-        n += tot;
+    for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += y;
     }
-    const int lo = (int)((int64_t)sp * n / a.splits);
-    const int n_my = (int)((int64_t)(sp + 1) * n / a.splits) - lo;
-    const int n_tiles = (n_my + kRows - 1) / kRows;
+    if (lane == 31) scan_tmp[warp] = incl;
+    __syncthreads();
+    int n = 0, pos = incl - cnt;
+#pragma unroll
+    for (int w = 0; w < 8; w++) {
+        const int c = scan_tmp[w];
+        if (w < warp) pos += c;
+        n += c;
+    }
+#pragma unroll
+    for (int e = 0; e < kPer; e++)
+        if (v8[e] >= 0) list[pos++] = v8[e];
+    __syncthreads();
+    // this split's tiles of 64 rows
+    const int nt_all = (n + kRows - 1) / kRows;
+    const int t_lo = (int)((int64_t)sp * nt_all / a.splits);
+    const int t_hi = (int)((int64_t)(sp + 1) * nt_all / a.splits);
+    const int lo = t_lo * kRows;
+    const int n_my = (t_hi * kRows < n ? t_hi * kRows : n) - lo;
+    const int n_tiles = t_hi - t_lo;
+
+    // the query (this CTA's 320 columns, two bf16 per TMEM column) moves from
+    // its staging copy to TMEM, one head per lane, by the softmax warps
+    if (is_softmax) {
+        if (tc::mbar_wait(q_full, 0, a.err, abort)) {
+            const uint8_t *qs = sc + 2 * kTileBytes;
+#pragma unroll 1
+            for (int c = 0; c < kLB * 8 / 4; c++) {          // 10 x 4 pieces of 16 bytes
+                uint32_t r[16];
+#pragma unroll
+                for (int u = 0; u < 4; u++) {
+                    const int piece = 4 * c + u, blk = piece >> 3, ch = piece & 7;
+                    const uint4 v = *reinterpret_cast<const uint4 *>(
+                        qs + blk * kQBlk + h * 128 + ((ch ^ (h & 7)) << 4));
+                    r[4 * u] = v.x; r[4 * u + 1] = v.y; r[4 * u + 2] = v.z; r[4 * u + 3] = v.w;
+                }
+                tc::tmem_st16(tmem + lane_addr + kColQ + c * 16, r);
+            }
+            tc::tmem_wait_st();
+        }
+        tc::tc_fence_before();
+        tc::mbar_arrive(q_ready);
+        tc::mbar_arrive(q_free);
+    }
 
     if (n_tiles == 0) {                                      // nothing selected here
-        if (threadIdx.x == 160) tc::mbar_wait(q_full, 0, a.err, abort);   // Q copy landed
         if (is_softmax) {
             if (a.splits > 1) {
-                float4 *po = reinterpret_cast<float4 *>(a.part_o + ((int64_t)unit * kHq + h) * kDh);
-                for (int c = 0; c < kDh / 4; c++) po[c] = make_float4(0.f, 0.f, 0.f, 0.f);
+                float4 *po = reinterpret_cast<float4 *>(a.part_o + (int64_t)unit * kHq * kDh) + h;
+                for (int c = 0; c < kDh / 4; c++) po[c * kHq] = make_float4(0.f, 0.f, 0.f, 0.f);
                 a.part_ml[(int64_t)unit * kHq + h] = make_float2(-INFINITY, 0.f);
             } else {
-                __nv_bfloat16 *o = a.out + (row * kHq + h) * kDc + half * kDh;
+                __nv_bfloat16 *o = a.out + (row * kHq + h) * kDc + cr * kDh;
                 for (int c = 0; c < kDh; c++) o[c] = __float2bfloat16_rn(0.f);
-                if (half == 0 && a.lse) a.lse[row * kHq + h] = -INFINITY;
+                if (cr == 0 && a.lse) a.lse[row * kHq + h] = -INFINITY;
             }
         }
     } else if (warp >= 5) {
-        // ---- gather: warp w copies rows 8w..8w+7 of each tile; lane l copies
-        // the 16-byte pieces l, l+32, l+64 (< 72) of each row
-        const int pw = warp - 5;
+        // ---- gather: the 128 threads copy the tile's 64 x 40 pieces of 16
+        // bytes, consecutive threads consecutive pieces of a row
+        const int gt = threadIdx.x - 160;
         const int64_t rbase = b * a.t_max;
+        const __nv_bfloat16 *kv_cols = a.kv + cr * kDh;     // this CTA's first column
         int issued = 0, signalled = 0;
         for (int i = 0; i < n_tiles; i++) {
             const int st = i % kStages;
@@ -219,20 +260,15 @@ sparse_mla_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const MlaArgs a) 
                 for (; signalled < issued; signalled++) tc::mbar_arrive(&c_full[signalled % kStages]);
                 if (!tc::mbar_wait(&c_empty[st], ph, a.err, abort)) break;
             }
+            if (i == 2 && !tc::mbar_wait(q_free, 0, a.err, abort)) break;   // stages 2..3 held the query
             uint8_t *tile = sc + st * kTileBytes;
-#pragma unroll 1
-            for (int jj = 0; jj < 8; jj++) {
-                const int j = pw * 8 + jj;
+#pragma unroll 4
+            for (int f = gt; f < kRows * kChunks; f += 128) {
+                const int j = f / kChunks, c = f - j * kChunks;
                 int r = i * kRows + j;
                 if (r >= n_my) r = n_my - 1;                 // padding: a valid row
-                const __nv_bfloat16 *src = a.kv + (rbase + list[lo + r]) * kDqk;
-#pragma unroll
-                for (int u = 0; u < 3; u++) {
-                    const int c = lane + 32 * u;
-                    if (c < 72)
-                        cp_async16(tile + (c >> 3) * kBlk + j * 128 + (((c & 7) ^ (j & 7)) << 4),
-                                   src + c * 8);
-                }
+                const __nv_bfloat16 *src = kv_cols + (rbase + list[lo + r]) * kDqk;
+                cp_async16(tile + (c >> 3) * kBlk + j * 128 + (((c & 7) ^ (j & 7)) << 4), src + c * 8);
             }
             cp_async_commit();
             issued = i + 1;
@@ -243,98 +279,126 @@ sparse_mla_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const MlaArgs a) 
                 signalled++;
             }
         }
-        cp_async_wait<0>();
-        tc::fence_proxy_async_smem();
-        for (; signalled < issued; signalled++) tc::mbar_arrive(&c_full[signalled % kStages]);
+        // publish the remaining tiles in order, each as soon as it has landed
+        for (; signalled < issued; signalled++) {
+            if (issued - signalled - 1 >= 1) cp_async_wait<1>();
+            else cp_async_wait<0>();
+            tc::fence_proxy_async_smem();
+            tc::mbar_arrive(&c_full[signalled % kStages]);
+        }
     } else if (warp == 0) {
         if (lane == 0) {
             const uint32_t id_qk = tc::instr_desc(tc::kFmtBF16, tc::kFmtBF16, 128, kRows);
             const uint32_t id_pv = tc::instr_desc(tc::kFmtBF16, tc::kFmtBF16, 128, kDh, true);
-            const uint32_t sc_addr = tc::smem_u32(sc), sq_addr = tc::smem_u32(sq);
-            bool ok = tc::mbar_wait(q_full, 0, a.err, abort);
-            // O += P C[:, half] for tile j (P(j) must be published)
+            const uint32_t sc_addr = tc::smem_u32(sc);
+            // this CTA's K steps (16 columns each) of the logit contraction:
+            // 18 of the 20 in its five blocks
+            const int ks_first = cr == 0 ? 0 : 2, ks_last = cr == 0 ? 4 * kLB - 2 : 4 * kLB;
+            bool ok = tc::mbar_wait(q_ready, 0, a.err, abort);
+            // O += P C[:, own 256] for tile j (P(j) must be published)
             auto pv_issue = [&](int j) {
-                const int st = j % kStages, pb = j & 1;
+                const int st = j % kStages;
                 tc::tc_fence_after();
 #pragma unroll
                 for (int ks = 0; ks < kRows / 16; ks++) {
-                    const uint64_t bd = tc::smem_desc(
-                        sc_addr + st * kTileBytes + half * (kDh / 64) * kBlk + ks * 2048, 1024,
-                        tc::kSwizzle128B, kBlk);
-                    tc::mma_f16_ts(tmem + kColO, tmem + kColP + pb * 16 + ks * 8, bd, id_pv,
-                                   j > 0 || ks > 0);
+                    const uint64_t bd = tc::smem_desc(sc_addr + st * kTileBytes + ks * 2048, 1024,
+                                                      tc::kSwizzle128B, kBlk);
+                    tc::mma_f16_ts(tmem + kColO, tmem + kColP + ks * 8, bd, id_pv, j > 0 || ks > 0);
                 }
                 tc::tc_commit(&c_empty[st]);
-                tc::tc_commit(&pv_done[pb]);
+                tc::tc_commit(pv_done);
             };
-            // S = Q C^T for tile i, one 64-column block at a time; the PV of the
-            // previous tile (pend >= 0) is slotted in as soon as its P is
-            // published, so its stage is released without waiting for all of
-            // this tile's MMAs
+            // S_r = Q_r C_r^T for tile i, A = Q from TMEM; the PV of the previous
+            // tile (pend >= 0) is slotted in as soon as its P is published
             auto qk = [&](int i, int pend) -> bool {
-                const int st = i % kStages, sb = i & 1;
+                const int st = i % kStages;
                 if (!tc::mbar_wait(&c_full[st], (uint32_t)(i / kStages) & 1u, a.err, abort)) return false;
-                if (!tc::mbar_wait(&s_empty[sb], ((uint32_t)(i >> 1) & 1u) ^ 1u, a.err, abort)) return false;
+                if (!tc::mbar_wait(s_empty, ((uint32_t)i & 1u) ^ 1u, a.err, abort)) return false;
                 tc::tc_fence_after();
-                const uint32_t d = tmem + kColS + sb * kRows;
 #pragma unroll 1
-                for (int cb = 0; cb < kNB; cb++) {
-                    if (pend >= 0 && tc::mbar_test_wait(&p_full[pend & 1], (uint32_t)(pend >> 1) & 1u)) {
+                for (int kk = ks_first; kk < ks_last; kk++) {
+                    if ((kk & 3) == 0 && pend >= 0 &&
+                        tc::mbar_test_wait(p_full, (uint32_t)pend & 1u)) {
                         pv_issue(pend);
                         pend = -1;
                     }
-#pragma unroll
-                    for (int ks = 0; ks < 4; ks++) {
-                        const uint64_t ad = tc::smem_desc(sq_addr + cb * kQBlk + ks * 32, 1024, tc::kSwizzle128B);
-                        const uint64_t bd = tc::smem_desc(sc_addr + st * kTileBytes + cb * kBlk + ks * 32,
-                                                          1024, tc::kSwizzle128B);
-                        tc::mma_f16(d, ad, bd, id_qk, (cb | ks) != 0);
-                    }
+                    const int cb = kk >> 2, ks = kk & 3;
+                    const uint64_t bd = tc::smem_desc(sc_addr + st * kTileBytes + cb * kBlk + ks * 32,
+                                                      1024, tc::kSwizzle128B);
+                    tc::mma_f16_ts(tmem + kColS, tmem + kColQ + kk * 8, bd, id_qk, kk != ks_first);
                 }
-                tc::tc_commit(&s_full[sb]);
+                tc::tc_commit(s_full);
                 if (pend >= 0) {
-                    if (!tc::mbar_wait(&p_full[pend & 1], (uint32_t)(pend >> 1) & 1u, a.err, abort)) return false;
+                    if (!tc::mbar_wait(p_full, (uint32_t)pend & 1u, a.err, abort)) return false;
                     pv_issue(pend);
                 }
                 return true;
             };
             if (ok) ok = qk(0, -1);
             for (int i = 1; ok && i < n_tiles; i++) ok = qk(i, i - 1);
-            if (ok && tc::mbar_wait(&p_full[(n_tiles - 1) & 1], (uint32_t)((n_tiles - 1) >> 1) & 1u, a.err, abort))
+            if (ok && tc::mbar_wait(p_full, (uint32_t)(n_tiles - 1) & 1u, a.err, abort))
                 pv_issue(n_tiles - 1);
         }
     } else {
         // ---- softmax warps
+        const uint32_t peer = (uint32_t)(cr ^ 1);
+        const uint32_t peer_rx = tc::map_shared_rank(rx, peer);
+        const uint32_t peer_rx_full = tc::map_shared_rank(rx_full, peer);
+        const uint32_t peer_tx_ok = tc::map_shared_rank(tx_ok, peer);
         float m_run = -INFINITY, l = 0.f;
         bool ok = true;
         for (int i = 0; i < n_tiles && ok; i++) {
-            const int sb = i & 1;
-            if (!tc::mbar_wait(&s_full[sb], (uint32_t)(i >> 1) & 1u, a.err, abort)) { ok = false; break; }
+            if (!tc::mbar_wait(s_full, (uint32_t)i & 1u, a.err, abort)) { ok = false; break; }
             tc::tc_fence_after();
-            uint32_t r0[16], r1[16];
-            tc::tmem_ld16(tmem + lane_addr + kColS + sb * kRows, r0);
-            tc::tmem_ld16(tmem + lane_addr + kColS + sb * kRows + 16, r1);
+            uint32_t own[kRows];
+#pragma unroll
+            for (int q = 0; q < kRows / 16; q++)
+                tc::tmem_ld16(tmem + lane_addr + kColS + q * 16,
+                              *reinterpret_cast<uint32_t(*)[16]>(own + q * 16));
             tc::tmem_wait_ld();
             tc::tc_fence_before();
-            tc::mbar_arrive(&s_empty[sb]);
+            tc::mbar_arrive(s_empty);
+            // exchange the partial logits: the partner must have read the
+            // previous tile's before they are overwritten
+            if (i > 0 && !tc::mbar_wait_cluster(tx_ok, (uint32_t)(i - 1) & 1u, a.err, abort)) {
+                ok = false;
+                break;
+            }
+#pragma unroll
+            for (int q = 0; q < kRows / 4; q++)
+                tc::st_cluster_v4(peer_rx + (uint32_t)((q * kHq + h) * 16),
+                                  __uint_as_float(own[4 * q]), __uint_as_float(own[4 * q + 1]),
+                                  __uint_as_float(own[4 * q + 2]), __uint_as_float(own[4 * q + 3]));
+            tc::mbar_arrive_cluster(peer_rx_full);
+            if (!tc::mbar_wait_cluster(rx_full, (uint32_t)i & 1u, a.err, abort)) { ok = false; break; }
             const int nv = n_my - i * kRows;
             float sv[kRows];
             float m_tile = -INFINITY;
 #pragma unroll
-            for (int j = 0; j < kRows; j++) {
-                const uint32_t bits = j < 16 ? r0[j] : r1[j - 16];
-                sv[j] = j < nv ? __uint_as_float(bits) * a.scale_log2 : -INFINITY;
-                m_tile = fmaxf(m_tile, sv[j]);
+            for (int q = 0; q < kRows / 4; q++) {
+                const float4 o = rx[q * kHq + h];
+                const float ov[4] = {o.x, o.y, o.z, o.w};
+#pragma unroll
+                for (int e = 0; e < 4; e++) {
+                    const int j = 4 * q + e;
+                    const float lg = __uint_as_float(own[j]) + ov[e];   // S_0 + S_1 in either CTA
+                    sv[j] = j < nv ? lg * a.scale_log2 : -INFINITY;
+                    m_tile = fmaxf(m_tile, sv[j]);
+                }
+            }
+            tc::mbar_arrive_cluster(peer_tx_ok);
+            // PV(i-1) must be done: it reads P, and O may be rescaled below
+            if (i > 0) {
+                if (!tc::mbar_wait(pv_done, (uint32_t)(i - 1) & 1u, a.err, abort)) {
+                    ok = false;
+                    break;
+                }
+                tc::tc_fence_after();
             }
             if (__any_sync(0xffffffffu, m_tile > m_run + 8.f)) {
                 const float m_new = fmaxf(m_run, m_tile);
                 const float alpha = m_run == -INFINITY ? 0.f : exp2f(m_run - m_new);
                 if (i > 0) {
-                    if (!tc::mbar_wait(&pv_done[(i - 1) & 1], (uint32_t)((i - 1) >> 1) & 1u, a.err, abort)) {
-                        ok = false;
-                        break;
-                    }
-                    tc::tc_fence_after();
 #pragma unroll 1
                     for (int c0 = 0; c0 < kDh; c0 += 16) {
                         uint32_t o[16];
@@ -349,28 +413,25 @@ sparse_mla_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const MlaArgs a) 
                 l *= alpha;
                 m_run = m_new;
             }
-            if (i >= 2 && !tc::mbar_wait(&pv_done[i & 1], (uint32_t)((i - 2) >> 1) & 1u, a.err, abort)) {
-                ok = false;
-                break;
-            }
-            uint32_t pk[16];
+            uint32_t pk[kRows / 2];
 #pragma unroll
-            for (int c = 0; c < 16; c++) {
+            for (int c = 0; c < kRows / 2; c++) {
                 const float p0 = exp2f(sv[2 * c] - m_run), p1 = exp2f(sv[2 * c + 1] - m_run);
                 l += p0 + p1;
                 const __nv_bfloat162 v = __floats2bfloat162_rn(p0, p1);
                 pk[c] = *reinterpret_cast<const uint32_t *>(&v);
             }
-            tc::tmem_st16(tmem + lane_addr + kColP + (i & 1) * 16, pk);
+            tc::tmem_st16(tmem + lane_addr + kColP, *reinterpret_cast<uint32_t(*)[16]>(pk));
+            tc::tmem_st16(tmem + lane_addr + kColP + 16, *reinterpret_cast<uint32_t(*)[16]>(pk + 16));
             tc::tmem_wait_st();
             tc::tc_fence_before();
-            tc::mbar_arrive(&p_full[i & 1]);
+            tc::mbar_arrive(p_full);
         }
-        if (ok && tc::mbar_wait(&pv_done[(n_tiles - 1) & 1], (uint32_t)((n_tiles - 1) >> 1) & 1u,
-                                a.err, abort)) {
+        if (ok && tc::mbar_wait(pv_done, (uint32_t)(n_tiles - 1) & 1u, a.err, abort)) {
             tc::tc_fence_after();
             if (a.splits > 1) {
-                float4 *po = reinterpret_cast<float4 *>(a.part_o + ((int64_t)unit * kHq + h) * kDh);
+                // [column / 4][head] float4s: a warp stores 512 contiguous bytes
+                float4 *po = reinterpret_cast<float4 *>(a.part_o + (int64_t)unit * kHq * kDh) + h;
 #pragma unroll 1
                 for (int c0 = 0; c0 < kDh; c0 += 16) {
                     uint32_t o[16];
@@ -378,13 +439,13 @@ sparse_mla_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const MlaArgs a) 
                     tc::tmem_wait_ld();
 #pragma unroll
                     for (int v = 0; v < 4; v++)
-                        po[c0 / 4 + v] = make_float4(__uint_as_float(o[4 * v]), __uint_as_float(o[4 * v + 1]),
-                                                     __uint_as_float(o[4 * v + 2]), __uint_as_float(o[4 * v + 3]));
+                        po[(c0 / 4 + v) * kHq] = make_float4(__uint_as_float(o[4 * v]), __uint_as_float(o[4 * v + 1]),
+                                                             __uint_as_float(o[4 * v + 2]), __uint_as_float(o[4 * v + 3]));
                 }
                 a.part_ml[(int64_t)unit * kHq + h] = make_float2(m_run, l);
             } else {
                 const float inv = l > 0.f ? 1.f / l : 0.f;
-                uint4 *o16 = reinterpret_cast<uint4 *>(a.out + (row * kHq + h) * kDc + half * kDh);
+                uint4 *o16 = reinterpret_cast<uint4 *>(a.out + (row * kHq + h) * kDc + cr * kDh);
 #pragma unroll 1
                 for (int c0 = 0; c0 < kDh; c0 += 16) {
                     uint32_t o[16], w[8];
@@ -399,80 +460,74 @@ sparse_mla_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const MlaArgs a) 
                     o16[c0 / 8] = make_uint4(w[0], w[1], w[2], w[3]);
                     o16[c0 / 8 + 1] = make_uint4(w[4], w[5], w[6], w[7]);
                 }
-                if (half == 0 && a.lse) a.lse[row * kHq + h] = l > 0.f ? (m_run + log2f(l)) * kLn2 : -INFINITY;
+                if (cr == 0 && a.lse) a.lse[row * kHq + h] = l > 0.f ? (m_run + log2f(l)) * kLn2 : -INFINITY;
             }
         }
     }
-
     tc::tc_fence_before();
     __syncthreads();
     if (warp == 0) {
         tc::tc_fence_after();
         tc::tmem_dealloc(tmem, kTmemCols);
     }
+    tc::cluster_sync_all();          // the partner no longer touches this CTA's shared memory
 }
 
 // Merges the splits of each (row, half): out = sum_s 2^(m_s - m) O_s / sum_s 2^(m_s - m) l_s.
-// One warp per head; lane l covers output columns 8l..8l+7 (coalesced rows).
-constexpr int kCombineHeads = 8;
-__global__ void __launch_bounds__(32 * kCombineHeads)
+// The partials are [column / 4][head] float4s; thread (head, quad) merges four
+// output columns of one head, consecutive threads consecutive heads (coalesced).
+constexpr int kCombineQuads = 2;                         // column quads per block
+__global__ void __launch_bounds__(kHq * kCombineQuads)
 sparse_mla_combine_kernel(const float *__restrict__ part_o, const float2 *__restrict__ part_ml,
                           int splits, __nv_bfloat16 *__restrict__ out, float *__restrict__ lse) {
-    const int groups = kHq / kCombineHeads;
+    constexpr int groups = (kDh / 4) / kCombineQuads;
     const int64_t rh = blockIdx.x / groups;                 // row * 2 + half
     const int64_t row = rh >> 1;
     const int half = (int)(rh & 1);
-    const int h = (int)(blockIdx.x % groups) * kCombineHeads + (threadIdx.x >> 5);
-    const int lane = threadIdx.x & 31;
-    const int64_t u0 = rh * splits;
-    // all (max, sum) pairs first, then the partial rows four splits at a time,
-    // so that the loads of a batch are in flight together
+    const int h = threadIdx.x % kHq;
+    const int c4 = (int)(blockIdx.x % groups) * kCombineQuads + threadIdx.x / kHq;
+    // partial of split sp: unit (row * splits + sp) * 2 + half
+    const int64_t u0 = row * splits * 2 + half;
     float m = -INFINITY;
-    for (int sp = 0; sp < splits; sp++) m = fmaxf(m, part_ml[(u0 + sp) * kHq + h].x);
+    for (int sp = 0; sp < splits; sp++) m = fmaxf(m, part_ml[(u0 + 2 * sp) * kHq + h].x);
     float L = 0.f;
-    float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    // four splits at a time, so that their loads are in flight together
     for (int sp0 = 0; sp0 < splits; sp0 += 4) {
         float2 ml[4];
-        float4 x[4], y[4];
+        float4 x[4];
 #pragma unroll
         for (int u = 0; u < 4; u++) {
             const int sp = sp0 + u;
-            ml[u] = sp < splits ? part_ml[(u0 + sp) * kHq + h] : make_float2(-INFINITY, 0.f);
-            if (sp < splits) {
-                const float4 *po =
-                    reinterpret_cast<const float4 *>(part_o + ((u0 + sp) * kHq + h) * kDh) + 2 * lane;
-                x[u] = po[0];
-                y[u] = po[1];
-            }
+            ml[u] = sp < splits ? part_ml[(u0 + 2 * sp) * kHq + h] : make_float2(-INFINITY, 0.f);
+            if (sp < splits)
+                x[u] = reinterpret_cast<const float4 *>(part_o + (u0 + 2 * sp) * kHq * kDh)[c4 * kHq + h];
         }
 #pragma unroll
         for (int u = 0; u < 4; u++) {
             if (ml[u].x == -INFINITY) continue;
             const float w = exp2f(ml[u].x - m);
             L += w * ml[u].y;
-            acc[0] += w * x[u].x; acc[1] += w * x[u].y; acc[2] += w * x[u].z; acc[3] += w * x[u].w;
-            acc[4] += w * y[u].x; acc[5] += w * y[u].y; acc[6] += w * y[u].z; acc[7] += w * y[u].w;
+            acc.x += w * x[u].x; acc.y += w * x[u].y; acc.z += w * x[u].z; acc.w += w * x[u].w;
         }
     }
     const float inv = L > 0.f ? 1.f / L : 0.f;
-    uint32_t wv[4];
-#pragma unroll
-    for (int e = 0; e < 4; e++) {
-        const __nv_bfloat162 v = __floats2bfloat162_rn(acc[2 * e] * inv, acc[2 * e + 1] * inv);
-        wv[e] = *reinterpret_cast<const uint32_t *>(&v);
-    }
-    reinterpret_cast<uint4 *>(out + (row * kHq + h) * kDc + half * kDh)[lane] =
-        make_uint4(wv[0], wv[1], wv[2], wv[3]);
-    if (half == 0 && lse && lane == 0) lse[row * kHq + h] = L > 0.f ? (m + log2f(L)) * kLn2 : -INFINITY;
+    const __nv_bfloat162 v0 = __floats2bfloat162_rn(acc.x * inv, acc.y * inv);
+    const __nv_bfloat162 v1 = __floats2bfloat162_rn(acc.z * inv, acc.w * inv);
+    reinterpret_cast<uint2 *>(out + (row * kHq + h) * kDc + half * kDh)[c4] =
+        make_uint2(*reinterpret_cast<const uint32_t *>(&v0), *reinterpret_cast<const uint32_t *>(&v1));
+    if (half == 0 && c4 == 0 && lse) lse[row * kHq + h] = L > 0.f ? (m + log2f(L)) * kLn2 : -INFINITY;
 }
 
+// Splits per row: as many pairs as fill the SMs once, then as few as give the
+// same number of tiles to the busiest split (fewer partials to combine).
 int mla_splits(int64_t rows, int k) {
-    const int64_t units = rows * 2;
-    int64_t sp = num_sms() / units;
-    const int64_t max_sp = (k + kRows - 1) / kRows;
-    if (sp > max_sp) sp = max_sp;
-    if (sp < 1) sp = 1;
-    return (int)sp;
+    const int64_t tiles = (k + kRows - 1) / kRows;
+    int64_t sp = num_sms() / (rows * 2);
+    if (sp > tiles) sp = tiles;
+    if (sp < 1) return 1;
+    const int64_t per = (tiles + sp - 1) / sp;
+    return (int)((tiles + per - 1) / per);
 }
 
 }  // namespace
@@ -527,11 +582,24 @@ dsa_status launch_sparse_mla_tc(const void *q, const void *kv, int64_t t_max, co
     if (cudaFuncSetAttribute(sparse_mla_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)kSmemBytes) != cudaSuccess)
         return DSA_ERR_CUDA;
-    sparse_mla_tc_kernel<<<(unsigned)(rows * 2 * a.splits), kThreads, kSmemBytes, stream>>>(tm_q, a);
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)(rows * a.splits * 2));
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = kSmemBytes;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (cudaLaunchKernelEx(&cfg, sparse_mla_tc_kernel, tm_q, a) != cudaSuccess) return DSA_ERR_CUDA;
     dsa_status st = launch_status();
     if (st != DSA_OK || a.splits == 1) return st;
-    sparse_mla_combine_kernel<<<(unsigned)(rows * 2 * (kHq / kCombineHeads)), 32 * kCombineHeads,
-                                0, stream>>>(a.part_o, a.part_ml, a.splits, a.out, lse);
+    sparse_mla_combine_kernel<<<(unsigned)(rows * 2 * ((kDh / 4) / kCombineQuads)),
+                                kHq * kCombineQuads, 0, stream>>>(a.part_o, a.part_ml, a.splits,
+                                                                  a.out, lse);
     return launch_status();
 }
 
