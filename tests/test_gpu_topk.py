@@ -116,3 +116,39 @@ def test_topk_query_chunk_rows_of_different_lengths(dsa):
     got = _gpu_topk(dsa, sc, sp, 2048)
     ref = oracle.topk_select(sc, sp, 2048)
     assert np.array_equal(got, ref)
+
+
+def _tied_block_row(T, n_top, n_tied, tied_positions, seed):
+    """Uniform [0, 1) scores, n_top of them in [6, 7) and n_tied exactly 5.0 at
+    the given positions: with k between n_top and n_top + n_tied the k-th
+    largest is 5.0 and only the lowest-positioned ties are taken."""
+    rng = np.random.default_rng(seed)
+    row = rng.random(T, dtype=np.float32)
+    rest = np.setdiff1d(np.arange(T), tied_positions)
+    top = rng.choice(rest, n_top, replace=False)
+    row[top] = 6.0 + rng.random(n_top, dtype=np.float32)
+    row[tied_positions] = 5.0
+    return row
+
+
+def test_topk_many_tied_candidates_spread_over_the_cluster(dsa):
+    """4000 ties at the threshold, spread over the row: every CTA sends a few
+    hundred candidates and CTA 0 radix-selects among them."""
+    T = 131072
+    rows = [_tied_block_row(T, 1500, 4000, np.linspace(0, T - 1, 4000).astype(np.int64), s)
+            for s in range(2)]
+    sc = np.stack(rows).reshape(2, 1, T)
+    got = _gpu_topk(dsa, sc, T - 1, 2048)
+    ref = oracle.topk_select(sc, T - 1, 2048)
+    assert np.array_equal(got, ref)
+
+
+def test_topk_tied_candidates_crowded_into_one_slice(dsa):
+    """1000 ties in the first 1000 positions: one CTA holds more threshold-bin
+    candidates than it may send to CTA 0, so the cluster-wide radix rounds run."""
+    T = 131072
+    rows = [_tied_block_row(T, 1500, 1000, np.arange(1000), s) for s in range(2)]
+    sc = np.stack(rows).reshape(2, 1, T)
+    got = _gpu_topk(dsa, sc, T - 1, 2048)
+    ref = oracle.topk_select(sc, T - 1, 2048)
+    assert np.array_equal(got, ref)
