@@ -391,6 +391,9 @@ def run_ours(args, wl, world, rank, local):
     peak, peak_kind = _peaks()
     stages = time_stages(dsa, wl, copies, iters=max(10, min(args.steps, 500)))
     t_score = stages["decode_index_scores"]
+    prefill = None
+    if not args.no_prefill:
+        prefill = time_prefill_scoring(dsa, measure_fp8_peak(sustained=False)["fp8_e4m3_tflops"])
     # keys + scales of every cached token, plus the new tokens' fp32 queries,
     # weights and keys (the scores written are not algorithmic)
     score_bytes = wl.B * wl.T * (wl.D + 4) + wl.B * (wl.H * wl.D * 4 + wl.H * 4 + wl.D * 4)
@@ -407,7 +410,11 @@ def run_ours(args, wl, world, rank, local):
                    "topk": wl.topk, "Hq": wl.Hq, "dc": wl.dc, "dr": wl.dr,
                    "l2": f"{len(copies)} rotating state copies, each larger than L2",
                    "parallelism": f"dp{world} (independent batches per rank)"},
-        "indexer_gscores_per_s": gscores,
+        # the scorer kernel's own rate (cached tokens scored per second), and the
+        # same count over the whole step
+        "indexer_gscores_per_s": wl.B * wl.T / t_score / 1e9,
+        "indexer_gscores_roofline": peak * 1e9 / (wl.D + 4) / 1e9,
+        "step_gscores_per_s": gscores,
         "step_roofline": {"bytes": step_bytes, "achieved_gbs": step_bytes / (ms_per_step * 1e-3)
                           / 1e9, "frac": step_bytes / (ms_per_step * 1e-3) / 1e9 / peak},
         "roofline": {"kernel": "decode_index_scores", "bound": "hbm", "achieved": achieved,
@@ -418,6 +425,7 @@ def run_ours(args, wl, world, rank, local):
         "gpu_launches": per_step_launches * args.steps,
         "kernels_per_step": per_step_launches, "kernels": kernel_names,
         "stage_us": {k: round(v * 1e6, 2) for k, v in stages.items()},
+        "prefill_scoring": prefill,
         "clocks": clk.summary(),
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -472,7 +480,51 @@ def run_e2e(dsa, wl, copies, args, world):
             "d2h_bytes_per_step": d2h}
 
 
-def measure_fp8_peak(n=8192, iters=20):
+def time_prefill_scoring(dsa, fp8_peak, iters=10):
+    """Indexer scoring of the causal prefill (T = 8192 queries against their own
+    8192 keys, 64 heads x 128, FP8): the FP8 tensor-bound workload.  Algorithmic
+    work = the causal (query, key) pairs only: T(T+1)/2 x H x D x 2 flop.  The
+    inputs are seeded random normals made on the device (performance only)."""
+    wl = workloads.WORKLOADS[3]
+    T, H, D = wl.T, wl.H, wl.D
+    g = torch.Generator(device="cuda").manual_seed(wl.seed(0))
+    q = torch.randn(1, T, H, D, device="cuda", generator=g)
+    w = torch.randn(1, T, H, device="cuda", generator=g)
+    keys = torch.randn(1, T, D, device="cuda", generator=g)
+    q_fp8 = torch.empty(1, T, H, D, dtype=torch.uint8, device="cuda")
+    q_scale = torch.empty(1, T, H, dtype=torch.float32, device="cuda")
+    k_cache = torch.empty(1, T, D, dtype=torch.uint8, device="cuda")
+    k_scale = torch.empty(1, T, dtype=torch.float32, device="cuda")
+    dsa.dsa_indexer_quant(q, q_fp8, q_scale)
+    dsa.dsa_indexer_quant(keys, k_cache, k_scale, n_rows=1, out_row_stride=T * D,
+                          scale_row_stride=T)
+    del q, keys
+    scores = torch.empty(1, T, T, dtype=torch.float32, device="cuda")
+
+    def one():
+        dsa.dsa_index_scores(q_fp8, q_scale, w, k_cache, k_scale, 0, T, wl.softmax_scale_idx,
+                             scores)
+
+    for _ in range(3):
+        one()
+    torch.cuda.synchronize()
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0.record()
+    for _ in range(iters):
+        one()
+    t1.record()
+    t1.synchronize()
+    t = t0.elapsed_time(t1) * 1e-3 / iters
+    flop = T * (T + 1) // 2 * H * D * 2
+    out = {"workload": wl.name, "queries": T, "keys": T, "gflop": flop / 1e9, "us": t * 1e6,
+           "tflops": flop / t / 1e12, "fp8_peak_tflops": fp8_peak, "frac": flop / t / 1e12 / fp8_peak,
+           "peak_kind": "measured in this run: torch._scaled_mm e4m3 8192^3, burst",
+           "note": "causal pairs only; the -inf scores of masked positions are written too"}
+    del scores
+    return out
+
+
+def measure_fp8_peak(n=8192, iters=20, sustained=True):
     """Dense e4m3 GEMM throughput (torch._scaled_mm, N^3, best of `iters`) -- the
     FP8 tensor-core denominator for the prefill scorer's roofline."""
     a = torch.randn(n, n, device="cuda").to(torch.float8_e4m3fn)
@@ -489,6 +541,8 @@ def measure_fp8_peak(n=8192, iters=20):
         t1.record()
         t1.synchronize()
         best = min(best, t0.elapsed_time(t1) * 1e-3)
+    if not sustained:
+        return {"fp8_e4m3_tflops": 2 * n ** 3 / best / 1e12, "n": n}
     with ClockSampler(torch.cuda.current_device()) as clk:
         t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         t0.record()
@@ -516,6 +570,8 @@ def main(argv=None):
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", type=int, default=4)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-prefill", action="store_true",
+                    help="skip the prefill scoring measurement")
     ap.add_argument("--fp8-peak", action="store_true",
                     help="measure the dense FP8 GEMM peak and exit")
     ap.add_argument("--copies", type=int, default=N_COPIES,

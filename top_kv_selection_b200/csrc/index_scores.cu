@@ -54,7 +54,7 @@ struct ScoreArgs {
     int64_t t_max;
     int64_t start_pos;
     int64_t T;
-    int S, H, NH, chunks;
+    int B, S, H, NH, chunks;
     uint32_t tmem_cols;
     float head_scale, softmax_scale;
     int *err;
@@ -184,9 +184,12 @@ score_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const ScoreArgs a) {
     float *knew_scale = reinterpret_cast<float *>(tmem_holder + 2);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int64_t row = blockIdx.x / a.chunks;
-    const int chunk = blockIdx.x - (int)(row * a.chunks);
-    const int64_t b = row / a.S, s = row - b * a.S;
+    // causal rows are taken longest first (query s = S-1 of every sequence,
+    // then S-2, ...), so the short rows fill the last wave
+    const int64_t ri = blockIdx.x / a.chunks;
+    const int chunk = blockIdx.x - (int)(ri * a.chunks);
+    const int64_t b = ri % a.B, s = a.S - 1 - ri / a.B;
+    const int64_t row = b * a.S + s;
     const int64_t limit = a.start_pos + s;
     const int64_t n_vis = a.T < limit + 1 ? a.T : limit + 1;
     const int64_t n_tiles = (n_vis + kTile - 1) / kTile;
@@ -377,6 +380,7 @@ dsa_status launch_tc(ScoreArgs a, const uint8_t *k_cache, int B, int S, int64_t 
         return DSA_ERR_CUDA;
     a.start_pos = start_pos;
     a.T = T;
+    a.B = B;
     a.S = S;
     a.NH = (a.H + 15) / 16 * 16;
     a.tmem_cols = pow2_cols(kAcc * a.NH);
