@@ -572,6 +572,8 @@ def main(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-prefill", action="store_true",
                     help="skip the prefill scoring measurement")
+    ap.add_argument("--prefill-only", action="store_true",
+                    help="only time the prefill scoring (T = 8192 causal) and exit")
     ap.add_argument("--fp8-peak", action="store_true",
                     help="measure the dense FP8 GEMM peak and exit")
     ap.add_argument("--copies", type=int, default=N_COPIES,
@@ -579,6 +581,13 @@ def main(argv=None):
     args = ap.parse_args(argv)
     if args.fp8_peak:
         print(json.dumps(measure_fp8_peak()), flush=True)
+        return
+    if args.prefill_only:
+        import __graft_entry__
+        __graft_entry__._builder().build()
+        import top_kv_selection_b200 as dsa
+        print(json.dumps(time_prefill_scoring(dsa, measure_fp8_peak(sustained=False)["fp8_e4m3_tflops"],
+                                              iters=max(1, args.steps))), flush=True)
         return
     wl = workloads.WORKLOADS[args.workload]
     if wl.mode != "decode":

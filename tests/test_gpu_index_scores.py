@@ -102,3 +102,20 @@ def test_decode_index_scores_matches_oracle(dsa, cfg, B, T, t_max, H):
         ref = oracle.index_scores(qf[None, None], qs[None, None], s["w"].numpy()[None, None],
                                   kf[None], ks[None], T - 1, T, wl.softmax_scale_idx)
         assert_scores_close(scores[b:b + 1].cpu().numpy()[:, None], ref)
+
+
+@pytest.mark.parametrize("B,S,H,D,T,sp,rows", [
+    (1, 702, 64, 128, 702, 0, (0, 1, 3, 4, 127, 128, 351, 697, 700, 701)),   # ragged last group
+    (2, 1195, 4, 64, 1195, 0, (0, 15, 16, 600, 1183, 1184, 1194)),          # 16 rows per group
+    (1, 600, 64, 128, 1000, 400, (0, 3, 4, 199, 599)),                      # chunk on a cache
+])
+def test_prefill_groups_match_oracle(dsa, B, S, H, D, T, sp, rows):
+    """Enough causal query rows for the grouped prefill scorer (several rows of
+    one sequence per CTA, the key tile shared); rows compared one by one."""
+    qf, qs, w, kf, ks = _quantised_case(B, S, H, D, T, seed=S + H)
+    sm = D ** -0.5
+    got = _run(dsa, qf, qs, w, kf, ks, sp, T, sm)
+    for s in rows:
+        ref = oracle.index_scores(qf[:, s:s + 1], qs[:, s:s + 1], w[:, s:s + 1], kf, ks, sp + s, T,
+                                  sm)
+        assert_scores_close(got[:, s:s + 1], ref)
