@@ -411,11 +411,17 @@ dsa_status launch_tc(ScoreArgs a, const uint8_t *k_cache, int B, int S, int64_t 
 //   warp 1      TMEM + tcgen05.mma kind::f8f6f4, M = 128 tokens,
 //               N = G * NH <= 256, into a double-buffered 2 x 256-column
 //               accumulator;
-//   warps 2..9  epilogue: warp w reads TMEM lane quarter w % 4 (its tokens)
-//               and the rows of half (w - 2) / 4 of the group, writing each
-//               row's causally masked score k_scale * sum_h w'_h ReLU(dot_h).
+//   warps 2..17 epilogue: warp w reads TMEM lane quarter w % 4 (its tokens)
+//               and the 64-column slice (w - 2) / 4 of the accumulator (64 / NH
+//               whole rows), writing each row's causally masked score
+//               k_scale * sum_h w'_h ReLU(dot_h); the weighted sum uses packed
+//               two-lane FMAs.
 // Groups are taken longest first (the last group of every sequence first).
-constexpr int kGThreads = 320;
+// The epilogue is CUDA-core bound at about the rate the FP8 MMA needs: per
+// 128-token tile, 128 x 256 (token, head, row) terms of one max and half a
+// packed FMA each.
+constexpr int kGEpiWarps = 16;
+constexpr int kGThreads = 64 + 32 * kGEpiWarps;
 constexpr int kGCols = 256;              // accumulator columns per buffer
 
 struct GroupArgs {
@@ -436,9 +442,12 @@ __host__ __device__ constexpr size_t group_smem_bytes() {
            (2 * kStages + 2 * kAcc + 1) * sizeof(uint64_t) + 16;
 }
 
-template <int D>
+template <int D, int NH>
 __global__ void __launch_bounds__(kGThreads, 1)
 score_group_kernel(const __grid_constant__ CUtensorMap tmap_k, const GroupArgs a) {
+    static_assert(NH == 16 || NH == 32 || NH == 64, "whole rows per 64-column slice");
+    constexpr int G = kGCols / NH;       // rows per group
+    constexpr int RS = 64 / NH;          // rows per epilogue slice
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -455,12 +464,12 @@ score_group_kernel(const __grid_constant__ CUtensorMap tmap_k, const GroupArgs a
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int64_t b = blockIdx.x % a.B;
-    const int64_t s0 = (int64_t)(a.n_groups - 1 - blockIdx.x / a.B) * a.G;
-    const int g_rows = a.S - s0 < a.G ? (int)(a.S - s0) : a.G;   // rows of this group
+    const int64_t s0 = (int64_t)(a.n_groups - 1 - blockIdx.x / a.B) * G;
+    const int g_rows = a.S - s0 < G ? (int)(a.S - s0) : G;       // rows of this group
     const int64_t last = a.start_pos + s0 + g_rows - 1;          // its longest row's last key
     const int64_t n_vis = a.T < last + 1 ? a.T : last + 1;
     const int n_tiles = (int)((n_vis + kTile - 1) / kTile);
-    const int N = a.G * a.NH;
+    constexpr int N = G * NH;
 
     // every row's scores beyond the group's last key tile are masked
     for (int r = 0; r < g_rows; r++) {
@@ -476,9 +485,9 @@ score_group_kernel(const __grid_constant__ CUtensorMap tmap_k, const GroupArgs a
         }
         for (int i = 0; i < kAcc; i++) {
             tc::mbar_init(&accf[i], 1);
-            tc::mbar_init(&acce[i], 8 * 32);
+            tc::mbar_init(&acce[i], kGEpiWarps * 32);
         }
-        tc::mbar_init(q_ready, 8 * 32);
+        tc::mbar_init(q_ready, kGEpiWarps * 32);
         *abort = 0;
         tc::fence_mbar_init();
         tc::tma_prefetch_desc(&tmap_k);
@@ -534,21 +543,21 @@ score_group_kernel(const __grid_constant__ CUtensorMap tmap_k, const GroupArgs a
     } else {
         // query operand: operand row r * NH + h holds row s0 + r, head h (zeros
         // for padded heads and rows past S), K-major and swizzled
-        const int t = threadIdx.x - 64;                      // 0..255
+        const int t = threadIdx.x - 64;                      // 0 .. 32 * kGEpiWarps - 1
         constexpr int kChunks = D / 16;
-        for (int i = t; i < kGCols * kChunks; i += 256) {
+        for (int i = t; i < kGCols * kChunks; i += 32 * kGEpiWarps) {
             const int orow = i / kChunks, c = i - orow * kChunks;
-            const int r = orow / a.NH, h = orow - r * a.NH;
+            const int r = orow / NH, h = orow - r * NH;
             uint4 v = make_uint4(0, 0, 0, 0);
-            if (orow < N && r < g_rows && h < a.H)
+            if (r < g_rows && h < a.H)
                 v = *reinterpret_cast<const uint4 *>(a.q_fp8 + ((b * a.S + s0 + r) * a.H + h) * D +
                                                      c * 16);
             *reinterpret_cast<uint4 *>(sq + orow * D + KSwizzle<D>::chunk(orow, c) * 16) = v;
         }
-        {
+        if (t < kGCols) {
             float x = 0.f;
-            const int r = t / a.NH, h = t - r * a.NH;
-            if (t < N && r < g_rows && h < a.H) {
+            const int r = t / NH, h = t - r * NH;
+            if (r < g_rows && h < a.H) {
                 const int64_t qi = (b * a.S + s0 + r) * a.H + h;
                 x = __fmul_rn(a.w[qi], a.head_scale);
                 x = __fmul_rn(x, a.q_scale[qi]);
@@ -557,12 +566,10 @@ score_group_kernel(const __grid_constant__ CUtensorMap tmap_k, const GroupArgs a
             wf[t] = x;
         }
         tc::fence_proxy_async_smem();
-        asm volatile("bar.sync 1, 256;" ::: "memory");
+        asm volatile("bar.sync 1, %0;" ::"n"(32 * kGEpiWarps) : "memory");
         tc::mbar_arrive(q_ready);
 
-        const int quarter = warp & 3, rh = (warp - 2) >> 2;
-        const int r_lo = rh == 0 ? 0 : (a.G + 1) / 2;
-        const int r_hi = rh == 0 ? (a.G + 1) / 2 : a.G;
+        const int quarter = warp & 3, slice = (warp - 2) >> 2;   // tokens, 64 columns
         const int tok = quarter * 32 + lane;
         const uint32_t lane_addr = (uint32_t)(quarter * 32) << 16;
         const float *ks_row = a.k_scale + b * a.t_max;
@@ -571,6 +578,7 @@ score_group_kernel(const __grid_constant__ CUtensorMap tmap_k, const GroupArgs a
             return ii < n_tiles && tt < n_vis ? __ldg(ks_row + tt) : 0.f;
         };
         float ks0 = load_ks(0), ks1 = load_ks(1), ks2 = load_ks(2);
+        const float4 *w4 = reinterpret_cast<const float4 *>(wf + slice * 64);
         for (int i = 0; i < n_tiles; i++) {
             const int ac = i % kAcc;
             const int64_t tp = (int64_t)i * kTile + tok;
@@ -580,38 +588,38 @@ score_group_kernel(const __grid_constant__ CUtensorMap tmap_k, const GroupArgs a
             ks2 = load_ks(i + 3);
             if (!tc::mbar_wait(&accf[ac], (uint32_t)(i / kAcc) & 1u, a.err, abort)) break;
             tc::tc_fence_after();
-            for (int r = r_lo; r < r_hi; r++) {
-                const uint32_t taddr = tmem_base + lane_addr + (uint32_t)(ac * kGCols + r * a.NH);
-                float acc4[4] = {0.f, 0.f, 0.f, 0.f};
-                for (int c0 = 0; c0 < a.NH; c0 += 64) {
-                    uint32_t v[4][16];
+            uint32_t v[64];
+            const uint32_t taddr = tmem_base + lane_addr + (uint32_t)(ac * kGCols + slice * 64);
 #pragma unroll
-                    for (int j = 0; j < 4; j++)
-                        if (c0 + 16 * j < a.NH) tc::tmem_ld16(taddr + c0 + 16 * j, v[j]);
-                    tc::tmem_wait_ld();
+            for (int j = 0; j < 4; j++)
+                tc::tmem_ld16(taddr + 16 * j, *reinterpret_cast<uint32_t(*)[16]>(v + 16 * j));
+            tc::tmem_wait_ld();
+            tc::tc_fence_before();
+            tc::mbar_arrive(&acce[ac]);          // the values are in registers
 #pragma unroll
-                    for (int j = 0; j < 4; j++) {
-                        if (c0 + 16 * j >= a.NH) break;
-                        const float4 *w4 = reinterpret_cast<const float4 *>(wf + r * a.NH + c0 + 16 * j);
+            for (int rl = 0; rl < RS; rl++) {
+                float2 acc01 = make_float2(0.f, 0.f), acc23 = make_float2(0.f, 0.f);
 #pragma unroll
-                        for (int e = 0; e < 4; e++) {
-                            const float4 wv = w4[e];
-                            acc4[0] = fmaf(wv.x, fmaxf(__uint_as_float(v[j][4 * e + 0]), 0.f), acc4[0]);
-                            acc4[1] = fmaf(wv.y, fmaxf(__uint_as_float(v[j][4 * e + 1]), 0.f), acc4[1]);
-                            acc4[2] = fmaf(wv.z, fmaxf(__uint_as_float(v[j][4 * e + 2]), 0.f), acc4[2]);
-                            acc4[3] = fmaf(wv.w, fmaxf(__uint_as_float(v[j][4 * e + 3]), 0.f), acc4[3]);
-                        }
-                    }
+                for (int h = 0; h < NH; h += 4) {
+                    const float4 wv = w4[(rl * NH + h) / 4];
+                    const int e = rl * NH + h;
+                    acc01 = __ffma2_rn(make_float2(wv.x, wv.y),
+                                       make_float2(fmaxf(__uint_as_float(v[e]), 0.f),
+                                                   fmaxf(__uint_as_float(v[e + 1]), 0.f)),
+                                       acc01);
+                    acc23 = __ffma2_rn(make_float2(wv.z, wv.w),
+                                       make_float2(fmaxf(__uint_as_float(v[e + 2]), 0.f),
+                                                   fmaxf(__uint_as_float(v[e + 3]), 0.f)),
+                                       acc23);
                 }
+                const int r = slice * RS + rl;
                 if (r < g_rows && tp < a.T) {
                     const int64_t srow = s0 + r;
-                    const int64_t vis = a.start_pos + srow + 1;
-                    const float acc = (acc4[0] + acc4[1]) + (acc4[2] + acc4[3]);
-                    a.scores[(b * a.S + srow) * a.T + tp] = tp < vis ? ks * acc : -INFINITY;
+                    const float acc = (acc01.x + acc01.y) + (acc23.x + acc23.y);
+                    a.scores[(b * a.S + srow) * a.T + tp] =
+                        tp < a.start_pos + srow + 1 ? ks * acc : -INFINITY;
                 }
             }
-            tc::tc_fence_before();
-            tc::mbar_arrive(&acce[ac]);
         }
     }
 
@@ -623,7 +631,7 @@ score_group_kernel(const __grid_constant__ CUtensorMap tmap_k, const GroupArgs a
     }
 }
 
-template <int D>
+template <int D, int NH>
 dsa_status launch_group(GroupArgs g, const uint8_t *k_cache, cudaStream_t stream) {
     CUtensorMap tmap;
     const uint64_t dims[3] = {(uint64_t)D, (uint64_t)g.t_max, (uint64_t)g.B};
@@ -634,19 +642,20 @@ dsa_status launch_group(GroupArgs g, const uint8_t *k_cache, cudaStream_t stream
     if (!encode_tmap(&tmap, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, k_cache, dims, strides, box, swz))
         return DSA_ERR_CUDA;
     const size_t smem = group_smem_bytes<D>();
-    if (cudaFuncSetAttribute(score_group_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)smem) != cudaSuccess)
+    if (cudaFuncSetAttribute(score_group_kernel<D, NH>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
         return DSA_ERR_CUDA;
-    score_group_kernel<D><<<(unsigned)((int64_t)g.B * g.n_groups), kGThreads, smem, stream>>>(tmap, g);
+    score_group_kernel<D, NH><<<(unsigned)((int64_t)g.B * g.n_groups), kGThreads, smem, stream>>>(
+        tmap, g);
     return launch_status();
 }
 
 // Rows per group of the prefill scorer for H heads, or 0 when one query row
-// per CTA with the key range split across CTAs is the better plan (too few
-// groups to fill the SMs, or more than 128 padded heads).
+// per CTA with the key range split across CTAs is the plan (too few groups to
+// fill the SMs, or padded heads other than 16, 32 or 64).
 int group_rows(int B, int S, int H) {
     const int NH = (H + 15) / 16 * 16;
-    if (NH > 128) return 0;
+    if (NH != 16 && NH != 32 && NH != 64) return 0;
     const int G = kGCols / NH;
     const int64_t groups = (int64_t)B * ((S + G - 1) / G);
     return groups >= num_sms() ? G : 0;
@@ -687,7 +696,14 @@ dsa_status launch_index_scores(const uint8_t *q_fp8, const float *q_scale, const
         g.head_scale = (float)(1.0 / sqrt((double)H));
         g.softmax_scale = softmax_scale;
         g.err = device_error_word();
-        return D == 128 ? launch_group<128>(g, k_cache, stream) : launch_group<64>(g, k_cache, stream);
+        switch (g.NH * 1000 + D) {
+            case 16128: return launch_group<128, 16>(g, k_cache, stream);
+            case 32128: return launch_group<128, 32>(g, k_cache, stream);
+            case 64128: return launch_group<128, 64>(g, k_cache, stream);
+            case 16064: return launch_group<64, 16>(g, k_cache, stream);
+            case 32064: return launch_group<64, 32>(g, k_cache, stream);
+            default: return launch_group<64, 64>(g, k_cache, stream);
+        }
     }
     return D == 128 ? launch_tc<128, false>(a, k_cache, B, S, start_pos, T, stream)
                     : launch_tc<64, false>(a, k_cache, B, S, start_pos, T, stream);
