@@ -37,8 +37,9 @@ N_COPIES = 3            # rotating device copies of the decode state (each > L2)
 # Source files of the dominant kernel (the indexer scorer); the committed ncu
 # summary records their hash, so its DRAM traffic is reported only while the
 # kernel is unchanged.
-SCORER_SOURCES = ("top_kv_selection_b200/csrc/index_scores.cu", "top_kv_selection_b200/csrc/quant.cuh",
-                  "top_kv_selection_b200/csrc/tc_ptx.cuh", "top_kv_selection_b200/csrc/common.cuh")
+SCORER_SOURCES = ("top_kv_selection_b200/csrc/index_scores.cu", "top_kv_selection_b200/csrc/scorer.cuh",
+                  "top_kv_selection_b200/csrc/quant.cuh", "top_kv_selection_b200/csrc/tc_ptx.cuh",
+                  "top_kv_selection_b200/csrc/common.cuh")
 SCORER_PROFILE = "profiles/index_scores_decode_B8_T131072.md"
 
 

@@ -4,13 +4,13 @@
  *
  * The path (lightning indexer, top-k token selection, sparse latent attention)
  * follows these pages:
- *   "DeepSeek-V3.2-Exp - Split indexer heads": the Indexer.forward excerpt
- *       (inference/model.py, lines 457-487): rotate_activation, act_quant,
+ *   "DeepSeek-V3.2-Exp - Split indexer heads": the Indexer.forward excerpt:
+ *       rotate_activation, act_quant,
  *       the key-cache write, the weight fold, fp8_index, the additive mask and
  *       topk(min(index_topk, end_pos)).
  *   "DeepSeek-V3.2-Exp - Causal mask": Transformer.forward (mask =
  *       full(-inf).triu_(1) when seqlen > 1) and the MLA prefill excerpt
- *       (model.py 574-589: index_mask = full(-inf).scatter_(topk, 0) + mask).
+ *       (index_mask = full(-inf).scatter_(topk, 0) + mask).
  *   "DeepSeek Sparse Attention, one decode step in one layer (V3.2 sizes)"
  *       diagram: I(t,s) = sum_j w_j ReLU(q_j . k_s), k = 2048, core attention
  *       in MQA mode over the gathered latents, each latent row key and value.

@@ -8,12 +8,12 @@
  * header, table or constant with the CUDA library; neither includes the other.
  *
  * Sources (web pages the method is taken from):
- *   [V32-IDX]  "DeepSeek-V3.2-Exp - Split indexer heads", Indexer.forward excerpt
- *              (inference/model.py lines 457-487): rotate_activation, act_quant,
+ *   [V32-IDX]  "DeepSeek-V3.2-Exp - Split indexer heads", Indexer.forward excerpt:
+ *              rotate_activation, act_quant,
  *              k cache write, weight fold, fp8_index, additive mask, topk.
- *   [V32-MASK] "DeepSeek-V3.2-Exp - Causal mask", Transformer.forward excerpt
- *              (model.py 880-908): mask = full(-inf).triu_(1) if seqlen > 1.
- *   [V32-MLA]  same page, MLA prefill excerpt (model.py 574-589): index_mask =
+ *   [V32-MASK] "DeepSeek-V3.2-Exp - Causal mask", Transformer.forward excerpt:
+ *              mask = full(-inf).triu_(1) if seqlen > 1.
+ *   [V32-MLA]  same page, MLA prefill excerpt: index_mask =
  *              full(-inf).scatter_(topk, 0) + mask, softmax, value mix.
  *   [DIAG]     "DeepSeek Sparse Attention, one decode step in one layer (V3.2
  *              sizes)" diagram: I(t,s) = sum_j w_j ReLU(q_j . k_s), k = 2048,
