@@ -21,7 +21,8 @@
 //            atomics rarely collide and the threshold bin is small), merged
 //            into CTA 0 with distributed shared-memory atomics;
 //   then the threshold-bin candidates' keys are gathered into CTA 0, which
-//   finds the exact k-th key alone (11 + 11 + 10-bit radix passes); if there
+//   finds the exact k-th key alone (by ranking every key directly when there
+//   are at most 1024 of them, else 11 + 11 + 10-bit radix passes); if there
 //   are too many candidates, the radix passes run cluster-wide instead.
 // Then every CTA counts its x > tau and x == tau, the counts are exchanged,
 // and each CTA writes its selected positions at its offset in position order.
@@ -231,6 +232,7 @@ topk_cluster_kernel(const float *__restrict__ scores, int S, int64_t T, int64_t 
     __shared__ ClusterCtl ctl;
     __shared__ unsigned s_bin, s_rank;
     __shared__ uint32_t s_tau;
+    __shared__ int s_ncand;
     __shared__ float s_lo, s_hi;
 
     const int64_t t0 = (int64_t)p * L;
@@ -345,19 +347,18 @@ topk_cluster_kernel(const float *__restrict__ scores, int S, int64_t T, int64_t 
     const int tb = (int)ctl.bin;
     unsigned rank = ctl.rank;
 
-    // threshold-bin candidates, in position order: thread i scans the
-    // contiguous segment [i*seg, (i+1)*seg) of the slice
+    // thread i owns the contiguous segment [i*seg, (i+1)*seg) of the slice
     const int seg = (len + kThreads - 1) / kThreads;
     const int s0 = threadIdx.x * seg < len ? threadIdx.x * seg : len;
     const int s1 = s0 + seg < len ? s0 + seg : len;
-    int n_cand;
-    {
-        int c = 0;
-        for (int i = s0; i < s1; i++) c += linear_bin(sv[pad(i)], g_lo, scale) == tb;
-        int pos = block_scan_int(c, itmp, &n_cand);
-        for (int i = s0; i < s1; i++)
-            if (linear_bin(sv[pad(i)], g_lo, scale) == tb) cand[pos++] = (uint16_t)i;
-    }
+    // threshold-bin candidates (slot indices, in any order: only their keys
+    // matter), appended in one pass
+    if (threadIdx.x == 0) s_ncand = 0;
+    __syncthreads();
+    for (int i = s0; i < s1; i++)
+        if (linear_bin(sv[pad(i)], g_lo, scale) == tb) cand[atomicAdd(&s_ncand, 1)] = (uint16_t)i;
+    __syncthreads();
+    const int n_cand = s_ncand;
     if (threadIdx.x == 0) ctl.n_cand = n_cand;
     cl.sync();                                                            // (4)
     int cand_off = 0, E = 0;
@@ -376,7 +377,28 @@ topk_cluster_kernel(const float *__restrict__ scores, int S, int64_t T, int64_t 
         cl.sync();                                                        // (5)
         if (p == 0) {
             unsigned rk;
-            cta_select_keys(gath, E, rank, hist, scan_tmp, &s_bin, &s_rank, &s_tau, &rk);
+            if (E <= kThreads) {
+                // few candidates: rank each key directly (keys larger, keys equal);
+                // the key whose range covers `rank` is tau, and rank - #larger of
+                // the keys equal to it are taken (every tau-equal thread agrees)
+                if ((int)threadIdx.x < E) {
+                    const uint32_t kj = gath[threadIdx.x];
+                    unsigned gt = 0, eq = 0;
+                    for (int i = 0; i < E; i++) {
+                        const uint32_t ki = gath[i];
+                        gt += ki > kj;
+                        eq += ki == kj;
+                    }
+                    if (gt < rank && gt + eq >= rank) {
+                        s_tau = kj;
+                        s_rank = rank - gt;
+                    }
+                }
+                __syncthreads();
+                rk = s_rank;
+            } else {
+                cta_select_keys(gath, E, rank, hist, scan_tmp, &s_bin, &s_rank, &s_tau, &rk);
+            }
             if (threadIdx.x < CN) {
                 ClusterCtl *rc = cl.map_shared_rank(&ctl, (int)threadIdx.x);
                 rc->bin = s_tau;
