@@ -355,8 +355,12 @@ topk_cluster_kernel(const float *__restrict__ scores, int S, int64_t T, int64_t 
     // matter), appended in one pass
     if (threadIdx.x == 0) s_ncand = 0;
     __syncthreads();
-    for (int i = s0; i < s1; i++)
-        if (linear_bin(sv[pad(i)], g_lo, scale) == tb) cand[atomicAdd(&s_ncand, 1)] = (uint16_t)i;
+    int above = 0;                        // this thread's values in bins above the threshold bin
+    for (int i = s0; i < s1; i++) {
+        const int bin = linear_bin(sv[pad(i)], g_lo, scale);
+        above += bin > tb;
+        if (bin == tb) cand[atomicAdd(&s_ncand, 1)] = (uint16_t)i;
+    }
     __syncthreads();
     const int n_cand = s_ncand;
     if (threadIdx.x == 0) ctl.n_cand = n_cand;
@@ -450,13 +454,21 @@ topk_cluster_kernel(const float *__restrict__ scores, int S, int64_t T, int64_t 
         q = (int)rank;
     }
 
-    // counts, exchanged through the cluster, give each CTA its output offset
-    int gt = 0, eq = 0;
-    for (int i = s0; i < s1; i++) {
-        const uint32_t key = score_key(sv[pad(i)]);
-        gt += key > tau;
-        eq += key == tau;
+    // counts, exchanged through the cluster, give each CTA its output offset.
+    // Every value above the threshold bin is > tau; of the candidates, each
+    // adds to its owner thread's count of keys > tau or == tau.
+    unsigned *t_gt = hist, *t_eq = hist + kThreads;        // hist is free again
+    t_gt[threadIdx.x] = 0;
+    t_eq[threadIdx.x] = 0;
+    __syncthreads();
+    for (int j = threadIdx.x; j < n_cand; j += kThreads) {
+        const int slot = cand[j];
+        const uint32_t key = score_key(sv[pad(slot)]);
+        if (key > tau) atomicAdd(&t_gt[slot / seg], 1u);
+        else if (key == tau) atomicAdd(&t_eq[slot / seg], 1u);
     }
+    __syncthreads();
+    const int gt = above + (int)t_gt[threadIdx.x], eq = (int)t_eq[threadIdx.x];
     int cta_gt, cta_eq;
     block_scan_int(gt, itmp, &cta_gt);
     const int eq_before_me = block_scan_int(eq, itmp, &cta_eq);
