@@ -150,6 +150,8 @@ sparse_mla_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const MlaArgs a) 
     tc::cluster_sync_all();          // both CTAs' barriers exist before any remote arrive
     tc::tc_fence_after();
     const uint32_t tmem = *tmem_holder;
+    // a kernel launched after this one (the split combine) may start its set-up
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     if (threadIdx.x == 0) {
         // this CTA's five 64-column blocks of the query, staged in ring
         // stages 2..3 until the softmax warps have moved them to TMEM
@@ -159,6 +161,10 @@ sparse_mla_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const MlaArgs a) 
                             (int)(row * kHq), q_full);
     }
 
+    // The selections come from the preceding kernel (the top-k): wait for it
+    // to complete (a no-op without a programmatic launch), then read them with
+    // plain loads, which stay after the wait.
+    asm volatile("griddepcontrol.wait;" ::: "memory");
     // valid selections of this row, in slot order (the same list in both CTAs):
     // threads 0..255 take 8 consecutive slots each, one block-wide scan
     constexpr int kPer = kMaxSel / 256;
@@ -167,7 +173,7 @@ sparse_mla_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const MlaArgs a) 
 #pragma unroll
     for (int e = 0; e < kPer; e++) {
         const int j = threadIdx.x * kPer + e;
-        int32_t t = threadIdx.x < 256 && j < a.k ? __ldg(a.idx + row * a.k + j) : -1;
+        int32_t t = threadIdx.x < 256 && j < a.k ? a.idx[row * a.k + j] : -1;
         if (t >= 0 && (int64_t)t <= limit) {
             if ((int64_t)t >= a.t_max) {
                 record_error(a.err, DSA_ERR_DEVICE);
@@ -478,8 +484,10 @@ sparse_mla_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const MlaArgs a) 
 // output columns of one head, consecutive threads consecutive heads (coalesced).
 constexpr int kCombineQuads = 2;                         // column quads per block
 __global__ void __launch_bounds__(kHq * kCombineQuads)
-sparse_mla_combine_kernel(const float *__restrict__ part_o, const float2 *__restrict__ part_ml,
-                          int splits, __nv_bfloat16 *__restrict__ out, float *__restrict__ lse) {
+sparse_mla_combine_kernel(const float *part_o, const float2 *part_ml, int splits,
+                          __nv_bfloat16 *__restrict__ out, float *__restrict__ lse) {
+    // the partials come from the preceding kernel: wait for it (plain loads below)
+    asm volatile("griddepcontrol.wait;" ::: "memory");
     constexpr int groups = (kDh / 4) / kCombineQuads;
     const int64_t rh = blockIdx.x / groups;                 // row * 2 + half
     const int64_t row = rh >> 1;
@@ -587,19 +595,32 @@ dsa_status launch_sparse_mla_tc(const void *q, const void *kv, int64_t t_max, co
     cfg.blockDim = dim3(kThreads);
     cfg.dynamicSmemBytes = kSmemBytes;
     cfg.stream = stream;
-    cudaLaunchAttribute attr[1];
+    // programmatic launch: the kernel's set-up overlaps the preceding kernel's
+    // tail; it waits for that kernel before reading the selections
+    cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeClusterDimension;
     attr[0].val.clusterDim.x = 2;
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
-    cfg.numAttrs = 1;
+    cfg.numAttrs = 2;
     if (cudaLaunchKernelEx(&cfg, sparse_mla_tc_kernel, tm_q, a) != cudaSuccess) return DSA_ERR_CUDA;
     dsa_status st = launch_status();
     if (st != DSA_OK || a.splits == 1) return st;
-    sparse_mla_combine_kernel<<<(unsigned)(rows * 2 * ((kDh / 4) / kCombineQuads)),
-                                kHq * kCombineQuads, 0, stream>>>(a.part_o, a.part_ml, a.splits,
-                                                                  a.out, lse);
+    cudaLaunchConfig_t ccfg = {};
+    ccfg.gridDim = dim3((unsigned)(rows * 2 * ((kDh / 4) / kCombineQuads)));
+    ccfg.blockDim = dim3(kHq * kCombineQuads);
+    ccfg.stream = stream;
+    cudaLaunchAttribute cattr[1];
+    cattr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    cattr[0].val.programmaticStreamSerializationAllowed = 1;
+    ccfg.attrs = cattr;
+    ccfg.numAttrs = 1;
+    if (cudaLaunchKernelEx(&ccfg, sparse_mla_combine_kernel, (const float *)a.part_o,
+                           (const float2 *)a.part_ml, a.splits, a.out, lse) != cudaSuccess)
+        return DSA_ERR_CUDA;
     return launch_status();
 }
 

@@ -206,6 +206,9 @@ constexpr int kGather = 8192;      // candidates CTA 0 can select alone
 __global__ void __launch_bounds__(kThreads, 1)
 topk_cluster_kernel(const float *__restrict__ scores, int S, int64_t T, int64_t start_pos, int K,
                     int L, int32_t *__restrict__ idx) {
+    // a kernel launched after this one (the sparse attention) may start its
+    // set-up now; it reads the selections only after waiting for this grid
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     cg::cluster_group cl = cg::this_cluster();
     const int CN = (int)cl.num_blocks();
     const int p = (int)cl.block_rank();
