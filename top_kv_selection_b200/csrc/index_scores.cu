@@ -185,6 +185,9 @@ score_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const ScoreArgs a) {
     // decode: this CTA appends the new key if its last tile holds position T-1
     const bool append = kRaw && n_my > 0 && tile_hi == n_tiles;
 
+    // a kernel launched after this one (the top-k) may be scheduled now; it
+    // waits for this grid before reading the scores
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     // causally masked positions of this row (prefill only), shared by the chunks
     for (int64_t t = n_vis + (int64_t)chunk * kThreads + threadIdx.x; t < a.T;
          t += (int64_t)a.chunks * kThreads)

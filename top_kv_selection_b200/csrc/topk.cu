@@ -204,7 +204,7 @@ __device__ void cta_select_keys(const uint32_t *keys, int n, unsigned rank, unsi
 constexpr int kGather = 8192;      // candidates CTA 0 can select alone
 
 __global__ void __launch_bounds__(kThreads, 1)
-topk_cluster_kernel(const float *__restrict__ scores, int S, int64_t T, int64_t start_pos, int K,
+topk_cluster_kernel(const float *scores, int S, int64_t T, int64_t start_pos, int K,
                     int L, int32_t *__restrict__ idx) {
     // a kernel launched after this one (the sparse attention) may start its
     // set-up now; it reads the selections only after waiting for this grid
@@ -244,6 +244,9 @@ topk_cluster_kernel(const float *__restrict__ scores, int S, int64_t T, int64_t 
     const int len = t1 > t0 ? (int)(t1 - t0) : 0;
     const float *src = scores + row * T + t0;
 
+    // The scores come from the preceding kernel (the scorer): wait for it (a
+    // no-op without a programmatic launch); plain loads stay after the wait.
+    asm volatile("griddepcontrol.wait;" ::: "memory");
     // load the slice, finite min / max; clear the histograms
     // (loads are issued in batches of eight per thread so their latencies overlap)
     float lo = INFINITY, hi = -INFINITY;
@@ -255,7 +258,7 @@ topk_cluster_kernel(const float *__restrict__ scores, int S, int64_t T, int64_t 
 #pragma unroll
             for (int u = 0; u < 8; u++) {
                 const int j = base + u * kThreads + threadIdx.x;
-                v[u] = j < n4 ? __ldg(reinterpret_cast<const float4 *>(src) + j)
+                v[u] = j < n4 ? reinterpret_cast<const float4 *>(src)[j]
                               : make_float4(NAN, NAN, NAN, NAN);
             }
 #pragma unroll
@@ -279,7 +282,7 @@ topk_cluster_kernel(const float *__restrict__ scores, int S, int64_t T, int64_t 
 #pragma unroll
         for (int u = 0; u < 8; u++) {
             const int i = base + u * kThreads + threadIdx.x;
-            v[u] = i < len ? __ldg(src + i) : NAN;
+            v[u] = i < len ? src[i] : NAN;
         }
 #pragma unroll
         for (int u = 0; u < 8; u++) {
@@ -623,13 +626,17 @@ dsa_status launch_topk_select(const float *scores, int B, int S, int64_t T, int6
     cfg.blockDim = dim3(kThreads);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = stream;
-    cudaLaunchAttribute attr[1];
+    cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeClusterDimension;
     attr[0].val.clusterDim.x = (unsigned)cn;
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
+    // programmatic launch: the launch overlaps the preceding kernel's tail; the
+    // kernel waits for that grid before reading the scores
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
-    cfg.numAttrs = 1;
+    cfg.numAttrs = 2;
     if (cudaLaunchKernelEx(&cfg, topk_cluster_kernel, scores, S, T, start_pos, K, L, idx) !=
         cudaSuccess)
         return DSA_ERR_CUDA;
