@@ -49,7 +49,7 @@ constexpr int kHq = 128, kDc = 512, kDr = 64, kDqk = kDc + kDr;
 constexpr int kLB = 5;                          // 64-column blocks held per CTA
 constexpr int kDh = 256;                        // output columns per CTA
 constexpr int kRows = 64;                       // gathered rows per tile (QK N)
-constexpr int kStages = 4;
+constexpr int kStages = 3;
 constexpr int kThreads = 288;               // warp 0 MMA, 1..4 softmax, 5..8 gather
 constexpr int kMaxSel = 2048;                   // selection slots held in shared memory
 // TMEM columns: O (fp32) | S (fp32) | P (bf16 pairs) | Q (bf16 pairs, this CTA's 320)
@@ -62,8 +62,10 @@ constexpr int kRxBytes = kHq * kRows * 4;       // partner's partial logits
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
 
-constexpr size_t kSmemBytes = 1024 + (size_t)kStages * kTileBytes + kRxBytes +
+constexpr size_t kSmemBytes = 1024 + (size_t)kStages * kTileBytes + 2 * kRxBytes +
                               kMaxSel * sizeof(int32_t) + 32 * sizeof(uint64_t) + 64;
+constexpr int kQStage = 1;                       // the query is staged in ring stages 1..2
+static_assert(kQStage + 2 <= kStages, "query staging");
 constexpr int kLag = 1;                          // gather tiles in flight per thread beyond the one issued
 constexpr int kQBlk = kHq * 128;                 // one 64-column block of the query (TMA box)
 
@@ -97,8 +99,10 @@ sparse_mla_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const MlaArgs a) 
     uint8_t *smem = reinterpret_cast<uint8_t *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t *sc = smem;                                      // C tiles
-    float4 *rx = reinterpret_cast<float4 *>(sc + kStages * kTileBytes);   // partner's logits [16][128]
-    int32_t *list = reinterpret_cast<int32_t *>(sc + kStages * kTileBytes + kRxBytes);
+    // this CTA's partial logits to send, and the partner's received: [16][128] float4
+    float4 *tx = reinterpret_cast<float4 *>(sc + kStages * kTileBytes);
+    float4 *rx = tx + kRxBytes / 16;
+    int32_t *list = reinterpret_cast<int32_t *>(sc + kStages * kTileBytes + 2 * kRxBytes);
     uint64_t *bars = reinterpret_cast<uint64_t *>(list + kMaxSel);
     uint64_t *c_full = bars, *c_empty = bars + kStages;
     uint64_t *s_full = bars + 2 * kStages, *s_empty = s_full + 1;
@@ -106,7 +110,7 @@ sparse_mla_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const MlaArgs a) 
     uint64_t *q_ready = pv_done + 1;    // the query is in TMEM
     uint64_t *q_full = q_ready + 1;     // the query's TMA copy (ring stages 2..3) landed
     uint64_t *q_free = q_full + 1;      // ... and has been moved to TMEM
-    uint64_t *rx_full = q_free + 1;     // partner's logits of the current tile landed
+    uint64_t *rx_full = q_free + 1;     // partner's logits of the current tile landed (bytes)
     uint64_t *tx_ok = rx_full + 1;      // partner has read what this CTA sent last
     uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(tx_ok + 1);
     volatile int *abort = reinterpret_cast<volatile int *>(tmem_holder + 1);
@@ -136,8 +140,8 @@ sparse_mla_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const MlaArgs a) 
         tc::mbar_init(q_ready, 128);
         tc::mbar_init(q_full, 1);
         tc::mbar_init(q_free, 128);
-        tc::mbar_init(rx_full, 128);
-        tc::mbar_init(tx_ok, 128);
+        tc::mbar_init(rx_full, 1);
+        tc::mbar_init(tx_ok, 1);
         *abort = 0;
         tc::fence_mbar_init();
         tc::tma_prefetch_desc(&tm_q);
@@ -154,10 +158,10 @@ sparse_mla_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const MlaArgs a) 
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     if (threadIdx.x == 0) {
         // this CTA's five 64-column blocks of the query, staged in ring
-        // stages 2..3 until the softmax warps have moved them to TMEM
+        // stages 1..2 until the softmax warps have moved them to TMEM
         tc::mbar_arrive_expect_tx(q_full, kLB * kQBlk);
         for (int j = 0; j < kLB; j++)
-            tc::tma_load_2d(sc + 2 * kTileBytes + j * kQBlk, &tm_q, (cr * 4 + j) * 64,
+            tc::tma_load_2d(sc + kQStage * kTileBytes + j * kQBlk, &tm_q, (cr * 4 + j) * 64,
                             (int)(row * kHq), q_full);
     }
 
@@ -216,7 +220,7 @@ sparse_mla_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const MlaArgs a) 
     // its staging copy to TMEM, one head per lane, by the softmax warps
     if (is_softmax) {
         if (tc::mbar_wait(q_full, 0, a.err, abort)) {
-            const uint8_t *qs = sc + 2 * kTileBytes;
+            const uint8_t *qs = sc + kQStage * kTileBytes;
 #pragma unroll 1
             for (int c = 0; c < kLB * 8 / 4; c++) {          // 10 x 4 pieces of 16 bytes
                 uint32_t r[16];
@@ -266,7 +270,7 @@ sparse_mla_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const MlaArgs a) 
                 for (; signalled < issued; signalled++) tc::mbar_arrive(&c_full[signalled % kStages]);
                 if (!tc::mbar_wait(&c_empty[st], ph, a.err, abort)) break;
             }
-            if (i == 2 && !tc::mbar_wait(q_free, 0, a.err, abort)) break;   // stages 2..3 held the query
+            if (i == kQStage && !tc::mbar_wait(q_free, 0, a.err, abort)) break;   // the query's staging
             uint8_t *tile = sc + st * kTileBytes;
 #pragma unroll 4
             for (int f = gt; f < kRows * kChunks; f += 128) {
@@ -347,14 +351,23 @@ sparse_mla_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const MlaArgs a) 
         }
     } else {
         // ---- softmax warps
+        // Per tile the 128 threads write this CTA's partial logits to `tx`, and
+        // one thread (the elected) pushes the 32 KB into the partner's `rx` with
+        // a bulk copy counted on the partner's rx_full; after reading `rx` the
+        // elected thread tells the partner (tx_ok) that it may send again,
+        // which also means this CTA's previous copy has landed.
         const uint32_t peer = (uint32_t)(cr ^ 1);
         const uint32_t peer_rx = tc::map_shared_rank(rx, peer);
         const uint32_t peer_rx_full = tc::map_shared_rank(rx_full, peer);
         const uint32_t peer_tx_ok = tc::map_shared_rank(tx_ok, peer);
+        const bool elected = threadIdx.x == 32;
         float m_run = -INFINITY, l = 0.f;
+        // A failed (timed-out) wait only clears `ok`: the thread carries on to the
+        // next named barrier, where all 128 threads leave the loop together.
         bool ok = true;
-        for (int i = 0; i < n_tiles && ok; i++) {
-            if (!tc::mbar_wait(s_full, (uint32_t)i & 1u, a.err, abort)) { ok = false; break; }
+        for (int i = 0; i < n_tiles; i++) {
+            if (elected) tc::mbar_arrive_expect_tx(rx_full, kRxBytes);   // tile i's bytes
+            if (ok && !tc::mbar_wait(s_full, (uint32_t)i & 1u, a.err, abort)) ok = false;
             tc::tc_fence_after();
             uint32_t own[kRows];
 #pragma unroll
@@ -364,19 +377,17 @@ sparse_mla_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const MlaArgs a) 
             tc::tmem_wait_ld();
             tc::tc_fence_before();
             tc::mbar_arrive(s_empty);
-            // exchange the partial logits: the partner must have read the
-            // previous tile's before they are overwritten
-            if (i > 0 && !tc::mbar_wait_cluster(tx_ok, (uint32_t)(i - 1) & 1u, a.err, abort)) {
+            // `tx` may be rewritten once the partner has read tile i-1
+            if (ok && i > 0 && !tc::mbar_wait_cluster(tx_ok, (uint32_t)(i - 1) & 1u, a.err, abort))
                 ok = false;
-                break;
-            }
 #pragma unroll
             for (int q = 0; q < kRows / 4; q++)
-                tc::st_cluster_v4(peer_rx + (uint32_t)((q * kHq + h) * 16),
-                                  __uint_as_float(own[4 * q]), __uint_as_float(own[4 * q + 1]),
-                                  __uint_as_float(own[4 * q + 2]), __uint_as_float(own[4 * q + 3]));
-            tc::mbar_arrive_cluster(peer_rx_full);
-            if (!tc::mbar_wait_cluster(rx_full, (uint32_t)i & 1u, a.err, abort)) { ok = false; break; }
+                tx[q * kHq + h] = make_float4(__uint_as_float(own[4 * q]), __uint_as_float(own[4 * q + 1]),
+                                              __uint_as_float(own[4 * q + 2]), __uint_as_float(own[4 * q + 3]));
+            tc::fence_proxy_async_smem();
+            if (tc::named_barrier_any(1, 128, !ok)) break;
+            if (elected) tc::bulk_copy_to_peer(peer_rx, tx, kRxBytes, peer_rx_full);
+            if (ok && !tc::mbar_wait(rx_full, (uint32_t)i & 1u, a.err, abort)) ok = false;
             const int nv = n_my - i * kRows;
             float sv[kRows];
             float m_tile = -INFINITY;
@@ -392,13 +403,11 @@ sparse_mla_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const MlaArgs a) 
                     m_tile = fmaxf(m_tile, sv[j]);
                 }
             }
-            tc::mbar_arrive_cluster(peer_tx_ok);
+            if (tc::named_barrier_any(1, 128, !ok)) break;      // every thread has read `rx`
+            if (elected) tc::mbar_arrive_cluster(peer_tx_ok);
             // PV(i-1) must be done: it reads P, and O may be rescaled below
             if (i > 0) {
-                if (!tc::mbar_wait(pv_done, (uint32_t)(i - 1) & 1u, a.err, abort)) {
-                    ok = false;
-                    break;
-                }
+                if (ok && !tc::mbar_wait(pv_done, (uint32_t)(i - 1) & 1u, a.err, abort)) ok = false;
                 tc::tc_fence_after();
             }
             if (__any_sync(0xffffffffu, m_tile > m_run + 8.f)) {
