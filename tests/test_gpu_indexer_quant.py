@@ -78,3 +78,18 @@ def test_indexer_quant_prefill_queries_full_size(dsa):
     ref_c, ref_s = oracle.indexer_quant(q[rows].numpy())
     assert np.array_equal(out.cpu().numpy()[rows], ref_c)
     assert np.array_equal(sc.cpu().numpy()[rows], ref_s)
+
+
+def test_indexer_quant_bit_exact_many_vectors(dsa):
+    """200,000 vectors of 128 (25.6 M quotients) over 2^-20 .. 2^20: every code and
+    scale equals the oracle's, which divides with C's correctly rounded division."""
+    n_vec, D = 200_000, 128
+    g = torch.Generator().manual_seed(20)
+    x = torch.randn(n_vec, D, generator=g) * torch.exp2(torch.randint(-20, 21, (n_vec, 1),
+                                                                      generator=g).float())
+    out = torch.empty(n_vec, D, dtype=torch.uint8, device="cuda")
+    sc = torch.empty(n_vec, dtype=torch.float32, device="cuda")
+    dsa.dsa_indexer_quant(x.cuda(), out, sc)
+    ref_c, ref_s = oracle.indexer_quant(x.numpy())
+    assert np.array_equal(sc.cpu().numpy(), ref_s)
+    assert np.array_equal(out.cpu().numpy(), ref_c)

@@ -11,7 +11,8 @@
 // ..., D/2 -- the same dataflow as the plain in-place transform, so the result
 // is bit-identical to it.  Then one multiply by fp32(D^-1/2), a warp max of
 // |x|, scale = max(amax, 1e-4) / 448 and the e4m3 codes of x / scale (round to
-// nearest even, saturate to +-448), both divisions correctly rounded.
+// nearest even, saturate to +-448), both divisions correctly rounded (the
+// per-element one by div_rn_by from the vector's reciprocal).
 #pragma once
 
 #include "common.cuh"
@@ -29,6 +30,17 @@ __device__ __forceinline__ uint32_t e4m3x2_rn_sat(float lo, float hi) {
     uint16_t r;
     asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(hi), "f"(lo));
     return r;
+}
+
+// x / s correctly rounded, given rs = RN(1/s) (one correctly rounded
+// reciprocal per vector): Markstein's FMA correction -- q0 = RN(x * rs),
+// e = x - q0 * s exactly (one FMA), q = RN(q0 + e * rs) -- which yields RN(x / s)
+// when no intermediate overflows or underflows (here |x / s| <= 448 and
+// s >= 1e-4 / 448).
+__device__ __forceinline__ float div_rn_by(float x, float s, float rs) {
+    const float q0 = __fmul_rn(x, rs);
+    const float e = __fmaf_rn(-q0, s, x);
+    return __fmaf_rn(e, rs, q0);
 }
 
 // Rotates and quantises the vector held in r (this lane's E elements).
@@ -65,10 +77,11 @@ __device__ __forceinline__ uint32_t rotate_quant_warp(float (&r)[D / 32], float 
     }
     amax = warp_max(amax);
     const float s = __fdiv_rn(fmaxf(amax, 1e-4f), 448.0f);
+    const float rs = __frcp_rn(s);
     uint32_t packed = 0;
 #pragma unroll
     for (int e = 0; e < E; e += 2)
-        packed |= e4m3x2_rn_sat(__fdiv_rn(r[e], s), __fdiv_rn(r[e + 1], s)) << (8 * e);
+        packed |= e4m3x2_rn_sat(div_rn_by(r[e], s, rs), div_rn_by(r[e + 1], s, rs)) << (8 * e);
     *scale = s;
     return packed;
 }
@@ -110,10 +123,11 @@ __device__ __forceinline__ void rotate_quant_lanes(float (&r)[64], uint32_t (&co
     }
     if constexpr (D == 128) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
     const float s = __fdiv_rn(fmaxf(amax, 1e-4f), 448.0f);
+    const float rs = __frcp_rn(s);
 #pragma unroll
     for (int j = 0; j < 16; j++)
-        codes[j] = e4m3x2_rn_sat(__fdiv_rn(r[4 * j], s), __fdiv_rn(r[4 * j + 1], s)) |
-                   e4m3x2_rn_sat(__fdiv_rn(r[4 * j + 2], s), __fdiv_rn(r[4 * j + 3], s)) << 16;
+        codes[j] = e4m3x2_rn_sat(div_rn_by(r[4 * j], s, rs), div_rn_by(r[4 * j + 1], s, rs)) |
+                   e4m3x2_rn_sat(div_rn_by(r[4 * j + 2], s, rs), div_rn_by(r[4 * j + 3], s, rs)) << 16;
     *scale = s;
 }
 
