@@ -205,7 +205,7 @@ constexpr int kGather = 8192;      // candidates CTA 0 can select alone
 
 __global__ void __launch_bounds__(kThreads, 1)
 topk_cluster_kernel(const float *scores, int S, int64_t T, int64_t start_pos, int K,
-                    int L, int32_t *__restrict__ idx) {
+                    int L, int store_bins, int32_t *__restrict__ idx) {
     // a kernel launched after this one (the sparse attention) may start its
     // set-up now; it reads the selections only after waiting for this grid
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
@@ -228,6 +228,9 @@ topk_cluster_kernel(const float *scores, int S, int64_t T, int64_t start_pos, in
     extern __shared__ float sv[];                                   // [pad(L)] scores
     uint32_t *gath = reinterpret_cast<uint32_t *>(sv + pad(L) + 1);  // [kGather] keys (CTA 0)
     uint16_t *cand = reinterpret_cast<uint16_t *>(gath + kGather);  // [L] candidate slots
+    // each value's linear bin, [slot within the thread's segment][thread], when
+    // shared memory holds it (else recomputed from the score)
+    uint16_t *bins = store_bins ? cand + L : nullptr;
     __shared__ unsigned hist[kBins];          // local histogram
     __shared__ unsigned hmerged[kBins];       // cluster histogram (CTA 0)
     __shared__ unsigned scan_tmp[33];
@@ -332,8 +335,18 @@ topk_cluster_kernel(const float *scores, int S, int64_t T, int64_t start_pos, in
                                                                   : 0.f;
 
     // round 0: linear bins, merged into CTA 0 with distributed shared-memory atomics
-    for (int i = threadIdx.x; i < len; i += kThreads)
-        atomicAdd(&hist[linear_bin(sv[pad(i)], g_lo, scale)], 1u);
+    // thread i owns the contiguous segment [i*seg, (i+1)*seg) of the slice
+    const int seg = (len + kThreads - 1) / kThreads;
+    const int s0 = threadIdx.x * seg < len ? threadIdx.x * seg : len;
+    const int s1 = s0 + seg < len ? s0 + seg : len;
+    for (int i = s0; i < s1; i++) {
+        const int bin = linear_bin(sv[pad(i)], g_lo, scale);
+        if (bins) bins[(i - s0) * kThreads + threadIdx.x] = (uint16_t)bin;
+        atomicAdd(&hist[bin], 1u);
+    }
+    auto bin_of = [&](int i) -> int {
+        return bins ? (int)bins[(i - s0) * kThreads + threadIdx.x] : linear_bin(sv[pad(i)], g_lo, scale);
+    };
     __syncthreads();
     {
         unsigned *h0 = cl.map_shared_rank(hmerged, 0);
@@ -353,17 +366,13 @@ topk_cluster_kernel(const float *scores, int S, int64_t T, int64_t start_pos, in
     const int tb = (int)ctl.bin;
     unsigned rank = ctl.rank;
 
-    // thread i owns the contiguous segment [i*seg, (i+1)*seg) of the slice
-    const int seg = (len + kThreads - 1) / kThreads;
-    const int s0 = threadIdx.x * seg < len ? threadIdx.x * seg : len;
-    const int s1 = s0 + seg < len ? s0 + seg : len;
     // threshold-bin candidates (slot indices, in any order: only their keys
     // matter), appended in one pass
     if (threadIdx.x == 0) s_ncand = 0;
     __syncthreads();
     int above = 0;                        // this thread's values in bins above the threshold bin
     for (int i = s0; i < s1; i++) {
-        const int bin = linear_bin(sv[pad(i)], g_lo, scale);
+        const int bin = bin_of(i);
         above += bin > tb;
         if (bin == tb) cand[atomicAdd(&s_ncand, 1)] = (uint16_t)i;
     }
@@ -498,11 +507,18 @@ topk_cluster_kernel(const float *scores, int S, int64_t T, int64_t start_pos, in
     int tot;
     int pos = off + block_scan_int(gt + my_q, itmp, &tot);
     for (int i = s0; i < s1; i++) {
-        const uint32_t key = score_key(sv[pad(i)]);
-        bool take = key > tau;
-        if (key == tau && my_q > 0) {
-            take = true;
-            my_q--;
+        // bins are monotone in the score: above the threshold bin means > tau,
+        // below means < tau; only threshold-bin values need their key
+        const int bin = bin_of(i);
+        if (bin < tb) continue;
+        bool take = bin > tb;
+        if (!take) {
+            const uint32_t key = score_key(sv[pad(i)]);
+            take = key > tau;
+            if (key == tau && my_q > 0) {
+                take = true;
+                my_q--;
+            }
         }
         if (take && pos < m) dst[pos++] = (int32_t)(t0 + i);
     }
@@ -612,8 +628,12 @@ dsa_status launch_topk_select(const float *scores, int B, int S, int64_t T, int6
         topk_row_kernel<<<(unsigned)rows, kThreads, 0, stream>>>(scores, S, T, start_pos, K, idx);
         return launch_status();
     }
-    const size_t smem = (size_t)(L + L / 32 + 1) * sizeof(float) + kGather * sizeof(uint32_t) +
-                        (size_t)L * sizeof(uint16_t);
+    size_t smem = (size_t)(L + L / 32 + 1) * sizeof(float) + kGather * sizeof(uint32_t) +
+                  (size_t)L * sizeof(uint16_t);
+    // per-value bins too, when they fit beside the static shared memory (~17 KB)
+    const size_t bins_bytes = (size_t)((L + kThreads - 1) / kThreads) * kThreads * sizeof(uint16_t);
+    const int store_bins = smem + bins_bytes <= (size_t)(208 * 1024) ? 1 : 0;
+    if (store_bins) smem += bins_bytes;
     if (cudaFuncSetAttribute(topk_cluster_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)smem) != cudaSuccess)
         return DSA_ERR_CUDA;
@@ -637,7 +657,7 @@ dsa_status launch_topk_select(const float *scores, int B, int S, int64_t T, int6
     attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 2;
-    if (cudaLaunchKernelEx(&cfg, topk_cluster_kernel, scores, S, T, start_pos, K, L, idx) !=
+    if (cudaLaunchKernelEx(&cfg, topk_cluster_kernel, scores, S, T, start_pos, K, L, store_bins, idx) !=
         cudaSuccess)
         return DSA_ERR_CUDA;
     return launch_status();
