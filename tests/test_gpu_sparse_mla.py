@@ -119,3 +119,23 @@ def test_sparse_mla_prefill_rows_bf16(dsa):
     out, lse = _gpu(dsa, q, kv, idx, sp, sm, dc)
     ref, ref_lse = oracle.sparse_mla(q.float().numpy(), kv.float().numpy(), idx.numpy(), sp, sm, dc)
     assert_attention_close(out, ref, "bf16", lse, ref_lse)
+
+
+def test_sparse_mla_split_partials_keep_range(dsa):
+    """Latent values far beyond the fp16 range of the split partials.
+
+    The cache is scaled by 2^20 and the query by 2^-20 (exact in bf16), so the
+    logits, the softmax and the log-sum-exp are unchanged and the output is
+    2^20 times the unscaled one; one row over 2048 selections runs as many
+    splits, whose partials are stored in fp16 with a power-of-two scale.
+    """
+    B, S, Hq, dc, dr, t_max, k = 1, 1, 128, 512, 64, 4096, 2048
+    q, kv, idx = _case(B, S, Hq, dc, dr, t_max, k, t_max - 1, torch.bfloat16, seed=33)
+    sm = (dc + dr) ** -0.5
+    big = 2.0 ** 20
+    out, lse = _gpu(dsa, (q.float() / big).to(torch.bfloat16), (kv.float() * big).to(torch.bfloat16),
+                    idx, t_max - 1, sm, dc)
+    assert np.all(np.isfinite(out))
+    ref, ref_lse = oracle.sparse_mla(q.float().numpy(), kv.float().numpy(), idx.numpy(), t_max - 1,
+                                     sm, dc)
+    assert_attention_close(out / big, ref, "bf16", lse, ref_lse)

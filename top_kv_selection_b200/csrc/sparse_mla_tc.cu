@@ -36,8 +36,12 @@
 // Both CTAs run the same softmax on the same logits, so their P, running max
 // and sum agree exactly; each accumulates its own half of the output.
 // TMEM: O 256 | S 2 x 64 | P 2 x 32 columns.
-// With several splits per row, unnormalised partial outputs and (max, sum)
-// pairs go to the workspace and a combine kernel merges them.
+// With several splits per row, each split's output normalised by its own sum
+// and divided by a power of two that keeps it below 2^14 (fp16: an 11-bit
+// significand, finer than the bf16 result), with its (max, sum, power of two),
+// goes to the workspace, and a combine kernel merges them.
+#include <cuda_fp16.h>
+
 #include "common.cuh"
 #include "tc_ptx.cuh"
 #include "tmap.cuh"
@@ -75,8 +79,8 @@ struct MlaArgs {
     const int32_t *idx;
     __nv_bfloat16 *out;
     float *lse;
-    float *part_o;      // [units][128][256]  (splits > 1), unit = (row * splits + sp) * 2 + r
-    float2 *part_ml;    // [units][128]
+    __half *part_o;     // [units][256 / 8][128][8]  (splits > 1), unit = (row * splits + sp) * 2 + r
+    float4 *part_ml;    // [units][128] (max, sum, scale of the fp16 partial, 0)
     int64_t t_max;
     int64_t start_pos;
     int S, k, splits;
@@ -243,9 +247,9 @@ sparse_mla_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const MlaArgs a) 
     if (n_tiles == 0) {                                      // nothing selected here
         if (is_softmax) {
             if (a.splits > 1) {
-                float4 *po = reinterpret_cast<float4 *>(a.part_o + (int64_t)unit * kHq * kDh) + h;
-                for (int c = 0; c < kDh / 4; c++) po[c * kHq] = make_float4(0.f, 0.f, 0.f, 0.f);
-                a.part_ml[(int64_t)unit * kHq + h] = make_float2(-INFINITY, 0.f);
+                uint4 *po = reinterpret_cast<uint4 *>(a.part_o + (int64_t)unit * kHq * kDh) + h;
+                for (int c = 0; c < kDh / 8; c++) po[c * kHq] = make_uint4(0u, 0u, 0u, 0u);
+                a.part_ml[(int64_t)unit * kHq + h] = make_float4(-INFINITY, 0.f, 1.f, 0.f);
             } else {
                 __nv_bfloat16 *o = a.out + (row * kHq + h) * kDc + cr * kDh;
                 for (int c = 0; c < kDh; c++) o[c] = __float2bfloat16_rn(0.f);
@@ -445,19 +449,38 @@ sparse_mla_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const MlaArgs a) 
         if (ok && tc::mbar_wait(pv_done, (uint32_t)(n_tiles - 1) & 1u, a.err, abort)) {
             tc::tc_fence_after();
             if (a.splits > 1) {
-                // [column / 4][head] float4s: a warp stores 512 contiguous bytes
-                float4 *po = reinterpret_cast<float4 *>(a.part_o + (int64_t)unit * kHq * kDh) + h;
+                // O / (l * sc) as [column / 8][head] groups of eight halves (a
+                // warp stores 512 contiguous bytes), sc the power of two that
+                // keeps |O / l| / sc <= 2^14 (a first pass finds max |O|)
+                float amax = 0.f;
 #pragma unroll 1
                 for (int c0 = 0; c0 < kDh; c0 += 16) {
                     uint32_t o[16];
                     tc::tmem_ld16(tmem + lane_addr + kColO + c0, o);
                     tc::tmem_wait_ld();
 #pragma unroll
-                    for (int v = 0; v < 4; v++)
-                        po[(c0 / 4 + v) * kHq] = make_float4(__uint_as_float(o[4 * v]), __uint_as_float(o[4 * v + 1]),
-                                                             __uint_as_float(o[4 * v + 2]), __uint_as_float(o[4 * v + 3]));
+                    for (int e = 0; e < 16; e++) amax = fmaxf(amax, fabsf(__uint_as_float(o[e])));
                 }
-                a.part_ml[(int64_t)unit * kHq + h] = make_float2(m_run, l);
+                const float inv_l = l > 0.f ? 1.f / l : 0.f;
+                float sc = 1.f;
+                while (amax * inv_l > 16384.f * sc) sc *= 2.f;
+                const float inv = inv_l / sc;
+                uint4 *po = reinterpret_cast<uint4 *>(a.part_o + (int64_t)unit * kHq * kDh) + h;
+#pragma unroll 1
+                for (int c0 = 0; c0 < kDh; c0 += 16) {
+                    uint32_t o[16], w[8];
+                    tc::tmem_ld16(tmem + lane_addr + kColO + c0, o);
+                    tc::tmem_wait_ld();
+#pragma unroll
+                    for (int e = 0; e < 8; e++) {
+                        const __half2 v = __floats2half2_rn(__uint_as_float(o[2 * e]) * inv,
+                                                            __uint_as_float(o[2 * e + 1]) * inv);
+                        w[e] = *reinterpret_cast<const uint32_t *>(&v);
+                    }
+                    po[(c0 / 8) * kHq] = make_uint4(w[0], w[1], w[2], w[3]);
+                    po[(c0 / 8 + 1) * kHq] = make_uint4(w[4], w[5], w[6], w[7]);
+                }
+                a.part_ml[(int64_t)unit * kHq + h] = make_float4(m_run, l, sc, 0.f);
             } else {
                 const float inv = l > 0.f ? 1.f / l : 0.f;
                 uint4 *o16 = reinterpret_cast<uint4 *>(a.out + (row * kHq + h) * kDc + cr * kDh);
@@ -488,52 +511,64 @@ sparse_mla_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const MlaArgs a) 
     tc::cluster_sync_all();          // the partner no longer touches this CTA's shared memory
 }
 
-// Merges the splits of each (row, half): out = sum_s 2^(m_s - m) O_s / sum_s 2^(m_s - m) l_s.
-// The partials are [column / 4][head] float4s; thread (head, quad) merges four
-// output columns of one head, consecutive threads consecutive heads (coalesced).
-constexpr int kCombineQuads = 2;                         // column quads per block
-__global__ void __launch_bounds__(kHq * kCombineQuads)
-sparse_mla_combine_kernel(const float *part_o, const float2 *part_ml, int splits,
+// Merges the splits of each (row, half): with w_s = 2^(m_s - m) l_s and the
+// stored partials Y_s = O_s / (l_s sc_s), out = sum_s w_s sc_s Y_s / sum_s w_s.
+// The partials are [column / 8][head] groups of eight halves; thread (head,
+// octet) merges eight output columns of one head, consecutive threads
+// consecutive heads (coalesced).
+constexpr int kCombineOcts = 1;                          // column octets per block
+__global__ void __launch_bounds__(kHq * kCombineOcts)
+sparse_mla_combine_kernel(const __half *part_o, const float4 *part_ml, int splits,
                           __nv_bfloat16 *__restrict__ out, float *__restrict__ lse) {
     // the partials come from the preceding kernel: wait for it (plain loads below)
     asm volatile("griddepcontrol.wait;" ::: "memory");
-    constexpr int groups = (kDh / 4) / kCombineQuads;
+    constexpr int groups = (kDh / 8) / kCombineOcts;
     const int64_t rh = blockIdx.x / groups;                 // row * 2 + half
     const int64_t row = rh >> 1;
     const int half = (int)(rh & 1);
     const int h = threadIdx.x % kHq;
-    const int c4 = (int)(blockIdx.x % groups) * kCombineQuads + threadIdx.x / kHq;
+    const int c8 = (int)(blockIdx.x % groups) * kCombineOcts + threadIdx.x / kHq;
     // partial of split sp: unit (row * splits + sp) * 2 + half
     const int64_t u0 = row * splits * 2 + half;
     float m = -INFINITY;
     for (int sp = 0; sp < splits; sp++) m = fmaxf(m, part_ml[(u0 + 2 * sp) * kHq + h].x);
     float L = 0.f;
-    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
     // four splits at a time, so that their loads are in flight together
     for (int sp0 = 0; sp0 < splits; sp0 += 4) {
-        float2 ml[4];
-        float4 x[4];
+        float4 ml[4];
+        uint4 x[4];
 #pragma unroll
         for (int u = 0; u < 4; u++) {
             const int sp = sp0 + u;
-            ml[u] = sp < splits ? part_ml[(u0 + 2 * sp) * kHq + h] : make_float2(-INFINITY, 0.f);
+            ml[u] = sp < splits ? part_ml[(u0 + 2 * sp) * kHq + h] : make_float4(-INFINITY, 0.f, 1.f, 0.f);
             if (sp < splits)
-                x[u] = reinterpret_cast<const float4 *>(part_o + (u0 + 2 * sp) * kHq * kDh)[c4 * kHq + h];
+                x[u] = reinterpret_cast<const uint4 *>(part_o + (u0 + 2 * sp) * kHq * kDh)[c8 * kHq + h];
         }
 #pragma unroll
         for (int u = 0; u < 4; u++) {
             if (ml[u].x == -INFINITY) continue;
-            const float w = exp2f(ml[u].x - m);
-            L += w * ml[u].y;
-            acc.x += w * x[u].x; acc.y += w * x[u].y; acc.z += w * x[u].z; acc.w += w * x[u].w;
+            const float w = exp2f(ml[u].x - m) * ml[u].y;
+            L += w;
+            const float ws = w * ml[u].z;
+            const uint32_t xs[4] = {x[u].x, x[u].y, x[u].z, x[u].w};
+#pragma unroll
+            for (int e = 0; e < 4; e++) {
+                const float2 f = __half22float2(*reinterpret_cast<const __half2 *>(&xs[e]));
+                acc[2 * e] += ws * f.x;
+                acc[2 * e + 1] += ws * f.y;
+            }
         }
     }
     const float inv = L > 0.f ? 1.f / L : 0.f;
-    const __nv_bfloat162 v0 = __floats2bfloat162_rn(acc.x * inv, acc.y * inv);
-    const __nv_bfloat162 v1 = __floats2bfloat162_rn(acc.z * inv, acc.w * inv);
-    reinterpret_cast<uint2 *>(out + (row * kHq + h) * kDc + half * kDh)[c4] =
-        make_uint2(*reinterpret_cast<const uint32_t *>(&v0), *reinterpret_cast<const uint32_t *>(&v1));
-    if (half == 0 && c4 == 0 && lse) lse[row * kHq + h] = L > 0.f ? (m + log2f(L)) * kLn2 : -INFINITY;
+    uint32_t w8[4];
+#pragma unroll
+    for (int e = 0; e < 4; e++) {
+        const __nv_bfloat162 v = __floats2bfloat162_rn(acc[2 * e] * inv, acc[2 * e + 1] * inv);
+        w8[e] = *reinterpret_cast<const uint32_t *>(&v);
+    }
+    reinterpret_cast<uint4 *>(out + (row * kHq + h) * kDc + half * kDh)[c8] = make_uint4(w8[0], w8[1], w8[2], w8[3]);
+    if (half == 0 && c8 == 0 && lse) lse[row * kHq + h] = L > 0.f ? (m + log2f(L)) * kLn2 : -INFINITY;
 }
 
 // Splits per row: as many pairs as fill the SMs once, then as few as give the
@@ -558,8 +593,8 @@ size_t sparse_mla_tc_workspace_bytes(int B, int S, int k) {
     const int sp = mla_splits(rows, k);
     if (sp <= 1) return 0;
     const int64_t units = rows * 2 * sp;
-    return align_up((size_t)units * kHq * kDh * sizeof(float), 256) +
-           (size_t)units * kHq * sizeof(float2);
+    return align_up((size_t)units * kHq * kDh * sizeof(__half), 256) +
+           (size_t)units * kHq * sizeof(float4);
 }
 
 dsa_status launch_sparse_mla_tc(const void *q, const void *kv, int64_t t_max, const int32_t *idx,
@@ -592,9 +627,9 @@ dsa_status launch_sparse_mla_tc(const void *q, const void *kv, int64_t t_max, co
     a.part_ml = nullptr;
     if (a.splits > 1) {
         const int64_t units = rows * 2 * a.splits;
-        a.part_o = static_cast<float *>(ws);
-        a.part_ml = reinterpret_cast<float2 *>(static_cast<char *>(ws) +
-                                               align_up((size_t)units * kHq * kDh * sizeof(float), 256));
+        a.part_o = static_cast<__half *>(ws);
+        a.part_ml = reinterpret_cast<float4 *>(static_cast<char *>(ws) +
+                                               align_up((size_t)units * kHq * kDh * sizeof(__half), 256));
     }
     if (cudaFuncSetAttribute(sparse_mla_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)kSmemBytes) != cudaSuccess)
@@ -619,16 +654,16 @@ dsa_status launch_sparse_mla_tc(const void *q, const void *kv, int64_t t_max, co
     dsa_status st = launch_status();
     if (st != DSA_OK || a.splits == 1) return st;
     cudaLaunchConfig_t ccfg = {};
-    ccfg.gridDim = dim3((unsigned)(rows * 2 * ((kDh / 4) / kCombineQuads)));
-    ccfg.blockDim = dim3(kHq * kCombineQuads);
+    ccfg.gridDim = dim3((unsigned)(rows * 2 * ((kDh / 8) / kCombineOcts)));
+    ccfg.blockDim = dim3(kHq * kCombineOcts);
     ccfg.stream = stream;
     cudaLaunchAttribute cattr[1];
     cattr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     cattr[0].val.programmaticStreamSerializationAllowed = 1;
     ccfg.attrs = cattr;
     ccfg.numAttrs = 1;
-    if (cudaLaunchKernelEx(&ccfg, sparse_mla_combine_kernel, (const float *)a.part_o,
-                           (const float2 *)a.part_ml, a.splits, a.out, lse) != cudaSuccess)
+    if (cudaLaunchKernelEx(&ccfg, sparse_mla_combine_kernel, (const __half *)a.part_o,
+                           (const float4 *)a.part_ml, a.splits, a.out, lse) != cudaSuccess)
         return DSA_ERR_CUDA;
     return launch_status();
 }
