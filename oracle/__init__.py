@@ -62,6 +62,14 @@ def _load():
     lib.oracle_act_quant.restype = None
     lib.oracle_indexer_quant.argtypes = [P, i64, i32, P, P]
     lib.oracle_indexer_quant.restype = None
+    lib.oracle_rope_half.argtypes = [P, i32, P]
+    lib.oracle_rope_half.restype = None
+    lib.oracle_scale_ue8m0.argtypes = [f32]
+    lib.oracle_scale_ue8m0.restype = f32
+    lib.oracle_act_quant_fmt.argtypes = [P, i32, i32, i32, P, P]
+    lib.oracle_act_quant_fmt.restype = None
+    lib.oracle_indexer_prologue.argtypes = [P, P, i32, i32, i32, i32, i32, P, i32, P, P, P, P]
+    lib.oracle_indexer_prologue.restype = None
     lib.oracle_weight_fold.argtypes = [f32, i32, f32, f32]
     lib.oracle_weight_fold.restype = f32
     lib.oracle_index_scores.argtypes = [P, P, P, P, P, i64, i32, i32, i32, i32, i64, i64,
@@ -151,6 +159,65 @@ def indexer_quant(x: np.ndarray):
     sc = np.empty(x.shape[:-1], dtype=np.float32)
     lib.oracle_indexer_quant(_p(x), n_vec, D, _p(out), _p(sc))
     return out, sc
+
+
+def rope_half(x: np.ndarray, cs: np.ndarray) -> np.ndarray:
+    """Non-interleaved rotary embedding of the first R = 2 * cs.shape[-2] elements
+    of each trailing vector of x, with the angles cs [..., R/2, 2] (cos, sin)
+    broadcast over the leading dims of x except the last."""
+    lib = _load()
+    x = _c(x, np.float32).copy()
+    R = 2 * cs.shape[-2]
+    D = x.shape[-1]
+    flat = x.reshape(-1, D)
+    csb = np.broadcast_to(_c(cs, np.float32), x.shape[:-1] + (R // 2, 2)).reshape(-1, R // 2, 2)
+    for r in range(flat.shape[0]):
+        row = np.ascontiguousarray(flat[r])
+        c = np.ascontiguousarray(csb[r])
+        lib.oracle_rope_half(_p(row), R, _p(c))
+        flat[r] = row
+    return flat.reshape(x.shape)
+
+
+def scale_ue8m0(s: float) -> np.float32:
+    return np.float32(_load().oracle_scale_ue8m0(s))
+
+
+def act_quant_fmt(x: np.ndarray, block: int, fmt: int):
+    """act_quant with scale format fmt (0 fp32, 1 ue8m0): returns (codes, scales)."""
+    lib = _load()
+    x = _c(x, np.float32)
+    n = x.shape[-1]
+    flat = x.reshape(-1, n)
+    y = np.empty(flat.shape, dtype=np.uint8)
+    s = np.empty((flat.shape[0], n // block), dtype=np.float32)
+    for r in range(flat.shape[0]):
+        row = np.ascontiguousarray(flat[r])
+        yr = np.empty(n, dtype=np.uint8)
+        sr = np.empty(n // block, dtype=np.float32)
+        lib.oracle_act_quant_fmt(_p(row), n, block, fmt, _p(yr), _p(sr))
+        y[r], s[r] = yr, sr
+    return y.reshape(x.shape), s.reshape(x.shape[:-1] + (n // block,))
+
+
+def indexer_prologue(q: np.ndarray, k: np.ndarray, cs: np.ndarray, fmt: int = 0):
+    """RoPE (first R dims, not interleaved) + rotate_activation + act_quant of the
+    indexer's queries q [B,S,H,D] and keys k [B,S,D]; cs [S, R/2, 2] (cos, sin),
+    R = 0 when cs has no columns.  Returns (q_fp8, q_scale, k_fp8, k_scale)."""
+    lib = _load()
+    q = _c(q, np.float32)
+    k = _c(k, np.float32)
+    B, S, H, D = q.shape
+    cs = _c(cs, np.float32).reshape(S, -1, 2) if cs is not None else np.zeros((S, 0, 2), np.float32)
+    R = 2 * cs.shape[1]
+    qf = np.empty(q.shape, dtype=np.uint8)
+    qs = np.empty((B, S, H), dtype=np.float32)
+    kf = np.empty(k.shape, dtype=np.uint8)
+    ks = np.empty((B, S), dtype=np.float32)
+    cs_buf = np.ascontiguousarray(cs if R else np.zeros((S, 1, 2), np.float32))
+    lib.oracle_indexer_prologue(_p(q), _p(k), B, S, H, D, R, _p(cs_buf), fmt, _p(qf), _p(qs),
+                                _p(kf), _p(ks))
+    return qf, qs, kf, ks
 
 
 def weight_fold(w: float, H: int, q_scale: float, softmax_scale: float) -> np.float32:

@@ -162,6 +162,99 @@ void oracle_indexer_quant(const float *x, int64_t n_vec, int D, uint8_t *out, fl
 }
 
 /*
+ * Rotary embedding of the first R elements of one vector, not interleaved
+ * [V32-IDX: q_pe = first rope_head_dim elements; apply_rotary_emb(q_pe,
+ * freqs_cis, False); q = cat(q_pe, q_nope)].  Element j and element j + R/2
+ * (j < R/2) are the real and imaginary parts of one complex number, which is
+ * multiplied by the position's unit complex cs[2j] + i cs[2j+1] (cos, sin of
+ * frequency j): (x1 + i x2)(c + i s) = (x1 c - x2 s) + i (x1 s + x2 c), each
+ * product and sum rounded to fp32.  Elements R .. D-1 are not touched.
+ */
+void oracle_rope_half(float *x, int R, const float *cs)
+{
+    int half = R / 2;
+    for (int j = 0; j < half; j++) {
+        float c = cs[2 * j], sn = cs[2 * j + 1];
+        float x1 = x[j], x2 = x[j + half];
+        float re_a = x1 * c, re_b = x2 * sn;
+        float im_a = x1 * sn, im_b = x2 * c;
+        x[j] = re_a - re_b;
+        x[j + half] = im_a + im_b;
+    }
+}
+
+/*
+ * The ue8m0 scale format [V32-IDX: act_quant(x, block_size, scale_fmt)]: the
+ * scale is stored as a bare power of two, here the smallest power of two not
+ * below the fp32 scale max(amax, 1e-4) / 448, so that |x / scale| stays within
+ * the e4m3 range.
+ */
+float oracle_scale_ue8m0(float s)
+{
+    int e;
+    double m = frexp((double)s, &e);          /* s = m * 2^e, 0.5 <= m < 1 */
+    if (m == 0.5)
+        return s;
+    return (float)ldexp(1.0, e);
+}
+
+/* act_quant with the scale format: fmt 0 = fp32 scale, 1 = ue8m0 scale. */
+void oracle_act_quant_fmt(const float *x, int n, int block, int fmt, uint8_t *y, float *scale)
+{
+    for (int b0 = 0; b0 < n; b0 += block) {
+        float amax = 0.0f;
+        for (int i = b0; i < b0 + block; i++) {
+            float a = fabsf(x[i]);
+            if (a > amax)
+                amax = a;
+        }
+        float clamped = amax > 1e-4f ? amax : 1e-4f;
+        float s = clamped / 448.0f;
+        if (fmt == 1)
+            s = oracle_scale_ue8m0(s);
+        scale[b0 / block] = s;
+        for (int i = b0; i < b0 + block; i++)
+            y[i] = oracle_e4m3_encode(x[i] / s);
+    }
+}
+
+/*
+ * The indexer's query and key preparation [V32-IDX, Indexer.forward]: for
+ * every query head vector q[b, s, h, :] and key vector k[b, s, :] (D each, fp32):
+ * rotary embedding of the first R elements with the angles of row s of cs
+ * ([S][R/2][2], the caller's freqs_cis rows start_pos .. start_pos + S - 1),
+ * rotate_activation, act_quant with block = D and the scale format fmt.
+ * Query codes / scales go to q_fp8 [B,S,H,D] / q_scale [B,S,H]; key codes /
+ * scales to k_fp8 [B,S,D] / k_scale [B,S] (the rows a cache append writes at
+ * positions start_pos .. start_pos + S - 1).
+ */
+void oracle_indexer_prologue(const float *q, const float *k, int B, int S, int H, int D, int R,
+                             const float *cs, int fmt, uint8_t *q_fp8, float *q_scale,
+                             uint8_t *k_fp8, float *k_scale)
+{
+    float *tmp = (float *)malloc(sizeof(float) * (size_t)D);
+    for (int b = 0; b < B; b++) {
+        for (int s = 0; s < S; s++) {
+            const float *cs_s = cs + (size_t)s * (size_t)R;
+            for (int h = 0; h <= H; h++) {
+                /* h < H: query head h; h == H: the key */
+                int64_t v = ((int64_t)b * S + s) * H + h;
+                const float *src = h < H ? q + v * D : k + ((int64_t)b * S + s) * D;
+                memcpy(tmp, src, sizeof(float) * (size_t)D);
+                oracle_rope_half(tmp, R, cs_s);
+                oracle_fwht_f32(tmp, D);
+                if (h < H)
+                    oracle_act_quant_fmt(tmp, D, D, fmt, q_fp8 + v * D, q_scale + v);
+                else
+                    oracle_act_quant_fmt(tmp, D, D, fmt, k_fp8 + ((int64_t)b * S + s) * D,
+                                         k_scale + (int64_t)b * S + s);
+            }
+        }
+    }
+    free(tmp);
+}
+
+/*
  * Weight fold [V32-IDX]: weights * n_heads^-1/2, then * q_scale * softmax_scale,
  * each product in fp32 and in that order.
  */
