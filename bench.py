@@ -392,9 +392,10 @@ def run_ours(args, wl, world, rank, local):
     peak, peak_kind = _peaks()
     stages = time_stages(dsa, wl, copies, iters=max(10, min(args.steps, 500)))
     t_score = stages["decode_index_scores"]
-    prefill = None
+    prefill = prologue = None
     if not args.no_prefill:
         prefill = time_prefill_scoring(dsa, measure_fp8_peak(sustained=False)["fp8_e4m3_tflops"])
+        prologue = time_indexer_prologue(dsa, peak)
     # keys + scales of every cached token, plus the new tokens' fp32 queries,
     # weights and keys (the scores written are not algorithmic)
     score_bytes = wl.B * wl.T * (wl.D + 4) + wl.B * (wl.H * wl.D * 4 + wl.H * 4 + wl.D * 4)
@@ -427,6 +428,7 @@ def run_ours(args, wl, world, rank, local):
         "kernels_per_step": per_step_launches, "kernels": kernel_names,
         "stage_us": {k: round(v * 1e6, 2) for k, v in stages.items()},
         "prefill_scoring": prefill,
+        "indexer_prologue": prologue,
         "clocks": clk.summary(),
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -525,6 +527,45 @@ def time_prefill_scoring(dsa, fp8_peak, iters=10):
     return out
 
 
+def time_indexer_prologue(dsa, peak_gbs, iters=20):
+    """The fused indexer prologue (RoPE on 64 of 128 dims, not interleaved ->
+    rotate_activation -> act_quant -> key cache append) over the queries and keys
+    of the T = 8192 prefill, bf16 inputs as a projection produces them.  HBM-bound:
+    algorithmic bytes = the bf16 inputs, the codes and scales written and the
+    rotary table; 2 inputs + outputs > 126 MB of L2, so every launch streams."""
+    wl = workloads.WORKLOADS[3]
+    T, H, D, R = wl.T, wl.H, wl.D, 64
+    g = torch.Generator(device="cuda").manual_seed(wl.seed(1))
+    q = torch.randn(1, T, H, D, device="cuda", generator=g).to(torch.bfloat16)
+    k = torch.randn(1, T, D, device="cuda", generator=g).to(torch.bfloat16)
+    th = torch.rand(T, R // 2, device="cuda", generator=g) * 6.283185307179586
+    cs = torch.stack([torch.cos(th), torch.sin(th)], dim=-1).contiguous()
+    q_fp8 = torch.empty(1, T, H, D, dtype=torch.uint8, device="cuda")
+    q_scale = torch.empty(1, T, H, dtype=torch.float32, device="cuda")
+    k_cache = torch.empty(1, T, D, dtype=torch.uint8, device="cuda")
+    k_scale = torch.empty(1, T, dtype=torch.float32, device="cuda")
+
+    def one():
+        dsa.dsa_indexer_prologue(q, k, cs, 0, q_fp8, q_scale, k_cache, k_scale)
+
+    for _ in range(3):
+        one()
+    torch.cuda.synchronize()
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0.record()
+    for _ in range(iters):
+        one()
+    t1.record()
+    t1.synchronize()
+    t = t0.elapsed_time(t1) * 1e-3 / iters
+    nbytes = T * (H + 1) * (2 * D + D + 4) + T * (R // 2) * 8
+    out = {"workload": "prefill_T8192_bf16_rope64", "vectors": T * (H + 1), "bytes": nbytes,
+           "us": t * 1e6, "achieved_gbs": nbytes / t / 1e9, "peak_gbs": peak_gbs,
+           "frac": nbytes / t / 1e9 / peak_gbs, "bound": "hbm"}
+    del q, k, q_fp8, k_cache
+    return out
+
+
 def measure_fp8_peak(n=8192, iters=20, sustained=True):
     """Dense e4m3 GEMM throughput (torch._scaled_mm, N^3, best of `iters`) -- the
     FP8 tensor-core denominator for the prefill scorer's roofline."""
@@ -573,6 +614,8 @@ def main(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-prefill", action="store_true",
                     help="skip the prefill scoring measurement")
+    ap.add_argument("--prologue-only", action="store_true",
+                    help="time only the fused indexer prologue on the T=8192 prefill")
     ap.add_argument("--prefill-only", action="store_true",
                     help="only time the prefill scoring (T = 8192 causal) and exit")
     ap.add_argument("--fp8-peak", action="store_true",
@@ -582,6 +625,13 @@ def main(argv=None):
     args = ap.parse_args(argv)
     if args.fp8_peak:
         print(json.dumps(measure_fp8_peak()), flush=True)
+        return
+    if args.prologue_only:
+        import __graft_entry__
+        __graft_entry__._builder().build()
+        import top_kv_selection_b200 as dsa
+        print(json.dumps(time_indexer_prologue(dsa, _peaks()[0], iters=max(1, args.steps))),
+              flush=True)
         return
     if args.prefill_only:
         import __graft_entry__

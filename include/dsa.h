@@ -61,6 +61,12 @@ typedef enum dsa_dtype {
     DSA_BF16 = 1               /* bfloat16      */
 } dsa_dtype;
 
+/* act_quant's scale_fmt: a plain fp32 scale, or ue8m0 (a bare power of two). */
+typedef enum dsa_scale_fmt {
+    DSA_SCALE_F32 = 0,
+    DSA_SCALE_UE8M0 = 1
+} dsa_scale_fmt;
+
 /* Text for a status code (static storage, never NULL). */
 const char *dsa_status_string(dsa_status status);
 
@@ -98,6 +104,42 @@ dsa_status dsa_get_device_error(dsa_stream_t stream, int32_t *device_status);
 dsa_status dsa_indexer_quant(const void *x, dsa_dtype x_dtype, int64_t n_rows, int64_t n_vec,
                              int d, uint8_t *out_fp8, int64_t out_row_stride, float *out_scale,
                              int64_t scale_row_stride, dsa_stream_t stream);
+
+/*
+ * The indexer's query and key preparation in one pass (Indexer.forward,
+ * "Split indexer heads": split off the first rope_head_dim elements, rotary
+ * embedding with interleaved = False, concatenate, rotate_activation,
+ * act_quant(x, block_size, scale_fmt), k_cache / k_scale_cache append at
+ * start_pos .. start_pos + S - 1).
+ * Rotary part, for every query head vector and key vector: element j and
+ * element j + rope_dim/2 (j < rope_dim/2) are the real and imaginary parts of
+ * one complex number, multiplied by rope_cs[s][j] = (cos, sin) of the token's
+ * angle for frequency j: x1' = x1*c - x2*s, x2' = x1*s + x2*c, each product
+ * and sum rounded to fp32 (bf16 inputs are widened to fp32 first; the result
+ * stays fp32).  Then rotation and quantisation as dsa_indexer_quant, except
+ * that with DSA_SCALE_UE8M0 the scale max(amax, 1e-4) / 448 is rounded up to
+ * the smallest power of two not below it.
+ *
+ *   q        [B,S,H,d] F32 or BF16 (x_dtype), contiguous, 16-byte aligned
+ *   k        [B,S,d]   same dtype, contiguous, 16-byte aligned
+ *   rope_cs  [S, rope_dim/2, 2] fp32, 16-byte aligned: row s is the angle of
+ *            position start_pos + s (the caller's freqs_cis[start_pos + s] as
+ *            (re, im)); unused (may be NULL) when rope_dim = 0
+ *   q_fp8    [B,S,H,d] e4m3 codes (16-byte aligned), q_scale [B,S,H] fp32
+ *   k_cache  [B,t_max,d] e4m3 codes (16-byte aligned), k_scale [B,t_max] fp32:
+ *            rows start_pos .. start_pos + S - 1 of each sequence are
+ *            written, nothing else
+ * d must be 64 or 128 and rope_dim one of 0, 8, 16, 32, 64 (or 128 when
+ * d = 128), else DSA_ERR_UNSUPPORTED; start_pos + S <= t_max, else
+ * DSA_ERR_INVALID_ARG, as are NULL or misaligned buffers.  H may be 0 (keys
+ * only; q, q_fp8 and q_scale may then be NULL).  All buffers are caller-owned
+ * device memory; the call is asynchronous on `stream`.
+ */
+dsa_status dsa_indexer_prologue(const void *q, const void *k, dsa_dtype x_dtype, int B, int S,
+                                int H, int d, int rope_dim, const float *rope_cs,
+                                dsa_scale_fmt scale_fmt, int64_t start_pos, int64_t t_max,
+                                uint8_t *q_fp8, float *q_scale, uint8_t *k_cache,
+                                float *k_scale, dsa_stream_t stream);
 
 /*
  * fp8_index with the weight fold and the additive causal mask

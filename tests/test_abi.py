@@ -66,6 +66,31 @@ def test_indexer_quant_argument_checks(dsa):
     assert L.dsa_indexer_quant(NULL, 0, 1, 0, 128, NULL, 0, NULL, 0, NULL) == dsa.DSA_OK
 
 
+def test_indexer_prologue_argument_checks(dsa):
+    L = dsa._lib
+    F, U = dsa.DSA_SCALE_F32, dsa.DSA_SCALE_UE8M0
+
+    def call(q=FAKE, k=FAKE, dt=0, B=1, S=2, H=4, d=128, R=64, cs=FAKE, fmt=F, sp=0, t_max=8,
+             qf=FAKE, qs=FAKE, kc=FAKE, ks=FAKE):
+        return L.dsa_indexer_prologue(q, k, dt, B, S, H, d, R, cs, fmt, sp, t_max, qf, qs, kc, ks,
+                                      NULL)
+
+    assert call(d=96) == dsa.DSA_ERR_UNSUPPORTED
+    for R in (24, 4, 256):                      # not a power of two / below d/16 / above d
+        assert call(R=R) == dsa.DSA_ERR_UNSUPPORTED
+    assert call(dt=7) == dsa.DSA_ERR_INVALID_ARG
+    assert call(fmt=2) == dsa.DSA_ERR_INVALID_ARG
+    assert call(sp=7, S=2, t_max=8) == dsa.DSA_ERR_INVALID_ARG   # rows 7, 8 past the cache
+    assert call(cs=NULL) == dsa.DSA_ERR_INVALID_ARG
+    assert call(k=NULL) == dsa.DSA_ERR_INVALID_ARG
+    assert call(q=ODD) == dsa.DSA_ERR_INVALID_ARG
+    assert call(kc=ODD) == dsa.DSA_ERR_INVALID_ARG
+    assert call(B=-1) == dsa.DSA_ERR_INVALID_ARG
+    # empty problems succeed without a launch (no GPU here)
+    assert call(B=0, q=NULL, k=NULL, cs=NULL, fmt=U) == dsa.DSA_OK
+    assert call(S=0) == dsa.DSA_OK
+
+
 def test_index_scores_argument_checks(dsa):
     L = dsa._lib
     args = lambda **kw: [kw.get("q", FAKE), FAKE, FAKE, kw.get("k", FAKE), FAKE,

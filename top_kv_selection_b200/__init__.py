@@ -26,6 +26,7 @@ _lib = ctypes.CDLL(LIB_PATH)
 DSA_OK, DSA_ERR_INVALID_ARG, DSA_ERR_UNSUPPORTED, DSA_ERR_CUDA = 0, 1, 2, 3
 DSA_ERR_TIMEOUT, DSA_ERR_DEVICE, DSA_ERR_WORKSPACE = 4, 5, 6
 DSA_F32, DSA_BF16 = 0, 1
+DSA_SCALE_F32, DSA_SCALE_UE8M0 = 0, 1
 DSA_NOALLOC_SCRATCH_BYTES = 32 << 20
 
 _P, _i32, _i64, _f32, _sz = (ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_float,
@@ -36,6 +37,8 @@ _SIGNATURES = {
     "dsa_version": ([], _i32),
     "dsa_get_device_error": ([_P, _P], _i32),
     "dsa_indexer_quant": ([_P, _i32, _i64, _i64, _i32, _P, _i64, _P, _i64, _P], _i32),
+    "dsa_indexer_prologue": ([_P, _P, _i32, _i32, _i32, _i32, _i32, _i32, _P, _i32, _i64, _i64,
+                              _P, _P, _P, _P, _P], _i32),
     "dsa_index_scores": ([_P, _P, _P, _P, _P, _i64, _i32, _i32, _i32, _i32, _i64, _i64, _f32,
                           _P, _P], _i32),
     "dsa_decode_index_scores": ([_P, _P, _P, _P, _P, _i64, _i32, _i32, _i32, _i64, _f32, _P, _P],
@@ -125,6 +128,22 @@ def dsa_indexer_quant(x: torch.Tensor, out_fp8: torch.Tensor, out_scale: torch.T
         _ptr(x), _dtype(x), n_rows, n_vec, d, ctypes.c_void_p(out_fp8.data_ptr()),
         out_row_stride, ctypes.c_void_p(out_scale.data_ptr()), scale_row_stride,
         _stream(stream)))
+
+
+def dsa_indexer_prologue(q: torch.Tensor | None, k: torch.Tensor, rope_cs: torch.Tensor | None,
+                         start_pos: int, q_fp8: torch.Tensor | None, q_scale: torch.Tensor | None,
+                         k_cache: torch.Tensor, k_scale: torch.Tensor,
+                         scale_fmt: int = DSA_SCALE_F32, stream=None) -> None:
+    """RoPE (first rope_dim elements, not interleaved) + rotate_activation + act_quant of
+    q [B,S,H,d] and k [B,S,d]; keys appended to k_cache [B,t_max,d] / k_scale [B,t_max]
+    at start_pos.  rope_cs [S, rope_dim/2, 2] fp32 (cos, sin), or None for no rotary part."""
+    B, S, d = k.shape
+    H = q.shape[2] if q is not None else 0
+    rope_dim = 2 * rope_cs.shape[1] if rope_cs is not None else 0
+    t_max = k_cache.shape[1]
+    _check("dsa_indexer_prologue", _lib.dsa_indexer_prologue(
+        _ptr(q), _ptr(k), _dtype(k), B, S, H, d, rope_dim, _ptr(rope_cs), scale_fmt, start_pos,
+        t_max, _ptr(q_fp8), _ptr(q_scale), _ptr(k_cache), _ptr(k_scale), _stream(stream)))
 
 
 def dsa_index_scores(q_fp8: torch.Tensor, q_scale: torch.Tensor, w: torch.Tensor,

@@ -43,11 +43,21 @@ __device__ __forceinline__ float div_rn_by(float x, float s, float rs) {
     return __fmaf_rn(e, rs, q0);
 }
 
+// The ue8m0 scale format: the smallest power of two not below s (s positive
+// and normal): keep the exponent when the significand bits are zero, else
+// step it up by one.
+__device__ __forceinline__ float pow2_ceil(float s) {
+    const uint32_t b = __float_as_uint(s);
+    return (b & 0x007FFFFFu) ? __uint_as_float((b & 0x7F800000u) + 0x00800000u) : s;
+}
+
 // Rotates and quantises the vector held in r (this lane's E elements).
 // Returns this lane's E codes packed little-endian; *scale gets the vector's
-// scale (same value in every lane).  All 32 lanes must call it.
+// scale (same value in every lane), rounded up to a power of two when ue8m0.
+// All 32 lanes must call it.
 template <int D>
-__device__ __forceinline__ uint32_t rotate_quant_warp(float (&r)[D / 32], float *scale) {
+__device__ __forceinline__ uint32_t rotate_quant_warp(float (&r)[D / 32], float *scale,
+                                                      bool ue8m0 = false) {
     constexpr int E = D / 32;
     const int lane = threadIdx.x & 31;
 #pragma unroll
@@ -76,7 +86,8 @@ __device__ __forceinline__ uint32_t rotate_quant_warp(float (&r)[D / 32], float 
         amax = fmaxf(amax, fabsf(r[e]));
     }
     amax = warp_max(amax);
-    const float s = __fdiv_rn(fmaxf(amax, 1e-4f), 448.0f);
+    float s = __fdiv_rn(fmaxf(amax, 1e-4f), 448.0f);
+    if (ue8m0) s = pow2_ceil(s);
     const float rs = __frcp_rn(s);
     uint32_t packed = 0;
 #pragma unroll
@@ -95,7 +106,7 @@ __device__ __forceinline__ uint32_t rotate_quant_warp(float (&r)[D / 32], float 
 // 4j .. 4j + 3 of this lane's slice, little-endian.
 template <int D>
 __device__ __forceinline__ void rotate_quant_lanes(float (&r)[64], uint32_t (&codes)[16],
-                                                   float *scale) {
+                                                   float *scale, bool ue8m0 = false) {
     static_assert(D == 64 || D == 128, "one or two lanes per vector");
 #pragma unroll
     for (int h = 1; h < 64; h <<= 1) {
@@ -122,7 +133,8 @@ __device__ __forceinline__ void rotate_quant_lanes(float (&r)[64], uint32_t (&co
         amax = fmaxf(amax, fabsf(r[e]));
     }
     if constexpr (D == 128) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
-    const float s = __fdiv_rn(fmaxf(amax, 1e-4f), 448.0f);
+    float s = __fdiv_rn(fmaxf(amax, 1e-4f), 448.0f);
+    if (ue8m0) s = pow2_ceil(s);
     const float rs = __frcp_rn(s);
 #pragma unroll
     for (int j = 0; j < 16; j++)
