@@ -70,6 +70,12 @@ def _load():
     lib.oracle_act_quant_fmt.restype = None
     lib.oracle_indexer_prologue.argtypes = [P, P, i32, i32, i32, i32, i32, P, i32, P, P, P, P]
     lib.oracle_indexer_prologue.restype = None
+    lib.oracle_latent_row_bytes.argtypes = [i32, i32]
+    lib.oracle_latent_row_bytes.restype = i64
+    lib.oracle_latent_quant.argtypes = [P, i32, i32, P]
+    lib.oracle_latent_quant.restype = None
+    lib.oracle_latent_dequant.argtypes = [P, i32, i32, P]
+    lib.oracle_latent_dequant.restype = None
     lib.oracle_weight_fold.argtypes = [f32, i32, f32, f32]
     lib.oracle_weight_fold.restype = f32
     lib.oracle_index_scores.argtypes = [P, P, P, P, P, i64, i32, i32, i32, i32, i64, i64,
@@ -218,6 +224,46 @@ def indexer_prologue(q: np.ndarray, k: np.ndarray, cs: np.ndarray, fmt: int = 0)
     lib.oracle_indexer_prologue(_p(q), _p(k), B, S, H, D, R, _p(cs_buf), fmt, _p(qf), _p(qs),
                                 _p(kf), _p(ks))
     return qf, qs, kf, ks
+
+
+def latent_row_bytes(dc: int, dr: int) -> int:
+    return int(_load().oracle_latent_row_bytes(dc, dr))
+
+
+def latent_quant(kv: np.ndarray, dc: int) -> np.ndarray:
+    """FP8 latent rows: kv [..., dc + dr] -> uint8 [..., latent_row_bytes(dc, dr)]."""
+    lib = _load()
+    kv = _c(kv, np.float32)
+    dr = kv.shape[-1] - dc
+    nbytes = latent_row_bytes(dc, dr)
+    flat = kv.reshape(-1, dc + dr)
+    out = np.empty((flat.shape[0], nbytes), dtype=np.uint8)
+    for r in range(flat.shape[0]):
+        row = np.ascontiguousarray(flat[r])
+        o = np.empty(nbytes, dtype=np.uint8)
+        lib.oracle_latent_quant(_p(row), dc, dr, _p(o))
+        out[r] = o
+    return out.reshape(kv.shape[:-1] + (nbytes,))
+
+
+def latent_dequant(rows: np.ndarray, dc: int, dr: int) -> np.ndarray:
+    """Decoded FP8 latent rows: uint8 [..., bytes] -> fp32 [..., dc + dr]."""
+    lib = _load()
+    rows = _c(rows, np.uint8)
+    flat = rows.reshape(-1, rows.shape[-1])
+    out = np.empty((flat.shape[0], dc + dr), dtype=np.float32)
+    for r in range(flat.shape[0]):
+        row = np.ascontiguousarray(flat[r])
+        o = np.empty(dc + dr, dtype=np.float32)
+        lib.oracle_latent_dequant(_p(row), dc, dr, _p(o))
+        out[r] = o
+    return out.reshape(rows.shape[:-1] + (dc + dr,))
+
+
+def sparse_mla_fp8(q, kv_rows, idx, start_pos: int, sm_scale: float, dc: int, dr: int):
+    """Sparse attention over an FP8 latent cache: the rows are decoded, then the
+    same fp64 attention as sparse_mla."""
+    return sparse_mla(q, latent_dequant(kv_rows, dc, dr), idx, start_pos, sm_scale, dc)
 
 
 def weight_fold(w: float, H: int, q_scale: float, softmax_scale: float) -> np.float32:

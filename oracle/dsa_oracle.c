@@ -255,6 +255,59 @@ void oracle_indexer_prologue(const float *q, const float *k, int B, int S, int H
 }
 
 /*
+ * FP8 latent row [DIAG: "cache: latents (T x 576, FP8 + bf16 RoPE)", "Stored per
+ * token per layer: 656 B latent row"].  The latent part c (the first dc values)
+ * is quantised in blocks of 128 exactly as act_quant does (one fp32 scale per
+ * block); the rotary part (the last dr values) stays bf16, rounded to nearest
+ * even.  Row layout: [dc e4m3 codes | dc/128 fp32 scales | dr bf16 values],
+ * 512 + 16 + 128 = 656 bytes at the V3.2 sizes.
+ */
+int64_t oracle_latent_row_bytes(int dc, int dr)
+{
+    return (int64_t)dc + (int64_t)(dc / 128) * 4 + (int64_t)dr * 2;
+}
+
+static uint16_t bf16_rne(float x)
+{
+    uint32_t b;
+    memcpy(&b, &x, 4);
+    if ((b & 0x7F800000u) == 0x7F800000u && (b & 0x007FFFFFu))
+        return (uint16_t)((b >> 16) | 0x40);              /* quiet NaN */
+    b += 0x7FFFu + ((b >> 16) & 1u);
+    return (uint16_t)(b >> 16);
+}
+
+void oracle_latent_quant(const float *x, int dc, int dr, uint8_t *row)
+{
+    int nb = dc / 128;
+    float *sc = (float *)malloc(sizeof(float) * (size_t)(nb > 0 ? nb : 1));
+    oracle_act_quant(x, dc, 128, row, sc);
+    memcpy(row + dc, sc, sizeof(float) * (size_t)nb);
+    for (int i = 0; i < dr; i++) {
+        uint16_t h = bf16_rne(x[dc + i]);
+        memcpy(row + dc + 4 * nb + 2 * i, &h, 2);
+    }
+    free(sc);
+}
+
+/* Decoded row: c[i] = e4m3(code_i) * scale[i / 128] (rounded to fp32), k_pe from bf16. */
+void oracle_latent_dequant(const uint8_t *row, int dc, int dr, float *x)
+{
+    int nb = dc / 128;
+    for (int i = 0; i < dc; i++) {
+        float s;
+        memcpy(&s, row + dc + 4 * (i / 128), 4);
+        x[i] = (float)(oracle_e4m3_decode(row[i]) * (double)s);
+    }
+    for (int i = 0; i < dr; i++) {
+        uint16_t h;
+        memcpy(&h, row + dc + 4 * nb + 2 * i, 2);
+        uint32_t b = (uint32_t)h << 16;
+        memcpy(&x[dc + i], &b, 4);
+    }
+}
+
+/*
  * Weight fold [V32-IDX]: weights * n_heads^-1/2, then * q_scale * softmax_scale,
  * each product in fp32 and in that order.
  */
