@@ -261,9 +261,15 @@ def latent_dequant(rows: np.ndarray, dc: int, dr: int) -> np.ndarray:
 
 
 def sparse_mla_fp8(q, kv_rows, idx, start_pos: int, sm_scale: float, dc: int, dr: int):
-    """Sparse attention over an FP8 latent cache: the rows are decoded, then the
+    """Sparse attention over an FP8 latent cache.  The attention computes in bf16
+    (bf16 operands, fp32-or-wider softmax and accumulation), so each decoded row
+    enters it as a bf16 operand: decode, round to bf16 (nearest even), then the
     same fp64 attention as sparse_mla."""
-    return sparse_mla(q, latent_dequant(kv_rows, dc, dr), idx, start_pos, sm_scale, dc)
+    dec = latent_dequant(kv_rows, dc, dr)
+    b = dec.view(np.uint32).astype(np.uint64)
+    rounded = ((b + 0x7FFF + ((b >> 16) & 1)) >> 16) << 16    # bf16, nearest even (finite values)
+    dec_bf16 = rounded.astype(np.uint32).view(np.float32)
+    return sparse_mla(q, dec_bf16, idx, start_pos, sm_scale, dc)
 
 
 def weight_fold(w: float, H: int, q_scale: float, softmax_scale: float) -> np.float32:

@@ -72,14 +72,16 @@ def test_latent_blocks_are_independent():
     assert np.array_equal(s1[:, 1], s0[:, 1] * np.float32(8.0))
 
 
-def test_sparse_attention_over_fp8_rows_is_attention_over_decoded_rows():
+def test_sparse_attention_over_fp8_rows_is_attention_over_decoded_bf16_rows():
     rng = np.random.default_rng(54)
     q = rng.standard_normal((1, 2, 8, 576)).astype(np.float32)
     kv = rng.standard_normal((1, 300, 576)).astype(np.float32)
     idx = np.sort(rng.permutation(300)[:40]).astype(np.int32).reshape(1, 1, 40).repeat(2, axis=1)
     rows = oracle.latent_quant(kv, 512)
     o8, l8 = oracle.sparse_mla_fp8(q, rows, idx, 299, 576 ** -0.5, 512, 64)
-    od, ld = oracle.sparse_mla(q, oracle.latent_dequant(rows, 512, 64), idx, 299, 576 ** -0.5, 512)
+    # the decoded rows enter the bf16 attention as bf16 operands (torch's rounding)
+    dec = torch.from_numpy(oracle.latent_dequant(rows, 512, 64)).to(torch.bfloat16).float().numpy()
+    od, ld = oracle.sparse_mla(q, dec, idx, 299, 576 ** -0.5, 512)
     assert np.array_equal(o8, od) and np.array_equal(l8, ld)
     # and it tracks the unquantised attention to within the FP8 error
     o, _ = oracle.sparse_mla(q, kv, idx, 299, 576 ** -0.5, 512)
