@@ -392,10 +392,14 @@ def run_ours(args, wl, world, rank, local):
     peak, peak_kind = _peaks()
     stages = time_stages(dsa, wl, copies, iters=max(10, min(args.steps, 500)))
     t_score = stages["decode_index_scores"]
-    prefill = prologue = None
+    prefill = prologue = attn_fp8 = None
     if not args.no_prefill:
         prefill = time_prefill_scoring(dsa, measure_fp8_peak(sustained=False)["fp8_e4m3_tflops"])
         prologue = time_indexer_prologue(dsa, peak)
+    try:
+        attn_fp8 = time_sparse_mla_fp8(dsa, peak, wl)
+    except Exception as exc:                       # reported, never fatal to the main line
+        attn_fp8 = {"error": f"{type(exc).__name__}: {exc}"[:200]}
     # keys + scales of every cached token, plus the new tokens' fp32 queries,
     # weights and keys (the scores written are not algorithmic)
     score_bytes = wl.B * wl.T * (wl.D + 4) + wl.B * (wl.H * wl.D * 4 + wl.H * 4 + wl.D * 4)
@@ -429,6 +433,7 @@ def run_ours(args, wl, world, rank, local):
         "stage_us": {k: round(v * 1e6, 2) for k, v in stages.items()},
         "prefill_scoring": prefill,
         "indexer_prologue": prologue,
+        "sparse_mla_fp8": attn_fp8,
         "clocks": clk.summary(),
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -564,6 +569,50 @@ def time_indexer_prologue(dsa, peak_gbs, iters=20):
            "frac": nbytes / t / 1e9 / peak_gbs, "bound": "hbm"}
     del q, k, q_fp8, k_cache
     return out
+
+
+def time_sparse_mla_fp8(dsa, peak_gbs, wl, iters=32, sets=16):
+    """Sparse attention over the FP8 latent cache (656 B rows) at the decode
+    workload's sizes: B queries x 2048 selected rows of a B x T cache.  The
+    selections rotate over `sets` independent random draws, so the rows gathered
+    across the timed iterations (sets x B x 2048 x 656 B) exceed L2.  Algorithmic
+    bytes per call: the FP8 rows gathered, the bf16 queries and outputs."""
+    B, T, Hq, dc, dr, k = wl.B, wl.T, wl.Hq, wl.dc, wl.dr, wl.topk
+    g = torch.Generator(device="cuda").manual_seed(wl.seed(2))
+    rb = dsa.dsa_latent_row_bytes(dc, dr)
+    cache = torch.empty(B, T, rb, dtype=torch.uint8, device="cuda")
+    for b in range(B):                                   # quantise one sequence at a time
+        kv = torch.randn(1, T, dc + dr, device="cuda", generator=g).to(torch.bfloat16)
+        dsa.dsa_latent_quant(kv, cache[b:b + 1], dc)
+        del kv
+    q = torch.randn(B, 1, Hq, dc + dr, device="cuda", generator=g).to(torch.bfloat16)
+    idxs = [torch.stack([torch.randperm(T, device="cuda", generator=g)[:k] for _ in range(B)])
+            .to(torch.int32).reshape(B, 1, k).contiguous() for _ in range(sets)]
+    out = torch.empty(B, 1, Hq, dc, dtype=torch.bfloat16, device="cuda")
+    lse = torch.empty(B, 1, Hq, dtype=torch.float32, device="cuda")
+    ws = torch.empty(dsa.dsa_sparse_mla_attn_fp8_workspace_size(B, 1, Hq, dc, dr, k),
+                     dtype=torch.uint8, device="cuda")
+
+    def one(i):
+        dsa.dsa_sparse_mla_attn_fp8(q, cache, idxs[i % sets], T - 1, wl.sm_scale, dc, out, lse, ws)
+
+    for i in range(3):
+        one(i)
+    torch.cuda.synchronize()
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0.record()
+    for i in range(iters):
+        one(i)
+    t1.record()
+    t1.synchronize()
+    t = t0.elapsed_time(t1) * 1e-3 / iters
+    nbytes = B * k * rb + B * Hq * (dc + dr) * 2 + B * Hq * dc * 2
+    res = {"workload": f"{wl.name}_fp8_latent", "rows": B * k, "row_bytes": rb, "bytes": nbytes,
+           "us": t * 1e6, "achieved_gbs": nbytes / t / 1e9, "peak_gbs": peak_gbs,
+           "frac": nbytes / t / 1e9 / peak_gbs, "bound": "hbm",
+           "note": "decode pass to bf16 rows in the workspace, then the bf16 sparse attention"}
+    del cache, idxs, ws
+    return res
 
 
 def measure_fp8_peak(n=8192, iters=20, sustained=True):

@@ -142,6 +142,49 @@ dsa_status dsa_indexer_prologue(const void *q, const void *k, dsa_dtype x_dtype,
                                 float *k_scale, dsa_stream_t stream);
 
 /*
+ * The FP8 latent cache ("DeepSeek Sparse Attention, one decode step in one
+ * layer (V3.2 sizes)": latents stored as "FP8 + bf16 RoPE", 656 B per row).
+ * Row layout, latent_row_bytes(dc, dr) = dc + 4*dc/128 + 2*dr bytes:
+ *   [dc e4m3 codes | dc/128 fp32 scales | dr bf16 rotary values]
+ * The latent part is quantised in blocks of 128 exactly as act_quant does
+ * (scale = max(amax, 1e-4) / 448, code = e4m3_rn_satfinite(x / scale), both
+ * divisions correctly rounded); the rotary part is rounded to bf16 (nearest
+ * even).  Supported: dc in {128, 256, 384, 512}, dr a multiple of 8 up to 64,
+ * dc + dr <= 576 (else DSA_ERR_UNSUPPORTED).
+ */
+int64_t dsa_latent_row_bytes(int dc, int dr);
+
+/*
+ * Quantise latent rows into the FP8 cache layout above.
+ *   kv   [n_rows, n_vec, dc + dr] F32 or BF16 (x_dtype), contiguous, 4-byte aligned
+ *   out  row (r, v) -> out + r * out_row_stride + v * latent_row_bytes(dc, dr)
+ * A cache append at start_pos: kv = new rows [B, S, dc + dr], n_rows = B, n_vec = S,
+ * out = cache + start_pos * row_bytes, out_row_stride = t_max * row_bytes.
+ * out and out_row_stride must be multiples of 4.
+ */
+dsa_status dsa_latent_quant(const void *kv, dsa_dtype x_dtype, int64_t n_rows, int64_t n_vec,
+                            int dc, int dr, uint8_t *out, int64_t out_row_stride,
+                            dsa_stream_t stream);
+
+/*
+ * Sparse latent attention (as dsa_sparse_mla_attn, bf16) over the FP8 latent
+ * cache kv_fp8 [B, t_max, latent_row_bytes(dc, dr)].  Each query row's selected
+ * rows are decoded (code * block scale, rounded to bf16; rotary part as
+ * stored) into the workspace, then attended with the bf16 sparse attention.
+ *   q    [B,S,Hq,dc+dr] bf16 (16-byte aligned), idx [B,S,k] int32 (-1 = empty)
+ *   out  [B,S,Hq,dc] bf16 (16-byte aligned), lse [B,S,Hq] fp32 or NULL
+ * Workspace: dsa_sparse_mla_attn_fp8_workspace_size bytes (16-byte aligned),
+ * else DSA_ERR_WORKSPACE.  Masking as dsa_sparse_mla_attn (indices > start_pos + s
+ * and -1 slots are skipped; indices >= t_max set DSA_ERR_DEVICE).
+ */
+size_t dsa_sparse_mla_attn_fp8_workspace_size(int B, int S, int Hq, int dc, int dr, int k);
+dsa_status dsa_sparse_mla_attn_fp8(const void *q, const uint8_t *kv_fp8, int64_t t_max,
+                                   const int32_t *idx, int B, int S, int Hq, int dc, int dr,
+                                   int k, int64_t start_pos, float sm_scale, void *out,
+                                   float *lse, void *workspace, size_t workspace_bytes,
+                                   dsa_stream_t stream);
+
+/*
  * fp8_index with the weight fold and the additive causal mask
  * (Indexer.forward; mask from Transformer.forward; formula from the diagram):
  *   w'[b,s,h]  = fp32(fp32(fp32(w * fp32(H^-1/2)) * q_scale) * softmax_scale)

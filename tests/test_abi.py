@@ -91,6 +91,34 @@ def test_indexer_prologue_argument_checks(dsa):
     assert call(S=0) == dsa.DSA_OK
 
 
+def test_latent_fp8_argument_checks(dsa):
+    L = dsa._lib
+    assert L.dsa_latent_row_bytes(512, 64) == 656
+    assert L.dsa_latent_quant(FAKE, 1, 1, 8, 500, 64, FAKE, 0, NULL) == dsa.DSA_ERR_UNSUPPORTED
+    assert L.dsa_latent_quant(FAKE, 1, 1, 8, 512, 72, FAKE, 0, NULL) == dsa.DSA_ERR_UNSUPPORTED
+    assert L.dsa_latent_quant(FAKE, 9, 1, 8, 512, 64, FAKE, 0, NULL) == dsa.DSA_ERR_INVALID_ARG
+    assert L.dsa_latent_quant(NULL, 1, 1, 8, 512, 64, FAKE, 0, NULL) == dsa.DSA_ERR_INVALID_ARG
+    # cache append with a row stride shorter than the rows it must hold
+    assert L.dsa_latent_quant(FAKE, 1, 2, 8, 512, 64, FAKE, 656, NULL) == dsa.DSA_ERR_INVALID_ARG
+    assert L.dsa_latent_quant(NULL, 1, 1, 0, 512, 64, NULL, 0, NULL) == dsa.DSA_OK
+    assert L.dsa_sparse_mla_attn_fp8_workspace_size(1, 1, 128, 500, 64, 16) == 0
+    need = L.dsa_sparse_mla_attn_fp8_workspace_size(1, 1, 128, 512, 64, 16)
+    assert need >= 16 * 576 * 2 + 16 * 4
+
+    def attn(q=FAKE, kv=FAKE, t_max=100, idx=FAKE, B=1, S=1, k=16, sp=99, out=FAKE, ws=FAKE,
+             wsb=None):
+        return L.dsa_sparse_mla_attn_fp8(q, kv, t_max, idx, B, S, 128, 512, 64, k, sp, 0.04, out,
+                                         NULL, ws, need if wsb is None else wsb, NULL)
+
+    assert attn(sp=100) == dsa.DSA_ERR_INVALID_ARG          # start_pos + S > t_max
+    assert attn(q=ODD) == dsa.DSA_ERR_INVALID_ARG
+    assert attn(idx=NULL) == dsa.DSA_ERR_INVALID_ARG
+    assert attn(k=0) == dsa.DSA_ERR_INVALID_ARG
+    assert attn(wsb=need - 1) == dsa.DSA_ERR_WORKSPACE
+    assert attn(ws=NULL) == dsa.DSA_ERR_WORKSPACE
+    assert attn(B=0) == dsa.DSA_OK
+
+
 def test_index_scores_argument_checks(dsa):
     L = dsa._lib
     args = lambda **kw: [kw.get("q", FAKE), FAKE, FAKE, kw.get("k", FAKE), FAKE,

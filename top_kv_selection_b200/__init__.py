@@ -39,6 +39,11 @@ _SIGNATURES = {
     "dsa_indexer_quant": ([_P, _i32, _i64, _i64, _i32, _P, _i64, _P, _i64, _P], _i32),
     "dsa_indexer_prologue": ([_P, _P, _i32, _i32, _i32, _i32, _i32, _i32, _P, _i32, _i64, _i64,
                               _P, _P, _P, _P, _P], _i32),
+    "dsa_latent_row_bytes": ([_i32, _i32], _i64),
+    "dsa_latent_quant": ([_P, _i32, _i64, _i64, _i32, _i32, _P, _i64, _P], _i32),
+    "dsa_sparse_mla_attn_fp8_workspace_size": ([_i32, _i32, _i32, _i32, _i32, _i32], _sz),
+    "dsa_sparse_mla_attn_fp8": ([_P, _P, _i64, _P, _i32, _i32, _i32, _i32, _i32, _i32, _i64,
+                                 _f32, _P, _P, _P, _sz, _P], _i32),
     "dsa_index_scores": ([_P, _P, _P, _P, _P, _i64, _i32, _i32, _i32, _i32, _i64, _i64, _f32,
                           _P, _P], _i32),
     "dsa_decode_index_scores": ([_P, _P, _P, _P, _P, _i64, _i32, _i32, _i32, _i64, _f32, _P, _P],
@@ -144,6 +149,41 @@ def dsa_indexer_prologue(q: torch.Tensor | None, k: torch.Tensor, rope_cs: torch
     _check("dsa_indexer_prologue", _lib.dsa_indexer_prologue(
         _ptr(q), _ptr(k), _dtype(k), B, S, H, d, rope_dim, _ptr(rope_cs), scale_fmt, start_pos,
         t_max, _ptr(q_fp8), _ptr(q_scale), _ptr(k_cache), _ptr(k_scale), _stream(stream)))
+
+
+def dsa_latent_row_bytes(dc: int, dr: int) -> int:
+    return int(_lib.dsa_latent_row_bytes(dc, dr))
+
+
+def dsa_latent_quant(kv: torch.Tensor, out: torch.Tensor, dc: int, n_rows: int = 1,
+                     out_row_stride: int = 0, stream=None) -> None:
+    """FP8 latent rows of kv ([n_rows, n_vec, dc + dr] as laid out) into out (uint8 rows of
+    dsa_latent_row_bytes bytes; a cache append passes a view at the cache row and the cache
+    row stride in bytes)."""
+    dqk = kv.shape[-1]
+    n_vec = kv.numel() // dqk // n_rows
+    _check("dsa_latent_quant", _lib.dsa_latent_quant(
+        _ptr(kv), _dtype(kv), n_rows, n_vec, dc, dqk - dc, ctypes.c_void_p(out.data_ptr()),
+        out_row_stride, _stream(stream)))
+
+
+def dsa_sparse_mla_attn_fp8_workspace_size(B: int, S: int, Hq: int, dc: int, dr: int,
+                                           k: int) -> int:
+    return int(_lib.dsa_sparse_mla_attn_fp8_workspace_size(B, S, Hq, dc, dr, k))
+
+
+def dsa_sparse_mla_attn_fp8(q: torch.Tensor, kv_fp8: torch.Tensor, idx: torch.Tensor,
+                            start_pos: int, sm_scale: float, dc: int, out: torch.Tensor,
+                            lse: torch.Tensor | None, workspace: torch.Tensor,
+                            stream=None) -> None:
+    """q [B,S,Hq,dc+dr] bf16, kv_fp8 [B,t_max,row_bytes] uint8, idx [B,S,k] int32 ->
+    out [B,S,Hq,dc] bf16, lse [B,S,Hq] fp32."""
+    B, S, Hq, dqk = q.shape
+    t_max = kv_fp8.shape[1]
+    k = idx.shape[-1]
+    _check("dsa_sparse_mla_attn_fp8", _lib.dsa_sparse_mla_attn_fp8(
+        _ptr(q), _ptr(kv_fp8), t_max, _ptr(idx), B, S, Hq, dc, dqk - dc, k, start_pos,
+        sm_scale, _ptr(out), _ptr(lse), _ptr(workspace), workspace.numel(), _stream(stream)))
 
 
 def dsa_index_scores(q_fp8: torch.Tensor, q_scale: torch.Tensor, w: torch.Tensor,
