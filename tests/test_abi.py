@@ -28,7 +28,8 @@ def header_functions():
 def test_header_declares_the_hot_path_entry_points():
     names = header_functions()
     for n in ("dsa_indexer_quant", "dsa_index_scores", "dsa_topk_select",
-              "dsa_sparse_mla_attn", "dsa_decode_step"):
+              "dsa_sparse_mla_attn", "dsa_decode_step", "dsa_decode_step_noalloc",
+              "dsa_indexer_prologue", "dsa_latent_quant", "dsa_sparse_mla_attn_fp8"):
         assert n in names
 
 
