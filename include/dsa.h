@@ -5,20 +5,21 @@
  * The path (lightning indexer, top-k token selection, sparse latent attention)
  * follows these pages:
  *   "DeepSeek-V3.2-Exp - Split indexer heads": the Indexer.forward excerpt:
- *       rotate_activation, act_quant,
- *       the key-cache write, the weight fold, fp8_index, the additive mask and
- *       topk(min(index_topk, end_pos)).
+ *       the non-interleaved rotary embedding of q_pe / k_pe, rotate_activation,
+ *       act_quant (with its scale_fmt), the key-cache write, the weight fold,
+ *       fp8_index, the additive mask and topk(min(index_topk, end_pos)).
  *   "DeepSeek-V3.2-Exp - Causal mask": Transformer.forward (mask =
  *       full(-inf).triu_(1) when seqlen > 1) and the MLA prefill excerpt
  *       (index_mask = full(-inf).scatter_(topk, 0) + mask).
  *   "DeepSeek Sparse Attention, one decode step in one layer (V3.2 sizes)"
  *       diagram: I(t,s) = sum_j w_j ReLU(q_j . k_s), k = 2048, core attention
- *       in MQA mode over the gathered latents, each latent row key and value.
+ *       in MQA mode over the gathered latents, each latent row key and value,
+ *       latents cached as "FP8 + bf16 RoPE" in 656-byte rows.
  *
  * Conventions for every entry point:
  *   - Memory: every tensor argument is a caller-owned DEVICE pointer, row-major
- *     and contiguous with the layout stated below, 16-byte aligned.  The
- *     library allocates nothing.  Scratch memory is passed in as `workspace`
+ *     and contiguous with the layout stated below, 16-byte aligned unless the
+ *     entry point states a weaker alignment.  The library allocates nothing.  Scratch memory is passed in as `workspace`
  *     (size from the matching *_workspace_size call); it need not be zeroed.
  *   - Execution: every call only enqueues kernels on `stream` and returns; it
  *     never synchronises.  Calls on one stream run in order.  Two calls that
