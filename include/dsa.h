@@ -59,7 +59,11 @@ typedef enum dsa_status {
 
 typedef enum dsa_dtype {
     DSA_F32 = 0,               /* IEEE binary32 */
-    DSA_BF16 = 1               /* bfloat16      */
+    DSA_BF16 = 1,              /* bfloat16      */
+    /* The FP8 latent cache layout of dsa_latent_row_bytes (656-byte rows at
+     * the V3.2 sizes).  Accepted only by dsa_decode_step(_noalloc) as the
+     * kv_cache type; q_mla and out are then bf16. */
+    DSA_FP8_LATENT = 2
 } dsa_dtype;
 
 /* act_quant's scale_fmt: a plain fp32 scale, or ue8m0 (a bare power of two). */
@@ -270,6 +274,9 @@ dsa_status dsa_sparse_mla_attn(const void *q, const void *kv_cache, int64_t t_ma
  *   kv_cache [B,t_max,dc+dr] (dt): row T-1 must already hold the new latent
  *   q_mla [B,Hq,dc+dr] (dt)   idx [B,K] int32   out [B,Hq,dc] (dt)
  *   lse [B,Hq] fp32 or NULL
+ * dt = DSA_FP8_LATENT: kv_cache is the FP8 latent cache [B, t_max,
+ * dsa_latent_row_bytes(dc, dr)] (16-byte aligned), attended as
+ * dsa_sparse_mla_attn_fp8 does; q_mla and out are bf16.
  */
 size_t dsa_decode_step_workspace_size(int B, int H, int D, int64_t T, int index_topk, int Hq,
                                       int dc, int dr, dsa_dtype dt);

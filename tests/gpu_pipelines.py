@@ -5,11 +5,13 @@ import torch
 import workloads
 
 
-def decode_batch(dsa, wl, T=None, B=None, t_max=None):
+def decode_batch(dsa, wl, T=None, B=None, t_max=None, fp8_latent=False):
     """Build a decode step's device state for sequences 0..B-1 and run it once.
 
     The cache holds positions 0..T-2 quantised by dsa_indexer_quant; the step
-    appends the new key at T-1.  Returns (host inputs per sequence, device results).
+    appends the new key at T-1.  With fp8_latent the latent rows are quantised
+    by dsa_latent_quant into the FP8 latent cache, which the step attends over.
+    Returns (host inputs per sequence, device results).
     """
     T = wl.T if T is None else T
     B = wl.B if B is None else B
@@ -28,12 +30,18 @@ def decode_batch(dsa, wl, T=None, B=None, t_max=None):
         if T > 1:
             dsa.dsa_indexer_quant(s["keys"][:T - 1].to(dev), k_cache[b], k_scale[b])
         kv[b, :T] = s["kv"].to(dev)
+    kv_dt = dsa.DSA_BF16 if dt == torch.bfloat16 else dsa.DSA_F32
+    if fp8_latent:
+        rb = dsa.dsa_latent_row_bytes(wl.dc, wl.dr)
+        kv8 = torch.zeros(B, t_max, rb, dtype=torch.uint8, device=dev)
+        dsa.dsa_latent_quant(kv, kv8, wl.dc, n_rows=B, out_row_stride=t_max * rb)
+        kv, kv_dt = kv8, dsa.DSA_FP8_LATENT
     K = min(wl.topk, T)
     idx = torch.empty(B, K, dtype=torch.int32, device=dev)
     out = torch.empty(B, wl.Hq, wl.dc, dtype=dt, device=dev)
     lse = torch.empty(B, wl.Hq, dtype=torch.float32, device=dev)
     need = dsa.dsa_decode_step_workspace_size(B, wl.H, wl.D, T, wl.topk, wl.Hq, wl.dc, wl.dr,
-                                              dsa.DSA_BF16 if dt == torch.bfloat16 else dsa.DSA_F32)
+                                              kv_dt)
     ws = torch.empty(need, dtype=torch.uint8, device=dev)
     state = dict(q_idx=q_idx, w=w, k_new=k_new, k_cache=k_cache, k_scale=k_scale, kv=kv,
                  q_mla=q_mla, idx=idx, out=out, lse=lse, ws=ws, T=T)

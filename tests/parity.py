@@ -9,12 +9,16 @@ Tolerances:
     the other must have an oracle score within the score tolerance of the
     oracle's k-th score (a boundary tie); the -1 padding must match exactly.
   * attention: 2e-2 absolute in bf16, 1e-4 absolute in fp32 test mode; lse 1e-3
-    absolute (bf16 inputs) / 1e-5 (fp32).
+    absolute (bf16 inputs) / 1e-5 (fp32).  In bf16 the error must also stay
+    within 2e-2 of the reference's root-mean-square output: the outputs are
+    convex mixes of ~N(0,1) rows, so their rms is far below 1 and the absolute
+    bound alone would pass a lost tile of the value mix.
 """
 import numpy as np
 
 SCORE_RTOL = 1e-3
 ATTN_ATOL = {"bf16": 2e-2, "f32": 1e-4}
+ATTN_RMS_RTOL = {"bf16": 2e-2}
 LSE_ATOL = {"bf16": 1e-3, "f32": 1e-5}
 
 
@@ -59,6 +63,10 @@ def assert_attention_close(gpu_out, ref_out, dtype, gpu_lse=None, ref_lse=None):
     ref_out = np.asarray(ref_out, dtype=np.float64)
     err = np.abs(gpu_out - ref_out).max() if gpu_out.size else 0.0
     assert err <= ATTN_ATOL[dtype], f"attention max abs err {err}"
+    if dtype in ATTN_RMS_RTOL and gpu_out.size:
+        rms = float(np.sqrt(np.mean(ref_out ** 2)))
+        assert err <= ATTN_RMS_RTOL[dtype] * rms + 1e-30, (
+            f"attention max abs err {err} vs rms {rms} ({err / max(rms, 1e-30):.3g} of rms)")
     if gpu_lse is not None:
         gl = np.asarray(gpu_lse, dtype=np.float64)
         rl = np.asarray(ref_lse, dtype=np.float64)

@@ -103,16 +103,23 @@ def test_latent_fp8_argument_checks(dsa):
     assert L.dsa_latent_quant(FAKE, 1, 2, 8, 512, 64, FAKE, 656, NULL) == dsa.DSA_ERR_INVALID_ARG
     assert L.dsa_latent_quant(NULL, 1, 1, 0, 512, 64, NULL, 0, NULL) == dsa.DSA_OK
     assert L.dsa_sparse_mla_attn_fp8_workspace_size(1, 1, 128, 500, 64, 16) == 0
-    need = L.dsa_sparse_mla_attn_fp8_workspace_size(1, 1, 128, 512, 64, 16)
-    assert need >= 16 * 576 * 2 + 16 * 4
+    # V3.2 shapes decode in the gather: a workspace only for split partials
+    # (none when one unit covers the row), never for decoded rows
+    assert L.dsa_sparse_mla_attn_fp8_workspace_size(1, 1, 128, 512, 64, 16) == 0
+    need = L.dsa_sparse_mla_attn_fp8_workspace_size(1, 1, 128, 512, 64, 2048)
+    assert need > 0
+    # other shapes decode into the workspace first
+    assert (L.dsa_sparse_mla_attn_fp8_workspace_size(1, 1, 16, 256, 32, 16) >=
+            16 * 288 * 2 + 16 * 4)
 
-    def attn(q=FAKE, kv=FAKE, t_max=100, idx=FAKE, B=1, S=1, k=16, sp=99, out=FAKE, ws=FAKE,
+    def attn(q=FAKE, kv=FAKE, t_max=3000, idx=FAKE, B=1, S=1, k=2048, sp=99, out=FAKE, ws=FAKE,
              wsb=None):
         return L.dsa_sparse_mla_attn_fp8(q, kv, t_max, idx, B, S, 128, 512, 64, k, sp, 0.04, out,
                                          NULL, ws, need if wsb is None else wsb, NULL)
 
-    assert attn(sp=100) == dsa.DSA_ERR_INVALID_ARG          # start_pos + S > t_max
+    assert attn(sp=3000) == dsa.DSA_ERR_INVALID_ARG         # start_pos + S > t_max
     assert attn(q=ODD) == dsa.DSA_ERR_INVALID_ARG
+    assert attn(kv=ODD) == dsa.DSA_ERR_INVALID_ARG          # 16-byte rows for the V3.2 shapes
     assert attn(idx=NULL) == dsa.DSA_ERR_INVALID_ARG
     assert attn(k=0) == dsa.DSA_ERR_INVALID_ARG
     assert attn(wsb=need - 1) == dsa.DSA_ERR_WORKSPACE

@@ -36,7 +36,7 @@ def _check_sequence(wl, seq, state, b, T):
     (1, 5000, 2),      # V3.2 shapes, ragged context
     (1, 1, 1),         # a single token: K = 1
     (1, 2048, 2),      # T == k: every position
-    (1, 700, 1),       # T < k: padded with -1? no: K = min(k, T) = T slots, all filled
+    (1, 700, 1),       # T < k: K = min(k, T) = T slots, all filled
     (0, 300, 2),       # tiny heads, fp32 test mode
 ])
 def test_decode_step_small(dsa, cfg, T, B):
@@ -89,3 +89,28 @@ def test_decode_step_deterministic(dsa):
     run_decode(dsa, wl, st)
     torch.cuda.synchronize()
     assert torch.equal(idx1, st["idx"]) and torch.equal(out1, st["out"])
+
+
+@pytest.mark.parametrize("T,B", [(5000, 2), (131072, 8)])
+def test_decode_step_fp8_latent_cache(dsa, T, B):
+    """The decode step over the FP8 latent cache (656-byte rows): the selection
+    is the bf16 step's, the attention matches the oracle's attention over its
+    own FP8 rows at the oracle's selection."""
+    wl = workloads.WORKLOADS[1 if T < 100000 else 4]
+    seqs, st = decode_batch(dsa, wl, T=T, B=B, fp8_latent=True)
+    rows = st["kv"].cpu().numpy()
+    for b in (0, B - 1):
+        seq = seqs[b]
+        k_fp8, k_sc = oracle.indexer_quant(seq["keys"].numpy())
+        q_fp8, q_sc = oracle.indexer_quant(seq["q_idx"].numpy())
+        sc = oracle.index_scores(q_fp8[None, None], q_sc[None, None], seq["w"].numpy()[None, None],
+                                 k_fp8[None], k_sc[None], start_pos=T - 1, T=T,
+                                 softmax_scale=wl.softmax_scale_idx)
+        ref_idx = oracle.topk_select(sc, start_pos=T - 1, k=wl.topk)
+        assert_selection_matches(st["idx"][b].cpu().numpy(), ref_idx[0, 0], sc[0, 0])
+        assert np.array_equal(rows[b, :T], oracle.latent_quant(seq["kv"].float().numpy(), wl.dc))
+        ref, ref_lse = oracle.sparse_mla_fp8(seq["q_mla"].float().numpy()[None, None], rows[b:b + 1],
+                                             ref_idx, T - 1, wl.sm_scale, wl.dc, wl.dr)
+        assert_attention_close(st["out"][b].float().cpu().numpy(), ref[0, 0], "bf16",
+                               st["lse"][b].cpu().numpy(), ref_lse[0, 0])
+    assert dsa.dsa_get_device_error() == 0

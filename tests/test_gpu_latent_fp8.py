@@ -1,7 +1,8 @@
 """The FP8 latent cache on the GPU against the oracle: row quantisation
 bit-identical (codes, block scales, bf16 rotary part), and sparse attention
-over FP8 rows within the bf16 attention tolerance (the GPU rounds each decoded
-value to bf16 before the attention; the oracle keeps it in fp32)."""
+over FP8 rows within the bf16 attention tolerance.  Both sides decode a row
+as code * block scale rounded to bf16 (the attention's operand type), so the
+decoded operands are identical and only the attention's arithmetic differs."""
 import numpy as np
 import pytest
 import torch
@@ -50,6 +51,8 @@ def test_latent_quant_matches_oracle(dsa, dtype, dc, dr):
     (1, 5, 2000, 512, 1500, 1.0),         # query rows with their own causal limits
     (3, 1, 300, 2048, 299, 1.0),          # fewer cached rows than k
     (1, 1, 5000, 1, 4999, 1.0),           # a single selected row
+    (8, 1, 4096, 2048, 4095, 1.0),        # 256-row units (the decode bench's B)
+    (5, 1, 3000, 2048, 2999, 0.8),        # 192-row units
 ])
 def test_sparse_mla_fp8_matches_oracle(dsa, B, S, t_max, k, sp, fill):
     Hq, dc, dr = 128, 512, 64
@@ -86,3 +89,23 @@ def test_sparse_mla_fp8_empty_rows(dsa):
     dsa.dsa_sparse_mla_attn_fp8(q, cache, idx, t_max - 1, 0.04, dc, out, lse, ws)
     torch.cuda.synchronize()
     assert torch.all(out == 0) and torch.all(torch.isinf(lse) & (lse < 0))
+
+
+def test_sparse_mla_fp8_other_shape_two_launch_path(dsa):
+    """dc = 256: decoded into the workspace, then the bf16 attention."""
+    B, S, Hq, dc, dr, t_max, k, sp = 1, 2, 16, 256, 32, 800, 128, 700
+    g = torch.Generator().manual_seed(9)
+    q = torch.randn(B, S, Hq, dc + dr, generator=g).to(torch.bfloat16)
+    kv = torch.randn(B, t_max, dc + dr, generator=g).to(torch.bfloat16)
+    idx = workloads.random_indices(B, S, k, t_max, sp, seed=9, fill=0.9)
+    cache = _gpu_rows(dsa, kv, dc)
+    rows = cache.cpu().numpy()
+    sm = (dc + dr) ** -0.5
+    ws = torch.empty(max(dsa.dsa_sparse_mla_attn_fp8_workspace_size(B, S, Hq, dc, dr, k), 1),
+                     dtype=torch.uint8, device="cuda")
+    out = torch.empty(B, S, Hq, dc, dtype=torch.bfloat16, device="cuda")
+    lse = torch.empty(B, S, Hq, dtype=torch.float32, device="cuda")
+    dsa.dsa_sparse_mla_attn_fp8(q.cuda(), cache, idx.cuda(), sp, sm, dc, out, lse, ws)
+    torch.cuda.synchronize()
+    ref, ref_lse = oracle.sparse_mla_fp8(q.float().numpy(), rows, idx.numpy(), sp, sm, dc, dr)
+    assert_attention_close(out.float().cpu().numpy(), ref, "bf16", lse.cpu().numpy(), ref_lse)

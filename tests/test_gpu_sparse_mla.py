@@ -44,6 +44,9 @@ def _gpu(dsa, q, kv, idx, sp, sm, dc):
     (3, 1, 128, 512, 64, 300, 2048, 299, "bf16", 1.0),  # fewer rows than k
     (1, 1, 128, 512, 64, 5000, 1, 4999, "bf16", 1.0),   # a single selected row
     (1, 3, 128, 512, 64, 4096, 2048, 3000, "f32", 1.0),  # V3.2 shape in fp32 test mode
+    (4, 1, 128, 512, 64, 4096, 2048, 4095, "bf16", 1.0),  # 128-row units
+    (5, 1, 128, 512, 64, 3000, 2048, 2999, "bf16", 0.8),  # 192-row units, -1 slots
+    (8, 1, 128, 512, 64, 4096, 2048, 4095, "bf16", 1.0),  # 256-row units (the decode bench's B)
 ])
 def test_sparse_mla_matches_oracle(dsa, B, S, Hq, dc, dr, t_max, k, sp, dtype, fill):
     tdt = torch.bfloat16 if dtype == "bf16" else torch.float32

@@ -25,7 +25,7 @@ _lib = ctypes.CDLL(LIB_PATH)
 
 DSA_OK, DSA_ERR_INVALID_ARG, DSA_ERR_UNSUPPORTED, DSA_ERR_CUDA = 0, 1, 2, 3
 DSA_ERR_TIMEOUT, DSA_ERR_DEVICE, DSA_ERR_WORKSPACE = 4, 5, 6
-DSA_F32, DSA_BF16 = 0, 1
+DSA_F32, DSA_BF16, DSA_FP8_LATENT = 0, 1, 2
 DSA_SCALE_F32, DSA_SCALE_UE8M0 = 0, 1
 DSA_NOALLOC_SCRATCH_BYTES = 32 << 20
 
@@ -110,6 +110,11 @@ def _dtype(t: torch.Tensor) -> int:
     if t.dtype == torch.bfloat16:
         return DSA_BF16
     raise ValueError(f"unsupported dtype {t.dtype}")
+
+
+def _kv_dtype(kv_cache: torch.Tensor, q_mla: torch.Tensor) -> int:
+    """The decode step's cache type: uint8 rows are the FP8 latent cache."""
+    return DSA_FP8_LATENT if kv_cache.dtype == torch.uint8 else _dtype(q_mla)
 
 
 def dsa_get_device_error(stream=None) -> int:
@@ -254,8 +259,9 @@ def dsa_decode_step(q_idx: torch.Tensor, w: torch.Tensor, k_new: torch.Tensor,
                     sm_scale: float, idx: torch.Tensor, out: torch.Tensor,
                     lse: torch.Tensor | None, workspace: torch.Tensor, stream=None) -> None:
     """One decode step (see include/dsa.h): q_idx [B,H,D], w [B,H], k_new [B,D] fp32;
-    k_cache [B,t_max,D] uint8, k_scale [B,t_max]; kv_cache [B,t_max,dc+dr];
-    q_mla [B,Hq,dc+dr]; idx [B,K]; out [B,Hq,dc]."""
+    k_cache [B,t_max,D] uint8, k_scale [B,t_max]; kv_cache [B,t_max,dc+dr] (or uint8
+    [B,t_max,row_bytes]: the FP8 latent cache, q_mla bf16); q_mla [B,Hq,dc+dr];
+    idx [B,K]; out [B,Hq,dc]."""
     B, H, D = q_idx.shape
     Hq, dqk = q_mla.shape[1], q_mla.shape[2]
     dc = out.shape[-1]
@@ -263,7 +269,7 @@ def dsa_decode_step(q_idx: torch.Tensor, w: torch.Tensor, k_new: torch.Tensor,
     _check("dsa_decode_step", _lib.dsa_decode_step(
         _ptr(q_idx), _ptr(w), _ptr(k_new), _ptr(k_cache), _ptr(k_scale), t_max, _ptr(kv_cache),
         _ptr(q_mla), B, H, D, Hq, dc, dqk - dc, T, index_topk, softmax_scale, sm_scale,
-        _dtype(q_mla), _ptr(idx), _ptr(out), _ptr(lse), _ptr(workspace),
+        _kv_dtype(kv_cache, q_mla), _ptr(idx), _ptr(out), _ptr(lse), _ptr(workspace),
         workspace.numel() * workspace.element_size(), _stream(stream)))
 
 
@@ -282,4 +288,4 @@ def dsa_decode_step_noalloc(q_idx: torch.Tensor, w: torch.Tensor, k_new: torch.T
     _check("dsa_decode_step_noalloc", _lib.dsa_decode_step_noalloc(
         _ptr(q_idx), _ptr(w), _ptr(k_new), _ptr(k_cache), _ptr(k_scale), t_max, _ptr(kv_cache),
         _ptr(q_mla), B, H, D, Hq, dc, dqk - dc, T, index_topk, softmax_scale, sm_scale,
-        _dtype(q_mla), _ptr(idx), _ptr(out), _ptr(lse), _stream(stream)))
+        _kv_dtype(kv_cache, q_mla), _ptr(idx), _ptr(out), _ptr(lse), _stream(stream)))

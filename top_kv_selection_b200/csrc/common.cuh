@@ -112,6 +112,18 @@ size_t sparse_mla_tc_workspace_bytes(int B, int S, int k);
 dsa_status launch_sparse_mla_tc(const void *q, const void *kv, int64_t t_max, const int32_t *idx,
                                 int B, int S, int k, int64_t start_pos, float sm_scale, void *out,
                                 float *lse, void *ws, cudaStream_t stream);
+bool sparse_mla_fp8_tc_supported(int Hq, int dc, int dr, int k);
+dsa_status launch_sparse_mla_fp8_tc(const void *q, const uint8_t *kv8, int64_t t_max,
+                                    const int32_t *idx, int B, int S, int k, int64_t start_pos,
+                                    float sm_scale, void *out, float *lse, void *ws,
+                                    cudaStream_t stream);
+// FP8 latent cache (latent_fp8.cu): 656-byte rows at the V3.2 shapes
+bool latent_fp8_shape_ok(int dc, int dr);
+size_t sparse_mla_fp8_workspace_bytes(int B, int S, int Hq, int dc, int dr, int k);
+dsa_status launch_sparse_mla_fp8(const void *q, const uint8_t *kv_fp8, int64_t t_max,
+                                 const int32_t *idx, int B, int S, int Hq, int dc, int dr, int k,
+                                 int64_t start_pos, float sm_scale, void *out, float *lse,
+                                 void *workspace, cudaStream_t stream);
 dsa_status launch_sparse_mla(const void *q, const void *kv, int64_t t_max, const int32_t *idx,
                              int B, int S, int Hq, int dc, int dr, int k, int64_t start_pos,
                              float sm_scale, dsa_dtype dt, void *out, float *lse, void *ws,

@@ -32,7 +32,8 @@ DecodeWs carve(void *base, int B, int, int, int64_t T, int index_topk, int Hq, i
     w.scores = reinterpret_cast<float *>(take((size_t)B * T * sizeof(float)));
     w.topk_ws = take(topk_workspace_bytes(B, 1, T, index_topk));
     const int K = (int64_t)index_topk < T ? index_topk : (int)T;
-    w.attn_ws = take(sparse_mla_workspace_bytes(B, 1, Hq, dc, dr, K, dt));
+    w.attn_ws = take(dt == DSA_FP8_LATENT ? sparse_mla_fp8_workspace_bytes(B, 1, Hq, dc, dr, K)
+                                          : sparse_mla_workspace_bytes(B, 1, Hq, dc, dr, K, dt));
     w.total = off;
     return w;
 }
@@ -55,11 +56,12 @@ extern "C" dsa_status dsa_decode_step(const float *q_idx, const float *w, const 
                                       size_t workspace_bytes, dsa_stream_t stream) {
     if (B < 0 || H < 1 || Hq < 1 || index_topk < 1 || T < 1 || T > t_max || T > INT32_MAX)
         return DSA_ERR_INVALID_ARG;
-    if (dt != DSA_F32 && dt != DSA_BF16) return DSA_ERR_INVALID_ARG;
+    if (dt != DSA_F32 && dt != DSA_BF16 && dt != DSA_FP8_LATENT) return DSA_ERR_INVALID_ARG;
     if (D != 64 && D != 128) return DSA_ERR_UNSUPPORTED;
     if (H > 256) return DSA_ERR_UNSUPPORTED;
     if (dc == 0 || dc % 32 != 0 || dc > 512 || dr < 0 || dr % 8 != 0 || dc + dr > 576)
         return DSA_ERR_UNSUPPORTED;
+    if (dt == DSA_FP8_LATENT && !dsa::latent_fp8_shape_ok(dc, dr)) return DSA_ERR_UNSUPPORTED;
     if (B == 0) return DSA_OK;
     if (!q_idx || !w || !k_new || !k_cache || !k_scale || !kv_cache || !q_mla || !idx || !out)
         return DSA_ERR_INVALID_ARG;
@@ -79,6 +81,10 @@ extern "C" dsa_status dsa_decode_step(const float *q_idx, const float *w, const 
                                       s)) != DSA_OK)
         return st;
     const int K = (int64_t)index_topk < T ? index_topk : (int)T;
+    if (dt == DSA_FP8_LATENT)
+        return dsa::launch_sparse_mla_fp8(q_mla, static_cast<const uint8_t *>(kv_cache), t_max,
+                                          idx, B, 1, Hq, dc, dr, K, T - 1, sm_scale, out, lse,
+                                          ws.attn_ws, s);
     return dsa::launch_sparse_mla(q_mla, kv_cache, t_max, idx, B, 1, Hq, dc, dr, K, T - 1,
                                   sm_scale, dt, out, lse, ws.attn_ws, s);
 }

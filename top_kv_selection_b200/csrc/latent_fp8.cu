@@ -8,11 +8,13 @@
 // max(amax, 1e-4) / 448, code e4m3_rn_satfinite(x / scale), both divisions
 // correctly rounded), the rotary part is rounded to bf16.
 //
-// Attention over the FP8 cache runs in two launches: a gather pass decodes
-// each query row's selected rows (code * block scale, rounded to bf16; the
-// rotary part copied) into a workspace, one row per selection slot, and the
-// bf16 sparse attention of sparse_mla.cu / sparse_mla_tc.cu then attends over
-// it with every query row as its own sequence and slot j at position j.
+// Attention over the FP8 cache: at the V3.2 shapes (128 heads, 512 + 64) the
+// tensor-core kernel of sparse_mla_tc.cu decodes each latent chunk while
+// gathering it.  Other shapes run in two launches: a gather pass decodes each
+// query row's selected rows (code * block scale, rounded to bf16; the rotary
+// part copied) into a workspace, one row per selection slot, and the bf16
+// sparse attention of sparse_mla.cu then attends over it with every query row
+// as its own sequence and slot j at position j.
 #include <cuda_fp8.h>
 
 #include "common.cuh"
@@ -142,9 +144,15 @@ struct Fp8Ws {
     size_t total() const { return rows_bytes + idx_bytes + attn_bytes; }
 };
 
-Fp8Ws fp8_workspace(int B, int S, int Hq, int dc, int dr, int k) {
+Fp8Ws fp8_workspace(int B, int S, int Hq, int dc, int dr, int k, bool tc) {
     const int64_t rows = (int64_t)B * S;
     Fp8Ws w;
+    if (tc) {
+        w.rows_bytes = 0;
+        w.idx_bytes = 0;
+        w.attn_bytes = sparse_mla_tc_workspace_bytes(B, S, k);
+        return w;
+    }
     w.rows_bytes = align_up((size_t)rows * k * (dc + dr) * sizeof(__nv_bfloat16), 256);
     w.idx_bytes = align_up((size_t)rows * k * sizeof(int32_t), 256);
     w.attn_bytes = sparse_mla_workspace_bytes((int)rows, 1, Hq, dc, dr, k, DSA_BF16);
@@ -152,6 +160,37 @@ Fp8Ws fp8_workspace(int B, int S, int Hq, int dc, int dr, int k) {
 }
 
 }  // namespace
+
+bool latent_fp8_shape_ok(int dc, int dr) { return fp8_shape_ok(dc, dr); }
+
+size_t sparse_mla_fp8_workspace_bytes(int B, int S, int Hq, int dc, int dr, int k) {
+    return fp8_workspace(B, S, Hq, dc, dr, k, sparse_mla_fp8_tc_supported(Hq, dc, dr, k)).total();
+}
+
+dsa_status launch_sparse_mla_fp8(const void *q, const uint8_t *kv_fp8, int64_t t_max,
+                                 const int32_t *idx, int B, int S, int Hq, int dc, int dr, int k,
+                                 int64_t start_pos, float sm_scale, void *out, float *lse,
+                                 void *workspace, cudaStream_t st) {
+    // the decode-in-gather kernel reads rows with 16-byte loads (the entry
+    // point requires a 16-byte aligned cache for these shapes)
+    if (sparse_mla_fp8_tc_supported(Hq, dc, dr, k))
+        return launch_sparse_mla_fp8_tc(q, kv_fp8, t_max, idx, B, S, k, start_pos, sm_scale, out,
+                                        lse, workspace, st);
+    const Fp8Ws w = fp8_workspace(B, S, Hq, dc, dr, k, false);
+    char *ws = static_cast<char *>(workspace);
+    __nv_bfloat16 *g_rows = reinterpret_cast<__nv_bfloat16 *>(ws);
+    int32_t *g_idx = reinterpret_cast<int32_t *>(ws + w.rows_bytes);
+    void *attn_ws = w.attn_bytes ? ws + w.rows_bytes + w.idx_bytes : nullptr;
+    const int64_t rows = (int64_t)B * S;
+    latent_gather_kernel<<<(unsigned)grid_for(rows * k), 256, 0, st>>>(
+        kv_fp8, t_max, idx, rows, S, k, dc, dr, start_pos, g_rows, g_idx, device_error_word());
+    const dsa_status e = launch_status();
+    if (e != DSA_OK) return e;
+    // every query row is a sequence of k decoded rows; slot j sits at position j
+    return launch_sparse_mla(q, g_rows, k, g_idx, (int)rows, 1, Hq, dc, dr, k, k - 1, sm_scale,
+                             DSA_BF16, out, lse, attn_ws, st);
+}
+
 }  // namespace dsa
 
 extern "C" int64_t dsa_latent_row_bytes(int dc, int dr) { return dsa::row_bytes(dc, dr); }
@@ -183,7 +222,7 @@ extern "C" dsa_status dsa_latent_quant(const void *kv, dsa_dtype x_dtype, int64_
 extern "C" size_t dsa_sparse_mla_attn_fp8_workspace_size(int B, int S, int Hq, int dc, int dr,
                                                          int k) {
     if (B <= 0 || S <= 0 || Hq <= 0 || k <= 0 || !dsa::fp8_shape_ok(dc, dr)) return 0;
-    return dsa::fp8_workspace(B, S, Hq, dc, dr, k).total();
+    return dsa::sparse_mla_fp8_workspace_bytes(B, S, Hq, dc, dr, k);
 }
 
 extern "C" dsa_status dsa_sparse_mla_attn_fp8(const void *q, const uint8_t *kv_fp8, int64_t t_max,
@@ -200,20 +239,12 @@ extern "C" dsa_status dsa_sparse_mla_attn_fp8(const void *q, const uint8_t *kv_f
     if (!dsa::aligned16(q) || !dsa::aligned16(out) || (reinterpret_cast<uintptr_t>(kv_fp8) & 3) ||
         (reinterpret_cast<uintptr_t>(idx) & 3))
         return DSA_ERR_INVALID_ARG;
-    const dsa::Fp8Ws w = dsa::fp8_workspace(B, S, Hq, dc, dr, k);
-    if (!workspace || workspace_bytes < w.total() || !dsa::aligned16(workspace))
+    if (dsa::sparse_mla_fp8_tc_supported(Hq, dc, dr, k) && !dsa::aligned16(kv_fp8))
+        return DSA_ERR_INVALID_ARG;
+    const size_t need = dsa::sparse_mla_fp8_workspace_bytes(B, S, Hq, dc, dr, k);
+    if (need > 0 && (!workspace || workspace_bytes < need || !dsa::aligned16(workspace)))
         return DSA_ERR_WORKSPACE;
-    const cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-    char *ws = static_cast<char *>(workspace);
-    __nv_bfloat16 *g_rows = reinterpret_cast<__nv_bfloat16 *>(ws);
-    int32_t *g_idx = reinterpret_cast<int32_t *>(ws + w.rows_bytes);
-    void *attn_ws = w.attn_bytes ? ws + w.rows_bytes + w.idx_bytes : nullptr;
-    const int64_t rows = (int64_t)B * S;
-    dsa::latent_gather_kernel<<<(unsigned)dsa::grid_for(rows * k), 256, 0, st>>>(
-        kv_fp8, t_max, idx, rows, S, k, dc, dr, start_pos, g_rows, g_idx, dsa::device_error_word());
-    const dsa_status e = dsa::launch_status();
-    if (e != DSA_OK) return e;
-    // every query row is a sequence of k decoded rows; slot j sits at position j
-    return dsa::launch_sparse_mla(q, g_rows, k, g_idx, (int)rows, 1, Hq, dc, dr, k, k - 1, sm_scale,
-                                  DSA_BF16, out, lse, attn_ws, st);
+    return dsa::launch_sparse_mla_fp8(q, kv_fp8, t_max, idx, B, S, Hq, dc, dr, k, start_pos,
+                                      sm_scale, out, lse, workspace,
+                                      reinterpret_cast<cudaStream_t>(stream));
 }
