@@ -321,24 +321,36 @@ def oracle_decode_sample(wl, n_seq: int, repeats: int = 1):
     return per_seq
 
 
+def bench_config(wl, world):
+    """The workload description both arms print (identical dicts)."""
+    return {"workload": wl.name, "B": wl.B, "T": wl.T, "H": wl.H, "D": wl.D, "topk": wl.topk,
+            "Hq": wl.Hq, "dc": wl.dc, "dr": wl.dr,
+            "l2": "inputs larger than L2 (a decode state is 1.4 GB)",
+            "parallelism": f"dp{world} (independent batches per rank)"}
+
+
 def run_reference(args, wl, world, rank):
     if rank != 0:
         return
-    # one "step" of the reference arm = the oracle's decode pass for ONE
-    # sequence of the batch; steps/s of the whole batch = 1 / (B * t_seq)
-    warm = oracle_decode_sample(wl, 1, repeats=max(args.warmup, 0)) if args.warmup else []
+    # One timed step of the reference arm is a bounded sample of the workload:
+    # the oracle's decode pass for ONE sequence of the batch (sequences are
+    # independent and alike).  ms_per_step is that timed work; the metric,
+    # steps/s of the whole B-sequence step, is 1 / (B * t_seq).
+    if args.warmup:
+        oracle_decode_sample(wl, 1, repeats=max(args.warmup, 0))
     times = []
     for k in range(args.steps):
         times += oracle_decode_sample(wl, 1, repeats=1)
     t_seq = sum(times) / len(times)
     value = 1.0 / (wl.B * t_seq)
     line = {
-        "metric": "dsa_decode_steps_per_s", "value": value, "unit": "steps/s", "n_gpus": 1,
-        "steps": args.steps, "warmup": args.warmup, "ms_per_step": wl.B * t_seq * 1e3,
+        "metric": "dsa_decode_steps_per_s", "value": value, "unit": "steps/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": t_seq * 1e3,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic", "impl": "reference",
-        "config": {"workload": wl.name, "B": wl.B, "T": wl.T, "H": wl.H, "D": wl.D,
-                   "topk": wl.topk, "Hq": wl.Hq, "dc": wl.dc, "dr": wl.dr},
+        "config": bench_config(wl, world),
+        "timed_step": f"one of the {wl.B} sequences of a decode step per timed step "
+                      f"(ms_per_step); value = 1 / ({wl.B} x that time)",
         "cpu_baseline": {"value": value, "unit": "steps/s", "cores": 1, "kind": "oracle",
                          "sample": f"sequence 0 of {wl.B}, one decode step per timed step "
                                    f"(T={wl.T}), extrapolated x{wl.B}; cache prebuilt"},
@@ -357,7 +369,8 @@ def run_ours(args, wl, world, rank, local):
     __graft_entry__._builder().build()
     import top_kv_selection_b200 as dsa
 
-    copies = build_state(dsa, wl, rank_seed_offset=0, n_copies=args.copies)
+    # every rank draws its own independent sequences
+    copies = build_state(dsa, wl, rank_seed_offset=rank * wl.B, n_copies=args.copies)
     torch.cuda.synchronize()
     per_step_launches, kernel_names = count_launches_per_step(wl, dsa, copies[0])
 
@@ -412,10 +425,8 @@ def run_ours(args, wl, world, rank, local):
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "fp8_e4m3+bf16", "data": "synthetic",
-        "config": {"workload": wl.name, "B": wl.B, "T": wl.T, "H": wl.H, "D": wl.D,
-                   "topk": wl.topk, "Hq": wl.Hq, "dc": wl.dc, "dr": wl.dr,
-                   "l2": f"{len(copies)} rotating state copies, each larger than L2",
-                   "parallelism": f"dp{world} (independent batches per rank)"},
+        "config": bench_config(wl, world),
+        "l2_detail": f"{len(copies)} rotating decode-state copies, each larger than L2",
         # the scorer kernel's own rate (cached tokens scored per second), and the
         # same count over the whole step
         "indexer_gscores_per_s": wl.B * wl.T / t_score / 1e9,
@@ -610,7 +621,7 @@ def time_sparse_mla_fp8(dsa, peak_gbs, wl, iters=32, sets=16):
     res = {"workload": f"{wl.name}_fp8_latent", "rows": B * k, "row_bytes": rb, "bytes": nbytes,
            "us": t * 1e6, "achieved_gbs": nbytes / t / 1e9, "peak_gbs": peak_gbs,
            "frac": nbytes / t / 1e9 / peak_gbs, "bound": "hbm",
-           "note": "decode pass to bf16 rows in the workspace, then the bf16 sparse attention"}
+           "note": "656-byte rows decoded to bf16 while they are gathered, inside the attention kernel"}
     del cache, idxs, ws
     return res
 
@@ -692,7 +703,20 @@ def main(argv=None):
     wl = workloads.WORKLOADS[args.workload]
     if wl.mode != "decode":
         raise SystemExit("bench.py times decode workloads (1, 2 or 4)")
+    if args.gpus > 1 and "WORLD_SIZE" not in os.environ:
+        # one process per GPU: start the ranks under torch.distributed.run
+        import socket
+        with socket.socket() as sk:
+            sk.bind(("127.0.0.1", 0))
+            port = sk.getsockname()[1]
+        cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1",
+               f"--nproc-per-node={args.gpus}", "--master-addr", "127.0.0.1",
+               "--master-port", str(port), os.path.abspath(__file__),
+               *(sys.argv[1:] if argv is None else argv)]
+        os.execv(sys.executable, cmd)
     world, rank, local = _dist_init()
+    if world != args.gpus:
+        raise SystemExit(f"--gpus {args.gpus} but the launcher started {world} ranks")
     try:
         if args.impl == "reference":
             run_reference(args, wl, world, rank)

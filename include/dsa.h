@@ -7,10 +7,12 @@
  *   "DeepSeek-V3.2-Exp - Split indexer heads": the Indexer.forward excerpt:
  *       the non-interleaved rotary embedding of q_pe / k_pe, rotate_activation,
  *       act_quant (with its scale_fmt), the key-cache write, the weight fold,
- *       fp8_index, the additive mask and topk(min(index_topk, end_pos)).
- *   "DeepSeek-V3.2-Exp - Causal mask": Transformer.forward (mask =
- *       full(-inf).triu_(1) when seqlen > 1) and the MLA prefill excerpt
- *       (index_mask = full(-inf).scatter_(topk, 0) + mask).
+ *       fp8_index, the additive mask and the top-k of min(index_topk, end_pos)
+ *       positions.
+ *   "DeepSeek-V3.2-Exp - Causal mask": Transformer.forward (a -inf mask above
+ *       the diagonal when more than one token is new) and the MLA prefill
+ *       excerpt (an index mask, -inf except at the selected positions, plus
+ *       that causal mask).
  *   "DeepSeek Sparse Attention, one decode step in one layer (V3.2 sizes)"
  *       diagram: I(t,s) = sum_j w_j ReLU(q_j . k_s), k = 2048, core attention
  *       in MQA mode over the gathered latents, each latent row key and value,
@@ -221,7 +223,7 @@ dsa_status dsa_decode_index_scores(const float *q_idx, const float *w, const flo
                                    dsa_stream_t stream);
 
 /*
- * topk(min(index_topk, end_pos)) (Indexer.forward), restricted to the causal
+ * The top-k step of Indexer.forward (min(index_topk, end_pos) positions), restricted to the causal
  * positions t <= start_pos + s of each row:
  *   idx[b,s,:] holds the m = min(K, start_pos+s+1, T) positions with the
  *   largest scores, K = min(k, T), ties broken towards the lower position,
@@ -302,6 +304,9 @@ dsa_status dsa_decode_step(const float *q_idx, const float *w, const float *k_ne
  * rejected with DSA_ERR_WORKSPACE before anything is launched.
  *   - The first call on a device resolves the array's device address (with
  *     that device current); make that first call before any stream capture.
+ *     A call that finds a different CUDA context current on the device (after
+ *     cudaDeviceReset, say) resolves it again, so that call too should come
+ *     before any stream capture.
  *   - All calls on a device share the one array and it keeps the previous
  *     call's contents (nothing in it needs to start at zero).  Calls that
  *     overlap on the GPU (other streams, other threads) race on it: serialise

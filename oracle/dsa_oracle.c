@@ -12,9 +12,10 @@
  *              rotate_activation, act_quant,
  *              k cache write, weight fold, fp8_index, additive mask, topk.
  *   [V32-MASK] "DeepSeek-V3.2-Exp - Causal mask", Transformer.forward excerpt:
- *              mask = full(-inf).triu_(1) if seqlen > 1.
- *   [V32-MLA]  same page, MLA prefill excerpt: index_mask =
- *              full(-inf).scatter_(topk, 0) + mask, softmax, value mix.
+ *              with more than one new token, a mask that is -inf above the
+ *              diagonal (future positions), none otherwise.
+ *   [V32-MLA]  same page, MLA prefill excerpt: an index mask that is -inf except
+ *              at the selected positions, plus the causal mask; softmax; value mix.
  *   [DIAG]     "DeepSeek Sparse Attention, one decode step in one layer (V3.2
  *              sizes)" diagram: I(t,s) = sum_j w_j ReLU(q_j . k_s), k = 2048,
  *              core attention in MQA mode over the selected latents, each latent
@@ -163,8 +164,8 @@ void oracle_indexer_quant(const float *x, int64_t n_vec, int D, uint8_t *out, fl
 
 /*
  * Rotary embedding of the first R elements of one vector, not interleaved
- * [V32-IDX: q_pe = first rope_head_dim elements; apply_rotary_emb(q_pe,
- * freqs_cis, False); q = cat(q_pe, q_nope)].  Element j and element j + R/2
+ * [V32-IDX: the first rope_head_dim elements get the rotary embedding, not
+ * interleaved, and are put back in front of the rest].  Element j and element j + R/2
  * (j < R/2) are the real and imaginary parts of one complex number, which is
  * multiplied by the position's unit complex cs[2j] + i cs[2j+1] (cos, sin of
  * frequency j): (x1 + i x2)(c + i s) = (x1 c - x2 s) + i (x1 s + x2 c), each

@@ -25,3 +25,10 @@ def test_reference_arm_prints_the_contract_line():
     assert d["e2e"]["value"] == d["value"]
     assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["e2e"]["d2h_bytes_per_step"] == 0
     assert d["config"]["workload"].startswith("decode_")
+    # the same workload description as the GPU arm prints, and a per-step time
+    # that is the work actually timed (one sequence per step)
+    sys.path.insert(0, ROOT)
+    import bench
+    import workloads
+    assert d["config"] == bench.bench_config(workloads.WORKLOADS[1], 1)
+    assert abs(d["value"] * workloads.WORKLOADS[1].B * d["ms_per_step"] * 1e-3 - 1) < 1e-6

@@ -142,3 +142,17 @@ def test_sparse_mla_split_partials_keep_range(dsa):
     ref, ref_lse = oracle.sparse_mla(q.float().numpy(), kv.float().numpy(), idx.numpy(), t_max - 1,
                                      sm, dc)
     assert_attention_close(out / big, ref, "bf16", lse, ref_lse)
+
+
+@pytest.mark.parametrize("B,k", [(40, 512), (20, 1024)])
+def test_sparse_mla_rows_of_two_and_four_units(dsa, B, k):
+    """Rows whose selections span 2 (k = 512) or 4 (k = 1024) units of 256 rows
+    when the rows fill the GPU, merged by the split combine."""
+    Hq, dc, dr, t_max = 128, 512, 64, 3000
+    q, kv, idx = _case(B, 1, Hq, dc, dr, t_max, k, t_max - 1, torch.bfloat16, seed=B + k, fill=0.9)
+    sm = 576 ** -0.5
+    out, lse = _gpu(dsa, q, kv, idx, t_max - 1, sm, dc)
+    for b in (0, B // 2, B - 1):
+        ref, ref_lse = oracle.sparse_mla(q[b:b + 1].float().numpy(), kv[b:b + 1].float().numpy(),
+                                         idx[b:b + 1].numpy(), t_max - 1, sm, dc)
+        assert_attention_close(out[b:b + 1], ref, "bf16", lse[b:b + 1], ref_lse)

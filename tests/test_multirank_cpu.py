@@ -50,8 +50,8 @@ def test_bench_reference_arm_under_torchrun_two_ranks():
     prints one JSON line, rank 1 exits 0 without work."""
     env = dict(os.environ, CUDA_VISIBLE_DEVICES="")
     cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", "--nproc-per-node=2",
-           "--master-addr", "127.0.0.1", "--master-port", "29533", "bench.py", "--impl",
-           "reference", "--workload", "1", "--steps", "1", "--warmup", "0"]
+           "--master-addr", "127.0.0.1", "--master-port", "29533", "bench.py", "--gpus", "2",
+           "--impl", "reference", "--workload", "1", "--steps", "1", "--warmup", "0"]
     r = subprocess.run(cmd, cwd=ROOT, env=env, capture_output=True, text=True, timeout=600)
     assert r.returncode == 0, r.stderr[-2000:]
     lines = [l for l in r.stdout.splitlines() if l.startswith("{")]
@@ -59,3 +59,25 @@ def test_bench_reference_arm_under_torchrun_two_ranks():
     d = json.loads(lines[0])
     assert d["impl"] == "reference" and d["value"] > 0 and d["cpu_baseline"]["kind"] == "oracle"
     assert d["e2e"]["h2d_bytes_per_step"] == 0
+
+
+@pytest.mark.slow
+def test_bench_gpus_flag_starts_the_ranks_itself():
+    """`bench.py --gpus 2` without a launcher starts two ranks under
+    torch.distributed.run (one process per device); rank 0 prints one line."""
+    env = dict(os.environ, CUDA_VISIBLE_DEVICES="")
+    env.pop("WORLD_SIZE", None)
+    cmd = [sys.executable, "bench.py", "--gpus", "2", "--impl", "reference", "--workload", "1",
+           "--steps", "1", "--warmup", "0"]
+    r = subprocess.run(cmd, cwd=ROOT, env=env, capture_output=True, text=True, timeout=600)
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = [l for l in r.stdout.splitlines() if l.startswith("{")]
+    assert len(lines) == 1 and json.loads(lines[0])["n_gpus"] == 2
+
+
+def test_bench_rejects_a_world_size_that_differs_from_gpus():
+    env = dict(os.environ, CUDA_VISIBLE_DEVICES="", WORLD_SIZE="1", RANK="0", LOCAL_RANK="0")
+    r = subprocess.run([sys.executable, "bench.py", "--gpus", "2", "--impl", "reference",
+                        "--workload", "1", "--steps", "1", "--warmup", "0"], cwd=ROOT, env=env,
+                       capture_output=True, text=True, timeout=600)
+    assert r.returncode != 0 and "--gpus 2" in r.stderr

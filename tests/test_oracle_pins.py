@@ -206,8 +206,8 @@ def test_golden_v32_row_sizes():
 # weight fold and fp8_index scoring
 # --------------------------------------------------------------------------- #
 def test_weight_fold_matches_page_expression_in_torch():
-    # the Indexer.forward lines, evaluated by torch in fp32:
-    # weights = weights_proj(x) * n_heads ** -0.5 ; weights * q_scale * softmax_scale
+    # the Indexer.forward weight step, evaluated by torch in fp32: the projected
+    # weights times H^-1/2, then times each head's query scale and the softmax scale
     rng = np.random.default_rng(8)
     for H in (4, 64, 3):
         w = torch.from_numpy(rng.standard_normal(H).astype(np.float32))
@@ -416,8 +416,9 @@ def test_sparse_equals_dense_causal_when_k_ge_T():
 
 
 def test_sparse_equals_index_mask_formulation():
-    """The MLA prefill lines: index_mask = full(-inf).scatter_(topk, 0) + causal mask,
-    added to the scaled scores, softmax, mix (latent row as key and value)."""
+    """The MLA prefill excerpt's formulation: an index mask, -inf except at the
+    selected positions, plus the causal mask, added to the scaled scores;
+    softmax; mix (latent row as key and value)."""
     rng = np.random.default_rng(15)
     T, Hq, dc, dr, k = 30, 4, 32, 8, 6
     q = torch.from_numpy(rng.standard_normal((1, T, Hq, dc + dr)))

@@ -1,10 +1,10 @@
 """Pins of the oracle's indexer prologue: non-interleaved RoPE, the ue8m0 scale
 format and their composition with rotate_activation and act_quant.
 
-The page ("DeepSeek-V3.2-Exp - Split indexer heads", Indexer.forward) applies
-apply_rotary_emb(q_pe, freqs_cis, False) to the first rope_head_dim elements,
-then rotate_activation and act_quant(x, block_size, scale_fmt); it does not
-print the rotary function or the scale format.  These tests check the oracle
+The page ("DeepSeek-V3.2-Exp - Split indexer heads", Indexer.forward) gives the
+first rope_head_dim elements the rotary embedding (not interleaved), then
+rotates and quantises with the configured scale format; it does not print the
+rotary function or the scale format.  These tests check the oracle
 against numpy complex arithmetic, scipy's Hadamard matrix, torch's e4m3 cast,
 exact special angles and invariants, so that a swapped pairing (interleaved
 instead of split halves), a sign slip or a wrong rounding of the scale fails.

@@ -1,4 +1,8 @@
-// api.cu -- status strings, version and the sticky device error word.
+// api.cu -- status strings, version, the sticky device error word, and the
+// per-context cache of device-symbol addresses.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
 #include "common.cuh"
 
 // First error code recorded by any kernel of the library on this device
@@ -6,17 +10,48 @@
 __device__ int dsa_device_error_word_storage = 0;
 
 namespace dsa {
+namespace {
+
+PFN_cuCtxGetCurrent_v4000 ctx_get_current_fn() {
+    static PFN_cuCtxGetCurrent_v4000 fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuCtxGetCurrent_v4000>(p);
+    });
+    return fn;
+}
+
+void *current_context() {
+    auto fn = ctx_get_current_fn();
+    CUcontext c = nullptr;
+    if (!fn || fn(&c) != CUDA_SUCCESS) return nullptr;
+    return c;
+}
+
+SymbolCache g_error_word_cache;
+
+}  // namespace
+
+void *symbol_address(const void *symbol, SymbolCache *cache) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= SymbolCache::kMaxDevices)
+        return nullptr;
+    std::lock_guard<std::mutex> lock(cache->mutex);
+    void *ctx = current_context();
+    if (cache->ptr[dev] && ctx && ctx == cache->ctx[dev]) return cache->ptr[dev];
+    void *p = nullptr;
+    if (cudaGetSymbolAddress(&p, symbol) != cudaSuccess || !p) return nullptr;
+    cache->ptr[dev] = p;
+    cache->ctx[dev] = current_context();     // the runtime's context now exists
+    return p;
+}
 
 int *device_error_word() {
-    static int *cached[64] = {nullptr};
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
-    if (!cached[dev]) {
-        void *p = nullptr;
-        if (cudaGetSymbolAddress(&p, dsa_device_error_word_storage) != cudaSuccess) return nullptr;
-        cached[dev] = static_cast<int *>(p);
-    }
-    return cached[dev];
+    return static_cast<int *>(symbol_address(&dsa_device_error_word_storage, &g_error_word_cache));
 }
 
 }  // namespace dsa

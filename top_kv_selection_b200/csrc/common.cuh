@@ -6,11 +6,26 @@
 #include <cuda_fp8.h>
 #include <stdint.h>
 
+#include <mutex>
+
 #include "dsa.h"
 
 namespace dsa {
 
 // ---------------------------------------------------------------- host side
+// Device address of a __device__ variable (its host-side name is only a
+// stand-in) on the current device, cached per device together with the CUDA
+// context it was resolved in: a new context (after cudaDeviceReset, say)
+// resolves it again.  Thread-safe.  Returns nullptr if the runtime cannot
+// resolve it.
+struct SymbolCache {
+    static constexpr int kMaxDevices = 64;
+    std::mutex mutex;
+    void *ctx[kMaxDevices] = {nullptr};
+    void *ptr[kMaxDevices] = {nullptr};
+};
+void *symbol_address(const void *symbol, SymbolCache *cache);
+
 // Device pointer of the sticky error word of the current device (the word
 // lives in api.cu).  Returns nullptr if the runtime cannot resolve it.
 int *device_error_word();
@@ -103,8 +118,13 @@ dsa_status launch_decode_scores(const float *q_raw, const float *w, const float 
                                 cudaStream_t stream);
 
 size_t topk_workspace_bytes(int B, int S, int64_t T, int k);
+// prefetch_rows: optional cache whose rows at the selected positions are
+// requested into L2 as they are selected (row (b, t) at prefetch_rows +
+// (b * prefetch_t_max + t) * prefetch_row_bytes; bytes a multiple of 16).
 dsa_status launch_topk_select(const float *scores, int B, int S, int64_t T, int64_t start_pos,
-                              int k, int32_t *idx, void *ws, cudaStream_t stream);
+                              int k, int32_t *idx, void *ws, cudaStream_t stream,
+                              const void *prefetch_rows = nullptr, int64_t prefetch_t_max = 0,
+                              int prefetch_row_bytes = 0);
 
 size_t sparse_mla_workspace_bytes(int B, int S, int Hq, int dc, int dr, int k, dsa_dtype dt);
 bool sparse_mla_tc_supported(int Hq, int dc, int dr, int k, dsa_dtype dt);

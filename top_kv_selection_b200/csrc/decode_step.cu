@@ -77,8 +77,12 @@ extern "C" dsa_status dsa_decode_step(const float *q_idx, const float *w, const 
     if ((st = dsa::launch_decode_scores(q_idx, w, k_new, k_cache, k_scale, t_max, B, H, D, T,
                                         softmax_scale, ws.scores, s)) != DSA_OK)
         return st;
-    if ((st = dsa::launch_topk_select(ws.scores, B, 1, T, T - 1, index_topk, idx, ws.topk_ws,
-                                      s)) != DSA_OK)
+    // the top-k asks L2 for the latent rows it selects, ahead of the attention's gather
+    const int row_bytes = dt == DSA_FP8_LATENT ? (int)dsa_latent_row_bytes(dc, dr)
+                                               : (dc + dr) * (dt == DSA_BF16 ? 2 : 4);
+    if ((st = dsa::launch_topk_select(ws.scores, B, 1, T, T - 1, index_topk, idx, ws.topk_ws, s,
+                                      row_bytes % 16 == 0 ? kv_cache : nullptr, t_max,
+                                      row_bytes)) != DSA_OK)
         return st;
     const int K = (int64_t)index_topk < T ? index_topk : (int)T;
     if (dt == DSA_FP8_LATENT)

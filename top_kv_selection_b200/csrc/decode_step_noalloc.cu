@@ -12,32 +12,20 @@
 // The array's host-side name is only a stand-in for the symbol, not a device
 // address, so the host code below resolves the real address once per device
 // (with that device current) and hands it to the kernels as a pointer.
-#include <mutex>
-
 #include "common.cuh"
 
 static __device__ __align__(256) unsigned char dsa_noalloc_scratch[DSA_NOALLOC_SCRATCH_BYTES];
 
 namespace {
 
-constexpr int kMaxDevices = 64;
-std::mutex g_scratch_mutex;
-void *g_scratch_ptr[kMaxDevices] = {nullptr};
+dsa::SymbolCache g_scratch_cache;
 
 // Device address of the scratch array on the current device, resolved on the
-// first call for that device.
+// first call for that device (and again if the device's context was replaced).
 dsa_status scratch_address(void **out) {
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess) return DSA_ERR_CUDA;
-    if (dev < 0 || dev >= kMaxDevices) return DSA_ERR_UNSUPPORTED;
-    std::lock_guard<std::mutex> lock(g_scratch_mutex);
-    if (!g_scratch_ptr[dev]) {
-        void *p = nullptr;
-        if (cudaGetSymbolAddress(&p, dsa_noalloc_scratch) != cudaSuccess || !p)
-            return DSA_ERR_CUDA;
-        g_scratch_ptr[dev] = p;
-    }
-    *out = g_scratch_ptr[dev];
+    void *p = dsa::symbol_address(dsa_noalloc_scratch, &g_scratch_cache);
+    if (!p) return DSA_ERR_CUDA;
+    *out = p;
     return DSA_OK;
 }
 

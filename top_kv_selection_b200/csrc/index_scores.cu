@@ -1,9 +1,12 @@
 // index_scores.cu -- fp8_index scoring with the weight fold and the causal mask.
 //
-// Page: "DeepSeek-V3.2-Exp - Split indexer heads", Indexer.forward:
-//   weights = weights_proj(x) * n_heads^-1/2; weights = weights * q_scale * softmax_scale
-//   index_score = fp8_index(q_fp8, weights, k_cache, k_scale); index_score += mask
-// and the diagram's I(t,s) = sum_j w_j ReLU(q_j . k_s).
+// Page: "DeepSeek-V3.2-Exp - Split indexer heads", Indexer.forward, weight
+// and scoring steps: the per-head weights are scaled by H^-1/2, by each
+// head's query scale and by the indexer's softmax scale; fp8_index then
+// scores every cached key, and the additive mask is applied.  The scoring
+// formula is the one of the diagram "DeepSeek Sparse Attention, one decode
+// step in one layer (V3.2 sizes)": a weighted sum over heads of the ReLU of
+// the query-key dot products.
 //
 // Tensor-core scorer (sm_100a).  One CTA owns a contiguous range of 128-token
 // tiles of one query row (b, s) and streams them once from HBM:

@@ -3,11 +3,12 @@
 // rotate_activation, act_quant (fp32 or ue8m0 scale), and the key's cache
 // append.
 //
-// Page: "DeepSeek-V3.2-Exp - Split indexer heads", Indexer.forward
-// (q_pe, q_nope = split(q, [rope_head_dim, ...]); q_pe = apply_rotary_emb(q_pe,
-//  freqs_cis, False); q = cat(q_pe, q_nope); the same for k; rotate_activation;
-//  act_quant(., block_size, scale_fmt); k_cache[:, start_pos:end_pos] = k_fp8;
-//  k_scale_cache[:, start_pos:end_pos] = k_scale).
+// Page: "DeepSeek-V3.2-Exp - Split indexer heads", Indexer.forward, query
+// and key preparation: the first rope_head_dim elements of each query head
+// and of the key get the rotary embedding (not interleaved) and are put back
+// in front of the rest; both are then rotated (rotate_activation) and
+// quantised (act_quant with the configured scale format), and the key's codes
+// and scale are written into the caches at positions start_pos .. end_pos-1.
 //
 // G = D / 64 adjacent lanes hold one D-vector, 64 contiguous elements each
 // (lane part p: elements [64p, 64p + 64)), as in quant.cuh's

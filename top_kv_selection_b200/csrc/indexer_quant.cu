@@ -1,8 +1,9 @@
 // indexer_quant.cu -- rotate_activation + act_quant of indexer queries and keys.
 //
-// Page: "DeepSeek-V3.2-Exp - Split indexer heads", Indexer.forward
-// (q = rotate_activation(q); k = rotate_activation(k); act_quant(., block_size);
-//  k_cache[:, start_pos:end_pos] = k_fp8; k_scale_cache[...] = k_scale).
+// Page: "DeepSeek-V3.2-Exp - Split indexer heads", Indexer.forward: queries
+// and keys are rotated (rotate_activation) and quantised blockwise to FP8
+// (act_quant), and the key's codes and scale are written into the caches at
+// positions start_pos .. end_pos-1.
 //
 // One warp rotates and quantises one d-vector entirely in registers (see
 // quant.cuh for the butterfly order and the rounding).

@@ -3,8 +3,8 @@
 // Pages: "DeepSeek Sparse Attention, one decode step in one layer (V3.2 sizes)"
 // (core attention in MQA mode: 128 heads over the 2048 gathered latents, each
 // latent row is key and value) and the MLA prefill excerpt of "DeepSeek-V3.2-Exp
-// - Causal mask" (scores masked by index_mask = full(-inf).scatter_(topk, 0)
-// plus the causal mask, softmax, value mix).  The latent row is [c | k_pe]
+// - Causal mask" (an index mask that is -inf everywhere except at the selected
+// positions, plus the causal mask, added to the scores; softmax; value mix).  The latent row is [c | k_pe]
 // (wkv_a output order); the query is already in latent space.
 //
 // bf16 at the V3.2 shapes (128 heads, 512 + 64) runs the tensor-core kernel of

@@ -7,9 +7,10 @@
 // Causal mask" (index mask + causal mask, softmax, value mix).
 //
 // Shapes: Hq = 128 heads (the MMA M), rows [c (512) | k_pe (64)].
-// Work unit: one query row and a contiguous share of U <= 256 of its selected
-// rows (in slot order), computed by TWO independent CTAs that differ only in
-// which half of the 512 output columns they produce.  Each CTA
+// Work unit: one query row and U <= 256 consecutive slots of its selection
+// (slots holding -1 or a future position count as empty rows), computed by
+// TWO independent CTAs that differ only in which half of the 512 output
+// columns they produce.  Each CTA
 //   1. gathers the U rows in nine 64-column chunks (eight latent blocks and
 //      the rotary block) into 128B-swizzled K-major tiles, and accumulates the
 //      full logits S = Q C^T (M = 128 heads, N = U, K = 576) in TMEM with 36
@@ -20,28 +21,38 @@
 //      the logits it came from);
 //   3. accumulates O = P C[:, own 256 columns] (M = 128, N = 256, K = U) with
 //      A = P read from TMEM and B = the CTA's four own latent chunks, which
-//      were gathered last and stay in shared memory (read MN-major), so the
-//      value mix needs no second gather;
+//      stay in shared memory after the logits (read MN-major), so the value
+//      mix needs no second gather;
 //   4. writes its 256 output columns: bf16 out (+ lse) when the row has one
 //      unit, else a normalised fp16 partial with its (max, sum, power-of-two
-//      range) for the split combine.
+//      ranges).  The partials of a row's units ("splits") are then merged:
+//      when the whole grid fits on the GPU at once it is launched as a
+//      cooperative grid, and after a grid-wide barrier every CTA merges its
+//      own slice of the output columns; otherwise a combine kernel merges.
 // The two CTAs of a unit read the same rows; the second read is served from
 // L2 (each CTA also prefetches half of the unit's rows into L2 at its start).
 //
-// Shared memory: five 32 KB chunk regions G0..G4 and the CTA's four own query
-// blocks (64 KB).  The query's five other blocks are staged by TMA in G2..G4
-// and consumed first, so the own latent chunks (chunks 5..8) can land in
-// G1..G4 -- consecutive regions, one MN-major operand with a 32 KB stride
-// between its 64-column blocks.  Chunk order and regions:
-//   chunk   0    1    2    3    4      5..8
-//   block   4 other latent blocks, rope, 4 own latent blocks
-//   region  G0   G1   G0   G1   G0     G1 G2 G3 G4
-// TMEM: S / P in columns [0, U), O in [256, 512).
+// Shared memory: six 32 KB chunk regions R0..R5 and the query's rotary block.
+// While the logits accumulate, the query's 512 latent columns sit in TMEM (the
+// output columns are not in use yet) and are the MMA's A operand there, so
+// the regions hold gathered rows only and six chunks are in flight at once.
+// Chunk order, regions and the MMA each chunk waits for before it may be
+// written:
+//   chunk    0     1     2     3     4     5     6     7     8
+//   block    own0  own1  oth0  oth1  oth2  oth3  own2  own3  rope
+//   region   R0    R1    R2    R3    R4    R5    R2    R3    R4
+//   waits    -     -     -     -     -     -     2     3     4
+// The own latent chunks end in R0..R3: consecutive regions, one MN-major
+// operand with a 32 KB stride between its 64-column blocks.
+// TMEM: S / P in columns [0, U); the query's latent part in [256, 512) during
+// the logits, then O in [256, 512).
 //
 // The FP8 variant reads 656-byte rows [512 e4m3 | 4 fp32 block scales | 64
-// bf16] and decodes each latent chunk while gathering it (code * block scale,
-// rounded to bf16 -- the same decoded operand as the oracle's), so the rows
-// cross HBM once at 656 bytes and no decoded copy is ever written to memory.
+// bf16].  The codes of a latent chunk are copied into the upper half of its
+// region and decoded in place (code * block scale, rounded to bf16 -- the same
+// decoded operand as the oracle's), so the rows cross HBM once at 656 bytes
+// and no decoded copy is ever written to memory.
+#include <cooperative_groups.h>
 #include <cuda_fp16.h>
 #include <cuda_fp8.h>
 
@@ -55,48 +66,45 @@ namespace {
 constexpr int kHq = 128, kDc = 512, kDr = 64, kDqk = kDc + kDr;
 constexpr int kUnitMax = 256;                   // selected rows per unit (max MMA N)
 constexpr int kChunks = 9;                      // 8 latent blocks + the rotary block
+constexpr int kRegions = 6;
 constexpr int kRegion = kUnitMax * 128;         // one chunk of 256 rows: 32 KB
 constexpr int kQBlk = kHq * 128;                // one 64-column block of the query: 16 KB
-constexpr int kOwnQ = 5 * kRegion;              // the own query blocks follow G0..G4
-constexpr int kBig = kOwnQ + 4 * kQBlk;         // 224 KB of operands
+constexpr int kQRope = kRegions * kRegion;      // the query's rotary block
+constexpr int kScales = kQRope + kQBlk;         // FP8: the unit's block scales, 16 B per row
+constexpr int kList = kScales + kUnitMax * 16;  // the unit's rows (int32)
+constexpr int kBars = kList + kUnitMax * 4;
 constexpr int kWork = 256;                      // gather / softmax / epilogue threads
 constexpr int kThreads = kWork + 32;            // + one TMA / MMA warp
 constexpr int kMaxSel = 2048;                   // selection slots per query row
-constexpr int kLag = 1;                         // gather chunks in flight beyond the newest
-constexpr uint32_t kColS = 0, kColO = 256, kTmemCols = 512;
+constexpr uint32_t kColS = 0, kColQ = 256, kColO = 256, kTmemCols = 512;
 constexpr int kRowFp8 = kDc + 4 * (kDc / 128) + 2 * kDr;   // 656
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
 
-constexpr size_t kSmemBytes = 1024 + (size_t)kBig + kUnitMax * sizeof(int32_t) +
-                              32 * sizeof(uint64_t) + 64;
+constexpr size_t kSmemBytes = 1024 + (size_t)kBars + 32 * sizeof(uint64_t) + 64;
 
-// chunk schedule of the CTA with output half `half`
+// chunk schedule of the CTA with output half `half` (see the table above)
 __device__ __forceinline__ int chunk_block(int k, int half) {
-    return k < 4 ? (1 - half) * 4 + k : (k == 4 ? 8 : half * 4 + (k - 5));
+    const int own = half * 4, oth = (1 - half) * 4;
+    return k < 2 ? own + k : (k < 6 ? oth + (k - 2) : (k < 8 ? own + (k - 4) : 8));
 }
-__device__ __forceinline__ int chunk_region(int k) { return k < 5 ? (k & 1) : k - 4; }
-__device__ __forceinline__ int q_offset(int k) {
-    return k < 5 ? 2 * kRegion + k * kQBlk : kOwnQ + (k - 5) * kQBlk;
-}
-// the MMA whose completion frees the region chunk k is written into
-//   chunk k    0   1   2   3   4   5   6   7   8
-//   waits on   -   -   0   1   2   3   1   3   4
-__device__ __forceinline__ int chunk_dep(int k) {
-    return k < 2 ? -1 : (k < 6 ? k - 2 : (k == 6 ? 1 : (k == 7 ? 3 : 4)));
-}
+__device__ __forceinline__ int chunk_region(int k) { return k < 6 ? k : k - 4; }
+__device__ __forceinline__ int chunk_dep(int k) { return k < 6 ? -1 : k - 4; }
 
 struct MlaArgs {
+    const __nv_bfloat16 *q;    // [rows, 128, 576]
     const __nv_bfloat16 *kv;   // bf16 rows [B, t_max, 576]
     const uint8_t *kv8;        // FP8 rows [B, t_max, 656]
     const int32_t *idx;
     __nv_bfloat16 *out;
     float *lse;
-    __half *part_o;            // [units][256 / 8][128][8]  (splits > 1), unit = (row * splits + sp) * 2 + half
-    float4 *part_ml;           // [units][128] (max, sum, scale of the fp16 partial, 0)
+    __half *part_o;            // [blocks][256 / 8][128][8] (split combine kernel)
+    float4 *part_ml;           // [blocks][128] (max, sum, fp16 range of columns 0..127, of 128..255)
     int64_t t_max;
     int64_t start_pos;
+    int64_t row0;              // first query row of this launch
     int S, k, splits, unit_rows;
+    int coop;                  // cooperative grid: the splits are merged in this kernel
     float scale_log2;          // sm_scale * log2(e)
     int *err;
 };
@@ -108,13 +116,44 @@ __device__ __forceinline__ void cp_async16(uint32_t dst, const void *src, uint32
                  : "memory");
 }
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-template <int N> __device__ __forceinline__ void cp_async_wait() {
-    asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+// Arrives on `bar` once every cp.async this thread issued so far has landed
+// (the arrival counts against the barrier's initial count); the thread does
+// not wait.
+__device__ __forceinline__ void cp_async_arrive(uint64_t *bar) {
+    asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(tc::smem_u32(bar))
+                 : "memory");
+}
+// waits until at most n of this thread's cp.async groups are pending (0 <= n <= 5)
+__device__ __forceinline__ void cp_async_wait_n(int n) {
+    switch (n) {
+        case 0: asm volatile("cp.async.wait_group 0;" ::: "memory"); break;
+        case 1: asm volatile("cp.async.wait_group 1;" ::: "memory"); break;
+        case 2: asm volatile("cp.async.wait_group 2;" ::: "memory"); break;
+        case 3: asm volatile("cp.async.wait_group 3;" ::: "memory"); break;
+        case 4: asm volatile("cp.async.wait_group 4;" ::: "memory"); break;
+        default: asm volatile("cp.async.wait_group 5;" ::: "memory"); break;
+    }
 }
 __device__ __forceinline__ void st_shared_v4(uint32_t addr, uint4 v) {
     asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(v.x), "r"(v.y),
                  "r"(v.z), "r"(v.w)
                  : "memory");
+}
+__device__ __forceinline__ uint4 ld_shared_v4(uint32_t addr) {
+    uint4 v;
+    asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                 : "r"(addr)
+                 : "memory");
+    return v;
+}
+
+// 2^x by the SFU (relative error about 2^-22, far below the bf16 rounding of
+// P; 2^-inf = +0).
+__device__ __forceinline__ float ex2(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
 }
 
 // Eight e4m3 codes (two words) times the block scale, rounded to bf16 pairs.
@@ -135,32 +174,107 @@ __device__ __forceinline__ uint4 decode8(uint32_t w0, uint32_t w1, float sc) {
     return make_uint4(o[0], o[1], o[2], o[3]);
 }
 
+// Merges output columns [8 c8, 8 c8 + 8) of head h of one (row, half) from
+// its splits' fp16 partials (blocks blk0 .. blk0 + splits - 1), for NC octets
+// c8[0..NC) at once: with w_s = 2^(m_s - M) l_s and Y_s = O_s / (l_s sc_s),
+// out = sum_s w_s sc_s Y_s / sum_s w_s and lse = (M + log2 sum_s w_s) ln 2.
+// The loads of eight splits are in flight together; further batches rescale
+// the running sums.
+template <int NC>
+__device__ __forceinline__ void merge_octets(const __half *part_o, const float4 *part_ml, int splits,
+                                             int64_t blk0, int64_t row, int half, const int (&c8)[NC],
+                                             int h, __nv_bfloat16 *out, float *lse) {
+    float M = -INFINITY, L = 0.f;
+    float acc[NC][8];
+#pragma unroll
+    for (int n = 0; n < NC; n++)
+#pragma unroll
+        for (int e = 0; e < 8; e++) acc[n][e] = 0.f;
+    for (int s0 = 0; s0 < splits; s0 += 8) {
+        float4 ml[8];
+        uint4 x[8][NC];
+#pragma unroll
+        for (int u = 0; u < 8; u++) {
+            const int sp = s0 + u;
+            ml[u] = sp < splits ? part_ml[(blk0 + sp) * kHq + h] : make_float4(-INFINITY, 0.f, 1.f, 1.f);
+#pragma unroll
+            for (int n = 0; n < NC; n++)
+                if (sp < splits)
+                    x[u][n] = reinterpret_cast<const uint4 *>(part_o + (blk0 + sp) * kHq * 256)[c8[n] * kHq + h];
+        }
+        float mb = M;
+#pragma unroll
+        for (int u = 0; u < 8; u++) mb = fmaxf(mb, ml[u].x);
+        if (mb == -INFINITY) continue;
+        if (mb > M) {                                  // rescale the running sums
+            const float r = M == -INFINITY ? 0.f : ex2(M - mb);
+            L *= r;
+#pragma unroll
+            for (int n = 0; n < NC; n++)
+#pragma unroll
+                for (int e = 0; e < 8; e++) acc[n][e] *= r;
+            M = mb;
+        }
+#pragma unroll
+        for (int u = 0; u < 8; u++) {
+            if (ml[u].x == -INFINITY) continue;
+            const float w = ex2(ml[u].x - M) * ml[u].y;
+            L += w;
+#pragma unroll
+            for (int n = 0; n < NC; n++) {
+                const float ws = w * (c8[n] < 16 ? ml[u].z : ml[u].w);
+                const uint32_t xs[4] = {x[u][n].x, x[u][n].y, x[u][n].z, x[u][n].w};
+#pragma unroll
+                for (int e = 0; e < 4; e++) {
+                    const float2 f = __half22float2(*reinterpret_cast<const __half2 *>(&xs[e]));
+                    acc[n][2 * e] = fmaf(ws, f.x, acc[n][2 * e]);
+                    acc[n][2 * e + 1] = fmaf(ws, f.y, acc[n][2 * e + 1]);
+                }
+            }
+        }
+    }
+    const float inv = L > 0.f ? 1.f / L : 0.f;
+#pragma unroll
+    for (int n = 0; n < NC; n++) {
+        uint32_t w8[4];
+#pragma unroll
+        for (int e = 0; e < 4; e++) {
+            const __nv_bfloat162 v = __floats2bfloat162_rn(acc[n][2 * e] * inv, acc[n][2 * e + 1] * inv);
+            w8[e] = *reinterpret_cast<const uint32_t *>(&v);
+        }
+        reinterpret_cast<uint4 *>(out + (row * kHq + h) * kDc + half * 256)[c8[n]] =
+            make_uint4(w8[0], w8[1], w8[2], w8[3]);
+        if (half == 0 && c8[n] == 0 && lse) lse[row * kHq + h] = L > 0.f ? (M + log2f(L)) * kLn2 : -INFINITY;
+    }
+}
+
 template <bool kFp8>
 __global__ void __launch_bounds__(kThreads, 1)
 sparse_mla_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const MlaArgs a) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = reinterpret_cast<uint8_t *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    int32_t *list = reinterpret_cast<int32_t *>(sm + kBig);              // the unit's rows
-    uint64_t *bars = reinterpret_cast<uint64_t *>(list + kUnitMax);
+    int32_t *list = reinterpret_cast<int32_t *>(sm + kList);             // the unit's rows
+    uint64_t *bars = reinterpret_cast<uint64_t *>(sm + kBars);
     uint64_t *chunk_full = bars;                 // [9] chunk k gathered (256 arrivals)
     uint64_t *mma_done = bars + kChunks;         // [9] chunk k's logit MMAs complete
-    uint64_t *q_full = bars + 2 * kChunks;       // the query's TMA copy landed
-    uint64_t *p_full = q_full + 1;               // P is in TMEM (256 arrivals)
-    uint64_t *o_full = p_full + 1;               // the value mix is complete
-    uint64_t *mma_fin = o_full + 1;              // every issued MMA is complete
-    uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(bars + 24);
+    uint64_t *q_full = bars + 2 * kChunks;       // the query's rotary block landed (TMA)
+    uint64_t *q_ready = q_full + 1;              // the query's latent part is in TMEM (256 arrivals)
+    uint64_t *p_full = q_ready + 1;              // [2] P of each row group is in TMEM (256 arrivals)
+    uint64_t *o_full = p_full + 2;               // [2] each output column half is complete
+    uint64_t *mma_fin = o_full + 2;              // every issued MMA is complete
+    uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(bars + 28);   // after the 25 barriers
     volatile int *abort = reinterpret_cast<volatile int *>(tmem_holder + 1);
     int *scan_tmp = const_cast<int *>(abort) + 1;                         // 9 ints
     // softmax exchange (max, sum, output range of the two column halves):
-    // region G0, free once the logits are complete
-    float *red = reinterpret_cast<float *>(sm);
+    // region R5, free once the logits are complete
+    float *red = reinterpret_cast<float *>(sm + 5 * kRegion);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int unit = blockIdx.x;                 // (row * splits + sp) * 2 + half
-    const int half = unit & 1;
-    const int sp = (unit >> 1) % a.splits;
-    const int64_t row = (unit >> 1) / a.splits;
+    // blockIdx.x = ((row - row0) * 2 + half) * splits + sp
+    const int sp = (int)(blockIdx.x % (unsigned)a.splits);
+    const int half = (int)((blockIdx.x / (unsigned)a.splits) & 1u);
+    const int64_t row = a.row0 + blockIdx.x / (unsigned)a.splits / 2;
     const int64_t b = row / a.S, s = row - b * a.S;
     const int64_t limit = a.start_pos + s;
     const int U = a.unit_rows;
@@ -173,8 +287,11 @@ sparse_mla_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const MlaArgs a) 
                 tc::mbar_init(&mma_done[i], 1);
             }
             tc::mbar_init(q_full, 1);
-            tc::mbar_init(p_full, kWork);
-            tc::mbar_init(o_full, 1);
+            tc::mbar_init(q_ready, kWork);
+            for (int i = 0; i < 2; i++) {
+                tc::mbar_init(&p_full[i], kWork);
+                tc::mbar_init(&o_full[i], 1);
+            }
             tc::mbar_init(mma_fin, 1);
             *abort = 0;
             tc::fence_mbar_init();
@@ -189,11 +306,13 @@ sparse_mla_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const MlaArgs a) 
     tc::tc_fence_after();
     const uint32_t tmem = *tmem_holder;
     if (warp == kWork / 32 && lane == 0) {
-        // the query's nine 64-column blocks (the own four to their own region)
+        // the query: its rotary block stays in shared memory (the MMA's A
+        // operand there); its eight latent blocks are staged in R2..R5 and
+        // moved to TMEM by the work threads
         tc::mbar_arrive_expect_tx(q_full, kChunks * kQBlk);
-        for (int k = 0; k < kChunks; k++)
-            tc::tma_load_2d(sm + q_offset(k), &tm_q, chunk_block(k, half) * 64, (int)(row * kHq),
-                            q_full);
+        tc::tma_load_2d(sm + kQRope, &tm_q, kDc, (int)(row * kHq), q_full);
+        for (int cb = 0; cb < 8; cb++)
+            tc::tma_load_2d(sm + 2 * kRegion + cb * kQBlk, &tm_q, cb * 64, (int)(row * kHq), q_full);
     }
     // a kernel launched after this one (the split combine) may start its set-up
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
@@ -201,18 +320,17 @@ sparse_mla_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const MlaArgs a) 
     // (a no-op without a programmatic launch), then read them with plain loads.
     asm volatile("griddepcontrol.wait;" ::: "memory");
 
-    // valid selections of this row in slot order; this unit takes positions
-    // [lo, lo + U) of that list.  Threads 0..255 hold 8 consecutive slots each.
+    // This unit is the slots [lo, lo + U) of the row's selection, slot lo + j
+    // as row j.  A slot counts when it holds a causal position (>= 0 and <=
+    // start_pos + s); vmask has one bit per row.  (A top-k selection lists
+    // its positions first and pads with -1, so its units are dense.)
     const int lo = sp * U;
-    int n_total = 0;
+    uint32_t *vmask = reinterpret_cast<uint32_t *>(scan_tmp);          // [8]
     {
-        constexpr int kPer = kMaxSel / kWork;
-        int32_t v8[kPer];
-        int cnt = 0;
-#pragma unroll
-        for (int e = 0; e < kPer; e++) {
-            const int j = threadIdx.x * kPer + e;
-            int32_t t = threadIdx.x < kWork && j < a.k ? a.idx[row * a.k + j] : -1;
+        const int j = threadIdx.x;
+        int32_t t = -1;
+        if (j < U && lo + j < a.k) {
+            t = a.idx[row * a.k + lo + j];
             if (t >= 0 && (int64_t)t <= limit) {
                 if ((int64_t)t >= a.t_max) {
                     record_error(a.err, DSA_ERR_DEVICE);
@@ -221,54 +339,25 @@ sparse_mla_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const MlaArgs a) 
             } else {
                 t = -1;
             }
-            v8[e] = t;
-            cnt += t >= 0 ? 1 : 0;
         }
-        int incl = cnt;
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-            const int y = __shfl_up_sync(0xffffffffu, incl, o);
-            if (lane >= o) incl += y;
-        }
-        if (lane == 31) scan_tmp[warp] = incl;
-        __syncthreads();
-        int pos = incl - cnt;
-#pragma unroll
-        for (int w = 0; w < kThreads / 32; w++) {
-            const int c = scan_tmp[w];
-            if (w < warp) pos += c;
-            n_total += c;
-        }
-#pragma unroll
-        for (int e = 0; e < kPer; e++) {
-            if (v8[e] < 0) continue;
-            if (pos >= lo && pos < lo + U) list[pos - lo] = v8[e];
-            pos++;
-        }
+        if (j < kUnitMax) list[j] = t;
+        const uint32_t bal = __ballot_sync(0xffffffffu, t >= 0);
+        if (warp < kUnitMax / 32 && lane == 0) vmask[warp] = bal;
     }
     __syncthreads();
-    int n_my = n_total - lo;
-    n_my = n_my < 0 ? 0 : (n_my > U ? U : n_my);
+    uint32_t any = 0;
+#pragma unroll
+    for (int w = 0; w < kUnitMax / 32; w++) any |= vmask[w];
     const int64_t rbase = b * a.t_max;
-    // each CTA of the unit prefetches every other row into L2 (its partner the rest)
-    {
-        const int j = 2 * (int)threadIdx.x + half;
-        if (j < n_my) {
-            if constexpr (kFp8)
-                tc::prefetch_l2_bulk(a.kv8 + (rbase + list[j]) * kRowFp8, kRowFp8);
-            else
-                tc::prefetch_l2_bulk(a.kv + (rbase + list[j]) * kDqk, kDqk * 2);
-        }
-    }
 
-    if (n_my == 0) {
+    if (!any) {
         // nothing selected in this unit: an empty partial (or a zero output)
         if (threadIdx.x < kWork) {
             const int h = threadIdx.x & (kHq - 1), c = threadIdx.x >> 7;
             if (a.splits > 1) {
-                uint4 *po = reinterpret_cast<uint4 *>(a.part_o + (int64_t)unit * kHq * 256) + h;
+                uint4 *po = reinterpret_cast<uint4 *>(a.part_o + (int64_t)blockIdx.x * kHq * 256) + h;
                 for (int o8 = 16 * c; o8 < 16 * c + 16; o8++) po[o8 * kHq] = make_uint4(0u, 0u, 0u, 0u);
-                if (c == 0) a.part_ml[(int64_t)unit * kHq + h] = make_float4(-INFINITY, 0.f, 1.f, 0.f);
+                if (c == 0) a.part_ml[(int64_t)blockIdx.x * kHq + h] = make_float4(-INFINITY, 0.f, 1.f, 1.f);
             } else {
                 uint4 *o16 = reinterpret_cast<uint4 *>(a.out + (row * kHq + h) * kDc + half * 256 + c * 128);
                 for (int j = 0; j < 16; j++) o16[j] = make_uint4(0u, 0u, 0u, 0u);
@@ -277,34 +366,25 @@ sparse_mla_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const MlaArgs a) 
         }
         if (warp == kWork / 32 && lane == 0) tc::mbar_wait(q_full, 0, a.err, abort);
     } else if (warp < kWork / 32) {
-        // ------------------------------------------------------------ gather
         const int gt = threadIdx.x;
+        const int q4 = warp & 3, c = warp >> 2;          // TMEM lane quarter, column half
+        const int h = q4 * 32 + lane;                    // head
+        const uint32_t lane_addr = (uint32_t)(q4 * 32) << 16;
         bool ok = true;
-        int issued = 0, signalled = 0;
-        // publish every chunk issued so far (before blocking on a region)
-        auto publish_all = [&]() {
-            cp_async_wait<0>();
-            tc::fence_proxy_async_smem();
-            for (; signalled < issued; signalled++) tc::mbar_arrive(&chunk_full[signalled]);
-        };
-        for (int k = 0; k < kChunks; k++) {
-            const int dep = chunk_dep(k);
-            if (dep >= 0 && !tc::mbar_test_wait(&mma_done[dep], 0)) {
-                publish_all();
-                if (!tc::mbar_wait(&mma_done[dep], 0, a.err, abort)) {
-                    ok = false;
-                    break;
-                }
-            }
+        // ------------------------------------------------------------ gather
+        // Issue chunk k: 16-byte cp.async pieces (rows past the unit's end are
+        // zero-filled: finite values that meet P = 0).  bf16 rows and the FP8
+        // rotary block land in their swizzled tile; FP8 codes land in the
+        // upper half of the region, to be decoded in place.
+        auto issue = [&](int k) {
             const int cb = chunk_block(k, half);
             const uint32_t rg = sbase + chunk_region(k) * kRegion;
             if (!kFp8 || cb == 8) {
-                // 16-byte pieces straight into the swizzled tile; rows past the
-                // unit's end are zero-filled (finite values times P = 0)
                 for (int f = gt; f < U * 8; f += kWork) {
                     const int j = f >> 3, p = f & 7;
-                    const bool v = j < n_my;
-                    const int64_t t = v ? (int64_t)list[j] : 0;
+                    const int32_t tl = list[j];
+                    const bool v = tl >= 0;
+                    const int64_t t = v ? (int64_t)tl : 0;
                     const void *src;
                     if constexpr (kFp8)
                         src = a.kv8 + (rbase + t) * kRowFp8 + kDc + 4 * (kDc / 128) + p * 16;
@@ -313,187 +393,317 @@ sparse_mla_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const MlaArgs a) 
                     cp_async16(rg + j * 128 + ((p ^ (j & 7)) << 4), src, v ? 16u : 0u);
                 }
             } else {
-                // FP8 latent block cb: 16 codes per piece, decoded with the
-                // block's scale into two 16-byte bf16 pieces of the tile row
-                constexpr int kPer = kUnitMax * 4 / kWork;   // pieces per thread (4)
+                for (int f = gt; f < U * 4; f += kWork) {
+                    const int j = f >> 2, p = f & 3;
+                    const int32_t tl = list[j];
+                    const bool v = tl >= 0;
+                    const int64_t t = v ? (int64_t)tl : 0;
+                    cp_async16(rg + kRegion / 2 + j * 64 + p * 16,
+                               a.kv8 + (rbase + t) * kRowFp8 + cb * 64 + p * 16, v ? 16u : 0u);
+                }
+                if (k == 0 && gt < U) {                   // the row's four block scales
+                    const int32_t tl = list[gt];
+                    const bool v = tl >= 0;
+                    const int64_t t = v ? (int64_t)tl : 0;
+                    cp_async16(sbase + kScales + gt * 16, a.kv8 + (rbase + t) * kRowFp8 + kDc,
+                               v ? 16u : 0u);
+                }
+            }
+            cp_async_commit();
+        };
+        // Chunk k has landed for this thread (`pending` later groups may still
+        // be in flight): FP8 latent codes are decoded in place (every thread's
+        // codes must have landed before any are read, and every read must be
+        // done before the first write), then the chunk is published.
+        auto publish = [&](int k, int pending) {
+            cp_async_wait_n(pending);
+            const int cb = chunk_block(k, half);
+            if (kFp8 && cb != 8) {
+                const uint32_t rg = sbase + chunk_region(k) * kRegion;
+                constexpr int kPer = kUnitMax * 4 / kWork;   // 16-code pieces per thread
                 uint4 cw[kPer];
                 float sc[kPer];
+                tc::named_barrier(1, kWork);
 #pragma unroll
                 for (int u = 0; u < kPer; u++) {
                     const int f = gt + u * kWork, j = f >> 2, p = f & 3;
-                    cw[u] = make_uint4(0u, 0u, 0u, 0u);
-                    sc[u] = 0.f;
-                    if (j < n_my) {
-                        const uint8_t *r8 = a.kv8 + (rbase + list[j]) * kRowFp8;
-                        cw[u] = *reinterpret_cast<const uint4 *>(r8 + cb * 64 + p * 16);
-                        sc[u] = *reinterpret_cast<const float *>(r8 + kDc + 4 * (cb >> 1));
+                    if (j < U) {
+                        cw[u] = ld_shared_v4(rg + kRegion / 2 + j * 64 + p * 16);
+                        sc[u] = reinterpret_cast<const float *>(sm + kScales + j * 16)[cb >> 1];
                     }
                 }
+                tc::named_barrier(1, kWork);
 #pragma unroll
                 for (int u = 0; u < kPer; u++) {
                     const int f = gt + u * kWork, j = f >> 2, p = f & 3;
                     if (j >= U) continue;
-                    const uint4 lo8 = decode8(cw[u].x, cw[u].y, sc[u]);
-                    const uint4 hi8 = decode8(cw[u].z, cw[u].w, sc[u]);
-                    st_shared_v4(rg + j * 128 + (((2 * p) ^ (j & 7)) << 4), lo8);
-                    st_shared_v4(rg + j * 128 + (((2 * p + 1) ^ (j & 7)) << 4), hi8);
+                    st_shared_v4(rg + j * 128 + (((2 * p) ^ (j & 7)) << 4), decode8(cw[u].x, cw[u].y, sc[u]));
+                    st_shared_v4(rg + j * 128 + (((2 * p + 1) ^ (j & 7)) << 4), decode8(cw[u].z, cw[u].w, sc[u]));
                 }
             }
-            cp_async_commit();
-            issued = k + 1;
-            if (issued - signalled > kLag) {
-                cp_async_wait<kLag>();
-                tc::fence_proxy_async_smem();
-                tc::mbar_arrive(&chunk_full[signalled]);
-                signalled++;
+            tc::fence_proxy_async_smem();
+            tc::mbar_arrive(&chunk_full[k]);
+        };
+        // chunks 0 and 1 go to free regions at once; 2..5 once the query's
+        // latent part has left its staging in R2..R5.  bf16 chunks are
+        // published by the copies themselves (an arrival when this thread's
+        // copies have landed); FP8 latent chunks are decoded in place first.
+        auto start = [&](int k) {
+            issue(k);
+            if constexpr (!kFp8) cp_async_arrive(&chunk_full[k]);
+            else cp_async_commit();
+        };
+        start(0);
+        start(1);
+        // the query's latent part (head h, columns [256c, 256c + 256)) from its
+        // swizzled staging to TMEM columns kColQ + [128c, 128c + 128), two bf16
+        // per column
+        if (ok && !tc::mbar_wait(q_full, 0, a.err, abort)) ok = false;
+#pragma unroll 1
+        for (int blk = 0; blk < 4; blk++) {
+            const int cb = 4 * c + blk;
+            const uint32_t src = sbase + 2 * kRegion + cb * kQBlk + h * 128;
+#pragma unroll
+            for (int hf = 0; hf < 2; hf++) {
+                uint32_t r[16];
+#pragma unroll
+                for (int i = 0; i < 4; i++) {
+                    const uint4 v = ld_shared_v4(src + (((4 * hf + i) ^ (h & 7)) << 4));
+                    r[4 * i] = v.x; r[4 * i + 1] = v.y; r[4 * i + 2] = v.z; r[4 * i + 3] = v.w;
+                }
+                tc::tmem_st16(tmem + lane_addr + kColQ + cb * 32 + hf * 16, r);
             }
         }
-        publish_all();
+        tc::tmem_wait_st();
+        tc::tc_fence_before();
+        tc::mbar_arrive(q_ready);
+        tc::named_barrier(1, kWork);            // the staging is no longer read
+        for (int k = 2; k < kRegions; k++) start(k);
+        if constexpr (kFp8)
+            for (int k = 0; k < kRegions; k++) publish(k, kRegions - 1 - k);
+        // chunks 6..8 reuse regions: wait for the MMA that read them last
+        for (int k = kRegions; k < kChunks; k++) {
+            if (ok && !tc::mbar_wait(&mma_done[chunk_dep(k)], 0, a.err, abort)) ok = false;
+            if (ok) start(k);
+            else if constexpr (kFp8) cp_async_commit();
+            else tc::mbar_arrive(&chunk_full[k]);
+        }
+        if constexpr (kFp8)
+            for (int k = kRegions; k < kChunks; k++) publish(k, kChunks - 1 - k);
 
         // ----------------------------------------------------------- softmax
-        // thread (head h, column half c): logits of rows [c U/2, (c+1) U/2)
-        const int q4 = warp & 3, c = warp >> 2;
-        const int h = q4 * 32 + lane;
-        const uint32_t lane_addr = (uint32_t)(q4 * 32) << 16;
+        // thread (head h, column half c): logits of rows [c U/2, (c+1) U/2).
+        // This thread's logits (up to 128) in two TMEM reads of 64 columns per
+        // pass (nine warps leave at most 168 registers a thread).  Logits of
+        // rows past the unit's end count as -inf; eight independent max and
+        // sum chains keep the dependent latency short.
         const int hc = U / 2, base = c * hc;
         if (ok && !tc::mbar_wait(&mma_done[kChunks - 1], 0, a.err, abort)) ok = false;
         tc::tc_fence_after();
-        float mx = -INFINITY;
-        for (int i = 0; i < hc; i += 32) {
-            uint32_t r0[16], r1[16];
-            tc::tmem_ld16(tmem + lane_addr + kColS + base + i, r0);
-            tc::tmem_ld16(tmem + lane_addr + kColS + base + i + 16, r1);
-            tc::tmem_wait_ld();
+        // validity bits of rows [base + 64g, base + 64g + 64), none past hc
+        auto rowbits = [&](int g, uint32_t &w0, uint32_t &w1) {
+            w0 = vmask[(base + 64 * g) >> 5];
+            w1 = 64 * g + 32 < hc ? vmask[((base + 64 * g) >> 5) + 1] : 0u;
+        };
+        float mx8[8];
 #pragma unroll
-            for (int e = 0; e < 16; e++) {
-                if (base + i + e < n_my) mx = fmaxf(mx, __uint_as_float(r0[e]) * a.scale_log2);
-                if (base + i + 16 + e < n_my) mx = fmaxf(mx, __uint_as_float(r1[e]) * a.scale_log2);
+        for (int e = 0; e < 8; e++) mx8[e] = -INFINITY;
+#pragma unroll
+        for (int g = 0; g < 2; g++) {
+            if (64 * g >= hc) break;
+            uint32_t sv[64];
+#pragma unroll
+            for (int i = 0; i < 4; i++)
+                if (64 * g + 16 * i < hc)
+                    tc::tmem_ld16(tmem + lane_addr + kColS + base + 64 * g + 16 * i,
+                                  *reinterpret_cast<uint32_t(*)[16]>(sv + 16 * i));
+            tc::tmem_wait_ld();
+            uint32_t w0, w1;
+            rowbits(g, w0, w1);
+            const bool part = (w0 & w1) != 0xffffffffu;
+#pragma unroll
+            for (int e = 0; e < 64; e++) {
+                float x = __uint_as_float(sv[e]) * a.scale_log2;
+                if (part && !(((e < 32 ? w0 : w1) >> (e & 31)) & 1u)) x = -INFINITY;
+                mx8[e & 7] = fmaxf(mx8[e & 7], x);
             }
         }
+        const float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
+                               fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
         red[c * kHq + h] = mx;
         tc::named_barrier(1, kWork);
         const float m = fmaxf(red[h], red[kHq + h]);       // finite: row 0 is valid
-        float l = 0.f;
-        for (int i = 0; i < hc; i += 32) {
-            uint32_t r0[16], r1[16], pk[16];
-            tc::tmem_ld16(tmem + lane_addr + kColS + base + i, r0);
-            tc::tmem_ld16(tmem + lane_addr + kColS + base + i + 16, r1);
-            tc::tmem_wait_ld();
+        float l8[8];
 #pragma unroll
-            for (int e = 0; e < 8; e++) {
-                const int j0 = base + i + 2 * e;
-                const float p0 = j0 < n_my ? exp2f(fmaf(__uint_as_float(r0[2 * e]), a.scale_log2, -m)) : 0.f;
-                const float p1 = j0 + 1 < n_my ? exp2f(fmaf(__uint_as_float(r0[2 * e + 1]), a.scale_log2, -m)) : 0.f;
-                const float p2 = j0 + 16 < n_my ? exp2f(fmaf(__uint_as_float(r1[2 * e]), a.scale_log2, -m)) : 0.f;
-                const float p3 = j0 + 17 < n_my ? exp2f(fmaf(__uint_as_float(r1[2 * e + 1]), a.scale_log2, -m)) : 0.f;
-                l += (p0 + p1) + (p2 + p3);
-                const __nv_bfloat162 v01 = __floats2bfloat162_rn(p0, p1);
-                const __nv_bfloat162 v23 = __floats2bfloat162_rn(p2, p3);
-                pk[e] = *reinterpret_cast<const uint32_t *>(&v01);
-                pk[8 + e] = *reinterpret_cast<const uint32_t *>(&v23);
+        for (int e = 0; e < 8; e++) l8[e] = 0.f;
+        // P of this thread's rows over the first half of its logits, 32 rows
+        // (16 columns) per store
+#pragma unroll
+        for (int g = 0; g < 2; g++) {
+            if (64 * g >= hc) break;
+            uint32_t sv[64];
+#pragma unroll
+            for (int i = 0; i < 4; i++)
+                if (64 * g + 16 * i < hc)
+                    tc::tmem_ld16(tmem + lane_addr + kColS + base + 64 * g + 16 * i,
+                                  *reinterpret_cast<uint32_t(*)[16]>(sv + 16 * i));
+            tc::tmem_wait_ld();
+            uint32_t w0, w1;
+            rowbits(g, w0, w1);
+            const bool part = (w0 & w1) != 0xffffffffu;
+#pragma unroll
+            for (int i = 0; i < 2; i++) {
+                uint32_t pk[16];
+#pragma unroll
+                for (int e = 0; e < 16; e++) {
+                    const int x = 32 * i + 2 * e;
+                    float t0 = fmaf(__uint_as_float(sv[x]), a.scale_log2, -m);
+                    float t1 = fmaf(__uint_as_float(sv[x + 1]), a.scale_log2, -m);
+                    const uint32_t wb = i == 0 ? w0 : w1;
+                    if (part && !((wb >> (2 * e)) & 1u)) t0 = -INFINITY;
+                    if (part && !((wb >> (2 * e + 1)) & 1u)) t1 = -INFINITY;
+                    const float p0 = ex2(t0), p1 = ex2(t1);
+                    l8[e & 7] += p0 + p1;
+                    const __nv_bfloat162 v01 = __floats2bfloat162_rn(p0, p1);
+                    pk[e] = *reinterpret_cast<const uint32_t *>(&v01);
+                }
+                // rows [base + 64g + 32i, +32) -> columns base + 32g + 16i (their
+                // logits were read above)
+                if (64 * g + 32 * i < hc)
+                    tc::tmem_st16(tmem + lane_addr + kColS + base + 32 * g + 16 * i, pk);
             }
-            // P of rows [base + i, base + i + 32) over the logits already read
-            tc::tmem_st16(tmem + lane_addr + kColS + base + i / 2, pk);
         }
         tc::tmem_wait_st();
         tc::tc_fence_before();
         tc::mbar_arrive(p_full);
-        red[2 * kHq + c * kHq + h] = l;
+        red[2 * kHq + c * kHq + h] = ((l8[0] + l8[1]) + (l8[2] + l8[3])) + ((l8[4] + l8[5]) + (l8[6] + l8[7]));
         tc::named_barrier(1, kWork);
         const float lt = red[2 * kHq + h] + red[3 * kHq + h];
 
         // ---------------------------------------------------------- epilogue
-        // thread (h, c) writes output columns [128c, 128c + 128) of this CTA's 256
+        // thread (h, c) owns output columns [128c, 128c + 128) of this CTA's 256
         if (ok && !tc::mbar_wait(o_full, 0, a.err, abort)) ok = false;
         tc::tc_fence_after();
         const uint32_t ocol = tmem + lane_addr + kColO + c * 128;
-        if (a.splits > 1) {
-            // O / (l * sc) in fp16, sc the power of two that keeps |O / l| / sc
-            // <= 2^14, as [column / 8][head] groups of eight halves
-            float amax = 0.f;
-            for (int j = 0; j < 128; j += 16) {
-                uint32_t o[16];
-                tc::tmem_ld16(ocol + j, o);
-                tc::tmem_wait_ld();
-#pragma unroll
-                for (int e = 0; e < 16; e++) amax = fmaxf(amax, fabsf(__uint_as_float(o[e])));
-            }
-            red[4 * kHq + c * kHq + h] = amax;
-            tc::named_barrier(1, kWork);
-            amax = fmaxf(red[4 * kHq + h], red[5 * kHq + h]);
-            const float inv_l = lt > 0.f ? 1.f / lt : 0.f;
-            float scl = 1.f;
-            while (amax * inv_l > 16384.f * scl) scl *= 2.f;
-            const float inv = inv_l / scl;
-            uint4 *po = reinterpret_cast<uint4 *>(a.part_o + (int64_t)unit * kHq * 256) + h;
-            for (int j = 0; j < 128; j += 16) {
-                uint32_t o[16], w[8];
-                tc::tmem_ld16(ocol + j, o);
-                tc::tmem_wait_ld();
-#pragma unroll
-                for (int e = 0; e < 8; e++) {
-                    const __half2 v = __floats2half2_rn(__uint_as_float(o[2 * e]) * inv,
-                                                        __uint_as_float(o[2 * e + 1]) * inv);
-                    w[e] = *reinterpret_cast<const uint32_t *>(&v);
-                }
-                if (ok) {
-                    const int o8 = (c * 128 + j) / 8;
-                    po[o8 * kHq] = make_uint4(w[0], w[1], w[2], w[3]);
-                    po[(o8 + 1) * kHq] = make_uint4(w[4], w[5], w[6], w[7]);
-                }
-            }
-            if (ok && c == 0) a.part_ml[(int64_t)unit * kHq + h] = make_float4(m, lt, scl, 0.f);
-        } else {
+        if (a.splits == 1) {
             const float inv = lt > 0.f ? 1.f / lt : 0.f;
             uint4 *o16 = reinterpret_cast<uint4 *>(a.out + (row * kHq + h) * kDc + half * 256 + c * 128);
-            for (int j = 0; j < 128; j += 16) {
-                uint32_t o[16], w[8];
-                tc::tmem_ld16(ocol + j, o);
+#pragma unroll
+            for (int g = 0; g < 2; g++) {
+                uint32_t ov[64];
+#pragma unroll
+                for (int i = 0; i < 4; i++)
+                    tc::tmem_ld16(ocol + 64 * g + 16 * i, *reinterpret_cast<uint32_t(*)[16]>(ov + 16 * i));
                 tc::tmem_wait_ld();
 #pragma unroll
-                for (int e = 0; e < 8; e++) {
-                    const __nv_bfloat162 v = __floats2bfloat162_rn(__uint_as_float(o[2 * e]) * inv,
-                                                                   __uint_as_float(o[2 * e + 1]) * inv);
-                    w[e] = *reinterpret_cast<const uint32_t *>(&v);
-                }
-                if (ok) {
-                    o16[j / 8] = make_uint4(w[0], w[1], w[2], w[3]);
-                    o16[j / 8 + 1] = make_uint4(w[4], w[5], w[6], w[7]);
+                for (int o8 = 0; o8 < 8; o8++) {
+                    uint32_t w[4];
+#pragma unroll
+                    for (int e = 0; e < 4; e++) {
+                        const __nv_bfloat162 v = __floats2bfloat162_rn(__uint_as_float(ov[8 * o8 + 2 * e]) * inv,
+                                                                       __uint_as_float(ov[8 * o8 + 2 * e + 1]) * inv);
+                        w[e] = *reinterpret_cast<const uint32_t *>(&v);
+                    }
+                    if (ok) o16[g * 8 + o8] = make_uint4(w[0], w[1], w[2], w[3]);
                 }
             }
             if (ok && half == 0 && c == 0 && a.lse)
                 a.lse[row * kHq + h] = lt > 0.f ? (m + log2f(lt)) * kLn2 : -INFINITY;
+        } else {
+            // O / (l * sc) in fp16 for the split combine, sc the power of two
+            // that keeps this column half's |O / l| / sc <= 2^14, as
+            // [column / 8][head] groups of eight halves
+            uint32_t ov[2][64];
+            float amax = 0.f;
+#pragma unroll
+            for (int g = 0; g < 2; g++) {
+#pragma unroll
+                for (int i = 0; i < 4; i++)
+                    tc::tmem_ld16(ocol + 64 * g + 16 * i, *reinterpret_cast<uint32_t(*)[16]>(ov[g] + 16 * i));
+            }
+            tc::tmem_wait_ld();
+#pragma unroll
+            for (int g = 0; g < 2; g++)
+#pragma unroll
+                for (int e = 0; e < 64; e++) amax = fmaxf(amax, fabsf(__uint_as_float(ov[g][e])));
+            const float inv_l = lt > 0.f ? 1.f / lt : 0.f;
+            float scl = 1.f;
+            while (amax * inv_l > 16384.f * scl) scl *= 2.f;
+            const float inv = inv_l / scl;
+            uint4 *po = reinterpret_cast<uint4 *>(a.part_o + (int64_t)blockIdx.x * kHq * 256) + h;
+#pragma unroll
+            for (int g = 0; g < 2; g++) {
+#pragma unroll
+                for (int o8 = 0; o8 < 8; o8++) {
+                    uint32_t w[4];
+#pragma unroll
+                    for (int e = 0; e < 4; e++) {
+                        const __half2 v = __floats2half2_rn(__uint_as_float(ov[g][8 * o8 + 2 * e]) * inv,
+                                                            __uint_as_float(ov[g][8 * o8 + 2 * e + 1]) * inv);
+                        w[e] = *reinterpret_cast<const uint32_t *>(&v);
+                    }
+                    if (ok) po[(c * 16 + g * 8 + o8) * kHq] = make_uint4(w[0], w[1], w[2], w[3]);
+                }
+            }
+            // (max, sum, range of columns [0, 128), range of columns [128, 256))
+            float *ml = reinterpret_cast<float *>(a.part_ml + (int64_t)blockIdx.x * kHq + h);
+            if (ok) {
+                if (c == 0) {
+                    ml[0] = m;
+                    ml[1] = lt;
+                }
+                ml[2 + c] = scl;
+            }
         }
-    } else if (lane == 0) {
+    } else if (lane > 0) {
+        // lanes 1..31 of the MMA warp: each CTA of the unit prefetches every
+        // other row into L2 (its partner the rest), whole rows at a time
+        for (int j = 2 * (lane - 1) + half; j < U; j += 62) {
+            if (list[j] < 0) continue;
+            if constexpr (kFp8)
+                tc::prefetch_l2_bulk(a.kv8 + (rbase + list[j]) * kRowFp8, kRowFp8);
+            else
+                tc::prefetch_l2_bulk(a.kv + (rbase + list[j]) * kDqk, kDqk * 2);
+        }
+    } else {
         // ------------------------------------------------------ TMA / MMA
         const uint32_t id_qk = tc::instr_desc(tc::kFmtBF16, tc::kFmtBF16, 128, U);
-        const uint32_t id_pv = tc::instr_desc(tc::kFmtBF16, tc::kFmtBF16, 128, 256, true);
-        bool ok = tc::mbar_wait(q_full, 0, a.err, abort);
+        bool ok = tc::mbar_wait(q_full, 0, a.err, abort) && tc::mbar_wait(q_ready, 0, a.err, abort);
         for (int k = 0; ok && k < kChunks; k++) {
             if (!tc::mbar_wait(&chunk_full[k], 0, a.err, abort)) {
                 ok = false;
                 break;
             }
+            // the chunk's bytes were written through the generic proxy (cp.async
+            // or stores): order them before the tensor core's reads
+            tc::fence_proxy_async_smem();
             tc::tc_fence_after();
-            const uint32_t qa = sbase + q_offset(k), ca = sbase + chunk_region(k) * kRegion;
+            const int cb = chunk_block(k, half);
+            const uint32_t ca = sbase + chunk_region(k) * kRegion;
 #pragma unroll
             for (int ks = 0; ks < 4; ks++) {
-                const uint64_t ad = tc::smem_desc(qa + ks * 32, 1024, tc::kSwizzle128B);
                 const uint64_t bd = tc::smem_desc(ca + ks * 32, 1024, tc::kSwizzle128B);
-                tc::mma_f16(tmem + kColS, ad, bd, id_qk, k > 0 || ks > 0);
+                if (cb < 8)        // A = the query's latent block cb in TMEM
+                    tc::mma_f16_ts(tmem + kColS, tmem + kColQ + cb * 32 + ks * 8, bd, id_qk,
+                                   k > 0 || ks > 0);
+                else               // A = the query's rotary block in shared memory
+                    tc::mma_f16(tmem + kColS,
+                                tc::smem_desc(sbase + kQRope + ks * 32, 1024, tc::kSwizzle128B), bd,
+                                id_qk, k > 0 || ks > 0);
             }
             tc::tc_commit(&mma_done[k]);
         }
         if (ok && tc::mbar_wait(p_full, 0, a.err, abort)) {
             tc::tc_fence_after();
             // O += P C[:, own 256]: K-step ks covers rows [16 ks, 16 ks + 16),
-            // whose P sits in the first quarter of its column half
+            // whose P sits in the first quarter of its column half; B = the own
+            // chunks in R0..R3
+            const uint32_t id_pv = tc::instr_desc(tc::kFmtBF16, tc::kFmtBF16, 128, 256, true);
             const int hc = U / 2;
             for (int ks = 0; ks < U / 16; ks++) {
                 const int r0 = 16 * ks, c = r0 / hc;
                 const uint32_t pa = tmem + kColS + c * hc + (r0 - c * hc) / 2;
-                const uint64_t bd = tc::smem_desc(sbase + kRegion + ks * 2048, 1024,
-                                                  tc::kSwizzle128B, kRegion);
+                const uint64_t bd = tc::smem_desc(sbase + ks * 2048, 1024, tc::kSwizzle128B, kRegion);
                 tc::mma_f16_ts(tmem + kColO, pa, bd, id_pv, ks > 0);
             }
             tc::tc_commit(o_full);
@@ -508,65 +718,42 @@ sparse_mla_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const MlaArgs a) 
         tc::tc_fence_after();
         tc::tmem_dealloc(tmem, kTmemCols);
     }
+    if (a.coop) {
+        // every split of every row has written its partial: merge this
+        // split's slice of its (row, half)'s output columns (32 / splits
+        // octets of eight columns)
+        cooperative_groups::this_grid().sync();
+        const int npo = 32 / a.splits;
+        const int h = threadIdx.x & (kHq - 1), o = threadIdx.x >> 7;
+        const int64_t blk0 = (int64_t)blockIdx.x - sp;
+        if (threadIdx.x < kWork) {
+            // thread (h, o): octets o, o + 2, ... of the slice, two at a time
+            int oc = o;
+            for (; oc + 2 < npo; oc += 4) {
+                const int c8[2] = {npo * sp + oc, npo * sp + oc + 2};
+                merge_octets<2>(a.part_o, a.part_ml, a.splits, blk0, row, half, c8, h, a.out, a.lse);
+            }
+            if (oc < npo) {
+                const int c8[1] = {npo * sp + oc};
+                merge_octets<1>(a.part_o, a.part_ml, a.splits, blk0, row, half, c8, h, a.out, a.lse);
+            }
+        }
+    }
 }
 
-// Merges the splits of each (row, half): with w_s = 2^(m_s - m) l_s and the
-// stored partials Y_s = O_s / (l_s sc_s), out = sum_s w_s sc_s Y_s / sum_s w_s.
-// The partials are [column / 8][head] groups of eight halves; thread (head,
-// octet) merges eight output columns of one head, consecutive threads
-// consecutive heads (coalesced).
+// Merges the splits of each (row, half) when the attention grid is not
+// cooperative: thread (head, octet) merges eight output columns of one head,
+// consecutive threads consecutive heads (coalesced reads of the partials).
 __global__ void __launch_bounds__(kHq)
-sparse_mla_combine_kernel(const __half *part_o, const float4 *part_ml, int splits,
+sparse_mla_combine_kernel(const __half *part_o, const float4 *part_ml, int splits, int64_t row0,
                           __nv_bfloat16 *__restrict__ out, float *__restrict__ lse) {
     // the partials come from the preceding kernel: wait for it (plain loads below)
     asm volatile("griddepcontrol.wait;" ::: "memory");
     constexpr int groups = 256 / 8;
-    const int64_t rh = blockIdx.x / groups;                 // row * 2 + half
-    const int64_t row = rh >> 1;
-    const int half = (int)(rh & 1);
-    const int h = threadIdx.x;
-    const int c8 = (int)(blockIdx.x % groups);
-    // partial of split sp: unit (row * splits + sp) * 2 + half
-    const int64_t u0 = row * splits * 2 + half;
-    float m = -INFINITY;
-    for (int sp = 0; sp < splits; sp++) m = fmaxf(m, part_ml[(u0 + 2 * sp) * kHq + h].x);
-    float L = 0.f;
-    float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-    // four splits at a time, so that their loads are in flight together
-    for (int sp0 = 0; sp0 < splits; sp0 += 4) {
-        float4 ml[4];
-        uint4 x[4];
-#pragma unroll
-        for (int u = 0; u < 4; u++) {
-            const int sp = sp0 + u;
-            ml[u] = sp < splits ? part_ml[(u0 + 2 * sp) * kHq + h] : make_float4(-INFINITY, 0.f, 1.f, 0.f);
-            if (sp < splits)
-                x[u] = reinterpret_cast<const uint4 *>(part_o + (u0 + 2 * sp) * kHq * 256)[c8 * kHq + h];
-        }
-#pragma unroll
-        for (int u = 0; u < 4; u++) {
-            if (ml[u].x == -INFINITY) continue;
-            const float w = exp2f(ml[u].x - m) * ml[u].y;
-            L += w;
-            const float ws = w * ml[u].z;
-            const uint32_t xs[4] = {x[u].x, x[u].y, x[u].z, x[u].w};
-#pragma unroll
-            for (int e = 0; e < 4; e++) {
-                const float2 f = __half22float2(*reinterpret_cast<const __half2 *>(&xs[e]));
-                acc[2 * e] += ws * f.x;
-                acc[2 * e + 1] += ws * f.y;
-            }
-        }
-    }
-    const float inv = L > 0.f ? 1.f / L : 0.f;
-    uint32_t w8[4];
-#pragma unroll
-    for (int e = 0; e < 4; e++) {
-        const __nv_bfloat162 v = __floats2bfloat162_rn(acc[2 * e] * inv, acc[2 * e + 1] * inv);
-        w8[e] = *reinterpret_cast<const uint32_t *>(&v);
-    }
-    reinterpret_cast<uint4 *>(out + (row * kHq + h) * kDc + half * 256)[c8] = make_uint4(w8[0], w8[1], w8[2], w8[3]);
-    if (half == 0 && c8 == 0 && lse) lse[row * kHq + h] = L > 0.f ? (m + log2f(L)) * kLn2 : -INFINITY;
+    const int64_t rh = blockIdx.x / groups;                 // (row - row0) * 2 + half
+    const int c8[1] = {(int)(blockIdx.x % groups)};
+    merge_octets<1>(part_o, part_ml, splits, rh * splits, row0 + (rh >> 1), (int)(rh & 1), c8,
+                    threadIdx.x, out, lse);
 }
 
 // Rows per unit: the smallest of 64, 128, 192, 256 whose units (two CTAs
@@ -577,11 +764,27 @@ int mla_unit_rows(int64_t rows, int k) {
     return kUnitMax;
 }
 
+// Split partials of one query row (both output halves of every split).
+size_t partial_bytes_per_row(int splits) {
+    return (size_t)2 * splits * kHq * (256 * sizeof(__half) + sizeof(float4));
+}
+
+// Query rows per launch: all of them, unless their split partials would pass
+// kWsBudget; then the rows run in launches of this many (each reusing the
+// workspace after its combine).
+constexpr size_t kWsBudget = size_t(256) << 20;
+int64_t rows_per_launch(int64_t rows, int splits) {
+    if (splits <= 1) return rows;
+    int64_t r = (int64_t)(kWsBudget / partial_bytes_per_row(splits));
+    if (r < 1) r = 1;
+    return r < rows ? r : rows;
+}
+
 size_t workspace_bytes(int64_t rows, int k) {
     const int u = mla_unit_rows(rows, k);
     const int sp = (k + u - 1) / u;
     if (sp <= 1) return 0;
-    const int64_t units = rows * 2 * sp;
+    const int64_t units = rows_per_launch(rows, sp) * 2 * sp;
     return align_up((size_t)units * kHq * 256 * sizeof(__half), 256) +
            (size_t)units * kHq * sizeof(float4);
 }
@@ -601,6 +804,7 @@ dsa_status launch(const void *q, const void *kv, int64_t t_max, const int32_t *i
             return DSA_ERR_CUDA;
     }
     MlaArgs a = {};
+    a.q = static_cast<const __nv_bfloat16 *>(q);
     a.kv = kFp8 ? nullptr : static_cast<const __nv_bfloat16 *>(kv);
     a.kv8 = kFp8 ? static_cast<const uint8_t *>(kv) : nullptr;
     a.idx = idx;
@@ -614,8 +818,9 @@ dsa_status launch(const void *q, const void *kv, int64_t t_max, const int32_t *i
     a.splits = (k + a.unit_rows - 1) / a.unit_rows;
     a.scale_log2 = sm_scale * kLog2e;
     a.err = device_error_word();
+    const int64_t chunk = rows_per_launch(rows, a.splits);
     if (a.splits > 1) {
-        const int64_t units = rows * 2 * a.splits;
+        const int64_t units = chunk * 2 * a.splits;
         a.part_o = static_cast<__half *>(ws);
         a.part_ml = reinterpret_cast<float4 *>(static_cast<char *>(ws) +
                                                align_up((size_t)units * kHq * 256 * sizeof(__half), 256));
@@ -623,35 +828,69 @@ dsa_status launch(const void *q, const void *kv, int64_t t_max, const int32_t *i
     if (cudaFuncSetAttribute(sparse_mla_tc_kernel<kFp8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)kSmemBytes) != cudaSuccess)
         return DSA_ERR_CUDA;
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3((unsigned)(rows * a.splits * 2));
-    cfg.blockDim = dim3(kThreads);
-    cfg.dynamicSmemBytes = kSmemBytes;
-    cfg.stream = stream;
-    // programmatic launch: the kernel's set-up overlaps the preceding kernel's
-    // tail; it waits for that kernel before reading the selections
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[0].val.programmaticStreamSerializationAllowed = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    if (cudaLaunchKernelEx(&cfg, sparse_mla_tc_kernel<kFp8>, tm_q, a) != cudaSuccess)
-        return DSA_ERR_CUDA;
-    dsa_status st = launch_status();
-    if (st != DSA_OK || a.splits == 1) return st;
-    cudaLaunchConfig_t ccfg = {};
-    ccfg.gridDim = dim3((unsigned)(rows * 2 * (256 / 8)));
-    ccfg.blockDim = dim3(kHq);
-    ccfg.stream = stream;
-    cudaLaunchAttribute cattr[1];
-    cattr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    cattr[0].val.programmaticStreamSerializationAllowed = 1;
-    ccfg.attrs = cattr;
-    ccfg.numAttrs = 1;
-    if (cudaLaunchKernelEx(&ccfg, sparse_mla_combine_kernel, (const __half *)a.part_o,
-                           (const float4 *)a.part_ml, a.splits, a.out, lse) != cudaSuccess)
-        return DSA_ERR_CUDA;
-    return launch_status();
+    // The splits are merged inside the attention grid when the grid can be
+    // cooperative (all of its CTAs resident at once, one launch) and each
+    // split gets whole octets of columns; else a combine kernel follows.
+    bool coop = false;
+    if (a.splits > 1 && 32 % a.splits == 0 && chunk == rows) {
+        int per_sm = 0;
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, sparse_mla_tc_kernel<kFp8>,
+                                                          kThreads, kSmemBytes) == cudaSuccess &&
+            (int64_t)per_sm * num_sms() >= rows * a.splits * 2)
+            coop = true;
+    }
+    for (int64_t r0 = 0; r0 < rows; r0 += chunk) {
+        const int64_t n = rows - r0 < chunk ? rows - r0 : chunk;
+        a.row0 = r0;
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3((unsigned)(n * a.splits * 2));
+        cfg.blockDim = dim3(kThreads);
+        cfg.dynamicSmemBytes = kSmemBytes;
+        cfg.stream = stream;
+        // programmatic launch: the kernel's set-up overlaps the preceding
+        // kernel's tail; it waits for that kernel before reading the selections
+        cudaLaunchAttribute attr[2];
+        attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[0].val.programmaticStreamSerializationAllowed = 1;
+        attr[1].id = cudaLaunchAttributeCooperative;
+        attr[1].val.cooperative = 1;
+        cfg.attrs = attr;
+        bool launched = false;
+        if (coop) {
+            // cooperative, first with the programmatic launch, then without it
+            a.coop = 1;
+            for (int first = 0; first < 2 && !launched; first++) {
+                cfg.attrs = attr + first;
+                cfg.numAttrs = 2 - first;
+                launched = cudaLaunchKernelEx(&cfg, sparse_mla_tc_kernel<kFp8>, tm_q, a) == cudaSuccess;
+                if (!launched) (void)cudaGetLastError();
+            }
+        }
+        if (!launched) {
+            a.coop = 0;
+            cfg.attrs = attr;
+            cfg.numAttrs = 1;
+            if (cudaLaunchKernelEx(&cfg, sparse_mla_tc_kernel<kFp8>, tm_q, a) != cudaSuccess)
+                return DSA_ERR_CUDA;
+        }
+        dsa_status st = launch_status();
+        if (st != DSA_OK) return st;
+        if (a.splits == 1 || a.coop) continue;
+        cudaLaunchConfig_t ccfg = {};
+        ccfg.gridDim = dim3((unsigned)(n * 2 * (256 / 8)));
+        ccfg.blockDim = dim3(kHq);
+        ccfg.stream = stream;
+        cudaLaunchAttribute cattr[1];
+        cattr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        cattr[0].val.programmaticStreamSerializationAllowed = 1;
+        ccfg.attrs = cattr;
+        ccfg.numAttrs = 1;
+        if (cudaLaunchKernelEx(&ccfg, sparse_mla_combine_kernel, (const __half *)a.part_o,
+                               (const float4 *)a.part_ml, a.splits, r0, a.out, lse) != cudaSuccess)
+            return DSA_ERR_CUDA;
+        if ((st = launch_status()) != DSA_OK) return st;
+    }
+    return DSA_OK;
 }
 
 }  // namespace

@@ -1,8 +1,9 @@
 // topk.cu -- per-query top-k selection over the causal positions.
 //
-// Page: "DeepSeek-V3.2-Exp - Split indexer heads", Indexer.forward:
-//   topk_indices = index_score.topk(min(index_topk, end_pos), dim=-1)[1]
-// with the causal mask of "DeepSeek-V3.2-Exp - Causal mask" applied first.
+// Page: "DeepSeek-V3.2-Exp - Split indexer heads", Indexer.forward, top-k
+// step: each query keeps the positions of its min(index_topk, end_pos)
+// largest index scores, after the causal mask of "DeepSeek-V3.2-Exp - Causal
+// mask" (Transformer.forward) has set the future positions to -inf.
 // Rows with fewer causal positions than K are padded with -1 (the warm-up
 // sentinel of the DeepSeek-V4 mask visualiser) instead of masked positions.
 //
@@ -203,9 +204,24 @@ __device__ void cta_select_keys(const uint32_t *keys, int n, unsigned rank, unsi
 
 constexpr int kGather = 8192;      // candidates CTA 0 can select alone
 
+// Rows of a cache the next kernel gathers at the selected positions: the
+// top-k asks L2 for each selected row as it writes the position (a no-op
+// when base is null), so that the gather finds them there.
+struct RowPrefetch {
+    const uint8_t *base;    // row (b, t) at base + (b * t_max + t) * bytes
+    int64_t t_max;
+    int bytes;              // a multiple of 16
+    __device__ __forceinline__ void operator()(int64_t b, int64_t t) const {
+        if (base)
+            asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(base + (b * t_max + t) * bytes),
+                         "r"(bytes)
+                         : "memory");
+    }
+};
+
 __global__ void __launch_bounds__(kThreads, 1)
 topk_cluster_kernel(const float *scores, int S, int64_t T, int64_t start_pos, int K,
-                    int L, int store_bins, int32_t *__restrict__ idx) {
+                    int L, int store_bins, int32_t *__restrict__ idx, const RowPrefetch pf) {
     // a kernel launched after this one (the sparse attention) may start its
     // set-up now; it reads the selections only after waiting for this grid
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
@@ -213,15 +229,22 @@ topk_cluster_kernel(const float *scores, int S, int64_t T, int64_t start_pos, in
     const int CN = (int)cl.num_blocks();
     const int p = (int)cl.block_rank();
     const int64_t row = blockIdx.x / CN;
-    const int64_t s = row % S;
+    const int64_t s = row % S, bseq = row / S;
     int64_t n_valid = start_pos + s + 1;
     if (n_valid > T) n_valid = T;
     const int m = (int64_t)K < n_valid ? K : (int)n_valid;
     int32_t *dst = idx + row * K;
+    // The scores come from the preceding kernel (the scorer), and a kernel
+    // before that may still read this row's old selections (an attention
+    // launched ahead of this top-k): wait for the preceding grid (a no-op
+    // without a programmatic launch) before reading or writing anything.
+    asm volatile("griddepcontrol.wait;" ::: "memory");
 
     if (m == n_valid) {                   // every causal position is selected
-        for (int i = p * kThreads + threadIdx.x; i < K; i += CN * kThreads)
+        for (int i = p * kThreads + threadIdx.x; i < K; i += CN * kThreads) {
             dst[i] = i < m ? i : -1;
+            if (i < m) pf(bseq, i);
+        }
         return;                           // uniform across the cluster
     }
 
@@ -247,9 +270,6 @@ topk_cluster_kernel(const float *scores, int S, int64_t T, int64_t start_pos, in
     const int len = t1 > t0 ? (int)(t1 - t0) : 0;
     const float *src = scores + row * T + t0;
 
-    // The scores come from the preceding kernel (the scorer): wait for it (a
-    // no-op without a programmatic launch); plain loads stay after the wait.
-    asm volatile("griddepcontrol.wait;" ::: "memory");
     // load the slice, finite min / max; clear the histograms
     // (loads are issued in batches of eight per thread so their latencies overlap)
     float lo = INFINITY, hi = -INFINITY;
@@ -520,7 +540,10 @@ topk_cluster_kernel(const float *scores, int S, int64_t T, int64_t start_pos, in
                 my_q--;
             }
         }
-        if (take && pos < m) dst[pos++] = (int32_t)(t0 + i);
+        if (take && pos < m) {
+            dst[pos++] = (int32_t)(t0 + i);
+            pf(bseq, t0 + i);
+        }
     }
     for (int i = m + p * kThreads + threadIdx.x; i < K; i += CN * kThreads) dst[i] = -1;
 }
@@ -617,7 +640,9 @@ void cluster_plan(int64_t n, int *cn, int *slice) {
 size_t topk_workspace_bytes(int, int, int64_t, int) { return 0; }
 
 dsa_status launch_topk_select(const float *scores, int B, int S, int64_t T, int64_t start_pos,
-                              int k, int32_t *idx, void *, cudaStream_t stream) {
+                              int k, int32_t *idx, void *, cudaStream_t stream,
+                              const void *prefetch_rows, int64_t prefetch_t_max,
+                              int prefetch_row_bytes) {
     if ((int64_t)B * S * T == 0) return DSA_OK;
     const int K = (int64_t)k < T ? k : (int)T;
     const int64_t rows = (int64_t)B * S;
@@ -657,8 +682,12 @@ dsa_status launch_topk_select(const float *scores, int B, int S, int64_t T, int6
     attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 2;
-    if (cudaLaunchKernelEx(&cfg, topk_cluster_kernel, scores, S, T, start_pos, K, L, store_bins, idx) !=
-        cudaSuccess)
+    RowPrefetch pf;
+    pf.base = static_cast<const uint8_t *>(prefetch_rows);
+    pf.t_max = prefetch_t_max;
+    pf.bytes = prefetch_row_bytes;
+    if (cudaLaunchKernelEx(&cfg, topk_cluster_kernel, scores, S, T, start_pos, K, L, store_bins, idx,
+                           pf) != cudaSuccess)
         return DSA_ERR_CUDA;
     return launch_status();
 }
