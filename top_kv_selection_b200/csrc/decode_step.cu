@@ -14,12 +14,15 @@ namespace {
 
 struct DecodeWs {
     float *scores;     // [B,T]
-    void *topk_ws;
+    uint32_t *hist;    // [B][kHistBins]: the scores counted by their top 12 key bits
     void *attn_ws;
     size_t total;
 };
 
-DecodeWs carve(void *base, int B, int, int, int64_t T, int index_topk, int Hq, int dc, int dr,
+// kHistBins bin counts per row
+size_t hist_bytes(int B) { return (size_t)B * kHistBins * sizeof(uint32_t); }
+
+DecodeWs carve(void *base, int B, int H, int D, int64_t T, int index_topk, int Hq, int dc, int dr,
                dsa_dtype dt) {
     DecodeWs w{};
     size_t off = 0;
@@ -30,7 +33,8 @@ DecodeWs carve(void *base, int B, int, int, int64_t T, int index_topk, int Hq, i
         return r;
     };
     w.scores = reinterpret_cast<float *>(take((size_t)B * T * sizeof(float)));
-    w.topk_ws = take(topk_workspace_bytes(B, 1, T, index_topk));
+    // the histograms: the part that starts each step at zero
+    w.hist = reinterpret_cast<uint32_t *>(take(hist_bytes(B)));
     const int K = (int64_t)index_topk < T ? index_topk : (int)T;
     w.attn_ws = take(dt == DSA_FP8_LATENT ? sparse_mla_fp8_workspace_bytes(B, 1, Hq, dc, dr, K)
                                           : sparse_mla_workspace_bytes(B, 1, Hq, dc, dr, K, dt));
@@ -74,15 +78,17 @@ extern "C" dsa_status dsa_decode_step(const float *q_idx, const float *w, const 
         return DSA_ERR_WORKSPACE;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     dsa_status st;
+    // the histograms start at zero
+    if (cudaMemsetAsync(ws.hist, 0, dsa::hist_bytes(B), s) != cudaSuccess) return DSA_ERR_CUDA;
     if ((st = dsa::launch_decode_scores(q_idx, w, k_new, k_cache, k_scale, t_max, B, H, D, T,
-                                        softmax_scale, ws.scores, s)) != DSA_OK)
+                                        softmax_scale, ws.scores, s, ws.hist)) != DSA_OK)
         return st;
     // the top-k asks L2 for the latent rows it selects, ahead of the attention's gather
     const int row_bytes = dt == DSA_FP8_LATENT ? (int)dsa_latent_row_bytes(dc, dr)
                                                : (dc + dr) * (dt == DSA_BF16 ? 2 : 4);
-    if ((st = dsa::launch_topk_select(ws.scores, B, 1, T, T - 1, index_topk, idx, ws.topk_ws, s,
-                                      row_bytes % 16 == 0 ? kv_cache : nullptr, t_max,
-                                      row_bytes)) != DSA_OK)
+    if ((st = dsa::launch_topk_select(ws.scores, B, 1, T, T - 1, index_topk, idx, nullptr, s,
+                                      row_bytes % 16 == 0 ? kv_cache : nullptr, t_max, row_bytes,
+                                      ws.hist)) != DSA_OK)
         return st;
     const int K = (int64_t)index_topk < T ? index_topk : (int)T;
     if (dt == DSA_FP8_LATENT)

@@ -52,6 +52,8 @@ struct ScoreArgs {
     const float *w;
     const float *k_scale;
     float *scores;
+    uint32_t *row_hist;        // decode: per row, the histogram of the scores' 12-bit key
+                               //   bins (zeroed before the launch), or null
     int64_t t_max;
     int64_t start_pos;
     int64_t T;
@@ -61,10 +63,17 @@ struct ScoreArgs {
     int *err;
 };
 
-template <int D>
+// Key-tile ring depth: the decode scorer gives one stage's shared memory to
+// the histogram of its scores (two CTAs must still fit on an SM).
+template <bool kRaw> constexpr int ring_stages() { return kRaw ? kStages - 1 : kStages; }
+constexpr int kHistBits = 12;                      // top key bits the histogram resolves
+static_assert(kHistBins == 1 << kHistBits, "histogram bins");
+
+template <int D, bool kRaw>
 __host__ __device__ constexpr size_t score_smem_bytes(int NH) {
-    return 1024 + (size_t)kStages * kTile * D + (size_t)NH * D + kMaxHeads * sizeof(float) +
-           (2 * kStages + 2 * kAcc + 2) * sizeof(uint64_t) + 16;
+    return 1024 + (size_t)ring_stages<kRaw>() * kTile * D + (size_t)NH * D +
+           kMaxHeads * sizeof(float) + (2 * ring_stages<kRaw>() + 2 * kAcc + 2) * sizeof(uint64_t) +
+           16 + (kRaw ? kHistBins * sizeof(uint32_t) : 0);
 }
 
 // Query operand (K-major, swizzled, padded heads zero) and folded weights
@@ -157,20 +166,23 @@ __device__ __forceinline__ void append_key(const ScoreArgs &a, int64_t b, float 
 template <int D, bool kRaw>
 __global__ void __launch_bounds__(kThreads, 2)
 score_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const ScoreArgs a) {
+    constexpr int NS = ring_stages<kRaw>();
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t *sk = smem;
-    uint8_t *sq = sk + kStages * kTile * D;
+    uint8_t *sq = sk + NS * kTile * D;
     float *wf = reinterpret_cast<float *>(sq + a.NH * D);
     uint64_t *full = reinterpret_cast<uint64_t *>(wf + kMaxHeads);
-    uint64_t *empty = full + kStages;
-    uint64_t *accf = empty + kStages;
+    uint64_t *empty = full + NS;
+    uint64_t *accf = empty + NS;
     uint64_t *acce = accf + kAcc;
     uint64_t *q_ready = acce + kAcc, *k_ready = q_ready + 1;
     uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(k_ready + 1);
     volatile int *abort = reinterpret_cast<volatile int *>(tmem_holder + 1);
     float *knew_scale = reinterpret_cast<float *>(tmem_holder + 2);
+    // decode: histogram of this CTA's scores by the top 12 bits of their key
+    uint32_t *s_hist = reinterpret_cast<uint32_t *>(tmem_holder + 4);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     // causal rows are taken longest first (query s = S-1 of every sequence,
@@ -223,7 +235,7 @@ score_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const ScoreArgs a) {
     }
 
     if (threadIdx.x == 0) {
-        for (int i = 0; i < kStages; i++) {
+        for (int i = 0; i < NS; i++) {
             tc::mbar_init(&full[i], 1);
             tc::mbar_init(&empty[i], 1);
         }
@@ -251,8 +263,8 @@ score_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const ScoreArgs a) {
             const uint64_t pol = tc::l2_evict_first_policy();
             int issued = 0;
             for (int i = 0; i < n_my; i++) {
-                const int st = i % kStages;
-                const uint32_t ph = (uint32_t)(i / kStages) & 1u;
+                const int st = i % NS;
+                const uint32_t ph = (uint32_t)(i / NS) & 1u;
                 if (!tc::mbar_wait(&empty[st], ph ^ 1u, a.err, abort)) break;
                 if (append && i == n_my - 1 && !tc::mbar_wait(k_ready, 0, a.err, abort)) break;
                 tc::mbar_arrive_expect_tx(&full[st], kTile * D);
@@ -261,8 +273,8 @@ score_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const ScoreArgs a) {
                 issued = i + 1;
             }
             // wait (bounded) for the last loads still landing in shared memory
-            for (int j = issued > kStages ? issued - kStages : 0; j < issued; j++)
-                tc::mbar_wait(&full[j % kStages], (uint32_t)(j / kStages) & 1u, a.err, abort);
+            for (int j = issued > NS ? issued - NS : 0; j < issued; j++)
+                tc::mbar_wait(&full[j % NS], (uint32_t)(j / NS) & 1u, a.err, abort);
         }
     } else if (warp == 1) {
         if (lane == 0) {
@@ -270,8 +282,8 @@ score_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const ScoreArgs a) {
             const uint32_t sk_addr = tc::smem_u32(sk), sq_addr = tc::smem_u32(sq);
             const bool q_ok = tc::mbar_wait(q_ready, 0, a.err, abort);
             for (int i = 0; q_ok && i < n_my; i++) {
-                const int st = i % kStages, ac = i % kAcc;
-                if (!tc::mbar_wait(&full[st], (uint32_t)(i / kStages) & 1u, a.err, abort)) break;
+                const int st = i % NS, ac = i % kAcc;
+                if (!tc::mbar_wait(&full[st], (uint32_t)(i / NS) & 1u, a.err, abort)) break;
                 if (!tc::mbar_wait(&acce[ac], ((uint32_t)(i / kAcc) & 1u) ^ 1u, a.err, abort))
                     break;
                 tc::tc_fence_after();
@@ -306,6 +318,11 @@ score_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const ScoreArgs a) {
         }
         const uint32_t lane_addr = (uint32_t)((warp & 3) * 32) << 16;
         float *out = a.scores + row * a.T;
+        const bool hist = kRaw && a.row_hist != nullptr;
+        if (hist) {
+            for (int i = threadIdx.x - 64; i < kHistBins; i += 128) s_hist[i] = 0;
+            asm volatile("bar.sync 2, 128;" ::: "memory");
+        }
         for (int i = 0; i < n_my; i++) {
             const int ac = i % kAcc;
             const int64_t t = (tile_lo + i) * kTile + tok;
@@ -341,7 +358,20 @@ score_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const ScoreArgs a) {
             const float acc = (acc4[0] + acc4[1]) + (acc4[2] + acc4[3]);
             tc::tc_fence_before();
             tc::mbar_arrive(&acce[ac]);
-            if (t < n_vis) out[t] = ks * acc;
+            if (t < n_vis) {
+                const float sc = ks * acc;
+                out[t] = sc;
+                if (hist) atomicAdd(&s_hist[score_key(sc) >> (32 - kHistBits)], 1u);
+            }
+        }
+        if (hist) {
+            // this CTA's nonzero bins into the row's histogram
+            asm volatile("bar.sync 2, 128;" ::: "memory");
+            uint32_t *rh = a.row_hist + row * kHistBins;
+            for (int i = threadIdx.x - 64; i < kHistBins; i += 128) {
+                const uint32_t c = s_hist[i];
+                if (c) atomicAdd(rh + i, c);
+            }
         }
     }
 
@@ -357,6 +387,19 @@ uint32_t pow2_cols(int n) {
     uint32_t c = 32;
     while (c < (uint32_t)n) c <<= 1;
     return c;
+}
+
+// CTAs per query row: enough to fill the SMs once (two per SM when their
+// shared memory and TMEM allow), at most one per 128-token tile.
+template <int D, bool kRaw>
+int score_chunks(int64_t rows, int NH, int64_t vis_max) {
+    const size_t smem = score_smem_bytes<D, kRaw>(NH);
+    const int per_sm = smem * 2 <= 227 * 1024 && pow2_cols(kAcc * NH) <= 256 ? 2 : 1;
+    const int64_t max_tiles = (vis_max + kTile - 1) / kTile;
+    int64_t chunks = (int64_t)num_sms() * per_sm / rows;
+    if (chunks > max_tiles) chunks = max_tiles;
+    if (chunks < 1) chunks = 1;
+    return (int)chunks;
 }
 
 template <int D, bool kRaw>
@@ -379,15 +422,11 @@ dsa_status launch_tc(ScoreArgs a, const uint8_t *k_cache, int B, int S, int64_t 
     a.head_scale = (float)(1.0 / sqrt((double)a.H));
     a.err = device_error_word();
 
-    const size_t smem = score_smem_bytes<D>(a.NH);
-    const int per_sm = smem * 2 <= 227 * 1024 && a.tmem_cols <= 256 ? 2 : 1;
+    const size_t smem = score_smem_bytes<D, kRaw>(a.NH);
     const int64_t rows = (int64_t)B * S;
     const int64_t vis_max = T < start_pos + S ? T : start_pos + S;
-    const int64_t max_tiles = (vis_max + kTile - 1) / kTile;
-    int64_t chunks = (int64_t)num_sms() * per_sm / rows;
-    if (chunks > max_tiles) chunks = max_tiles;
-    if (chunks < 1) chunks = 1;
-    a.chunks = (int)chunks;
+    a.chunks = score_chunks<D, kRaw>(rows, a.NH, vis_max);
+    const int64_t chunks = a.chunks;
     if (cudaFuncSetAttribute(score_tc_kernel<D, kRaw>,
                              cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
         return DSA_ERR_CUDA;
@@ -421,9 +460,10 @@ dsa_status launch_index_scores(const uint8_t *q_fp8, const float *q_scale, const
 dsa_status launch_decode_scores(const float *q_raw, const float *w, const float *k_new,
                                 uint8_t *k_cache, float *k_scale, int64_t t_max, int B, int H,
                                 int D, int64_t T, float softmax_scale, float *scores,
-                                cudaStream_t stream) {
+                                cudaStream_t stream, uint32_t *row_hist) {
     if ((int64_t)B * T == 0) return DSA_OK;
     ScoreArgs a = {};
+    a.row_hist = row_hist;
     a.q_raw = q_raw;
     a.k_new = k_new;
     a.k_cache_w = k_cache;

@@ -13,27 +13,35 @@
 // finding tau = the m-th largest value and q = m - #(x > tau), then taking
 // every x > tau plus the first q positions with x == tau.
 //
-// Cluster kernel (rows up to ~300K positions): a thread-block cluster of CN
-// CTAs owns one row; CTA p keeps the scores of positions [p*L, (p+1)*L) in
-// shared memory.  tau is found in rounds whose histograms are merged through
-// distributed shared memory by CTA 0, which broadcasts the decision:
-//   round 0: 2048 bins linear in value between the row's finite min and max
-//            (well spread for smooth score distributions, so shared-memory
-//            atomics rarely collide and the threshold bin is small), merged
-//            into CTA 0 with distributed shared-memory atomics;
-//   then the threshold-bin candidates' keys are gathered into CTA 0, which
-//   finds the exact k-th key alone (by ranking every key directly when there
-//   are at most 1024 of them, else 11 + 11 + 10-bit radix passes); if there
-//   are too many candidates, the radix passes run cluster-wide instead.
-// Then every CTA counts its x > tau and x == tau, the counts are exchanged,
-// and each CTA writes its selected positions at its offset in position order.
-// Cluster barriers are hardware barriers between co-scheduled CTAs.
+// Scores are compared through an order-preserving 32-bit key (score_key).
+// Cluster kernel (rows up to ~460K positions): a thread-block cluster of CN
+// CTAs owns one row; CTA p keeps the keys of positions [p L, (p+1) L) in
+// shared memory.  tau is found by radix rounds on the key bits, each a
+// histogram of the keys still in play, merged into CTA 0 with distributed
+// shared-memory atomics and read back by every CTA, which all find the same
+// threshold bin (no broadcast step):
+//   round 0: the top 12 key bits of every key (sign, exponent, 3 mantissa
+//            bits: bins an eighth of an octave wide);
+//   when the keys in the threshold bin are few enough (kCap), they are
+//   gathered with their positions into CTA 0, and every CTA reads them back
+//   and finds tau among them by radix passes in its own shared memory;
+//   otherwise further 12-bit rounds narrow the prefix first.
+// The counts each CTA needs for its output offset (keys above tau, and the
+// tau-equal keys of lower CTAs) come from the counts every CTA published and
+// from the gathered keys' positions, so that the positions are written in
+// ascending order with three cluster barriers on the common path.
+//
+// Decode kernel (one query per sequence, the scorer's per-row histogram of
+// the top 12 key bits at hand): the same cluster layout, but every CTA finds
+// the threshold bin from that histogram itself, so round 0 and its merge
+// disappear and the scores are read once.
 //
 // Fallback kernel (longer rows): one CTA per row, four 8-bit radix passes
 // over the row in global memory, then the same ordered compaction.
 #include <cooperative_groups.h>
 
 #include "common.cuh"
+#include "tc_ptx.cuh"
 
 namespace cg = cooperative_groups;
 
@@ -42,8 +50,11 @@ namespace {
 
 constexpr int kThreads = 1024;
 constexpr int kWarps = kThreads / 32;
-constexpr int kBins = 2048;
-constexpr int kMaxSlice = 28672;     // scores per CTA kept in shared memory
+constexpr int kBits = 12;                 // key bits a cluster round resolves
+constexpr int kBins = 1 << kBits;         // 4096
+constexpr int kCap = 8192;                // keys CTA 0 gathers for the exact selection
+constexpr int kMaxSlice = 28672;          // keys per CTA kept in shared memory
+constexpr int kMaxCluster = 16;
 
 // Block-wide exclusive scan of a 0/1 flag; *total receives the block total.
 // All threads must call it.
@@ -71,138 +82,82 @@ __device__ __forceinline__ int block_scan_flag(bool flag, int *warp_tot, int *to
     return r;
 }
 
-// Block-wide exclusive scan of an int; *total receives the block total.
-__device__ __forceinline__ int block_scan_int(int v, int *tmp, int *total) {
+// Block-wide exclusive scan of two ints at once; totals in *ta, *tb.
+__device__ __forceinline__ void block_scan2(int a, int b, int *ea, int *eb, int2 *tmp, int *ta,
+                                            int *tb) {
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    int incl = v;
+    int ia = a, ib = b;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
-        const int n = __shfl_up_sync(0xffffffffu, incl, o);
-        if (lane >= o) incl += n;
+        const int na = __shfl_up_sync(0xffffffffu, ia, o);
+        const int nb = __shfl_up_sync(0xffffffffu, ib, o);
+        if (lane >= o) {
+            ia += na;
+            ib += nb;
+        }
     }
-    if (lane == 31) tmp[warp] = incl;
+    if (lane == 31) tmp[warp] = make_int2(ia, ib);
     __syncthreads();
     if (warp == 0) {
-        const int wv = lane < kWarps ? tmp[lane] : 0;
-        int wi = wv;
+        const int2 v = tmp[lane];
+        int wa = v.x, wb = v.y;
 #pragma unroll
         for (int o = 1; o < 32; o <<= 1) {
-            const int n = __shfl_up_sync(0xffffffffu, wi, o);
-            if (lane >= o) wi += n;
-        }
-        if (lane < kWarps) tmp[lane] = wi - wv;
-        if (lane == 31) tmp[32] = wi;
-    }
-    __syncthreads();
-    const int r = tmp[warp] + incl - v;
-    *total = tmp[32];
-    __syncthreads();
-    return r;
-}
-
-// Block-wide sum of an int (result in every thread).
-__device__ __forceinline__ int block_sum(int v, int *tmp) {
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-    if ((threadIdx.x & 31) == 0) tmp[threadIdx.x >> 5] = v;
-    __syncthreads();
-    int r = 0;
-    for (int w = 0; w < kWarps; w++) r += tmp[w];
-    __syncthreads();
-    return r;
-}
-
-// Finds, in a histogram of `nb` bins counted from the top, the bin where the
-// running count reaches `rank` (1-based); returns the bin and the rank left
-// inside it.  Executed by the whole block; `hist` is in shared memory.
-__device__ __forceinline__ void find_rank_bin(const unsigned *hist, int nb, unsigned rank,
-                                              unsigned *out_bin, unsigned *out_rank,
-                                              unsigned *scan_tmp) {
-    // inclusive suffix sums over bins, in chunks of kThreads bins from the top
-    unsigned above = 0;
-    for (int base = nb - 1; base >= 0; base -= kThreads) {
-        const int bin = base - (int)threadIdx.x;
-        unsigned v = bin >= 0 ? hist[bin] : 0u;
-        // inclusive scan in thread order (= descending bins)
-        unsigned incl = v;
-        const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-            unsigned n = __shfl_up_sync(0xffffffffu, incl, o);
-            if (lane >= o) incl += n;
-        }
-        if (lane == 31) scan_tmp[warp] = incl;
-        __syncthreads();
-        if (warp == 0) {
-            unsigned wv = scan_tmp[lane];
-            unsigned wi = wv;
-#pragma unroll
-            for (int o = 1; o < 32; o <<= 1) {
-                unsigned n = __shfl_up_sync(0xffffffffu, wi, o);
-                if (lane >= o) wi += n;
+            const int na = __shfl_up_sync(0xffffffffu, wa, o);
+            const int nb = __shfl_up_sync(0xffffffffu, wb, o);
+            if (lane >= o) {
+                wa += na;
+                wb += nb;
             }
-            scan_tmp[lane] = wi - wv;       // exclusive prefix of warp totals
-            if (lane == 31) scan_tmp[32] = wi;
         }
-        __syncthreads();
-        const unsigned before = above + scan_tmp[warp] + incl - v;   // count strictly above bin
-        if (bin >= 0 && before < rank && before + v >= rank) {
-            *out_bin = (unsigned)bin;
-            *out_rank = rank - before;
-        }
-        above += scan_tmp[32];
-        __syncthreads();
-        if (above >= rank) break;
+        tmp[lane] = make_int2(wa - v.x, wb - v.y);
+        if (lane == 31) tmp[32] = make_int2(wa, wb);
     }
+    __syncthreads();
+    *ea = tmp[warp].x + ia - a;
+    *eb = tmp[warp].y + ib - b;
+    *ta = tmp[32].x;
+    *tb = tmp[32].y;
     __syncthreads();
 }
 
-__device__ __forceinline__ int linear_bin(float x, float lo, float scale) {
-    if (!(x >= lo)) return 0;                       // NaN, -inf
-    const float t = __fmul_rn(__fsub_rn(x, lo), scale);
-    return t >= (float)(kBins - 1) ? kBins - 1 : (int)t;
+// In a histogram of nb = 4 * kThreads or fewer bins (bin index = key digit,
+// larger is better), finds the bin holding the rank-th largest key (1-based)
+// and the count of keys in the bins above it.  Thread t owns the 4 bins
+// nb - 4t - 4 .. nb - 4t - 1 (descending); get(i) reads bin i.  Every thread
+// of the block calls it and gets the same answer.
+template <typename Get>
+__device__ __forceinline__ void find_rank(Get get, int nb, unsigned rank, unsigned *bin_out,
+                                          unsigned *above_out, unsigned *cnt_out, int2 *tmp) {
+    const int t = threadIdx.x;
+    const int b0 = nb - 4 * t - 1;                 // this thread's highest bin
+    unsigned c[4];
+#pragma unroll
+    for (int j = 0; j < 4; j++) c[j] = b0 - j >= 0 ? get(b0 - j) : 0u;
+    const int mine = (int)(c[0] + c[1] + c[2] + c[3]);
+    int before, unused, total, unused2;
+    block_scan2(mine, 0, &before, &unused, tmp, &total, &unused2);
+    unsigned above = (unsigned)before;
+    __shared__ unsigned s_out[3];
+#pragma unroll
+    for (int j = 0; j < 4; j++) {
+        if (b0 - j >= 0 && above < rank && above + c[j] >= rank) {
+            s_out[0] = (unsigned)(b0 - j);
+            s_out[1] = above;
+            s_out[2] = c[j];
+        }
+        above += c[j];
+    }
+    __syncthreads();
+    *bin_out = s_out[0];
+    *above_out = s_out[1];
+    *cnt_out = s_out[2];
+    __syncthreads();
 }
-
-struct ClusterCtl {
-    float lo, hi;           // this CTA's finite min / max
-    unsigned bin, rank;     // broadcast by CTA 0
-    int n_cand;             // this CTA's threshold-bin candidates
-    int n_gt, n_eq;         // this CTA's counts of x > tau, x == tau
-};
 
 // Slice element i lives at sv[pad(i)]: one spare word every 32 keeps the
 // per-thread contiguous segments (stride seg words) off a single bank.
 __device__ __forceinline__ int pad(int i) { return i + (i >> 5); }
-
-// Exact rank search among n keys held in shared memory by one CTA: the
-// rank-th largest key (11 + 11 + 10-bit radix passes) and the rank left
-// among the keys equal to it.
-__device__ void cta_select_keys(const uint32_t *keys, int n, unsigned rank, unsigned *hist,
-                                unsigned *scan_tmp, unsigned *s_bin, unsigned *s_rank,
-                                uint32_t *tau_out, unsigned *rank_out) {
-    uint32_t prefix = 0, mask = 0;
-    const int shifts[3] = {21, 10, 0};
-    const int widths[3] = {11, 11, 10};
-    for (int rd = 0; rd < 3; rd++) {
-        const uint32_t dm = (1u << widths[rd]) - 1u;
-        for (int i = threadIdx.x; i <= (int)dm; i += kThreads) hist[i] = 0;
-        __syncthreads();
-        for (int j = threadIdx.x; j < n; j += kThreads) {
-            const uint32_t key = keys[j];
-            if ((key & mask) == prefix) atomicAdd(&hist[(key >> shifts[rd]) & dm], 1u);
-        }
-        __syncthreads();
-        find_rank_bin(hist, (int)dm + 1, rank, s_bin, s_rank, scan_tmp);
-        prefix |= *s_bin << shifts[rd];
-        mask |= dm << shifts[rd];
-        rank = *s_rank;
-        __syncthreads();
-    }
-    *tau_out = prefix;
-    *rank_out = rank;
-}
-
-constexpr int kGather = 8192;      // candidates CTA 0 can select alone
 
 // Rows of a cache the next kernel gathers at the selected positions: the
 // top-k asks L2 for each selected row as it writes the position (a no-op
@@ -219,9 +174,41 @@ struct RowPrefetch {
     }
 };
 
+// Shared by the CTAs of a cluster through distributed shared memory.  Other
+// CTAs only write into CTA 0 (atomics, appends, counts) and CTA 0 only writes
+// small results back; nobody reads another CTA's shared memory in bulk.
+struct TopkShared {
+    unsigned hist[kBins];           // this CTA's histogram; CTA 0's is the cluster's sum
+    unsigned res[4];                // from CTA 0: prefix, prefix bits, rank in group, group size
+    unsigned out[3];                // from CTA 0: tau, this CTA's output offset, its tau-equal quota
+    int n_cand;                     // CTA 0: keys gathered
+    int cnt_gt[kMaxCluster];        // CTA 0: per CTA, keys above the prefix group
+    int cnt_in[kMaxCluster];        // CTA 0: per CTA, keys inside it
+    int sel_gt[kMaxCluster];        // CTA 0: per CTA, gathered keys above tau
+    int sel_eq[kMaxCluster];        // CTA 0: per CTA, gathered keys equal to tau
+};
+
+// The prefix group's threshold bin in CTA 0's merged histogram, found by CTA
+// 0 and written into every CTA's res (call with the whole cluster; a cluster
+// barrier must follow before res is read).
+__device__ __forceinline__ void cta0_find_and_send(cg::cluster_group &cl, TopkShared &sh, int nb,
+                                                   uint32_t prefix, int pbits, unsigned rank,
+                                                   int2 *tmp) {
+    if (cl.block_rank() != 0) return;
+    unsigned bin, above, cnt;
+    find_rank([&](int i) { return sh.hist[i]; }, 1 << nb, rank, &bin, &above, &cnt, tmp);
+    if (threadIdx.x < cl.num_blocks()) {
+        TopkShared *r = cl.map_shared_rank(&sh, (int)threadIdx.x);
+        r->res[0] = (prefix << nb) | bin;
+        r->res[1] = (unsigned)(pbits + nb);
+        r->res[2] = rank - above;
+        r->res[3] = cnt;
+    }
+}
+
 __global__ void __launch_bounds__(kThreads, 1)
-topk_cluster_kernel(const float *scores, int S, int64_t T, int64_t start_pos, int K,
-                    int L, int store_bins, int32_t *__restrict__ idx, const RowPrefetch pf) {
+topk_cluster_kernel(const float *scores, int S, int64_t T, int64_t start_pos, int K, int L,
+                    int32_t *__restrict__ idx, const RowPrefetch pf) {
     // a kernel launched after this one (the sparse attention) may start its
     // set-up now; it reads the selections only after waiting for this grid
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
@@ -248,21 +235,13 @@ topk_cluster_kernel(const float *scores, int S, int64_t T, int64_t start_pos, in
         return;                           // uniform across the cluster
     }
 
-    extern __shared__ float sv[];                                   // [pad(L)] scores
-    uint32_t *gath = reinterpret_cast<uint32_t *>(sv + pad(L) + 1);  // [kGather] keys (CTA 0)
-    uint16_t *cand = reinterpret_cast<uint16_t *>(gath + kGather);  // [L] candidate slots
-    // each value's linear bin, [slot within the thread's segment][thread], when
-    // shared memory holds it (else recomputed from the score)
-    uint16_t *bins = store_bins ? cand + L : nullptr;
-    __shared__ unsigned hist[kBins];          // local histogram
-    __shared__ unsigned hmerged[kBins];       // cluster histogram (CTA 0)
-    __shared__ unsigned scan_tmp[33];
-    __shared__ int itmp[33];
-    __shared__ ClusterCtl ctl;
-    __shared__ unsigned s_bin, s_rank;
-    __shared__ uint32_t s_tau;
-    __shared__ int s_ncand;
-    __shared__ float s_lo, s_hi;
+    extern __shared__ uint32_t dyn[];
+    uint32_t *keys = dyn;                                           // [pad(L) + 1]
+    uint32_t *ck = keys + pad(L) + 1;                               // CTA 0: [kCap] gathered keys
+    int32_t *cp = reinterpret_cast<int32_t *>(ck + kCap);           // CTA 0: [kCap] their positions
+    __shared__ TopkShared sh;
+    __shared__ int2 scan_tmp[33];
+    TopkShared *sh0 = cl.map_shared_rank(&sh, 0);
 
     const int64_t t0 = (int64_t)p * L;
     int64_t t1 = t0 + L;
@@ -270,275 +249,222 @@ topk_cluster_kernel(const float *scores, int S, int64_t T, int64_t start_pos, in
     const int len = t1 > t0 ? (int)(t1 - t0) : 0;
     const float *src = scores + row * T + t0;
 
-    // load the slice, finite min / max; clear the histograms
-    // (loads are issued in batches of eight per thread so their latencies overlap)
-    float lo = INFINITY, hi = -INFINITY;
-    const bool vec = ((reinterpret_cast<uintptr_t>(src) & 15) == 0);
-    if (vec) {
+    // clear, then let the other CTAs know (the barrier's wait comes after the
+    // slice is loaded, so its latency is hidden)
+    for (int i = threadIdx.x; i < kBins; i += kThreads) sh.hist[i] = 0;
+    if (threadIdx.x < kMaxCluster) {
+        sh.sel_gt[threadIdx.x] = 0;
+        sh.sel_eq[threadIdx.x] = 0;
+    }
+    if (threadIdx.x == 0) sh.n_cand = 0;
+    __syncthreads();
+    asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
+
+    // keys of the slice and the histogram of their top 12 bits
+    auto put = [&](int i, float x) {
+        const uint32_t key = score_key(x);
+        keys[pad(i)] = key;
+        atomicAdd(&sh.hist[key >> (32 - kBits)], 1u);
+    };
+    if ((reinterpret_cast<uintptr_t>(src) & 15) == 0) {
         const int n4 = len >> 2;
-        for (int base = 0; base < n4; base += 8 * kThreads) {
-            float4 v[8];
+        for (int base = 0; base < n4; base += 4 * kThreads) {
+            float4 v[4];
 #pragma unroll
-            for (int u = 0; u < 8; u++) {
+            for (int u = 0; u < 4; u++) {
                 const int j = base + u * kThreads + threadIdx.x;
-                v[u] = j < n4 ? reinterpret_cast<const float4 *>(src)[j]
-                              : make_float4(NAN, NAN, NAN, NAN);
+                v[u] = j < n4 ? reinterpret_cast<const float4 *>(src)[j] : make_float4(0.f, 0.f, 0.f, 0.f);
             }
 #pragma unroll
-            for (int u = 0; u < 8; u++) {
+            for (int u = 0; u < 4; u++) {
                 const int j = base + u * kThreads + threadIdx.x;
                 if (j >= n4) continue;
-                const float xs[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
-#pragma unroll
-                for (int e = 0; e < 4; e++) {
-                    sv[pad(4 * j + e)] = xs[e];
-                    if (isfinite(xs[e])) {
-                        lo = fminf(lo, xs[e]);
-                        hi = fmaxf(hi, xs[e]);
-                    }
+                put(4 * j, v[u].x);
+                put(4 * j + 1, v[u].y);
+                put(4 * j + 2, v[u].z);
+                put(4 * j + 3, v[u].w);
+            }
+        }
+        for (int i = (len & ~3) + threadIdx.x; i < len; i += kThreads) put(i, src[i]);
+    } else {
+        for (int i = threadIdx.x; i < len; i += kThreads) put(i, src[i]);
+    }
+    __syncthreads();
+    asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
+
+    // ---- round 0: the 12-bit bin holding the m-th largest key
+    uint32_t prefix;
+    int pbits;
+    unsigned rank, n_group;
+    {
+        if (p != 0)
+            for (int i = threadIdx.x; i < kBins; i += kThreads) {
+                const unsigned c = sh.hist[i];
+                if (c) atomicAdd(&sh0->hist[i], c);
+            }
+        cl.sync();
+        cta0_find_and_send(cl, sh, kBits, 0u, 0, (unsigned)m, scan_tmp);
+        cl.sync();
+        prefix = sh.res[0];
+        pbits = (int)sh.res[1];
+        rank = sh.res[2];
+        n_group = sh.res[3];
+    }
+    // further 12-bit rounds while the group is too large to gather (rare:
+    // scores within a few percent of each other, or many exact ties)
+    while (n_group > (unsigned)kCap && pbits < 32) {
+        const int nb = 32 - pbits < kBits ? 32 - pbits : kBits;
+        const int sh_lo = 32 - pbits - nb;
+        for (int i = threadIdx.x; i < kBins; i += kThreads) sh.hist[i] = 0;
+        cl.sync();                                  // CTA 0's histogram is clear
+        for (int i = threadIdx.x; i < len; i += kThreads) {
+            const uint32_t key = keys[pad(i)];
+            if ((key >> (32 - pbits)) == prefix)
+                atomicAdd(&sh.hist[(key >> sh_lo) & ((1u << nb) - 1u)], 1u);
+        }
+        __syncthreads();
+        if (p != 0)
+            for (int i = threadIdx.x; i < (1 << nb); i += kThreads) {
+                const unsigned c = sh.hist[i];
+                if (c) atomicAdd(&sh0->hist[i], c);
+            }
+        cl.sync();
+        cta0_find_and_send(cl, sh, nb, prefix, pbits, rank, scan_tmp);
+        cl.sync();
+        prefix = sh.res[0];
+        pbits = (int)sh.res[1];
+        rank = sh.res[2];
+        n_group = sh.res[3];
+    }
+
+    // ---- this CTA's keys above the group and inside it, counted into CTA 0;
+    // the group's keys themselves are gathered there when they are few
+    const bool gather = n_group <= (unsigned)kCap && pbits < 32;
+    const int gshift = 32 - pbits;
+    int n_gt = 0, n_in = 0;
+    uint32_t *rk = cl.map_shared_rank(ck, 0);
+    int32_t *rp = cl.map_shared_rank(cp, 0);
+    for (int i0 = 0; i0 < len; i0 += kThreads) {
+        const int i = i0 + threadIdx.x;
+        uint32_t key = 0;
+        bool in = false;
+        if (i < len) {
+            key = keys[pad(i)];
+            const uint32_t g = gshift == 32 ? 0u : key >> gshift;
+            n_gt += g > prefix;
+            in = g == prefix;
+            n_in += in;
+        }
+        if (gather) {
+            // warp-aggregated append into CTA 0's list
+            const unsigned bal = __ballot_sync(0xffffffffu, in);
+            const int lane = threadIdx.x & 31;
+            int base = 0;
+            if (lane == 0 && bal) base = atomicAdd(&sh0->n_cand, __popc(bal));
+            base = __shfl_sync(0xffffffffu, base, 0);
+            if (in) {
+                const int slot = base + __popc(bal & ((1u << lane) - 1u));
+                if (slot < kCap) {
+                    rk[slot] = key;
+                    rp[slot] = (int32_t)(t0 + i);
                 }
             }
         }
     }
-    for (int base = vec ? (len & ~3) : 0; base < len; base += 8 * kThreads) {
-        float v[8];
-#pragma unroll
-        for (int u = 0; u < 8; u++) {
-            const int i = base + u * kThreads + threadIdx.x;
-            v[u] = i < len ? src[i] : NAN;
-        }
-#pragma unroll
-        for (int u = 0; u < 8; u++) {
-            const int i = base + u * kThreads + threadIdx.x;
-            if (i >= len) continue;
-            sv[pad(i)] = v[u];
-            if (isfinite(v[u])) {
-                lo = fminf(lo, v[u]);
-                hi = fmaxf(hi, v[u]);
-            }
+    {
+        int e_gt, e_in, tot_gt, tot_in;
+        block_scan2(n_gt, n_in, &e_gt, &e_in, scan_tmp, &tot_gt, &tot_in);
+        if (threadIdx.x == 0) {
+            sh0->cnt_gt[p] = tot_gt;
+            sh0->cnt_in[p] = tot_in;
         }
     }
-    for (int i = threadIdx.x; i < kBins; i += kThreads) {
-        hist[i] = 0;
-        hmerged[i] = 0;
-    }
-    lo = -warp_max(-lo);
-    hi = warp_max(hi);
-    if ((threadIdx.x & 31) == 0) {
-        reinterpret_cast<float *>(itmp)[threadIdx.x >> 5] = lo;
-        scan_tmp[threadIdx.x >> 5] = __float_as_uint(hi);
-    }
-    __syncthreads();
-    if (threadIdx.x == 0) {
-        float l = INFINITY, h = -INFINITY;
-        for (int w = 0; w < kWarps; w++) {
-            l = fminf(l, reinterpret_cast<float *>(itmp)[w]);
-            h = fmaxf(h, __uint_as_float(scan_tmp[w]));
-        }
-        ctl.lo = l;
-        ctl.hi = h;
-    }
-    cl.sync();                                                            // (1)
-    if (threadIdx.x == 0) {
-        float l = INFINITY, h = -INFINITY;
-        for (int r = 0; r < CN; r++) {
-            const ClusterCtl *rc = cl.map_shared_rank(&ctl, r);
-            l = fminf(l, rc->lo);
-            h = fmaxf(h, rc->hi);
-        }
-        s_lo = l;
-        s_hi = h;
-    }
-    __syncthreads();
-    const float g_lo = s_lo, g_hi = s_hi;
-    const float scale = (g_hi > g_lo && isfinite(g_hi - g_lo)) ? __fdiv_rn((float)kBins, g_hi - g_lo)
-                                                                  : 0.f;
+    cl.sync();                                                      // counts and keys in CTA 0
 
-    // round 0: linear bins, merged into CTA 0 with distributed shared-memory atomics
-    // thread i owns the contiguous segment [i*seg, (i+1)*seg) of the slice
+    // ---- CTA 0: tau (the rank-th largest key of the group), q (tau-equal keys
+    // taken), and every CTA's output offset and tau-equal quota
+    if (p == 0) {
+        uint32_t tau;
+        int q;
+        if (gather) {
+            // radix passes on the gathered keys' remaining bits (at most 11 at a time)
+            const int E = (int)n_group;
+            uint32_t tp = prefix;
+            int tbits = pbits;
+            unsigned rk_left = rank;
+            while (tbits < 32) {
+                const int nb = 32 - tbits < 11 ? 32 - tbits : 11;
+                const int sh_lo = 32 - tbits - nb;
+                for (int i = threadIdx.x; i < (1 << nb); i += kThreads) sh.hist[i] = 0;
+                __syncthreads();
+                for (int j = threadIdx.x; j < E; j += kThreads) {
+                    const uint32_t key = ck[j];
+                    if ((key >> (32 - tbits)) == tp) atomicAdd(&sh.hist[(key >> sh_lo) & ((1u << nb) - 1u)], 1u);
+                }
+                __syncthreads();
+                unsigned bin, above, cnt;
+                find_rank([&](int i) { return sh.hist[i]; }, 1 << nb, rk_left, &bin, &above, &cnt, scan_tmp);
+                tp = (tp << nb) | bin;
+                tbits += nb;
+                rk_left -= above;
+            }
+            tau = tp;
+            q = (int)rk_left;
+            // per CTA: gathered keys above tau and equal to tau
+            for (int j = threadIdx.x; j < E; j += kThreads) {
+                const uint32_t key = ck[j];
+                const int c = (int)(cp[j] / L);
+                if (key > tau) atomicAdd(&sh.sel_gt[c], 1);
+                else if (key == tau) atomicAdd(&sh.sel_eq[c], 1);
+            }
+            __syncthreads();
+        } else {
+            // the group is one key value: its keys are all tau-equal
+            tau = prefix;
+            q = (int)rank;
+        }
+        if (threadIdx.x < CN) {
+            const int t = (int)threadIdx.x;
+            int gt = 0, eq = 0;
+            for (int r = 0; r < t; r++) {
+                gt += sh.cnt_gt[r] + (gather ? sh.sel_gt[r] : 0);
+                eq += gather ? sh.sel_eq[r] : sh.cnt_in[r];
+            }
+            const int mine = gather ? sh.sel_eq[t] : sh.cnt_in[t];
+            int my_q = q - eq;
+            my_q = my_q < 0 ? 0 : (my_q > mine ? mine : my_q);
+            TopkShared *r = cl.map_shared_rank(&sh, t);
+            r->out[0] = tau;
+            r->out[1] = (unsigned)(gt + (q < eq ? q : eq));
+            r->out[2] = (unsigned)my_q;
+        }
+    }
+    cl.sync();                            // results delivered; no CTA touches another's memory after this
+    const uint32_t tau = sh.out[0];
+    const int off = (int)sh.out[1], my_q = (int)sh.out[2];
+
+    // ---- ordered write: thread i owns the contiguous segment [i seg, (i+1) seg)
     const int seg = (len + kThreads - 1) / kThreads;
     const int s0 = threadIdx.x * seg < len ? threadIdx.x * seg : len;
     const int s1 = s0 + seg < len ? s0 + seg : len;
+    int c_gt = 0, c_eq = 0;
     for (int i = s0; i < s1; i++) {
-        const int bin = linear_bin(sv[pad(i)], g_lo, scale);
-        if (bins) bins[(i - s0) * kThreads + threadIdx.x] = (uint16_t)bin;
-        atomicAdd(&hist[bin], 1u);
+        const uint32_t key = keys[pad(i)];
+        c_gt += key > tau;
+        c_eq += key == tau;
     }
-    auto bin_of = [&](int i) -> int {
-        return bins ? (int)bins[(i - s0) * kThreads + threadIdx.x] : linear_bin(sv[pad(i)], g_lo, scale);
-    };
-    __syncthreads();
-    {
-        unsigned *h0 = cl.map_shared_rank(hmerged, 0);
-        for (int b = threadIdx.x; b < kBins; b += kThreads)
-            if (hist[b]) atomicAdd(h0 + b, hist[b]);
-    }
-    cl.sync();                                                            // (2)
-    if (p == 0) {
-        find_rank_bin(hmerged, kBins, (unsigned)m, &s_bin, &s_rank, scan_tmp);
-        if (threadIdx.x < CN) {
-            ClusterCtl *rc = cl.map_shared_rank(&ctl, (int)threadIdx.x);
-            rc->bin = s_bin;
-            rc->rank = s_rank;
-        }
-    }
-    cl.sync();                                                            // (3)
-    const int tb = (int)ctl.bin;
-    unsigned rank = ctl.rank;
-
-    // threshold-bin candidates (slot indices, in any order: only their keys
-    // matter), appended in one pass
-    if (threadIdx.x == 0) s_ncand = 0;
-    __syncthreads();
-    int above = 0;                        // this thread's values in bins above the threshold bin
+    int e_gt, e_eq, tot_gt, tot_eq;
+    block_scan2(c_gt, c_eq, &e_gt, &e_eq, scan_tmp, &tot_gt, &tot_eq);
+    // tau-equal keys this thread takes: the CTA's quota goes to the lowest positions
+    int take_eq = my_q - e_eq;
+    take_eq = take_eq < 0 ? 0 : (take_eq > c_eq ? c_eq : take_eq);
+    int pos = off + e_gt + (my_q < e_eq ? my_q : e_eq);
     for (int i = s0; i < s1; i++) {
-        const int bin = bin_of(i);
-        above += bin > tb;
-        if (bin == tb) cand[atomicAdd(&s_ncand, 1)] = (uint16_t)i;
-    }
-    __syncthreads();
-    const int n_cand = s_ncand;
-    if (threadIdx.x == 0) ctl.n_cand = n_cand;
-    cl.sync();                                                            // (4)
-    int cand_off = 0, E = 0;
-    for (int r = 0; r < CN; r++) {
-        const int c = cl.map_shared_rank(&ctl, r)->n_cand;
-        if (r < p) cand_off += c;
-        E += c;
-    }
-
-    uint32_t tau;
-    int q;
-    if (E <= kGather) {
-        // few candidates: CTA 0 selects among all of them alone
-        uint32_t *g0 = cl.map_shared_rank(gath, 0);
-        for (int j = threadIdx.x; j < n_cand; j += kThreads) g0[cand_off + j] = score_key(sv[pad(cand[j])]);
-        cl.sync();                                                        // (5)
-        if (p == 0) {
-            unsigned rk;
-            if (E <= kThreads) {
-                // few candidates: rank each key directly (keys larger, keys equal);
-                // the key whose range covers `rank` is tau, and rank - #larger of
-                // the keys equal to it are taken (every tau-equal thread agrees)
-                if ((int)threadIdx.x < E) {
-                    const uint32_t kj = gath[threadIdx.x];
-                    unsigned gt = 0, eq = 0;
-                    for (int i = 0; i < E; i++) {
-                        const uint32_t ki = gath[i];
-                        gt += ki > kj;
-                        eq += ki == kj;
-                    }
-                    if (gt < rank && gt + eq >= rank) {
-                        s_tau = kj;
-                        s_rank = rank - gt;
-                    }
-                }
-                __syncthreads();
-                rk = s_rank;
-            } else {
-                cta_select_keys(gath, E, rank, hist, scan_tmp, &s_bin, &s_rank, &s_tau, &rk);
-            }
-            if (threadIdx.x < CN) {
-                ClusterCtl *rc = cl.map_shared_rank(&ctl, (int)threadIdx.x);
-                rc->bin = s_tau;
-                rc->rank = rk;
-            }
-        }
-        cl.sync();                                                        // (6)
-        tau = ctl.bin;
-        q = (int)ctl.rank;
-    } else {
-        // many candidates: radix rounds over each CTA's own candidates,
-        // histograms merged into CTA 0 with distributed atomics
-        uint32_t prefix = 0, mask = 0;
-        const int shifts[3] = {21, 10, 0};
-        const int widths[3] = {11, 11, 10};
-        for (int rd = 0; rd < 3; rd++) {
-            const int sh = shifts[rd];
-            const uint32_t dm = (1u << widths[rd]) - 1u;
-            for (int i = threadIdx.x; i < kBins; i += kThreads) {
-                hist[i] = 0;
-                hmerged[i] = 0;
-            }
-            cl.sync();
-            for (int j = threadIdx.x; j < n_cand; j += kThreads) {
-                const uint32_t key = score_key(sv[pad(cand[j])]);
-                if ((key & mask) == prefix) atomicAdd(&hist[(key >> sh) & dm], 1u);
-            }
-            __syncthreads();
-            {
-                unsigned *h0 = cl.map_shared_rank(hmerged, 0);
-                for (int b = threadIdx.x; b <= (int)dm; b += kThreads)
-                    if (hist[b]) atomicAdd(h0 + b, hist[b]);
-            }
-            cl.sync();
-            if (p == 0) {
-                find_rank_bin(hmerged, (int)dm + 1, rank, &s_bin, &s_rank, scan_tmp);
-                if (threadIdx.x < CN) {
-                    ClusterCtl *rc = cl.map_shared_rank(&ctl, (int)threadIdx.x);
-                    rc->bin = s_bin;
-                    rc->rank = s_rank;
-                }
-            }
-            cl.sync();
-            prefix |= ctl.bin << sh;
-            mask |= dm << sh;
-            rank = ctl.rank;
-        }
-        tau = prefix;
-        q = (int)rank;
-    }
-
-    // counts, exchanged through the cluster, give each CTA its output offset.
-    // Every value above the threshold bin is > tau; of the candidates, each
-    // adds to its owner thread's count of keys > tau or == tau.
-    unsigned *t_gt = hist, *t_eq = hist + kThreads;        // hist is free again
-    t_gt[threadIdx.x] = 0;
-    t_eq[threadIdx.x] = 0;
-    __syncthreads();
-    for (int j = threadIdx.x; j < n_cand; j += kThreads) {
-        const int slot = cand[j];
-        const uint32_t key = score_key(sv[pad(slot)]);
-        if (key > tau) atomicAdd(&t_gt[slot / seg], 1u);
-        else if (key == tau) atomicAdd(&t_eq[slot / seg], 1u);
-    }
-    __syncthreads();
-    const int gt = above + (int)t_gt[threadIdx.x], eq = (int)t_eq[threadIdx.x];
-    int cta_gt, cta_eq;
-    block_scan_int(gt, itmp, &cta_gt);
-    const int eq_before_me = block_scan_int(eq, itmp, &cta_eq);
-    if (threadIdx.x == 0) {
-        ctl.n_gt = cta_gt;
-        ctl.n_eq = cta_eq;
-    }
-    cl.sync();                                                            // (7)
-    int off = 0, eq_before = 0;
-    for (int r = 0; r < p; r++) {
-        const ClusterCtl *rc = cl.map_shared_rank(&ctl, r);
-        int quota = q - eq_before;
-        quota = quota < 0 ? 0 : (quota > rc->n_eq ? rc->n_eq : quota);
-        off += rc->n_gt + quota;
-        eq_before += rc->n_eq;
-    }
-    cl.sync();                            // (8) no CTA leaves while others read its counts
-    // tau-equal positions this thread takes: the first (q - earlier ones)
-    int my_q = q - eq_before - eq_before_me;
-    my_q = my_q < 0 ? 0 : (my_q > eq ? eq : my_q);
-    int tot;
-    int pos = off + block_scan_int(gt + my_q, itmp, &tot);
-    for (int i = s0; i < s1; i++) {
-        // bins are monotone in the score: above the threshold bin means > tau,
-        // below means < tau; only threshold-bin values need their key
-        const int bin = bin_of(i);
-        if (bin < tb) continue;
-        bool take = bin > tb;
-        if (!take) {
-            const uint32_t key = score_key(sv[pad(i)]);
-            take = key > tau;
-            if (key == tau && my_q > 0) {
-                take = true;
-                my_q--;
-            }
+        const uint32_t key = keys[pad(i)];
+        bool take = key > tau;
+        if (key == tau && take_eq > 0) {
+            take = true;
+            take_eq--;
         }
         if (take && pos < m) {
             dst[pos++] = (int32_t)(t0 + i);
@@ -546,6 +472,407 @@ topk_cluster_kernel(const float *scores, int S, int64_t T, int64_t start_pos, in
         }
     }
     for (int i = m + p * kThreads + threadIdx.x; i < K; i += CN * kThreads) dst[i] = -1;
+}
+
+// ------------------------------------------------------------ decode top-k
+// The decode step's top-k, when the scorer has counted the row's scores by
+// their top 12 key bits: a cluster of CN CTAs of 512 threads per row, each
+// thread holding 32 consecutive positions' keys in registers.  Every CTA reads
+// the row's histogram and finds the same 12-bit threshold bin on its own, so
+// the scores are read once and no histogram is merged.  Each CTA reserves a
+// range of CTA 0's candidate list with one atomic and stores the keys of its
+// span that fall in the bin there, with their positions (distributed shared
+// memory); CTA 0 finds tau among them (a 10-bit histogram pass, then one warp
+// ranks the few keys left, or further passes when they are many) and every
+// CTA's output offset and tau-equal quota, and sends each CTA its numbers.
+// Two cluster barriers on the common path; global memory sees only the
+// scores, the histogram and the output.  When the threshold bin holds more
+// keys than CTA 0 can gather, 12-bit rounds over the register keys, merged
+// into CTA 0, narrow it first.
+constexpr int kDecThreads = 512;
+constexpr int kDecWarps = kDecThreads / 32;
+constexpr int kDecPer = 32;                         // positions per thread
+constexpr int kDecSpan = kDecThreads * kDecPer;     // positions per CTA: 16384
+constexpr int kDecCap = 8192;                       // keys CTA 0 gathers
+constexpr int kDecSub = 1024;                       // bins of a 10-bit pass
+constexpr int kDecFew = 32;                         // keys one warp ranks directly
+
+struct DecShared {
+    unsigned hist[kBins];             // CTA 0: histogram of the current pass or round
+    uint2 cand[kDecCap];              // CTA 0: gathered (key, position), CTA by CTA
+    int n_cand;                       // CTA 0: slots reserved
+    int base[kMaxCluster];            // CTA 0: per CTA, its first slot
+    int cnt_gt[kMaxCluster];          // CTA 0: per CTA, keys above the group
+    int cnt_in[kMaxCluster];          // CTA 0: per CTA, keys inside it
+    int sel_gt[kMaxCluster];          // CTA 0: per CTA, gathered keys above tau
+    int sel_eq[kMaxCluster];          // CTA 0: per CTA, gathered keys equal to tau
+    unsigned res[4];                  // from CTA 0: prefix, prefix bits, rank in group, group size
+    unsigned out[3];                  // from CTA 0: tau, output offset, tau-equal quota
+    int my_base;
+    int n_few;
+    uint32_t few[kDecFew];
+    unsigned s_out[3];
+    int wtmp[kDecWarps];
+    int2 wtmp2[kDecWarps];
+};
+
+// Sum over lanes 0..n-1 of v (n <= 32), in every lane.
+__device__ __forceinline__ int warp_sum_first(int v, int lane, int n) {
+    int x = lane < n ? v : 0;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
+    return x;
+}
+
+// Rank search over register-held counts: thread t holds the N bins
+// b0 - N + 1 .. b0 (b0 = nb - N t - 1), c[j] the count of bin b0 - j (zero
+// for bins below 0).  Finds the bin holding the rank-th largest key in
+// descending bin order, the count above it and its own count; every thread
+// gets the answer.
+template <int N>
+__device__ __forceinline__ void find_rank_regs(const unsigned (&c)[N], int b0, unsigned rank,
+                                               unsigned *bin_out, unsigned *above_out,
+                                               unsigned *cnt_out, DecShared &sh) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    unsigned mine = 0;
+#pragma unroll
+    for (int j = 0; j < N; j++) mine += c[j];
+    unsigned incl = mine;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const unsigned y = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += y;
+    }
+    if (lane == 31) sh.wtmp[warp] = (int)incl;
+    __syncthreads();
+    unsigned above = incl - mine +
+                     (unsigned)warp_sum_first(lane < kDecWarps ? sh.wtmp[lane] : 0, lane, warp);
+#pragma unroll
+    for (int j = 0; j < N; j++) {
+        if (b0 - j >= 0 && above < rank && above + c[j] >= rank) {
+            sh.s_out[0] = (unsigned)(b0 - j);
+            sh.s_out[1] = above;
+            sh.s_out[2] = c[j];
+        }
+        above += c[j];
+    }
+    __syncthreads();
+    *bin_out = sh.s_out[0];
+    *above_out = sh.s_out[1];
+    *cnt_out = sh.s_out[2];
+    __syncthreads();
+}
+
+// Block-wide exclusive scan of two ints, with their totals in every thread.
+__device__ __forceinline__ int2 block_scan2_dec(int a, int b, DecShared &sh, int2 *total) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    int ia = a, ib = b;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int na = __shfl_up_sync(0xffffffffu, ia, o);
+        const int nb = __shfl_up_sync(0xffffffffu, ib, o);
+        if (lane >= o) {
+            ia += na;
+            ib += nb;
+        }
+    }
+    if (lane == 31) sh.wtmp2[warp] = make_int2(ia, ib);
+    __syncthreads();
+    const int2 w = lane < kDecWarps ? sh.wtmp2[lane] : make_int2(0, 0);
+    int2 r;
+    r.x = ia - a + warp_sum_first(w.x, lane, warp);
+    r.y = ib - b + warp_sum_first(w.y, lane, warp);
+    total->x = warp_sum_first(w.x, lane, kDecWarps);
+    total->y = warp_sum_first(w.y, lane, kDecWarps);
+    __syncthreads();
+    return r;
+}
+
+__global__ void __launch_bounds__(kDecThreads, 1)
+topk_decode_kernel(const float *scores, int64_t T, int K, int32_t *__restrict__ idx,
+                   const RowPrefetch pf, const uint32_t *row_hist) {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    cg::cluster_group cl = cg::this_cluster();
+    const int CN = (int)cl.num_blocks();
+    const int p = (int)cl.block_rank();
+    const int64_t row = blockIdx.x / CN;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int m = (int64_t)K < T ? K : (int)T;
+    int32_t *dst = idx + row * K;
+    if (m == T) {                          // every position selected (the same for every row)
+        asm volatile("griddepcontrol.wait;" ::: "memory");
+        for (int i = p * kDecThreads + tid; i < K; i += CN * kDecThreads) {
+            dst[i] = i < m ? i : -1;
+            if (i < m) pf(row, i);
+        }
+        return;
+    }
+    extern __shared__ __align__(16) uint8_t dec_smem[];
+    DecShared &sh = *reinterpret_cast<DecShared *>(dec_smem);
+    DecShared *sh0 = cl.map_shared_rank(&sh, 0);
+    if (p == 0) {
+        for (int i = tid; i < kBins; i += kDecThreads) sh.hist[i] = 0;
+        if (tid == 0) sh.n_cand = 0;
+    }
+    if (tid == 0) sh.n_few = 0;
+    __syncthreads();
+    // cleared: the other CTAs may write here once they have waited
+    asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
+    // the scores and the histogram come from the scorer
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+
+    // this thread's 8 bins of the row's histogram (4088 - 8t .. 4095 - 8t)
+    // and its 32 positions, loaded together
+    unsigned hc[8];
+    {
+        const uint4 *h4 = reinterpret_cast<const uint4 *>(row_hist + row * kBins + kBins - 8 * (tid + 1));
+        const uint4 x0 = h4[0], x1 = h4[1];
+        hc[0] = x1.w; hc[1] = x1.z; hc[2] = x1.y; hc[3] = x1.x;
+        hc[4] = x0.w; hc[5] = x0.z; hc[6] = x0.y; hc[7] = x0.x;
+    }
+    const int64_t t0 = (int64_t)p * kDecSpan + (int64_t)tid * kDecPer;
+    const float *src = scores + row * T + t0;
+    uint32_t key[kDecPer];
+    if (t0 + kDecPer <= T && (reinterpret_cast<uintptr_t>(src) & 15) == 0) {
+#pragma unroll
+        for (int j = 0; j < kDecPer / 4; j++) {
+            const float4 v = reinterpret_cast<const float4 *>(src)[j];
+            key[4 * j] = score_key(v.x);
+            key[4 * j + 1] = score_key(v.y);
+            key[4 * j + 2] = score_key(v.z);
+            key[4 * j + 3] = score_key(v.w);
+        }
+    } else {
+#pragma unroll
+        for (int j = 0; j < kDecPer; j++) key[j] = t0 + j < T ? score_key(src[j]) : 0u;
+    }
+    const int nv = T - t0 <= 0 ? 0 : (T - t0 >= kDecPer ? kDecPer : (int)(T - t0));
+
+    unsigned bin, above, n_group;
+    find_rank_regs<8>(hc, kBins - 8 * tid - 1, (unsigned)m, &bin, &above, &n_group, sh);
+    uint32_t prefix = bin;
+    int pbits = kBits;
+    unsigned rank = (unsigned)m - above;           // rank of tau within the group
+    asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
+
+    // too many keys to gather (rare: scores within a few percent of each
+    // other, or many exact ties): 12-bit rounds over the register keys,
+    // merged into CTA 0's histogram (clear on entry, cleared after each round)
+    while (n_group > (unsigned)kDecCap && pbits < 32) {
+        const int nb = 32 - pbits < kBits ? 32 - pbits : kBits;
+        const int sh_lo = 32 - pbits - nb;
+#pragma unroll
+        for (int j = 0; j < kDecPer; j++)
+            if (j < nv && (key[j] >> (32 - pbits)) == prefix)
+                atomicAdd(&sh0->hist[(key[j] >> sh_lo) & ((1u << nb) - 1u)], 1u);
+        cl.sync();
+        if (p == 0) {
+            unsigned c8[8];
+#pragma unroll
+            for (int j = 0; j < 8; j++) {
+                const int b = kBins - 8 * tid - 1 - j;
+                c8[j] = b < (1 << nb) ? sh.hist[b] : 0u;
+            }
+            unsigned b2, a2, n2;
+            find_rank_regs<8>(c8, kBins - 8 * tid - 1, rank, &b2, &a2, &n2, sh);
+            for (int i = tid; i < kBins; i += kDecThreads) sh.hist[i] = 0;
+            if (tid < CN) {
+                DecShared *r = cl.map_shared_rank(&sh, tid);
+                r->res[0] = (prefix << nb) | b2;
+                r->res[1] = (unsigned)(pbits + nb);
+                r->res[2] = rank - a2;
+                r->res[3] = n2;
+            }
+        }
+        cl.sync();
+        prefix = sh.res[0];
+        pbits = (int)sh.res[1];
+        rank = sh.res[2];
+        n_group = sh.res[3];
+    }
+
+    // ---- this CTA's keys above the group and inside it; the group's keys
+    // stored into a range of CTA 0's list (one atomic per CTA) when they are
+    // few enough to gather
+    const bool gather = n_group <= (unsigned)kDecCap && pbits < 32;
+    const int gshift = 32 - pbits;
+    int n_gt = 0, n_in = 0;
+#pragma unroll
+    for (int j = 0; j < kDecPer; j++) {
+        const uint32_t g = gshift == 32 ? 0u : key[j] >> gshift;
+        n_gt += j < nv && g > prefix;
+        n_in += j < nv && g == prefix;
+    }
+    int2 tot;
+    const int2 ex = block_scan2_dec(n_gt, n_in, sh, &tot);
+    if (tid == 0) {
+        sh0->cnt_gt[p] = tot.x;
+        sh0->cnt_in[p] = tot.y;
+        if (gather) {
+            const int b = atomicAdd(&sh0->n_cand, tot.y);
+            sh0->base[p] = b;
+            sh.my_base = b;
+        }
+    }
+    if (gather) {
+        __syncthreads();
+        if (n_in) {
+            int slot = sh.my_base + ex.y;
+#pragma unroll
+            for (int j = 0; j < kDecPer; j++)
+                if (j < nv && (key[j] >> gshift) == prefix) {
+                    if (slot < kDecCap) sh0->cand[slot] = make_uint2(key[j], (uint32_t)(t0 + j));
+                    slot++;
+                }
+        }
+    }
+    cl.sync();                                   // counts and keys in CTA 0
+
+    // ---- CTA 0: tau, q (tau-equal keys taken), every CTA's offset and quota
+    if (p == 0) {
+        uint32_t tau;
+        int q;
+        if (gather) {
+            const int E = sh.n_cand < kDecCap ? sh.n_cand : kDecCap;
+            uint32_t tp = prefix;
+            int tb = pbits;
+            unsigned rk = rank, cnt = n_group;
+            while (tb < 32) {
+                if (cnt <= (unsigned)kDecFew) {
+                    // at most 32 keys share the prefix: one warp ranks them
+                    const int sh_p = 32 - tb;
+                    for (int j = tid; j < E; j += kDecThreads) {
+                        const uint32_t k = sh.cand[j].x;
+                        if ((k >> sh_p) == tp) {
+                            const int f = atomicAdd(&sh.n_few, 1);
+                            if (f < kDecFew) sh.few[f] = k;
+                        }
+                    }
+                    __syncthreads();
+                    if (warp == 0) {
+                        const int n = sh.n_few < kDecFew ? sh.n_few : kDecFew;
+                        const bool valid = lane < n;
+                        const uint32_t kl = valid ? sh.few[lane] : 0u;
+                        int gt = 0, eq = 0;
+                        for (int i = 0; i < n; i++) {
+                            const uint32_t ki = __shfl_sync(0xffffffffu, kl, i);
+                            gt += ki > kl;
+                            eq += ki == kl;
+                        }
+                        if (valid && (unsigned)gt < rk && (unsigned)(gt + eq) >= rk) {
+                            sh.s_out[0] = kl;
+                            sh.s_out[1] = rk - (unsigned)gt;
+                        }
+                    }
+                    __syncthreads();
+                    tp = sh.s_out[0];
+                    rk = sh.s_out[1];
+                    break;
+                }
+                const int nb = 32 - tb < 10 ? 32 - tb : 10;
+                const int sh_lo = 32 - tb - nb;
+                for (int i = tid; i < kDecSub; i += kDecThreads) sh.hist[i] = 0;
+                __syncthreads();
+                for (int j = tid; j < E; j += kDecThreads) {
+                    const uint32_t k = sh.cand[j].x;
+                    if ((k >> (32 - tb)) == tp) atomicAdd(&sh.hist[(k >> sh_lo) & ((1u << nb) - 1u)], 1u);
+                }
+                __syncthreads();
+                // thread t: bins 1023 - 2t and 1022 - 2t (zero above the pass's range)
+                unsigned c2[2];
+#pragma unroll
+                for (int j = 0; j < 2; j++) {
+                    const int b = kDecSub - 2 * tid - 1 - j;
+                    c2[j] = b < (1 << nb) ? sh.hist[b] : 0u;
+                }
+                unsigned b1, a1, n1;
+                find_rank_regs<2>(c2, kDecSub - 2 * tid - 1, rk, &b1, &a1, &n1, sh);
+                tp = (tp << nb) | b1;
+                tb += nb;
+                rk -= a1;
+                cnt = n1;
+            }
+            tau = tp;
+            q = (int)rk;
+            // per CTA (its contiguous range of the list): keys above tau, equal to it
+            for (int r = warp; r < CN; r += kDecWarps) {
+                const int lo = sh.base[r], n = sh.cnt_in[r];
+                int gt = 0, eq = 0;
+                for (int j = lane; j < n; j += 32) {
+                    if (lo + j >= kDecCap) break;
+                    const uint32_t k = sh.cand[lo + j].x;
+                    gt += k > tau;
+                    eq += k == tau;
+                }
+                gt = warp_sum_first(gt, lane, 32);
+                eq = warp_sum_first(eq, lane, 32);
+                if (lane == 0) {
+                    sh.sel_gt[r] = gt;
+                    sh.sel_eq[r] = eq;
+                }
+            }
+            __syncthreads();
+        } else {
+            // the group is one key value: its keys are all tau-equal
+            tau = prefix;
+            q = (int)rank;
+        }
+        if (warp == 0) {
+            // exclusive prefix over the CTAs of (keys above tau, tau-equal keys)
+            const bool in = lane < CN;
+            const int gt_r = in ? sh.cnt_gt[lane] + (gather ? sh.sel_gt[lane] : 0) : 0;
+            const int eq_r = in ? (gather ? sh.sel_eq[lane] : sh.cnt_in[lane]) : 0;
+            int g = gt_r, e = eq_r;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int ng = __shfl_up_sync(0xffffffffu, g, o);
+                const int ne = __shfl_up_sync(0xffffffffu, e, o);
+                if (lane >= o) {
+                    g += ng;
+                    e += ne;
+                }
+            }
+            if (in) {
+                const int gt_below = g - gt_r, eq_below = e - eq_r;
+                int my_q = q - eq_below;
+                my_q = my_q < 0 ? 0 : (my_q > eq_r ? eq_r : my_q);
+                DecShared *r = cl.map_shared_rank(&sh, lane);
+                r->out[0] = tau;
+                r->out[1] = (unsigned)(gt_below + (q < eq_below ? q : eq_below));
+                r->out[2] = (unsigned)my_q;
+            }
+        }
+    }
+    cl.sync();                  // results delivered; no CTA touches another's memory after this
+    const uint32_t tau = sh.out[0];
+    const int off = (int)sh.out[1], my_q = (int)sh.out[2];
+
+    // ---- ordered write of this thread's 32 positions
+    int c_gt = 0, c_eq = 0;
+#pragma unroll
+    for (int j = 0; j < kDecPer; j++) {
+        c_gt += j < nv && key[j] > tau;
+        c_eq += j < nv && key[j] == tau;
+    }
+    int2 tot2;
+    const int2 e2 = block_scan2_dec(c_gt, c_eq, sh, &tot2);
+    int take_eq = my_q - e2.y;
+    take_eq = take_eq < 0 ? 0 : (take_eq > c_eq ? c_eq : take_eq);
+    int pos = off + e2.x + (my_q < e2.y ? my_q : e2.y);
+#pragma unroll
+    for (int j = 0; j < kDecPer; j++) {
+        if (j >= nv) break;
+        bool sel = key[j] > tau;
+        if (key[j] == tau && take_eq > 0) {
+            sel = true;
+            take_eq--;
+        }
+        if (sel && pos < m) {
+            dst[pos++] = (int32_t)(t0 + j);
+            pf(row, t0 + j);
+        }
+    }
+    for (int i = m + p * kDecThreads + tid; i < K; i += CN * kDecThreads) dst[i] = -1;
 }
 
 // One CTA per row, the row read from global memory (rows too long for the
@@ -642,23 +969,52 @@ size_t topk_workspace_bytes(int, int, int64_t, int) { return 0; }
 dsa_status launch_topk_select(const float *scores, int B, int S, int64_t T, int64_t start_pos,
                               int k, int32_t *idx, void *, cudaStream_t stream,
                               const void *prefetch_rows, int64_t prefetch_t_max,
-                              int prefetch_row_bytes) {
+                              int prefetch_row_bytes, const uint32_t *row_hist) {
     if ((int64_t)B * S * T == 0) return DSA_OK;
     const int K = (int64_t)k < T ? k : (int)T;
     const int64_t rows = (int64_t)B * S;
     const int64_t n_max = T < start_pos + S ? T : start_pos + S;
+    RowPrefetch pf;
+    pf.base = static_cast<const uint8_t *>(prefetch_rows);
+    pf.t_max = prefetch_t_max;
+    pf.bytes = prefetch_row_bytes;
+    if (row_hist && S == 1 && start_pos == T - 1 && (T + kDecSpan - 1) / kDecSpan <= kMaxCluster) {
+        // the decode top-k: one cluster per row, the threshold bin from the scorer's histogram
+        const int dcn = (int)((T + kDecSpan - 1) / kDecSpan);
+        const int dsmem = (int)sizeof(DecShared);
+        if (cudaFuncSetAttribute(topk_decode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 dsmem) != cudaSuccess ||
+            (dcn > 8 && cudaFuncSetAttribute(topk_decode_kernel,
+                                             cudaFuncAttributeNonPortableClusterSizeAllowed,
+                                             1) != cudaSuccess))
+            return DSA_ERR_CUDA;
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3((unsigned)(rows * dcn));
+        cfg.blockDim = dim3(kDecThreads);
+        cfg.dynamicSmemBytes = (size_t)dsmem;
+        cfg.stream = stream;
+        cudaLaunchAttribute attr[2];
+        attr[0].id = cudaLaunchAttributeClusterDimension;
+        attr[0].val.clusterDim.x = (unsigned)dcn;
+        attr[0].val.clusterDim.y = 1;
+        attr[0].val.clusterDim.z = 1;
+        // programmatic launch: the set-up overlaps the scorer's tail
+        attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[1].val.programmaticStreamSerializationAllowed = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 2;
+        if (cudaLaunchKernelEx(&cfg, topk_decode_kernel, scores, T, K, idx, pf, row_hist) != cudaSuccess)
+            return DSA_ERR_CUDA;
+        return launch_status();
+    }
     int cn, L;
     cluster_plan(n_max, &cn, &L);
     if (cn == 0) {
         topk_row_kernel<<<(unsigned)rows, kThreads, 0, stream>>>(scores, S, T, start_pos, K, idx);
         return launch_status();
     }
-    size_t smem = (size_t)(L + L / 32 + 1) * sizeof(float) + kGather * sizeof(uint32_t) +
-                  (size_t)L * sizeof(uint16_t);
-    // per-value bins too, when they fit beside the static shared memory (~17 KB)
-    const size_t bins_bytes = (size_t)((L + kThreads - 1) / kThreads) * kThreads * sizeof(uint16_t);
-    const int store_bins = smem + bins_bytes <= (size_t)(208 * 1024) ? 1 : 0;
-    if (store_bins) smem += bins_bytes;
+    // keys of the slice (padded) and the gathered keys with their positions
+    const size_t smem = (size_t)(L + L / 32 + 1) * sizeof(uint32_t) + (size_t)kCap * 8;
     if (cudaFuncSetAttribute(topk_cluster_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)smem) != cudaSuccess)
         return DSA_ERR_CUDA;
@@ -682,12 +1038,8 @@ dsa_status launch_topk_select(const float *scores, int B, int S, int64_t T, int6
     attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 2;
-    RowPrefetch pf;
-    pf.base = static_cast<const uint8_t *>(prefetch_rows);
-    pf.t_max = prefetch_t_max;
-    pf.bytes = prefetch_row_bytes;
-    if (cudaLaunchKernelEx(&cfg, topk_cluster_kernel, scores, S, T, start_pos, K, L, store_bins, idx,
-                           pf) != cudaSuccess)
+    if (cudaLaunchKernelEx(&cfg, topk_cluster_kernel, scores, S, T, start_pos, K, L, idx, pf) !=
+        cudaSuccess)
         return DSA_ERR_CUDA;
     return launch_status();
 }
