@@ -7,45 +7,35 @@
 // Causal mask" (index mask + causal mask, softmax, value mix).
 //
 // Shapes: Hq = 128 heads (the MMA M), rows [c (512) | k_pe (64)].
-// Work unit: one query row and U <= 256 consecutive slots of its selection
-// (slots holding -1 or a future position count as empty rows), computed by
-// TWO independent CTAs that differ only in which half of the 512 output
-// columns they produce.  Each CTA
-//   1. gathers the U rows in nine 64-column chunks (eight latent blocks and
-//      the rotary block) into 128B-swizzled K-major tiles, and accumulates the
-//      full logits S = Q C^T (M = 128 heads, N = U, K = 576) in TMEM with 36
-//      tcgen05.mma kind::f16 -- the logits are complete in every CTA, so no
-//      partial logits ever move between CTAs;
-//   2. runs an exact softmax over the U logits of each head (two passes over
-//      TMEM: the max, then exp2, the sum and P as bf16 written in place over
-//      the logits it came from);
-//   3. accumulates O = P C[:, own 256 columns] (M = 128, N = 256, K = U) with
-//      A = P read from TMEM and B = the CTA's four own latent chunks, which
-//      stay in shared memory after the logits (read MN-major), so the value
-//      mix needs no second gather;
-//   4. writes its 256 output columns: bf16 out (+ lse) when the row has one
-//      unit, else a normalised fp16 partial with its (max, sum, power-of-two
-//      ranges).  The partials of a row's units ("splits") are then merged:
-//      when the whole grid fits on the GPU at once it is launched as a
-//      cooperative grid, and after a grid-wide barrier every CTA merges its
-//      own slice of the output columns; otherwise a combine kernel merges.
-// The two CTAs of a unit read the same rows; the second read is served from
-// L2 (each CTA also prefetches half of the unit's rows into L2 at its start).
+// Work unit: one query row and U = 128 consecutive slots of its selection
+// (slots holding -1 or a future position count as empty rows), computed by one
+// CTA, which
+//   1. gathers the unit's rows in nine 64-column chunks (eight latent blocks
+//      and the rotary block), each into its own 16 KB 128B-swizzled K-major
+//      tile -- all nine stay resident, so every gather is issued up front --
+//      and accumulates the logits S = Q C^T (M = 128 heads, N = 128, K = 576)
+//      in TMEM with 36 tcgen05.mma kind::f16, A = the query's latent part
+//      from TMEM and its rotary block from shared memory;
+//   2. runs an exact softmax over the unit's 128 logits of each head (the
+//      thread's logits stay in registers between the max and the exp2 pass)
+//      and writes P as bf16 into shared memory, the A operand of the value mix;
+//   3. accumulates O = P C[:, 0:512] as two N = 256 halves (M = 128, K = 128)
+//      whose B operands are the latent chunks already resident (read
+//      MN-major), into all 512 TMEM columns;
+//   4. writes bf16 out (+ lse) when the row has one unit, else a normalised
+//      fp16 partial with its (max, sum, power-of-two ranges).  The partials of
+//      a row's units ("splits") are merged: when the whole grid fits on the
+//      GPU at once it is launched as a cooperative grid, and after a grid-wide
+//      barrier every CTA merges its own slice of the output columns;
+//      otherwise a combine kernel merges.
 //
-// Shared memory: six 32 KB chunk regions R0..R5 and the query's rotary block.
-// While the logits accumulate, the query's 512 latent columns sit in TMEM (the
-// output columns are not in use yet) and are the MMA's A operand there, so
-// the regions hold gathered rows only and six chunks are in flight at once.
-// Chunk order, regions and the MMA each chunk waits for before it may be
-// written:
-//   chunk    0     1     2     3     4     5     6     7     8
-//   block    own0  own1  oth0  oth1  oth2  oth3  own2  own3  rope
-//   region   R0    R1    R2    R3    R4    R5    R2    R3    R4
-//   waits    -     -     -     -     -     -     2     3     4
-// The own latent chunks end in R0..R3: consecutive regions, one MN-major
-// operand with a 32 KB stride between its 64-column blocks.
-// TMEM: S / P in columns [0, U); the query's latent part in [256, 512) during
-// the logits, then O in [256, 512).
+// Shared memory: nine chunk regions R0..R8 (R k holds chunk k), the query's
+// rotary block, and P (two 16 KB K-major blocks).  The query's latent blocks
+// are staged by TMA in P's space (blocks 0, 1) and in R2..R7 (blocks 2..7)
+// before the work threads move them to TMEM, so chunks 0, 1 and 8 are gathered
+// at once and chunks 2..7 once the staging is free.
+// TMEM: S in columns [0, 128) and the query's latent part in [256, 512) while
+// the logits accumulate; then O in [0, 512).
 //
 // The FP8 variant reads 656-byte rows [512 e4m3 | 4 fp32 block scales | 64
 // bf16].  The codes of a latent chunk are copied into the upper half of its
@@ -64,32 +54,29 @@ namespace dsa {
 namespace {
 
 constexpr int kHq = 128, kDc = 512, kDr = 64, kDqk = kDc + kDr;
-constexpr int kUnitMax = 256;                   // selected rows per unit (max MMA N)
+constexpr int kU = 128;                         // selected rows per unit (the MMA N of the logits)
 constexpr int kChunks = 9;                      // 8 latent blocks + the rotary block
-constexpr int kRegions = 6;
-constexpr int kRegion = kUnitMax * 128;         // one chunk of 256 rows: 32 KB
+constexpr int kRegion = kU * 128;               // one chunk of 128 rows: 16 KB
 constexpr int kQBlk = kHq * 128;                // one 64-column block of the query: 16 KB
-constexpr int kQRope = kRegions * kRegion;      // the query's rotary block
-constexpr int kScales = kQRope + kQBlk;         // FP8: the unit's block scales, 16 B per row
-constexpr int kList = kScales + kUnitMax * 16;  // the unit's rows (int32)
-constexpr int kBars = kList + kUnitMax * 4;
+constexpr int kQRope = kChunks * kRegion;       // the query's rotary block
+constexpr int kP = kQRope + kQBlk;              // P: two K-major blocks of 64 slots
+constexpr int kScales = kP + 2 * kQBlk;         // FP8: the unit's block scales, 16 B per row
+constexpr int kList = kScales + kU * 16;        // the unit's rows (int32)
+constexpr int kBars = kList + kU * 4;
 constexpr int kWork = 256;                      // gather / softmax / epilogue threads
 constexpr int kThreads = kWork + 32;            // + one TMA / MMA warp
 constexpr int kMaxSel = 2048;                   // selection slots per query row
-constexpr uint32_t kColS = 0, kColQ = 256, kColO = 256, kTmemCols = 512;
+constexpr int kOct = kDc / 8;                   // output octets per head: 64
+constexpr uint32_t kColS = 0, kColQ = 256, kColO = 0, kTmemCols = 512;
 constexpr int kRowFp8 = kDc + 4 * (kDc / 128) + 2 * kDr;   // 656
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
 
 constexpr size_t kSmemBytes = 1024 + (size_t)kBars + 32 * sizeof(uint64_t) + 64;
+static_assert(kSmemBytes <= 227 * 1024, "shared memory");
 
-// chunk schedule of the CTA with output half `half` (see the table above)
-__device__ __forceinline__ int chunk_block(int k, int half) {
-    const int own = half * 4, oth = (1 - half) * 4;
-    return k < 2 ? own + k : (k < 6 ? oth + (k - 2) : (k < 8 ? own + (k - 4) : 8));
-}
-__device__ __forceinline__ int chunk_region(int k) { return k < 6 ? k : k - 4; }
-__device__ __forceinline__ int chunk_dep(int k) { return k < 6 ? -1 : k - 4; }
+// where the query's latent block cb is staged by TMA
+__device__ __forceinline__ int q_stage(int cb) { return cb < 2 ? kP + cb * kQBlk : cb * kRegion; }
 
 struct MlaArgs {
     const __nv_bfloat16 *q;    // [rows, 128, 576]
@@ -98,12 +85,12 @@ struct MlaArgs {
     const int32_t *idx;
     __nv_bfloat16 *out;
     float *lse;
-    __half *part_o;            // [blocks][256 / 8][128][8] (split combine kernel)
-    float4 *part_ml;           // [blocks][128] (max, sum, fp16 range of columns 0..127, of 128..255)
+    __half *part_o;            // [blocks][64 octets][128][8] (split partials)
+    float4 *part_ml;           // [blocks][128] (max, sum, fp16 range of columns 0..255, of 256..511)
     int64_t t_max;
     int64_t start_pos;
     int64_t row0;              // first query row of this launch
-    int S, k, splits, unit_rows;
+    int S, k, splits;
     int coop;                  // cooperative grid: the splits are merged in this kernel
     float scale_log2;          // sm_scale * log2(e)
     int *err;
@@ -174,16 +161,16 @@ __device__ __forceinline__ uint4 decode8(uint32_t w0, uint32_t w1, float sc) {
     return make_uint4(o[0], o[1], o[2], o[3]);
 }
 
-// Merges output columns [8 c8, 8 c8 + 8) of head h of one (row, half) from
-// its splits' fp16 partials (blocks blk0 .. blk0 + splits - 1), for NC octets
+// Merges output columns [8 c8, 8 c8 + 8) of head h of one query row from its
+// splits' fp16 partials (blocks blk0 .. blk0 + splits - 1), for NC octets
 // c8[0..NC) at once: with w_s = 2^(m_s - M) l_s and Y_s = O_s / (l_s sc_s),
 // out = sum_s w_s sc_s Y_s / sum_s w_s and lse = (M + log2 sum_s w_s) ln 2.
 // The loads of eight splits are in flight together; further batches rescale
 // the running sums.
 template <int NC>
 __device__ __forceinline__ void merge_octets(const __half *part_o, const float4 *part_ml, int splits,
-                                             int64_t blk0, int64_t row, int half, const int (&c8)[NC],
-                                             int h, __nv_bfloat16 *out, float *lse) {
+                                             int64_t blk0, int64_t row, const int (&c8)[NC], int h,
+                                             __nv_bfloat16 *out, float *lse) {
     float M = -INFINITY, L = 0.f;
     float acc[NC][8];
 #pragma unroll
@@ -200,7 +187,7 @@ __device__ __forceinline__ void merge_octets(const __half *part_o, const float4 
 #pragma unroll
             for (int n = 0; n < NC; n++)
                 if (sp < splits)
-                    x[u][n] = reinterpret_cast<const uint4 *>(part_o + (blk0 + sp) * kHq * 256)[c8[n] * kHq + h];
+                    x[u][n] = reinterpret_cast<const uint4 *>(part_o + (blk0 + sp) * kHq * kDc)[c8[n] * kHq + h];
         }
         float mb = M;
 #pragma unroll
@@ -222,7 +209,7 @@ __device__ __forceinline__ void merge_octets(const __half *part_o, const float4 
             L += w;
 #pragma unroll
             for (int n = 0; n < NC; n++) {
-                const float ws = w * (c8[n] < 16 ? ml[u].z : ml[u].w);
+                const float ws = w * (c8[n] < kOct / 2 ? ml[u].z : ml[u].w);
                 const uint32_t xs[4] = {x[u][n].x, x[u][n].y, x[u][n].z, x[u][n].w};
 #pragma unroll
                 for (int e = 0; e < 4; e++) {
@@ -242,9 +229,8 @@ __device__ __forceinline__ void merge_octets(const __half *part_o, const float4 
             const __nv_bfloat162 v = __floats2bfloat162_rn(acc[n][2 * e] * inv, acc[n][2 * e + 1] * inv);
             w8[e] = *reinterpret_cast<const uint32_t *>(&v);
         }
-        reinterpret_cast<uint4 *>(out + (row * kHq + h) * kDc + half * 256)[c8[n]] =
-            make_uint4(w8[0], w8[1], w8[2], w8[3]);
-        if (half == 0 && c8[n] == 0 && lse) lse[row * kHq + h] = L > 0.f ? (M + log2f(L)) * kLn2 : -INFINITY;
+        reinterpret_cast<uint4 *>(out + (row * kHq + h) * kDc)[c8[n]] = make_uint4(w8[0], w8[1], w8[2], w8[3]);
+        if (c8[n] == 0 && lse) lse[row * kHq + h] = L > 0.f ? (M + log2f(L)) * kLn2 : -INFINITY;
     }
 }
 
@@ -257,41 +243,35 @@ sparse_mla_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const MlaArgs a) 
     int32_t *list = reinterpret_cast<int32_t *>(sm + kList);             // the unit's rows
     uint64_t *bars = reinterpret_cast<uint64_t *>(sm + kBars);
     uint64_t *chunk_full = bars;                 // [9] chunk k gathered (256 arrivals)
-    uint64_t *mma_done = bars + kChunks;         // [9] chunk k's logit MMAs complete
-    uint64_t *q_full = bars + 2 * kChunks;       // the query's rotary block landed (TMA)
+    uint64_t *q_full = bars + kChunks;           // the query landed (TMA)
     uint64_t *q_ready = q_full + 1;              // the query's latent part is in TMEM (256 arrivals)
-    uint64_t *p_full = q_ready + 1;              // [2] P of each row group is in TMEM (256 arrivals)
-    uint64_t *o_full = p_full + 2;               // [2] each output column half is complete
-    uint64_t *mma_fin = o_full + 2;              // every issued MMA is complete
-    uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(bars + 28);   // after the 25 barriers
+    uint64_t *s_done = q_ready + 1;              // every logit MMA is complete
+    uint64_t *p_full = s_done + 1;               // P is in shared memory (256 arrivals)
+    uint64_t *o_full = p_full + 1;               // O is complete
+    uint64_t *mma_fin = o_full + 1;              // every issued MMA is complete
+    uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(bars + 16);   // after the 15 barriers
     volatile int *abort = reinterpret_cast<volatile int *>(tmem_holder + 1);
-    int *scan_tmp = const_cast<int *>(abort) + 1;                         // 9 ints
-    // softmax exchange (max, sum, output range of the two column halves):
-    // region R5, free once the logits are complete
-    float *red = reinterpret_cast<float *>(sm + 5 * kRegion);
+    uint32_t *vmask = reinterpret_cast<uint32_t *>(const_cast<int *>(abort) + 1);   // [4]
+    // softmax exchange (max and sum of the two slot halves): the query's
+    // rotary block, free once the logits are complete
+    float *red = reinterpret_cast<float *>(sm + kQRope);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    // blockIdx.x = ((row - row0) * 2 + half) * splits + sp
+    // blockIdx.x = (row - row0) * splits + sp
     const int sp = (int)(blockIdx.x % (unsigned)a.splits);
-    const int half = (int)((blockIdx.x / (unsigned)a.splits) & 1u);
-    const int64_t row = a.row0 + blockIdx.x / (unsigned)a.splits / 2;
+    const int64_t row = a.row0 + blockIdx.x / (unsigned)a.splits;
     const int64_t b = row / a.S, s = row - b * a.S;
     const int64_t limit = a.start_pos + s;
-    const int U = a.unit_rows;
     const uint32_t sbase = tc::smem_u32(sm);
 
     if (warp == kWork / 32) {
         if (lane == 0) {
-            for (int i = 0; i < kChunks; i++) {
-                tc::mbar_init(&chunk_full[i], kWork);
-                tc::mbar_init(&mma_done[i], 1);
-            }
+            for (int i = 0; i < kChunks; i++) tc::mbar_init(&chunk_full[i], kWork);
             tc::mbar_init(q_full, 1);
             tc::mbar_init(q_ready, kWork);
-            for (int i = 0; i < 2; i++) {
-                tc::mbar_init(&p_full[i], kWork);
-                tc::mbar_init(&o_full[i], 1);
-            }
+            tc::mbar_init(s_done, 1);
+            tc::mbar_init(p_full, kWork);
+            tc::mbar_init(o_full, 1);
             tc::mbar_init(mma_fin, 1);
             *abort = 0;
             tc::fence_mbar_init();
@@ -307,12 +287,12 @@ sparse_mla_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const MlaArgs a) 
     const uint32_t tmem = *tmem_holder;
     if (warp == kWork / 32 && lane == 0) {
         // the query: its rotary block stays in shared memory (the MMA's A
-        // operand there); its eight latent blocks are staged in R2..R5 and
-        // moved to TMEM by the work threads
+        // operand there); its eight latent blocks are staged in P's space and
+        // R2..R7 and moved to TMEM by the work threads
         tc::mbar_arrive_expect_tx(q_full, kChunks * kQBlk);
         tc::tma_load_2d(sm + kQRope, &tm_q, kDc, (int)(row * kHq), q_full);
         for (int cb = 0; cb < 8; cb++)
-            tc::tma_load_2d(sm + 2 * kRegion + cb * kQBlk, &tm_q, cb * 64, (int)(row * kHq), q_full);
+            tc::tma_load_2d(sm + q_stage(cb), &tm_q, cb * 64, (int)(row * kHq), q_full);
     }
     // a kernel launched after this one (the split combine) may start its set-up
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
@@ -320,16 +300,15 @@ sparse_mla_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const MlaArgs a) 
     // (a no-op without a programmatic launch), then read them with plain loads.
     asm volatile("griddepcontrol.wait;" ::: "memory");
 
-    // This unit is the slots [lo, lo + U) of the row's selection, slot lo + j
+    // This unit is the slots [lo, lo + 128) of the row's selection, slot lo + j
     // as row j.  A slot counts when it holds a causal position (>= 0 and <=
     // start_pos + s); vmask has one bit per row.  (A top-k selection lists
     // its positions first and pads with -1, so its units are dense.)
-    const int lo = sp * U;
-    uint32_t *vmask = reinterpret_cast<uint32_t *>(scan_tmp);          // [8]
-    {
+    const int lo = sp * kU;
+    if (threadIdx.x < kU) {
         const int j = threadIdx.x;
         int32_t t = -1;
-        if (j < U && lo + j < a.k) {
+        if (lo + j < a.k) {
             t = a.idx[row * a.k + lo + j];
             if (t >= 0 && (int64_t)t <= limit) {
                 if ((int64_t)t >= a.t_max) {
@@ -340,14 +319,12 @@ sparse_mla_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const MlaArgs a) 
                 t = -1;
             }
         }
-        if (j < kUnitMax) list[j] = t;
+        list[j] = t;
         const uint32_t bal = __ballot_sync(0xffffffffu, t >= 0);
-        if (warp < kUnitMax / 32 && lane == 0) vmask[warp] = bal;
+        if (lane == 0) vmask[warp] = bal;
     }
     __syncthreads();
-    uint32_t any = 0;
-#pragma unroll
-    for (int w = 0; w < kUnitMax / 32; w++) any |= vmask[w];
+    const uint32_t any = vmask[0] | vmask[1] | vmask[2] | vmask[3];
     const int64_t rbase = b * a.t_max;
 
     if (!any) {
@@ -355,33 +332,33 @@ sparse_mla_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const MlaArgs a) 
         if (threadIdx.x < kWork) {
             const int h = threadIdx.x & (kHq - 1), c = threadIdx.x >> 7;
             if (a.splits > 1) {
-                uint4 *po = reinterpret_cast<uint4 *>(a.part_o + (int64_t)blockIdx.x * kHq * 256) + h;
-                for (int o8 = 16 * c; o8 < 16 * c + 16; o8++) po[o8 * kHq] = make_uint4(0u, 0u, 0u, 0u);
+                uint4 *po = reinterpret_cast<uint4 *>(a.part_o + (int64_t)blockIdx.x * kHq * kDc) + h;
+                for (int o8 = 32 * c; o8 < 32 * c + 32; o8++) po[o8 * kHq] = make_uint4(0u, 0u, 0u, 0u);
                 if (c == 0) a.part_ml[(int64_t)blockIdx.x * kHq + h] = make_float4(-INFINITY, 0.f, 1.f, 1.f);
             } else {
-                uint4 *o16 = reinterpret_cast<uint4 *>(a.out + (row * kHq + h) * kDc + half * 256 + c * 128);
-                for (int j = 0; j < 16; j++) o16[j] = make_uint4(0u, 0u, 0u, 0u);
-                if (half == 0 && c == 0 && a.lse) a.lse[row * kHq + h] = -INFINITY;
+                uint4 *o16 = reinterpret_cast<uint4 *>(a.out + (row * kHq + h) * kDc + c * 256);
+                for (int j = 0; j < 32; j++) o16[j] = make_uint4(0u, 0u, 0u, 0u);
+                if (c == 0 && a.lse) a.lse[row * kHq + h] = -INFINITY;
             }
         }
         if (warp == kWork / 32 && lane == 0) tc::mbar_wait(q_full, 0, a.err, abort);
     } else if (warp < kWork / 32) {
         const int gt = threadIdx.x;
-        const int q4 = warp & 3, c = warp >> 2;          // TMEM lane quarter, column half
+        const int q4 = warp & 3, c = warp >> 2;          // TMEM lane quarter; slot half / column half
         const int h = q4 * 32 + lane;                    // head
         const uint32_t lane_addr = (uint32_t)(q4 * 32) << 16;
         bool ok = true;
         // ------------------------------------------------------------ gather
-        // Issue chunk k: 16-byte cp.async pieces (rows past the unit's end are
+        // Issue chunk k into region k: 16-byte cp.async pieces (empty rows are
         // zero-filled: finite values that meet P = 0).  bf16 rows and the FP8
         // rotary block land in their swizzled tile; FP8 codes land in the
         // upper half of the region, to be decoded in place.
         auto issue = [&](int k) {
-            const int cb = chunk_block(k, half);
-            const uint32_t rg = sbase + chunk_region(k) * kRegion;
-            if (!kFp8 || cb == 8) {
-                for (int f = gt; f < U * 8; f += kWork) {
-                    const int j = f >> 3, p = f & 7;
+            const uint32_t rg = sbase + k * kRegion;
+            if (!kFp8 || k == 8) {
+#pragma unroll
+                for (int u = 0; u < kU * 8 / kWork; u++) {
+                    const int f = gt + u * kWork, j = f >> 3, p = f & 7;
                     const int32_t tl = list[j];
                     const bool v = tl >= 0;
                     const int64_t t = v ? (int64_t)tl : 0;
@@ -389,19 +366,20 @@ sparse_mla_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const MlaArgs a) 
                     if constexpr (kFp8)
                         src = a.kv8 + (rbase + t) * kRowFp8 + kDc + 4 * (kDc / 128) + p * 16;
                     else
-                        src = a.kv + (rbase + t) * kDqk + cb * 64 + p * 8;
+                        src = a.kv + (rbase + t) * kDqk + k * 64 + p * 8;
                     cp_async16(rg + j * 128 + ((p ^ (j & 7)) << 4), src, v ? 16u : 0u);
                 }
             } else {
-                for (int f = gt; f < U * 4; f += kWork) {
-                    const int j = f >> 2, p = f & 3;
+#pragma unroll
+                for (int u = 0; u < kU * 4 / kWork; u++) {
+                    const int f = gt + u * kWork, j = f >> 2, p = f & 3;
                     const int32_t tl = list[j];
                     const bool v = tl >= 0;
                     const int64_t t = v ? (int64_t)tl : 0;
                     cp_async16(rg + kRegion / 2 + j * 64 + p * 16,
-                               a.kv8 + (rbase + t) * kRowFp8 + cb * 64 + p * 16, v ? 16u : 0u);
+                               a.kv8 + (rbase + t) * kRowFp8 + k * 64 + p * 16, v ? 16u : 0u);
                 }
-                if (k == 0 && gt < U) {                   // the row's four block scales
+                if (k == 0 && gt < kU) {                  // the row's four block scales
                     const int32_t tl = list[gt];
                     const bool v = tl >= 0;
                     const int64_t t = v ? (int64_t)tl : 0;
@@ -410,33 +388,32 @@ sparse_mla_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const MlaArgs a) 
                 }
             }
             cp_async_commit();
+            // bf16 chunks are published by the copies themselves (an arrival
+            // when this thread's copies so far have landed)
+            if constexpr (!kFp8) cp_async_arrive(&chunk_full[k]);
         };
-        // Chunk k has landed for this thread (`pending` later groups may still
-        // be in flight): FP8 latent codes are decoded in place (every thread's
-        // codes must have landed before any are read, and every read must be
-        // done before the first write), then the chunk is published.
+        // FP8: chunk k has landed for this thread (`pending` later groups may
+        // still be in flight); its latent codes are decoded in place (every
+        // thread's codes must have landed before any are read, and every read
+        // must be done before the first write), then the chunk is published.
         auto publish = [&](int k, int pending) {
             cp_async_wait_n(pending);
-            const int cb = chunk_block(k, half);
-            if (kFp8 && cb != 8) {
-                const uint32_t rg = sbase + chunk_region(k) * kRegion;
-                constexpr int kPer = kUnitMax * 4 / kWork;   // 16-code pieces per thread
+            if (k != 8) {
+                const uint32_t rg = sbase + k * kRegion;
+                constexpr int kPer = kU * 4 / kWork;         // 16-code pieces per thread
                 uint4 cw[kPer];
                 float sc[kPer];
                 tc::named_barrier(1, kWork);
 #pragma unroll
                 for (int u = 0; u < kPer; u++) {
                     const int f = gt + u * kWork, j = f >> 2, p = f & 3;
-                    if (j < U) {
-                        cw[u] = ld_shared_v4(rg + kRegion / 2 + j * 64 + p * 16);
-                        sc[u] = reinterpret_cast<const float *>(sm + kScales + j * 16)[cb >> 1];
-                    }
+                    cw[u] = ld_shared_v4(rg + kRegion / 2 + j * 64 + p * 16);
+                    sc[u] = reinterpret_cast<const float *>(sm + kScales + j * 16)[k >> 1];
                 }
                 tc::named_barrier(1, kWork);
 #pragma unroll
                 for (int u = 0; u < kPer; u++) {
                     const int f = gt + u * kWork, j = f >> 2, p = f & 3;
-                    if (j >= U) continue;
                     st_shared_v4(rg + j * 128 + (((2 * p) ^ (j & 7)) << 4), decode8(cw[u].x, cw[u].y, sc[u]));
                     st_shared_v4(rg + j * 128 + (((2 * p + 1) ^ (j & 7)) << 4), decode8(cw[u].z, cw[u].w, sc[u]));
                 }
@@ -444,25 +421,18 @@ sparse_mla_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const MlaArgs a) 
             tc::fence_proxy_async_smem();
             tc::mbar_arrive(&chunk_full[k]);
         };
-        // chunks 0 and 1 go to free regions at once; 2..5 once the query's
-        // latent part has left its staging in R2..R5.  bf16 chunks are
-        // published by the copies themselves (an arrival when this thread's
-        // copies have landed); FP8 latent chunks are decoded in place first.
-        auto start = [&](int k) {
-            issue(k);
-            if constexpr (!kFp8) cp_async_arrive(&chunk_full[k]);
-            else cp_async_commit();
-        };
-        start(0);
-        start(1);
-        // the query's latent part (head h, columns [256c, 256c + 256)) from its
-        // swizzled staging to TMEM columns kColQ + [128c, 128c + 128), two bf16
-        // per column
+        // chunks 0, 1 and 8 go to free regions at once; 2..7 once the query's
+        // latent part has left its staging
+        issue(0);
+        issue(1);
+        issue(8);
+        // the query's latent part (head h, blocks 4c..4c+3) from its swizzled
+        // staging to TMEM columns kColQ + 32 cb, two bf16 per column
         if (ok && !tc::mbar_wait(q_full, 0, a.err, abort)) ok = false;
 #pragma unroll 1
         for (int blk = 0; blk < 4; blk++) {
             const int cb = 4 * c + blk;
-            const uint32_t src = sbase + 2 * kRegion + cb * kQBlk + h * 128;
+            const uint32_t src = sbase + q_stage(cb) + h * 128;
 #pragma unroll
             for (int hf = 0; hf < 2; hf++) {
                 uint32_t r[16];
@@ -478,102 +448,71 @@ sparse_mla_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const MlaArgs a) 
         tc::tc_fence_before();
         tc::mbar_arrive(q_ready);
         tc::named_barrier(1, kWork);            // the staging is no longer read
-        for (int k = 2; k < kRegions; k++) start(k);
-        if constexpr (kFp8)
-            for (int k = 0; k < kRegions; k++) publish(k, kRegions - 1 - k);
-        // chunks 6..8 reuse regions: wait for the MMA that read them last
-        for (int k = kRegions; k < kChunks; k++) {
-            if (ok && !tc::mbar_wait(&mma_done[chunk_dep(k)], 0, a.err, abort)) ok = false;
-            if (ok) start(k);
-            else if constexpr (kFp8) cp_async_commit();
-            else tc::mbar_arrive(&chunk_full[k]);
+        for (int k = 2; k < 8; k++) issue(k);
+        if constexpr (kFp8) {
+            // in issue order: 0, 1, 8, 2, ..., 7
+            publish(0, 8);
+            publish(1, 7);
+            publish(8, 6);
+            for (int k = 2; k < 8; k++) publish(k, 7 - k);
         }
-        if constexpr (kFp8)
-            for (int k = kRegions; k < kChunks; k++) publish(k, kChunks - 1 - k);
 
         // ----------------------------------------------------------- softmax
-        // thread (head h, column half c): logits of rows [c U/2, (c+1) U/2).
-        // This thread's logits (up to 128) in two TMEM reads of 64 columns per
-        // pass (nine warps leave at most 168 registers a thread).  Logits of
-        // rows past the unit's end count as -inf; eight independent max and
-        // sum chains keep the dependent latency short.
-        const int hc = U / 2, base = c * hc;
-        if (ok && !tc::mbar_wait(&mma_done[kChunks - 1], 0, a.err, abort)) ok = false;
+        // thread (head h, slot half c): the logits of rows [64c, 64c + 64),
+        // kept in registers between the max and the exp2 pass; rows of no
+        // selection count as -inf; eight independent chains for the max and
+        // the sum
+        if (ok && !tc::mbar_wait(s_done, 0, a.err, abort)) ok = false;
         tc::tc_fence_after();
-        // validity bits of rows [base + 64g, base + 64g + 64), none past hc
-        auto rowbits = [&](int g, uint32_t &w0, uint32_t &w1) {
-            w0 = vmask[(base + 64 * g) >> 5];
-            w1 = 64 * g + 32 < hc ? vmask[((base + 64 * g) >> 5) + 1] : 0u;
-        };
+        uint32_t sv[64];
+#pragma unroll
+        for (int i = 0; i < 4; i++)
+            tc::tmem_ld16(tmem + lane_addr + kColS + 64 * c + 16 * i,
+                          *reinterpret_cast<uint32_t(*)[16]>(sv + 16 * i));
+        tc::tmem_wait_ld();
+        const uint32_t w0 = vmask[2 * c], w1 = vmask[2 * c + 1];
+        const bool part = (w0 & w1) != 0xffffffffu;
         float mx8[8];
 #pragma unroll
         for (int e = 0; e < 8; e++) mx8[e] = -INFINITY;
 #pragma unroll
-        for (int g = 0; g < 2; g++) {
-            if (64 * g >= hc) break;
-            uint32_t sv[64];
-#pragma unroll
-            for (int i = 0; i < 4; i++)
-                if (64 * g + 16 * i < hc)
-                    tc::tmem_ld16(tmem + lane_addr + kColS + base + 64 * g + 16 * i,
-                                  *reinterpret_cast<uint32_t(*)[16]>(sv + 16 * i));
-            tc::tmem_wait_ld();
-            uint32_t w0, w1;
-            rowbits(g, w0, w1);
-            const bool part = (w0 & w1) != 0xffffffffu;
-#pragma unroll
-            for (int e = 0; e < 64; e++) {
-                float x = __uint_as_float(sv[e]) * a.scale_log2;
-                if (part && !(((e < 32 ? w0 : w1) >> (e & 31)) & 1u)) x = -INFINITY;
-                mx8[e & 7] = fmaxf(mx8[e & 7], x);
-            }
+        for (int e = 0; e < 64; e++) {
+            float x = __uint_as_float(sv[e]) * a.scale_log2;
+            if (part && !(((e < 32 ? w0 : w1) >> (e & 31)) & 1u)) x = -INFINITY;
+            mx8[e & 7] = fmaxf(mx8[e & 7], x);
         }
         const float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
                                fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
         red[c * kHq + h] = mx;
         tc::named_barrier(1, kWork);
-        const float m = fmaxf(red[h], red[kHq + h]);       // finite: row 0 is valid
+        const float m = fmaxf(red[h], red[kHq + h]);       // finite: the unit has a row
         float l8[8];
 #pragma unroll
         for (int e = 0; e < 8; e++) l8[e] = 0.f;
-        // P of this thread's rows over the first half of its logits, 32 rows
-        // (16 columns) per store
+        // P of rows [64c, 64c + 64) is the K-major block c of the A operand:
+        // head h's 128-byte row, 16-byte piece i = rows 8i .. 8i + 7
+        const uint32_t prow = sbase + kP + c * kQBlk + h * 128;
 #pragma unroll
-        for (int g = 0; g < 2; g++) {
-            if (64 * g >= hc) break;
-            uint32_t sv[64];
+        for (int i = 0; i < 8; i++) {
+            uint32_t pk[4];
 #pragma unroll
-            for (int i = 0; i < 4; i++)
-                if (64 * g + 16 * i < hc)
-                    tc::tmem_ld16(tmem + lane_addr + kColS + base + 64 * g + 16 * i,
-                                  *reinterpret_cast<uint32_t(*)[16]>(sv + 16 * i));
-            tc::tmem_wait_ld();
-            uint32_t w0, w1;
-            rowbits(g, w0, w1);
-            const bool part = (w0 & w1) != 0xffffffffu;
-#pragma unroll
-            for (int i = 0; i < 2; i++) {
-                uint32_t pk[16];
-#pragma unroll
-                for (int e = 0; e < 16; e++) {
-                    const int x = 32 * i + 2 * e;
-                    float t0 = fmaf(__uint_as_float(sv[x]), a.scale_log2, -m);
-                    float t1 = fmaf(__uint_as_float(sv[x + 1]), a.scale_log2, -m);
-                    const uint32_t wb = i == 0 ? w0 : w1;
-                    if (part && !((wb >> (2 * e)) & 1u)) t0 = -INFINITY;
-                    if (part && !((wb >> (2 * e + 1)) & 1u)) t1 = -INFINITY;
-                    const float p0 = ex2(t0), p1 = ex2(t1);
-                    l8[e & 7] += p0 + p1;
-                    const __nv_bfloat162 v01 = __floats2bfloat162_rn(p0, p1);
-                    pk[e] = *reinterpret_cast<const uint32_t *>(&v01);
-                }
-                // rows [base + 64g + 32i, +32) -> columns base + 32g + 16i (their
-                // logits were read above)
-                if (64 * g + 32 * i < hc)
-                    tc::tmem_st16(tmem + lane_addr + kColS + base + 32 * g + 16 * i, pk);
+            for (int e = 0; e < 4; e++) {
+                const int x = 8 * i + 2 * e;
+                float t0 = fmaf(__uint_as_float(sv[x]), a.scale_log2, -m);
+                float t1 = fmaf(__uint_as_float(sv[x + 1]), a.scale_log2, -m);
+                const uint32_t wb = x < 32 ? w0 : w1;
+                if (part && !((wb >> (x & 31)) & 1u)) t0 = -INFINITY;
+                if (part && !((wb >> ((x + 1) & 31)) & 1u)) t1 = -INFINITY;
+                const float p0 = ex2(t0), p1 = ex2(t1);
+                l8[(2 * e) & 7] += p0;
+                l8[(2 * e + 1) & 7] += p1;
+                const __nv_bfloat162 v01 = __floats2bfloat162_rn(p0, p1);
+                pk[e] = *reinterpret_cast<const uint32_t *>(&v01);
             }
+            st_shared_v4(prow + ((i ^ (h & 7)) << 4), make_uint4(pk[0], pk[1], pk[2], pk[3]));
         }
-        tc::tmem_wait_st();
+        // P is read by the tensor core (async proxy)
+        tc::fence_proxy_async_smem();
         tc::tc_fence_before();
         tc::mbar_arrive(p_full);
         red[2 * kHq + c * kHq + h] = ((l8[0] + l8[1]) + (l8[2] + l8[3])) + ((l8[4] + l8[5]) + (l8[6] + l8[7]));
@@ -581,15 +520,15 @@ sparse_mla_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const MlaArgs a) 
         const float lt = red[2 * kHq + h] + red[3 * kHq + h];
 
         // ---------------------------------------------------------- epilogue
-        // thread (h, c) owns output columns [128c, 128c + 128) of this CTA's 256
+        // thread (h, c) owns output columns [256c, 256c + 256)
         if (ok && !tc::mbar_wait(o_full, 0, a.err, abort)) ok = false;
         tc::tc_fence_after();
-        const uint32_t ocol = tmem + lane_addr + kColO + c * 128;
+        const uint32_t ocol = tmem + lane_addr + kColO + c * 256;
         if (a.splits == 1) {
             const float inv = lt > 0.f ? 1.f / lt : 0.f;
-            uint4 *o16 = reinterpret_cast<uint4 *>(a.out + (row * kHq + h) * kDc + half * 256 + c * 128);
-#pragma unroll
-            for (int g = 0; g < 2; g++) {
+            uint4 *o16 = reinterpret_cast<uint4 *>(a.out + (row * kHq + h) * kDc + c * 256);
+#pragma unroll 1
+            for (int g = 0; g < 4; g++) {
                 uint32_t ov[64];
 #pragma unroll
                 for (int i = 0; i < 4; i++)
@@ -607,45 +546,48 @@ sparse_mla_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const MlaArgs a) 
                     if (ok) o16[g * 8 + o8] = make_uint4(w[0], w[1], w[2], w[3]);
                 }
             }
-            if (ok && half == 0 && c == 0 && a.lse)
-                a.lse[row * kHq + h] = lt > 0.f ? (m + log2f(lt)) * kLn2 : -INFINITY;
+            if (ok && c == 0 && a.lse) a.lse[row * kHq + h] = lt > 0.f ? (m + log2f(lt)) * kLn2 : -INFINITY;
         } else {
-            // O / (l * sc) in fp16 for the split combine, sc the power of two
+            // O / (l * sc) in fp16 for the split merge, sc the power of two
             // that keeps this column half's |O / l| / sc <= 2^14, as
-            // [column / 8][head] groups of eight halves
-            uint32_t ov[2][64];
+            // [column / 8][head] groups of eight halves; the half's range is
+            // found in a first read of its columns
             float amax = 0.f;
-#pragma unroll
-            for (int g = 0; g < 2; g++) {
+#pragma unroll 1
+            for (int g = 0; g < 4; g++) {
+                uint32_t ov[64];
 #pragma unroll
                 for (int i = 0; i < 4; i++)
-                    tc::tmem_ld16(ocol + 64 * g + 16 * i, *reinterpret_cast<uint32_t(*)[16]>(ov[g] + 16 * i));
+                    tc::tmem_ld16(ocol + 64 * g + 16 * i, *reinterpret_cast<uint32_t(*)[16]>(ov + 16 * i));
+                tc::tmem_wait_ld();
+#pragma unroll
+                for (int e = 0; e < 64; e++) amax = fmaxf(amax, fabsf(__uint_as_float(ov[e])));
             }
-            tc::tmem_wait_ld();
-#pragma unroll
-            for (int g = 0; g < 2; g++)
-#pragma unroll
-                for (int e = 0; e < 64; e++) amax = fmaxf(amax, fabsf(__uint_as_float(ov[g][e])));
             const float inv_l = lt > 0.f ? 1.f / lt : 0.f;
             float scl = 1.f;
             while (amax * inv_l > 16384.f * scl) scl *= 2.f;
             const float inv = inv_l / scl;
-            uint4 *po = reinterpret_cast<uint4 *>(a.part_o + (int64_t)blockIdx.x * kHq * 256) + h;
+            uint4 *po = reinterpret_cast<uint4 *>(a.part_o + (int64_t)blockIdx.x * kHq * kDc) + h;
+#pragma unroll 1
+            for (int g = 0; g < 4; g++) {
+                uint32_t ov[64];
 #pragma unroll
-            for (int g = 0; g < 2; g++) {
+                for (int i = 0; i < 4; i++)
+                    tc::tmem_ld16(ocol + 64 * g + 16 * i, *reinterpret_cast<uint32_t(*)[16]>(ov + 16 * i));
+                tc::tmem_wait_ld();
 #pragma unroll
                 for (int o8 = 0; o8 < 8; o8++) {
                     uint32_t w[4];
 #pragma unroll
                     for (int e = 0; e < 4; e++) {
-                        const __half2 v = __floats2half2_rn(__uint_as_float(ov[g][8 * o8 + 2 * e]) * inv,
-                                                            __uint_as_float(ov[g][8 * o8 + 2 * e + 1]) * inv);
+                        const __half2 v = __floats2half2_rn(__uint_as_float(ov[8 * o8 + 2 * e]) * inv,
+                                                            __uint_as_float(ov[8 * o8 + 2 * e + 1]) * inv);
                         w[e] = *reinterpret_cast<const uint32_t *>(&v);
                     }
-                    if (ok) po[(c * 16 + g * 8 + o8) * kHq] = make_uint4(w[0], w[1], w[2], w[3]);
+                    if (ok) po[(c * 32 + g * 8 + o8) * kHq] = make_uint4(w[0], w[1], w[2], w[3]);
                 }
             }
-            // (max, sum, range of columns [0, 128), range of columns [128, 256))
+            // (max, sum, range of columns [0, 256), range of columns [256, 512))
             float *ml = reinterpret_cast<float *>(a.part_ml + (int64_t)blockIdx.x * kHq + h);
             if (ok) {
                 if (c == 0) {
@@ -656,9 +598,9 @@ sparse_mla_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const MlaArgs a) 
             }
         }
     } else if (lane > 0) {
-        // lanes 1..31 of the MMA warp: each CTA of the unit prefetches every
-        // other row into L2 (its partner the rest), whole rows at a time
-        for (int j = 2 * (lane - 1) + half; j < U; j += 62) {
+        // lanes 1..31 of the MMA warp: the unit's rows into L2, whole rows at
+        // a time, ahead of the chunk gathers
+        for (int j = lane - 1; j < kU; j += 31) {
             if (list[j] < 0) continue;
             if constexpr (kFp8)
                 tc::prefetch_l2_bulk(a.kv8 + (rbase + list[j]) * kRowFp8, kRowFp8);
@@ -667,9 +609,11 @@ sparse_mla_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const MlaArgs a) 
         }
     } else {
         // ------------------------------------------------------ TMA / MMA
-        const uint32_t id_qk = tc::instr_desc(tc::kFmtBF16, tc::kFmtBF16, 128, U);
+        const uint32_t id_qk = tc::instr_desc(tc::kFmtBF16, tc::kFmtBF16, 128, kU);
         bool ok = tc::mbar_wait(q_full, 0, a.err, abort) && tc::mbar_wait(q_ready, 0, a.err, abort);
-        for (int k = 0; ok && k < kChunks; k++) {
+        // chunks in issue order: 0, 1, 8, 2, ..., 7
+        for (int i = 0; ok && i < kChunks; i++) {
+            const int k = i < 2 ? i : (i == 2 ? 8 : i - 1);
             if (!tc::mbar_wait(&chunk_full[k], 0, a.err, abort)) {
                 ok = false;
                 break;
@@ -678,33 +622,35 @@ sparse_mla_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const MlaArgs a) 
             // or stores): order them before the tensor core's reads
             tc::fence_proxy_async_smem();
             tc::tc_fence_after();
-            const int cb = chunk_block(k, half);
-            const uint32_t ca = sbase + chunk_region(k) * kRegion;
+            const uint32_t ca = sbase + k * kRegion;
 #pragma unroll
             for (int ks = 0; ks < 4; ks++) {
                 const uint64_t bd = tc::smem_desc(ca + ks * 32, 1024, tc::kSwizzle128B);
-                if (cb < 8)        // A = the query's latent block cb in TMEM
-                    tc::mma_f16_ts(tmem + kColS, tmem + kColQ + cb * 32 + ks * 8, bd, id_qk,
-                                   k > 0 || ks > 0);
+                if (k < 8)         // A = the query's latent block k in TMEM
+                    tc::mma_f16_ts(tmem + kColS, tmem + kColQ + k * 32 + ks * 8, bd, id_qk,
+                                   i > 0 || ks > 0);
                 else               // A = the query's rotary block in shared memory
                     tc::mma_f16(tmem + kColS,
                                 tc::smem_desc(sbase + kQRope + ks * 32, 1024, tc::kSwizzle128B), bd,
-                                id_qk, k > 0 || ks > 0);
+                                id_qk, i > 0 || ks > 0);
             }
-            tc::tc_commit(&mma_done[k]);
         }
+        if (ok) tc::tc_commit(s_done);
         if (ok && tc::mbar_wait(p_full, 0, a.err, abort)) {
             tc::tc_fence_after();
-            // O += P C[:, own 256]: K-step ks covers rows [16 ks, 16 ks + 16),
-            // whose P sits in the first quarter of its column half; B = the own
-            // chunks in R0..R3
+            // O[:, 256 hv + n] += P C[:, 256 hv + n]: K-step ks covers rows
+            // [16 ks, 16 ks + 16); A = P (K-major, block ks / 4), B = the latent
+            // chunks 4 hv .. 4 hv + 3 (MN-major, 16 KB between 64-column blocks)
             const uint32_t id_pv = tc::instr_desc(tc::kFmtBF16, tc::kFmtBF16, 128, 256, true);
-            const int hc = U / 2;
-            for (int ks = 0; ks < U / 16; ks++) {
-                const int r0 = 16 * ks, c = r0 / hc;
-                const uint32_t pa = tmem + kColS + c * hc + (r0 - c * hc) / 2;
-                const uint64_t bd = tc::smem_desc(sbase + ks * 2048, 1024, tc::kSwizzle128B, kRegion);
-                tc::mma_f16_ts(tmem + kColO, pa, bd, id_pv, ks > 0);
+            for (int ks = 0; ks < kU / 16; ks++) {
+                const uint64_t pa = tc::smem_desc(sbase + kP + (ks >> 2) * kQBlk + (ks & 3) * 32, 1024,
+                                                  tc::kSwizzle128B);
+#pragma unroll
+                for (int hv = 0; hv < 2; hv++) {
+                    const uint64_t bd = tc::smem_desc(sbase + 4 * hv * kRegion + ks * 2048, 1024,
+                                                      tc::kSwizzle128B, kRegion);
+                    tc::mma_f16(tmem + kColO + 256 * hv, pa, bd, id_pv, ks > 0);
+                }
             }
             tc::tc_commit(o_full);
         }
@@ -720,10 +666,10 @@ sparse_mla_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const MlaArgs a) 
     }
     if (a.coop) {
         // every split of every row has written its partial: merge this
-        // split's slice of its (row, half)'s output columns (32 / splits
-        // octets of eight columns)
+        // split's slice of its row's output columns (64 / splits octets of
+        // eight columns)
         cooperative_groups::this_grid().sync();
-        const int npo = 32 / a.splits;
+        const int npo = kOct / a.splits;
         const int h = threadIdx.x & (kHq - 1), o = threadIdx.x >> 7;
         const int64_t blk0 = (int64_t)blockIdx.x - sp;
         if (threadIdx.x < kWork) {
@@ -731,17 +677,17 @@ sparse_mla_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const MlaArgs a) 
             int oc = o;
             for (; oc + 2 < npo; oc += 4) {
                 const int c8[2] = {npo * sp + oc, npo * sp + oc + 2};
-                merge_octets<2>(a.part_o, a.part_ml, a.splits, blk0, row, half, c8, h, a.out, a.lse);
+                merge_octets<2>(a.part_o, a.part_ml, a.splits, blk0, row, c8, h, a.out, a.lse);
             }
             if (oc < npo) {
                 const int c8[1] = {npo * sp + oc};
-                merge_octets<1>(a.part_o, a.part_ml, a.splits, blk0, row, half, c8, h, a.out, a.lse);
+                merge_octets<1>(a.part_o, a.part_ml, a.splits, blk0, row, c8, h, a.out, a.lse);
             }
         }
     }
 }
 
-// Merges the splits of each (row, half) when the attention grid is not
+// Merges the splits of each query row when the attention grid is not
 // cooperative: thread (head, octet) merges eight output columns of one head,
 // consecutive threads consecutive heads (coalesced reads of the partials).
 __global__ void __launch_bounds__(kHq)
@@ -749,29 +695,19 @@ sparse_mla_combine_kernel(const __half *part_o, const float4 *part_ml, int split
                           __nv_bfloat16 *__restrict__ out, float *__restrict__ lse) {
     // the partials come from the preceding kernel: wait for it (plain loads below)
     asm volatile("griddepcontrol.wait;" ::: "memory");
-    constexpr int groups = 256 / 8;
-    const int64_t rh = blockIdx.x / groups;                 // (row - row0) * 2 + half
-    const int c8[1] = {(int)(blockIdx.x % groups)};
-    merge_octets<1>(part_o, part_ml, splits, rh * splits, row0 + (rh >> 1), (int)(rh & 1), c8,
-                    threadIdx.x, out, lse);
+    const int64_t r = blockIdx.x / kOct;                 // row - row0
+    const int c8[1] = {(int)(blockIdx.x % kOct)};
+    merge_octets<1>(part_o, part_ml, splits, r * splits, row0 + r, c8, threadIdx.x, out, lse);
 }
 
-// Rows per unit: the smallest of 64, 128, 192, 256 whose units (two CTAs
-// each) fit on the SMs at once; 256 when none does.
-int mla_unit_rows(int64_t rows, int k) {
-    for (int u = 64; u <= kUnitMax; u += 64)
-        if (rows * 2 * ((k + u - 1) / u) <= num_sms()) return u;
-    return kUnitMax;
-}
-
-// Split partials of one query row (both output halves of every split).
+// Split partials of one query row.
 size_t partial_bytes_per_row(int splits) {
-    return (size_t)2 * splits * kHq * (256 * sizeof(__half) + sizeof(float4));
+    return (size_t)splits * kHq * (kDc * sizeof(__half) + sizeof(float4));
 }
 
 // Query rows per launch: all of them, unless their split partials would pass
 // kWsBudget; then the rows run in launches of this many (each reusing the
-// workspace after its combine).
+// workspace after its merge).
 constexpr size_t kWsBudget = size_t(256) << 20;
 int64_t rows_per_launch(int64_t rows, int splits) {
     if (splits <= 1) return rows;
@@ -781,11 +717,10 @@ int64_t rows_per_launch(int64_t rows, int splits) {
 }
 
 size_t workspace_bytes(int64_t rows, int k) {
-    const int u = mla_unit_rows(rows, k);
-    const int sp = (k + u - 1) / u;
+    const int sp = (k + kU - 1) / kU;
     if (sp <= 1) return 0;
-    const int64_t units = rows_per_launch(rows, sp) * 2 * sp;
-    return align_up((size_t)units * kHq * 256 * sizeof(__half), 256) +
+    const int64_t units = rows_per_launch(rows, sp) * sp;
+    return align_up((size_t)units * kHq * kDc * sizeof(__half), 256) +
            (size_t)units * kHq * sizeof(float4);
 }
 
@@ -814,16 +749,15 @@ dsa_status launch(const void *q, const void *kv, int64_t t_max, const int32_t *i
     a.start_pos = start_pos;
     a.S = S;
     a.k = k;
-    a.unit_rows = mla_unit_rows(rows, k);
-    a.splits = (k + a.unit_rows - 1) / a.unit_rows;
+    a.splits = (k + kU - 1) / kU;
     a.scale_log2 = sm_scale * kLog2e;
     a.err = device_error_word();
     const int64_t chunk = rows_per_launch(rows, a.splits);
     if (a.splits > 1) {
-        const int64_t units = chunk * 2 * a.splits;
+        const int64_t units = chunk * a.splits;
         a.part_o = static_cast<__half *>(ws);
         a.part_ml = reinterpret_cast<float4 *>(static_cast<char *>(ws) +
-                                               align_up((size_t)units * kHq * 256 * sizeof(__half), 256));
+                                               align_up((size_t)units * kHq * kDc * sizeof(__half), 256));
     }
     if (cudaFuncSetAttribute(sparse_mla_tc_kernel<kFp8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)kSmemBytes) != cudaSuccess)
@@ -832,18 +766,18 @@ dsa_status launch(const void *q, const void *kv, int64_t t_max, const int32_t *i
     // cooperative (all of its CTAs resident at once, one launch) and each
     // split gets whole octets of columns; else a combine kernel follows.
     bool coop = false;
-    if (a.splits > 1 && 32 % a.splits == 0 && chunk == rows) {
+    if (a.splits > 1 && kOct % a.splits == 0 && chunk == rows) {
         int per_sm = 0;
         if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, sparse_mla_tc_kernel<kFp8>,
                                                           kThreads, kSmemBytes) == cudaSuccess &&
-            (int64_t)per_sm * num_sms() >= rows * a.splits * 2)
+            (int64_t)per_sm * num_sms() >= rows * a.splits)
             coop = true;
     }
     for (int64_t r0 = 0; r0 < rows; r0 += chunk) {
         const int64_t n = rows - r0 < chunk ? rows - r0 : chunk;
         a.row0 = r0;
         cudaLaunchConfig_t cfg = {};
-        cfg.gridDim = dim3((unsigned)(n * a.splits * 2));
+        cfg.gridDim = dim3((unsigned)(n * a.splits));
         cfg.blockDim = dim3(kThreads);
         cfg.dynamicSmemBytes = kSmemBytes;
         cfg.stream = stream;
@@ -877,7 +811,7 @@ dsa_status launch(const void *q, const void *kv, int64_t t_max, const int32_t *i
         if (st != DSA_OK) return st;
         if (a.splits == 1 || a.coop) continue;
         cudaLaunchConfig_t ccfg = {};
-        ccfg.gridDim = dim3((unsigned)(n * 2 * (256 / 8)));
+        ccfg.gridDim = dim3((unsigned)(n * kOct));
         ccfg.blockDim = dim3(kHq);
         ccfg.stream = stream;
         cudaLaunchAttribute cattr[1];
