@@ -89,6 +89,22 @@ int dsa_version(void);
 dsa_status dsa_get_device_error(dsa_stream_t stream, int32_t *device_status);
 
 /*
+ * Diagnostic of the bounded device waits (failure detection; the pages have
+ * no counterpart).  Every wait of this library's kernels on a barrier (a TMA
+ * load, a tensor-core commit, a peer CTA) gives up after a budget of SM clock
+ * cycles, records DSA_ERR_TIMEOUT in the device word above and lets the kernel
+ * return normally: no trap, and the context stays usable.  This call launches
+ * one CTA that waits through that same routine on a shared-memory barrier,
+ * with a budget of budget_cycles (1 .. 2e9, about a second at 2 GHz, the
+ * budget the kernels use).  With complete = 0 nobody arrives, so the wait
+ * expires after about budget_cycles and DSA_ERR_TIMEOUT is recorded; with
+ * complete != 0 the barrier completes at once and nothing is recorded.
+ * Returns DSA_ERR_INVALID_ARG for a budget outside that range (nothing
+ * launched), DSA_ERR_CUDA if the launch fails.
+ */
+dsa_status dsa_wait_selftest(int64_t budget_cycles, int complete, dsa_stream_t stream);
+
+/*
  * rotate_activation + act_quant (Indexer.forward, "Split indexer heads"):
  * each d-vector is rotated by the orthonormal Walsh-Hadamard transform
  * (butterflies in fp32 with strides 1, 2, ..., d/2, then one multiply by

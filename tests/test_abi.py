@@ -179,3 +179,11 @@ def test_decode_step_argument_checks(dsa):
     assert call(T=0) == dsa.DSA_ERR_INVALID_ARG
     assert call(ws_bytes=need - 1) == dsa.DSA_ERR_WORKSPACE
     assert call(ws=NULL) == dsa.DSA_ERR_WORKSPACE
+
+
+def test_wait_selftest_argument_checks(dsa):
+    L = dsa._lib
+    # a budget outside 1 .. 2e9 cycles is refused before anything is launched
+    assert L.dsa_wait_selftest(0, 0, NULL) == dsa.DSA_ERR_INVALID_ARG
+    assert L.dsa_wait_selftest(-5, 1, NULL) == dsa.DSA_ERR_INVALID_ARG
+    assert L.dsa_wait_selftest(2_000_000_001, 0, NULL) == dsa.DSA_ERR_INVALID_ARG

@@ -91,6 +91,27 @@ def test_decode_step_deterministic(dsa):
     assert torch.equal(idx1, st["idx"]) and torch.equal(out1, st["out"])
 
 
+def test_decode_step_repeats_bitwise_50_steps(dsa):
+    """50 back-to-back decode steps on one state at the long-context shapes
+    (B = 8, T = 131072, the launch configuration the benchmark times): the
+    selections, outputs and lse are bitwise the first step's every time (the
+    re-appended key writes the same codes; the scorer's histogram atomics, the
+    cluster top-k and the split merge are order-independent)."""
+    wl = workloads.WORKLOADS[4]
+    _, st = decode_batch(dsa, wl)
+    idx1, out1, lse1 = st["idx"].clone(), st["out"].clone(), st["lse"].clone()
+    outs = []
+    for i in range(50):
+        run_decode(dsa, wl, st)
+        outs.append((st["idx"].clone(), st["out"].clone(), st["lse"].clone()))
+    torch.cuda.synchronize()
+    assert dsa.dsa_get_device_error() == dsa.DSA_OK
+    for i, (idx, out, lse) in enumerate(outs):
+        assert torch.equal(idx, idx1), f"step {i}: selection differs"
+        assert torch.equal(out, out1), f"step {i}: output differs"
+        assert torch.equal(lse, lse1), f"step {i}: lse differs"
+
+
 @pytest.mark.parametrize("T,B", [(5000, 2), (131072, 8)])
 def test_decode_step_fp8_latent_cache(dsa, T, B):
     """The decode step over the FP8 latent cache (656-byte rows): the selection

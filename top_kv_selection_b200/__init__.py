@@ -36,6 +36,7 @@ _SIGNATURES = {
     "dsa_status_string": ([_i32], ctypes.c_char_p),
     "dsa_version": ([], _i32),
     "dsa_get_device_error": ([_P, _P], _i32),
+    "dsa_wait_selftest": ([_i64, _i32, _P], _i32),
     "dsa_indexer_quant": ([_P, _i32, _i64, _i64, _i32, _P, _i64, _P, _i64, _P], _i32),
     "dsa_indexer_prologue": ([_P, _P, _i32, _i32, _i32, _i32, _i32, _i32, _P, _i32, _i64, _i64,
                               _P, _P, _P, _P, _P], _i32),
@@ -122,6 +123,14 @@ def dsa_get_device_error(stream=None) -> int:
     code = ctypes.c_int32(0)
     _check("dsa_get_device_error", _lib.dsa_get_device_error(_stream(stream), ctypes.byref(code)))
     return code.value
+
+
+def dsa_wait_selftest(budget_cycles: int, complete: bool = False, stream=None) -> None:
+    """Run one bounded device wait of budget_cycles SM cycles: with complete=False
+    nobody arrives, so it expires and records DSA_ERR_TIMEOUT (read it with
+    dsa_get_device_error); with complete=True it succeeds at once."""
+    _check("dsa_wait_selftest", _lib.dsa_wait_selftest(int(budget_cycles), 1 if complete else 0,
+                                                       _stream(stream)))
 
 
 def dsa_indexer_quant(x: torch.Tensor, out_fp8: torch.Tensor, out_scale: torch.Tensor,

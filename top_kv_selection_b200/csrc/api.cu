@@ -1,9 +1,11 @@
-// api.cu -- status strings, version, the sticky device error word, and the
-// per-context cache of device-symbol addresses.
+// api.cu -- status strings, version, the sticky device error word, the
+// per-context cache of device-symbol addresses, and the diagnostic of the
+// bounded device waits.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
 #include "common.cuh"
+#include "tc_ptx.cuh"
 
 // First error code recorded by any kernel of the library on this device
 // (0 = none).  Kernels never trap; they record here and skip the access.
@@ -83,4 +85,35 @@ extern "C" dsa_status dsa_get_device_error(dsa_stream_t stream, int32_t *device_
     if (host != 0 && cudaMemset(word, 0, sizeof(int)) != cudaSuccess) return DSA_ERR_CUDA;
     *device_status = host;
     return DSA_OK;
+}
+
+namespace {
+
+// One CTA waits on a shared-memory barrier through the wait routine every
+// kernel of the library uses, with the given budget; nobody arrives unless
+// `complete`, so the wait either succeeds at once or expires and records
+// DSA_ERR_TIMEOUT.
+__global__ void __launch_bounds__(32) wait_selftest_kernel(long long budget, int complete, int *err) {
+    __shared__ __align__(8) uint64_t bar;
+    __shared__ int abort_flag;
+    if (threadIdx.x == 0) {
+        dsa::tc::mbar_init(&bar, 1);
+        abort_flag = 0;
+        dsa::tc::fence_mbar_init();
+    }
+    __syncthreads();
+    if (complete && threadIdx.x == 0) dsa::tc::mbar_arrive(&bar);
+    dsa::tc::mbar_wait(&bar, 0, err, &abort_flag, budget);
+    __syncthreads();
+}
+
+}  // namespace
+
+extern "C" dsa_status dsa_wait_selftest(int64_t budget_cycles, int complete, dsa_stream_t stream) {
+    if (budget_cycles < 1 || budget_cycles > dsa::tc::kWaitBudget) return DSA_ERR_INVALID_ARG;
+    int *err = dsa::device_error_word();
+    if (!err) return DSA_ERR_CUDA;
+    wait_selftest_kernel<<<1, 32, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
+        (long long)budget_cycles, complete, err);
+    return dsa::launch_status();
 }

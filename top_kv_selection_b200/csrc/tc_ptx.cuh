@@ -74,16 +74,16 @@ __device__ __forceinline__ void prefetch_l2_bulk(const void *src, uint32_t bytes
 constexpr long long kWaitBudget = 2000000000LL;
 
 // Waits for the phase with the given parity.  Returns false (and records
-// DSA_ERR_TIMEOUT in the error word) if the budget runs out or if another
-// thread of the CTA already gave up (*abort set); never spins forever.
+// DSA_ERR_TIMEOUT in the error word) if `budget` SM clock cycles pass or if
+// another thread of the CTA already gave up (*abort set); never spins forever.
 __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, int *err,
-                                          volatile int *abort) {
+                                          volatile int *abort, long long budget = kWaitBudget) {
     if (mbar_try_wait(bar, parity)) return true;
     const long long t0 = clock64();
     while (true) {
         if (mbar_try_wait(bar, parity)) return true;
         if (*abort) return false;
-        if (clock64() - t0 > kWaitBudget) {
+        if (clock64() - t0 > budget) {
             record_error(err, DSA_ERR_TIMEOUT);
             *abort = 1;
             return false;
