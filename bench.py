@@ -406,9 +406,14 @@ def run_ours(args, wl, world, rank, local):
     stages = time_stages(dsa, wl, copies, iters=max(10, min(args.steps, 500)))
     t_score = stages["decode_index_scores"]
     prefill = prologue = attn_fp8 = None
+    prefill_chain = None
     if not args.no_prefill:
         prefill = time_prefill_scoring(dsa, measure_fp8_peak(sustained=False)["fp8_e4m3_tflops"])
         prologue = time_indexer_prologue(dsa, peak)
+        try:
+            prefill_chain = time_prefill_chain(dsa, peak)
+        except Exception as exc:                   # reported, never fatal to the main line
+            prefill_chain = {"error": f"{type(exc).__name__}: {exc}"[:200]}
     try:
         attn_fp8 = time_sparse_mla_fp8(dsa, peak, wl)
     except Exception as exc:                       # reported, never fatal to the main line
@@ -444,6 +449,7 @@ def run_ours(args, wl, world, rank, local):
         "stage_us": {k: round(v * 1e6, 2) for k, v in stages.items()},
         "prefill_scoring": prefill,
         "indexer_prologue": prologue,
+        "prefill_chain": prefill_chain,
         "sparse_mla_fp8": attn_fp8,
         "clocks": clk.summary(),
     }
@@ -582,6 +588,120 @@ def time_indexer_prologue(dsa, peak_gbs, iters=20):
     return out
 
 
+BF16_FALLBACK_TFLOPS = 1590.0
+
+
+def _bf16_peak():
+    """Dense bf16 tensor peak (TFLOP/s) for the prefill attention's roofline:
+    the driver's measured cuBLAS figure when present, else the pool's earlier
+    measurement."""
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            p = json.load(f)
+        for key in ("bf16_tflops", "bf16_tflops_burst"):
+            if key in p:
+                return float(p[key]), "measured"
+    return BF16_FALLBACK_TFLOPS, "fallback"
+
+
+def time_prefill_chain(dsa, hbm_peak, iters=3):
+    """The causal prefill of one T = 8192 sequence end to end on the device:
+    the fused indexer prologue (RoPE, rotate_activation, act_quant, key cache
+    write), the causal index scores (64 heads x 128, FP8), the per-row top-2048
+    and the sparse MLA attention (128 heads over the selected latent rows,
+    512 + 64 bf16).  Every stage is timed on its own with CUDA events, then the
+    four back to back.  Inputs are seeded random normals made on the device
+    (performance only; parity is the tests' job).
+
+    Rooflines: the top-k reads the causal scores and writes the selections
+    (HBM-bound); the attention's algorithmic work is the valid (query, selected
+    row) pairs, sum_s min(s + 1, 2048), times 128 heads x (576 + 512) x 2 flop
+    = 4.09 TFLOP, against the dense bf16 tensor peak."""
+    wl = workloads.WORKLOADS[3]
+    T, H, D, R = wl.T, wl.H, wl.D, 64
+    Hq, dc, dr, k = wl.Hq, wl.dc, wl.dr, wl.topk
+    dev = "cuda"
+    g = torch.Generator(device=dev).manual_seed(wl.seed(3))
+    q = torch.randn(1, T, H, D, device=dev, generator=g).to(torch.bfloat16)
+    keys = torch.randn(1, T, D, device=dev, generator=g).to(torch.bfloat16)
+    th = torch.rand(T, R // 2, device=dev, generator=g) * 6.283185307179586
+    cs = torch.stack([torch.cos(th), torch.sin(th)], dim=-1).contiguous()
+    w = torch.randn(1, T, H, device=dev, generator=g)
+    q_fp8 = torch.empty(1, T, H, D, dtype=torch.uint8, device=dev)
+    q_scale = torch.empty(1, T, H, dtype=torch.float32, device=dev)
+    k_cache = torch.empty(1, T, D, dtype=torch.uint8, device=dev)
+    k_scale = torch.empty(1, T, dtype=torch.float32, device=dev)
+    scores = torch.empty(1, T, T, dtype=torch.float32, device=dev)
+    idx = torch.empty(1, T, k, dtype=torch.int32, device=dev)
+    topk_ws = torch.empty(max(1, dsa.dsa_topk_select_workspace_size(1, T, T, k)), dtype=torch.uint8,
+                          device=dev)
+    kv = torch.randn(1, T, dc + dr, device=dev, generator=g).to(torch.bfloat16)
+    q_mla = torch.empty(1, T, Hq, dc + dr, dtype=torch.bfloat16, device=dev)
+    for s0 in range(0, T, 1024):                       # 1.2 GB of queries, made in slices
+        q_mla[:, s0:s0 + 1024] = torch.randn(1, min(1024, T - s0), Hq, dc + dr, device=dev,
+                                             generator=g).to(torch.bfloat16)
+    out = torch.empty(1, T, Hq, dc, dtype=torch.bfloat16, device=dev)
+    lse = torch.empty(1, T, Hq, dtype=torch.float32, device=dev)
+    attn_ws = torch.empty(max(1, dsa.dsa_sparse_mla_attn_workspace_size(1, T, Hq, dc, dr, k,
+                                                                        dsa.DSA_BF16)),
+                          dtype=torch.uint8, device=dev)
+
+    def prologue():
+        dsa.dsa_indexer_prologue(q, keys, cs, 0, q_fp8, q_scale, k_cache, k_scale)
+
+    def score():
+        dsa.dsa_index_scores(q_fp8, q_scale, w, k_cache, k_scale, 0, T, wl.softmax_scale_idx, scores)
+
+    def topk():
+        dsa.dsa_topk_select(scores, 0, k, idx, topk_ws)
+
+    def attn():
+        dsa.dsa_sparse_mla_attn(q_mla, kv, idx, 0, wl.sm_scale, out, lse, attn_ws)
+
+    def chain():
+        prologue()
+        score()
+        topk()
+        attn()
+
+    def timed(fn):
+        fn()
+        torch.cuda.synchronize()
+        t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        t0.record()
+        for _ in range(iters):
+            fn()
+        t1.record()
+        t1.synchronize()
+        return t0.elapsed_time(t1) * 1e-3 / iters
+
+    t_pro, t_sc, t_tk, t_at, t_ch = (timed(f) for f in (prologue, score, topk, attn, chain))
+    if dsa.dsa_get_device_error() != 0:
+        raise RuntimeError("device error word set during the prefill chain")
+    bf16_peak, bf16_kind = _bf16_peak()
+    pairs = sum(min(s + 1, k) for s in range(T))
+    attn_flop = pairs * Hq * (dc + dr + dc) * 2
+    topk_bytes = T * (T + 1) // 2 * 4 + T * k * 4
+    res = {
+        "workload": wl.name, "T": T, "k": k,
+        "prologue_us": t_pro * 1e6, "scores_us": t_sc * 1e6,
+        "topk": {"rows": T, "positions": T, "k": k, "us": t_tk * 1e6, "bytes": topk_bytes,
+                 "achieved_gbs": topk_bytes / t_tk / 1e9, "peak_gbs": hbm_peak,
+                 "frac": topk_bytes / t_tk / 1e9 / hbm_peak, "bound": "hbm",
+                 "note": "bytes = the causal scores read once + the selections written"},
+        "sparse_mla": {"queries": T, "selected_pairs": pairs, "tflop": attn_flop / 1e12,
+                       "us": t_at * 1e6, "tflops": attn_flop / t_at / 1e12,
+                       "peak_tflops": bf16_peak, "peak_kind": f"{bf16_kind} bf16 dense",
+                       "frac": attn_flop / t_at / 1e12 / bf16_peak, "bound": "tensor"},
+        "chain_us": t_ch * 1e6,
+        "chain_note": "prologue -> scores -> top-k -> attention back to back on one stream",
+    }
+    del q_mla, out, scores, attn_ws
+    torch.cuda.empty_cache()
+    return res
+
+
 def time_sparse_mla_fp8(dsa, peak_gbs, wl, iters=32, sets=16):
     """Sparse attention over the FP8 latent cache (656 B rows) at the decode
     workload's sizes: B queries x 2048 selected rows of a B x T cache.  The
@@ -678,6 +798,9 @@ def main(argv=None):
                     help="time only the fused indexer prologue on the T=8192 prefill")
     ap.add_argument("--prefill-only", action="store_true",
                     help="only time the prefill scoring (T = 8192 causal) and exit")
+    ap.add_argument("--prefill-chain-only", action="store_true",
+                    help="only time the T = 8192 prefill chain (prologue, scores, top-k, "
+                         "attention) and exit")
     ap.add_argument("--fp8-peak", action="store_true",
                     help="measure the dense FP8 GEMM peak and exit")
     ap.add_argument("--copies", type=int, default=N_COPIES,
@@ -699,6 +822,13 @@ def main(argv=None):
         import top_kv_selection_b200 as dsa
         print(json.dumps(time_prefill_scoring(dsa, measure_fp8_peak(sustained=False)["fp8_e4m3_tflops"],
                                               iters=max(1, args.steps))), flush=True)
+        return
+    if args.prefill_chain_only:
+        import __graft_entry__
+        __graft_entry__._builder().build()
+        import top_kv_selection_b200 as dsa
+        print(json.dumps(time_prefill_chain(dsa, _peaks()[0], iters=max(1, min(args.steps, 10)))),
+              flush=True)
         return
     wl = workloads.WORKLOADS[args.workload]
     if wl.mode != "decode":
