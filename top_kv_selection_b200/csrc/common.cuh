@@ -112,10 +112,12 @@ dsa_status launch_index_scores(const uint8_t *q_fp8, const float *q_scale, const
 
 // Decode step: rotate + quantise the new queries and key inside the scorer,
 // append the key at T-1, score positions 0..T-1 of each sequence.  With
-// row_hist ([B][kHistBins], zeroed before the launch), the scorer also counts
-// its scores by the top 12 bits of their key into the row's histogram, for
-// the decode top-k (see topk.cu).
+// row_hist ([B][decode_hist_chunks()][kHistBins]), each of the scorer's CTAs
+// also counts its scores by the top 12 bits of their key and writes that
+// histogram, every bin, into its own slot, for the decode top-k (topk.cu),
+// which sums a row's slots; nothing needs zeroing first.
 constexpr int kHistBins = 4096;
+int decode_hist_chunks(int B, int H, int D, int64_t T);
 dsa_status launch_decode_scores(const float *q_raw, const float *w, const float *k_new,
                                 uint8_t *k_cache, float *k_scale, int64_t t_max, int B, int H,
                                 int D, int64_t T, float softmax_scale, float *scores,
@@ -125,14 +127,15 @@ size_t topk_workspace_bytes(int B, int S, int64_t T, int k);
 // prefetch_rows: optional cache whose rows at the selected positions are
 // requested into L2 as they are selected (row (b, t) at prefetch_rows +
 // (b * prefetch_t_max + t) * prefetch_row_bytes; bytes a multiple of 16).
-// row_hist: the decode step's top-k (S = 1, start_pos = T - 1, T up to
-// 262144) takes the per-row histograms of the scores' top 12 key bits made by
-// the decode scorer and runs one cluster per row that reads the scores once;
-// without them the general cluster kernel runs.
+// row_hist / hist_chunks: the decode step's top-k (S = 1, start_pos = T - 1,
+// T up to 262144) takes the decode scorer's per-CTA histograms of the scores'
+// top 12 key bits ([B][hist_chunks][kHistBins]) and runs one cluster per row
+// that reads the scores once; without them the general cluster kernel runs.
 dsa_status launch_topk_select(const float *scores, int B, int S, int64_t T, int64_t start_pos,
                               int k, int32_t *idx, void *ws, cudaStream_t stream,
                               const void *prefetch_rows = nullptr, int64_t prefetch_t_max = 0,
-                              int prefetch_row_bytes = 0, const uint32_t *row_hist = nullptr);
+                              int prefetch_row_bytes = 0, const uint32_t *row_hist = nullptr,
+                              int hist_chunks = 0);
 
 size_t sparse_mla_workspace_bytes(int B, int S, int Hq, int dc, int dr, int k, dsa_dtype dt);
 bool sparse_mla_tc_supported(int Hq, int dc, int dr, int k, dsa_dtype dt);

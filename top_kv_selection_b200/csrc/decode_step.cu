@@ -14,13 +14,13 @@ namespace {
 
 struct DecodeWs {
     float *scores;     // [B,T]
-    uint32_t *hist;    // [B][kHistBins]: the scores counted by their top 12 key bits
+    uint32_t *hist;    // [B][chunks][kHistBins]: each scorer CTA's scores counted by their
+                       //   top 12 key bits
+    int hist_chunks;
     void *attn_ws;
     size_t total;
 };
 
-// kHistBins bin counts per row
-size_t hist_bytes(int B) { return (size_t)B * kHistBins * sizeof(uint32_t); }
 
 DecodeWs carve(void *base, int B, int H, int D, int64_t T, int index_topk, int Hq, int dc, int dr,
                dsa_dtype dt) {
@@ -33,8 +33,10 @@ DecodeWs carve(void *base, int B, int H, int D, int64_t T, int index_topk, int H
         return r;
     };
     w.scores = reinterpret_cast<float *>(take((size_t)B * T * sizeof(float)));
-    // the histograms: the part that starts each step at zero
-    w.hist = reinterpret_cast<uint32_t *>(take(hist_bytes(B)));
+    // the scorer CTAs' histograms (each slot fully written every step)
+    w.hist_chunks = decode_hist_chunks(B, H, D, T);
+    w.hist = reinterpret_cast<uint32_t *>(
+        take((size_t)B * w.hist_chunks * kHistBins * sizeof(uint32_t)));
     const int K = (int64_t)index_topk < T ? index_topk : (int)T;
     w.attn_ws = take(dt == DSA_FP8_LATENT ? sparse_mla_fp8_workspace_bytes(B, 1, Hq, dc, dr, K)
                                           : sparse_mla_workspace_bytes(B, 1, Hq, dc, dr, K, dt));
@@ -78,8 +80,6 @@ extern "C" dsa_status dsa_decode_step(const float *q_idx, const float *w, const 
         return DSA_ERR_WORKSPACE;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     dsa_status st;
-    // the histograms start at zero
-    if (cudaMemsetAsync(ws.hist, 0, dsa::hist_bytes(B), s) != cudaSuccess) return DSA_ERR_CUDA;
     if ((st = dsa::launch_decode_scores(q_idx, w, k_new, k_cache, k_scale, t_max, B, H, D, T,
                                         softmax_scale, ws.scores, s, ws.hist)) != DSA_OK)
         return st;
@@ -88,7 +88,7 @@ extern "C" dsa_status dsa_decode_step(const float *q_idx, const float *w, const 
                                                : (dc + dr) * (dt == DSA_BF16 ? 2 : 4);
     if ((st = dsa::launch_topk_select(ws.scores, B, 1, T, T - 1, index_topk, idx, nullptr, s,
                                       row_bytes % 16 == 0 ? kv_cache : nullptr, t_max, row_bytes,
-                                      ws.hist)) != DSA_OK)
+                                      ws.hist, ws.hist_chunks)) != DSA_OK)
         return st;
     const int K = (int64_t)index_topk < T ? index_topk : (int)T;
     if (dt == DSA_FP8_LATENT)

@@ -52,8 +52,9 @@ struct ScoreArgs {
     const float *w;
     const float *k_scale;
     float *scores;
-    uint32_t *row_hist;        // decode: per row, the histogram of the scores' 12-bit key
-                               //   bins (zeroed before the launch), or null
+    uint32_t *row_hist;        // decode: per (row, chunk) CTA, the histogram of its scores'
+                               //   12-bit key bins ([rows][chunks][kHistBins], every bin
+                               //   written), or null
     int64_t t_max;
     int64_t start_pos;
     int64_t T;
@@ -207,7 +208,13 @@ score_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const ScoreArgs a) {
     for (int64_t t = n_vis + (int64_t)chunk * kThreads + threadIdx.x; t < a.T;
          t += (int64_t)a.chunks * kThreads)
         a.scores[row * a.T + t] = -INFINITY;
-    if (n_my <= 0) return;
+    if (n_my <= 0) {
+        // no tiles: an empty histogram for this CTA's slot
+        if (kRaw && a.row_hist)
+            for (int i = threadIdx.x; i < kHistBins; i += kThreads)
+                a.row_hist[(row * a.chunks + chunk) * kHistBins + i] = 0u;
+        return;
+    }
 
     // epilogue warps: issue the query, weight, first key-scale and new-key
     // loads before the key stream starts
@@ -365,13 +372,11 @@ score_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const ScoreArgs a) {
             }
         }
         if (hist) {
-            // this CTA's nonzero bins into the row's histogram
+            // this CTA's histogram, every bin, into its own slot (nothing has
+            // to be zeroed before the launch; the top-k sums a row's slots)
             asm volatile("bar.sync 2, 128;" ::: "memory");
-            uint32_t *rh = a.row_hist + row * kHistBins;
-            for (int i = threadIdx.x - 64; i < kHistBins; i += 128) {
-                const uint32_t c = s_hist[i];
-                if (c) atomicAdd(rh + i, c);
-            }
+            uint32_t *rh = a.row_hist + (row * a.chunks + chunk) * kHistBins;
+            for (int i = threadIdx.x - 64; i < kHistBins; i += 128) rh[i] = s_hist[i];
         }
     }
 
@@ -455,6 +460,12 @@ dsa_status launch_index_scores(const uint8_t *q_fp8, const float *q_scale, const
                                      start_pos, T, softmax_scale, scores, stream);
     return D == 128 ? launch_tc<128, false>(a, k_cache, B, S, start_pos, T, stream)
                     : launch_tc<64, false>(a, k_cache, B, S, start_pos, T, stream);
+}
+
+int decode_hist_chunks(int B, int H, int D, int64_t T) {
+    if (B <= 0 || T <= 0) return 0;
+    const int NH = (H + 15) / 16 * 16;
+    return D == 128 ? score_chunks<128, true>(B, NH, T) : score_chunks<64, true>(B, NH, T);
 }
 
 dsa_status launch_decode_scores(const float *q_raw, const float *w, const float *k_new,

@@ -475,11 +475,13 @@ topk_cluster_kernel(const float *scores, int S, int64_t T, int64_t start_pos, in
 }
 
 // ------------------------------------------------------------ decode top-k
-// The decode step's top-k, when the scorer has counted the row's scores by
-// their top 12 key bits: a cluster of CN CTAs of 512 threads per row, each
-// thread holding 32 consecutive positions' keys in registers.  Every CTA reads
-// the row's histogram and finds the same 12-bit threshold bin on its own, so
-// the scores are read once and no histogram is merged.  Each CTA reserves a
+// The decode step's top-k, when the scorer's CTAs have counted their scores
+// by the top 12 key bits: a cluster of CN CTAs of 512 threads per row, each
+// thread holding 32 consecutive positions' keys in registers.  CTA p sums its
+// slice of the bins over the row's scorer histograms and stores the sums into
+// every CTA of the cluster, so that after one cluster barrier every CTA holds
+// the row's histogram and finds the same 12-bit threshold bin on its own; the
+// scores are read once.  Each CTA reserves a
 // range of CTA 0's candidate list with one atomic and stores the keys of its
 // span that fall in the bin there, with their positions (distributed shared
 // memory); CTA 0 finds tau among them (a 10-bit histogram pass, then one warp
@@ -499,6 +501,7 @@ constexpr int kDecFew = 32;                         // keys one warp ranks direc
 
 struct DecShared {
     unsigned hist[kBins];             // CTA 0: histogram of the current pass or round
+    unsigned rowhist[kBins];          // the row's histogram, a slice from each CTA
     uint2 cand[kDecCap];              // CTA 0: gathered (key, position), CTA by CTA
     int n_cand;                       // CTA 0: slots reserved
     int base[kMaxCluster];            // CTA 0: per CTA, its first slot
@@ -590,7 +593,7 @@ __device__ __forceinline__ int2 block_scan2_dec(int a, int b, DecShared &sh, int
 
 __global__ void __launch_bounds__(kDecThreads, 1)
 topk_decode_kernel(const float *scores, int64_t T, int K, int32_t *__restrict__ idx,
-                   const RowPrefetch pf, const uint32_t *row_hist) {
+                   const RowPrefetch pf, const uint32_t *row_hist, int hist_chunks) {
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     cg::cluster_group cl = cg::this_cluster();
     const int CN = (int)cl.num_blocks();
@@ -621,14 +624,33 @@ topk_decode_kernel(const float *scores, int64_t T, int K, int32_t *__restrict__ 
     // the scores and the histogram come from the scorer
     asm volatile("griddepcontrol.wait;" ::: "memory");
 
-    // this thread's 8 bins of the row's histogram (4088 - 8t .. 4095 - 8t)
-    // and its 32 positions, loaded together
-    unsigned hc[8];
+    // this CTA's slice of the bins, summed over the row's scorer histograms
+    // (thread t: bins b0 + t, b0 + t + 512, ...), and this thread's 32
+    // positions, loaded together
+    const int bpc = (kBins + CN - 1) / CN;           // bins per CTA
+    const int b_lo = p * bpc, b_hi = b_lo + bpc < kBins ? b_lo + bpc : kBins;
+    constexpr int kMaxSlice = kBins / kDecThreads;   // bins a thread sums (CN = 1)
+    unsigned bsum[kMaxSlice];
     {
-        const uint4 *h4 = reinterpret_cast<const uint4 *>(row_hist + row * kBins + kBins - 8 * (tid + 1));
-        const uint4 x0 = h4[0], x1 = h4[1];
-        hc[0] = x1.w; hc[1] = x1.z; hc[2] = x1.y; hc[3] = x1.x;
-        hc[4] = x0.w; hc[5] = x0.z; hc[6] = x0.y; hc[7] = x0.x;
+        // up to kSumBatch histograms' loads in flight at once per bin
+        constexpr int kSumBatch = 40;
+        const uint32_t *rh = row_hist + row * hist_chunks * kBins;
+#pragma unroll 1
+        for (int u = 0; u < kMaxSlice; u++) {
+            const int bb = b_lo + tid + u * kDecThreads;
+            unsigned acc = 0;
+            if (bb < b_hi) {
+                for (int c0 = 0; c0 < hist_chunks; c0 += kSumBatch) {
+                    unsigned v[kSumBatch];
+#pragma unroll
+                    for (int c = 0; c < kSumBatch; c++)
+                        v[c] = c0 + c < hist_chunks ? __ldg(rh + (c0 + c) * kBins + bb) : 0u;
+#pragma unroll
+                    for (int c = 0; c < kSumBatch; c++) acc += v[c];
+                }
+            }
+            bsum[u] = acc;
+        }
     }
     const int64_t t0 = (int64_t)p * kDecSpan + (int64_t)tid * kDecPer;
     const float *src = scores + row * T + t0;
@@ -648,12 +670,31 @@ topk_decode_kernel(const float *scores, int64_t T, int K, int32_t *__restrict__ 
     }
     const int nv = T - t0 <= 0 ? 0 : (T - t0 >= kDecPer ? kDecPer : (int)(T - t0));
 
+    // every CTA has started (and CTA 0 has cleared its merge state): store the
+    // slice's sums into every CTA's copy of the row histogram, then meet again
+    asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
+    for (int r = 0; r < CN; r++) {
+        unsigned *peer = cl.map_shared_rank(sh.rowhist, r);
+#pragma unroll
+        for (int u = 0; u < kMaxSlice; u++) {
+            const int bb = b_lo + tid + u * kDecThreads;
+            if (bb < b_hi) peer[bb] = bsum[u];
+        }
+    }
+    cl.sync();
+    // this thread's 8 bins of the row's histogram (4088 - 8t .. 4095 - 8t)
+    unsigned hc[8];
+    {
+        const uint4 *h4 = reinterpret_cast<const uint4 *>(sh.rowhist + kBins - 8 * (tid + 1));
+        const uint4 x0 = h4[0], x1 = h4[1];
+        hc[0] = x1.w; hc[1] = x1.z; hc[2] = x1.y; hc[3] = x1.x;
+        hc[4] = x0.w; hc[5] = x0.z; hc[6] = x0.y; hc[7] = x0.x;
+    }
     unsigned bin, above, n_group;
     find_rank_regs<8>(hc, kBins - 8 * tid - 1, (unsigned)m, &bin, &above, &n_group, sh);
     uint32_t prefix = bin;
     int pbits = kBits;
     unsigned rank = (unsigned)m - above;           // rank of tau within the group
-    asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
 
     // too many keys to gather (rare: scores within a few percent of each
     // other, or many exact ties): 12-bit rounds over the register keys,
@@ -969,7 +1010,7 @@ size_t topk_workspace_bytes(int, int, int64_t, int) { return 0; }
 dsa_status launch_topk_select(const float *scores, int B, int S, int64_t T, int64_t start_pos,
                               int k, int32_t *idx, void *, cudaStream_t stream,
                               const void *prefetch_rows, int64_t prefetch_t_max,
-                              int prefetch_row_bytes, const uint32_t *row_hist) {
+                              int prefetch_row_bytes, const uint32_t *row_hist, int hist_chunks) {
     if ((int64_t)B * S * T == 0) return DSA_OK;
     const int K = (int64_t)k < T ? k : (int)T;
     const int64_t rows = (int64_t)B * S;
@@ -978,7 +1019,8 @@ dsa_status launch_topk_select(const float *scores, int B, int S, int64_t T, int6
     pf.base = static_cast<const uint8_t *>(prefetch_rows);
     pf.t_max = prefetch_t_max;
     pf.bytes = prefetch_row_bytes;
-    if (row_hist && S == 1 && start_pos == T - 1 && (T + kDecSpan - 1) / kDecSpan <= kMaxCluster) {
+    if (row_hist && hist_chunks > 0 && S == 1 && start_pos == T - 1 &&
+        (T + kDecSpan - 1) / kDecSpan <= kMaxCluster) {
         // the decode top-k: one cluster per row, the threshold bin from the scorer's histogram
         const int dcn = (int)((T + kDecSpan - 1) / kDecSpan);
         const int dsmem = (int)sizeof(DecShared);
@@ -1003,7 +1045,8 @@ dsa_status launch_topk_select(const float *scores, int B, int S, int64_t T, int6
         attr[1].val.programmaticStreamSerializationAllowed = 1;
         cfg.attrs = attr;
         cfg.numAttrs = 2;
-        if (cudaLaunchKernelEx(&cfg, topk_decode_kernel, scores, T, K, idx, pf, row_hist) != cudaSuccess)
+        if (cudaLaunchKernelEx(&cfg, topk_decode_kernel, scores, T, K, idx, pf, row_hist,
+                               hist_chunks) != cudaSuccess)
             return DSA_ERR_CUDA;
         return launch_status();
     }
