@@ -205,10 +205,14 @@ score_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const ScoreArgs a) {
     // waits for this grid before reading the scores
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     // causally masked positions of this row (prefill only), shared by the chunks
-    for (int64_t t = n_vis + (int64_t)chunk * kThreads + threadIdx.x; t < a.T;
-         t += (int64_t)a.chunks * kThreads)
-        a.scores[row * a.T + t] = -INFINITY;
+    auto write_masked = [&]() {
+        for (int64_t t = n_vis + (int64_t)chunk * kThreads + threadIdx.x; t < a.T;
+             t += (int64_t)a.chunks * kThreads)
+            a.scores[row * a.T + t] = -INFINITY;
+    };
     if (n_my <= 0) {
+        asm volatile("griddepcontrol.wait;" ::: "memory");
+        write_masked();
         // no tiles: an empty histogram for this CTA's slot
         if (kRaw && a.row_hist)
             for (int i = threadIdx.x; i < kHistBins; i += kThreads)
@@ -216,8 +220,6 @@ score_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const ScoreArgs a) {
         return;
     }
 
-    // epilogue warps: issue the query, weight, first key-scale and new-key
-    // loads before the key stream starts
     using Prefetch = QueryPrefetch<D, kRaw>;
     Prefetch pf;
     float kr[D / 32];
@@ -233,13 +235,6 @@ score_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const ScoreArgs a) {
     // so the key's scale passes between lanes of one warp
     const bool appender = append && warp >= 2 && (warp & 3) == (int)(((a.T - 1) % kTile) >> 5);
     float ks0 = 0.f, ks1 = 0.f, ks2 = 0.f;
-    if (warp >= 2) {
-        pf.load(a, row, 0);
-        if (appender) load_lane_slice<D, float>(a.k_new + b * D, kr);
-        ks0 = load_ks(0);     // the new key's entry is reloaded once it is appended
-        ks1 = load_ks(1);
-        ks2 = load_ks(2);
-    }
 
     if (threadIdx.x == 0) {
         for (int i = 0; i < NS; i++) {
@@ -256,20 +251,51 @@ score_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const ScoreArgs a) {
         tc::fence_mbar_init();
         tc::tma_prefetch_desc(&tmap_k);
     }
+    __syncthreads();        // the barriers are initialised
+    // The accumulators: warp 1 allocates them while the epilogue warps build
+    // the query operand; the two meet at named barrier 3 (warps 1..5) before
+    // either touches TMEM.  Allocation is the last thing done before the wait
+    // below, so with a programmatic launch it overlaps the preceding kernel.
     if (warp == 1) {
         tc::tmem_alloc(tmem_holder, a.tmem_cols);
         tc::tmem_relinquish();
     }
-    tc::tc_fence_before();
-    __syncthreads();
-    tc::tc_fence_after();
-    const uint32_t tmem_base = *tmem_holder;
+    // Everything below reads the step's inputs (queries, weights, the key
+    // cache) or writes its outputs: wait for the preceding kernel (a no-op
+    // without a programmatic launch).
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    write_masked();
+    // epilogue warps: issue the query, weight, first key-scale and new-key
+    // loads before the key stream starts
+    if (warp >= 2) {
+        pf.load(a, row, 0);
+        if (appender) load_lane_slice<D, float>(a.k_new + b * D, kr);
+        ks0 = load_ks(0);     // the new key's entry is reloaded once it is appended
+        ks1 = load_ks(1);
+        ks2 = load_ks(2);
+    }
+    // the first ring of key tiles (the tile holding the appended key waits
+    // for it in the loop below)
+    const int early = n_my - (append ? 1 : 0) < NS ? n_my - (append ? 1 : 0) : NS;
+    const uint64_t pol = tc::l2_evict_first_policy();
+    if (threadIdx.x == 0)
+        for (int i = 0; i < early; i++) {
+            tc::mbar_arrive_expect_tx(&full[i], kTile * D);
+            tc::tma_load_3d(sk + i * kTile * D, &tmap_k, 0, (int)((tile_lo + i) * kTile), (int)b,
+                            &full[i], pol);
+        }
+    uint32_t tmem_base = 0;
+    if (warp == 1) {
+        tc::tc_fence_before();
+        asm volatile("bar.sync 3, 160;" ::: "memory");
+        tc::tc_fence_after();
+        tmem_base = *tmem_holder;
+    }
 
     if (warp == 0) {
         if (lane == 0) {
-            const uint64_t pol = tc::l2_evict_first_policy();
-            int issued = 0;
-            for (int i = 0; i < n_my; i++) {
+            int issued = early;
+            for (int i = early; i < n_my; i++) {
                 const int st = i % NS;
                 const uint32_t ph = (uint32_t)(i / NS) & 1u;
                 if (!tc::mbar_wait(&empty[st], ph ^ 1u, a.err, abort)) break;
@@ -330,6 +356,10 @@ score_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const ScoreArgs a) {
             for (int i = threadIdx.x - 64; i < kHistBins; i += 128) s_hist[i] = 0;
             asm volatile("bar.sync 2, 128;" ::: "memory");
         }
+        // the accumulators' TMEM address, from warp 1
+        asm volatile("bar.sync 3, 160;" ::: "memory");
+        tc::tc_fence_after();
+        tmem_base = *tmem_holder;
         for (int i = 0; i < n_my; i++) {
             const int ac = i % kAcc;
             const int64_t t = (tile_lo + i) * kTile + tok;
@@ -435,7 +465,19 @@ dsa_status launch_tc(ScoreArgs a, const uint8_t *k_cache, int B, int S, int64_t 
     if (cudaFuncSetAttribute(score_tc_kernel<D, kRaw>,
                              cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
         return DSA_ERR_CUDA;
-    score_tc_kernel<D, kRaw><<<(unsigned)(rows * chunks), kThreads, smem, stream>>>(tmap, a);
+    // programmatic launch: the CTAs' set-up (barriers, TMEM) overlaps the
+    // preceding kernel's tail; the kernel waits for it before touching memory
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)(rows * chunks));
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (cudaLaunchKernelEx(&cfg, score_tc_kernel<D, kRaw>, tmap, a) != cudaSuccess) return DSA_ERR_CUDA;
     return launch_status();
 }
 

@@ -24,10 +24,11 @@
 //      MN-major), into all 512 TMEM columns;
 //   4. writes bf16 out (+ lse) when the row has one unit, else a normalised
 //      fp16 partial with its (max, sum, power-of-two ranges).  The partials of
-//      a row's units ("splits") are merged: when the whole grid fits on the
-//      GPU at once it is launched as a cooperative grid, and after a grid-wide
-//      barrier every CTA merges its own slice of the output columns;
-//      otherwise a combine kernel merges.
+//      a row's units ("splits") are merged by a combine kernel launched right
+//      behind (programmatic launch: its CTAs are resident, waiting, while the
+//      attention finishes).  The attention itself is a plain programmatic
+//      launch too, so its CTAs start their set-up (barriers, TMEM, the query's
+//      TMA) on the SMs the top-k leaves free.
 //
 // Shared memory: nine chunk regions R0..R8 (R k holds chunk k), the query's
 // rotary block, and P (two 16 KB K-major blocks).  The query's latent blocks
@@ -42,7 +43,6 @@
 // region and decoded in place (code * block scale, rounded to bf16 -- the same
 // decoded operand as the oracle's), so the rows cross HBM once at 656 bytes
 // and no decoded copy is ever written to memory.
-#include <cooperative_groups.h>
 #include <cuda_fp16.h>
 #include <cuda_fp8.h>
 
@@ -91,7 +91,6 @@ struct MlaArgs {
     int64_t start_pos;
     int64_t row0;              // first query row of this launch
     int S, k, splits;
-    int coop;                  // cooperative grid: the splits are merged in this kernel
     float scale_log2;          // sm_scale * log2(e)
     int *err;
 };
@@ -664,32 +663,11 @@ sparse_mla_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const MlaArgs a) 
         tc::tc_fence_after();
         tc::tmem_dealloc(tmem, kTmemCols);
     }
-    if (a.coop) {
-        // every split of every row has written its partial: merge this
-        // split's slice of its row's output columns (64 / splits octets of
-        // eight columns)
-        cooperative_groups::this_grid().sync();
-        const int npo = kOct / a.splits;
-        const int h = threadIdx.x & (kHq - 1), o = threadIdx.x >> 7;
-        const int64_t blk0 = (int64_t)blockIdx.x - sp;
-        if (threadIdx.x < kWork) {
-            // thread (h, o): octets o, o + 2, ... of the slice, two at a time
-            int oc = o;
-            for (; oc + 2 < npo; oc += 4) {
-                const int c8[2] = {npo * sp + oc, npo * sp + oc + 2};
-                merge_octets<2>(a.part_o, a.part_ml, a.splits, blk0, row, c8, h, a.out, a.lse);
-            }
-            if (oc < npo) {
-                const int c8[1] = {npo * sp + oc};
-                merge_octets<1>(a.part_o, a.part_ml, a.splits, blk0, row, c8, h, a.out, a.lse);
-            }
-        }
-    }
 }
 
-// Merges the splits of each query row when the attention grid is not
-// cooperative: thread (head, octet) merges eight output columns of one head,
-// consecutive threads consecutive heads (coalesced reads of the partials).
+// Merges the splits of each query row: thread (head, octet) merges eight
+// output columns of one head, consecutive threads consecutive heads
+// (coalesced reads of the partials).
 __global__ void __launch_bounds__(kHq)
 sparse_mla_combine_kernel(const __half *part_o, const float4 *part_ml, int splits, int64_t row0,
                           __nv_bfloat16 *__restrict__ out, float *__restrict__ lse) {
@@ -762,17 +740,6 @@ dsa_status launch(const void *q, const void *kv, int64_t t_max, const int32_t *i
     if (cudaFuncSetAttribute(sparse_mla_tc_kernel<kFp8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)kSmemBytes) != cudaSuccess)
         return DSA_ERR_CUDA;
-    // The splits are merged inside the attention grid when the grid can be
-    // cooperative (all of its CTAs resident at once, one launch) and each
-    // split gets whole octets of columns; else a combine kernel follows.
-    bool coop = false;
-    if (a.splits > 1 && kOct % a.splits == 0 && chunk == rows) {
-        int per_sm = 0;
-        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, sparse_mla_tc_kernel<kFp8>,
-                                                          kThreads, kSmemBytes) == cudaSuccess &&
-            (int64_t)per_sm * num_sms() >= rows * a.splits)
-            coop = true;
-    }
     for (int64_t r0 = 0; r0 < rows; r0 += chunk) {
         const int64_t n = rows - r0 < chunk ? rows - r0 : chunk;
         a.row0 = r0;
@@ -783,33 +750,16 @@ dsa_status launch(const void *q, const void *kv, int64_t t_max, const int32_t *i
         cfg.stream = stream;
         // programmatic launch: the kernel's set-up overlaps the preceding
         // kernel's tail; it waits for that kernel before reading the selections
-        cudaLaunchAttribute attr[2];
+        cudaLaunchAttribute attr[1];
         attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
         attr[0].val.programmaticStreamSerializationAllowed = 1;
-        attr[1].id = cudaLaunchAttributeCooperative;
-        attr[1].val.cooperative = 1;
         cfg.attrs = attr;
-        bool launched = false;
-        if (coop) {
-            // cooperative, first with the programmatic launch, then without it
-            a.coop = 1;
-            for (int first = 0; first < 2 && !launched; first++) {
-                cfg.attrs = attr + first;
-                cfg.numAttrs = 2 - first;
-                launched = cudaLaunchKernelEx(&cfg, sparse_mla_tc_kernel<kFp8>, tm_q, a) == cudaSuccess;
-                if (!launched) (void)cudaGetLastError();
-            }
-        }
-        if (!launched) {
-            a.coop = 0;
-            cfg.attrs = attr;
-            cfg.numAttrs = 1;
-            if (cudaLaunchKernelEx(&cfg, sparse_mla_tc_kernel<kFp8>, tm_q, a) != cudaSuccess)
-                return DSA_ERR_CUDA;
-        }
+        cfg.numAttrs = 1;
+        if (cudaLaunchKernelEx(&cfg, sparse_mla_tc_kernel<kFp8>, tm_q, a) != cudaSuccess)
+            return DSA_ERR_CUDA;
         dsa_status st = launch_status();
         if (st != DSA_OK) return st;
-        if (a.splits == 1 || a.coop) continue;
+        if (a.splits == 1) continue;
         cudaLaunchConfig_t ccfg = {};
         ccfg.gridDim = dim3((unsigned)(n * kOct));
         ccfg.blockDim = dim3(kHq);
