@@ -467,42 +467,96 @@ def run_ours(args, wl, world, rank, local):
         print(json.dumps(line), flush=True)
 
 
-def run_e2e(dsa, wl, copies, args, world):
-    """Same step through the public API with host buffers: the step's inputs are
-    copied from pinned host memory and the result read back, inside the timed region."""
-    B = wl.B
+def run_e2e(dsa, wl, copies, args, world, graph_steps=12):
+    """Same step through the public API with host buffers.  Every step's inputs
+    are copied from pinned host memory and its selections and output read back
+    into pinned host memory, inside the timed region; as a serving loop would,
+    the copies run on their own streams (host-to-device, device-to-host) and
+    overlap the neighbouring steps' kernels.  Events order each device state's
+    reuse: the inputs of step i are written once step i - n (same state) has
+    read them, and step i's kernels start once step i - n's results have been
+    read back.  `graph_steps` steps (copies, calls and events) are captured in
+    a CUDA graph and replayed, as a decode server replays its step graph; if
+    the capture fails the same loop runs eagerly."""
+    n = len(copies)
     st = copies[0]
     host_in = {k: st[k].cpu().pin_memory() for k in ("q_idx", "w", "k_new", "q_mla")}
-    new_row = st["kv"][:, wl.T - 1].cpu().pin_memory()
-    host_idx = torch.empty(st["idx"].shape, dtype=torch.int32).pin_memory()
-    host_out = torch.empty(st["out"].shape, dtype=st["out"].dtype).pin_memory()
+    new_row = st["kv"][:, wl.T - 1].contiguous().cpu().pin_memory()
+    host_idx = [torch.empty(st["idx"].shape, dtype=torch.int32).pin_memory() for _ in range(n)]
+    host_out = [torch.empty(st["out"].shape, dtype=st["out"].dtype).pin_memory() for _ in range(n)]
+    row_dev = [torch.empty_like(new_row, device="cuda") for _ in range(n)]
     h2d = sum(t.numel() * t.element_size() for t in host_in.values()) + \
         new_row.numel() * new_row.element_size()
-    d2h = host_idx.numel() * 4 + host_out.numel() * host_out.element_size()
-    stream = torch.cuda.current_stream()
+    d2h = host_idx[0].numel() * 4 + host_out[0].numel() * host_out[0].element_size()
+    up, down = torch.cuda.Stream(), torch.cuda.Stream()
 
-    def one(i):
-        s = copies[i % len(copies)]
-        for k, t in host_in.items():
-            s[k].copy_(t, non_blocking=True)
-        s["kv"][:, wl.T - 1].copy_(new_row, non_blocking=True)
-        decode_step(dsa, wl, s)
-        host_idx.copy_(s["idx"], non_blocking=True)
-        host_out.copy_(s["out"], non_blocking=True)
+    def steps(count):
+        compute = torch.cuda.current_stream()
+        up.wait_stream(compute)
+        down.wait_stream(compute)
+        in_read, out_read = [None] * n, [None] * n
+        for i in range(count):
+            j = i % n
+            s = copies[j]
+            with torch.cuda.stream(up):
+                if in_read[j] is not None:
+                    up.wait_event(in_read[j])
+                for k, t in host_in.items():
+                    s[k].copy_(t, non_blocking=True)
+                row_dev[j].copy_(new_row, non_blocking=True)
+                s["kv"][:, wl.T - 1].copy_(row_dev[j])
+                inputs = torch.cuda.Event()
+                inputs.record(up)
+            compute.wait_event(inputs)
+            if out_read[j] is not None:
+                compute.wait_event(out_read[j])
+            decode_step(dsa, wl, s, stream=compute)
+            done = torch.cuda.Event()
+            done.record(compute)
+            in_read[j] = done
+            with torch.cuda.stream(down):
+                down.wait_event(done)
+                host_idx[j].copy_(s["idx"], non_blocking=True)
+                host_out[j].copy_(s["out"], non_blocking=True)
+                back = torch.cuda.Event()
+                back.record(down)
+            out_read[j] = back
+        compute.wait_stream(up)
+        compute.wait_stream(down)
 
-    for i in range(max(args.warmup, 1)):
-        one(i)
+    steps(max(args.warmup, n))
     torch.cuda.synchronize()
+    graph = None
+    try:
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            steps(graph_steps)
+        torch.cuda.synchronize()
+        g.replay()
+        torch.cuda.synchronize()
+        if dsa.dsa_get_device_error() == 0:
+            graph = g
+    except Exception:                           # the eager loop below instead
+        torch.cuda.synchronize()
+    reps = max(1, -(-args.steps // graph_steps)) if graph is not None else 0
+    n_steps = reps * graph_steps if graph is not None else args.steps
+    stream = torch.cuda.current_stream()
     _barrier(world)
     t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     t0.record(stream)
-    for i in range(args.steps):
-        one(i)
+    if graph is not None:
+        for _ in range(reps):
+            graph.replay()
+    else:
+        steps(n_steps)
     t1.record(stream)
     t1.synchronize()
     el = _max_over_ranks(world, t0.elapsed_time(t1) * 1e-3)
-    return {"value": world * args.steps / el, "unit": "steps/s", "h2d_bytes_per_step": h2d,
-            "d2h_bytes_per_step": d2h}
+    return {"value": world * n_steps / el, "unit": "steps/s", "h2d_bytes_per_step": h2d,
+            "d2h_bytes_per_step": d2h, "steps": n_steps,
+            "how": (f"CUDA graph of {graph_steps} steps replayed {reps} times" if graph is not None
+                    else "eager loop (graph capture failed)") +
+                   "; copies on their own streams, overlapping the neighbouring steps' kernels"}
 
 
 def time_prefill_scoring(dsa, fp8_peak, iters=10):
