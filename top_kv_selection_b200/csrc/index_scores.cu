@@ -266,7 +266,9 @@ score_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const ScoreArgs a) {
     asm volatile("griddepcontrol.wait;" ::: "memory");
     write_masked();
     // epilogue warps: issue the query, weight, first key-scale and new-key
-    // loads before the key stream starts
+    // loads before the key stream starts (named barrier 4, warps 0 and 2..5:
+    // the first ring of key tiles is issued only after them, so that the
+    // query's loads are not queued behind every CTA's ring in HBM)
     if (warp >= 2) {
         pf.load(a, row, 0);
         if (appender) load_lane_slice<D, float>(a.k_new + b * D, kr);
@@ -274,6 +276,7 @@ score_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const ScoreArgs a) {
         ks1 = load_ks(1);
         ks2 = load_ks(2);
     }
+    if (warp != 1) asm volatile("bar.sync 4, 160;" ::: "memory");
     // the first ring of key tiles (the tile holding the appended key waits
     // for it in the loop below)
     const int early = n_my - (append ? 1 : 0) < NS ? n_my - (append ? 1 : 0) : NS;

@@ -612,6 +612,10 @@ topk_decode_kernel(const float *scores, int64_t T, int K, int32_t *__restrict__ 
     }
     extern __shared__ __align__(16) uint8_t dec_smem[];
     DecShared &sh = *reinterpret_cast<DecShared *>(dec_smem);
+    // this CTA's keys, [j][thread]: the per-key loops below read them from here
+    // and stay rolled (one pass per CTA, so unrolled code would be fetched
+    // cold on every SM)
+    uint32_t *skey = reinterpret_cast<uint32_t *>(dec_smem + sizeof(DecShared));
     DecShared *sh0 = cl.map_shared_rank(&sh, 0);
     if (p == 0) {
         for (int i = tid; i < kBins; i += kDecThreads) sh.hist[i] = 0;
@@ -669,6 +673,9 @@ topk_decode_kernel(const float *scores, int64_t T, int K, int32_t *__restrict__ 
         for (int j = 0; j < kDecPer; j++) key[j] = t0 + j < T ? score_key(src[j]) : 0u;
     }
     const int nv = T - t0 <= 0 ? 0 : (T - t0 >= kDecPer ? kDecPer : (int)(T - t0));
+#pragma unroll
+    for (int j = 0; j < kDecPer; j++) skey[j * kDecThreads + tid] = key[j];
+    auto key_at = [&](int j) { return skey[j * kDecThreads + tid]; };
 
     // every CTA has started (and CTA 0 has cleared its merge state): store the
     // slice's sums into every CTA's copy of the row histogram, then meet again
@@ -702,10 +709,12 @@ topk_decode_kernel(const float *scores, int64_t T, int K, int32_t *__restrict__ 
     while (n_group > (unsigned)kDecCap && pbits < 32) {
         const int nb = 32 - pbits < kBits ? 32 - pbits : kBits;
         const int sh_lo = 32 - pbits - nb;
-#pragma unroll
-        for (int j = 0; j < kDecPer; j++)
-            if (j < nv && (key[j] >> (32 - pbits)) == prefix)
-                atomicAdd(&sh0->hist[(key[j] >> sh_lo) & ((1u << nb) - 1u)], 1u);
+#pragma unroll 1
+        for (int j = 0; j < nv; j++) {
+            const uint32_t kj = key_at(j);
+            if ((kj >> (32 - pbits)) == prefix)
+                atomicAdd(&sh0->hist[(kj >> sh_lo) & ((1u << nb) - 1u)], 1u);
+        }
         cl.sync();
         if (p == 0) {
             unsigned c8[8];
@@ -738,11 +747,11 @@ topk_decode_kernel(const float *scores, int64_t T, int K, int32_t *__restrict__ 
     const bool gather = n_group <= (unsigned)kDecCap && pbits < 32;
     const int gshift = 32 - pbits;
     int n_gt = 0, n_in = 0;
-#pragma unroll
-    for (int j = 0; j < kDecPer; j++) {
-        const uint32_t g = gshift == 32 ? 0u : key[j] >> gshift;
-        n_gt += j < nv && g > prefix;
-        n_in += j < nv && g == prefix;
+#pragma unroll 1
+    for (int j = 0; j < nv; j++) {
+        const uint32_t g = gshift == 32 ? 0u : key_at(j) >> gshift;
+        n_gt += g > prefix;
+        n_in += g == prefix;
     }
     int2 tot;
     const int2 ex = block_scan2_dec(n_gt, n_in, sh, &tot);
@@ -759,12 +768,14 @@ topk_decode_kernel(const float *scores, int64_t T, int K, int32_t *__restrict__ 
         __syncthreads();
         if (n_in) {
             int slot = sh.my_base + ex.y;
-#pragma unroll
-            for (int j = 0; j < kDecPer; j++)
-                if (j < nv && (key[j] >> gshift) == prefix) {
-                    if (slot < kDecCap) sh0->cand[slot] = make_uint2(key[j], (uint32_t)(t0 + j));
+#pragma unroll 1
+            for (int j = 0; j < nv; j++) {
+                const uint32_t kj = key_at(j);
+                if ((kj >> gshift) == prefix) {
+                    if (slot < kDecCap) sh0->cand[slot] = make_uint2(kj, (uint32_t)(t0 + j));
                     slot++;
                 }
+            }
         }
     }
     cl.sync();                                   // counts and keys in CTA 0
@@ -890,21 +901,22 @@ topk_decode_kernel(const float *scores, int64_t T, int K, int32_t *__restrict__ 
 
     // ---- ordered write of this thread's 32 positions
     int c_gt = 0, c_eq = 0;
-#pragma unroll
-    for (int j = 0; j < kDecPer; j++) {
-        c_gt += j < nv && key[j] > tau;
-        c_eq += j < nv && key[j] == tau;
+#pragma unroll 1
+    for (int j = 0; j < nv; j++) {
+        const uint32_t kj = key_at(j);
+        c_gt += kj > tau;
+        c_eq += kj == tau;
     }
     int2 tot2;
     const int2 e2 = block_scan2_dec(c_gt, c_eq, sh, &tot2);
     int take_eq = my_q - e2.y;
     take_eq = take_eq < 0 ? 0 : (take_eq > c_eq ? c_eq : take_eq);
     int pos = off + e2.x + (my_q < e2.y ? my_q : e2.y);
-#pragma unroll
-    for (int j = 0; j < kDecPer; j++) {
-        if (j >= nv) break;
-        bool sel = key[j] > tau;
-        if (key[j] == tau && take_eq > 0) {
+#pragma unroll 1
+    for (int j = 0; j < nv; j++) {
+        const uint32_t kj = key_at(j);
+        bool sel = kj > tau;
+        if (kj == tau && take_eq > 0) {
             sel = true;
             take_eq--;
         }
@@ -1023,7 +1035,7 @@ dsa_status launch_topk_select(const float *scores, int B, int S, int64_t T, int6
         (T + kDecSpan - 1) / kDecSpan <= kMaxCluster) {
         // the decode top-k: one cluster per row, the threshold bin from the scorer's histogram
         const int dcn = (int)((T + kDecSpan - 1) / kDecSpan);
-        const int dsmem = (int)sizeof(DecShared);
+        const int dsmem = (int)sizeof(DecShared) + kDecSpan * (int)sizeof(uint32_t);
         if (cudaFuncSetAttribute(topk_decode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  dsmem) != cudaSuccess ||
             (dcn > 8 && cudaFuncSetAttribute(topk_decode_kernel,
