@@ -254,6 +254,36 @@ dsa_status dsa_topk_select(const float *scores, int B, int S, int64_t T, int64_t
                            dsa_stream_t stream);
 
 /*
+ * The indexer of DeepSeek-V4's compressed sparse attention (CSA branch of
+ * "visualize_attention_masks.py (DeepSeek-V4)"): the keys are compressed
+ * entries of `compress` (m >= 1) tokens each, and entry e is causally
+ * available to the query at absolute position i = start_pos + s once all its
+ * tokens are in, i.e. e < (i + 1) / m (integer division).  The page shows only
+ * this availability rule and the -1 warm-up sentinel of the top-k; how the
+ * compressor builds an entry's key is not shown, so the entries' indexer keys
+ * are an input, in the cache layout of dsa_index_scores.  With m = 1 these two
+ * calls are dsa_index_scores and dsa_topk_select.
+ *
+ * dsa_index_scores_csa: as dsa_index_scores over T entries (k_cache / k_scale
+ * rows are entries), scores [B,S,T] fp32, entry e of query s masked (-inf)
+ * unless e < (start_pos + s + 1) / m.  (start_pos + S) / m must not exceed T.
+ *
+ * dsa_topk_select_csa: idx[b,s,:] (K = min(k, T) slots) holds the
+ * min(K, available entries) entry ids with the largest scores among the row's
+ * available entries, ties towards the lower entry, in ascending order; the
+ * other slots hold -1 (warm-up: fewer entries than k available yet).
+ * Workspace as dsa_topk_select.  Both return DSA_ERR_INVALID_ARG for m < 1.
+ */
+dsa_status dsa_index_scores_csa(const uint8_t *q_fp8, const float *q_scale, const float *w,
+                                const uint8_t *k_cache, const float *k_scale, int64_t t_max,
+                                int B, int S, int H, int D, int64_t start_pos, int64_t T,
+                                int compress, float softmax_scale, float *scores,
+                                dsa_stream_t stream);
+dsa_status dsa_topk_select_csa(const float *scores, int B, int S, int64_t T, int64_t start_pos,
+                               int compress, int k, int32_t *idx, void *workspace,
+                               size_t workspace_bytes, dsa_stream_t stream);
+
+/*
  * Sparse latent attention, MQA mode (diagram "core attention"; semantics of
  * the MLA prefill excerpt with the index mask and the causal mask):
  *   for each (b, s, head) over the selected rows c_j = kv_cache[b, idx_j, :]:

@@ -83,6 +83,13 @@ def _load():
     lib.oracle_index_scores.restype = None
     lib.oracle_topk_select.argtypes = [P, i32, i32, i64, i64, i32, P]
     lib.oracle_topk_select.restype = None
+    lib.oracle_csa_available.argtypes = [i64, i32]
+    lib.oracle_csa_available.restype = i64
+    lib.oracle_index_scores_csa.argtypes = [P, P, P, P, P, i64, i32, i32, i32, i32, i64, i64,
+                                            i32, f32, P]
+    lib.oracle_index_scores_csa.restype = None
+    lib.oracle_topk_select_csa.argtypes = [P, i32, i32, i64, i64, i32, i32, P]
+    lib.oracle_topk_select_csa.restype = None
     lib.oracle_sparse_mla.argtypes = [P, P, i64, P, i32, i32, i32, i32, i32, i32, i64, f32,
                                       P, P]
     lib.oracle_sparse_mla.restype = None
@@ -306,6 +313,42 @@ def topk_select(scores, start_pos: int, k: int) -> np.ndarray:
     K = min(k, T)
     idx = np.empty((B, S, K), dtype=np.int32)
     lib.oracle_topk_select(_p(scores), B, S, T, start_pos, k, _p(idx))
+    return idx
+
+
+def csa_available(i: int, m: int) -> int:
+    """Compressed entries (m tokens each) available to the query at position i."""
+    return int(_load().oracle_csa_available(i, m))
+
+
+def index_scores_csa(q_fp8, q_scale, w, k_cache, k_scale, start_pos: int, T: int, m: int,
+                     softmax_scale: float) -> np.ndarray:
+    """fp8_index over compressed entries with the CSA availability mask.
+    q_fp8 [B,S,H,D], k_cache [B,t_max,D] (entry keys) -> [B,S,T] over entries."""
+    lib = _load()
+    q_fp8 = _c(q_fp8, np.uint8)
+    B, S, H, D = q_fp8.shape
+    k_cache = _c(k_cache, np.uint8)
+    t_max = k_cache.shape[1]
+    q_scale = _c(q_scale, np.float32)
+    w = _c(w, np.float32)
+    k_scale = _c(k_scale, np.float32)
+    assert q_scale.shape == (B, S, H) and w.shape == (B, S, H)
+    assert k_cache.shape == (B, t_max, D) and k_scale.shape == (B, t_max) and T <= t_max
+    out = np.empty((B, S, T), dtype=np.float32)
+    lib.oracle_index_scores_csa(_p(q_fp8), _p(q_scale), _p(w), _p(k_cache), _p(k_scale), t_max,
+                                B, S, H, D, start_pos, T, m, softmax_scale, _p(out))
+    return out
+
+
+def topk_select_csa(scores, start_pos: int, m: int, k: int) -> np.ndarray:
+    """scores [B,S,T] over entries -> idx [B,S,min(k,T)] int32 entry ids, ascending, -1 padded."""
+    lib = _load()
+    scores = _c(scores, np.float32)
+    B, S, T = scores.shape
+    K = min(k, T)
+    idx = np.empty((B, S, K), dtype=np.int32)
+    lib.oracle_topk_select_csa(_p(scores), B, S, T, start_pos, m, k, _p(idx))
     return idx
 
 

@@ -20,6 +20,11 @@
  *              sizes)" diagram: I(t,s) = sum_j w_j ReLU(q_j . k_s), k = 2048,
  *              core attention in MQA mode over the selected latents, each latent
  *              row is key and value.
+ *   [V4-CSA]   "visualize_attention_masks.py (DeepSeek-V4)", CSA branch: the
+ *              indexer scores compressed entries (m tokens each, m the compress
+ *              rate); an entry is causally available to the query at position i
+ *              once its m tokens are in, i.e. entry < (i + 1) // m; the top-k
+ *              lists entry ids and pads with -1 (warm-up sentinel).
  *
  * Readings where the pages are silent (each is also listed in the design notes):
  *   - rotate_activation: orthonormal Walsh-Hadamard transform in natural
@@ -406,6 +411,26 @@ static int by_pos_asc(const void *pa, const void *pb)
 }
 
 /*
+ * One row: ranks positions 0 .. n_valid - 1 of `row` by (score desc, position
+ * asc), keeps the first min(K, n_valid), writes them in ascending position
+ * order into dst[0 .. K) and fills the remaining slots with -1.
+ */
+static void select_row(const float *row, int64_t n_valid, int K, scored_pos *buf, int32_t *dst)
+{
+    for (int64_t t = 0; t < n_valid; t++) {
+        buf[t].score = row[t];
+        buf[t].pos = t;
+    }
+    qsort(buf, (size_t)n_valid, sizeof(scored_pos), by_score_desc_pos_asc);
+    int m = (int64_t)K < n_valid ? K : (int)n_valid;
+    for (int j = 0; j < m; j++)
+        dst[j] = (int32_t)buf[j].pos;
+    qsort(dst, (size_t)m, sizeof(int32_t), by_pos_asc);
+    for (int j = m; j < K; j++)
+        dst[j] = -1;
+}
+
+/*
  * scores [B,S,T]; idx [B,S,K] with K = min(k, T).  Row (b,s) ranks the causal
  * positions t <= start_pos + s by (score desc, t asc), keeps the first
  * min(K, start_pos + s + 1), writes them in ascending position order and fills
@@ -421,18 +446,63 @@ void oracle_topk_select(const float *scores, int B, int S, int64_t T, int64_t st
         int64_t n_valid = start_pos + s + 1;
         if (n_valid > T)
             n_valid = T;
-        for (int64_t t = 0; t < n_valid; t++) {
-            buf[t].score = scores[row * T + t];
-            buf[t].pos = t;
-        }
-        qsort(buf, (size_t)n_valid, sizeof(scored_pos), by_score_desc_pos_asc);
-        int m = (int64_t)K < n_valid ? K : (int)n_valid;
-        int32_t *dst = idx + row * K;
-        for (int j = 0; j < m; j++)
-            dst[j] = (int32_t)buf[j].pos;
-        qsort(dst, (size_t)m, sizeof(int32_t), by_pos_asc);
-        for (int j = m; j < K; j++)
-            dst[j] = -1;
+        select_row(scores + row * T, n_valid, K, buf, idx + row * K);
+    }
+    free(buf);
+}
+
+/* ------------------------------------------------------------------------- */
+/* V4 compressed sparse attention (CSA) indexer [V4-CSA]                      */
+/* ------------------------------------------------------------------------- */
+
+/* Entries of m tokens available to the query at absolute position i. */
+int64_t oracle_csa_available(int64_t i, int m)
+{
+    return (i + 1) / m;
+}
+
+/*
+ * fp8_index over compressed entries: k_cache [B,t_max,D] / k_scale [B,t_max]
+ * hold the entries' indexer keys (entry e at row e); scores [B,S,T] over
+ * entries 0 .. T-1.  Every entry is scored as [V32-IDX]'s keys are (no mask),
+ * then entry e of query s is masked (-inf) unless
+ * e < oracle_csa_available(start_pos + s, m).
+ */
+void oracle_index_scores_csa(const uint8_t *q_fp8, const float *q_scale, const float *w,
+                             const uint8_t *k_cache, const float *k_scale, int64_t t_max,
+                             int B, int S, int H, int D, int64_t start_pos, int64_t T, int m,
+                             float softmax_scale, float *scores)
+{
+    /* start_pos = T: every entry of every row is within the token-level causal
+       limit, so nothing is masked there */
+    oracle_index_scores(q_fp8, q_scale, w, k_cache, k_scale, t_max, B, S, H, D, T, T,
+                        softmax_scale, scores);
+    for (int64_t row = 0; row < (int64_t)B * S; row++) {
+        int s = (int)(row % S);
+        int64_t avail = oracle_csa_available(start_pos + s, m);
+        for (int64_t e = avail < 0 ? 0 : avail; e < T; e++)
+            scores[row * T + e] = -INFINITY;
+    }
+}
+
+/*
+ * Top-k over compressed entries: idx [B,S,K], K = min(k, T); row (b,s) keeps
+ * the min(K, n_avail) best of its n_avail = min(T, available entries) by
+ * (score desc, entry asc), in ascending entry order, padded with -1.
+ */
+void oracle_topk_select_csa(const float *scores, int B, int S, int64_t T, int64_t start_pos,
+                            int m, int k, int32_t *idx)
+{
+    int K = (int64_t)k < T ? k : (int)T;
+    scored_pos *buf = (scored_pos *)malloc(sizeof(scored_pos) * (size_t)(T > 0 ? T : 1));
+    for (int64_t row = 0; row < (int64_t)B * S; row++) {
+        int s = (int)(row % S);
+        int64_t n_valid = oracle_csa_available(start_pos + s, m);
+        if (n_valid > T)
+            n_valid = T;
+        if (n_valid < 0)
+            n_valid = 0;
+        select_row(scores + row * T, n_valid, K, buf, idx + row * K);
     }
     free(buf);
 }

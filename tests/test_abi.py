@@ -187,3 +187,19 @@ def test_wait_selftest_argument_checks(dsa):
     assert L.dsa_wait_selftest(0, 0, NULL) == dsa.DSA_ERR_INVALID_ARG
     assert L.dsa_wait_selftest(-5, 1, NULL) == dsa.DSA_ERR_INVALID_ARG
     assert L.dsa_wait_selftest(2_000_000_001, 0, NULL) == dsa.DSA_ERR_INVALID_ARG
+
+
+def test_csa_argument_checks(dsa):
+    L = dsa._lib
+    def scores(**kw):
+        return L.dsa_index_scores_csa(FAKE, FAKE, FAKE, FAKE, FAKE, kw.get("t_max", 1000), 1,
+                                      kw.get("S", 1), 64, 128, kw.get("sp", 3999),
+                                      kw.get("T", 1000), kw.get("m", 4), 0.088, FAKE, NULL)
+    assert scores(m=0) == dsa.DSA_ERR_INVALID_ARG
+    assert scores(sp=4003) == dsa.DSA_ERR_INVALID_ARG           # entry 1000 would be visible
+    assert scores(T=1001) == dsa.DSA_ERR_INVALID_ARG            # more entries than the cache holds
+    def topk(**kw):
+        return L.dsa_topk_select_csa(FAKE, 1, 1, kw.get("T", 1000), kw.get("sp", 3999),
+                                     kw.get("m", 4), 2048, FAKE, NULL, 0, NULL)
+    assert topk(m=0) == dsa.DSA_ERR_INVALID_ARG
+    assert topk(sp=4003) == dsa.DSA_ERR_INVALID_ARG

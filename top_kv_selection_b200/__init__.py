@@ -50,6 +50,9 @@ _SIGNATURES = {
     "dsa_decode_index_scores": ([_P, _P, _P, _P, _P, _i64, _i32, _i32, _i32, _i64, _f32, _P, _P],
                                 _i32),
     "dsa_topk_select_workspace_size": ([_i32, _i32, _i64, _i32], _sz),
+    "dsa_index_scores_csa": ([_P, _P, _P, _P, _P, _i64, _i32, _i32, _i32, _i32, _i64, _i64, _i32,
+                              _f32, _P, _P], _i32),
+    "dsa_topk_select_csa": ([_P, _i32, _i32, _i64, _i64, _i32, _i32, _P, _P, _sz, _P], _i32),
     "dsa_topk_select": ([_P, _i32, _i32, _i64, _i64, _i32, _P, _P, _sz, _P], _i32),
     "dsa_sparse_mla_attn_workspace_size": ([_i32, _i32, _i32, _i32, _i32, _i32, _i32], _sz),
     "dsa_sparse_mla_attn": ([_P, _P, _i64, _P, _i32, _i32, _i32, _i32, _i32, _i32, _i64, _f32,
@@ -234,6 +237,32 @@ def dsa_topk_select(scores: torch.Tensor, start_pos: int, k: int, idx: torch.Ten
     ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
     _check("dsa_topk_select", _lib.dsa_topk_select(
         _ptr(scores), B, S, T, start_pos, k, _ptr(idx), _ptr(workspace), ws_bytes,
+        _stream(stream)))
+
+
+def dsa_index_scores_csa(q_fp8: torch.Tensor, q_scale: torch.Tensor, w: torch.Tensor,
+                         k_cache: torch.Tensor, k_scale: torch.Tensor, start_pos: int, T: int,
+                         compress: int, softmax_scale: float, scores: torch.Tensor,
+                         stream=None) -> None:
+    """fp8_index over compressed entries (m = compress tokens each): scores [B,S,T] over
+    the T entries of k_cache [B,t_max,D], entry e of query s masked unless
+    e < (start_pos + s + 1) // m."""
+    B, S, H, D = q_fp8.shape
+    t_max = k_cache.shape[1]
+    _check("dsa_index_scores_csa", _lib.dsa_index_scores_csa(
+        _ptr(q_fp8), _ptr(q_scale), _ptr(w), _ptr(k_cache), _ptr(k_scale), t_max, B, S, H, D,
+        start_pos, T, compress, softmax_scale, _ptr(scores), _stream(stream)))
+
+
+def dsa_topk_select_csa(scores: torch.Tensor, start_pos: int, compress: int, k: int,
+                        idx: torch.Tensor, workspace: torch.Tensor | None = None,
+                        stream=None) -> None:
+    """scores [B,S,T] over entries -> idx [B,S,min(k,T)] entry ids (ascending, -1 padded)
+    among the (start_pos + s + 1) // compress available entries of each row."""
+    B, S, T = scores.shape
+    ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    _check("dsa_topk_select_csa", _lib.dsa_topk_select_csa(
+        _ptr(scores), B, S, T, start_pos, compress, k, _ptr(idx), _ptr(workspace), ws_bytes,
         _stream(stream)))
 
 

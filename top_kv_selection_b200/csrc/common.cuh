@@ -108,7 +108,8 @@ dsa_status launch_indexer_quant(const void *x, dsa_dtype x_dtype, int64_t n_rows
 dsa_status launch_index_scores(const uint8_t *q_fp8, const float *q_scale, const float *w,
                                const uint8_t *k_cache, const float *k_scale, int64_t t_max, int B,
                                int S, int H, int D, int64_t start_pos, int64_t T,
-                               float softmax_scale, float *scores, cudaStream_t stream);
+                               float softmax_scale, float *scores, cudaStream_t stream,
+                               int compress = 1);
 
 // Decode step: rotate + quantise the new queries and key inside the scorer,
 // append the key at T-1, score positions 0..T-1 of each sequence.  With
@@ -127,6 +128,8 @@ size_t topk_workspace_bytes(int B, int S, int64_t T, int k);
 // prefetch_rows: optional cache whose rows at the selected positions are
 // requested into L2 as they are selected (row (b, t) at prefetch_rows +
 // (b * prefetch_t_max + t) * prefetch_row_bytes; bytes a multiple of 16).
+// compress: the scores are over compressed entries of this many tokens; row s
+// keeps the best of its (start_pos + s + 1) / compress available entries.
 // row_hist / hist_chunks: the decode step's top-k (S = 1, start_pos = T - 1,
 // T up to 262144) takes the decode scorer's per-CTA histograms of the scores'
 // top 12 key bits ([B][hist_chunks][kHistBins]) and runs one cluster per row
@@ -135,7 +138,7 @@ dsa_status launch_topk_select(const float *scores, int B, int S, int64_t T, int6
                               int k, int32_t *idx, void *ws, cudaStream_t stream,
                               const void *prefetch_rows = nullptr, int64_t prefetch_t_max = 0,
                               int prefetch_row_bytes = 0, const uint32_t *row_hist = nullptr,
-                              int hist_chunks = 0);
+                              int hist_chunks = 0, int compress = 1);
 
 size_t sparse_mla_workspace_bytes(int B, int S, int Hq, int dc, int dr, int k, dsa_dtype dt);
 bool sparse_mla_tc_supported(int Hq, int dc, int dr, int k, dsa_dtype dt);

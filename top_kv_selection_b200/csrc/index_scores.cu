@@ -59,6 +59,7 @@ struct ScoreArgs {
     int64_t start_pos;
     int64_t T;
     int B, S, H, NH, chunks;
+    int compress;              // keys are compressed entries of this many tokens (1: tokens)
     uint32_t tmem_cols;
     float head_scale, softmax_scale;
     int *err;
@@ -192,8 +193,10 @@ score_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const ScoreArgs a) {
     const int chunk = blockIdx.x - (int)(ri * a.chunks);
     const int64_t b = ri % a.B, s = a.S - 1 - ri / a.B;
     const int64_t row = b * a.S + s;
-    const int64_t limit = a.start_pos + s;
-    const int64_t n_vis = a.T < limit + 1 ? a.T : limit + 1;
+    // keys visible to this query: positions <= start_pos + s, or with compressed
+    // entries of m tokens, the entries whose m tokens are all in
+    const int64_t avail = (a.start_pos + s + 1) / (a.compress > 1 ? a.compress : 1);
+    const int64_t n_vis = a.T < avail ? a.T : avail;
     const int64_t n_tiles = (n_vis + kTile - 1) / kTile;
     const int64_t tile_lo = chunk * n_tiles / a.chunks;
     const int64_t tile_hi = (chunk + 1) * n_tiles / a.chunks;
@@ -462,7 +465,8 @@ dsa_status launch_tc(ScoreArgs a, const uint8_t *k_cache, int B, int S, int64_t 
 
     const size_t smem = score_smem_bytes<D, kRaw>(a.NH);
     const int64_t rows = (int64_t)B * S;
-    const int64_t vis_max = T < start_pos + S ? T : start_pos + S;
+    const int64_t avail_max = (start_pos + S) / (a.compress > 1 ? a.compress : 1);
+    const int64_t vis_max = T < avail_max ? T : avail_max;
     a.chunks = score_chunks<D, kRaw>(rows, a.NH, vis_max);
     const int64_t chunks = a.chunks;
     if (cudaFuncSetAttribute(score_tc_kernel<D, kRaw>,
@@ -489,7 +493,8 @@ dsa_status launch_tc(ScoreArgs a, const uint8_t *k_cache, int B, int S, int64_t 
 dsa_status launch_index_scores(const uint8_t *q_fp8, const float *q_scale, const float *w,
                                const uint8_t *k_cache, const float *k_scale, int64_t t_max, int B,
                                int S, int H, int D, int64_t start_pos, int64_t T,
-                               float softmax_scale, float *scores, cudaStream_t stream) {
+                               float softmax_scale, float *scores, cudaStream_t stream,
+                               int compress) {
     if ((int64_t)B * S * T == 0) return DSA_OK;
     ScoreArgs a = {};
     a.q_fp8 = q_fp8;
@@ -500,7 +505,8 @@ dsa_status launch_index_scores(const uint8_t *q_fp8, const float *q_scale, const
     a.t_max = t_max;
     a.H = H;
     a.softmax_scale = softmax_scale;
-    if (prefill_group_rows(B, S, H))
+    a.compress = compress;
+    if (compress == 1 && prefill_group_rows(B, S, H))
         return launch_prefill_scores(q_fp8, q_scale, w, k_cache, k_scale, t_max, B, S, H, D,
                                      start_pos, T, softmax_scale, scores, stream);
     return D == 128 ? launch_tc<128, false>(a, k_cache, B, S, start_pos, T, stream)
@@ -530,6 +536,7 @@ dsa_status launch_decode_scores(const float *q_raw, const float *w, const float 
     a.t_max = t_max;
     a.H = H;
     a.softmax_scale = softmax_scale;
+    a.compress = 1;
     return D == 128 ? launch_tc<128, true>(a, k_cache, B, 1, T - 1, T, stream)
                     : launch_tc<64, true>(a, k_cache, B, 1, T - 1, T, stream);
 }
@@ -552,7 +559,29 @@ extern "C" dsa_status dsa_index_scores(const uint8_t *q_fp8, const float *q_scal
     if (!dsa::aligned16(q_fp8) || !dsa::aligned16(k_cache)) return DSA_ERR_INVALID_ARG;
     return dsa::launch_index_scores(q_fp8, q_scale, w, k_cache, k_scale, t_max, B, S, H, D,
                                     start_pos, T, softmax_scale, scores,
-                                    reinterpret_cast<cudaStream_t>(stream));
+                                    reinterpret_cast<cudaStream_t>(stream), 1);
+}
+
+extern "C" dsa_status dsa_index_scores_csa(const uint8_t *q_fp8, const float *q_scale,
+                                           const float *w, const uint8_t *k_cache,
+                                           const float *k_scale, int64_t t_max, int B, int S,
+                                           int H, int D, int64_t start_pos, int64_t T,
+                                           int compress, float softmax_scale, float *scores,
+                                           dsa_stream_t stream) {
+    if (B < 0 || S < 0 || T < 0 || start_pos < 0 || H < 1 || compress < 1)
+        return DSA_ERR_INVALID_ARG;
+    if (D != 64 && D != 128) return DSA_ERR_UNSUPPORTED;
+    if (H > 256) return DSA_ERR_UNSUPPORTED;
+    if ((int64_t)B * S * T == 0) return DSA_OK;
+    // every entry the last query may see must be in the cache
+    if (T > t_max || (start_pos + S) / compress > T) return DSA_ERR_INVALID_ARG;
+    if (t_max > INT32_MAX || B > 65535 || (int64_t)B * S > INT32_MAX / 512)
+        return DSA_ERR_UNSUPPORTED;
+    if (!q_fp8 || !q_scale || !w || !k_cache || !k_scale || !scores) return DSA_ERR_INVALID_ARG;
+    if (!dsa::aligned16(q_fp8) || !dsa::aligned16(k_cache)) return DSA_ERR_INVALID_ARG;
+    return dsa::launch_index_scores(q_fp8, q_scale, w, k_cache, k_scale, t_max, B, S, H, D,
+                                    start_pos, T, softmax_scale, scores,
+                                    reinterpret_cast<cudaStream_t>(stream), compress);
 }
 
 extern "C" dsa_status dsa_decode_index_scores(const float *q_idx, const float *w,

@@ -208,7 +208,7 @@ __device__ __forceinline__ void cta0_find_and_send(cg::cluster_group &cl, TopkSh
 
 __global__ void __launch_bounds__(kThreads, 1)
 topk_cluster_kernel(const float *scores, int S, int64_t T, int64_t start_pos, int K, int L,
-                    int32_t *__restrict__ idx, const RowPrefetch pf) {
+                    int32_t *__restrict__ idx, const RowPrefetch pf, int compress) {
     // a kernel launched after this one (the sparse attention) may start its
     // set-up now; it reads the selections only after waiting for this grid
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
@@ -217,7 +217,7 @@ topk_cluster_kernel(const float *scores, int S, int64_t T, int64_t start_pos, in
     const int p = (int)cl.block_rank();
     const int64_t row = blockIdx.x / CN;
     const int64_t s = row % S, bseq = row / S;
-    int64_t n_valid = start_pos + s + 1;
+    int64_t n_valid = (start_pos + s + 1) / compress;
     if (n_valid > T) n_valid = T;
     const int m = (int64_t)K < n_valid ? K : (int)n_valid;
     int32_t *dst = idx + row * K;
@@ -932,14 +932,14 @@ topk_decode_kernel(const float *scores, int64_t T, int K, int32_t *__restrict__ 
 // cluster kernel's shared memory).
 __global__ void __launch_bounds__(kThreads)
 topk_row_kernel(const float *__restrict__ scores, int S, int64_t T, int64_t start_pos, int K,
-                int32_t *__restrict__ idx) {
+                int32_t *__restrict__ idx, int compress) {
     __shared__ unsigned hist[256];
     __shared__ int warp_tot[33];
     __shared__ unsigned s_sel, s_remaining;
 
     const int64_t row = blockIdx.x;
     const int64_t s = row % S;
-    int64_t n_valid = start_pos + s + 1;
+    int64_t n_valid = (start_pos + s + 1) / compress;
     if (n_valid > T) n_valid = T;
     const int m = (int64_t)K < n_valid ? K : (int)n_valid;
     const float *src = scores + row * T;
@@ -1022,16 +1022,18 @@ size_t topk_workspace_bytes(int, int, int64_t, int) { return 0; }
 dsa_status launch_topk_select(const float *scores, int B, int S, int64_t T, int64_t start_pos,
                               int k, int32_t *idx, void *, cudaStream_t stream,
                               const void *prefetch_rows, int64_t prefetch_t_max,
-                              int prefetch_row_bytes, const uint32_t *row_hist, int hist_chunks) {
+                              int prefetch_row_bytes, const uint32_t *row_hist, int hist_chunks,
+                              int compress) {
     if ((int64_t)B * S * T == 0) return DSA_OK;
     const int K = (int64_t)k < T ? k : (int)T;
     const int64_t rows = (int64_t)B * S;
-    const int64_t n_max = T < start_pos + S ? T : start_pos + S;
+    const int64_t avail_max = (start_pos + S) / compress;
+    const int64_t n_max = T < avail_max ? T : avail_max;
     RowPrefetch pf;
     pf.base = static_cast<const uint8_t *>(prefetch_rows);
     pf.t_max = prefetch_t_max;
     pf.bytes = prefetch_row_bytes;
-    if (row_hist && hist_chunks > 0 && S == 1 && start_pos == T - 1 &&
+    if (row_hist && hist_chunks > 0 && compress == 1 && S == 1 && start_pos == T - 1 &&
         (T + kDecSpan - 1) / kDecSpan <= kMaxCluster) {
         // the decode top-k: one cluster per row, the threshold bin from the scorer's histogram
         const int dcn = (int)((T + kDecSpan - 1) / kDecSpan);
@@ -1065,7 +1067,8 @@ dsa_status launch_topk_select(const float *scores, int B, int S, int64_t T, int6
     int cn, L;
     cluster_plan(n_max, &cn, &L);
     if (cn == 0) {
-        topk_row_kernel<<<(unsigned)rows, kThreads, 0, stream>>>(scores, S, T, start_pos, K, idx);
+        topk_row_kernel<<<(unsigned)rows, kThreads, 0, stream>>>(scores, S, T, start_pos, K, idx,
+                                                                  compress);
         return launch_status();
     }
     // keys of the slice (padded) and the gathered keys with their positions
@@ -1093,8 +1096,8 @@ dsa_status launch_topk_select(const float *scores, int B, int S, int64_t T, int6
     attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 2;
-    if (cudaLaunchKernelEx(&cfg, topk_cluster_kernel, scores, S, T, start_pos, K, L, idx, pf) !=
-        cudaSuccess)
+    if (cudaLaunchKernelEx(&cfg, topk_cluster_kernel, scores, S, T, start_pos, K, L, idx, pf,
+                           compress) != cudaSuccess)
         return DSA_ERR_CUDA;
     return launch_status();
 }
@@ -1118,4 +1121,21 @@ extern "C" dsa_status dsa_topk_select(const float *scores, int B, int S, int64_t
     if (need > 0 && (!workspace || workspace_bytes < need)) return DSA_ERR_WORKSPACE;
     return dsa::launch_topk_select(scores, B, S, T, start_pos, k, idx, workspace,
                                    reinterpret_cast<cudaStream_t>(stream));
+}
+
+extern "C" dsa_status dsa_topk_select_csa(const float *scores, int B, int S, int64_t T,
+                                          int64_t start_pos, int compress, int k, int32_t *idx,
+                                          void *workspace, size_t workspace_bytes,
+                                          dsa_stream_t stream) {
+    if (B < 0 || S < 0 || T < 0 || start_pos < 0 || k < 1 || compress < 1)
+        return DSA_ERR_INVALID_ARG;
+    if ((int64_t)B * S * T == 0) return DSA_OK;
+    if (T > INT32_MAX || (start_pos + S) / compress > T) return DSA_ERR_INVALID_ARG;
+    if ((int64_t)B * S * 16 > INT32_MAX) return DSA_ERR_UNSUPPORTED;
+    if (!scores || !idx) return DSA_ERR_INVALID_ARG;
+    const size_t need = dsa::topk_workspace_bytes(B, S, T, k);
+    if (need > 0 && (!workspace || workspace_bytes < need)) return DSA_ERR_WORKSPACE;
+    return dsa::launch_topk_select(scores, B, S, T, start_pos, k, idx, workspace,
+                                   reinterpret_cast<cudaStream_t>(stream), nullptr, 0, 0,
+                                   nullptr, 0, compress);
 }
