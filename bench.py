@@ -418,6 +418,10 @@ def run_ours(args, wl, world, rank, local):
         attn_fp8 = time_sparse_mla_fp8(dsa, peak, wl)
     except Exception as exc:                       # reported, never fatal to the main line
         attn_fp8 = {"error": f"{type(exc).__name__}: {exc}"[:200]}
+    try:
+        csa = time_csa_decode(dsa, peak, wl)
+    except Exception as exc:                       # reported, never fatal to the main line
+        csa = {"error": f"{type(exc).__name__}: {exc}"[:200]}
     # keys + scales of every cached token, plus the new tokens' fp32 queries,
     # weights and keys (the scores written are not algorithmic)
     score_bytes = wl.B * wl.T * (wl.D + 4) + wl.B * (wl.H * wl.D * 4 + wl.H * 4 + wl.D * 4)
@@ -451,6 +455,7 @@ def run_ours(args, wl, world, rank, local):
         "indexer_prologue": prologue,
         "prefill_chain": prefill_chain,
         "sparse_mla_fp8": attn_fp8,
+        "csa_indexer": csa,
         "clocks": clk.summary(),
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -640,6 +645,65 @@ def time_indexer_prologue(dsa, peak_gbs, iters=20):
            "frac": nbytes / t / 1e9 / peak_gbs, "bound": "hbm"}
     del q, k, q_fp8, k_cache
     return out
+
+
+def time_csa_decode(dsa, peak_gbs, wl, m=4, iters=20, copies=3):
+    """The V4 CSA indexer at the decode workload's sizes: B sequences of T tokens
+    compressed at rate m into T / m entries, 64 heads x 128, k = 2048 over the
+    entries: dsa_index_scores_csa then dsa_topk_select_csa, timed together and
+    the scorer alone.  Rotating entry caches (each B x T/m x 132 B) are seeded
+    random normals made on the device (performance only).  Algorithmic bytes of
+    the scorer: the entries' keys and scales plus the queries."""
+    B, H, D, k = wl.B, wl.H, wl.D, wl.topk
+    E = wl.T // m
+    sp = wl.T - 1
+    g = torch.Generator(device="cuda").manual_seed(wl.seed(5))
+    states = []
+    for _ in range(copies):
+        keys = torch.randn(B, E, D, device="cuda", generator=g)
+        kf = torch.empty(B, E, D, dtype=torch.uint8, device="cuda")
+        ksc = torch.empty(B, E, dtype=torch.float32, device="cuda")
+        dsa.dsa_indexer_quant(keys, kf, ksc, n_rows=B, out_row_stride=E * D, scale_row_stride=E)
+        del keys
+        q = torch.randn(B, 1, H, D, device="cuda", generator=g)
+        qf = torch.empty(B, 1, H, D, dtype=torch.uint8, device="cuda")
+        qs = torch.empty(B, 1, H, dtype=torch.float32, device="cuda")
+        dsa.dsa_indexer_quant(q, qf, qs)
+        w = torch.randn(B, 1, H, device="cuda", generator=g)
+        states.append((qf, qs, w, kf, ksc))
+    scores = torch.empty(B, 1, E, dtype=torch.float32, device="cuda")
+    idx = torch.empty(B, 1, min(k, E), dtype=torch.int32, device="cuda")
+    ws = torch.empty(max(1, dsa.dsa_topk_select_workspace_size(B, 1, E, k)), dtype=torch.uint8,
+                     device="cuda")
+
+    def score(i):
+        qf, qs, w, kf, ksc = states[i % copies]
+        dsa.dsa_index_scores_csa(qf, qs, w, kf, ksc, sp, E, m, wl.softmax_scale_idx, scores)
+
+    def both(i):
+        score(i)
+        dsa.dsa_topk_select_csa(scores, sp, m, k, idx, ws)
+
+    def timed(fn):
+        for i in range(3):
+            fn(i)
+        torch.cuda.synchronize()
+        t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        t0.record()
+        for i in range(iters):
+            fn(i)
+        t1.record()
+        t1.synchronize()
+        return t0.elapsed_time(t1) * 1e-3 / iters
+
+    t_sc, t_both = timed(score), timed(both)
+    nbytes = B * E * (D + 4) + B * H * (D + 8)
+    return {"workload": f"{wl.name}_csa_m{m}", "entries": E, "compress": m, "k": k,
+            "scores_us": t_sc * 1e6, "scores_plus_topk_us": t_both * 1e6, "scorer_bytes": nbytes,
+            "achieved_gbs": nbytes / t_sc / 1e9, "peak_gbs": peak_gbs,
+            "frac": nbytes / t_sc / 1e9 / peak_gbs, "bound": "hbm",
+            "note": "entry keys are an input (the compressor is not on the pages); "
+                    "top-k over (start_pos + 1) // m available entries"}
 
 
 BF16_FALLBACK_TFLOPS = 1590.0
