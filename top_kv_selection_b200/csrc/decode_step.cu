@@ -83,12 +83,10 @@ extern "C" dsa_status dsa_decode_step(const float *q_idx, const float *w, const 
     if ((st = dsa::launch_decode_scores(q_idx, w, k_new, k_cache, k_scale, t_max, B, H, D, T,
                                         softmax_scale, ws.scores, s, ws.hist)) != DSA_OK)
         return st;
-    // the top-k asks L2 for the latent rows it selects, ahead of the attention's gather
-    const int row_bytes = dt == DSA_FP8_LATENT ? (int)dsa_latent_row_bytes(dc, dr)
-                                               : (dc + dr) * (dt == DSA_BF16 ? 2 : 4);
+    // (the attention prefetches its own rows into L2; a prefetch issued by the
+    // top-k as it writes each position measured slower in the chained step)
     if ((st = dsa::launch_topk_select(ws.scores, B, 1, T, T - 1, index_topk, idx, nullptr, s,
-                                      row_bytes % 16 == 0 ? kv_cache : nullptr, t_max, row_bytes,
-                                      ws.hist, ws.hist_chunks)) != DSA_OK)
+                                      nullptr, 0, 0, ws.hist, ws.hist_chunks)) != DSA_OK)
         return st;
     const int K = (int64_t)index_topk < T ? index_topk : (int)T;
     if (dt == DSA_FP8_LATENT)

@@ -164,8 +164,9 @@ __device__ __forceinline__ uint4 decode8(uint32_t w0, uint32_t w1, float sc) {
 // splits' fp16 partials (blocks blk0 .. blk0 + splits - 1), for NC octets
 // c8[0..NC) at once: with w_s = 2^(m_s - M) l_s and Y_s = O_s / (l_s sc_s),
 // out = sum_s w_s sc_s Y_s / sum_s w_s and lse = (M + log2 sum_s w_s) ln 2.
-// The loads of eight splits are in flight together; further batches rescale
-// the running sums.
+// The loads of kMergeBatch splits are in flight together (all sixteen of a
+// 2048-slot row); further batches rescale the running sums.
+constexpr int kMergeBatch = 16;
 template <int NC>
 __device__ __forceinline__ void merge_octets(const __half *part_o, const float4 *part_ml, int splits,
                                              int64_t blk0, int64_t row, const int (&c8)[NC], int h,
@@ -176,11 +177,11 @@ __device__ __forceinline__ void merge_octets(const __half *part_o, const float4 
     for (int n = 0; n < NC; n++)
 #pragma unroll
         for (int e = 0; e < 8; e++) acc[n][e] = 0.f;
-    for (int s0 = 0; s0 < splits; s0 += 8) {
-        float4 ml[8];
-        uint4 x[8][NC];
+    for (int s0 = 0; s0 < splits; s0 += kMergeBatch) {
+        float4 ml[kMergeBatch];
+        uint4 x[kMergeBatch][NC];
 #pragma unroll
-        for (int u = 0; u < 8; u++) {
+        for (int u = 0; u < kMergeBatch; u++) {
             const int sp = s0 + u;
             ml[u] = sp < splits ? part_ml[(blk0 + sp) * kHq + h] : make_float4(-INFINITY, 0.f, 1.f, 1.f);
 #pragma unroll
@@ -190,7 +191,7 @@ __device__ __forceinline__ void merge_octets(const __half *part_o, const float4 
         }
         float mb = M;
 #pragma unroll
-        for (int u = 0; u < 8; u++) mb = fmaxf(mb, ml[u].x);
+        for (int u = 0; u < kMergeBatch; u++) mb = fmaxf(mb, ml[u].x);
         if (mb == -INFINITY) continue;
         if (mb > M) {                                  // rescale the running sums
             const float r = M == -INFINITY ? 0.f : ex2(M - mb);
@@ -202,7 +203,7 @@ __device__ __forceinline__ void merge_octets(const __half *part_o, const float4 
             M = mb;
         }
 #pragma unroll
-        for (int u = 0; u < 8; u++) {
+        for (int u = 0; u < kMergeBatch; u++) {
             if (ml[u].x == -INFINITY) continue;
             const float w = ex2(ml[u].x - M) * ml[u].y;
             L += w;

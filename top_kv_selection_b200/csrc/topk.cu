@@ -747,7 +747,7 @@ topk_decode_kernel(const float *scores, int64_t T, int K, int32_t *__restrict__ 
     const bool gather = n_group <= (unsigned)kDecCap && pbits < 32;
     const int gshift = 32 - pbits;
     int n_gt = 0, n_in = 0;
-#pragma unroll 1
+#pragma unroll 4
     for (int j = 0; j < nv; j++) {
         const uint32_t g = gshift == 32 ? 0u : key_at(j) >> gshift;
         n_gt += g > prefix;
@@ -768,7 +768,7 @@ topk_decode_kernel(const float *scores, int64_t T, int K, int32_t *__restrict__ 
         __syncthreads();
         if (n_in) {
             int slot = sh.my_base + ex.y;
-#pragma unroll 1
+#pragma unroll 4
             for (int j = 0; j < nv; j++) {
                 const uint32_t kj = key_at(j);
                 if ((kj >> gshift) == prefix) {
@@ -901,7 +901,7 @@ topk_decode_kernel(const float *scores, int64_t T, int K, int32_t *__restrict__ 
 
     // ---- ordered write of this thread's 32 positions
     int c_gt = 0, c_eq = 0;
-#pragma unroll 1
+#pragma unroll 4
     for (int j = 0; j < nv; j++) {
         const uint32_t kj = key_at(j);
         c_gt += kj > tau;
@@ -912,7 +912,7 @@ topk_decode_kernel(const float *scores, int64_t T, int K, int32_t *__restrict__ 
     int take_eq = my_q - e2.y;
     take_eq = take_eq < 0 ? 0 : (take_eq > c_eq ? c_eq : take_eq);
     int pos = off + e2.x + (my_q < e2.y ? my_q : e2.y);
-#pragma unroll 1
+#pragma unroll 4
     for (int j = 0; j < nv; j++) {
         const uint32_t kj = key_at(j);
         bool sel = kj > tau;
