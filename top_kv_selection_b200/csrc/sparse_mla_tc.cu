@@ -672,6 +672,8 @@ sparse_mla_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const MlaArgs a) 
 __global__ void __launch_bounds__(kHq)
 sparse_mla_combine_kernel(const __half *part_o, const float4 *part_ml, int splits, int64_t row0,
                           __nv_bfloat16 *__restrict__ out, float *__restrict__ lse) {
+    // the next kernel (the next step's scorer) may start its set-up now
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     // the partials come from the preceding kernel: wait for it (plain loads below)
     asm volatile("griddepcontrol.wait;" ::: "memory");
     const int64_t r = blockIdx.x / kOct;                 // row - row0
