@@ -75,6 +75,8 @@ def test_scores_prefill_full_size_sampled_rows(dsa):
     (1, 2, 4193, 4200, 128),       # two passes over the heads; T-1 in the last quarter
     (1, 1, 2081, 2081, 256),       # four passes; T-1 in the second quarter
     (1, 2, 129, 129, 64),          # T-1 opens a tile of its own
+    (0, 2, 3000, 3001, 96),        # D = 64: the staged query's third box in the last key stage
+    (1, 2, 700, 700, 20),          # staged query rows end inside its second box
 ])
 def test_decode_index_scores_matches_oracle(dsa, cfg, B, T, t_max, H):
     """The indexer half of a decode step: quantise the new queries and key, append

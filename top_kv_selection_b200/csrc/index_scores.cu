@@ -60,6 +60,8 @@ struct ScoreArgs {
     int64_t T;
     int B, S, H, NH, chunks;
     int compress;              // keys are compressed entries of this many tokens (1: tokens)
+    int q_copies;              // decode: the fp32 query row arrives in this many TMA boxes
+    int q_box_bytes;           //   of this size into shared memory (0 boxes: direct loads)
     uint32_t tmem_cols;
     float head_scale, softmax_scale;
     int *err;
@@ -74,9 +76,18 @@ static_assert(kHistBins == 1 << kHistBits, "histogram bins");
 template <int D, bool kRaw>
 __host__ __device__ constexpr size_t score_smem_bytes(int NH) {
     return 1024 + (size_t)ring_stages<kRaw>() * kTile * D + (size_t)NH * D +
-           kMaxHeads * sizeof(float) + (2 * ring_stages<kRaw>() + 2 * kAcc + 2) * sizeof(uint64_t) +
+           kMaxHeads * sizeof(float) + (2 * ring_stages<kRaw>() + 2 * kAcc + 3) * sizeof(uint64_t) +
            16 + (kRaw ? kHistBins * sizeof(uint32_t) : 0);
 }
+
+// Decode: the fp32 query row [H, D] of a sequence reaches shared memory as
+// 8 KB TMA boxes of 64 rows x 128 bytes, 128-byte swizzled (16-byte chunk c of
+// row r lands at chunk c ^ (r % 8)), so that the lanes of a head-slice read it
+// back with at most two-way bank conflicts; global loads of 64 contiguous
+// floats per lane would touch 32 cache lines per warp instruction.  Boxes 0
+// and 1 land in the histogram's region, the rest in the last key stage.
+constexpr int kQBoxRows = 64;
+constexpr int kQBoxBytes = kQBoxRows * 128;
 
 // Query operand (K-major, swizzled, padded heads zero) and folded weights
 // w' = ((w * H^-1/2) * q_scale) * softmax_scale, built by the four epilogue
@@ -94,6 +105,33 @@ template <int D, bool kRaw> struct QueryPrefetch {
     __device__ __forceinline__ static int head(int pass) {
         const int t = threadIdx.x - 64;
         return pass * kPass + (t >> 5) * (32 / G) + (t & 31) / G;
+    }
+    // the head's weight only (the query itself comes from shared memory)
+    __device__ __forceinline__ void load_w(const ScoreArgs &a, int64_t row, int pass) {
+        const int h = head(pass), part = (threadIdx.x - 64) % G;
+        w = h < a.H && part == 0 ? a.w[row * a.H + h] : 0.f;
+        qs = 0.f;
+    }
+    // this lane's 64 floats from the staged, swizzled query row (decode)
+    __device__ __forceinline__ void load_staged(const ScoreArgs &a, const uint8_t *box01,
+                                                const uint8_t *box2, int pass) {
+        const int h = head(pass), part = (threadIdx.x - 64) % G;
+        const bool ok = h < a.H;
+        const int slice = h * G + part;             // 256-byte slice of the row
+#pragma unroll
+        for (int half = 0; half < 2; half++) {
+            const int R = slice * 2 + half;         // 128-byte row of the query
+            const int c = R / kQBoxRows, rr = R % kQBoxRows;
+            const uint8_t *line = (c < 2 ? box01 + c * kQBoxBytes : box2 + (c - 2) * kQBoxBytes) +
+                                  rr * 128;
+#pragma unroll
+            for (int j = 0; j < 8; j++) {
+                const float4 v = ok ? *reinterpret_cast<const float4 *>(line + ((j ^ (rr & 7)) << 4))
+                                    : make_float4(0.f, 0.f, 0.f, 0.f);
+                float *d = r + 32 * half + 4 * j;
+                d[0] = v.x; d[1] = v.y; d[2] = v.z; d[3] = v.w;
+            }
+        }
     }
     __device__ __forceinline__ void load(const ScoreArgs &a, int64_t row, int pass) {
         const int h = head(pass), part = (threadIdx.x - 64) % G;
@@ -167,24 +205,32 @@ __device__ __forceinline__ void append_key(const ScoreArgs &a, int64_t b, float 
 
 template <int D, bool kRaw>
 __global__ void __launch_bounds__(kThreads, 2)
-score_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const ScoreArgs a) {
+score_tc_kernel(const __grid_constant__ CUtensorMap tmap_k,
+                const __grid_constant__ CUtensorMap tmap_q, const ScoreArgs a) {
     constexpr int NS = ring_stages<kRaw>();
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t *sk = smem;
     uint8_t *sq = sk + NS * kTile * D;
-    float *wf = reinterpret_cast<float *>(sq + a.NH * D);
+    // decode: histogram of this CTA's scores by the top 12 bits of their key
+    // (1024-byte aligned: before the query operand is built it holds the
+    // first two boxes of the staged fp32 query row)
+    uint32_t *s_hist = reinterpret_cast<uint32_t *>(sq + a.NH * D);
+    float *wf = reinterpret_cast<float *>(sq + a.NH * D + (kRaw ? kHistBins * sizeof(uint32_t) : 0));
     uint64_t *full = reinterpret_cast<uint64_t *>(wf + kMaxHeads);
     uint64_t *empty = full + NS;
     uint64_t *accf = empty + NS;
     uint64_t *acce = accf + kAcc;
-    uint64_t *q_ready = acce + kAcc, *k_ready = q_ready + 1;
-    uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(k_ready + 1);
+    uint64_t *q_ready = acce + kAcc, *k_ready = q_ready + 1, *q_full = k_ready + 1;
+    uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(q_full + 1);
     volatile int *abort = reinterpret_cast<volatile int *>(tmem_holder + 1);
     float *knew_scale = reinterpret_cast<float *>(tmem_holder + 2);
-    // decode: histogram of this CTA's scores by the top 12 bits of their key
-    uint32_t *s_hist = reinterpret_cast<uint32_t *>(tmem_holder + 4);
+    // decode with a staged query: its boxes 2.. occupy the last key stage
+    // until the query operand is built
+    const bool staged = kRaw && a.q_copies > 0;
+    uint8_t *q_box01 = reinterpret_cast<uint8_t *>(s_hist);
+    uint8_t *q_box2 = sk + (NS - 1) * kTile * D;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     // causal rows are taken longest first (query s = S-1 of every sequence,
@@ -250,9 +296,11 @@ score_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const ScoreArgs a) {
         }
         tc::mbar_init(q_ready, 4 * 32);
         tc::mbar_init(k_ready, 1);
+        tc::mbar_init(q_full, 1);
         *abort = 0;
         tc::fence_mbar_init();
         tc::tma_prefetch_desc(&tmap_k);
+        if (staged) tc::tma_prefetch_desc(&tmap_q);
     }
     __syncthreads();        // the barriers are initialised
     // The accumulators: warp 1 allocates them while the epilogue warps build
@@ -268,12 +316,21 @@ score_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const ScoreArgs a) {
     // without a programmatic launch).
     asm volatile("griddepcontrol.wait;" ::: "memory");
     write_masked();
-    // epilogue warps: issue the query, weight, first key-scale and new-key
-    // loads before the key stream starts (named barrier 4, warps 0 and 2..5:
-    // the first ring of key tiles is issued only after them, so that the
-    // query's loads are not queued behind every CTA's ring in HBM)
+    // the staged query row first, ahead of every other request of the CTA
+    if (staged && threadIdx.x == 0) {
+        tc::mbar_arrive_expect_tx(q_full, (uint32_t)(a.q_copies * a.q_box_bytes));
+        const uint64_t keep = tc::l2_evict_last_policy();   // every chunk of the row reads it
+        for (int c = 0; c < a.q_copies; c++)
+            tc::tma_load_3d(c < 2 ? q_box01 + c * kQBoxBytes : q_box2 + (c - 2) * kQBoxBytes,
+                            &tmap_q, 0, c * kQBoxRows, (int)b, q_full, keep);
+    }
+    // epilogue warps: issue the query (unless staged), weight, first key-scale
+    // and new-key loads before the key stream starts (named barrier 4, warps 0
+    // and 2..5: the first ring of key tiles is issued only after them, so that
+    // these loads are not queued behind every CTA's ring in HBM)
     if (warp >= 2) {
-        pf.load(a, row, 0);
+        if (staged) pf.load_w(a, row, 0);
+        else pf.load(a, row, 0);
         if (appender) load_lane_slice<D, float>(a.k_new + b * D, kr);
         ks0 = load_ks(0);     // the new key's entry is reloaded once it is appended
         ks1 = load_ks(1);
@@ -281,8 +338,10 @@ score_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const ScoreArgs a) {
     }
     if (warp != 1) asm volatile("bar.sync 4, 160;" ::: "memory");
     // the first ring of key tiles (the tile holding the appended key waits
-    // for it in the loop below)
-    const int early = n_my - (append ? 1 : 0) < NS ? n_my - (append ? 1 : 0) : NS;
+    // for it in the loop below; with a staged query the last stage waits
+    // until the query operand is built)
+    const int ring0 = staged ? NS - 1 : NS;
+    const int early = n_my - (append ? 1 : 0) < ring0 ? n_my - (append ? 1 : 0) : ring0;
     const uint64_t pol = tc::l2_evict_first_policy();
     if (threadIdx.x == 0)
         for (int i = 0; i < early; i++) {
@@ -305,6 +364,7 @@ score_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const ScoreArgs a) {
                 const int st = i % NS;
                 const uint32_t ph = (uint32_t)(i / NS) & 1u;
                 if (!tc::mbar_wait(&empty[st], ph ^ 1u, a.err, abort)) break;
+                if (staged && i == NS - 1 && !tc::mbar_wait(q_ready, 0, a.err, abort)) break;
                 if (append && i == n_my - 1 && !tc::mbar_wait(k_ready, 0, a.err, abort)) break;
                 tc::mbar_arrive_expect_tx(&full[st], kTile * D);
                 tc::tma_load_3d(sk + st * kTile * D, &tmap_k, 0, (int)((tile_lo + i) * kTile),
@@ -314,6 +374,7 @@ score_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const ScoreArgs a) {
             // wait (bounded) for the last loads still landing in shared memory
             for (int j = issued > NS ? issued - NS : 0; j < issued; j++)
                 tc::mbar_wait(&full[j % NS], (uint32_t)(j / NS) & 1u, a.err, abort);
+            if (staged) tc::mbar_wait(q_full, 0, a.err, abort);
         }
     } else if (warp == 1) {
         if (lane == 0) {
@@ -341,7 +402,21 @@ score_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const ScoreArgs a) {
         }
     } else {
         for (int pass = 0; pass * Prefetch::kPass < a.NH; pass++) {
-            if (pass > 0) pf.load(a, row, pass);
+            if constexpr (kRaw) {
+                if (staged) {
+                    if (pass > 0) pf.load_w(a, row, pass);
+                    if (tc::mbar_wait(q_full, 0, a.err, abort)) {
+                        pf.load_staged(a, q_box01, q_box2, pass);
+                    } else {
+#pragma unroll
+                        for (int e = 0; e < 64; e++) pf.r[e] = 0.f;
+                    }
+                } else if (pass > 0) {
+                    pf.load(a, row, pass);
+                }
+            } else {
+                if (pass > 0) pf.load(a, row, pass);
+            }
             pf.store(a, pass, sq, wf);
         }
         for (int h = a.H + (threadIdx.x - 64); h < kMaxHeads; h += 128) wf[h] = 0.f;
@@ -446,7 +521,7 @@ int score_chunks(int64_t rows, int NH, int64_t vis_max) {
 template <int D, bool kRaw>
 dsa_status launch_tc(ScoreArgs a, const uint8_t *k_cache, int B, int S, int64_t start_pos,
                      int64_t T, cudaStream_t stream) {
-    CUtensorMap tmap;
+    CUtensorMap tmap, tmap_q;
     const uint64_t dims[3] = {(uint64_t)D, (uint64_t)a.t_max, (uint64_t)B};
     const uint64_t strides[2] = {(uint64_t)D, (uint64_t)a.t_max * D};
     const uint32_t box[3] = {(uint32_t)D, (uint32_t)kTile, 1};
@@ -454,6 +529,26 @@ dsa_status launch_tc(ScoreArgs a, const uint8_t *k_cache, int B, int S, int64_t 
         D == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
     if (!encode_tmap(&tmap, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, k_cache, dims, strides, box, swz))
         return DSA_ERR_CUDA;
+    tmap_q = tmap;      // unused unless the decode query is staged
+    a.q_copies = 0;
+    if (kRaw) {
+        // the query row [H, D] fp32 as rows of 128 bytes; staged when its
+        // boxes fit the histogram region (2 boxes) and the last key stage
+        const int64_t q_rows = (int64_t)a.H * D / 32;
+        const int64_t copies = (q_rows + kQBoxRows - 1) / kQBoxRows;
+        const int64_t room = 2 + (int64_t)kTile * D / kQBoxBytes;
+        if (copies <= room) {
+            const uint64_t qd[3] = {32, (uint64_t)q_rows, (uint64_t)B};
+            const uint64_t qs[2] = {128, (uint64_t)q_rows * 128};
+            const uint32_t box_rows = (uint32_t)(q_rows < kQBoxRows ? q_rows : kQBoxRows);
+            const uint32_t qb[3] = {32, box_rows, 1};
+            if (!encode_tmap(&tmap_q, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, a.q_raw, qd, qs, qb,
+                             CU_TENSOR_MAP_SWIZZLE_128B))
+                return DSA_ERR_CUDA;
+            a.q_copies = (int)copies;
+            a.q_box_bytes = (int)box_rows * 128;
+        }
+    }
     a.start_pos = start_pos;
     a.T = T;
     a.B = B;
@@ -484,7 +579,8 @@ dsa_status launch_tc(ScoreArgs a, const uint8_t *k_cache, int B, int S, int64_t 
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    if (cudaLaunchKernelEx(&cfg, score_tc_kernel<D, kRaw>, tmap, a) != cudaSuccess) return DSA_ERR_CUDA;
+    if (cudaLaunchKernelEx(&cfg, score_tc_kernel<D, kRaw>, tmap, tmap_q, a) != cudaSuccess)
+        return DSA_ERR_CUDA;
     return launch_status();
 }
 
