@@ -381,22 +381,51 @@ def run_ours(args, wl, world, rank, local):
     if dsa.dsa_get_device_error() != 0:
         raise RuntimeError("device error word set during warm-up")
 
+    # the steps run as a decode server issues them: a CUDA graph of
+    # graph_steps consecutive steps (the copies in rotation) replayed, the last
+    # steps % graph_steps launched directly
+    graph_steps = len(copies) * max(1, 12 // len(copies))
+    graph = None
+    if not args.eager and args.steps >= graph_steps:
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph):
+            for i in range(graph_steps):
+                decode_step(dsa, wl, copies[i % len(copies)])
+        graph.replay()                                  # untimed
+        torch.cuda.synchronize()
+    n_replays = args.steps // graph_steps if graph is not None else 0
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     _barrier(world)
     torch.cuda.synchronize()
     with ClockSampler(torch.cuda.current_device()) as clk:
         start.record(stream)
-        for i in range(args.steps):
+        for _ in range(n_replays):
+            graph.replay()
+        for i in range(n_replays * graph_steps, args.steps):
             decode_step(dsa, wl, copies[i % len(copies)])
         end.record(stream)
         end.synchronize()
     torch.cuda.synchronize()
     _barrier(world)
+    if dsa.dsa_get_device_error() != 0:
+        raise RuntimeError("device error word set during the timed steps")
     elapsed = start.elapsed_time(end) * 1e-3
     elapsed = _max_over_ranks(world, elapsed)
     ms_per_step = elapsed / args.steps * 1e3
     value = world * args.steps / elapsed
     gscores = world * args.steps * wl.B * wl.T / elapsed / 1e9
+
+    del graph
+    # the same steps launched one by one (reported beside the graph-replayed figure)
+    eager_ms = None
+    if n_replays:
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for i in range(args.steps):
+            decode_step(dsa, wl, copies[i % len(copies)])
+        e1.record(stream)
+        e1.synchronize()
+        eager_ms = _max_over_ranks(world, e0.elapsed_time(e1) * 1e-3) / args.steps * 1e3
 
     # e2e: per-step inputs from pinned host memory, result back to the host
     e2e = run_e2e(dsa, wl, copies, args, world)
@@ -436,6 +465,10 @@ def run_ours(args, wl, world, rank, local):
         "dtype": "fp8_e4m3+bf16", "data": "synthetic",
         "config": bench_config(wl, world),
         "l2_detail": f"{len(copies)} rotating decode-state copies, each larger than L2",
+        "launch": (f"CUDA graph of {graph_steps} steps replayed {n_replays}x"
+                   + (f" + {args.steps - n_replays * graph_steps} direct" if
+                      args.steps % graph_steps else "") if n_replays else "direct launches"),
+        "eager_ms_per_step": eager_ms,
         # the scorer kernel's own rate (cached tokens scored per second), and the
         # same count over the whole step
         "indexer_gscores_per_s": wl.B * wl.T / t_score / 1e9,
@@ -921,6 +954,8 @@ def main(argv=None):
                          "attention) and exit")
     ap.add_argument("--fp8-peak", action="store_true",
                     help="measure the dense FP8 GEMM peak and exit")
+    ap.add_argument("--eager", action="store_true",
+                    help="time the decode steps launched one by one instead of graph-replayed")
     ap.add_argument("--copies", type=int, default=N_COPIES,
                     help="rotating device copies of the decode state (each larger than L2)")
     args = ap.parse_args(argv)
