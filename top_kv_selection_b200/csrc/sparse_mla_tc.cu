@@ -21,9 +21,12 @@
 //      and writes P as bf16 into shared memory, the A operand of the value mix;
 //   3. accumulates O = P C[:, 0:512] as two N = 256 halves (M = 128, K = 128)
 //      whose B operands are the latent chunks already resident (read
-//      MN-major), into all 512 TMEM columns;
+//      MN-major), into all 512 TMEM columns, committing each half on its own;
 //   4. writes bf16 out (+ lse) when the row has one unit, else a normalised
-//      fp16 partial with its (max, sum, power-of-two ranges).  The partials of
+//      fp16 partial with its (max, sum, power-of-two ranges), half by half as
+//      the MMAs complete, so that the first half's stores overlap the second
+//      half's MMAs.  The once-per-CTA loops here are rolled: straight-line code
+//      that runs once stalls on instruction fetch.  The partials of
 //      a row's units ("splits") are merged by a combine kernel launched right
 //      behind (programmatic launch: its CTAs are resident, waiting, while the
 //      attention finishes).  The attention itself is a plain programmatic
@@ -247,9 +250,9 @@ sparse_mla_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const MlaArgs a) 
     uint64_t *q_ready = q_full + 1;              // the query's latent part is in TMEM (256 arrivals)
     uint64_t *s_done = q_ready + 1;              // every logit MMA is complete
     uint64_t *p_full = s_done + 1;               // P is in shared memory (256 arrivals)
-    uint64_t *o_full = p_full + 1;               // O is complete
-    uint64_t *mma_fin = o_full + 1;              // every issued MMA is complete
-    uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(bars + 16);   // after the 15 barriers
+    uint64_t *o_full = p_full + 1;               // [2] column half hv of O is complete
+    uint64_t *mma_fin = o_full + 2;              // every issued MMA is complete
+    uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(bars + 16);   // after the 16 barriers
     volatile int *abort = reinterpret_cast<volatile int *>(tmem_holder + 1);
     uint32_t *vmask = reinterpret_cast<uint32_t *>(const_cast<int *>(abort) + 1);   // [4]
     // softmax exchange (max and sum of the two slot halves): the query's
@@ -271,7 +274,8 @@ sparse_mla_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const MlaArgs a) 
             tc::mbar_init(q_ready, kWork);
             tc::mbar_init(s_done, 1);
             tc::mbar_init(p_full, kWork);
-            tc::mbar_init(o_full, 1);
+            tc::mbar_init(&o_full[0], 1);
+            tc::mbar_init(&o_full[1], 1);
             tc::mbar_init(mma_fin, 1);
             *abort = 0;
             tc::fence_mbar_init();
@@ -464,22 +468,27 @@ sparse_mla_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const MlaArgs a) 
         // the sum
         if (ok && !tc::mbar_wait(s_done, 0, a.err, abort)) ok = false;
         tc::tc_fence_after();
-        uint32_t sv[64];
-#pragma unroll
-        for (int i = 0; i < 4; i++)
-            tc::tmem_ld16(tmem + lane_addr + kColS + 64 * c + 16 * i,
-                          *reinterpret_cast<uint32_t(*)[16]>(sv + 16 * i));
-        tc::tmem_wait_ld();
+        // (rolled over four groups of 16 logits, re-read from TMEM in the
+        // second pass: this code runs once per CTA, and straight-line code
+        // of that length stalls on instruction fetch)
         const uint32_t w0 = vmask[2 * c], w1 = vmask[2 * c + 1];
         const bool part = (w0 & w1) != 0xffffffffu;
+        const uint32_t scol = tmem + lane_addr + kColS + 64 * c;
         float mx8[8];
 #pragma unroll
         for (int e = 0; e < 8; e++) mx8[e] = -INFINITY;
+#pragma unroll 1
+        for (int i = 0; i < 4; i++) {
+            uint32_t sv[16];
+            tc::tmem_ld16(scol + 16 * i, sv);
+            tc::tmem_wait_ld();
+            const uint32_t wb = (i < 2 ? w0 : w1) >> (16 * (i & 1));
 #pragma unroll
-        for (int e = 0; e < 64; e++) {
-            float x = __uint_as_float(sv[e]) * a.scale_log2;
-            if (part && !(((e < 32 ? w0 : w1) >> (e & 31)) & 1u)) x = -INFINITY;
-            mx8[e & 7] = fmaxf(mx8[e & 7], x);
+            for (int e = 0; e < 16; e++) {
+                float x = __uint_as_float(sv[e]) * a.scale_log2;
+                if (part && !((wb >> e) & 1u)) x = -INFINITY;
+                mx8[e & 7] = fmaxf(mx8[e & 7], x);
+            }
         }
         const float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
                                fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
@@ -492,24 +501,31 @@ sparse_mla_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const MlaArgs a) 
         // P of rows [64c, 64c + 64) is the K-major block c of the A operand:
         // head h's 128-byte row, 16-byte piece i = rows 8i .. 8i + 7
         const uint32_t prow = sbase + kP + c * kQBlk + h * 128;
+#pragma unroll 1
+        for (int i = 0; i < 4; i++) {
+            uint32_t sv[16];
+            tc::tmem_ld16(scol + 16 * i, sv);
+            tc::tmem_wait_ld();
+            const uint32_t wb = (i < 2 ? w0 : w1) >> (16 * (i & 1));
 #pragma unroll
-        for (int i = 0; i < 8; i++) {
-            uint32_t pk[4];
+            for (int hp = 0; hp < 2; hp++) {
+                uint32_t pk[4];
 #pragma unroll
-            for (int e = 0; e < 4; e++) {
-                const int x = 8 * i + 2 * e;
-                float t0 = fmaf(__uint_as_float(sv[x]), a.scale_log2, -m);
-                float t1 = fmaf(__uint_as_float(sv[x + 1]), a.scale_log2, -m);
-                const uint32_t wb = x < 32 ? w0 : w1;
-                if (part && !((wb >> (x & 31)) & 1u)) t0 = -INFINITY;
-                if (part && !((wb >> ((x + 1) & 31)) & 1u)) t1 = -INFINITY;
-                const float p0 = ex2(t0), p1 = ex2(t1);
-                l8[(2 * e) & 7] += p0;
-                l8[(2 * e + 1) & 7] += p1;
-                const __nv_bfloat162 v01 = __floats2bfloat162_rn(p0, p1);
-                pk[e] = *reinterpret_cast<const uint32_t *>(&v01);
+                for (int e = 0; e < 4; e++) {
+                    const int x = 8 * hp + 2 * e;
+                    float t0 = fmaf(__uint_as_float(sv[x]), a.scale_log2, -m);
+                    float t1 = fmaf(__uint_as_float(sv[x + 1]), a.scale_log2, -m);
+                    if (part && !((wb >> x) & 1u)) t0 = -INFINITY;
+                    if (part && !((wb >> (x + 1)) & 1u)) t1 = -INFINITY;
+                    const float p0 = ex2(t0), p1 = ex2(t1);
+                    l8[(2 * e) & 7] += p0;
+                    l8[(2 * e + 1) & 7] += p1;
+                    const __nv_bfloat162 v01 = __floats2bfloat162_rn(p0, p1);
+                    pk[e] = *reinterpret_cast<const uint32_t *>(&v01);
+                }
+                st_shared_v4(prow + (((2 * i + hp) ^ (h & 7)) << 4),
+                             make_uint4(pk[0], pk[1], pk[2], pk[3]));
             }
-            st_shared_v4(prow + ((i ^ (h & 7)) << 4), make_uint4(pk[0], pk[1], pk[2], pk[3]));
         }
         // P is read by the tensor core (async proxy)
         tc::fence_proxy_async_smem();
@@ -520,22 +536,20 @@ sparse_mla_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const MlaArgs a) 
         const float lt = red[2 * kHq + h] + red[3 * kHq + h];
 
         // ---------------------------------------------------------- epilogue
-        // thread (h, c) owns output columns [256c, 256c + 256)
-        if (ok && !tc::mbar_wait(o_full, 0, a.err, abort)) ok = false;
-        tc::tc_fence_after();
-        const uint32_t ocol = tmem + lane_addr + kColO + c * 256;
         if (a.splits == 1) {
+            // thread (h, c) owns output columns [256c, 256c + 256)
+            if (ok && !tc::mbar_wait(&o_full[c], 0, a.err, abort)) ok = false;
+            tc::tc_fence_after();
+            const uint32_t ocol = tmem + lane_addr + kColO + c * 256;
             const float inv = lt > 0.f ? 1.f / lt : 0.f;
             uint4 *o16 = reinterpret_cast<uint4 *>(a.out + (row * kHq + h) * kDc + c * 256);
 #pragma unroll 1
-            for (int g = 0; g < 4; g++) {
-                uint32_t ov[64];
-#pragma unroll
-                for (int i = 0; i < 4; i++)
-                    tc::tmem_ld16(ocol + 64 * g + 16 * i, *reinterpret_cast<uint32_t(*)[16]>(ov + 16 * i));
+            for (int g = 0; g < 16; g++) {
+                uint32_t ov[16];
+                tc::tmem_ld16(ocol + 16 * g, ov);
                 tc::tmem_wait_ld();
 #pragma unroll
-                for (int o8 = 0; o8 < 8; o8++) {
+                for (int o8 = 0; o8 < 2; o8++) {
                     uint32_t w[4];
 #pragma unroll
                     for (int e = 0; e < 4; e++) {
@@ -543,58 +557,63 @@ sparse_mla_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const MlaArgs a) 
                                                                        __uint_as_float(ov[8 * o8 + 2 * e + 1]) * inv);
                         w[e] = *reinterpret_cast<const uint32_t *>(&v);
                     }
-                    if (ok) o16[g * 8 + o8] = make_uint4(w[0], w[1], w[2], w[3]);
+                    if (ok) o16[2 * g + o8] = make_uint4(w[0], w[1], w[2], w[3]);
                 }
             }
             if (ok && c == 0 && a.lse) a.lse[row * kHq + h] = lt > 0.f ? (m + log2f(lt)) * kLn2 : -INFINITY;
         } else {
-            // O / (l * sc) in fp16 for the split merge, sc the power of two
-            // that keeps this column half's |O / l| / sc <= 2^14, as
-            // [column / 8][head] groups of eight halves; the half's range is
-            // found in a first read of its columns
-            float amax = 0.f;
-#pragma unroll 1
-            for (int g = 0; g < 4; g++) {
-                uint32_t ov[64];
-#pragma unroll
-                for (int i = 0; i < 4; i++)
-                    tc::tmem_ld16(ocol + 64 * g + 16 * i, *reinterpret_cast<uint32_t(*)[16]>(ov + 16 * i));
-                tc::tmem_wait_ld();
-#pragma unroll
-                for (int e = 0; e < 64; e++) amax = fmaxf(amax, fabsf(__uint_as_float(ov[e])));
-            }
+            // O / (l * sc) in fp16 for the split merge, as [column / 8][head]
+            // groups of eight halves, sc per column half: the power of two
+            // that keeps the half's |O / l| / sc <= 2^14.  The halves are
+            // written in MMA completion order, both threads of a head taking
+            // 128 columns of each; a half is written with sc = 1 and written
+            // again only when the head's max |O| over its 256 columns (the two
+            // threads' maxima) asks for a larger range.
             const float inv_l = lt > 0.f ? 1.f / lt : 0.f;
-            float scl = 1.f;
-            while (amax * inv_l > 16384.f * scl) scl *= 2.f;
-            const float inv = inv_l / scl;
             uint4 *po = reinterpret_cast<uint4 *>(a.part_o + (int64_t)blockIdx.x * kHq * kDc) + h;
+            float *ml = reinterpret_cast<float *>(a.part_ml + (int64_t)blockIdx.x * kHq + h);
+            float *xmax = red + 4 * kHq;          // [half][c][head]
+            auto write_cols = [&](uint32_t ocol, int oct0, float inv, bool track) -> float {
+                float amax = 0.f;
 #pragma unroll 1
-            for (int g = 0; g < 4; g++) {
-                uint32_t ov[64];
+                for (int g = 0; g < 8; g++) {
+                    uint32_t ov[16];
+                    tc::tmem_ld16(ocol + 16 * g, ov);
+                    tc::tmem_wait_ld();
 #pragma unroll
-                for (int i = 0; i < 4; i++)
-                    tc::tmem_ld16(ocol + 64 * g + 16 * i, *reinterpret_cast<uint32_t(*)[16]>(ov + 16 * i));
-                tc::tmem_wait_ld();
+                    for (int o8 = 0; o8 < 2; o8++) {
+                        uint32_t w[4];
 #pragma unroll
-                for (int o8 = 0; o8 < 8; o8++) {
-                    uint32_t w[4];
-#pragma unroll
-                    for (int e = 0; e < 4; e++) {
-                        const __half2 v = __floats2half2_rn(__uint_as_float(ov[8 * o8 + 2 * e]) * inv,
-                                                            __uint_as_float(ov[8 * o8 + 2 * e + 1]) * inv);
-                        w[e] = *reinterpret_cast<const uint32_t *>(&v);
+                        for (int e = 0; e < 4; e++) {
+                            const float x0 = __uint_as_float(ov[8 * o8 + 2 * e]);
+                            const float x1 = __uint_as_float(ov[8 * o8 + 2 * e + 1]);
+                            if (track) amax = fmaxf(amax, fmaxf(fabsf(x0), fabsf(x1)));
+                            const __half2 v = __floats2half2_rn(x0 * inv, x1 * inv);
+                            w[e] = *reinterpret_cast<const uint32_t *>(&v);
+                        }
+                        if (ok) po[(oct0 + 2 * g + o8) * kHq] = make_uint4(w[0], w[1], w[2], w[3]);
                     }
-                    if (ok) po[(c * 32 + g * 8 + o8) * kHq] = make_uint4(w[0], w[1], w[2], w[3]);
                 }
+                return amax;
+            };
+#pragma unroll 1
+            for (int hv = 0; hv < 2; hv++) {
+                if (ok && !tc::mbar_wait(&o_full[hv], 0, a.err, abort)) ok = false;
+                tc::tc_fence_after();
+                const uint32_t ocol = tmem + lane_addr + kColO + 256 * hv + 128 * c;
+                const int oct0 = 32 * hv + 16 * c;
+                xmax[(2 * hv + c) * kHq + h] = write_cols(ocol, oct0, inv_l, true);
+                tc::named_barrier(1, kWork);
+                const float amax = fmaxf(xmax[2 * hv * kHq + h], xmax[(2 * hv + 1) * kHq + h]);
+                float scl = 1.f;
+                while (amax * inv_l > 16384.f * scl) scl *= 2.f;
+                if (scl != 1.f) write_cols(ocol, oct0, inv_l / scl, false);
+                if (ok && c == 0) ml[2 + hv] = scl;
             }
             // (max, sum, range of columns [0, 256), range of columns [256, 512))
-            float *ml = reinterpret_cast<float *>(a.part_ml + (int64_t)blockIdx.x * kHq + h);
-            if (ok) {
-                if (c == 0) {
-                    ml[0] = m;
-                    ml[1] = lt;
-                }
-                ml[2 + c] = scl;
+            if (ok && c == 0) {
+                ml[0] = m;
+                ml[1] = lt;
             }
         }
     } else if (lane > 0) {
@@ -641,18 +660,19 @@ sparse_mla_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const MlaArgs a) 
             // O[:, 256 hv + n] += P C[:, 256 hv + n]: K-step ks covers rows
             // [16 ks, 16 ks + 16); A = P (K-major, block ks / 4), B = the latent
             // chunks 4 hv .. 4 hv + 3 (MN-major, 16 KB between 64-column blocks)
+            // Half 0 is committed before half 1 is issued, so that its
+            // epilogue overlaps the second half's MMAs.
             const uint32_t id_pv = tc::instr_desc(tc::kFmtBF16, tc::kFmtBF16, 128, 256, true);
-            for (int ks = 0; ks < kU / 16; ks++) {
-                const uint64_t pa = tc::smem_desc(sbase + kP + (ks >> 2) * kQBlk + (ks & 3) * 32, 1024,
-                                                  tc::kSwizzle128B);
-#pragma unroll
-                for (int hv = 0; hv < 2; hv++) {
+            for (int hv = 0; hv < 2; hv++) {
+                for (int ks = 0; ks < kU / 16; ks++) {
+                    const uint64_t pa = tc::smem_desc(sbase + kP + (ks >> 2) * kQBlk + (ks & 3) * 32,
+                                                      1024, tc::kSwizzle128B);
                     const uint64_t bd = tc::smem_desc(sbase + 4 * hv * kRegion + ks * 2048, 1024,
                                                       tc::kSwizzle128B, kRegion);
                     tc::mma_f16(tmem + kColO + 256 * hv, pa, bd, id_pv, ks > 0);
                 }
+                tc::tc_commit(&o_full[hv]);
             }
-            tc::tc_commit(o_full);
         }
         // every issued MMA completes before TMEM is released
         tc::tc_commit(mma_fin);
