@@ -495,6 +495,7 @@ constexpr int kDecThreads = 512;
 constexpr int kDecWarps = kDecThreads / 32;
 constexpr int kDecPer = 32;                         // positions per thread
 constexpr int kDecSpan = kDecThreads * kDecPer;     // positions per CTA: 16384
+constexpr int kKeyPitch = kDecPer + 1;              // a thread's keys in shared memory (padded)
 constexpr int kDecCap = 8192;                       // keys CTA 0 gathers
 constexpr int kDecSub = 1024;                       // bins of a 10-bit pass
 constexpr int kDecFew = 32;                         // keys one warp ranks directly
@@ -612,9 +613,9 @@ topk_decode_kernel(const float *scores, int64_t T, int K, int32_t *__restrict__ 
     }
     extern __shared__ __align__(16) uint8_t dec_smem[];
     DecShared &sh = *reinterpret_cast<DecShared *>(dec_smem);
-    // this CTA's keys, [j][thread]: the per-key loops below read them from here
-    // and stay rolled (one pass per CTA, so unrolled code would be fetched
-    // cold on every SM)
+    // this CTA's keys, thread t's 32 positions at skey[t * 33 + j]: the per-key
+    // loops below read them from here and stay rolled (one pass per CTA, so
+    // unrolled code would be fetched cold on every SM)
     uint32_t *skey = reinterpret_cast<uint32_t *>(dec_smem + sizeof(DecShared));
     DecShared *sh0 = cl.map_shared_rank(&sh, 0);
     if (p == 0) {
@@ -628,9 +629,22 @@ topk_decode_kernel(const float *scores, int64_t T, int K, int32_t *__restrict__ 
     // the scores and the histogram come from the scorer
     asm volatile("griddepcontrol.wait;" ::: "memory");
 
-    // this CTA's slice of the bins, summed over the row's scorer histograms
-    // (thread t: bins b0 + t, b0 + t + 512, ...), and this thread's 32
-    // positions, loaded together
+    // This CTA's scores, loaded first as coalesced float4s (consecutive
+    // threads, consecutive 16 bytes; the thread that owns a position is not
+    // the one that loads it), then its slice of the bins, summed over the
+    // row's scorer histograms (thread t: bins b0 + t, b0 + t + 512, ...), with
+    // both sets of loads in flight together.
+    const int64_t span0 = (int64_t)p * kDecSpan;
+    const int64_t span_n = T - span0 <= 0 ? 0 : (T - span0 >= kDecSpan ? kDecSpan : T - span0);
+    const float *src = scores + row * T + span0;
+    const bool vec = span_n == kDecSpan && (reinterpret_cast<uintptr_t>(src) & 15) == 0;
+    constexpr int kLoads = kDecSpan / 4 / kDecThreads;   // float4s a thread loads
+    float4 kv4[kLoads];
+    if (vec) {
+#pragma unroll
+        for (int u = 0; u < kLoads; u++)
+            kv4[u] = reinterpret_cast<const float4 *>(src)[tid + u * kDecThreads];
+    }
     const int bpc = (kBins + CN - 1) / CN;           // bins per CTA
     const int b_lo = p * bpc, b_hi = b_lo + bpc < kBins ? b_lo + bpc : kBins;
     constexpr int kMaxSlice = kBins / kDecThreads;   // bins a thread sums (CN = 1)
@@ -656,26 +670,32 @@ topk_decode_kernel(const float *scores, int64_t T, int K, int32_t *__restrict__ 
             bsum[u] = acc;
         }
     }
-    const int64_t t0 = (int64_t)p * kDecSpan + (int64_t)tid * kDecPer;
-    const float *src = scores + row * T + t0;
-    uint32_t key[kDecPer];
-    if (t0 + kDecPer <= T && (reinterpret_cast<uintptr_t>(src) & 15) == 0) {
+    // the keys into shared memory: position o of the span at skey[(o / 32) * 33
+    // + o % 32] (a warp's stores fall in 32 different banks; so do the owners'
+    // reads of their j-th key); positions past T get key 0
 #pragma unroll
-        for (int j = 0; j < kDecPer / 4; j++) {
-            const float4 v = reinterpret_cast<const float4 *>(src)[j];
-            key[4 * j] = score_key(v.x);
-            key[4 * j + 1] = score_key(v.y);
-            key[4 * j + 2] = score_key(v.z);
-            key[4 * j + 3] = score_key(v.w);
+    for (int u = 0; u < kLoads; u++) {
+        const int o = 4 * (tid + u * kDecThreads);
+        float4 v;
+        if (vec) {
+            v = kv4[u];
+        } else {
+            v.x = o < span_n ? src[o] : 0.f;
+            v.y = o + 1 < span_n ? src[o + 1] : 0.f;
+            v.z = o + 2 < span_n ? src[o + 2] : 0.f;
+            v.w = o + 3 < span_n ? src[o + 3] : 0.f;
         }
-    } else {
-#pragma unroll
-        for (int j = 0; j < kDecPer; j++) key[j] = t0 + j < T ? score_key(src[j]) : 0u;
+        uint32_t *kr = skey + (o / kDecPer) * kKeyPitch + (o % kDecPer);
+        kr[0] = o < span_n ? score_key(v.x) : 0u;
+        kr[1] = o + 1 < span_n ? score_key(v.y) : 0u;
+        kr[2] = o + 2 < span_n ? score_key(v.z) : 0u;
+        kr[3] = o + 3 < span_n ? score_key(v.w) : 0u;
     }
+    const int64_t t0 = span0 + (int64_t)tid * kDecPer;
     const int nv = T - t0 <= 0 ? 0 : (T - t0 >= kDecPer ? kDecPer : (int)(T - t0));
-#pragma unroll
-    for (int j = 0; j < kDecPer; j++) skey[j * kDecThreads + tid] = key[j];
-    auto key_at = [&](int j) { return skey[j * kDecThreads + tid]; };
+    // every thread's keys are in place before their owners read them
+    __syncthreads();
+    auto key_at = [&](int j) { return skey[tid * kKeyPitch + j]; };
 
     // every CTA has started (and CTA 0 has cleared its merge state): store the
     // slice's sums into every CTA's copy of the row histogram, then meet again
@@ -1037,7 +1057,7 @@ dsa_status launch_topk_select(const float *scores, int B, int S, int64_t T, int6
         (T + kDecSpan - 1) / kDecSpan <= kMaxCluster) {
         // the decode top-k: one cluster per row, the threshold bin from the scorer's histogram
         const int dcn = (int)((T + kDecSpan - 1) / kDecSpan);
-        const int dsmem = (int)sizeof(DecShared) + kDecSpan * (int)sizeof(uint32_t);
+        const int dsmem = (int)sizeof(DecShared) + kDecThreads * kKeyPitch * (int)sizeof(uint32_t);
         if (cudaFuncSetAttribute(topk_decode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  dsmem) != cudaSuccess ||
             (dcn > 8 && cudaFuncSetAttribute(topk_decode_kernel,
