@@ -766,13 +766,15 @@ topk_decode_kernel(const float *scores, int64_t T, int K, int32_t *__restrict__ 
     // few enough to gather
     const bool gather = n_group <= (unsigned)kDecCap && pbits < 32;
     const int gshift = 32 - pbits;
-    int n_gt = 0, n_in = 0;
+    // this thread's keys above the group and inside it, one bit per position
+    uint32_t m_gt = 0, m_in = 0;
 #pragma unroll 4
     for (int j = 0; j < nv; j++) {
         const uint32_t g = gshift == 32 ? 0u : key_at(j) >> gshift;
-        n_gt += g > prefix;
-        n_in += g == prefix;
+        m_gt |= (uint32_t)(g > prefix) << j;
+        m_in |= (uint32_t)(g == prefix) << j;
     }
+    const int n_gt = __popc(m_gt), n_in = __popc(m_in);
     int2 tot;
     const int2 ex = block_scan2_dec(n_gt, n_in, sh, &tot);
     if (tid == 0) {
@@ -786,16 +788,11 @@ topk_decode_kernel(const float *scores, int64_t T, int K, int32_t *__restrict__ 
     }
     if (gather) {
         __syncthreads();
-        if (n_in) {
-            int slot = sh.my_base + ex.y;
-#pragma unroll 4
-            for (int j = 0; j < nv; j++) {
-                const uint32_t kj = key_at(j);
-                if ((kj >> gshift) == prefix) {
-                    if (slot < kDecCap) sh0->cand[slot] = make_uint2(kj, (uint32_t)(t0 + j));
-                    slot++;
-                }
-            }
+        int slot = sh.my_base + ex.y;
+        for (uint32_t mm = m_in; mm; mm &= mm - 1u) {
+            const int j = __ffs(mm) - 1;
+            if (slot < kDecCap) sh0->cand[slot] = make_uint2(key_at(j), (uint32_t)(t0 + j));
+            slot++;
         }
     }
     cl.sync();                                   // counts and keys in CTA 0
@@ -919,31 +916,27 @@ topk_decode_kernel(const float *scores, int64_t T, int K, int32_t *__restrict__ 
     const uint32_t tau = sh.out[0];
     const int off = (int)sh.out[1], my_q = (int)sh.out[2];
 
-    // ---- ordered write of this thread's 32 positions
-    int c_gt = 0, c_eq = 0;
-#pragma unroll 4
-    for (int j = 0; j < nv; j++) {
+    // ---- ordered write of this thread's 32 positions: every key above the
+    // group is above tau; of the group's keys (few), those above tau and the
+    // lowest positions of the tau-equal ones within the quota
+    uint32_t m_sel = m_gt, m_eq = 0;
+    for (uint32_t mm = m_in; mm; mm &= mm - 1u) {
+        const int j = __ffs(mm) - 1;
         const uint32_t kj = key_at(j);
-        c_gt += kj > tau;
-        c_eq += kj == tau;
+        if (kj > tau) m_sel |= 1u << j;
+        else if (kj == tau) m_eq |= 1u << j;
     }
+    const int c_gt = __popc(m_sel), c_eq = __popc(m_eq);
     int2 tot2;
     const int2 e2 = block_scan2_dec(c_gt, c_eq, sh, &tot2);
     int take_eq = my_q - e2.y;
     take_eq = take_eq < 0 ? 0 : (take_eq > c_eq ? c_eq : take_eq);
+    for (uint32_t mm = m_eq; take_eq > 0 && mm; mm &= mm - 1u, take_eq--) m_sel |= mm & (0u - mm);
     int pos = off + e2.x + (my_q < e2.y ? my_q : e2.y);
-#pragma unroll 4
-    for (int j = 0; j < nv; j++) {
-        const uint32_t kj = key_at(j);
-        bool sel = kj > tau;
-        if (kj == tau && take_eq > 0) {
-            sel = true;
-            take_eq--;
-        }
-        if (sel && pos < m) {
-            dst[pos++] = (int32_t)(t0 + j);
-            pf(row, t0 + j);
-        }
+    for (uint32_t mm = m_sel; mm && pos < m; mm &= mm - 1u) {
+        const int j = __ffs(mm) - 1;
+        dst[pos++] = (int32_t)(t0 + j);
+        pf(row, t0 + j);
     }
     for (int i = m + p * kDecThreads + tid; i < K; i += CN * kDecThreads) dst[i] = -1;
 }
