@@ -670,6 +670,18 @@ topk_decode_kernel(const float *scores, int64_t T, int K, int32_t *__restrict__ 
             bsum[u] = acc;
         }
     }
+    // every CTA has started (and CTA 0 has cleared its merge state): store the
+    // slice's sums into every CTA's copy of the row histogram (distributed
+    // shared memory), while the score loads are still landing
+    asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
+    for (int r = 0; r < CN; r++) {
+        unsigned *peer = cl.map_shared_rank(sh.rowhist, r);
+#pragma unroll
+        for (int u = 0; u < kMaxSlice; u++) {
+            const int bb = b_lo + tid + u * kDecThreads;
+            if (bb < b_hi) peer[bb] = bsum[u];
+        }
+    }
     // the keys into shared memory: position o of the span at skey[(o / 32) * 33
     // + o % 32] (a warp's stores fall in 32 different banks; so do the owners'
     // reads of their j-th key); positions past T get key 0
@@ -693,21 +705,9 @@ topk_decode_kernel(const float *scores, int64_t T, int K, int32_t *__restrict__ 
     }
     const int64_t t0 = span0 + (int64_t)tid * kDecPer;
     const int nv = T - t0 <= 0 ? 0 : (T - t0 >= kDecPer ? kDecPer : (int)(T - t0));
-    // every thread's keys are in place before their owners read them
-    __syncthreads();
     auto key_at = [&](int j) { return skey[tid * kKeyPitch + j]; };
-
-    // every CTA has started (and CTA 0 has cleared its merge state): store the
-    // slice's sums into every CTA's copy of the row histogram, then meet again
-    asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
-    for (int r = 0; r < CN; r++) {
-        unsigned *peer = cl.map_shared_rank(sh.rowhist, r);
-#pragma unroll
-        for (int u = 0; u < kMaxSlice; u++) {
-            const int bb = b_lo + tid + u * kDecThreads;
-            if (bb < b_hi) peer[bb] = bsum[u];
-        }
-    }
+    // the row's histogram is complete in every CTA, and every thread's keys
+    // are in place before their owners read them
     cl.sync();
     // this thread's 8 bins of the row's histogram (4088 - 8t .. 4095 - 8t)
     unsigned hc[8];
