@@ -65,7 +65,7 @@ __device__ __forceinline__ void load64(const Tin *src, bool valid, float (&r)[64
 }
 
 template <int D, int R, typename Tin>
-__global__ void __launch_bounds__(256) indexer_prologue_kernel(const PrologueArgs a) {
+__global__ void __launch_bounds__(256, 2) indexer_prologue_kernel(const PrologueArgs a) {
     constexpr int G = D / 64;                  // lanes per vector
     const int lane = threadIdx.x & 31;
     const int part = lane % G;

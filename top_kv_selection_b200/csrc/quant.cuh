@@ -104,42 +104,78 @@ __device__ __forceinline__ uint32_t rotate_quant_warp(float (&r)[D / 32], float 
 // lane pair L, L ^ 1.  Every lane of the warp must call it (lanes of a vector
 // that does not exist pass zeros).  codes[j] holds the e4m3 codes of elements
 // 4j .. 4j + 3 of this lane's slice, little-endian.
+//
+// Stages h >= 2, the scaling and the division run on packed fp32 pairs (one
+// instruction for two elements, each rounded as the scalar operation would
+// be: a - b as a + (-b), p - a as fma(a, -1, p), fma(-q0, s, x) as
+// fma(q0, -s, x)), so the results are bit-identical to the scalar form.
 template <int D>
 __device__ __forceinline__ void rotate_quant_lanes(float (&r)[64], uint32_t (&codes)[16],
                                                    float *scale, bool ue8m0 = false) {
     static_assert(D == 64 || D == 128, "one or two lanes per vector");
 #pragma unroll
-    for (int h = 1; h < 64; h <<= 1) {
+    for (int e = 0; e < 64; e += 2) {
+        const float a = r[e], b = r[e + 1];
+        r[e] = a + b;
+        r[e + 1] = a - b;
+    }
 #pragma unroll
-        for (int e = 0; e < 64; e++) {
+    for (int h = 2; h < 64; h <<= 1) {
+#pragma unroll
+        for (int e = 0; e < 64; e += 2) {
             if (e & h) continue;
-            const float a = r[e], b = r[e + h];
-            r[e] = a + b;
-            r[e + h] = a - b;
+            const float2 a = make_float2(r[e], r[e + 1]);
+            const float2 b = make_float2(r[e + h], r[e + h + 1]);
+            const float2 sum = __fadd2_rn(a, b);
+            const float2 dif = __fadd2_rn(a, make_float2(-b.x, -b.y));
+            r[e] = sum.x;
+            r[e + 1] = sum.y;
+            r[e + h] = dif.x;
+            r[e + h + 1] = dif.y;
         }
     }
     if constexpr (D == 128) {
-        const bool upper = (threadIdx.x & 1) != 0;
+        // lower lane: a + p; upper lane: p - a = fma(a, -1, p)
+        const float sg = (threadIdx.x & 1) ? -1.f : 1.f;
+        const float2 sg2 = make_float2(sg, sg);
 #pragma unroll
-        for (int e = 0; e < 64; e++) {
-            const float p = __shfl_xor_sync(0xffffffffu, r[e], 1);
-            r[e] = upper ? __fsub_rn(p, r[e]) : __fadd_rn(r[e], p);
+        for (int e = 0; e < 64; e += 2) {
+            const float2 p = make_float2(__shfl_xor_sync(0xffffffffu, r[e], 1),
+                                         __shfl_xor_sync(0xffffffffu, r[e + 1], 1));
+            const float2 v = __ffma2_rn(make_float2(r[e], r[e + 1]), sg2, p);
+            r[e] = v.x;
+            r[e + 1] = v.y;
         }
     }
-    float amax = 0.f;
+    const float2 hs = make_float2(HadamardScale<D>::value, HadamardScale<D>::value);
+    float am0 = 0.f, am1 = 0.f;
 #pragma unroll
-    for (int e = 0; e < 64; e++) {
-        r[e] = __fmul_rn(r[e], HadamardScale<D>::value);
-        amax = fmaxf(amax, fabsf(r[e]));
+    for (int e = 0; e < 64; e += 2) {
+        const float2 v = __fmul2_rn(make_float2(r[e], r[e + 1]), hs);
+        r[e] = v.x;
+        r[e + 1] = v.y;
+        am0 = fmaxf(am0, fabsf(v.x));
+        am1 = fmaxf(am1, fabsf(v.y));
     }
+    float amax = fmaxf(am0, am1);
     if constexpr (D == 128) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
     float s = __fdiv_rn(fmaxf(amax, 1e-4f), 448.0f);
     if (ue8m0) s = pow2_ceil(s);
     const float rs = __frcp_rn(s);
+    // x / s correctly rounded, two at a time (div_rn_by on each element)
+    const float2 rs2 = make_float2(rs, rs), ns2 = make_float2(-s, -s);
+    auto div2 = [&](float x0, float x1) {
+        const float2 x = make_float2(x0, x1);
+        const float2 q0 = __fmul2_rn(x, rs2);
+        const float2 er = __ffma2_rn(q0, ns2, x);
+        return __ffma2_rn(er, rs2, q0);
+    };
 #pragma unroll
-    for (int j = 0; j < 16; j++)
-        codes[j] = e4m3x2_rn_sat(div_rn_by(r[4 * j], s, rs), div_rn_by(r[4 * j + 1], s, rs)) |
-                   e4m3x2_rn_sat(div_rn_by(r[4 * j + 2], s, rs), div_rn_by(r[4 * j + 3], s, rs)) << 16;
+    for (int j = 0; j < 16; j++) {
+        const float2 lo = div2(r[4 * j], r[4 * j + 1]);
+        const float2 hi = div2(r[4 * j + 2], r[4 * j + 3]);
+        codes[j] = e4m3x2_rn_sat(lo.x, lo.y) | e4m3x2_rn_sat(hi.x, hi.y) << 16;
+    }
     *scale = s;
 }
 
