@@ -39,53 +39,186 @@ struct PrologueArgs {
     int64_t start_pos, t_max;
     int B, S, H, R;
     int ue8m0;
+    int small;              // every vector index fits in 31 bits
 };
 
-// Loads 64 contiguous elements (fp32 or bf16) as fp32; zeros when !valid.
-template <typename Tin>
-__device__ __forceinline__ void load64(const Tin *src, bool valid, float (&r)[64]) {
-    if constexpr (sizeof(Tin) == 4) {
+// A warp's vectors pass through shared memory: the warp copies them with
+// coalesced 16-byte cp.async pieces (consecutive lanes, consecutive pieces), and
+// lane o, which owns 64 elements of one vector, then reads its CPL pieces.
+// Piece j of owner o sits at slot o * CPL + (j ^ (o % 8)): both the copies
+// (8 consecutive lanes hit 8 different 16-byte bank groups) and the owners'
+// reads (lanes o .. o + 7 at the same j, likewise) are free of bank conflicts.
+// Two buffers per warp: the next vectors are in flight while these are
+// rotated.
+__device__ __forceinline__ void cp_async16_zfill(uint32_t dst, const void *src, bool valid) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src),
+                 "r"(valid ? 16u : 0u)
+                 : "memory");
+}
+
+template <int D, typename Tin> struct Stage {
+    static constexpr int G = D / 64;                        // lanes per vector
+    static constexpr int kVecs = 32 / G;                    // vectors per warp and pass
+    static constexpr int kVecBytes = D * (int)sizeof(Tin);
+    static constexpr int kBytes = kVecs * kVecBytes;        // one buffer
+    static constexpr int kCPL = 64 * (int)sizeof(Tin) / 16; // pieces a lane owns (8 or 16)
+    static constexpr int kPieces = kBytes / 16;
+
+    // copies the vectors [base, base + kVecs) (zeros past `total`) into buf
+    __device__ __forceinline__ static void issue(uint32_t buf, const PrologueArgs &a, int64_t base,
+                                                 int64_t nq, int64_t total, int lane) {
+        constexpr int kPerVec = kVecBytes / 16;
 #pragma unroll
-        for (int i = 0; i < 16; i++) {
-            const float4 t = valid ? reinterpret_cast<const float4 *>(src)[i] : make_float4(0.f, 0.f, 0.f, 0.f);
-            r[4 * i] = t.x; r[4 * i + 1] = t.y; r[4 * i + 2] = t.z; r[4 * i + 3] = t.w;
+        for (int i = 0; i < kPieces / 32; i++) {
+            const int c = lane + 32 * i;
+            const int64_t v = base + c / kPerVec;
+            const int off = (c % kPerVec) * 16;
+            const bool valid = v < total;
+            const uint8_t *src =
+                v < nq ? static_cast<const uint8_t *>(a.q) + v * kVecBytes
+                       : static_cast<const uint8_t *>(a.k) + (valid ? v - nq : 0) * kVecBytes;
+            const int o = c / kCPL, j = c % kCPL;
+            cp_async16_zfill(buf + (uint32_t)(o * kCPL + (j ^ (o & 7))) * 16u, src + off, valid);
         }
-    } else {
+    }
+    // lane o's 64 elements from buf, as fp32
+    __device__ __forceinline__ static void read(uint32_t buf, int o, float (&r)[64]) {
 #pragma unroll
-        for (int i = 0; i < 8; i++) {
-            const uint4 t = valid ? reinterpret_cast<const uint4 *>(src)[i] : make_uint4(0u, 0u, 0u, 0u);
-            const uint32_t w[4] = {t.x, t.y, t.z, t.w};
+        for (int j = 0; j < kCPL; j++) {
+            uint4 t;
+            asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+                         : "=r"(t.x), "=r"(t.y), "=r"(t.z), "=r"(t.w)
+                         : "r"(buf + (uint32_t)(o * kCPL + (j ^ (o & 7))) * 16u));
+            if constexpr (sizeof(Tin) == 4) {
+                r[4 * j] = __uint_as_float(t.x);
+                r[4 * j + 1] = __uint_as_float(t.y);
+                r[4 * j + 2] = __uint_as_float(t.z);
+                r[4 * j + 3] = __uint_as_float(t.w);
+            } else {
+                const uint32_t w[4] = {t.x, t.y, t.z, t.w};
 #pragma unroll
-            for (int h = 0; h < 4; h++) {
-                r[8 * i + 2 * h] = __uint_as_float(w[h] << 16);
-                r[8 * i + 2 * h + 1] = __uint_as_float(w[h] & 0xFFFF0000u);
+                for (int h = 0; h < 4; h++) {
+                    r[8 * j + 2 * h] = __uint_as_float(w[h] << 16);
+                    r[8 * j + 2 * h + 1] = __uint_as_float(w[h] & 0xFFFF0000u);
+                }
             }
         }
+    }
+};
+
+// Token (b * S + s) of query vector v, and the position s of vector v's token
+// (a query head vector or a key); 32-bit arithmetic when the problem fits.
+__device__ __forceinline__ int64_t token_of(const PrologueArgs &a, int64_t v) {
+    return a.small ? (int64_t)((uint32_t)v / (uint32_t)a.H) : v / a.H;
+}
+__device__ __forceinline__ int token_pos(const PrologueArgs &a, int64_t v, int64_t nq,
+                                         int64_t total) {
+    if (v >= total) return 0;
+    const int64_t t = v < nq ? token_of(a, v) : v - nq;
+    return a.small ? (int)((uint32_t)t % (uint32_t)a.S) : (int)(t % a.S);
+}
+
+// Two fp32 products rounded to nearest, never fused into a following add
+// (an explicit rounding mode keeps ptxas from contracting it into an fma).
+__device__ __forceinline__ float2 mul2_rn(float2 a, float2 b) {
+    float2 r;
+    asm("{\n\t.reg .b64 pa, pb, pr;\n\t"
+        "mov.b64 pa, {%2, %3};\n\tmov.b64 pb, {%4, %5};\n\t"
+        "mul.rn.f32x2 pr, pa, pb;\n\tmov.b64 {%0, %1}, pr;\n\t}"
+        : "=f"(r.x), "=f"(r.y)
+        : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+    return r;
+}
+
+// The angles of a pass whose vectors are all query heads of at most two
+// tokens (every pass when H >= 16 and H divides by 16) are copied next to its
+// vectors: rows t_lo and t_lo + 1 of the table, R floats pairs each; other
+// passes (the keys, few heads) read the table directly.
+__device__ __forceinline__ bool angles_staged(const PrologueArgs &a, int64_t base, int n,
+                                              int64_t nq, int64_t *t_lo) {
+    if (base + n > nq) return false;
+    const int64_t t0 = token_of(a, base), t1 = token_of(a, base + n - 1);
+    *t_lo = t0;
+    return t1 - t0 <= 1;
+}
+template <int R>
+__device__ __forceinline__ void issue_angles(uint32_t dst, const PrologueArgs &a, int64_t base,
+                                             int n, int64_t nq, int lane) {
+    int64_t t_lo;
+    if (!angles_staged(a, base, n, nq, &t_lo)) return;
+    const bool two = token_of(a, base + n - 1) > t_lo;
+    constexpr int kPer = R / 4;                  // 16-byte pieces per row
+#pragma unroll
+    for (int c = lane; c < 2 * kPer; c += 32) {
+        const int row = c / kPer;
+        const int64_t t = t_lo + row;
+        const int sp = row == 0 || two ? (a.small ? (int)((uint32_t)t % (uint32_t)a.S) : (int)(t % a.S)) : 0;
+        cp_async16_zfill(dst + (uint32_t)c * 16u, a.cs + (int64_t)sp * R + (c % kPer) * 4,
+                         row == 0 || two);
     }
 }
 
 template <int D, int R, typename Tin>
 __global__ void __launch_bounds__(256, 2) indexer_prologue_kernel(const PrologueArgs a) {
+    using St = Stage<D, Tin>;
     constexpr int G = D / 64;                  // lanes per vector
+    extern __shared__ __align__(16) uint8_t stage_smem[];
     const int lane = threadIdx.x & 31;
     const int part = lane % G;
     const int64_t nq = (int64_t)a.B * a.S * a.H;
     const int64_t total = nq + (int64_t)a.B * a.S;
-    const int64_t per_warp = 32 / G;
+    const int64_t per_warp = St::kVecs;
     const int64_t warps = (int64_t)gridDim.x * (blockDim.x >> 5);
-    for (int64_t base = ((int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5)) * per_warp;
-         base < total; base += warps * per_warp) {
+    const int64_t stride = warps * per_warp;
+    const int warp = threadIdx.x >> 5;
+    const uint32_t buf0 = (uint32_t)__cvta_generic_to_shared(stage_smem) +
+                          (uint32_t)(warp * 2 * St::kBytes);
+    // the staged angles: after the 8 warps' vector buffers, two rows per buffer
+    constexpr int kAngBytes = 2 * (R > 0 ? R : 4) * 4;
+    const int ang_off = 8 * 2 * St::kBytes + warp * 2 * kAngBytes;
+    const uint32_t ang0 = (uint32_t)__cvta_generic_to_shared(stage_smem) + (uint32_t)ang_off;
+    int64_t base = ((int64_t)blockIdx.x * (blockDim.x >> 5) + warp) * per_warp;
+    if (base < total) {
+        St::issue(buf0, a, base, nq, total, lane);
+        if constexpr (R > 0) issue_angles<R>(ang0, a, base, St::kVecs, nq, lane);
+        asm volatile("cp.async.commit_group;" ::: "memory");
+    }
+    for (int it = 0; base < total; base += stride, it++) {
+        const uint32_t cur = buf0 + (uint32_t)((it & 1) * St::kBytes);
+        // the next pass's vectors (and angles) into the other buffer (its reads
+        // ended at the __syncwarp of the previous pass), then this pass's pieces
+        if (base + stride < total) {
+            const int nb = (it + 1) & 1;
+            St::issue(buf0 + (uint32_t)(nb * St::kBytes), a, base + stride, nq, total, lane);
+            if constexpr (R > 0)
+                issue_angles<R>(ang0 + (uint32_t)(nb * kAngBytes), a, base + stride, St::kVecs, nq,
+                                lane);
+            asm volatile("cp.async.commit_group;" ::: "memory");
+            asm volatile("cp.async.wait_group 1;" ::: "memory");
+        } else {
+            asm volatile("cp.async.wait_group 0;" ::: "memory");
+        }
+        __syncwarp();
         const int64_t v = base + lane / G;   // both lanes of a vector agree on `valid`
         const bool valid = v < total;
         const bool is_q = v < nq;
-        const int64_t t = is_q ? v / a.H : v - nq;   // token index b * S + s
-        const int s = valid ? (int)(t % a.S) : 0;
+        const int64_t t = is_q ? token_of(a, v) : v - nq;   // token index b * S + s
+        const int s = valid ? token_pos(a, v, nq, total) : 0;
         float r[64];
-        if (is_q) load64<Tin>(static_cast<const Tin *>(a.q) + v * D + part * 64, valid, r);
-        else load64<Tin>(static_cast<const Tin *>(a.k) + t * D + part * 64, valid, r);
+        St::read(cur, lane, r);
+        // this vector's angles: the staged copy, or the table
+        const float4 *cs = nullptr;
+        if constexpr (R > 0) {
+            int64_t t_lo = 0;
+            cs = angles_staged(a, base, St::kVecs, nq, &t_lo)
+                     ? reinterpret_cast<const float4 *>(stage_smem + ang_off + (it & 1) * kAngBytes +
+                                                        (int)(t - t_lo) * R * 4)
+                     : reinterpret_cast<const float4 *>(a.cs + (int64_t)s * R);
+        }
         if constexpr (R > 0 && R <= 64) {
             if (part == 0 && valid) {
-                const float4 *cs = reinterpret_cast<const float4 *>(a.cs + (int64_t)s * R);
+                // lower x1 c - x2 s, upper x1 s + x2 c, each product and sum
+                // rounded once: two packed products and a packed sum
 #pragma unroll
                 for (int j2 = 0; j2 < R / 4; j2++) {            // two frequencies per float4
                     const float4 c2 = cs[j2];
@@ -101,7 +234,6 @@ __global__ void __launch_bounds__(256, 2) indexer_prologue_kernel(const Prologue
             }
         } else if constexpr (R == 128) {
             static_assert(D == 128, "rotary part within the vector");
-            const float4 *cs = reinterpret_cast<const float4 *>(a.cs + (int64_t)s * R);
             const bool upper = part == 1;
 #pragma unroll
             for (int j2 = 0; j2 < 32; j2++) {
@@ -116,6 +248,8 @@ __global__ void __launch_bounds__(256, 2) indexer_prologue_kernel(const Prologue
                 }
             }
         }
+        // every lane is done with this pass's buffer (vectors and angles)
+        __syncwarp();
         uint32_t codes[16];
         float sc;
         rotate_quant_lanes<D>(r, codes, &sc, a.ue8m0 != 0);
@@ -126,7 +260,8 @@ __global__ void __launch_bounds__(256, 2) indexer_prologue_kernel(const Prologue
                 dst = a.q_fp8 + v * D;
                 dscale = a.q_scale + v;
             } else {
-                const int64_t row = (t / a.S) * a.t_max + a.start_pos + s;
+                const int64_t bb = a.small ? (int64_t)((uint32_t)t / (uint32_t)a.S) : t / a.S;
+                const int64_t row = bb * a.t_max + a.start_pos + s;
                 dst = a.k_cache + row * D;
                 dscale = a.k_scale + row;
             }
@@ -141,12 +276,20 @@ __global__ void __launch_bounds__(256, 2) indexer_prologue_kernel(const Prologue
 
 template <int D, int R, typename Tin>
 dsa_status launch_r(const PrologueArgs &a, cudaStream_t stream) {
+    using St = Stage<D, Tin>;
     const int64_t total = (int64_t)a.B * a.S * (a.H + 1);
-    const int64_t per_block = 8 * (32 / (D / 64));
+    const int64_t per_block = 8 * St::kVecs;
     int64_t blocks = (total + per_block - 1) / per_block;
-    const int64_t cap = (int64_t)num_sms() * 16;
+    const size_t smem = (size_t)8 * 2 * St::kBytes + (size_t)8 * 2 * (2 * (R > 0 ? R : 4) * 4);
+    // every SM holds as many CTAs as its shared memory and registers allow;
+    // the warps stride over the vectors
+    const int per_sm = smem * 2 <= 227 * 1024 ? 2 : 1;
+    const int64_t cap = (int64_t)num_sms() * per_sm;
     if (blocks > cap) blocks = cap;
-    indexer_prologue_kernel<D, R, Tin><<<(unsigned)blocks, 256, 0, stream>>>(a);
+    if (cudaFuncSetAttribute(indexer_prologue_kernel<D, R, Tin>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
+        return DSA_ERR_CUDA;
+    indexer_prologue_kernel<D, R, Tin><<<(unsigned)blocks, 256, smem, stream>>>(a);
     return launch_status();
 }
 
@@ -208,6 +351,7 @@ extern "C" dsa_status dsa_indexer_prologue(const void *q, const void *k, dsa_dty
     a.H = H;
     a.R = rope_dim;
     a.ue8m0 = scale_fmt == DSA_SCALE_UE8M0 ? 1 : 0;
+    a.small = (int64_t)B * S * ((int64_t)H + 1) + 64 <= INT32_MAX ? 1 : 0;
     const cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     const bool bf = x_dtype == DSA_BF16;
     if (d == 128)
