@@ -56,7 +56,7 @@ __device__ __forceinline__ void cp_async16_zfill(uint32_t dst, const void *src, 
                  : "memory");
 }
 
-template <int D, typename Tin> struct Stage {
+template <int D, typename Tin, int X> struct Stage {
     static constexpr int G = D / 64;                        // lanes per vector
     static constexpr int kVecs = 32 / G;                    // vectors per warp and pass
     static constexpr int kVecBytes = D * (int)sizeof(Tin);
@@ -68,16 +68,22 @@ template <int D, typename Tin> struct Stage {
     __device__ __forceinline__ static void issue(uint32_t buf, const PrologueArgs &a, int64_t base,
                                                  int64_t nq, int64_t total, int lane) {
         constexpr int kPerVec = kVecBytes / 16;
+        constexpr int kEPC = 16 / (int)sizeof(Tin);           // elements per piece
+        static_assert(G == 1 || kEPC <= (1 << X), "a piece stays within one lane's elements");
 #pragma unroll
         for (int i = 0; i < kPieces / 32; i++) {
             const int c = lane + 32 * i;
             const int64_t v = base + c / kPerVec;
-            const int off = (c % kPerVec) * 16;
+            const int cc = c % kPerVec, off = cc * 16;
             const bool valid = v < total;
             const uint8_t *src =
                 v < nq ? static_cast<const uint8_t *>(a.q) + v * kVecBytes
                        : static_cast<const uint8_t *>(a.k) + (valid ? v - nq : 0) * kVecBytes;
-            const int o = c / kCPL, j = c % kCPL;
+            // owner lane (vector, part) and the piece's place among its registers
+            const int e0 = cc * kEPC;
+            const int p = G == 2 ? (e0 >> X) & 1 : 0;
+            const int i0 = G == 2 ? ((e0 >> (X + 1)) << X) | (e0 & ((1 << X) - 1)) : e0;
+            const int o = (c / kPerVec) * G + p, j = i0 / kEPC;
             cp_async16_zfill(buf + (uint32_t)(o * kCPL + (j ^ (o & 7))) * 16u, src + off, valid);
         }
     }
@@ -158,9 +164,22 @@ __device__ __forceinline__ void issue_angles(uint32_t dst, const PrologueArgs &a
     }
 }
 
+// The lane split of a 128-vector for rotary part R: on the bit just below the
+// rotary pair's bit, so that both lanes of a vector hold half of the pairs
+// (element j and j + R/2 in the same lane); bit 6 (contiguous halves) when
+// the part is too short for a 16-byte piece to stay in one lane.
+template <int D, int R, typename Tin> constexpr int lane_split() {
+    if (D != 128) return 6;
+    if (R == 128) return 5;
+    if (R == 64) return 4;
+    if (R == 32 && sizeof(Tin) == 2) return 3;
+    return 6;
+}
+
 template <int D, int R, typename Tin>
 __global__ void __launch_bounds__(256, 2) indexer_prologue_kernel(const PrologueArgs a) {
-    using St = Stage<D, Tin>;
+    constexpr int X = lane_split<D, R, Tin>();
+    using St = Stage<D, Tin, X>;
     constexpr int G = D / 64;                  // lanes per vector
     extern __shared__ __align__(16) uint8_t stage_smem[];
     const int lane = threadIdx.x & 31;
@@ -215,7 +234,26 @@ __global__ void __launch_bounds__(256, 2) indexer_prologue_kernel(const Prologue
                                                         (int)(t - t_lo) * R * 4)
                      : reinterpret_cast<const float4 *>(a.cs + (int64_t)s * R);
         }
-        if constexpr (R > 0 && R <= 64) {
+        if constexpr (R > 0 && X < 6) {
+            // both lanes: pairs (register m, register 2^X + m), m < 2^X, at
+            // frequency part * 2^X + m
+            if (valid) {
+                constexpr int M = 1 << X;
+                const float4 *cp = cs + part * (M / 2);
+#pragma unroll
+                for (int m2 = 0; m2 < M / 2; m2++) {
+                    const float4 c2 = cp[m2];
+                    const float cc[2] = {c2.x, c2.z}, ss[2] = {c2.y, c2.w};
+#pragma unroll
+                    for (int u = 0; u < 2; u++) {
+                        const int m = 2 * m2 + u;
+                        const float x1 = r[m], x2 = r[M + m];
+                        r[m] = __fsub_rn(__fmul_rn(x1, cc[u]), __fmul_rn(x2, ss[u]));
+                        r[M + m] = __fadd_rn(__fmul_rn(x1, ss[u]), __fmul_rn(x2, cc[u]));
+                    }
+                }
+            }
+        } else if constexpr (R > 0 && R <= 64) {
             if (part == 0 && valid) {
                 // lower x1 c - x2 s, upper x1 s + x2 c, each product and sum
                 // rounded once: two packed products and a packed sum
@@ -252,7 +290,7 @@ __global__ void __launch_bounds__(256, 2) indexer_prologue_kernel(const Prologue
         __syncwarp();
         uint32_t codes[16];
         float sc;
-        rotate_quant_lanes<D>(r, codes, &sc, a.ue8m0 != 0);
+        rotate_quant_lanes<D, X>(r, codes, &sc, a.ue8m0 != 0);
         if (valid) {
             uint8_t *dst;
             float *dscale;
@@ -265,10 +303,11 @@ __global__ void __launch_bounds__(256, 2) indexer_prologue_kernel(const Prologue
                 dst = a.k_cache + row * D;
                 dscale = a.k_scale + row;
             }
-            uint4 *d4 = reinterpret_cast<uint4 *>(dst + part * 64);
+            // registers 16i .. 16i + 15 are 16 consecutive elements
 #pragma unroll
             for (int i = 0; i < 4; i++)
-                d4[i] = make_uint4(codes[4 * i], codes[4 * i + 1], codes[4 * i + 2], codes[4 * i + 3]);
+                *reinterpret_cast<uint4 *>(dst + (G == 2 ? split_element<X>(16 * i, part) : 16 * i)) =
+                    make_uint4(codes[4 * i], codes[4 * i + 1], codes[4 * i + 2], codes[4 * i + 3]);
             if (part == 0) *dscale = sc;
         }
     }
@@ -276,7 +315,7 @@ __global__ void __launch_bounds__(256, 2) indexer_prologue_kernel(const Prologue
 
 template <int D, int R, typename Tin>
 dsa_status launch_r(const PrologueArgs &a, cudaStream_t stream) {
-    using St = Stage<D, Tin>;
+    using St = Stage<D, Tin, lane_split<D, R, Tin>()>;
     const int64_t total = (int64_t)a.B * a.S * (a.H + 1);
     const int64_t per_block = 8 * St::kVecs;
     int64_t blocks = (total + per_block - 1) / per_block;

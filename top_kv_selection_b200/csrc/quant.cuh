@@ -98,53 +98,65 @@ __device__ __forceinline__ uint32_t rotate_quant_warp(float (&r)[D / 32], float 
 }
 
 // The same rotation and quantisation with the vector split over G = D / 64
-// adjacent lanes, 64 contiguous elements each (lane part p holds elements
-// [64p, 64p + 64)).  Stages h = 1 .. 32 stay in registers; for D = 128 the last
-// stage h = 64 pairs part 0 (lower: a + b) with part 1 (upper: a - b) of the
-// lane pair L, L ^ 1.  Every lane of the warp must call it (lanes of a vector
-// that does not exist pass zeros).  codes[j] holds the e4m3 codes of elements
-// 4j .. 4j + 3 of this lane's slice, little-endian.
+// adjacent lanes, 64 elements each.  For D = 128 the lane pair splits the
+// vector on element bit X: lane part p holds the elements whose bit X is p, in
+// register order (register i holds element ((i >> X) << (X + 1)) | (p << X) |
+// (i & (2^X - 1)); X = 6, the default, gives part p the elements
+// [64p, 64p + 64)).  Butterfly stages run over element bits 0, 1, ..., D-1's
+// top bit in that order; the stage on bit X pairs the two lanes (the lane
+// holding the lower element takes a + b, the other a - b), every other stage
+// pairs two registers of a lane.  Every lane of the warp must call it (lanes
+// of a vector that does not exist pass zeros).  codes[j] holds the e4m3 codes
+// of registers 4j .. 4j + 3, little-endian.
 //
-// Stages h >= 2, the scaling and the division run on packed fp32 pairs (one
-// instruction for two elements, each rounded as the scalar operation would
-// be: a - b as a + (-b), p - a as fma(a, -1, p), fma(-q0, s, x) as
-// fma(q0, -s, x)), so the results are bit-identical to the scalar form.
-template <int D>
+// Stages on register strides >= 2, the scaling and the division run on packed
+// fp32 pairs (one instruction for two elements, each rounded as the scalar
+// operation would be: a - b as a + (-b), p - a as fma(a, -1, p),
+// fma(-q0, s, x) as fma(q0, -s, x)), so the results are bit-identical to the
+// scalar form.
+template <int D, int X = 6>
 __device__ __forceinline__ void rotate_quant_lanes(float (&r)[64], uint32_t (&codes)[16],
                                                    float *scale, bool ue8m0 = false) {
     static_assert(D == 64 || D == 128, "one or two lanes per vector");
+    static_assert(D == 64 ? X == 6 : (X >= 1 && X <= 6), "lane split bit");
+    constexpr int kBits = D == 128 ? 7 : 6;
 #pragma unroll
-    for (int e = 0; e < 64; e += 2) {
-        const float a = r[e], b = r[e + 1];
-        r[e] = a + b;
-        r[e + 1] = a - b;
-    }
+    for (int b = 0; b < kBits; b++) {
+        if (D == 128 && b == X) {
+            // lower lane: a + p; upper lane: p - a = fma(a, -1, p)
+            const float sg = (threadIdx.x & 1) ? -1.f : 1.f;
+            const float2 sg2 = make_float2(sg, sg);
 #pragma unroll
-    for (int h = 2; h < 64; h <<= 1) {
-#pragma unroll
-        for (int e = 0; e < 64; e += 2) {
-            if (e & h) continue;
-            const float2 a = make_float2(r[e], r[e + 1]);
-            const float2 b = make_float2(r[e + h], r[e + h + 1]);
-            const float2 sum = __fadd2_rn(a, b);
-            const float2 dif = __fadd2_rn(a, make_float2(-b.x, -b.y));
-            r[e] = sum.x;
-            r[e + 1] = sum.y;
-            r[e + h] = dif.x;
-            r[e + h + 1] = dif.y;
+            for (int e = 0; e < 64; e += 2) {
+                const float2 p = make_float2(__shfl_xor_sync(0xffffffffu, r[e], 1),
+                                             __shfl_xor_sync(0xffffffffu, r[e + 1], 1));
+                const float2 v = __ffma2_rn(make_float2(r[e], r[e + 1]), sg2, p);
+                r[e] = v.x;
+                r[e + 1] = v.y;
+            }
+            continue;
         }
-    }
-    if constexpr (D == 128) {
-        // lower lane: a + p; upper lane: p - a = fma(a, -1, p)
-        const float sg = (threadIdx.x & 1) ? -1.f : 1.f;
-        const float2 sg2 = make_float2(sg, sg);
+        const int h = (D == 128 && b > X) ? 1 << (b - 1) : 1 << b;   // register stride
+        if (h == 1) {
 #pragma unroll
-        for (int e = 0; e < 64; e += 2) {
-            const float2 p = make_float2(__shfl_xor_sync(0xffffffffu, r[e], 1),
-                                         __shfl_xor_sync(0xffffffffu, r[e + 1], 1));
-            const float2 v = __ffma2_rn(make_float2(r[e], r[e + 1]), sg2, p);
-            r[e] = v.x;
-            r[e + 1] = v.y;
+            for (int e = 0; e < 64; e += 2) {
+                const float a = r[e], c = r[e + 1];
+                r[e] = a + c;
+                r[e + 1] = a - c;
+            }
+        } else {
+#pragma unroll
+            for (int e = 0; e < 64; e += 2) {
+                if (e & h) continue;
+                const float2 a = make_float2(r[e], r[e + 1]);
+                const float2 c = make_float2(r[e + h], r[e + h + 1]);
+                const float2 sum = __fadd2_rn(a, c);
+                const float2 dif = __fadd2_rn(a, make_float2(-c.x, -c.y));
+                r[e] = sum.x;
+                r[e + 1] = sum.y;
+                r[e + h] = dif.x;
+                r[e + h + 1] = dif.y;
+            }
         }
     }
     const float2 hs = make_float2(HadamardScale<D>::value, HadamardScale<D>::value);
@@ -177,6 +189,12 @@ __device__ __forceinline__ void rotate_quant_lanes(float (&r)[64], uint32_t (&co
         codes[j] = e4m3x2_rn_sat(lo.x, lo.y) | e4m3x2_rn_sat(hi.x, hi.y) << 16;
     }
     *scale = s;
+}
+
+// Element of register i of lane part p under the lane split on bit X.
+template <int X>
+__host__ __device__ constexpr int split_element(int i, int p) {
+    return ((i >> X) << (X + 1)) | (p << X) | (i & ((1 << X) - 1));
 }
 
 // Loads this lane's E elements of a D-vector (fp32 or bf16).
