@@ -64,6 +64,9 @@ def _run(dsa, B, S, H, d, R, dtype, fmt, start_pos, t_max, seed, scale=1.0):
     (1, 4, 8, 128, 8, torch.bfloat16, 0, 2, 9),            # smallest rotary part
     (1, 4, 8, 128, 0, torch.float32, 1, 2, 10),            # no rotary part, ue8m0
     (3, 2, 0, 64, 32, torch.bfloat16, 0, 5, 9),            # keys only
+    (1, 6, 16, 128, 32, torch.bfloat16, 0, 3, 12),         # lanes split on bit 3, angles staged
+    (1, 6, 16, 128, 32, torch.float32, 1, 3, 12),          # rotary 32 in fp32: contiguous halves
+    (2, 3, 5, 128, 16, torch.bfloat16, 0, 0, 5),           # few heads: angles read from the table
 ])
 def test_prologue_matches_oracle(dsa, B, S, H, d, R, dtype, fmt, start_pos, t_max):
     _run(dsa, B, S, H, d, R, dtype, fmt, start_pos, t_max, seed=B * 100 + S * 10 + H + R)

@@ -24,12 +24,12 @@
 // The producer starts streaming at once; the query operand is built in
 // parallel by the epilogue warps, either from given FP8 codes or -- in the
 // decode step -- by rotating and quantising the new token's fp32 queries
-// (rotate_activation + act_quant, bit-identical to dsa_indexer_quant).  Their
-// global loads are issued at kernel entry, before the key stream fills the
-// memory queues, and the rotation keeps 64 elements per lane so that it is
-// almost all register arithmetic.  In the decode step the CTA holding position
-// T-1 also quantises the new key and appends it to the cache (the cache write
-// of Indexer.forward) before its last tile is fetched.
+// (rotate_activation + act_quant, bit-identical to dsa_indexer_quant).  The
+// fp32 query row arrives by TMA (swizzled boxes) right after the dependency
+// wait, ahead of the key stream, and the rotation keeps 64 elements per lane
+// so that it is almost all register arithmetic.  In the decode step the CTA
+// holding position T-1 also quantises the new key and appends it to the cache
+// (the cache write of Indexer.forward) before its last tile is fetched.
 #include "common.cuh"
 #include "quant.cuh"
 #include "tc_ptx.cuh"

@@ -303,11 +303,20 @@ __global__ void __launch_bounds__(256, 2) indexer_prologue_kernel(const Prologue
                 dst = a.k_cache + row * D;
                 dscale = a.k_scale + row;
             }
-            // registers 16i .. 16i + 15 are 16 consecutive elements
+            // registers run k .. run k + run - 1 are consecutive elements, run =
+            // min(16, 2^X) under the lane split (contiguous halves: 16)
+            static_assert(G == 1 || X >= 3, "8-code runs at least");
+            if constexpr (G == 2 && X == 3) {
 #pragma unroll
-            for (int i = 0; i < 4; i++)
-                *reinterpret_cast<uint4 *>(dst + (G == 2 ? split_element<X>(16 * i, part) : 16 * i)) =
-                    make_uint4(codes[4 * i], codes[4 * i + 1], codes[4 * i + 2], codes[4 * i + 3]);
+                for (int m = 0; m < 8; m++)
+                    *reinterpret_cast<uint2 *>(dst + split_element<X>(8 * m, part)) =
+                        make_uint2(codes[2 * m], codes[2 * m + 1]);
+            } else {
+#pragma unroll
+                for (int i = 0; i < 4; i++)
+                    *reinterpret_cast<uint4 *>(dst + (G == 2 ? split_element<X>(16 * i, part) : 16 * i)) =
+                        make_uint4(codes[4 * i], codes[4 * i + 1], codes[4 * i + 2], codes[4 * i + 3]);
+            }
             if (part == 0) *dscale = sc;
         }
     }

@@ -477,7 +477,9 @@ topk_cluster_kernel(const float *scores, int S, int64_t T, int64_t start_pos, in
 // ------------------------------------------------------------ decode top-k
 // The decode step's top-k, when the scorer's CTAs have counted their scores
 // by the top 12 key bits: a cluster of CN CTAs of 512 threads per row, each
-// thread holding 32 consecutive positions' keys in registers.  CTA p sums its
+// thread owning 32 consecutive positions (their keys in shared memory, loaded
+// as coalesced float4s; the thread keeps bitmasks of which are above the
+// threshold bin and which fall in it).  CTA p sums its
 // slice of the bins over the row's scorer histograms and stores the sums into
 // every CTA of the cluster, so that after one cluster barrier every CTA holds
 // the row's histogram and finds the same 12-bit threshold bin on its own; the
