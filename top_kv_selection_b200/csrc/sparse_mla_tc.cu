@@ -19,14 +19,14 @@
 //   2. runs an exact softmax over the unit's 128 logits of each head (the
 //      thread's logits stay in registers between the max and the exp2 pass)
 //      and writes P as bf16 into shared memory, the A operand of the value mix;
-//   3. accumulates O = P C[:, 0:512] as two N = 256 halves (M = 128, K = 128)
-//      whose B operands are the latent chunks already resident (read
-//      MN-major), into all 512 TMEM columns, committing each half on its own;
+//   3. accumulates O = P C[:, 0:512] (M = 128, K = 128), whose B operands are
+//      the latent chunks already resident (read MN-major), into all 512 TMEM
+//      columns as four N = 128 quarters, each committed on its own;
 //   4. writes bf16 out (+ lse) when the row has one unit, else a normalised
-//      fp16 partial with its (max, sum, power-of-two ranges), half by half as
-//      the MMAs complete, so that the first half's stores overlap the second
-//      half's MMAs.  The once-per-CTA loops here are rolled: straight-line code
-//      that runs once stalls on instruction fetch.  The partials of
+//      fp16 partial with its (max, sum, power-of-two ranges per column half),
+//      quarter by quarter as the MMAs complete, so that the stores overlap the
+//      following quarters' MMAs.  The once-per-CTA loops here are rolled:
+//      straight-line code that runs once stalls on instruction fetch.  The partials of
 //      a row's units ("splits") are merged by a combine kernel launched right
 //      behind (programmatic launch: its CTAs are resident, waiting, while the
 //      attention finishes).  The attention itself is a plain programmatic
@@ -250,9 +250,9 @@ sparse_mla_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const MlaArgs a) 
     uint64_t *q_ready = q_full + 1;              // the query's latent part is in TMEM (256 arrivals)
     uint64_t *s_done = q_ready + 1;              // every logit MMA is complete
     uint64_t *p_full = s_done + 1;               // P is in shared memory (256 arrivals)
-    uint64_t *o_full = p_full + 1;               // [2] column half hv of O is complete
-    uint64_t *mma_fin = o_full + 2;              // every issued MMA is complete
-    uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(bars + 16);   // after the 16 barriers
+    uint64_t *o_full = p_full + 1;               // [4] column quarter q of O is complete
+    uint64_t *mma_fin = o_full + 4;              // every issued MMA is complete
+    uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(bars + 20);   // after the 18 barriers
     volatile int *abort = reinterpret_cast<volatile int *>(tmem_holder + 1);
     uint32_t *vmask = reinterpret_cast<uint32_t *>(const_cast<int *>(abort) + 1);   // [4]
     // softmax exchange (max and sum of the two slot halves): the query's
@@ -274,8 +274,7 @@ sparse_mla_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const MlaArgs a) 
             tc::mbar_init(q_ready, kWork);
             tc::mbar_init(s_done, 1);
             tc::mbar_init(p_full, kWork);
-            tc::mbar_init(&o_full[0], 1);
-            tc::mbar_init(&o_full[1], 1);
+            for (int i = 0; i < 4; i++) tc::mbar_init(&o_full[i], 1);
             tc::mbar_init(mma_fin, 1);
             *abort = 0;
             tc::fence_mbar_init();
@@ -538,7 +537,8 @@ sparse_mla_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const MlaArgs a) 
         // ---------------------------------------------------------- epilogue
         if (a.splits == 1) {
             // thread (h, c) owns output columns [256c, 256c + 256)
-            if (ok && !tc::mbar_wait(&o_full[c], 0, a.err, abort)) ok = false;
+            if (ok && !tc::mbar_wait(&o_full[2 * c], 0, a.err, abort)) ok = false;
+            if (ok && !tc::mbar_wait(&o_full[2 * c + 1], 0, a.err, abort)) ok = false;
             tc::tc_fence_after();
             const uint32_t ocol = tmem + lane_addr + kColO + c * 256;
             const float inv = lt > 0.f ? 1.f / lt : 0.f;
@@ -576,7 +576,7 @@ sparse_mla_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const MlaArgs a) 
             auto write_cols = [&](uint32_t ocol, int oct0, float inv, bool track) -> float {
                 float amax = 0.f;
 #pragma unroll 1
-                for (int g = 0; g < 8; g++) {
+                for (int g = 0; g < 4; g++) {
                     uint32_t ov[16];
                     tc::tmem_ld16(ocol + 16 * g, ov);
                     tc::tmem_wait_ld();
@@ -596,18 +596,28 @@ sparse_mla_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const MlaArgs a) 
                 }
                 return amax;
             };
+            // quarter q: thread (h, c) writes columns [128q + 64c, 128q + 64c + 64)
+            float hmax = 0.f;
 #pragma unroll 1
-            for (int hv = 0; hv < 2; hv++) {
-                if (ok && !tc::mbar_wait(&o_full[hv], 0, a.err, abort)) ok = false;
+            for (int q = 0; q < 4; q++) {
+                if (ok && !tc::mbar_wait(&o_full[q], 0, a.err, abort)) ok = false;
                 tc::tc_fence_after();
-                const uint32_t ocol = tmem + lane_addr + kColO + 256 * hv + 128 * c;
-                const int oct0 = 32 * hv + 16 * c;
-                xmax[(2 * hv + c) * kHq + h] = write_cols(ocol, oct0, inv_l, true);
+                hmax = fmaxf(hmax, write_cols(tmem + lane_addr + kColO + 128 * q + 64 * c,
+                                              16 * q + 8 * c, inv_l, true));
+                if (!(q & 1)) continue;
+                // column half hv = q / 2 complete: its range, from both threads of the head
+                const int hv = q >> 1;
+                xmax[(2 * hv + c) * kHq + h] = hmax;
+                hmax = 0.f;
                 tc::named_barrier(1, kWork);
                 const float amax = fmaxf(xmax[2 * hv * kHq + h], xmax[(2 * hv + 1) * kHq + h]);
                 float scl = 1.f;
                 while (amax * inv_l > 16384.f * scl) scl *= 2.f;
-                if (scl != 1.f) write_cols(ocol, oct0, inv_l / scl, false);
+                if (scl != 1.f) {
+                    for (int q2 = q - 1; q2 <= q; q2++)
+                        write_cols(tmem + lane_addr + kColO + 128 * q2 + 64 * c, 16 * q2 + 8 * c,
+                                   inv_l / scl, false);
+                }
                 if (ok && c == 0) ml[2 + hv] = scl;
             }
             // (max, sum, range of columns [0, 256), range of columns [256, 512))
@@ -657,21 +667,21 @@ sparse_mla_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const MlaArgs a) 
         if (ok) tc::tc_commit(s_done);
         if (ok && tc::mbar_wait(p_full, 0, a.err, abort)) {
             tc::tc_fence_after();
-            // O[:, 256 hv + n] += P C[:, 256 hv + n]: K-step ks covers rows
+            // O[:, 128 q + n] += P C[:, 128 q + n]: K-step ks covers rows
             // [16 ks, 16 ks + 16); A = P (K-major, block ks / 4), B = the latent
-            // chunks 4 hv .. 4 hv + 3 (MN-major, 16 KB between 64-column blocks)
-            // Half 0 is committed before half 1 is issued, so that its
-            // epilogue overlaps the second half's MMAs.
-            const uint32_t id_pv = tc::instr_desc(tc::kFmtBF16, tc::kFmtBF16, 128, 256, true);
-            for (int hv = 0; hv < 2; hv++) {
+            // chunks 2q, 2q + 1 (MN-major, 16 KB between 64-column blocks).
+            // Each quarter is committed before the next is issued, so that its
+            // epilogue overlaps the following quarters' MMAs.
+            const uint32_t id_pv = tc::instr_desc(tc::kFmtBF16, tc::kFmtBF16, 128, 128, true);
+            for (int q = 0; q < 4; q++) {
                 for (int ks = 0; ks < kU / 16; ks++) {
                     const uint64_t pa = tc::smem_desc(sbase + kP + (ks >> 2) * kQBlk + (ks & 3) * 32,
                                                       1024, tc::kSwizzle128B);
-                    const uint64_t bd = tc::smem_desc(sbase + 4 * hv * kRegion + ks * 2048, 1024,
+                    const uint64_t bd = tc::smem_desc(sbase + 2 * q * kRegion + ks * 2048, 1024,
                                                       tc::kSwizzle128B, kRegion);
-                    tc::mma_f16(tmem + kColO + 256 * hv, pa, bd, id_pv, ks > 0);
+                    tc::mma_f16(tmem + kColO + 128 * q, pa, bd, id_pv, ks > 0);
                 }
-                tc::tc_commit(&o_full[hv]);
+                tc::tc_commit(&o_full[q]);
             }
         }
         // every issued MMA completes before TMEM is released
