@@ -483,10 +483,10 @@ topk_cluster_kernel(const float *scores, int S, int64_t T, int64_t start_pos, in
 // slice of the bins over the row's scorer histograms and stores the sums into
 // every CTA of the cluster, so that after one cluster barrier every CTA holds
 // the row's histogram and finds the same 12-bit threshold bin on its own; the
-// scores are read once.  Each CTA reserves a
-// range of CTA 0's candidate list with one atomic and stores the keys of its
-// span that fall in the bin there, with their positions (distributed shared
-// memory); CTA 0 finds tau among them (a 10-bit histogram pass, then one warp
+// scores are read once.  Each warp adds its counts into CTA 0's per-CTA
+// totals, reserves a range of CTA 0's candidate list with one atomic and
+// stores its keys that fall in the bin there, with their positions
+// (distributed shared memory); CTA 0 finds tau among them (a 10-bit histogram pass, then one warp
 // ranks the few keys left, or further passes when they are many) and every
 // CTA's output offset and tau-equal quota, and sends each CTA its numbers.
 // Two cluster barriers on the common path; global memory sees only the
@@ -505,16 +505,14 @@ constexpr int kDecFew = 32;                         // keys one warp ranks direc
 struct DecShared {
     unsigned hist[kBins];             // CTA 0: histogram of the current pass or round
     unsigned rowhist[kBins];          // the row's histogram, a slice from each CTA
-    uint2 cand[kDecCap];              // CTA 0: gathered (key, position), CTA by CTA
+    uint2 cand[kDecCap];              // CTA 0: gathered (key, position), warp by warp
     int n_cand;                       // CTA 0: slots reserved
-    int base[kMaxCluster];            // CTA 0: per CTA, its first slot
     int cnt_gt[kMaxCluster];          // CTA 0: per CTA, keys above the group
     int cnt_in[kMaxCluster];          // CTA 0: per CTA, keys inside it
     int sel_gt[kMaxCluster];          // CTA 0: per CTA, gathered keys above tau
     int sel_eq[kMaxCluster];          // CTA 0: per CTA, gathered keys equal to tau
     unsigned res[4];                  // from CTA 0: prefix, prefix bits, rank in group, group size
     unsigned out[3];                  // from CTA 0: tau, output offset, tau-equal quota
-    int my_base;
     int n_few;
     uint32_t few[kDecFew];
     unsigned s_out[3];
@@ -623,6 +621,12 @@ topk_decode_kernel(const float *scores, int64_t T, int K, int32_t *__restrict__ 
     if (p == 0) {
         for (int i = tid; i < kBins; i += kDecThreads) sh.hist[i] = 0;
         if (tid == 0) sh.n_cand = 0;
+        if (tid < kMaxCluster) {
+            sh.cnt_gt[tid] = 0;
+            sh.cnt_in[tid] = 0;
+            sh.sel_gt[tid] = 0;
+            sh.sel_eq[tid] = 0;
+        }
     }
     if (tid == 0) sh.n_few = 0;
     __syncthreads();
@@ -777,20 +781,27 @@ topk_decode_kernel(const float *scores, int64_t T, int K, int32_t *__restrict__ 
         m_in |= (uint32_t)(g == prefix) << j;
     }
     const int n_gt = __popc(m_gt), n_in = __popc(m_in);
-    int2 tot;
-    const int2 ex = block_scan2_dec(n_gt, n_in, sh, &tot);
-    if (tid == 0) {
-        sh0->cnt_gt[p] = tot.x;
-        sh0->cnt_in[p] = tot.y;
-        if (gather) {
-            const int b = atomicAdd(&sh0->n_cand, tot.y);
-            sh0->base[p] = b;
-            sh.my_base = b;
+    // per warp: its counts added into CTA 0's per-CTA totals, and (when the
+    // group is gathered) a range of CTA 0's list reserved with one atomic,
+    // each lane's keys at its place within the warp's range
+    int incl = n_in;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += y;
+    }
+    const int w_in = __shfl_sync(0xffffffffu, incl, 31);
+    const int w_gt = warp_sum_first(n_gt, lane, 32);
+    int wbase = 0;
+    if (lane == 0) {
+        if (w_gt) atomicAdd(&sh0->cnt_gt[p], w_gt);
+        if (w_in) {
+            atomicAdd(&sh0->cnt_in[p], w_in);
+            if (gather) wbase = atomicAdd(&sh0->n_cand, w_in);
         }
     }
-    if (gather) {
-        __syncthreads();
-        int slot = sh.my_base + ex.y;
+    if (gather && w_in) {
+        int slot = __shfl_sync(0xffffffffu, wbase, 0) + incl - n_in;
         for (uint32_t mm = m_in; mm; mm &= mm - 1u) {
             const int j = __ffs(mm) - 1;
             if (slot < kDecCap) sh0->cand[slot] = make_uint2(key_at(j), (uint32_t)(t0 + j));
@@ -865,22 +876,13 @@ topk_decode_kernel(const float *scores, int64_t T, int K, int32_t *__restrict__ 
             }
             tau = tp;
             q = (int)rk;
-            // per CTA (its contiguous range of the list): keys above tau, equal to it
-            for (int r = warp; r < CN; r += kDecWarps) {
-                const int lo = sh.base[r], n = sh.cnt_in[r];
-                int gt = 0, eq = 0;
-                for (int j = lane; j < n; j += 32) {
-                    if (lo + j >= kDecCap) break;
-                    const uint32_t k = sh.cand[lo + j].x;
-                    gt += k > tau;
-                    eq += k == tau;
-                }
-                gt = warp_sum_first(gt, lane, 32);
-                eq = warp_sum_first(eq, lane, 32);
-                if (lane == 0) {
-                    sh.sel_gt[r] = gt;
-                    sh.sel_eq[r] = eq;
-                }
+            // per CTA (a candidate's CTA is its position / kDecSpan): keys above
+            // tau, and equal to it
+            for (int j = tid; j < E; j += kDecThreads) {
+                const uint2 cj = sh.cand[j];
+                const int r = (int)(cj.y / (uint32_t)kDecSpan);
+                if (cj.x > tau) atomicAdd(&sh.sel_gt[r], 1);
+                else if (cj.x == tau) atomicAdd(&sh.sel_eq[r], 1);
             }
             __syncthreads();
         } else {
