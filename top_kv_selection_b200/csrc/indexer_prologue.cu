@@ -10,18 +10,20 @@
 // quantised (act_quant with the configured scale format), and the key's codes
 // and scale are written into the caches at positions start_pos .. end_pos-1.
 //
-// G = D / 64 adjacent lanes hold one D-vector, 64 contiguous elements each
-// (lane part p: elements [64p, 64p + 64)), as in quant.cuh's
-// rotate_quant_lanes; a warp holds 32 / G vectors (query head vectors first,
-// then the new tokens' keys).  Rotary pairs are element j and element j + R/2
-// (j < R/2).  For R <= 64 both live in part 0's registers; for R = 128 (D = 128)
-// they are the same register of the two lanes of a vector, one shuffle apart.
-// With (c, s) the angle of frequency j at the token's position, the lower
-// element becomes x1*c - x2*s and the upper x1*s + x2*c (x1 lower, x2 upper),
-// each product and sum rounded to fp32.  Then the butterfly, the scale and the
-// codes of rotate_quant_lanes.  HBM-bound: 4*D (fp32) or 2*D (bf16) bytes in
-// and D + 4 bytes out per vector, plus the angles (R/2 * 8 bytes per token,
-// L2-resident and the same address for every head of a token).
+// G = D / 64 adjacent lanes hold one D-vector, 64 elements each, as in
+// quant.cuh's rotate_quant_lanes; a warp holds 32 / G vectors (query head
+// vectors first, then the new tokens' keys).  Rotary pairs are element j and
+// element j + R/2 (j < R/2).  For D = 128 the two lanes split the vector on
+// the element bit just below the pair's (bit 4 for R = 64, bit 5 for R = 128,
+// bit 3 for R = 32 with bf16 input), so that both elements of a pair sit in
+// one lane and each lane holds half of the pairs; other rotary widths keep
+// contiguous halves, where every pair lies in part 0.  With (c, s) the angle
+// of frequency j at the token's position, the lower element becomes
+// x1*c - x2*s and the upper x1*s + x2*c (x1 lower, x2 upper), each product and
+// sum rounded to fp32.  Then the butterfly, the scale and the codes of
+// rotate_quant_lanes.  HBM-bound: 4*D (fp32) or 2*D (bf16) bytes in and D + 4
+// bytes out per vector, plus the angles (R/2 * 8 bytes per token, L2-resident
+// and staged once per warp pass when the pass covers at most two tokens).
 #include "common.cuh"
 #include "quant.cuh"
 
