@@ -50,6 +50,21 @@ __device__ __forceinline__ void record_error(int *word, int code) {
     if (word) atomicCAS(word, 0, code);
 }
 
+// Loads of a preceding kernel's output (or of anything written in the same
+// stream order) after griddepcontrol.wait: L2-coherent (.cg), and volatile so
+// that the compiler keeps them after the wait (a non-coherent __ldg may be
+// moved above it).
+__device__ __forceinline__ uint32_t ld_cg_u32(const uint32_t *p) {
+    uint32_t v;
+    asm volatile("ld.global.cg.u32 %0, [%1];" : "=r"(v) : "l"(p));
+    return v;
+}
+__device__ __forceinline__ float ld_cg_f32(const float *p) {
+    float v;
+    asm volatile("ld.global.cg.f32 %0, [%1];" : "=f"(v) : "l"(p));
+    return v;
+}
+
 // Order-preserving map from an fp32 score to an unsigned key: a > b as floats
 // <=> key(a) > key(b).  -0 maps to the key of +0; NaN maps to 0, below -inf.
 __device__ __forceinline__ uint32_t score_key(float f) {

@@ -278,7 +278,7 @@ score_tc_kernel(const __grid_constant__ CUtensorMap tmap_k,
     auto load_ks = [&](int ii) -> float {
         const int64_t tt = (tile_lo + ii) * kTile + tok;
         if (ii >= n_my || tt >= n_vis) return 0.f;
-        return (append && tt == a.T - 1) ? *knew_scale : __ldg(ks_row + tt);
+        return (append && tt == a.T - 1) ? *knew_scale : ld_cg_f32(ks_row + tt);
     };
     // the epilogue warp whose tokens include position T-1 appends the new key,
     // so the key's scale passes between lanes of one warp

@@ -668,7 +668,7 @@ topk_decode_kernel(const float *scores, int64_t T, int K, int32_t *__restrict__ 
                     unsigned v[kSumBatch];
 #pragma unroll
                     for (int c = 0; c < kSumBatch; c++)
-                        v[c] = c0 + c < hist_chunks ? __ldg(rh + (c0 + c) * kBins + bb) : 0u;
+                        v[c] = c0 + c < hist_chunks ? ld_cg_u32(rh + (c0 + c) * kBins + bb) : 0u;
 #pragma unroll
                     for (int c = 0; c < kSumBatch; c++) acc += v[c];
                 }
