@@ -135,3 +135,62 @@ def test_decode_step_fp8_latent_cache(dsa, T, B):
         assert_attention_close(st["out"][b].float().cpu().numpy(), ref[0, 0], "bf16",
                                st["lse"][b].cpu().numpy(), ref_lse[0, 0])
     assert dsa.dsa_get_device_error() == 0
+
+
+def test_decode_steps_growing_context(dsa):
+    """Four decode steps launched back to back on one stream, the context growing
+    by one token each step (T0 .. T0 + 3), with nothing between the launches:
+    every step's scorer reads the keys that the previous steps appended while the
+    kernels overlap through their programmatic launches.  Each step's selection,
+    output and appended key match the oracle's decode pass over the cache as it
+    stood at that step."""
+    wl = workloads.WORKLOADS[1]
+    B, T0, n = 2, 3000, 4
+    t_max = T0 + n - 1
+    dev = "cuda"
+    dt = torch.bfloat16
+    base = [workloads.decode_sequence(wl, b, T=t_max) for b in range(B)]
+    # per step: the new token's queries, weights and attention query
+    stepq = [[workloads.decode_sequence(wl, 100 + 10 * i + b, T=1) for b in range(B)]
+             for i in range(n)]
+    k_cache = torch.zeros(B, t_max, wl.D, dtype=torch.uint8, device=dev)
+    k_scale = torch.zeros(B, t_max, dtype=torch.float32, device=dev)
+    kv = torch.zeros(B, t_max, wl.dqk, dtype=dt, device=dev)
+    for b, s in enumerate(base):
+        dsa.dsa_indexer_quant(s["keys"][:T0 - 1].to(dev), k_cache[b], k_scale[b])
+        kv[b] = s["kv"].to(dev)
+    q_idx = torch.stack([torch.stack([stepq[i][b]["q_idx"] for b in range(B)])
+                         for i in range(n)]).to(dev)
+    w = torch.stack([torch.stack([stepq[i][b]["w"] for b in range(B)]) for i in range(n)]).to(dev)
+    q_mla = torch.stack([torch.stack([stepq[i][b]["q_mla"] for b in range(B)])
+                         for i in range(n)]).to(dev)
+    k_new = torch.stack([torch.stack([base[b]["keys"][T0 - 1 + i] for b in range(B)])
+                         for i in range(n)]).to(dev)
+    K = min(wl.topk, T0)
+    idx = torch.empty(n, B, K, dtype=torch.int32, device=dev)
+    out = torch.empty(n, B, wl.Hq, wl.dc, dtype=dt, device=dev)
+    lse = torch.empty(n, B, wl.Hq, dtype=torch.float32, device=dev)
+    need = max(dsa.dsa_decode_step_workspace_size(B, wl.H, wl.D, T0 + i, wl.topk, wl.Hq, wl.dc,
+                                                  wl.dr, dsa.DSA_BF16) for i in range(n))
+    ws = torch.empty(need, dtype=torch.uint8, device=dev)
+    torch.cuda.synchronize()
+    for i in range(n):
+        dsa.dsa_decode_step(q_idx[i], w[i], k_new[i], k_cache, k_scale, kv, q_mla[i], T0 + i,
+                            wl.topk, wl.softmax_scale_idx, wl.sm_scale, idx[i], out[i], lse[i],
+                            ws)
+    torch.cuda.synchronize()
+    assert dsa.dsa_get_device_error() == dsa.DSA_OK
+    for i in range(n):
+        T = T0 + i
+        for b in range(B):
+            r = oracle.decode_step(stepq[i][b]["q_idx"].numpy(), stepq[i][b]["w"].numpy(),
+                                   base[b]["keys"][:T].numpy(),
+                                   stepq[i][b]["q_mla"].float().numpy(),
+                                   base[b]["kv"][:T].float().numpy(), topk=wl.topk,
+                                   softmax_scale_idx=wl.softmax_scale_idx, sm_scale=wl.sm_scale,
+                                   dc=wl.dc)
+            assert np.array_equal(k_cache[b, T - 1].cpu().numpy(), r["k_fp8"][T - 1])
+            assert k_scale[b, T - 1].item() == r["k_scale"][T - 1]
+            assert_selection_matches(idx[i, b].cpu().numpy(), r["idx"], r["scores"])
+            assert_attention_close(out[i, b].float().cpu().numpy(), r["out"], wl.attn_dtype,
+                                   lse[i, b].cpu().numpy(), r["lse"])
