@@ -564,11 +564,12 @@ sparse_mla_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const MlaArgs a) 
         } else {
             // O / (l * sc) in fp16 for the split merge, as [column / 8][head]
             // groups of eight halves, sc per column half: the power of two
-            // that keeps the half's |O / l| / sc <= 2^14.  The halves are
+            // that keeps the half's |O / l| / sc <= 2^14.  The quarters are
             // written in MMA completion order, both threads of a head taking
-            // 128 columns of each; a half is written with sc = 1 and written
-            // again only when the head's max |O| over its 256 columns (the two
-            // threads' maxima) asks for a larger range.
+            // 64 columns of each; a half's two quarters are written with
+            // sc = 1 and written again only when the head's max |O| over the
+            // half's 256 columns (the two threads' maxima) asks for a larger
+            // range.
             const float inv_l = lt > 0.f ? 1.f / lt : 0.f;
             uint4 *po = reinterpret_cast<uint4 *>(a.part_o + (int64_t)blockIdx.x * kHq * kDc) + h;
             float *ml = reinterpret_cast<float *>(a.part_ml + (int64_t)blockIdx.x * kHq + h);
