@@ -167,9 +167,10 @@ __device__ __forceinline__ uint4 decode8(uint32_t w0, uint32_t w1, float sc) {
 // splits' fp16 partials (blocks blk0 .. blk0 + splits - 1), for NC octets
 // c8[0..NC) at once: with w_s = 2^(m_s - M) l_s and Y_s = O_s / (l_s sc_s),
 // out = sum_s w_s sc_s Y_s / sum_s w_s and lse = (M + log2 sum_s w_s) ln 2.
-// The loads of kMergeBatch splits are in flight together (all sixteen of a
-// 2048-slot row); further batches rescale the running sums.
-constexpr int kMergeBatch = 16;
+// The loads of kMergeBatch splits are in flight together (eight of the
+// sixteen of a 2048-slot row, for two octets at once); further batches
+// rescale the running sums.
+constexpr int kMergeBatch = 8;
 template <int NC>
 __device__ __forceinline__ void merge_octets(const __half *part_o, const float4 *part_ml, int splits,
                                              int64_t blk0, int64_t row, const int (&c8)[NC], int h,
@@ -697,19 +698,23 @@ sparse_mla_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const MlaArgs a) 
     }
 }
 
-// Merges the splits of each query row: thread (head, octet) merges eight
-// output columns of one head, consecutive threads consecutive heads
-// (coalesced reads of the partials).
+// Merges the splits of each query row: thread (head, octet pair) merges
+// sixteen output columns of one head, consecutive threads consecutive heads
+// (coalesced reads of the partials): 256 CTAs at B = 8, all resident beside
+// the attention's CTAs, waiting.  The next kernel (the next step's scorer) is
+// released only once the attention has completed, so that its CTAs do not
+// take the SMs that the attention's last CTAs are waiting for.
 __global__ void __launch_bounds__(kHq)
 sparse_mla_combine_kernel(const __half *part_o, const float4 *part_ml, int splits, int64_t row0,
                           __nv_bfloat16 *__restrict__ out, float *__restrict__ lse) {
-    // the next kernel (the next step's scorer) may start its set-up now
-    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     // the partials come from the preceding kernel: wait for it (plain loads below)
     asm volatile("griddepcontrol.wait;" ::: "memory");
-    const int64_t r = blockIdx.x / kOct;                 // row - row0
-    const int c8[1] = {(int)(blockIdx.x % kOct)};
-    merge_octets<1>(part_o, part_ml, splits, r * splits, row0 + r, c8, threadIdx.x, out, lse);
+    // the next kernel may start its set-up while the splits are merged
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    const int64_t r = blockIdx.x / (kOct / 2);           // row - row0
+    const int pair = (int)(blockIdx.x % (kOct / 2));
+    const int c8[2] = {2 * pair, 2 * pair + 1};
+    merge_octets<2>(part_o, part_ml, splits, r * splits, row0 + r, c8, threadIdx.x, out, lse);
 }
 
 // Split partials of one query row.
@@ -795,7 +800,7 @@ dsa_status launch(const void *q, const void *kv, int64_t t_max, const int32_t *i
         if (st != DSA_OK) return st;
         if (a.splits == 1) continue;
         cudaLaunchConfig_t ccfg = {};
-        ccfg.gridDim = dim3((unsigned)(n * kOct));
+        ccfg.gridDim = dim3((unsigned)(n * (kOct / 2)));
         ccfg.blockDim = dim3(kHq);
         ccfg.stream = stream;
         cudaLaunchAttribute cattr[1];
