@@ -364,10 +364,39 @@ def run_reference(args, wl, world, rank):
 # --------------------------------------------------------------------------- #
 # our arm
 # --------------------------------------------------------------------------- #
+def bind_local_cpus(device_index: int) -> list | None:
+    """Restrict this process to the CPUs NVML reports as local to the GPU (its
+    NUMA node), as a serving process is placed: pinned host buffers are then
+    allocated, and the copies and launches issued, next to the GPU's PCIe root.
+    Best effort: returns the CPU list, or None when NVML or the affinity call is
+    unavailable.  Reads only; changes no GPU setting."""
+    try:
+        import pynvml
+        pynvml.nvmlInit()
+        p = torch.cuda.get_device_properties(device_index)
+        try:
+            bus = f"{p.pci_domain_id:08X}:{p.pci_bus_id:02X}:{p.pci_device_id:02X}.0"
+            h = pynvml.nvmlDeviceGetHandleByPciBusId(bus)
+        except Exception:
+            h = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+        n_words = (os.cpu_count() + 63) // 64
+        words = pynvml.nvmlDeviceGetCpuAffinity(h, n_words)
+        cpus = [64 * i + b for i, w in enumerate(words) for b in range(64) if (w >> b) & 1]
+        cpus = [c for c in cpus if c < os.cpu_count()]
+        if not cpus:
+            return None
+        os.sched_setaffinity(0, cpus)
+        return cpus
+    except Exception:
+        return None
+
+
 def run_ours(args, wl, world, rank, local):
     import __graft_entry__
     __graft_entry__._builder().build()
     import top_kv_selection_b200 as dsa
+
+    local_cpus = bind_local_cpus(torch.cuda.current_device())
 
     # every rank draws its own independent sequences
     copies = build_state(dsa, wl, rank_seed_offset=rank * wl.B, n_copies=args.copies)
@@ -481,6 +510,8 @@ def run_ours(args, wl, world, rank, local):
                      "frac": achieved / peak, "traffic": profiled_traffic(),
                      "avg_launch_us": t_score * 1e6},
         "e2e": e2e,
+        "host_cpus": (f"{len(local_cpus)} GPU-local CPUs (NVML affinity)" if local_cpus
+                      else "not bound"),
         "gpu_launches": per_step_launches * args.steps,
         "kernels_per_step": per_step_launches, "kernels": kernel_names,
         "stage_us": {k: round(v * 1e6, 2) for k, v in stages.items()},
